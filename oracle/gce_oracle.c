@@ -1,0 +1,385 @@
+/*
+ * gce_oracle.c -- plain, slow, obviously-correct CPU oracle for the
+ * gradient-compression step with error-feedback memory.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may call, link or
+ * execute this file.  Its only callers are the tests under tests/, the
+ * smoke() check in __graft_entry__.py and the cpu_baseline / reference leg of
+ * bench.py.  It shares no code, header, table or constant generator with the
+ * CUDA library in gradient_compression_error_b200/csrc; the two are written
+ * independently from the same definitions.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared
+ *        (see oracle/build.py).  -ffp-contract=off keeps every float
+ *        multiply and add separately rounded, which the Mem-SGD reading below
+ *        requires.  Single-threaded; every function handles one unit
+ *        (one worker's layer) and touches nothing global.
+ *
+ * Sources (page title, section):
+ *   [MEM]  "Sparsified SGD with Memory", Method: the k-contraction operator
+ *          comp_k, the memory m_t that accumulates what was not sent, and the
+ *          update  g_t = comp_k(m_t + eta_t grad),
+ *                  m_{t+1} = m_t + eta_t grad - g_t.
+ *          Abstract / Motivation: top-k keeps the largest entries, rand-k
+ *          keeps random entries.  Key results: 0 < k <= d.
+ *   [ACC]  "Accordion: Adaptive Gradient Communication via Critical Learning
+ *          Regime Identification", Method: per-layer gradient-norm rate of
+ *          change detects critical regimes; inside one use the low-compression
+ *          level l_low (e.g. higher rank / higher K), outside it the
+ *          high-compression level l_high.
+ *   [UTIL] "On the Utility of Gradient Compression in Distributed Training
+ *          Systems", Method / Key results: PowerSGD is all-reduce compatible;
+ *          payloads are summed across data-parallel workers.
+ *   PowerSGD's steps are not printed on the pages (they only name it and its
+ *   rank).  This oracle takes the standard single power-iteration step with a
+ *   reused (warm-started) Q: P = M Q, orthonormalise P, Q' = M^T P,
+ *   decompress P Q'^T, residual into memory.
+ *
+ * Readings where the pages are silent (each listed in the design doc):
+ *   - residual rounding: v = fl32(m + fl32(eta * g)), two separate roundings,
+ *     no fused multiply-add;
+ *   - top-k order: key = |v| taken as the float's bits with the sign cleared;
+ *     larger key first, equal keys -> lower index first; the payload is
+ *     emitted in ascending index; selected memory becomes +0.0f;
+ *   - rand-k: uniform k-subset = the k smallest (hash key, index) pairs, the
+ *     hash being SplitMix64 (Steele, Lea, Flood 2014) keyed by
+ *     (seed, stream, worker, layer, step); values are not rescaled;
+ *   - PowerSGD orientation: M is rows x cols row-major, P rows x r,
+ *     Q cols x r (stored with row stride r_max); orthonormalisation is
+ *     modified Gram-Schmidt in column order, a zero column stays zero;
+ *   - Accordion: L2 norm of the raw gradient per layer at check steps, a
+ *     missing previous norm (prev < 0) means "critical", rel change >= the
+ *     threshold means "critical" (level LOW = l_low), else HIGH = l_high;
+ *   - k from a fraction in parts per million: k = max(1, floor(n*ppm/1e6)).
+ *
+ * Parity unpinned (nothing on the pages fixes it):
+ *   or_randk_base / the stream composition of the rand-k and Q-init hashes
+ *   (the SplitMix64 step itself is pinned by its published outputs);
+ *   or_powersgd_init_q's mapping of hash bits to [-1, 1).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_ERR_ARG (-1)
+#define OR_ERR_NOMEM (-2)
+
+/* ------------------------------------------------------------------ */
+/* Mem-SGD residual [MEM]: v = m + eta * g, two separate fp32 roundings. */
+static float or_residual(float m, float eta, float g)
+{
+    float t = eta * g;   /* fl32(eta * g) */
+    float v = m + t;     /* fl32(m + t)   */
+    return v;
+}
+
+/* |v| ordering key: the IEEE-754 bits of v with the sign bit cleared.  For
+ * finite floats this orders exactly like |v| (and +0 == -0). */
+static uint32_t or_abs_key(float v)
+{
+    uint32_t b;
+    memcpy(&b, &v, sizeof b);
+    return b & 0x7FFFFFFFu;
+}
+
+typedef struct {
+    uint32_t key;
+    int32_t idx;
+} or_pair;
+
+/* larger key first; equal keys -> lower index first */
+static int or_cmp_key_desc(const void* a, const void* b)
+{
+    const or_pair* x = (const or_pair*)a;
+    const or_pair* y = (const or_pair*)b;
+    if (x->key != y->key) return x->key > y->key ? -1 : 1;
+    return x->idx < y->idx ? -1 : (x->idx > y->idx ? 1 : 0);
+}
+
+/* smaller key first; equal keys -> lower index first */
+static int or_cmp_key_asc(const void* a, const void* b)
+{
+    const or_pair* x = (const or_pair*)a;
+    const or_pair* y = (const or_pair*)b;
+    if (x->key != y->key) return x->key < y->key ? -1 : 1;
+    return x->idx < y->idx ? -1 : (x->idx > y->idx ? 1 : 0);
+}
+
+static int or_cmp_idx_asc(const void* a, const void* b)
+{
+    const or_pair* x = (const or_pair*)a;
+    const or_pair* y = (const or_pair*)b;
+    return x->idx < y->idx ? -1 : (x->idx > y->idx ? 1 : 0);
+}
+
+/* k from a fraction given in parts per million: max(1, floor(n*ppm/1e6)). */
+int64_t or_k_from_ppm(int64_t n, int64_t ppm)
+{
+    int64_t k = (n * ppm) / 1000000;
+    return k < 1 ? 1 : k;
+}
+
+/* Shared tail of top-k and rand-k: given v[] and the selection order already
+ * applied to pairs[] (the first k pairs are the chosen set), emit the payload
+ * in ascending index and write the memory update m = v - g. */
+static void or_emit_selected(int64_t n, int64_t k, const float* v, or_pair* pairs,
+                             float* m, float* vals, int32_t* idx)
+{
+    qsort(pairs, (size_t)k, sizeof(or_pair), or_cmp_idx_asc);
+    for (int64_t i = 0; i < n; ++i) m[i] = v[i];          /* m_{t+1} = v - g ... */
+    for (int64_t j = 0; j < k; ++j) {
+        int32_t i = pairs[j].idx;
+        vals[j] = v[i];                                   /* g_t,i = v_i on S   */
+        idx[j] = i;
+        m[i] = 0.0f;                                      /* ... = +0 on S      */
+    }
+}
+
+/*
+ * One Mem-SGD top-k step for one worker's layer [MEM].
+ *   g[n]   gradient (read)          m[n]   memory (read, then overwritten)
+ *   vals[k], idx[k]                 payload, ascending idx
+ */
+int or_ef_topk(int64_t n, int64_t k, float eta, const float* g, float* m,
+               float* vals, int32_t* idx)
+{
+    if (n < 1 || k < 1 || k > n || n > INT32_MAX) return OR_ERR_ARG;
+    float* v = (float*)malloc((size_t)n * sizeof(float));
+    or_pair* pairs = (or_pair*)malloc((size_t)n * sizeof(or_pair));
+    if (!v || !pairs) { free(v); free(pairs); return OR_ERR_NOMEM; }
+    for (int64_t i = 0; i < n; ++i) {
+        v[i] = or_residual(m[i], eta, g[i]);
+        pairs[i].key = or_abs_key(v[i]);
+        pairs[i].idx = (int32_t)i;
+    }
+    qsort(pairs, (size_t)n, sizeof(or_pair), or_cmp_key_desc);
+    or_emit_selected(n, k, v, pairs, m, vals, idx);
+    free(v);
+    free(pairs);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* SplitMix64 (Steele, Lea, Flood, "Fast splittable pseudorandom number
+ * generators", OOPSLA 2014): the state advances by the golden-ratio gamma
+ * and each output is the state passed through the 64-bit finaliser. */
+#define OR_GAMMA 0x9E3779B97F4A7C15ull
+
+static uint64_t or_mix64(uint64_t z)
+{
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+/* The j-th output (j >= 1) of a SplitMix64 generator started at `state`. */
+uint64_t or_splitmix64_output(uint64_t state, uint64_t j)
+{
+    return or_mix64(state + j * OR_GAMMA);
+}
+
+/* Per-unit base state: each of seed, stream, worker, layer, step is folded in
+ * by taking the first SplitMix64 output from (previous + (value+1)*gamma). */
+uint64_t or_randk_base(uint64_t seed, uint64_t stream, uint64_t worker,
+                       uint64_t layer, uint64_t step)
+{
+    uint64_t h = or_splitmix64_output(seed, stream + 1);
+    h = or_splitmix64_output(h, worker + 1);
+    h = or_splitmix64_output(h, layer + 1);
+    h = or_splitmix64_output(h, step + 1);
+    return h;
+}
+
+/* rand-k key of coordinate i: high 32 bits of output i+1 from the base. */
+uint32_t or_randk_key(uint64_t base, int64_t i)
+{
+    return (uint32_t)(or_splitmix64_output(base, (uint64_t)i + 1) >> 32);
+}
+
+/*
+ * One Mem-SGD rand-k step for one worker's layer [MEM]: same update as top-k,
+ * the chosen set is the k coordinates with the smallest (key, index).
+ * Unscaled: g_i = v_i on the chosen set (comp_k stays a k-contraction).
+ */
+int or_ef_randk(int64_t n, int64_t k, float eta, const float* g, float* m,
+                float* vals, int32_t* idx, uint64_t seed, uint64_t worker,
+                uint64_t layer, uint64_t step)
+{
+    if (n < 1 || k < 1 || k > n || n > INT32_MAX) return OR_ERR_ARG;
+    float* v = (float*)malloc((size_t)n * sizeof(float));
+    or_pair* pairs = (or_pair*)malloc((size_t)n * sizeof(or_pair));
+    if (!v || !pairs) { free(v); free(pairs); return OR_ERR_NOMEM; }
+    uint64_t base = or_randk_base(seed, 0, worker, layer, step);
+    for (int64_t i = 0; i < n; ++i) {
+        v[i] = or_residual(m[i], eta, g[i]);
+        pairs[i].key = or_randk_key(base, i);
+        pairs[i].idx = (int32_t)i;
+    }
+    qsort(pairs, (size_t)n, sizeof(or_pair), or_cmp_key_asc);
+    or_emit_selected(n, k, v, pairs, m, vals, idx);
+    free(v);
+    free(pairs);
+    return OR_OK;
+}
+
+/* Uncompressed (1-D) layer: the payload is v itself and the memory empties. */
+int or_dense(int64_t n, float eta, const float* g, float* m, float* payload)
+{
+    if (n < 1) return OR_ERR_ARG;
+    for (int64_t i = 0; i < n; ++i) {
+        payload[i] = or_residual(m[i], eta, g[i]);
+        m[i] = 0.0f;
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* PowerSGD warm-start Q: entries uniform in [-1, 1) drawn from the hash with
+ * stream 1; x = (h >> 40) * 2^-23 - 1, exact in fp32.  Q is cols x r_max,
+ * row-major; element (c, j) uses counter c*r_max + j. */
+int or_powersgd_init_q(int64_t cols, int64_t r_max, uint64_t seed, uint64_t worker,
+                       uint64_t layer, float* Q)
+{
+    if (cols < 1 || r_max < 1) return OR_ERR_ARG;
+    uint64_t base = or_randk_base(seed, 1, worker, layer, 0);
+    for (int64_t c = 0; c < cols; ++c)
+        for (int64_t j = 0; j < r_max; ++j) {
+            uint64_t h = or_splitmix64_output(base, (uint64_t)(c * r_max + j) + 1);
+            Q[c * r_max + j] = (float)(h >> 40) * (1.0f / 8388608.0f) - 1.0f;
+        }
+    return OR_OK;
+}
+
+/*
+ * One PowerSGD rank-r step with error feedback for one worker's matrix.
+ *   g, m      rows x cols row-major fp32; m is read and overwritten with the
+ *             new residual M - P Q'^T
+ *   Q         cols x r_max (row stride r_max); columns 0..r-1 are read as the
+ *             warm start and overwritten with Q' = M^T P; others untouched
+ *   P         rows x r_max (row stride r_max); columns 0..r-1 receive the
+ *             orthonormalised P
+ *   Mhat      optional rows x cols output of the decompressed P Q'^T
+ * Arithmetic after M is formed runs in double and is stored as fp32.
+ */
+int or_powersgd(int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
+                const float* g, float* m, float* Q, float* P, float* Mhat)
+{
+    if (rows < 1 || cols < 1 || r < 1 || r > r_max || r > rows || r > cols)
+        return OR_ERR_ARG;
+    int64_t n = rows * cols;
+    double* M = (double*)malloc((size_t)n * sizeof(double));
+    double* Pd = (double*)malloc((size_t)(rows * r) * sizeof(double));
+    double* Qd = (double*)malloc((size_t)(cols * r) * sizeof(double));
+    if (!M || !Pd || !Qd) { free(M); free(Pd); free(Qd); return OR_ERR_NOMEM; }
+
+    /* M = m + eta*grad, formed exactly as the Mem-SGD residual */
+    for (int64_t i = 0; i < n; ++i) M[i] = (double)or_residual(m[i], eta, g[i]);
+
+    /* P = M Q */
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t j = 0; j < r; ++j) {
+            double s = 0.0;
+            for (int64_t c = 0; c < cols; ++c) s += M[a * cols + c] * (double)Q[c * r_max + j];
+            Pd[a * r + j] = s;
+        }
+
+    /* modified Gram-Schmidt over the columns of P, in order 0..r-1 */
+    for (int64_t j = 0; j < r; ++j) {
+        for (int64_t i = 0; i < j; ++i) {
+            double d = 0.0;
+            for (int64_t a = 0; a < rows; ++a) d += Pd[a * r + i] * Pd[a * r + j];
+            for (int64_t a = 0; a < rows; ++a) Pd[a * r + j] -= d * Pd[a * r + i];
+        }
+        double nn = 0.0;
+        for (int64_t a = 0; a < rows; ++a) nn += Pd[a * r + j] * Pd[a * r + j];
+        double nu = sqrt(nn);
+        for (int64_t a = 0; a < rows; ++a) Pd[a * r + j] = nu > 0.0 ? Pd[a * r + j] / nu : 0.0;
+    }
+
+    /* Q' = M^T P */
+    for (int64_t c = 0; c < cols; ++c)
+        for (int64_t j = 0; j < r; ++j) {
+            double s = 0.0;
+            for (int64_t a = 0; a < rows; ++a) s += M[a * cols + c] * Pd[a * r + j];
+            Qd[c * r + j] = s;
+        }
+
+    /* decompress P Q'^T, residual into memory */
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t c = 0; c < cols; ++c) {
+            double s = 0.0;
+            for (int64_t j = 0; j < r; ++j) s += Pd[a * r + j] * Qd[c * r + j];
+            m[a * cols + c] = (float)(M[a * cols + c] - s);
+            if (Mhat) Mhat[a * cols + c] = (float)s;
+        }
+
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t j = 0; j < r; ++j) P[a * r_max + j] = (float)Pd[a * r + j];
+    for (int64_t c = 0; c < cols; ++c)
+        for (int64_t j = 0; j < r; ++j) Q[c * r_max + j] = (float)Qd[c * r + j];
+
+    free(M);
+    free(Pd);
+    free(Qd);
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Accordion [ACC]: L2 norm of one layer's raw gradient, summed in index
+ * order in double. */
+double or_layer_norm(int64_t n, const float* g)
+{
+    double s = 0.0;
+    for (int64_t i = 0; i < n; ++i) s += (double)g[i] * (double)g[i];
+    return sqrt(s);
+}
+
+/*
+ * Accordion decision for one layer at a check step [ACC].
+ *   s_prev < 0 means "no earlier check": the layer is treated as critical.
+ *   rel = |s_prev - s_cur| / s_prev (s_prev == 0: rel = 0 if s_cur == 0,
+ *   else +inf).  rel >= threshold -> LOW (0, l_low: less compression),
+ *   else HIGH (1, l_high: more compression).
+ */
+int32_t or_accordion_decide(double s_prev, double s_cur, double threshold)
+{
+    if (s_prev < 0.0) return 0;
+    double rel;
+    if (s_prev == 0.0) rel = (s_cur == 0.0) ? 0.0 : INFINITY;
+    else rel = fabs(s_prev - s_cur) / s_prev;
+    return rel >= threshold ? 0 : 1;
+}
+
+/* ------------------------------------------------------------------ */
+/* Decode side [UTIL]: the aggregate of the workers' payloads, summed in worker
+ * order from +0.0 in fp32, then multiplied by `scale`.  These three helpers
+ * add one worker's payload into one layer's slice of the dense output. */
+void or_accum_sparse(int64_t k, const float* vals, const int32_t* idx, float* out)
+{
+    for (int64_t j = 0; j < k; ++j) out[idx[j]] = out[idx[j]] + vals[j];
+}
+
+void or_accum_dense(int64_t n, const float* payload, float* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = out[i] + payload[i];
+}
+
+/* out += P Q^T for one worker (P rows x r, Q cols x r, row stride r_max);
+ * each entry is formed in double and rounded once before the fp32 add. */
+void or_accum_lowrank(int64_t rows, int64_t cols, int64_t r, int64_t r_max,
+                      const float* P, const float* Q, float* out)
+{
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t c = 0; c < cols; ++c) {
+            double s = 0.0;
+            for (int64_t j = 0; j < r; ++j) s += (double)P[a * r_max + j] * (double)Q[c * r_max + j];
+            out[a * cols + c] = out[a * cols + c] + (float)s;
+        }
+}
+
+void or_scale(int64_t n, float scale, float* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = out[i] * scale;
+}
