@@ -1,0 +1,241 @@
+"""Python binding of the gce C ABI (include/gce.h): argument marshalling only.
+
+Every step of the gradient-compression path runs in the native library
+libgce.so (CUDA C++ for sm_100a) built in-tree by
+``python -m gradient_compression_error_b200.build``.  This module converts
+torch CUDA tensors into device pointers and the current CUDA stream into a
+``cudaStream_t``; it computes nothing itself.  If the library is missing the
+first call raises -- there is no fallback.
+
+The entry points keep the C names: ef_topk_step, ef_randk_step,
+powersgd_init_q, powersgd_step, accordion_init, accordion_select,
+decompress_accumulate, plus the Table wrapper of gce_table_* and the
+workspace / status helpers.
+"""
+import ctypes as C
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgce.so")
+
+KIND = {"topk": 0, "randk": 1, "powersgd": 2, "dense": 3}
+KIND_NAME = {v: k for k, v in KIND.items()}
+OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4}
+STATUS_K_RANGE = 1
+STATUS_FALLBACK = 2
+LEVEL_LOW, LEVEL_HIGH = 0, 1
+WS_HEADER_BYTES = 256
+
+ERRORS = {-1: "invalid argument", -2: "CUDA runtime error", -3: "workspace missing or too small",
+          -4: "device allocation failed", -5: "layer kinds do not fit this call"}
+
+
+class GceError(RuntimeError):
+    def __init__(self, fn, code):
+        super().__init__("%s returned %d (%s)" % (fn, code, ERRORS.get(code, "unknown")))
+        self.code = code
+
+
+class LayerDesc(C.Structure):
+    _fields_ = [("rows", C.c_int64), ("cols", C.c_int64), ("kind", C.c_int32), ("cap", C.c_int32)]
+
+
+class LayerInfo(C.Structure):
+    _fields_ = [("offset", C.c_int64), ("n", C.c_int64), ("rows", C.c_int64), ("cols", C.c_int64),
+                ("kind", C.c_int32), ("cap", C.c_int32), ("val_offset", C.c_int64),
+                ("p_offset", C.c_int64), ("q_offset", C.c_int64)]
+
+
+class Totals(C.Structure):
+    _fields_ = [("L", C.c_int64), ("N", C.c_int64), ("vals_per_worker", C.c_int64),
+                ("P_per_worker", C.c_int64), ("Q_per_worker", C.c_int64),
+                ("compressed_kind", C.c_int32)]
+
+
+# exported symbol -> (restype, argtypes); the full list the header declares
+_vp, _i32, _i64, _u64, _f32, _f64 = (C.c_void_p, C.c_int32, C.c_int64, C.c_uint64, C.c_float,
+                                     C.c_double)
+SIGNATURES = {
+    "gce_table_create": (C.c_int, [C.POINTER(LayerDesc), _i32, C.POINTER(_vp)]),
+    "gce_table_destroy": (C.c_int, [_vp]),
+    "gce_table_get_totals": (C.c_int, [_vp, C.POINTER(Totals)]),
+    "gce_table_get_layer": (C.c_int, [_vp, _i32, C.POINTER(LayerInfo)]),
+    "gce_workspace_bytes": (C.c_int, [_vp, _i32, _i32, C.POINTER(C.c_size_t)]),
+    "ef_topk_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, C.c_size_t, _vp]),
+    "ef_randk_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _u64, _u64, _vp, _vp, _vp,
+                                C.c_size_t, _vp]),
+    "powersgd_init_q": (C.c_int, [_vp, _i32, _u64, _vp, _vp]),
+    "powersgd_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                C.c_size_t, _vp]),
+    "accordion_init": (C.c_int, [_vp, _vp, _vp, _vp]),
+    "accordion_select": (C.c_int, [_vp, _vp, _i64, _i32, _f64, _i32, _i32, _vp, _vp, _vp, _vp,
+                                   _vp, C.c_size_t, _vp]),
+    "decompress_accumulate": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
+                                        C.c_size_t, _vp]),
+    "gce_status": (C.c_int, [_vp, _vp, C.POINTER(_i32)]),
+    "gce_launch_count": (_u64, []),
+    "gce_error_string": (C.c_char_p, [C.c_int]),
+    "gce_set_bracket_sigma": (C.c_int, [_f64]),
+}
+
+_lib = None
+
+
+def lib():
+    """Load libgce.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libgce.so is not built; run "
+                               "`python -m gradient_compression_error_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise GceError(fn, rc)
+
+
+def _ptr(t, dtype=None):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("expected a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("expected dtype %s, got %s" % (dtype, t.dtype))
+    return C.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+class Table:
+    """A gce_table: layers described by dicts {rows, cols, kind, cap}."""
+
+    def __init__(self, layers):
+        self.layers = [dict(l) for l in layers]
+        arr = (LayerDesc * len(layers))()
+        for i, l in enumerate(layers):
+            arr[i] = LayerDesc(int(l["rows"]), int(l["cols"]), KIND[l["kind"]], int(l.get("cap", 0)))
+        h = C.c_void_p()
+        _check("gce_table_create", lib().gce_table_create(arr, len(layers), C.byref(h)))
+        self.handle = h
+        tot = Totals()
+        _check("gce_table_get_totals", lib().gce_table_get_totals(h, C.byref(tot)))
+        self.L, self.N = tot.L, tot.N
+        self.vals_per_worker = tot.vals_per_worker
+        self.P_per_worker, self.Q_per_worker = tot.P_per_worker, tot.Q_per_worker
+        self.compressed_kind = tot.compressed_kind
+        self.info = []
+        for i in range(len(layers)):
+            li = LayerInfo()
+            _check("gce_table_get_layer", lib().gce_table_get_layer(h, i, C.byref(li)))
+            self.info.append({f: getattr(li, f) for f, _ in LayerInfo._fields_})
+
+    def close(self):
+        if self.handle is not None and self.handle.value:
+            lib().gce_table_destroy(self.handle)
+        self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def workspace_bytes(self, W, op):
+        n = C.c_size_t()
+        _check("gce_workspace_bytes", lib().gce_workspace_bytes(self.handle, int(W), OP[op],
+                                                                C.byref(n)))
+        return n.value
+
+    def workspace(self, W, op, device="cuda"):
+        """A zero-filled uint8 CUDA tensor of the size the operation needs."""
+        import torch
+        return torch.zeros(max(self.workspace_bytes(W, op), WS_HEADER_BYTES), dtype=torch.uint8,
+                           device=device)
+
+
+def _f32():
+    import torch
+    return torch.float32
+
+
+def _i32():
+    import torch
+    return torch.int32
+
+
+def ef_topk_step(table, W, grad, mem, eta, k_or_rank, vals, idx, ws, stream=None):
+    _check("ef_topk_step", lib().ef_topk_step(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), _ptr(vals, _f32()), _ptr(idx, _i32()), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def ef_randk_step(table, W, grad, mem, eta, k_or_rank, seed, step, vals, idx, ws, stream=None):
+    _check("ef_randk_step", lib().ef_randk_step(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), int(seed), int(step), _ptr(vals, _f32()), _ptr(idx, _i32()),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def powersgd_init_q(table, W, seed, Q, stream=None):
+    _check("powersgd_init_q", lib().powersgd_init_q(table.handle, int(W), int(seed),
+                                                    _ptr(Q, _f32()), _stream(stream)))
+
+
+def powersgd_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, dense_out, ws, stream=None):
+    _check("powersgd_step", lib().powersgd_step(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), _ptr(P, _f32()), _ptr(Q, _f32()), _ptr(vals, _f32()),
+        _ptr(dense_out, _f32()), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def accordion_init(table, prev_norm, level, stream=None):
+    import torch
+    _check("accordion_init", lib().accordion_init(table.handle, _ptr(prev_norm, torch.float64),
+                                                  _ptr(level, _i32()), _stream(stream)))
+
+
+def accordion_select(table, grad, step, interval, threshold, lvl_low, lvl_high, prev_norm, level,
+                     cur_norm, k_or_rank_out, ws, stream=None):
+    import torch
+    _check("accordion_select", lib().accordion_select(
+        table.handle, _ptr(grad, _f32()), int(step), int(interval), float(threshold),
+        int(lvl_low), int(lvl_high), _ptr(prev_norm, torch.float64), _ptr(level, _i32()),
+        _ptr(cur_norm, torch.float64), _ptr(k_or_rank_out, _i32()), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def decompress_accumulate(table, W, vals, idx, k_or_rank, P, Q, scale, out, ws, stream=None):
+    _check("decompress_accumulate", lib().decompress_accumulate(
+        table.handle, int(W), _ptr(vals, _f32()), _ptr(idx, _i32()), _ptr(k_or_rank, _i32()),
+        _ptr(P, _f32()), _ptr(Q, _f32()), float(scale), _ptr(out, _f32()), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def status(ws, stream=None):
+    """Wait for the stream, then read and clear the workspace status word."""
+    st = C.c_int32()
+    _check("gce_status", lib().gce_status(_ptr(ws), _stream(stream), C.byref(st)))
+    return st.value
+
+
+def launch_count():
+    return int(lib().gce_launch_count())
+
+
+def set_bracket_sigma(sigma):
+    _check("gce_set_bracket_sigma", lib().gce_set_bracket_sigma(float(sigma)))

@@ -1,0 +1,132 @@
+// common.cuh -- shared internals of the gce library (sm_100a): the layer
+// table, workspace carving, launch accounting and small device helpers.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+#include <vector>
+
+#include "gce.h"
+
+namespace gce {
+
+constexpr int kMaxRank = 4;
+
+// Device copy of one layer.  Offsets are in elements (grad/mem), slots
+// (vals/idx) or floats (P, Q) per worker.
+struct DevLayer {
+    int64_t offset, n, rows, cols;
+    int64_t val_off, p_off, q_off;
+    int64_t sp_off;  // offset among the compressed layers' elements (spill slots)
+    int32_t kind, cap;
+    int32_t tile0, ntiles;  // top-k / rand-k main tiles of this layer, per worker
+    int32_t sidx;           // index among compressed layers, -1 for DENSE
+    int32_t dc_tile0;       // first decode tile of this layer (all layers, per table)
+    int32_t dc_ntiles;      // decode tiles of this layer
+    int32_t dc_base;        // first slot of this layer's ntiles+1 tile bounds
+};
+
+}  // namespace gce
+
+struct gce_table {
+    int32_t L = 0;
+    int64_t N = 0, vals_pw = 0, P_pw = 0, Q_pw = 0;
+    int32_t ckind = -1;
+    std::vector<gce::DevLayer> layers;     // host copy
+    gce::DevLayer* d_layers = nullptr;
+    std::vector<int32_t> comp;             // compressed layer ids, in order
+    std::vector<int32_t> dense;            // DENSE layer ids
+    int32_t* d_comp = nullptr;
+    int32_t* d_dense = nullptr;
+    int64_t comp_N = 0;                    // elements in compressed layers, per worker
+    int64_t dense_N = 0;
+    int64_t max_comp_n = 0;
+    int32_t tiles_pw = 0;                  // main tiles (compressed layers) per worker
+    int32_t* d_tile_layer = nullptr;       // [tiles_pw] layer of each main tile
+    int32_t sunits_pw = 0;                 // top-k sample units per worker
+    int32_t* d_sunit_layer = nullptr;      // [sunits_pw] layer of each sample unit
+    int32_t* d_sunit_part = nullptr;       // [sunits_pw] part index within the layer
+    int32_t dtiles_pw = 0;                 // dense-layer tiles per worker
+    int32_t* d_dtile_layer = nullptr;
+    int32_t* d_dtile_start = nullptr;      // element start of each dense tile
+    int32_t dc_tiles = 0;                  // decode tiles over all layers
+    int32_t dc_slots = 0;                  // tile-bound slots per worker (tiles + L)
+    int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
+    int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker
+    int32_t* d_bunit_layer = nullptr;
+    int32_t* d_bunit_chunk = nullptr;
+};
+
+namespace gce {
+
+// ---- launch accounting -------------------------------------------------
+extern std::atomic<uint64_t> g_launches;
+
+inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+#define GCE_LAUNCH(kern, grid, block, smem, stream, ...)                        \
+    do {                                                                         \
+        ::gce::count_launch();                                                   \
+        kern<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+    } while (0)
+
+inline int check_launch() {
+    return cudaGetLastError() == cudaSuccess ? GCE_OK : GCE_ERR_CUDA;
+}
+
+// ---- device properties (cached per device) --------------------------------
+int sm_count();
+
+// ---- workspace carving ------------------------------------------------------
+struct Carver {
+    size_t off = GCE_WS_HEADER_BYTES;
+    template <class T>
+    size_t take(size_t count) {
+        size_t o = off;
+        off += (count * sizeof(T) + 255) & ~size_t(255);
+        return o;
+    }
+};
+
+template <class T>
+inline T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- device helpers -----------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__device__ __forceinline__ void set_status(int32_t* status, int32_t bit) {
+    atomicOr(status, bit);
+}
+
+// Mem-SGD residual v = fl32(m + fl32(eta*g)): explicit round-to-nearest
+// multiply then add, never contracted into an FMA.
+__device__ __forceinline__ float residual(float m, float eta, float g) {
+    return __fadd_rn(m, __fmul_rn(eta, g));
+}
+
+// |v| ordering key: the float's bits with the sign cleared.
+__device__ __forceinline__ uint32_t abs_key(float v) {
+    return __float_as_uint(v) & 0x7FFFFFFFu;
+}
+
+__device__ __forceinline__ float4 ld_stream4(const float* p) {
+    return __ldcs(reinterpret_cast<const float4*>(p));
+}
+
+// host entry points shared between translation units
+constexpr int kDcTileLog = 12;              // decode tile: 4096 output elements
+constexpr int kDcTile = 1 << kDcTileLog;
+constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
+
+int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
+                        float eta, float* vals, cudaStream_t st);
+
+}  // namespace gce

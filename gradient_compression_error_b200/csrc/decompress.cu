@@ -1,0 +1,155 @@
+// decompress.cu -- aggregate of W workers' compressed payloads into one dense
+// fp32 buffer, on sm_100a.
+//
+// "On the Utility of Gradient Compression in Distributed Training Systems",
+// Method / Key results: the workers' compressed gradients are combined
+// (all-reduce for PowerSGD, gather for sparse payloads); here the W data-
+// parallel replicas live in one GPU's HBM and the combination is a sum in
+// worker order from +0.0 with fp32 round-to-nearest adds, times `scale`.
+//
+// Design: each CTA owns one 4096-element tile of the output and accumulates
+// every worker's contribution to it in shared memory, in worker order, then
+// writes the tile once.  Sparse payloads are sorted by index, so a first
+// pass (bounds) turns each (worker, layer) list into per-tile entry ranges
+// by comparing neighbouring indices -- no searching.  DRAM traffic: the
+// payload read once plus one 4-byte write per output element.
+#include "common.cuh"
+
+namespace gce {
+
+size_t decompress_ws_bytes(const gce_table* t, int32_t W) {
+    Carver c;
+    c.take<int32_t>(int64_t(W) * t->dc_slots);
+    return c.off;
+}
+
+__device__ __forceinline__ int32_t layer_k(const DevLayer& L, const int32_t* k_or_rank, int32_t l) {
+    const int32_t k = k_or_rank ? k_or_rank[l] : L.cap;
+    return (k >= 1 && k <= L.cap) ? k : 0;  // out of range: the layer contributes nothing
+}
+
+// bounds[w][L.dc_base + tt] = first payload entry of (w, l) whose index lies in
+// decode tile tt or later; slot ntiles holds k.
+__global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restrict__ layers,
+                                                        const int32_t* __restrict__ bunit_layer,
+                                                        const int32_t* __restrict__ bunit_chunk,
+                                                        int32_t bunits_pw, int32_t W,
+                                                        int64_t vals_pw, int32_t dc_slots,
+                                                        const int32_t* __restrict__ k_or_rank,
+                                                        const int32_t* __restrict__ idx,
+                                                        int32_t* __restrict__ bounds) {
+    const int64_t total = int64_t(bunits_pw) * W;
+    for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
+        const int w = int(u / bunits_pw);
+        const int bu = int(u % bunits_pw);
+        const int32_t l = bunit_layer[bu];
+        const DevLayer L = layers[l];
+        const int32_t k = layer_k(L, k_or_rank, l);
+        int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base;
+        const int32_t nt = L.dc_ntiles;
+        const int64_t j0 = int64_t(bunit_chunk[bu]) * kDcBoundChunk;
+        if (k == 0) {
+            if (j0 == 0)
+                for (int32_t tt = threadIdx.x; tt <= nt; tt += blockDim.x) b[tt] = 0;
+            continue;
+        }
+        const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
+        const int64_t j1 = min64(j0 + kDcBoundChunk, k);
+        for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
+            const int32_t tj = min(max(ix[j], 0) >> kDcTileLog, nt);
+            const int32_t tp = j > 0 ? min(max(ix[j - 1], 0) >> kDcTileLog, nt) : -1;
+            for (int32_t tt = tp + 1; tt <= tj; ++tt) b[tt] = int32_t(j);
+            if (j == k - 1)
+                for (int32_t tt = tj + 1; tt <= nt; ++tt) b[tt] = k;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) dc_accum_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
+    int32_t dc_tiles, int32_t W, int64_t vals_pw, int64_t P_pw, int64_t Q_pw, int32_t dc_slots,
+    const int32_t* __restrict__ k_or_rank, const float* __restrict__ vals,
+    const int32_t* __restrict__ idx, const float* __restrict__ P, const float* __restrict__ Q,
+    const int32_t* __restrict__ bounds, float scale, float* __restrict__ out) {
+    __shared__ float acc[kDcTile];
+    for (int32_t t = blockIdx.x; t < dc_tiles; t += gridDim.x) {
+        const int32_t l = dc_tile_layer[t];
+        const DevLayer L = layers[l];
+        const int32_t tt = t - L.dc_tile0;
+        const int64_t start = int64_t(tt) << kDcTileLog;
+        const int cnt = int(min64(kDcTile, L.n - start));
+        float* o = out + L.offset + start;
+        if (L.kind == GCE_KIND_TOPK || L.kind == GCE_KIND_RANDK) {
+            const int32_t k = layer_k(L, k_or_rank, l);
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) acc[i] = 0.0f;
+            for (int w = 0; w < W; ++w) {
+                __syncthreads();
+                const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base + tt;
+                const int32_t a = min(max(b[0], 0), k), e = min(max(b[1], a), k);
+                const float* v = vals + int64_t(w) * vals_pw + L.val_off;
+                const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
+                for (int32_t j = a + threadIdx.x; j < e; j += blockDim.x) {
+                    const int64_t i = int64_t(ix[j]) - start;
+                    if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], v[j]);
+                }
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) o[i] = __fmul_rn(acc[i], scale);
+            __syncthreads();
+        } else if (L.kind == GCE_KIND_DENSE) {
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+                float s = 0.0f;
+                for (int w = 0; w < W; ++w)
+                    s = __fadd_rn(s, vals[int64_t(w) * vals_pw + L.val_off + start + i]);
+                o[i] = __fmul_rn(s, scale);
+            }
+        } else {  // POWERSGD: P Q^T over the first r columns
+            const int32_t r = layer_k(L, k_or_rank, l);
+            const int cap = L.cap;
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+                const int64_t e = start + i;
+                const int64_t row = e / L.cols, col = e - row * L.cols;
+                float s = 0.0f;
+                for (int w = 0; w < W; ++w) {
+                    const float* p = P + int64_t(w) * P_pw + L.p_off + row * cap;
+                    const float* q = Q + int64_t(w) * Q_pw + L.q_off + col * cap;
+                    float m = 0.0f;
+                    if (r > 0) {
+                        m = __fmul_rn(p[0], q[0]);
+                        for (int j = 1; j < r; ++j) m = __fmaf_rn(p[j], q[j], m);
+                    }
+                    s = __fadd_rn(s, m);
+                }
+                o[i] = __fmul_rn(s, scale);
+            }
+        }
+    }
+}
+
+}  // namespace gce
+
+using namespace gce;
+
+extern "C" int decompress_accumulate(const gce_table* t, int32_t W, const float* vals,
+                                     const int32_t* idx, const int32_t* k_or_rank, const float* P,
+                                     const float* Q, float scale, float* out, void* ws,
+                                     size_t ws_bytes, void* stream) {
+    if (!t || W < 1 || !out || !ws || !aligned16(out) || !aligned16(ws)) return GCE_ERR_ARG;
+    const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
+    if ((t->vals_pw > 0 && !vals) || (sparse && !idx)) return GCE_ERR_ARG;
+    if (t->ckind == GCE_KIND_POWERSGD && (!P || !Q)) return GCE_ERR_ARG;
+    if (ws_bytes < decompress_ws_bytes(t, W)) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* bounds = at<int32_t>(ws, GCE_WS_HEADER_BYTES);
+    const int sms = sm_count();
+    if (sparse && t->bunits_pw > 0) {
+        const int64_t units = int64_t(t->bunits_pw) * W;
+        GCE_LAUNCH(dc_bounds_kernel, int(min64(units, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
+                   t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
+                   k_or_rank, idx, bounds);
+    }
+    GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
+               t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots,
+               k_or_rank, vals, idx, P, Q, bounds, scale, out);
+    return check_launch();
+}

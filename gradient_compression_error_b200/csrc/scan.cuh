@@ -1,0 +1,92 @@
+// scan.cuh -- warp / block prefix sums and the radix-bin crossing search.
+#pragma once
+
+#include <cstdint>
+
+namespace gce {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+template <class T>
+__device__ __forceinline__ T warp_inclusive_scan(T x) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        T y = __shfl_up_sync(kFull, x, o);
+        if (lane >= o) x += y;
+    }
+    return x;
+}
+
+template <class T>
+__device__ __forceinline__ T warp_sum(T x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+    return x;
+}
+
+// Exclusive prefix sum over the block (blockDim.x a multiple of 32, <= 1024).
+// s_warp: 33 ints of shared scratch.  Returns the thread's exclusive prefix;
+// *total receives the block total.  Contains __syncthreads (call uniformly).
+__device__ __forceinline__ int block_exclusive_scan(int x, int* s_warp, int* total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    int incl = warp_inclusive_scan(x);
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    if (warp == 0) {
+        int v = lane < nw ? s_warp[lane] : 0;
+        int vi = warp_inclusive_scan(v);
+        if (lane < nw) s_warp[lane] = vi - v;
+        if (lane == 31) s_warp[32] = vi;  // lane 31 holds the block total
+    }
+    __syncthreads();
+    int res = s_warp[warp] + incl - x;
+    *total = s_warp[32];
+    __syncthreads();
+    return res;
+}
+
+// Run by one full warp.  h: nb >= 32 bins in shared memory, nb % 32 == 0.
+// Finds the bin b with above(b) < target <= above(b) + h[b], where above(b)
+// is the sum of all bins above b (the crossing of the count taken from the
+// top).  Returns -1 when the total is below target.  *above_out = above(b).
+__device__ __forceinline__ int warp_find_from_top(const int32_t* h, int nb, int64_t target,
+                                                  int64_t* above_out) {
+    const int lane = threadIdx.x & 31;
+    const int per = nb >> 5;
+    int64_t mine = 0;
+    for (int i = 0; i < per; ++i) mine += h[lane * per + i];
+    // inclusive suffix sum over lanes (this lane and every higher one)
+    int64_t incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int64_t y = __shfl_down_sync(kFull, incl, o);
+        if (lane + o < 32) incl += y;
+    }
+    const int64_t excl = incl - mine;
+    const unsigned ball = __ballot_sync(kFull, excl < target && target <= incl);
+    if (ball == 0) {
+        *above_out = __shfl_sync(kFull, incl, 0);
+        return -1;
+    }
+    const int src = __ffs(ball) - 1;
+    int res = -1;
+    int64_t above = 0;
+    if (lane == src) {
+        int64_t acc = excl;
+        for (int b = lane * per + per - 1; b >= lane * per; --b) {
+            if (acc + h[b] >= target) {
+                res = b;
+                above = acc;
+                break;
+            }
+            acc += h[b];
+        }
+    }
+    res = __shfl_sync(kFull, res, src);
+    above = __shfl_sync(kFull, above, src);
+    *above_out = above;
+    return res;
+}
+
+}  // namespace gce

@@ -1,0 +1,290 @@
+// table.cu -- layer table, workspace queries, status word, launch counter,
+// and the kernel for uncompressed (DENSE) layers shared by every step.
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "topk_layout.cuh"
+
+namespace gce {
+
+std::atomic<uint64_t> g_launches{0};
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// ---- DENSE layers: payload = fl32(m + fl32(eta*g)), memory -> +0 ----------
+constexpr int kDenseTile = 4096;
+
+__global__ void __launch_bounds__(256) dense_kernel(const DevLayer* __restrict__ layers,
+                                                    const int32_t* __restrict__ dtile_layer,
+                                                    const int32_t* __restrict__ dtile_start,
+                                                    int32_t dtiles_pw, int32_t W, int64_t N,
+                                                    int64_t vals_pw, const float* __restrict__ grad,
+                                                    float* __restrict__ mem, float eta,
+                                                    float* __restrict__ vals) {
+    const int64_t total = int64_t(dtiles_pw) * W;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+        const int w = int(t / dtiles_pw);
+        const int lt = int(t % dtiles_pw);
+        const DevLayer L = layers[dtile_layer[lt]];
+        const int64_t start = dtile_start[lt];
+        const int64_t cnt = min64(kDenseTile, L.n - start);
+        const float* g = grad + int64_t(w) * N + L.offset + start;
+        float* m = mem + int64_t(w) * N + L.offset + start;
+        float* out = vals + int64_t(w) * vals_pw + L.val_off + start;
+        for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+            out[i] = residual(m[i], eta, __ldcs(g + i));
+            m[i] = 0.0f;
+        }
+    }
+}
+
+int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
+                        float* vals, cudaStream_t st) {
+    if (t->dtiles_pw == 0) return GCE_OK;
+    if (!vals) return GCE_ERR_ARG;
+    int64_t total = int64_t(t->dtiles_pw) * W;
+    int grid = int(min64(total, int64_t(sm_count()) * 8));
+    GCE_LAUNCH(dense_kernel, grid, 256, 0, st, t->d_layers, t->d_dtile_layer, t->d_dtile_start,
+               t->dtiles_pw, W, t->N, t->vals_pw, grad, mem, eta, vals);
+    return check_launch();
+}
+
+}  // namespace gce
+
+using namespace gce;
+
+static void free_table(gce_table* t) {
+    if (!t) return;
+    cudaFree(t->d_layers);
+    cudaFree(t->d_comp);
+    cudaFree(t->d_dense);
+    cudaFree(t->d_tile_layer);
+    cudaFree(t->d_sunit_layer);
+    cudaFree(t->d_sunit_part);
+    cudaFree(t->d_dtile_layer);
+    cudaFree(t->d_dtile_start);
+    cudaFree(t->d_dc_tile_layer);
+    cudaFree(t->d_bunit_layer);
+    cudaFree(t->d_bunit_chunk);
+    delete t;
+}
+
+template <class T>
+static int upload(T** dst, const std::vector<T>& src) {
+    *dst = nullptr;
+    if (src.empty()) return GCE_OK;
+    if (cudaMalloc(dst, src.size() * sizeof(T)) != cudaSuccess) return GCE_ERR_NOMEM;
+    if (cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice) != cudaSuccess)
+        return GCE_ERR_CUDA;
+    return GCE_OK;
+}
+
+extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_table** out) {
+    if (!descs || !out || L < 1) return GCE_ERR_ARG;
+    *out = nullptr;
+    gce_table* t = new gce_table();
+    t->L = L;
+    int64_t off = 0, voff = 0, poff = 0, qoff = 0, spoff = 0;
+    int32_t tiles = 0;
+    std::vector<int32_t> tile_layer, sunit_layer, sunit_part, dtile_layer, dtile_start;
+    std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk;
+    int32_t dc_tiles = 0, dc_slots = 0;
+    for (int32_t l = 0; l < L; ++l) {
+        const gce_layer_desc& d = descs[l];
+        const int64_t n = d.rows * d.cols;
+        if (d.rows < 1 || d.cols < 1 || n > INT32_MAX || d.kind < 0 || d.kind > GCE_KIND_DENSE) {
+            delete t;
+            return GCE_ERR_ARG;
+        }
+        DevLayer x{};
+        x.offset = off;
+        x.n = n;
+        x.rows = d.rows;
+        x.cols = d.cols;
+        x.kind = d.kind;
+        x.cap = d.cap;
+        x.val_off = x.p_off = x.q_off = -1;
+        x.sp_off = -1;
+        x.sidx = -1;
+        if (d.kind == GCE_KIND_TOPK || d.kind == GCE_KIND_RANDK) {
+            if (d.cap < 1 || d.cap > n) { delete t; return GCE_ERR_ARG; }
+            x.val_off = voff;
+            voff += (d.cap + 3) & ~int64_t(3);  // keep every slice 16-byte aligned
+        } else if (d.kind == GCE_KIND_POWERSGD) {
+            if (d.cap < 1 || d.cap > kMaxRank || d.cap > d.rows || d.cap > d.cols) {
+                delete t;
+                return GCE_ERR_ARG;
+            }
+            x.p_off = poff;
+            x.q_off = qoff;
+            poff += (d.rows * d.cap + 3) & ~int64_t(3);
+            qoff += (d.cols * d.cap + 3) & ~int64_t(3);
+        } else {  // DENSE
+            x.val_off = voff;
+            voff += (n + 3) & ~int64_t(3);
+            for (int64_t s = 0; s < n; s += kDenseTile) {
+                dtile_layer.push_back(l);
+                dtile_start.push_back(int32_t(s));
+            }
+            t->dense.push_back(l);
+            t->dense_N += n;
+        }
+        if (d.kind != GCE_KIND_DENSE) {
+            if (t->ckind >= 0 && t->ckind != d.kind) { delete t; return GCE_ERR_KIND; }
+            t->ckind = d.kind;
+            x.sidx = int32_t(t->comp.size());
+            x.sp_off = spoff;
+            spoff += n;
+            t->comp.push_back(l);
+            t->max_comp_n = std::max(t->max_comp_n, n);
+            if (d.kind != GCE_KIND_POWERSGD) {
+                x.tile0 = tiles;
+                x.ntiles = int32_t((n + kTkTile - 1) / kTkTile);
+                for (int32_t i = 0; i < x.ntiles; ++i) tile_layer.push_back(l);
+                tiles += x.ntiles;
+                if (n >= kTkSampleMinN) {
+                    int32_t parts = int32_t((n + kTkSamplePart - 1) / kTkSamplePart);
+                    for (int32_t p = 0; p < parts; ++p) {
+                        sunit_layer.push_back(l);
+                        sunit_part.push_back(p);
+                    }
+                }
+            }
+        }
+        x.dc_tile0 = dc_tiles;
+        x.dc_ntiles = int32_t((n + kDcTile - 1) / kDcTile);
+        x.dc_base = dc_slots;
+        for (int32_t i = 0; i < x.dc_ntiles; ++i) dc_tile_layer.push_back(l);
+        dc_tiles += x.dc_ntiles;
+        dc_slots += x.dc_ntiles + 1;
+        if (d.kind == GCE_KIND_TOPK || d.kind == GCE_KIND_RANDK) {
+            const int32_t chunks = (d.cap + kDcBoundChunk - 1) / kDcBoundChunk;
+            for (int32_t c = 0; c < chunks; ++c) {
+                bunit_layer.push_back(l);
+                bunit_chunk.push_back(c);
+            }
+        }
+        off += n;
+        t->layers.push_back(x);
+    }
+    t->N = off;
+    t->vals_pw = voff;
+    t->P_pw = poff;
+    t->Q_pw = qoff;
+    t->comp_N = spoff;
+    t->tiles_pw = tiles;
+    t->sunits_pw = int32_t(sunit_layer.size());
+    t->dtiles_pw = int32_t(dtile_layer.size());
+    t->dc_tiles = dc_tiles;
+    t->dc_slots = dc_slots;
+    t->bunits_pw = int32_t(bunit_layer.size());
+    int rc = GCE_OK;
+    if (rc == GCE_OK) rc = upload(&t->d_layers, t->layers);
+    if (rc == GCE_OK) rc = upload(&t->d_comp, t->comp);
+    if (rc == GCE_OK) rc = upload(&t->d_dense, t->dense);
+    if (rc == GCE_OK) rc = upload(&t->d_tile_layer, tile_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_sunit_layer, sunit_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_sunit_part, sunit_part);
+    if (rc == GCE_OK) rc = upload(&t->d_dtile_layer, dtile_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_dtile_start, dtile_start);
+    if (rc == GCE_OK) rc = upload(&t->d_dc_tile_layer, dc_tile_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_bunit_layer, bunit_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_bunit_chunk, bunit_chunk);
+    if (rc != GCE_OK) {
+        free_table(t);
+        return rc;
+    }
+    *out = t;
+    return GCE_OK;
+}
+
+extern "C" int gce_table_destroy(gce_table* t) {
+    if (!t) return GCE_ERR_ARG;
+    free_table(t);
+    return GCE_OK;
+}
+
+extern "C" int gce_table_get_totals(const gce_table* t, gce_table_totals* out) {
+    if (!t || !out) return GCE_ERR_ARG;
+    out->L = t->L;
+    out->N = t->N;
+    out->vals_per_worker = t->vals_pw;
+    out->P_per_worker = t->P_pw;
+    out->Q_per_worker = t->Q_pw;
+    out->compressed_kind = t->ckind;
+    return GCE_OK;
+}
+
+extern "C" int gce_table_get_layer(const gce_table* t, int32_t l, gce_layer_info* out) {
+    if (!t || !out || l < 0 || l >= t->L) return GCE_ERR_ARG;
+    const DevLayer& x = t->layers[l];
+    out->offset = x.offset;
+    out->n = x.n;
+    out->rows = x.rows;
+    out->cols = x.cols;
+    out->kind = x.kind;
+    out->cap = x.cap;
+    out->val_offset = x.val_off;
+    out->p_offset = x.p_off;
+    out->q_offset = x.q_off;
+    return GCE_OK;
+}
+
+namespace gce {
+size_t topk_ws_bytes(const gce_table* t, int32_t W);
+size_t randk_ws_bytes(const gce_table* t, int32_t W);
+size_t powersgd_ws_bytes(const gce_table* t, int32_t W);
+size_t accordion_ws_bytes(const gce_table* t);
+size_t decompress_ws_bytes(const gce_table* t, int32_t W);
+}  // namespace gce
+
+extern "C" int gce_workspace_bytes(const gce_table* t, int32_t W, int32_t op, size_t* bytes) {
+    if (!t || !bytes || W < 1) return GCE_ERR_ARG;
+    switch (op) {
+        case GCE_OP_TOPK: *bytes = topk_ws_bytes(t, W); break;
+        case GCE_OP_RANDK: *bytes = randk_ws_bytes(t, W); break;
+        case GCE_OP_POWERSGD: *bytes = powersgd_ws_bytes(t, W); break;
+        case GCE_OP_ACCORDION: *bytes = accordion_ws_bytes(t); break;
+        case GCE_OP_DECOMPRESS: *bytes = decompress_ws_bytes(t, W); break;
+        default: return GCE_ERR_ARG;
+    }
+    return GCE_OK;
+}
+
+extern "C" int gce_status(void* ws, void* stream, int32_t* status) {
+    if (!ws || !status) return GCE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t h = 0;
+    if (cudaMemcpyAsync(&h, ws, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return GCE_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof h, st) != cudaSuccess) return GCE_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return GCE_ERR_CUDA;
+    *status = h;
+    return GCE_OK;
+}
+
+extern "C" uint64_t gce_launch_count(void) { return g_launches.load(); }
+
+extern "C" const char* gce_error_string(int code) {
+    switch (code) {
+        case GCE_OK: return "ok";
+        case GCE_ERR_ARG: return "invalid argument";
+        case GCE_ERR_CUDA: return "CUDA runtime error";
+        case GCE_ERR_WORKSPACE: return "workspace missing or too small";
+        case GCE_ERR_NOMEM: return "device allocation failed";
+        case GCE_ERR_KIND: return "layer kinds do not fit this call";
+        default: return "unknown error";
+    }
+}

@@ -1,0 +1,253 @@
+/*
+ * gce.h -- C ABI of the B200 (sm_100a) gradient-compression library:
+ * error-feedback top-k / rand-k (Mem-SGD), PowerSGD with a warm-started Q,
+ * Accordion's per-layer level switch, and the on-device aggregate of the
+ * compressed payloads of W data-parallel worker replicas.
+ *
+ * Sources (page title, section):
+ *   [MEM]  "Sparsified SGD with Memory", Method: the error-feedback update
+ *            g_t = comp_k(m_t + eta*grad),  m_{t+1} = m_t + eta*grad - g_t,
+ *          comp_k a k-contraction (top-k keeps the largest entries, rand-k
+ *          random ones: Abstract); Key results: 0 < k <= d.
+ *   [ACC]  "Accordion: Adaptive Gradient Communication via Critical Learning
+ *          Regime Identification", Method: the per-layer rate of change of
+ *          the gradient norm selects the low-compression level l_low inside
+ *          critical regimes and the high-compression level l_high outside.
+ *   [UTIL] "On the Utility of Gradient Compression in Distributed Training
+ *          Systems", Method / Key results: PowerSGD (rank r) is all-reduce
+ *          compatible; the encode-decode latency is what limits speedups.
+ *   PowerSGD's steps are not printed on the pages; this library implements
+ *   the standard single power-iteration step with a reused Q:
+ *   P = M Q, orthonormalise P (modified Gram-Schmidt), Q' = M^T P,
+ *   decompress P Q'^T, residual M - P Q'^T into memory.
+ *
+ * Conventions shared by every call:
+ *   - Pointers named grad, mem, vals, idx, P, Q, out, k_or_rank, prev_norm,
+ *     level, cur_norm and ws are DEVICE pointers owned by the caller; they
+ *     must be 16-byte aligned.  The library never allocates during a step
+ *     (only gce_table_create allocates, once).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every step call is asynchronous on that stream; a return of
+ *     GCE_OK means the work was enqueued.  Host-detectable errors return a
+ *     negative GCE_ERR_* before anything is enqueued; errors found on the
+ *     device set bits in the workspace status word (gce_status).  No call
+ *     aborts, throws or prints.
+ *   - Layout: W workers' buffers are stacked.  grad and mem are
+ *     [W][N] fp32; layer l of worker w starts at w*N + info.offset and is
+ *     rows x cols row-major.  Sparse payloads of (w, l) are vals/idx at
+ *     w*vals_per_worker + info.val_offset, k entries in ascending index
+ *     (layer-local int32); an uncompressed (DENSE) layer's payload is its n
+ *     values at the same place.  PowerSGD P of (w, l) is rows x r_max at
+ *     w*P_per_worker + info.p_offset and Q is cols x r_max at
+ *     w*Q_per_worker + info.q_offset (row stride r_max; rank r uses
+ *     columns 0..r-1 and leaves the others untouched).
+ *   - Inputs must be finite (NaN has no |v| order).
+ *   - Calls that share a workspace must not overlap on the GPU.
+ */
+#ifndef GCE_H
+#define GCE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GCE_API __attribute__((visibility("default")))
+#else
+#define GCE_API
+#endif
+
+/* return codes */
+#define GCE_OK 0
+#define GCE_ERR_ARG (-1)       /* bad argument (NULL, misaligned, out of range) */
+#define GCE_ERR_CUDA (-2)      /* a CUDA runtime call failed                     */
+#define GCE_ERR_WORKSPACE (-3) /* ws NULL or smaller than gce_workspace_bytes   */
+#define GCE_ERR_NOMEM (-4)     /* gce_table_create could not allocate           */
+#define GCE_ERR_KIND (-5)      /* the table's layer kinds do not fit this call  */
+
+/* device status bits, read with gce_status */
+#define GCE_STATUS_K_RANGE 1    /* a per-layer k / rank was out of range: layer skipped   */
+#define GCE_STATUS_FALLBACK 2   /* informational: an exact fallback path ran              */
+
+/* layer kinds */
+#define GCE_KIND_TOPK 0
+#define GCE_KIND_RANDK 1
+#define GCE_KIND_POWERSGD 2
+#define GCE_KIND_DENSE 3 /* sent uncompressed: payload = m + eta*grad, memory -> 0 */
+
+/* operations, for gce_workspace_bytes */
+#define GCE_OP_TOPK 0
+#define GCE_OP_RANDK 1
+#define GCE_OP_POWERSGD 2
+#define GCE_OP_ACCORDION 3
+#define GCE_OP_DECOMPRESS 4
+
+/* Accordion levels [ACC] */
+#define GCE_LEVEL_LOW 0  /* l_low: less compression (critical regime) */
+#define GCE_LEVEL_HIGH 1 /* l_high: more compression                 */
+
+typedef struct gce_table gce_table;
+
+/* One layer as the caller describes it.  cap: for TOPK / RANDK the largest k
+ * any step will use (payload slots, 1 <= cap <= rows*cols); for POWERSGD the
+ * largest rank r_max (1..4, <= min(rows, cols)); ignored for DENSE. */
+typedef struct gce_layer_desc {
+    int64_t rows;
+    int64_t cols; /* 1 for a 1-D layer */
+    int32_t kind;
+    int32_t cap;
+} gce_layer_desc;
+
+typedef struct gce_layer_info {
+    int64_t offset;     /* first element in a worker's flat buffer         */
+    int64_t n;          /* rows * cols                                     */
+    int64_t rows, cols;
+    int32_t kind, cap;
+    int64_t val_offset; /* vals/idx slot start (sparse, DENSE); -1 otherwise */
+    int64_t p_offset;   /* POWERSGD only; -1 otherwise                     */
+    int64_t q_offset;   /* POWERSGD only; -1 otherwise                     */
+} gce_layer_info;
+
+typedef struct gce_table_totals {
+    int64_t L;
+    int64_t N;               /* elements per worker                         */
+    int64_t vals_per_worker; /* floats (and int32 idx slots) per worker     */
+    int64_t P_per_worker;    /* floats                                      */
+    int64_t Q_per_worker;    /* floats                                      */
+    int32_t compressed_kind; /* TOPK / RANDK / POWERSGD, or -1 if all DENSE */
+} gce_table_totals;
+
+/*
+ * Build a layer table: copies `descs` (host, L entries) and uploads the
+ * device-side copy.  A table holds at most one compressed kind (TOPK, RANDK
+ * or POWERSGD) plus any number of DENSE layers.  Allocates device memory
+ * once; *out is owned by the caller and released with gce_table_destroy.
+ * Errors: GCE_ERR_ARG (L < 1, a bad shape or cap, n > 2^31-1 per layer),
+ * GCE_ERR_KIND (two compressed kinds), GCE_ERR_NOMEM / GCE_ERR_CUDA.
+ */
+GCE_API int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_table** out);
+GCE_API int gce_table_destroy(gce_table* table);
+GCE_API int gce_table_get_totals(const gce_table* table, gce_table_totals* out);
+GCE_API int gce_table_get_layer(const gce_table* table, int32_t l, gce_layer_info* out);
+
+/* Bytes of device workspace an operation needs for W workers (>= 1).  The
+ * caller allocates it once; its first GCE_WS_HEADER_BYTES hold the status
+ * word and must be zero before first use.  The same workspace may be reused
+ * by every call on the same table and W (never by two calls at once). */
+#define GCE_WS_HEADER_BYTES 256
+GCE_API int gce_workspace_bytes(const gce_table* table, int32_t W, int32_t op, size_t* bytes);
+
+/*
+ * Mem-SGD top-k step [MEM] for every (worker, TOPK layer), plus DENSE layers.
+ *   v = fl32(mem + fl32(eta * grad))      (two roundings, no FMA)
+ *   chosen set S: the k largest |v| (|v| ordered by the float's bits with
+ *   the sign cleared), equal |v| -> lower index first;
+ *   vals/idx <- (v_i, i) for i in S, ascending i;  mem <- v, and +0.0 on S.
+ * grad [W][N] read; mem [W][N] read and written; k_or_rank: device int32[L]
+ * with k per layer (1 <= k <= cap), or NULL for k = cap; entries of non-TOPK
+ * layers are ignored.  vals / idx: [W][vals_per_worker].  Results are
+ * bit-exact and independent of the launch configuration.
+ * A layer whose k is out of range is skipped and sets GCE_STATUS_K_RANGE.
+ */
+GCE_API int ef_topk_step(const gce_table* table, int32_t W, const float* grad, float* mem,
+                 float eta, const int32_t* k_or_rank, float* vals, int32_t* idx,
+                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Mem-SGD rand-k step [MEM]: as ef_topk_step, but S is the k coordinates with
+ * the smallest (key, index), key_i = high 32 bits of output i+1 of a
+ * SplitMix64 generator (Steele, Lea, Flood 2014) whose state is derived from
+ * (seed, stream 0, worker, layer, step) by successive SplitMix64 outputs; the
+ * chosen values are sent unscaled (comp_k stays a k-contraction).
+ */
+GCE_API int ef_randk_step(const gce_table* table, int32_t W, const float* grad, float* mem,
+                  float eta, const int32_t* k_or_rank, uint64_t seed, uint64_t step,
+                  float* vals, int32_t* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Initial (warm-start) Q for every (worker, POWERSGD layer): entries
+ * (h >> 40) * 2^-23 - 1 in [-1, 1), h the SplitMix64 output c*r_max + j + 1
+ * from the state of (seed, stream 1, worker, layer, step 0).  Q: [W][Q_per_worker].
+ */
+GCE_API int powersgd_init_q(const gce_table* table, int32_t W, uint64_t seed, float* Q,
+                    void* stream);
+
+/*
+ * PowerSGD rank-r step with error feedback for every (worker, POWERSGD layer),
+ * plus DENSE layers (payload to vals, memory -> 0):
+ *   M = fl32(mem + fl32(eta*grad)); P = M Q (warm start); P <- orthonormal
+ *   columns by modified Gram-Schmidt in column order (a zero column stays 0);
+ *   Q <- M^T P; mem <- M - P Q^T; dense_out (optional) <- P Q^T.
+ * k_or_rank: device int32[L] rank per layer (1 <= r <= cap) or NULL for
+ * r = cap.  P [W][P_per_worker] written; Q [W][Q_per_worker] read and
+ * written; vals [W][vals_per_worker] receives DENSE payloads (may be NULL if
+ * the table has no DENSE layer); dense_out [W][N] or NULL.  fp32 with fp64
+ * reductions; deterministic for a given table.
+ */
+GCE_API int powersgd_step(const gce_table* table, int32_t W, const float* grad, float* mem,
+                  float eta, const int32_t* k_or_rank, float* P, float* Q, float* vals,
+                  float* dense_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Accordion select [ACC] over every compressed layer of the table.
+ * Sets prev_norm[l] = -1 (no earlier check) and level[l] = LOW.
+ */
+GCE_API int accordion_init(const gce_table* table, double* prev_norm, int32_t* level, void* stream);
+/*
+ * grad: device fp32 [N] (one gradient, e.g. one worker's or an aggregate).
+ * If step % interval == 0 (a check step): s_l = sqrt(sum grad_i^2) per
+ * compressed layer (fp64 accumulation, fixed order), cur_norm[l] = s_l,
+ * rel = |prev - s_l| / prev (prev == 0: 0 if s_l == 0 else +inf),
+ * level[l] = (prev < 0 || rel >= threshold) ? LOW : HIGH, prev_norm[l] = s_l.
+ * Every step: k_or_rank_out[l] = the level's parameter -- for POWERSGD
+ * layers the rank lvl_low / lvl_high, for TOPK / RANDK layers
+ * k = max(1, floor(n * ppm / 1e6)) with ppm = lvl_low / lvl_high (parts per
+ * million of the layer); DENSE layers get 0.  lvl_low / lvl_high are host
+ * values.  prev_norm, cur_norm: device double[L]; level, k_or_rank_out:
+ * device int32[L].
+ */
+GCE_API int accordion_select(const gce_table* table, const float* grad, int64_t step,
+                     int32_t interval, double threshold, int32_t lvl_low, int32_t lvl_high,
+                     double* prev_norm, int32_t* level, double* cur_norm,
+                     int32_t* k_or_rank_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Aggregate [UTIL] of the W workers' payloads into a dense fp32 out [N]:
+ *   out = scale * sum_{w = 0..W-1} decode(payload_w), summed in worker order
+ *   from +0.0 with fp32 round-to-nearest adds, the product taken last.
+ * decode: sparse layers scatter vals at idx (first k entries); DENSE layers
+ * take their n values; POWERSGD layers P Q^T over the first r columns (each
+ * entry formed with fp32 FMAs in column order).  k_or_rank as for the step
+ * that produced the payloads (NULL = cap).  P/Q may be NULL when the table
+ * has no POWERSGD layer, idx when it has no sparse layer.  Sparse and DENSE
+ * results are bit-exact.  Sparse payloads must be in ascending index within
+ * each (worker, layer), as the steps write them.  ws: workspace of
+ * gce_workspace_bytes(GCE_OP_DECOMPRESS) bytes (per-tile entry ranges).
+ */
+GCE_API int decompress_accumulate(const gce_table* table, int32_t W, const float* vals,
+                          const int32_t* idx, const int32_t* k_or_rank, const float* P,
+                          const float* Q, float scale, float* out, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Wait for `stream`, then read and clear the status word of workspace `ws`
+ * (device pointer).  *status receives GCE_STATUS_* bits (0 = clean). */
+GCE_API int gce_status(void* ws, void* stream, int32_t* status);
+
+/* Number of kernels this library has launched since it was loaded. */
+GCE_API uint64_t gce_launch_count(void);
+
+/* Static description of a return code. */
+GCE_API const char* gce_error_string(int code);
+
+/* Tuning knob for the approximate pre-selection of top-k / rand-k: the safety
+ * margin in standard deviations (default 6).  Results never depend on it;
+ * small values only make the exact fallback run more often. */
+GCE_API int gce_set_bracket_sigma(double sigma);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* GCE_H */
