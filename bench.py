@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Benchmark of the gradient-compression hot path on B200: prints ONE JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--profile]
+
+Default workload (bert_base_topk1pct_w8): BERT-base-shaped fp32 gradients
+(109,482,240 elements per worker, 90 tensors) compressed with error-feedback
+top-k at 1 % of every tensor for W = 8 data-parallel worker replicas held in
+one GPU's HBM, and the W sparse payloads summed on the device.  One step =
+ef_topk_step (encode + memory update) + decompress_accumulate (decode), on
+fresh seeded N(0, 1) gradients resident in HBM.  The metric is gradient
+elements encoded+decoded per second (W * N per step); the roofline object
+reports the dominant kernel (the fused residual / memory / candidate pass)
+against the measured HBM copy bandwidth.
+
+Under torchrun (N > 1) every rank runs its own independent replica of the
+workload (the workload's W workers are simulated replicas; there is no data
+exchange between GPUs): value = elements of all ranks / max time over ranks.
+--impl reference times the CPU oracle (plain C, oracle/) on a bounded sample
+of the same workload on the host cores.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gradient elements encoded+decoded per sec (GB/s vs HBM roofline); ms per step"
+UNIT = "elements/s"
+DEFAULT_WORKLOAD = "bert_base_topk1pct_w8"
+MAIN_KERNEL = "tk_main_kernel<true>"
+MAIN_SOURCE = os.path.join(ROOT, "gradient_compression_error_b200", "csrc", "topk.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "tk_main_bert_base_w8_traffic.txt")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def workload_spec(name):
+    from gradient_compression_error_b200 import workloads as wl
+    if name == "bert_base_topk1pct_w8":
+        return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk")
+    if name == "memsgd_vector_2p20":
+        return dict(layers=wl.memsgd_vector(), W=1, cfg=1, method="topk")
+    if name.startswith("sweep_topk_e"):          # e.g. sweep_topk_e28_ppm10000
+        e, ppm = name[len("sweep_topk_e"):].split("_ppm")
+        return dict(layers=wl.sweep(int(e), "topk", int(ppm)), W=1, cfg=5, method="topk")
+    if name.startswith("sweep_randk_e"):
+        e, ppm = name[len("sweep_randk_e"):].split("_ppm")
+        return dict(layers=wl.sweep(int(e), "randk", int(ppm)), W=1, cfg=5, method="randk")
+    raise SystemExit("unknown workload %s" % name)
+
+
+def measured_hbm_gbs():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def ncu_traffic_per_launch():
+    """Per-launch DRAM bytes of the main kernel from the committed ncu summary,
+    or None when the kernel source changed since the capture."""
+    try:
+        src_hash = hashlib.sha256(open(MAIN_SOURCE, "rb").read()).hexdigest()
+        fields = {}
+        with open(TRAFFIC_FILE) as f:
+            for line in f:
+                if ":" in line:
+                    k, v = line.split(":", 1)
+                    fields[k.strip()] = v.strip()
+        if fields.get("source_sha256") != src_hash:
+            return None
+        return float(fields["dram_bytes_per_launch_full_size"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cpu_oracle_sample(spec, units, steps_seed):
+    """Run the oracle on `units` of the workload (host arrays from seeded
+    device gradients of worker w); returns (elements, seconds, threads)."""
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
+    import oracle
+    from gradient_compression_error_b200 import workloads as wl
+    import torch
+    layers = spec["layers"]
+    offs, o = [], 0
+    for l in layers:
+        offs.append(o)
+        o += l["rows"] * l["cols"]
+    threads = os.cpu_count() or 1
+    data = {}
+    for (w, l) in units:
+        n = layers[l]["rows"] * layers[l]["cols"]
+        g = torch.Generator()
+        g.manual_seed(wl.seed_for(spec["cfg"], w, steps_seed) + l)
+        data[(w, l)] = (torch.randn(n, generator=g).numpy().astype(np.float32),
+                        np.zeros(n, np.float32))
+
+    def one(u):
+        w, l = u
+        lay = layers[l]
+        gg, mm = data[u]
+        if spec["method"] == "topk":
+            vals, idx, m_new = oracle.ef_topk_unit(gg, mm, lay["cap"], wl.ETA)
+        else:
+            vals, idx, m_new = oracle.ef_randk_unit(gg, mm, lay["cap"], wl.ETA, 5, w, l, 0)
+        out = np.zeros(gg.size, np.float32)
+        oracle.accum_sparse(out, vals, idx)
+        return gg.size
+
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        elems = sum(ex.map(one, units))
+    dt = time.perf_counter() - t0
+    return elems, dt, threads
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    spec = workload_spec(args.workload)
+    L = len(spec["layers"])
+    # bounded sample per step: one worker's tensors, rotating over workers,
+    # capped near 6 M elements so a 13-step run stays within a few minutes
+    samples = []
+    for s in range(args.warmup + args.steps):
+        w = s % spec["W"]
+        units, tot = [], 0
+        for l in sorted(range(L), key=lambda l: -(spec["layers"][l]["rows"] * spec["layers"][l]["cols"])):
+            n = spec["layers"][l]["rows"] * spec["layers"][l]["cols"]
+            if tot + n <= 6_000_000 or not units:
+                units.append((w, l))
+                tot += n
+        samples.append(units)
+    times, elems_tot, threads = [], 0, 1
+    for s, units in enumerate(samples):
+        elems, dt, threads = cpu_oracle_sample(spec, units, s)
+        if s >= args.warmup:
+            times.append(dt)
+            elems_tot += elems
+    t = sum(times)
+    value = elems_tot / t
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (seeded N(0,1) gradients)",
+            "config": {"workload": args.workload, "W": spec["W"]},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": "per step: the largest tensors of one worker (rotating), "
+                                       "about 6 M elements, encode (top-k) + decode"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--profile", action="store_true", help="per-kernel table on stderr")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    import gradient_compression_error_b200 as gce
+    from gradient_compression_error_b200 import workloads as wl
+
+    spec = workload_spec(args.workload)
+    layers, W = spec["layers"], spec["W"]
+    table = gce.Table(wl.table_layers(layers))
+    N = table.N
+    K_total = sum(l["cap"] for l in layers)
+    dev = "cuda"
+    grads = [wl.gradients(layers, W, spec["cfg"], s) for s in range(2)]
+    mem = torch.zeros((W, N), dtype=torch.float32, device=dev)
+    vals = torch.zeros((W, table.vals_per_worker), dtype=torch.float32, device=dev)
+    idx = torch.zeros((W, table.vals_per_worker), dtype=torch.int32, device=dev)
+    ws = table.workspace(W, spec["method"])
+    ws_dc = table.workspace(W, "decompress")
+    out = torch.zeros(N, dtype=torch.float32, device=dev)
+    encode = gce.ef_topk_step if spec["method"] == "topk" else None
+
+    def step(s, grad):
+        if spec["method"] == "topk":
+            gce.ef_topk_step(table, W, grad, mem, wl.ETA, None, vals, idx, ws)
+        else:
+            gce.ef_randk_step(table, W, grad, mem, wl.ETA, None, 5, s, vals, idx, ws)
+        gce.decompress_accumulate(table, W, vals, idx, None, None, None, 1.0, out, ws_dc)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for s in range(args.warmup):
+        step(s, grads[s % 2])
+    torch.cuda.synchronize()
+    if gce.status(ws) & gce.STATUS_K_RANGE:
+        raise SystemExit("device status reports an out-of-range k")
+
+    clocks = ClockSampler(torch.cuda.current_device())
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.2)
+    l0 = gce.launch_count()
+    gce.profile_start()
+    ev0.record()
+    for s in range(args.steps):
+        step(args.warmup + s, grads[s % 2])
+    ev1.record()
+    torch.cuda.synchronize()
+    prof = gce.profile_stop()
+    launches = gce.launch_count() - l0
+    barrier()
+    clk = clocks.stop()
+    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    fallback_seen = bool(gce.status(ws) & gce.STATUS_FALLBACK)
+
+    elems_per_step = W * N
+    value = world * elems_per_step * args.steps / (t_ms / 1e3)
+    ms_step = t_ms / args.steps
+
+    main_ms, main_n = prof.get(MAIN_KERNEL if spec["method"] == "topk" else "rk_emit_kernel",
+                               (0.0, 0))
+    peak, peak_kind = measured_hbm_gbs()
+    bytes_per_launch = 12.0 * W * (N - sum(l["rows"] * l["cols"] for l in layers
+                                          if l["kind"] == "dense"))
+    achieved = bytes_per_launch / (main_ms / main_n / 1e3) / 1e9 if main_n else None
+    traffic = ncu_traffic_per_launch() if args.workload == DEFAULT_WORKLOAD else None
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": (achieved / peak) if achieved else None, "traffic": traffic,
+                "kernel": MAIN_KERNEL if spec["method"] == "topk" else "rk_emit_kernel",
+                "peak_source": peak_kind,
+                "algorithmic_bytes_per_launch": bytes_per_launch,
+                "avg_launch_ms": main_ms / main_n if main_n else None}
+    # whole-step algorithmic traffic: W(12N + 8K) encode + 16 W K + 4N decode
+    step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total + 4.0 * N
+    step_gbs = step_bytes / (ms_step / 1e3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hgrad = torch.empty((W, N), dtype=torch.float32, pin_memory=True)
+        hgrad.copy_(grads[0])
+        hout = torch.empty(N, dtype=torch.float32, pin_memory=True)
+        dgrad = grads[1]
+        ke = max(3, min(args.steps, 20))
+        step(0, dgrad)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for s in range(ke):
+            dgrad.copy_(hgrad, non_blocking=True)
+            step(s, dgrad)
+            hout.copy_(out, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        te = max_over_ranks(e0.elapsed_time(e1))
+        e2e = {"value": world * elems_per_step * ke / (te / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": W * N * 4, "d2h_bytes_per_step": N * 4, "steps": ke}
+        del hgrad, hout
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu:
+        units = [(0, l) for l in range(len(layers))]
+        elems, dt, threads = cpu_oracle_sample(spec, units, 0)
+        cpu = {"value": elems / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+               "sample": "worker 0: all %d tensors (%d elements), encode + decode, one step"
+                         % (len(layers), elems), "seconds": dt}
+
+    if args.profile and rank == 0:
+        tot = sum(v[0] for v in prof.values())
+        for name, (ms, n) in sorted(prof.items(), key=lambda x: -x[1][0]):
+            print("%-32s %8d launches %10.3f ms %6.1f%%" % (name, n, ms, 100 * ms / tot),
+                  file=sys.stderr)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded N(0,1) gradients, resident in HBM)",
+                "config": {"workload": args.workload, "W": W, "elements_per_worker": N,
+                           "tensors": len(layers), "k_total_per_worker": K_total,
+                           "eta": wl.ETA, "parallelism": "replicas x%d" % world,
+                           "l2": "inputs larger than L2 (%.1f GB of grad+memory per step)"
+                                 % (8.0 * W * N / 1e9),
+                           "step_algorithmic_GBps": step_gbs,
+                           "step_frac_of_hbm": step_gbs / peak,
+                           "fallback_seen": fallback_seen},
+                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+                "gpu_launches": launches, "clocks": clk}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -75,6 +75,10 @@ SIGNATURES = {
     "gce_launch_count": (_u64, []),
     "gce_error_string": (C.c_char_p, [C.c_int]),
     "gce_set_bracket_sigma": (C.c_int, [_f64]),
+    "gce_profile_start": (C.c_int, []),
+    "gce_profile_stop": (C.c_int, []),
+    "gce_profile_count": (C.c_int, []),
+    "gce_profile_get": (C.c_int, [_i32, C.c_char_p, _i32, C.POINTER(_f64), C.POINTER(_i64)]),
 }
 
 _lib = None
@@ -235,6 +239,22 @@ def status(ws, stream=None):
 
 def launch_count():
     return int(lib().gce_launch_count())
+
+
+def profile_start():
+    _check("gce_profile_start", lib().gce_profile_start())
+
+
+def profile_stop():
+    """Stop timing launches; returns {kernel name: (total ms, launches)}."""
+    _check("gce_profile_stop", lib().gce_profile_stop())
+    out = {}
+    for i in range(lib().gce_profile_count()):
+        buf = C.create_string_buffer(256)
+        ms, n = C.c_double(), C.c_int64()
+        _check("gce_profile_get", lib().gce_profile_get(i, buf, 256, C.byref(ms), C.byref(n)))
+        out[buf.value.decode()] = (ms.value, n.value)
+    return out
 
 
 def set_bracket_sigma(sigma):

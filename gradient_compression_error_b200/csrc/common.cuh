@@ -67,10 +67,18 @@ extern std::atomic<uint64_t> g_launches;
 
 inline void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// optional per-launch timing: two events on the launch's stream around it
+extern std::atomic<bool> g_prof_on;
+void prof_before(const char* name, cudaStream_t st);
+void prof_after(cudaStream_t st);
+
 #define GCE_LAUNCH(kern, grid, block, smem, stream, ...)                        \
     do {                                                                         \
         ::gce::count_launch();                                                   \
+        const bool gce_prof_ = ::gce::g_prof_on.load(std::memory_order_relaxed); \
+        if (gce_prof_) ::gce::prof_before(#kern, (stream));                      \
         kern<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+        if (gce_prof_) ::gce::prof_after((stream));                              \
     } while (0)
 
 inline int check_launch() {

@@ -1,0 +1,498 @@
+// randk.cu -- Mem-SGD error-feedback rand-k step on sm_100a.
+//
+// "Sparsified SGD with Memory", Method / Abstract: the same error-feedback
+// update as top-k with comp_k keeping k random coordinates, values unscaled.
+// The k coordinates are the k smallest (key, index) pairs, key_i = the high
+// 32 bits of output i+1 of a SplitMix64 generator (Steele, Lea, Flood 2014)
+// whose state is derived from (seed, stream 0, worker, layer, step).
+//
+// The choice does not depend on the data, so it is made before the memory
+// pass, without touching HBM:
+//   keys     hash every index once: a bitmask of key < lo (1 bit / element),
+//            the count below lo per tile, and a short list of the keys in
+//            [lo, hi] -- a band of +-sigma binomial deviations around the
+//            expected k-th smallest key
+//   resolve  exact (key, index) selection inside the band (one CTA per
+//            layer); the chosen band entries are OR-ed into the bitmask
+//   keys/resolve again with the band opened to everything for any layer
+//            whose band missed (exact fallback; results never depend on sigma)
+//   scan     per-tile output offsets
+//   emit     the only HBM pass: v = fl(m + fl(eta*g)), ordered write of the
+//            chosen (v, i), mem <- v or +0
+// DRAM traffic: 12 B per element + 8 B per chosen entry + 1/8 B of bitmask
+// written and read.
+#include <cmath>
+
+#include "common.cuh"
+#include "scan.cuh"
+#include "topk_layout.cuh"
+
+namespace gce {
+
+extern double bracket_sigma();
+
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+
+__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// state of (seed, stream, worker, layer, step): each field folded in as the
+// first SplitMix64 output from (previous + (field + 1) * gamma)
+__host__ __device__ __forceinline__ uint64_t hash_base(uint64_t seed, uint64_t stream,
+                                                       uint64_t worker, uint64_t layer,
+                                                       uint64_t step) {
+    uint64_t h = mix64(seed + (stream + 1) * kGamma);
+    h = mix64(h + (worker + 1) * kGamma);
+    h = mix64(h + (layer + 1) * kGamma);
+    h = mix64(h + (step + 1) * kGamma);
+    return h;
+}
+
+struct RkSeg {
+    int32_t k;       // 0: layer skipped
+    uint32_t lo, hi; // band of candidate keys
+    int32_t c_lo;    // keys below lo (main pass)
+    int32_t cand;    // band entries listed (main pass)
+    int32_t cand_redo;
+    int32_t fail;    // 1: the band missed the k-th key; redone exactly
+    uint32_t T;      // chosen iff key < T or (key == T and i <= iT)
+    int32_t iT;
+    uint64_t base;   // hash state of this (worker, layer, step)
+    int32_t pad[3];
+};
+static_assert(sizeof(RkSeg) == 56 || sizeof(RkSeg) == 64, "RkSeg layout");
+
+struct RkEntry {
+    uint32_t key;
+    int32_t i;
+};
+
+constexpr int kRkWords = kTkTile / 32;  // bitmask words per tile (256)
+
+struct RkLayout {
+    int64_t S = 0, TT = 0;
+    size_t segs = 0, tile_cnt = 0, bitmask = 0, cand = 0, total = 0;
+};
+
+static RkLayout rk_layout(const gce_table* t, int32_t W) {
+    RkLayout o;
+    Carver c;
+    const bool on = t->ckind == GCE_KIND_RANDK;
+    o.S = on ? int64_t(W) * int64_t(t->comp.size()) : 0;
+    o.TT = on ? int64_t(W) * t->tiles_pw : 0;
+    o.segs = c.take<RkSeg>(o.S);
+    o.tile_cnt = c.take<int32_t>(o.TT);
+    o.bitmask = c.take<uint32_t>(o.TT * kRkWords);
+    o.cand = c.take<RkEntry>(o.S ? int64_t(W) * t->comp_N : 0);
+    o.total = c.off;
+    return o;
+}
+
+size_t randk_ws_bytes(const gce_table* t, int32_t W) { return rk_layout(t, W).total; }
+
+__global__ void __launch_bounds__(256) rk_setup_kernel(const DevLayer* __restrict__ layers,
+                                                       const int32_t* __restrict__ comp,
+                                                       int32_t ncomp, int64_t S,
+                                                       const int32_t* __restrict__ k_or_rank,
+                                                       uint64_t seed, uint64_t step, double sigma,
+                                                       RkSeg* __restrict__ segs,
+                                                       int32_t* __restrict__ status) {
+    for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
+         s += int64_t(gridDim.x) * blockDim.x) {
+        const int32_t l = comp[s % ncomp];
+        const DevLayer L = layers[l];
+        const int32_t k = k_or_rank ? k_or_rank[l] : L.cap;
+        RkSeg g{};
+        if (k >= 1 && k <= L.cap && int64_t(k) <= L.n) {
+            g.k = k;
+        } else {
+            g.k = 0;
+            set_status(status, GCE_STATUS_K_RANGE);
+        }
+        // band: k -+ (sigma * binomial sd + sigma) keys around the expected position
+        const double n = double(L.n), p = double(k) / n;
+        const double d = sigma * (sqrt(n * p * (1.0 - p)) + 1.0);
+        const double scale = 4294967296.0 / n;
+        const double lo = (double(k) - d) * scale, hi = (double(k) + d) * scale;
+        g.lo = lo <= 0.0 ? 0u : (lo >= 4294967295.0 ? 0xFFFFFFFFu : uint32_t(lo));
+        g.hi = hi >= 4294967295.0 ? 0xFFFFFFFFu : (hi <= 0.0 ? 0u : uint32_t(hi));
+        if (g.hi < g.lo) g.hi = g.lo;
+        g.base = hash_base(seed, 0, uint64_t(s / ncomp), uint64_t(l), step);
+        segs[s] = g;
+    }
+}
+
+// kRedo: re-list a failed layer whole (band = every key, nothing below it).
+template <bool kRedo>
+__global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict__ layers,
+                                                      const int32_t* __restrict__ tile_layer,
+                                                      int32_t tiles_pw, int32_t W, int32_t ncomp,
+                                                      int64_t comp_N, RkSeg* __restrict__ segs,
+                                                      int32_t* __restrict__ tile_cnt,
+                                                      uint32_t* __restrict__ bitmask,
+                                                      RkEntry* __restrict__ cand) {
+    __shared__ int s_red[8];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t total = int64_t(tiles_pw) * W;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+        const int w = int(t / tiles_pw);
+        const int lt = int(t % tiles_pw);
+        const DevLayer L = layers[tile_layer[lt]];
+        const int64_t s = int64_t(w) * ncomp + L.sidx;
+        RkSeg& g = segs[s];
+        if (g.k == 0) continue;
+        if (kRedo && !g.fail) continue;
+        const uint32_t lo = kRedo ? 0u : g.lo, hi = kRedo ? 0xFFFFFFFFu : g.hi;
+        const uint64_t base = g.base;
+        const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
+        const int64_t e0 = tstart + int64_t(tid) * 32;
+        uint32_t keys[32];
+        uint32_t below = 0, inband = 0;
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const int64_t i = e0 + q;
+            const uint32_t key = uint32_t(mix64(base + uint64_t(i + 1) * kGamma) >> 32);
+            keys[q] = key;
+            if (i < L.n) {
+                below |= uint32_t(key < lo) << q;
+                inband |= uint32_t(key >= lo && key <= hi) << q;
+            }
+        }
+        bitmask[t * kRkWords + tid] = below;
+        // tile count of keys below the band
+        int c = warp_sum(__popc(below));
+        if (lane == 0) s_red[warp] = c;
+        __syncthreads();
+        if (tid == 0) {
+            int tot = 0;
+            for (int i = 0; i < 8; ++i) tot += s_red[i];
+            tile_cnt[t] = tot;
+            if (tot) atomicAdd(&g.c_lo, tot);
+        }
+        __syncthreads();
+        // band entries: order does not matter, the resolve sorts them out
+        const int nb = __popc(inband);
+        const int incl = warp_inclusive_scan(nb);
+        int wbase = 0;
+        if (lane == 31 && incl) wbase = atomicAdd(kRedo ? &g.cand_redo : &g.cand, incl);
+        wbase = __shfl_sync(kFull, wbase, 31);
+        RkEntry* out = cand + int64_t(w) * comp_N + L.sp_off + wbase + (incl - nb);
+        int pos = 0;
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+            if (inband & (1u << q)) out[pos++] = RkEntry{keys[q], int32_t(e0 + q)};
+    }
+}
+
+// One CTA: the rank-th smallest (key, index) pair (rank 1-based) of a list.
+__device__ void cta_select_pair(const RkEntry* __restrict__ list, int32_t count, int32_t rank,
+                                int32_t* h, uint32_t* s_pref, int32_t* s_rank, uint32_t* T,
+                                int32_t* iT) {
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        *s_pref = 0;
+        *s_rank = rank;
+    }
+    __syncthreads();
+    // key bits 31..21, 20..10, 9..0
+    const int kshift[3] = {21, 10, 0}, kbits[3] = {11, 11, 10};
+    for (int lv = 0; lv < 3; ++lv) {
+        const int nb = 1 << kbits[lv], sh = kshift[lv], top = sh + kbits[lv];
+        for (int b = tid; b < nb; b += blockDim.x) h[b] = 0;
+        __syncthreads();
+        const uint32_t pref = *s_pref;
+        for (int32_t j = tid; j < count; j += blockDim.x) {
+            const uint32_t key = list[j].key;
+            if (top >= 32 || (key >> top) == (pref >> top)) atomicAdd(&h[(key >> sh) & (nb - 1)], 1);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            int64_t below = 0;
+            const int b = warp_find_from_bottom(h, nb, *s_rank, &below);
+            if (tid == 0) {
+                *s_pref = pref | (uint32_t(max(b, 0)) << sh);
+                *s_rank = *s_rank - int32_t(below);
+            }
+        }
+        __syncthreads();
+    }
+    const uint32_t key_T = *s_pref;
+    if (tid == 0) *s_pref = 0;
+    __syncthreads();
+    // among keys == T: index bits 30..20, 19..9, 8..0
+    const int ishift[3] = {20, 9, 0}, ibits[3] = {11, 11, 9};
+    for (int lv = 0; lv < 3; ++lv) {
+        const int nb = 1 << ibits[lv], sh = ishift[lv], top = sh + ibits[lv];
+        for (int b = tid; b < nb; b += blockDim.x) h[b] = 0;
+        __syncthreads();
+        const uint32_t pref = *s_pref;
+        for (int32_t j = tid; j < count; j += blockDim.x) {
+            const RkEntry e = list[j];
+            const uint32_t i = uint32_t(e.i);
+            if (e.key == key_T && (i >> top) == (pref >> top)) atomicAdd(&h[(i >> sh) & (nb - 1)], 1);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            int64_t below = 0;
+            const int b = warp_find_from_bottom(h, nb, *s_rank, &below);
+            if (tid == 0) {
+                *s_pref = pref | (uint32_t(max(b, 0)) << sh);
+                *s_rank = *s_rank - int32_t(below);
+            }
+        }
+        __syncthreads();
+    }
+    *T = key_T;
+    *iT = int32_t(*s_pref);
+    __syncthreads();
+}
+
+// One CTA per layer: find (T, iT), then OR the chosen band entries into the
+// bitmask and add them to their tiles' counts.
+template <bool kRedo>
+__global__ void __launch_bounds__(1024) rk_resolve_kernel(const DevLayer* __restrict__ layers,
+                                                          const int32_t* __restrict__ comp,
+                                                          int32_t ncomp, int64_t S,
+                                                          int32_t tiles_pw, int64_t comp_N,
+                                                          RkSeg* __restrict__ segs,
+                                                          int32_t* __restrict__ tile_cnt,
+                                                          uint32_t* __restrict__ bitmask,
+                                                          const RkEntry* __restrict__ cand,
+                                                          int32_t* __restrict__ status) {
+    __shared__ int32_t h[2048];
+    __shared__ uint32_t s_pref;
+    __shared__ int32_t s_rank;
+    __shared__ int s_go;
+    for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
+        RkSeg& g = segs[s];
+        if (threadIdx.x == 0) {
+            int go = 0;
+            if (g.k > 0) {
+                if (!kRedo) {
+                    const int32_t need = g.k - g.c_lo;
+                    go = (need >= 1 && need <= g.cand);
+                    if (!go) {
+                        g.fail = 1;
+                        set_status(status, GCE_STATUS_FALLBACK);
+                    }
+                } else {
+                    go = g.fail;
+                }
+            }
+            s_go = go;
+        }
+        __syncthreads();
+        if (!s_go) {
+            __syncthreads();
+            continue;
+        }
+        const int w = int(s / ncomp);
+        const DevLayer L = layers[comp[s % ncomp]];
+        const RkEntry* list = cand + int64_t(w) * comp_N + L.sp_off;
+        const int32_t count = kRedo ? g.cand_redo : g.cand;
+        const int32_t rank = kRedo ? g.k : g.k - g.c_lo;
+        uint32_t T;
+        int32_t iT;
+        cta_select_pair(list, count, rank, h, &s_pref, &s_rank, &T, &iT);
+        if (threadIdx.x == 0) {
+            g.T = T;
+            g.iT = iT;
+        }
+        const int64_t t0 = int64_t(w) * tiles_pw + L.tile0;
+        for (int32_t j = threadIdx.x; j < count; j += blockDim.x) {
+            const RkEntry e = list[j];
+            if (e.key < T || (e.key == T && e.i <= iT)) {
+                const int64_t t = t0 + e.i / kTkTile;
+                const int r = e.i % kTkTile;
+                atomicOr(&bitmask[t * kRkWords + r / 32], 1u << (r % 32));
+                atomicAdd(&tile_cnt[t], 1);
+            }
+        }
+        __syncthreads();
+    }
+}
+
+__global__ void __launch_bounds__(1024) rk_scan_kernel(const DevLayer* __restrict__ layers,
+                                                       const int32_t* __restrict__ comp,
+                                                       int32_t ncomp, int64_t S, int32_t tiles_pw,
+                                                       const RkSeg* __restrict__ segs,
+                                                       int32_t* __restrict__ tile_cnt) {
+    __shared__ int s_warp[33];
+    for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
+        if (segs[s].k == 0) continue;
+        const int w = int(s / ncomp);
+        const DevLayer L = layers[comp[s % ncomp]];
+        int32_t* tc = tile_cnt + int64_t(w) * tiles_pw + L.tile0;
+        int carry = 0;
+        for (int b0 = 0; b0 < L.ntiles; b0 += blockDim.x) {
+            const int i = b0 + threadIdx.x;
+            const int x = i < L.ntiles ? tc[i] : 0;
+            int tot = 0;
+            const int ex = block_exclusive_scan(x, s_warp, &tot);
+            if (i < L.ntiles) tc[i] = carry + ex;
+            carry += tot;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
+    int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, const float* __restrict__ grad,
+    float* __restrict__ mem, float eta, const RkSeg* __restrict__ segs,
+    const int32_t* __restrict__ tile_off, const uint32_t* __restrict__ bitmask,
+    float* __restrict__ vals, int32_t* __restrict__ idx) {
+    constexpr int kIters = kTkPerThread / 4;
+    constexpr int kWarps = kTkThreads / 32;
+    __shared__ int32_t s_wt[kIters * kWarps];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t total = int64_t(tiles_pw) * W;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+        const int w = int(t / tiles_pw);
+        const int lt = int(t % tiles_pw);
+        const DevLayer L = layers[tile_layer[lt]];
+        const int64_t s = int64_t(w) * ncomp + L.sidx;
+        const int32_t k = segs[s].k;
+        if (k == 0) continue;
+        const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
+        const int cnt = int(min64(kTkTile, L.n - tstart));
+        const int64_t ebase = int64_t(w) * N + L.offset + tstart;
+        const float* g = grad + ebase;
+        float* m = mem + ebase;
+        const uint32_t* bm = bitmask + t * kRkWords;
+        float v[kTkPerThread];
+        uint32_t flags = 0;
+        const bool vec = cnt == kTkTile && (ebase & 3) == 0;
+#pragma unroll
+        for (int j = 0; j < kIters; ++j) {
+            const int e = j * (kTkThreads * 4) + tid * 4;
+            const uint32_t word = bm[e >> 5];
+            const uint32_t f = (word >> (e & 31)) & 0xFu;
+            float4 x;
+            if (vec) {
+                const float4 gg = ld_stream4(g + e);
+                const float4 mm = ld_stream4(m + e);
+                x.x = residual(mm.x, eta, gg.x);
+                x.y = residual(mm.y, eta, gg.y);
+                x.z = residual(mm.z, eta, gg.z);
+                x.w = residual(mm.w, eta, gg.w);
+                float4 o;
+                o.x = (f & 1u) ? 0.0f : x.x;
+                o.y = (f & 2u) ? 0.0f : x.y;
+                o.z = (f & 4u) ? 0.0f : x.z;
+                o.w = (f & 8u) ? 0.0f : x.w;
+                *reinterpret_cast<float4*>(m + e) = o;
+            } else {
+                float xs[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    xs[q] = 0.0f;
+                    if (e + q < cnt) {
+                        xs[q] = residual(m[e + q], eta, __ldcs(g + e + q));
+                        m[e + q] = (f & (1u << q)) ? 0.0f : xs[q];
+                    }
+                }
+                x = make_float4(xs[0], xs[1], xs[2], xs[3]);
+            }
+            v[4 * j + 0] = x.x;
+            v[4 * j + 1] = x.y;
+            v[4 * j + 2] = x.z;
+            v[4 * j + 3] = x.w;
+            flags |= f << (4 * j);
+        }
+        int incl[kIters];
+#pragma unroll
+        for (int j = 0; j < kIters; ++j) {
+            incl[j] = warp_inclusive_scan(__popc((flags >> (4 * j)) & 0xFu));
+            if (lane == 31) s_wt[j * kWarps + warp] = incl[j];
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const int a = s_wt[2 * lane], b = s_wt[2 * lane + 1];
+            const int x = warp_inclusive_scan(a + b);
+            s_wt[2 * lane] = x - a - b;
+            s_wt[2 * lane + 1] = x - b;
+        }
+        __syncthreads();
+        const int base = tile_off[t];
+        float* vout = vals + int64_t(w) * vals_pw + L.val_off;
+        int32_t* iout = idx + int64_t(w) * vals_pw + L.val_off;
+#pragma unroll
+        for (int j = 0; j < kIters; ++j) {
+            const uint32_t f = (flags >> (4 * j)) & 0xFu;
+            int pos = base + s_wt[j * kWarps + warp] + incl[j] - __popc(f);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                if ((f & (1u << q)) && pos < k) {
+                    vout[pos] = v[4 * j + q];
+                    iout[pos] = int32_t(tstart + j * (kTkThreads * 4) + tid * 4 + q);
+                }
+                pos += (f >> q) & 1u;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+template <class K>
+static int occupancy_of(K kernel, int threads) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1)
+        n = 1;
+    return n;
+}
+
+static int grid_cap(int64_t work, int per_sm) {
+    const int64_t cap = int64_t(sm_count()) * per_sm;
+    return int(max64(1, min64(work, cap)));
+}
+
+}  // namespace gce
+
+using namespace gce;
+
+extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
+                             const int32_t* k_or_rank, uint64_t seed, uint64_t step, float* vals,
+                             int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+    if (!t || W < 1 || !grad || !mem || !ws) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_RANDK && t->ckind != -1) return GCE_ERR_KIND;
+    if (!aligned16(grad) || !aligned16(mem) || !aligned16(ws)) return GCE_ERR_ARG;
+    if ((t->vals_pw > 0) && (!vals || !aligned16(vals))) return GCE_ERR_ARG;
+    if (t->ckind == GCE_KIND_RANDK && (!idx || !aligned16(idx))) return GCE_ERR_ARG;
+    if (k_or_rank && (reinterpret_cast<uintptr_t>(k_or_rank) & 3)) return GCE_ERR_ARG;
+    const RkLayout lay = rk_layout(t, W);
+    if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(ws);
+    if (lay.S > 0) {
+        const int32_t ncomp = int32_t(t->comp.size());
+        RkSeg* segs = at<RkSeg>(ws, lay.segs);
+        int32_t* tile_cnt = at<int32_t>(ws, lay.tile_cnt);
+        uint32_t* bitmask = at<uint32_t>(ws, lay.bitmask);
+        RkEntry* cand = at<RkEntry>(ws, lay.cand);
+        static int occ_emit = occupancy_of(rk_emit_kernel, kTkThreads);
+        GCE_LAUNCH(rk_setup_kernel, grid_cap((lay.S + 255) / 256, 4), 256, 0, st, t->d_layers,
+                   t->d_comp, ncomp, lay.S, k_or_rank, seed, step, bracket_sigma(), segs, status);
+        GCE_LAUNCH(rk_keys_kernel<false>, grid_cap(lay.TT, 8), 256, 0, st, t->d_layers,
+                   t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs, tile_cnt, bitmask,
+                   cand);
+        GCE_LAUNCH(rk_resolve_kernel<false>, grid_cap(lay.S, 2), 1024, 0, st, t->d_layers,
+                   t->d_comp, ncomp, lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, bitmask, cand,
+                   status);
+        GCE_LAUNCH(rk_keys_kernel<true>, grid_cap(lay.TT, 8), 256, 0, st, t->d_layers,
+                   t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs, tile_cnt, bitmask,
+                   cand);
+        GCE_LAUNCH(rk_resolve_kernel<true>, grid_cap(lay.S, 2), 1024, 0, st, t->d_layers,
+                   t->d_comp, ncomp, lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, bitmask, cand,
+                   status);
+        GCE_LAUNCH(rk_scan_kernel, grid_cap(lay.S, 2), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
+                   lay.S, t->tiles_pw, segs, tile_cnt);
+        GCE_LAUNCH(rk_emit_kernel, grid_cap(lay.TT, occ_emit), kTkThreads, 0, st, t->d_layers,
+                   t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw, grad, mem, eta, segs,
+                   tile_cnt, bitmask, vals, idx);
+        if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+    }
+    return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+}

@@ -89,4 +89,39 @@ __device__ __forceinline__ int warp_find_from_top(const int32_t* h, int nb, int6
     return res;
 }
 
+// As warp_find_from_top, counting from the bottom: returns b with
+// below(b) < target <= below(b) + h[b]; *below_out = below(b).
+__device__ __forceinline__ int warp_find_from_bottom(const int32_t* h, int nb, int64_t target,
+                                                     int64_t* below_out) {
+    const int lane = threadIdx.x & 31;
+    const int per = nb >> 5;
+    int64_t mine = 0;
+    for (int i = 0; i < per; ++i) mine += h[lane * per + i];
+    const int64_t incl = warp_inclusive_scan(mine);
+    const int64_t excl = incl - mine;
+    const unsigned ball = __ballot_sync(kFull, excl < target && target <= incl);
+    if (ball == 0) {
+        *below_out = __shfl_sync(kFull, incl, 31);
+        return -1;
+    }
+    const int src = __ffs(ball) - 1;
+    int res = -1;
+    int64_t below = 0;
+    if (lane == src) {
+        int64_t acc = excl;
+        for (int b = lane * per; b < lane * per + per; ++b) {
+            if (acc + h[b] >= target) {
+                res = b;
+                below = acc;
+                break;
+            }
+            acc += h[b];
+        }
+    }
+    res = __shfl_sync(kFull, res, src);
+    below = __shfl_sync(kFull, below, src);
+    *below_out = below;
+    return res;
+}
+
 }  // namespace gce

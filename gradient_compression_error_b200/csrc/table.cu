@@ -2,6 +2,7 @@
 // and the kernel for uncompressed (DENSE) layers shared by every step.
 #include <cstring>
 #include <mutex>
+#include <string>
 
 #include "common.cuh"
 #include "topk_layout.cuh"
@@ -9,6 +10,52 @@
 namespace gce {
 
 std::atomic<uint64_t> g_launches{0};
+std::atomic<bool> g_prof_on{false};
+
+// ---- launch timing (host side) -------------------------------------------------
+namespace {
+struct ProfRec {
+    const char* name;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::vector<ProfRec> g_prof_recs;
+std::vector<cudaEvent_t> g_prof_pool;
+size_t g_prof_used = 0;
+constexpr size_t kProfMax = 1 << 16;
+struct ProfAgg {
+    std::string name;
+    double ms;
+    int64_t n;
+};
+std::vector<ProfAgg> g_prof_agg;
+
+cudaEvent_t prof_event() {
+    if (g_prof_used < g_prof_pool.size()) return g_prof_pool[g_prof_used++];
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    g_prof_pool.push_back(e);
+    ++g_prof_used;
+    return e;
+}
+}  // namespace
+
+void prof_before(const char* name, cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof_recs.size() >= kProfMax) return;
+    ProfRec r{name, prof_event(), nullptr};
+    if (!r.a) return;
+    cudaEventRecord(r.a, st);
+    g_prof_recs.push_back(r);
+}
+
+void prof_after(cudaStream_t st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof_recs.empty() || g_prof_recs.back().b) return;
+    ProfRec& r = g_prof_recs.back();
+    r.b = prof_event();
+    if (r.b) cudaEventRecord(r.b, st);
+}
 
 int sm_count() {
     static int cached[64] = {0};
@@ -276,6 +323,56 @@ extern "C" int gce_status(void* ws, void* stream, int32_t* status) {
 }
 
 extern "C" uint64_t gce_launch_count(void) { return g_launches.load(); }
+
+extern "C" int gce_profile_start(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_recs.clear();
+    g_prof_agg.clear();
+    g_prof_used = 0;
+    g_prof_on.store(true);
+    return GCE_OK;
+}
+
+extern "C" int gce_profile_stop(void) {
+    g_prof_on.store(false);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    int rc = GCE_OK;
+    for (const ProfRec& r : g_prof_recs) {
+        if (!r.a || !r.b) continue;
+        if (cudaEventSynchronize(r.b) != cudaSuccess) { rc = GCE_ERR_CUDA; continue; }
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) { rc = GCE_ERR_CUDA; continue; }
+        bool found = false;
+        for (ProfAgg& a : g_prof_agg)
+            if (a.name == r.name) {
+                a.ms += ms;
+                a.n += 1;
+                found = true;
+                break;
+            }
+        if (!found) g_prof_agg.push_back(ProfAgg{r.name, double(ms), 1});
+    }
+    g_prof_recs.clear();
+    return rc;
+}
+
+extern "C" int gce_profile_count(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    return int(g_prof_agg.size());
+}
+
+extern "C" int gce_profile_get(int32_t i, char* name, int32_t name_len, double* total_ms,
+                               int64_t* launches) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (i < 0 || size_t(i) >= g_prof_agg.size() || !name || name_len < 1 || !total_ms || !launches)
+        return GCE_ERR_ARG;
+    const ProfAgg& a = g_prof_agg[i];
+    std::strncpy(name, a.name.c_str(), size_t(name_len) - 1);
+    name[name_len - 1] = 0;
+    *total_ms = a.ms;
+    *launches = a.n;
+    return GCE_OK;
+}
 
 extern "C" const char* gce_error_string(int code) {
     switch (code) {

@@ -581,3 +581,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, st);
 }
+
+namespace gce {
+double bracket_sigma() { return g_bracket_sigma; }
+}  // namespace gce

@@ -239,6 +239,18 @@ GCE_API int gce_status(void* ws, void* stream, int32_t* status);
 /* Number of kernels this library has launched since it was loaded. */
 GCE_API uint64_t gce_launch_count(void);
 
+/* Per-kernel timing.  Between gce_profile_start and gce_profile_stop every
+ * launch of this library is bracketed by two CUDA events recorded on its
+ * stream (at most 65536 launches are recorded).  gce_profile_stop waits for
+ * those events and sums the elapsed time per kernel; gce_profile_count /
+ * gce_profile_get then list (kernel name, total ms, launches).  Host-side
+ * bookkeeping only; the kernels themselves are unchanged. */
+GCE_API int gce_profile_start(void);
+GCE_API int gce_profile_stop(void);
+GCE_API int gce_profile_count(void);
+GCE_API int gce_profile_get(int32_t i, char* name, int32_t name_len, double* total_ms,
+                            int64_t* launches);
+
 /* Static description of a return code. */
 GCE_API const char* gce_error_string(int code);
 

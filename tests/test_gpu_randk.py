@@ -1,0 +1,103 @@
+"""GPU parity of ef_randk_step against the CPU oracle (bit-exact).
+
+Source: "Sparsified SGD with Memory", Abstract / Method: rand-k keeps k
+random coordinates under the same error-feedback update; both sides draw
+the coordinates from SplitMix64 keyed by (seed, worker, layer, step), each
+implemented from the generator's published definition.
+"""
+import numpy as np
+import pytest
+
+from gradient_compression_error_b200 import workloads
+from oracle import steps as osteps
+from tests.helpers import bits, gce, host, layer_slice, need_gpu, payload_slice, torch
+
+pytestmark = pytest.mark.gpu
+
+
+def run_randk(layers, W, T, seed, make_grad, eta=0.05, k_fn=None):
+    g = gce()
+    t = g.Table(workloads.table_layers(layers))
+    mem = torch.zeros((W, t.N), device="cuda")
+    vals = torch.zeros((W, max(4, t.vals_per_worker)), device="cuda")
+    idx = torch.zeros((W, max(4, t.vals_per_worker)), dtype=torch.int32, device="cuda")
+    ws = t.workspace(W, "randk")
+    hmem = np.zeros((W, t.N), np.float32)
+    for step in range(T):
+        grad = make_grad(step)
+        ks = [l["cap"] for l in layers] if k_fn is None else k_fn(step)
+        kt = None if k_fn is None else torch.tensor(ks, dtype=torch.int32, device="cuda")
+        expect = osteps.sparse_step(layers, host(grad), hmem, eta, ks, method="randk", seed=seed,
+                                    step=step, threads=8)
+        g.ef_randk_step(t, W, grad, mem, eta, kt, seed, step, vals, idx, ws)
+        hv, hi, hm = host(vals), host(idx), host(mem)
+        for (w, l), e in expect.items():
+            if layers[l]["kind"] == "dense":
+                n = layers[l]["rows"] * layers[l]["cols"]
+                assert np.array_equal(bits(hv[w, payload_slice(t, 0, l, n)]), bits(e))
+            else:
+                sl = payload_slice(t, 0, l, ks[l])
+                assert np.array_equal(hi[w, sl], e[1]), ("idx", step, w, l)
+                assert np.array_equal(bits(hv[w, sl]), bits(e[0])), ("vals", step, w, l)
+            ls = layer_slice(t, l)
+            assert np.array_equal(bits(hm[w, ls]), bits(hmem[w, ls])), ("mem", step, w, l)
+    return g, ws
+
+
+LAYERS = [dict(rows=1, cols=1, kind="randk", cap=1, sigma=1.0),
+          dict(rows=8193, cols=1, kind="randk", cap=80, sigma=1.0),
+          dict(rows=64, cols=1, kind="dense", cap=0, sigma=1.0),
+          dict(rows=200, cols=500, kind="randk", cap=100000, sigma=1.0),   # k = n
+          dict(rows=300017, cols=1, kind="randk", cap=3000, sigma=1.0),
+          dict(rows=1 << 20, cols=1, kind="randk", cap=104857, sigma=1.0)]
+
+
+def test_ragged_table_bit_exact():
+    need_gpu()
+    run_randk(LAYERS, 2, 3, 1234, lambda s: workloads.gradients(LAYERS, 2, 201, s))
+
+
+def test_k_changes_between_steps():
+    need_gpu()
+    layers = [dict(rows=100000, cols=1, kind="randk", cap=10000, sigma=1.0)]
+    ks = [[10000], [1000], [1]]
+    run_randk(layers, 1, 3, 7, lambda s: workloads.gradients(layers, 1, 202, s),
+              k_fn=lambda s: ks[s])
+
+
+def test_forced_fallback_is_still_exact():
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=500000, cols=1, kind="randk", cap=5000, sigma=1.0),
+              dict(rows=30000, cols=1, kind="randk", cap=300, sigma=1.0)]
+    try:
+        g.set_bracket_sigma(-50.0)    # empty band: every layer takes the exact fallback
+        g2, ws = run_randk(layers, 2, 2, 99, lambda s: workloads.gradients(layers, 2, 203, s))
+        assert g.status(ws) & g.STATUS_FALLBACK
+    finally:
+        g.set_bracket_sigma(6.0)
+
+
+def test_bert_base_w8_sampled_units():
+    """BERT-base shapes, rand-k 1 %, W = 8 at full size; oracle on sampled units."""
+    need_gpu()
+    g = gce()
+    layers = workloads.bert_base_topk(kind="randk")
+    W = 8
+    t = g.Table(workloads.table_layers(layers))
+    grad = workloads.gradients(layers, W, 4, 0)
+    mem = torch.zeros_like(grad)
+    vals = torch.zeros((W, t.vals_per_worker), device="cuda")
+    idx = torch.zeros((W, t.vals_per_worker), dtype=torch.int32, device="cuda")
+    g.ef_randk_step(t, W, grad, mem, 0.05, None, 5, 0, vals, idx, t.workspace(W, "randk"))
+    import oracle
+    hv, hi = host(vals), host(idx)
+    for (w, l) in [(0, 0), (7, 5), (4, 3), (1, len(layers) - 1)]:
+        ls = layer_slice(t, l)
+        n = layers[l]["rows"] * layers[l]["cols"]
+        ev, ei, em = oracle.ef_randk_unit(host(grad[w, ls]), np.zeros(n, np.float32),
+                                          layers[l]["cap"], 0.05, 5, w, l, 0)
+        sl = payload_slice(t, 0, l, layers[l]["cap"])
+        assert np.array_equal(hi[w, sl], ei)
+        assert np.array_equal(bits(hv[w, sl]), bits(ev))
+        assert np.array_equal(bits(host(mem[w, ls])), bits(em))
