@@ -58,6 +58,21 @@ struct gce_table {
     int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker
     int32_t* d_bunit_layer = nullptr;
     int32_t* d_bunit_chunk = nullptr;
+    // PowerSGD plan (built by gce::powersgd_plan)
+    void* d_ps = nullptr;                  // PsLayer[L]
+    int4* d_ps1_tiles = nullptr;           // (layer, row block, column chunk) of M Q and residual
+    int32_t ps1_ntiles = 0;
+    int4* d_ps3_tiles = nullptr;           // (layer, row block, column chunk) of M^T P
+    int32_t ps3_ntiles = 0;
+    int4* d_psq_tiles = nullptr;           // (layer, column block) of the Q reduction
+    int32_t psq_ntiles = 0;
+    int32_t* d_ps_layers = nullptr;        // POWERSGD layer ids
+    int32_t nps = 0;
+    int64_t ppart_pw = 0, pd_pw = 0, qpart_pw = 0;  // workspace floats / doubles per worker
+    // Accordion plan (built by gce::accordion_plan)
+    int2* d_ac_tiles = nullptr;            // (layer, chunk) of the norm reduction
+    int32_t ac_ntiles = 0;
+    int2* d_ac_layer = nullptr;            // per layer: (first norm tile, tile count)
 };
 
 namespace gce {
@@ -136,5 +151,30 @@ constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
 
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
                         float eta, float* vals, cudaStream_t st);
+int powersgd_plan(gce_table* t);   // called once by gce_table_create
+void powersgd_plan_free(gce_table* t);
+int accordion_plan(gce_table* t);  // called once by gce_table_create
+void accordion_plan_free(gce_table* t);
+
+// SplitMix64 (Steele, Lea, Flood 2014): 64-bit finaliser and golden gamma
+constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
+
+__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
+    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+    return z ^ (z >> 31);
+}
+
+// state of (seed, stream, worker, layer, step): each field folded in as the
+// first SplitMix64 output from (previous + (field + 1) * gamma)
+__host__ __device__ __forceinline__ uint64_t hash_base(uint64_t seed, uint64_t stream,
+                                                       uint64_t worker, uint64_t layer,
+                                                       uint64_t step) {
+    uint64_t h = mix64(seed + (stream + 1) * kGamma);
+    h = mix64(h + (worker + 1) * kGamma);
+    h = mix64(h + (layer + 1) * kGamma);
+    h = mix64(h + (step + 1) * kGamma);
+    return h;
+}
 
 }  // namespace gce

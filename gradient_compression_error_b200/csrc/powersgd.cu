@@ -1,0 +1,485 @@
+// powersgd.cu -- PowerSGD rank-r compression with error feedback on sm_100a.
+//
+// The pages name PowerSGD and its ranks ("Accordion ...", Method and Key
+// results: ranks 1/2/4; "On the Utility of Gradient Compression ...", Method
+// and Key results: all-reduce compatible) without printing its steps; this
+// file implements the standard single power-iteration step with a reused Q,
+// with the Mem-SGD memory of "Sparsified SGD with Memory", Method:
+//   M = fl(m + fl(eta*g))                         (residual, as Mem-SGD)
+//   P = M Q            (Q: warm start, cols x r)
+//   P <- orthonormal columns (modified Gram-Schmidt, column order, fp64)
+//   Q <- M^T P
+//   m <- M - P Q^T,  dense_out <- P Q^T
+//
+// r <= 4, so every product is a skinny contraction of about 2r flops per
+// element of M: far below the tensor-core ridge and below the CUDA-core one,
+// so the kernels are plain register-blocked FMA loops shaped for bandwidth:
+//   mq      one pass over grad and mem: M written back to mem, and per
+//           (16-row block, 1024-column chunk) tile each warp reduces its rows
+//           against the Q chunk staged in shared memory -> partial P
+//   orth    one CTA per matrix: partial P summed in fp64 in chunk order,
+//           then Gram-Schmidt with fp64 block reductions in a fixed order
+//   mtp     per (64-row block, 1024-column chunk): each thread owns 4
+//           columns and accumulates M^T P over the block's rows -> partials
+//   qred    the row-block partials summed in fp64 in block order -> Q
+//   resid   m <- M - P Q^T with the same product order as the decoder
+// DRAM traffic for matrices that stay in L2 between the passes: 12 B per
+// element (read grad, read mem, write mem once); otherwise mtp and resid
+// re-read M (+8 B) and resid writes it (+4 B; +4 B for dense_out).
+#include <cmath>
+
+#include "common.cuh"
+#include "scan.cuh"
+
+namespace gce {
+
+constexpr int kPsRB = 16;     // rows per M Q / residual tile
+constexpr int kPsCB = 1024;   // columns per chunk (256 threads x 4)
+constexpr int kPsRB3 = 64;    // rows per M^T P tile
+constexpr int kPsQB = 256;    // columns per Q-reduction tile
+
+struct PsLayer {
+    int64_t ppart_off;  // floats: nch1 x rows x cap partial P
+    int64_t pd_off;     // doubles: rows x cap
+    int64_t qpart_off;  // floats: nrb3 x cols x cap partial Q
+    int32_t nch1, nrb3;
+};
+
+int powersgd_plan(gce_table* t) {
+    std::vector<PsLayer> ps(t->L);
+    std::vector<int4> t1, t3, tq;
+    std::vector<int32_t> ids;
+    int64_t pp = 0, pd = 0, qp = 0;
+    for (int32_t l = 0; l < t->L; ++l) {
+        const DevLayer& L = t->layers[l];
+        PsLayer x{};
+        if (L.kind == GCE_KIND_POWERSGD) {
+            x.nch1 = int32_t((L.cols + kPsCB - 1) / kPsCB);
+            x.nrb3 = int32_t((L.rows + kPsRB3 - 1) / kPsRB3);
+            x.ppart_off = pp;
+            x.pd_off = pd;
+            x.qpart_off = qp;
+            pp += int64_t(x.nch1) * L.rows * L.cap;
+            pd += L.rows * L.cap;
+            qp += int64_t(x.nrb3) * L.cols * L.cap;
+            for (int32_t rb = 0; rb < (L.rows + kPsRB - 1) / kPsRB; ++rb)
+                for (int32_t ch = 0; ch < x.nch1; ++ch) t1.push_back(make_int4(l, rb, ch, 0));
+            for (int32_t rb = 0; rb < x.nrb3; ++rb)
+                for (int32_t ch = 0; ch < x.nch1; ++ch) t3.push_back(make_int4(l, rb, ch, 0));
+            for (int32_t cb = 0; cb < (L.cols + kPsQB - 1) / kPsQB; ++cb)
+                tq.push_back(make_int4(l, cb, 0, 0));
+            ids.push_back(l);
+        }
+        ps[l] = x;
+    }
+    t->ppart_pw = pp;
+    t->pd_pw = pd;
+    t->qpart_pw = qp;
+    t->ps1_ntiles = int32_t(t1.size());
+    t->ps3_ntiles = int32_t(t3.size());
+    t->psq_ntiles = int32_t(tq.size());
+    t->nps = int32_t(ids.size());
+    auto up = [](void** dst, const void* src, size_t bytes) -> int {
+        *dst = nullptr;
+        if (bytes == 0) return GCE_OK;
+        if (cudaMalloc(dst, bytes) != cudaSuccess) return GCE_ERR_NOMEM;
+        return cudaMemcpy(*dst, src, bytes, cudaMemcpyHostToDevice) == cudaSuccess ? GCE_OK
+                                                                                  : GCE_ERR_CUDA;
+    };
+    int rc = up(&t->d_ps, ps.data(), ps.size() * sizeof(PsLayer));
+    if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_ps1_tiles), t1.data(), t1.size() * sizeof(int4));
+    if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_ps3_tiles), t3.data(), t3.size() * sizeof(int4));
+    if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_psq_tiles), tq.data(), tq.size() * sizeof(int4));
+    if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_ps_layers), ids.data(), ids.size() * sizeof(int32_t));
+    return rc;
+}
+
+void powersgd_plan_free(gce_table* t) {
+    cudaFree(t->d_ps);
+    cudaFree(t->d_ps1_tiles);
+    cudaFree(t->d_ps3_tiles);
+    cudaFree(t->d_psq_tiles);
+    cudaFree(t->d_ps_layers);
+}
+
+struct PsWs {
+    size_t ppart = 0, pd = 0, qpart = 0, total = 0;
+};
+
+static PsWs ps_layout(const gce_table* t, int32_t W) {
+    PsWs o;
+    Carver c;
+    o.ppart = c.take<float>(int64_t(W) * t->ppart_pw);
+    o.pd = c.take<double>(int64_t(W) * t->pd_pw);
+    o.qpart = c.take<float>(int64_t(W) * t->qpart_pw);
+    o.total = c.off;
+    return o;
+}
+
+size_t powersgd_ws_bytes(const gce_table* t, int32_t W) { return ps_layout(t, W).total; }
+
+__device__ __forceinline__ int32_t ps_rank(const DevLayer& L, const int32_t* k_or_rank, int32_t l) {
+    const int32_t r = k_or_rank ? k_or_rank[l] : L.cap;
+    return (r >= 1 && r <= L.cap) ? r : 0;
+}
+
+// ---- Q initialisation --------------------------------------------------------------
+__global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
+                                 const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W,
+                                 int64_t Q_pw, uint64_t seed, float* __restrict__ Q) {
+    for (int64_t u = blockIdx.x; u < int64_t(nps) * W; u += gridDim.x) {
+        const int w = int(u / nps);
+        const int32_t l = ps_layers[u % nps];
+        const DevLayer L = layers[l];
+        const uint64_t base = hash_base(seed, 1, uint64_t(w), uint64_t(l), 0);
+        float* q = Q + int64_t(w) * Q_pw + L.q_off;
+        const int64_t n = L.cols * L.cap;
+        for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+            const uint64_t h = mix64(base + uint64_t(i + 1) * kGamma);
+            q[i] = __fsub_rn(__fmul_rn(float(h >> 40), 1.0f / 8388608.0f), 1.0f);
+        }
+    }
+}
+
+// ---- phase 1: M = m + eta*g (written back), partial P = M Q -------------------------------
+__global__ void __launch_bounds__(256) ps_mq_kernel(
+    const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
+    const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t Q_pw,
+    int64_t ppart_pw, const float* __restrict__ grad, float* __restrict__ mem, float eta,
+    const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, float* __restrict__ ppart) {
+    __shared__ float qs[kMaxRank][kPsCB];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
+        const int w = int(u / ntiles);
+        const int4 d = tiles[u % ntiles];
+        const DevLayer L = layers[d.x];
+        const PsLayer X = ps[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        if (r == 0) continue;
+        const int cap = L.cap;
+        const int64_t C = L.cols, R = L.rows;
+        const int64_t c0 = int64_t(d.z) * kPsCB;
+        const int cw = int(min64(kPsCB, C - c0));
+        const int64_t r0 = int64_t(d.y) * kPsRB;
+        const int rh = int(min64(kPsRB, R - r0));
+        const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
+        for (int i = tid; i < cw * r; i += blockDim.x) {
+            const int c = i / r, j = i - c * r;
+            qs[j][c] = q[int64_t(c) * cap + j];
+        }
+        __syncthreads();
+        for (int row = warp; row < rh; row += blockDim.x >> 5) {
+            const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
+            const float* g = grad + e;
+            float* m = mem + e;
+            float acc[kMaxRank] = {0.f, 0.f, 0.f, 0.f};
+            if (((e & 3) == 0) && ((cw & 3) == 0)) {
+                for (int c = lane * 4; c < cw; c += 128) {
+                    const float4 gg = ld_stream4(g + c);
+                    const float4 mm = *reinterpret_cast<const float4*>(m + c);
+                    float4 x;
+                    x.x = residual(mm.x, eta, gg.x);
+                    x.y = residual(mm.y, eta, gg.y);
+                    x.z = residual(mm.z, eta, gg.z);
+                    x.w = residual(mm.w, eta, gg.w);
+                    *reinterpret_cast<float4*>(m + c) = x;
+#pragma unroll
+                    for (int j = 0; j < kMaxRank; ++j) {
+                        if (j < r) {
+                            acc[j] = fmaf(x.x, qs[j][c], acc[j]);
+                            acc[j] = fmaf(x.y, qs[j][c + 1], acc[j]);
+                            acc[j] = fmaf(x.z, qs[j][c + 2], acc[j]);
+                            acc[j] = fmaf(x.w, qs[j][c + 3], acc[j]);
+                        }
+                    }
+                }
+            } else {
+                for (int c = lane; c < cw; c += 32) {
+                    const float x = residual(m[c], eta, __ldcs(g + c));
+                    m[c] = x;
+#pragma unroll
+                    for (int j = 0; j < kMaxRank; ++j)
+                        if (j < r) acc[j] = fmaf(x, qs[j][c], acc[j]);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kMaxRank; ++j) acc[j] = warp_sum(acc[j]);
+            if (lane < r) {
+                float a = acc[0];
+                if (lane == 1) a = acc[1];
+                if (lane == 2) a = acc[2];
+                if (lane == 3) a = acc[3];
+                ppart[int64_t(w) * ppart_pw + X.ppart_off + (int64_t(d.z) * R + r0 + row) * cap + lane] = a;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---- orthonormalise P (one CTA per matrix) ----------------------------------------------
+__device__ __forceinline__ double block_sum_d(double x, double* s_red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    x = warp_sum(x);
+    if (lane == 0) s_red[warp] = x;
+    __syncthreads();
+    double t = 0.0;
+    for (int i = 0; i < nw; ++i) t += s_red[i];
+    __syncthreads();
+    return t;
+}
+
+__global__ void __launch_bounds__(256) ps_orth_kernel(
+    const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
+    const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W, int64_t P_pw, int64_t ppart_pw,
+    int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ ppart,
+    double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status) {
+    __shared__ double s_red[32];
+    for (int64_t u = blockIdx.x; u < int64_t(nps) * W; u += gridDim.x) {
+        const int w = int(u / nps);
+        const int32_t l = ps_layers[u % nps];
+        const DevLayer L = layers[l];
+        const PsLayer X = ps[l];
+        const int r = ps_rank(L, k_or_rank, l);
+        if (r == 0) {
+            if (threadIdx.x == 0) set_status(status, GCE_STATUS_K_RANGE);
+            continue;
+        }
+        const int cap = L.cap;
+        const int64_t R = L.rows;
+        const float* pp = ppart + int64_t(w) * ppart_pw + X.ppart_off;
+        double* pd = pdw + int64_t(w) * pd_pw + X.pd_off;
+        for (int64_t i = threadIdx.x; i < R * r; i += blockDim.x) {
+            const int64_t row = i / r;
+            const int j = int(i - row * r);
+            double s = 0.0;
+            for (int ch = 0; ch < X.nch1; ++ch) s += double(pp[(int64_t(ch) * R + row) * cap + j]);
+            pd[row * cap + j] = s;
+        }
+        __syncthreads();
+        for (int j = 0; j < r; ++j) {
+            for (int i = 0; i < j; ++i) {
+                double part = 0.0;
+                for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
+                    part += pd[row * cap + i] * pd[row * cap + j];
+                const double dot = block_sum_d(part, s_red);
+                for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
+                    pd[row * cap + j] -= dot * pd[row * cap + i];
+                __syncthreads();
+            }
+            double part = 0.0;
+            for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
+                part += pd[row * cap + j] * pd[row * cap + j];
+            const double nu = sqrt(block_sum_d(part, s_red));
+            for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
+                pd[row * cap + j] = nu > 0.0 ? pd[row * cap + j] / nu : 0.0;
+            __syncthreads();
+        }
+        float* p = P + int64_t(w) * P_pw + L.p_off;
+        for (int64_t i = threadIdx.x; i < R * r; i += blockDim.x) {
+            const int64_t row = i / r;
+            const int j = int(i - row * r);
+            p[row * cap + j] = float(pd[row * cap + j]);
+        }
+        __syncthreads();
+    }
+}
+
+// ---- phase 3: partial Q = M^T P over 64-row blocks ---------------------------------------
+__global__ void __launch_bounds__(256) ps_mtp_kernel(
+    const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
+    const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t P_pw,
+    int64_t qpart_pw, const float* __restrict__ mem, const int32_t* __restrict__ k_or_rank,
+    const float* __restrict__ P, float* __restrict__ qpart) {
+    __shared__ float prow[kPsRB3][kMaxRank];
+    const int tid = threadIdx.x;
+    for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
+        const int w = int(u / ntiles);
+        const int4 d = tiles[u % ntiles];
+        const DevLayer L = layers[d.x];
+        const PsLayer X = ps[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        if (r == 0) continue;
+        const int cap = L.cap;
+        const int64_t C = L.cols;
+        const int64_t r0 = int64_t(d.y) * kPsRB3;
+        const int rh = int(min64(kPsRB3, L.rows - r0));
+        const int64_t c0 = int64_t(d.z) * kPsCB;
+        const int cw = int(min64(kPsCB, C - c0));
+        const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+        for (int i = tid; i < rh * kMaxRank; i += blockDim.x) {
+            const int row = i / kMaxRank, j = i % kMaxRank;
+            prow[row][j] = j < r ? p[int64_t(row) * cap + j] : 0.0f;
+        }
+        __syncthreads();
+        const int cc = tid * 4;
+        float acc[4][kMaxRank];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int j = 0; j < kMaxRank; ++j) acc[q][j] = 0.0f;
+        const int64_t ebase = int64_t(w) * N + L.offset + r0 * C + c0;
+        const bool vec = ((ebase & 3) == 0) && ((C & 3) == 0) && (cc + 3 < cw);
+        if (cc < cw) {
+            for (int row = 0; row < rh; ++row) {
+                const float* m = mem + ebase + int64_t(row) * C + cc;
+                float x[4];
+                if (vec) {
+                    const float4 mm = *reinterpret_cast<const float4*>(m);
+                    x[0] = mm.x; x[1] = mm.y; x[2] = mm.z; x[3] = mm.w;
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) x[q] = (cc + q < cw) ? m[q] : 0.0f;
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+#pragma unroll
+                    for (int j = 0; j < kMaxRank; ++j) acc[q][j] = fmaf(x[q], prow[row][j], acc[q][j]);
+            }
+            float* out = qpart + int64_t(w) * qpart_pw + X.qpart_off + (int64_t(d.y) * C + c0 + cc) * cap;
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (cc + q < cw)
+#pragma unroll
+                    for (int j = 0; j < kMaxRank; ++j)
+                        if (j < r) out[q * cap + j] = acc[q][j];
+        }
+        __syncthreads();
+    }
+}
+
+// ---- Q = sum of the row-block partials (fp64, block order) ----------------------------------
+__global__ void __launch_bounds__(256) ps_qred_kernel(
+    const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
+    const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t Q_pw, int64_t qpart_pw,
+    const int32_t* __restrict__ k_or_rank, const float* __restrict__ qpart, float* __restrict__ Q) {
+    for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
+        const int w = int(u / ntiles);
+        const int4 d = tiles[u % ntiles];
+        const DevLayer L = layers[d.x];
+        const PsLayer X = ps[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        if (r == 0) continue;
+        const int cap = L.cap;
+        const int64_t C = L.cols;
+        const int64_t c0 = int64_t(d.y) * kPsQB;
+        const int cw = int(min64(kPsQB, C - c0));
+        const float* qp = qpart + int64_t(w) * qpart_pw + X.qpart_off;
+        float* q = Q + int64_t(w) * Q_pw + L.q_off;
+        for (int i = threadIdx.x; i < cw * r; i += blockDim.x) {
+            const int64_t c = c0 + i / r;
+            const int j = i % r;
+            double s = 0.0;
+            for (int rb = 0; rb < X.nrb3; ++rb) s += double(qp[(int64_t(rb) * C + c) * cap + j]);
+            q[c * cap + j] = float(s);
+        }
+    }
+}
+
+// ---- residual: m <- M - P Q^T, dense_out <- P Q^T ---------------------------------------------
+__global__ void __launch_bounds__(256) ps_resid_kernel(
+    const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles, int32_t W,
+    int64_t N, int64_t P_pw, int64_t Q_pw, const int32_t* __restrict__ k_or_rank,
+    const float* __restrict__ P, const float* __restrict__ Q, float* __restrict__ mem,
+    float* __restrict__ dense_out) {
+    __shared__ float qs[kMaxRank][kPsCB];
+    __shared__ float prow[kPsRB][kMaxRank];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
+        const int w = int(u / ntiles);
+        const int4 d = tiles[u % ntiles];
+        const DevLayer L = layers[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        if (r == 0) continue;
+        const int cap = L.cap;
+        const int64_t C = L.cols, R = L.rows;
+        const int64_t c0 = int64_t(d.z) * kPsCB;
+        const int cw = int(min64(kPsCB, C - c0));
+        const int64_t r0 = int64_t(d.y) * kPsRB;
+        const int rh = int(min64(kPsRB, R - r0));
+        const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
+        for (int i = tid; i < cw * r; i += blockDim.x) {
+            const int c = i / r, j = i - c * r;
+            qs[j][c] = q[int64_t(c) * cap + j];
+        }
+        const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+        for (int i = tid; i < rh * r; i += blockDim.x) {
+            const int row = i / r, j = i - row * r;
+            prow[row][j] = p[int64_t(row) * cap + j];
+        }
+        __syncthreads();
+        for (int row = warp; row < rh; row += blockDim.x >> 5) {
+            const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
+            float* m = mem + e;
+            float* o = dense_out ? dense_out + e : nullptr;
+            float pr[kMaxRank];
+#pragma unroll
+            for (int j = 0; j < kMaxRank; ++j) pr[j] = j < r ? prow[row][j] : 0.0f;
+            for (int c = lane; c < cw; c += 32) {
+                float mh = __fmul_rn(pr[0], qs[0][c]);
+#pragma unroll
+                for (int j = 1; j < kMaxRank; ++j)
+                    if (j < r) mh = __fmaf_rn(pr[j], qs[j][c], mh);
+                m[c] = __fsub_rn(m[c], mh);
+                if (o) o[c] = mh;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+static int grid_of(int64_t work, int per_sm) {
+    return int(max64(1, min64(work, int64_t(sm_count()) * per_sm)));
+}
+
+}  // namespace gce
+
+using namespace gce;
+
+extern "C" int powersgd_init_q(const gce_table* t, int32_t W, uint64_t seed, float* Q, void* stream) {
+    if (!t || W < 1) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    if (t->nps == 0) return GCE_OK;
+    if (!Q || !aligned16(Q)) return GCE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    GCE_LAUNCH(ps_init_q_kernel, grid_of(int64_t(t->nps) * W, 4), 256, 0, st, t->d_layers,
+               t->d_ps_layers, t->nps, W, t->Q_pw, seed, Q);
+    return check_launch();
+}
+
+extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
+                             const int32_t* k_or_rank, float* P, float* Q, float* vals,
+                             float* dense_out, void* ws, size_t ws_bytes, void* stream) {
+    if (!t || W < 1 || !grad || !mem || !ws) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    if (!aligned16(grad) || !aligned16(mem) || !aligned16(ws)) return GCE_ERR_ARG;
+    if (t->nps > 0 && (!P || !Q || !aligned16(P) || !aligned16(Q))) return GCE_ERR_ARG;
+    if (dense_out && !aligned16(dense_out)) return GCE_ERR_ARG;
+    if (k_or_rank && (reinterpret_cast<uintptr_t>(k_or_rank) & 3)) return GCE_ERR_ARG;
+    const PsWs lay = ps_layout(t, W);
+    if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(ws);
+    if (t->nps > 0) {
+        float* ppart = at<float>(ws, lay.ppart);
+        double* pd = at<double>(ws, lay.pd);
+        float* qpart = at<float>(ws, lay.qpart);
+        const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
+        GCE_LAUNCH(ps_mq_kernel, grid_of(int64_t(t->ps1_ntiles) * W, 8), 256, 0, st, t->d_layers,
+                   ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw, t->ppart_pw, grad, mem,
+                   eta, k_or_rank, Q, ppart);
+        GCE_LAUNCH(ps_orth_kernel, grid_of(int64_t(t->nps) * W, 8), 256, 0, st, t->d_layers, ps,
+                   t->d_ps_layers, t->nps, W, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
+                   pd, P, status);
+        GCE_LAUNCH(ps_mtp_kernel, grid_of(int64_t(t->ps3_ntiles) * W, 8), 256, 0, st,
+                   t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->P_pw, t->qpart_pw,
+                   mem, k_or_rank, P, qpart);
+        GCE_LAUNCH(ps_qred_kernel, grid_of(int64_t(t->psq_ntiles) * W, 8), 256, 0, st,
+                   t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
+                   k_or_rank, qpart, Q);
+        GCE_LAUNCH(ps_resid_kernel, grid_of(int64_t(t->ps1_ntiles) * W, 8), 256, 0, st,
+                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
+                   k_or_rank, P, Q, mem, dense_out);
+        if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+    }
+    return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+}

@@ -31,26 +31,6 @@ namespace gce {
 
 extern double bracket_sigma();
 
-constexpr uint64_t kGamma = 0x9E3779B97F4A7C15ull;
-
-__host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
-    z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-    z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-    return z ^ (z >> 31);
-}
-
-// state of (seed, stream, worker, layer, step): each field folded in as the
-// first SplitMix64 output from (previous + (field + 1) * gamma)
-__host__ __device__ __forceinline__ uint64_t hash_base(uint64_t seed, uint64_t stream,
-                                                       uint64_t worker, uint64_t layer,
-                                                       uint64_t step) {
-    uint64_t h = mix64(seed + (stream + 1) * kGamma);
-    h = mix64(h + (worker + 1) * kGamma);
-    h = mix64(h + (layer + 1) * kGamma);
-    h = mix64(h + (step + 1) * kGamma);
-    return h;
-}
-
 struct RkSeg {
     int32_t k;       // 0: layer skipped
     uint32_t lo, hi; // band of candidate keys

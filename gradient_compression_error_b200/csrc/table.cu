@@ -125,6 +125,8 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_dc_tile_layer);
     cudaFree(t->d_bunit_layer);
     cudaFree(t->d_bunit_chunk);
+    powersgd_plan_free(t);
+    accordion_plan_free(t);
     delete t;
 }
 
@@ -249,6 +251,8 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_dc_tile_layer, dc_tile_layer);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_layer, bunit_layer);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_chunk, bunit_chunk);
+    if (rc == GCE_OK) rc = powersgd_plan(t);
+    if (rc == GCE_OK) rc = accordion_plan(t);
     if (rc != GCE_OK) {
         free_table(t);
         return rc;
