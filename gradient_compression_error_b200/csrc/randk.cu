@@ -200,6 +200,7 @@ __device__ void cta_select_pair(const RkEntry* __restrict__ list, int32_t count,
         __syncthreads();
     }
     const uint32_t key_T = *s_pref;
+    __syncthreads();  // every thread has read key_T before the prefix is reset
     if (tid == 0) *s_pref = 0;
     __syncthreads();
     // among keys == T: index bits 30..20, 19..9, 8..0

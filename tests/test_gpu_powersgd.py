@@ -54,6 +54,7 @@ class PsRun:
         r = [l["cap"] for l in self.layers] if ranks is None else ranks
         expect = osteps.powersgd_step(self.layers, host(grad), self.hmem, eta, r, self.hQ,
                                       threads=8)
+        Q_before = host(self.Q).copy()
         self.g.powersgd_step(self.t, self.W, grad, self.mem, eta, kt, self.P, self.Q, self.vals,
                              self.out, self.ws)
         torch.cuda.synchronize()
@@ -82,7 +83,9 @@ class PsRun:
                     relerr(hm[w, ls], self.hmem[w, ls], Mfull)]
             assert max(errs) <= TOL, (w, l, errs)
             worst = max(worst, max(errs))
-            assert np.array_equal(bits(Q_gpu[:, rr:]), bits(Q_ref[:, rr:]))   # untouched columns
+            # columns >= r are left as they were (the GPU's own previous values)
+            Q_prev = Q_before[w, info["q_offset"]:info["q_offset"] + cols * cap].reshape(cols, cap)
+            assert np.array_equal(bits(Q_gpu[:, rr:]), bits(Q_prev[:, rr:]))
         return worst
 
 
