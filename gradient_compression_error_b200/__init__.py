@@ -71,6 +71,8 @@ SIGNATURES = {
                                    _vp, C.c_size_t, _vp]),
     "decompress_accumulate": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
                                         C.c_size_t, _vp]),
+    "decompress_accumulate_noalloc": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _f32, _vp,
+                                                _vp]),
     "gce_status": (C.c_int, [_vp, _vp, C.POINTER(_i32)]),
     "gce_launch_count": (_u64, []),
     "gce_error_string": (C.c_char_p, [C.c_int]),
@@ -228,6 +230,14 @@ def decompress_accumulate(table, W, vals, idx, k_or_rank, P, Q, scale, out, ws, 
         table.handle, int(W), _ptr(vals, _f32()), _ptr(idx, _i32()), _ptr(k_or_rank, _i32()),
         _ptr(P, _f32()), _ptr(Q, _f32()), float(scale), _ptr(out, _f32()), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def decompress_accumulate_noalloc(table, W, vals, idx, k_or_rank, P, Q, scale, out, stream=None):
+    """decompress_accumulate for callers that cannot allocate a workspace: the
+    library's fixed 4 MiB scratch is used instead (see include/gce.h)."""
+    _check("decompress_accumulate_noalloc", lib().decompress_accumulate_noalloc(
+        table.handle, int(W), _ptr(vals, _f32()), _ptr(idx, _i32()), _ptr(k_or_rank, _i32()),
+        _ptr(P, _f32()), _ptr(Q, _f32()), float(scale), _ptr(out, _f32()), _stream(stream)))
 
 
 def status(ws, stream=None):

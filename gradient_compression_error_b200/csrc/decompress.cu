@@ -13,6 +13,8 @@
 // pass (bounds) turns each (worker, layer) list into per-tile entry ranges
 // by comparing neighbouring indices -- no searching.  DRAM traffic: the
 // payload read once plus one 4-byte write per output element.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace gce {
@@ -141,6 +143,62 @@ extern "C" int decompress_accumulate(const gce_table* t, int32_t W, const float*
     if (ws_bytes < decompress_ws_bytes(t, W)) return GCE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t* bounds = at<int32_t>(ws, GCE_WS_HEADER_BYTES);
+    const int sms = sm_count();
+    if (sparse && t->bunits_pw > 0) {
+        const int64_t units = int64_t(t->bunits_pw) * W;
+        GCE_LAUNCH(dc_bounds_kernel, int(min64(units, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
+                   t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
+                   k_or_rank, idx, bounds);
+    }
+    GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
+               t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots,
+               k_or_rank, vals, idx, P, Q, bounds, scale, out);
+    return check_launch();
+}
+
+// ---- decode without a caller workspace -------------------------------------------------
+// Some callers cannot hand the library a workspace: code that runs inside
+// another allocator (a caching allocator's out-of-memory hook, for one), code
+// whose device memory is all reserved up front by its framework, and code in
+// a latency-critical loop that must not pay cudaMalloc's implicit device-wide
+// synchronisation.  For them, decompress_accumulate_noalloc keeps its only
+// scratch -- the per-tile entry bounds -- in the fixed array below, which the
+// module reserves on every GPU that loads this library until the process
+// exits.  4 MiB: W x (decode tiles of 4096 elements + layers) <= 1,048,576
+// bound slots (the BERT-base table at W = 8 uses 214,144).
+constexpr int64_t kNoAllocBoundSlots = int64_t(1) << 20;
+static __device__ __align__(256) int32_t g_noalloc_bounds[kNoAllocBoundSlots];
+
+// Device address of g_noalloc_bounds on the current device, looked up once per
+// device (host code cannot use the symbol itself as a device address).
+static int32_t* noalloc_bounds_on_current_device() {
+    static std::mutex mu;
+    static int32_t* addr[64] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_bounds) != cudaSuccess || !p) return nullptr;
+        addr[dev] = static_cast<int32_t*>(p);
+    }
+    return addr[dev];
+}
+
+extern "C" int decompress_accumulate_noalloc(const gce_table* t, int32_t W, const float* vals,
+                                             const int32_t* idx, const int32_t* k_or_rank,
+                                             const float* P, const float* Q, float scale,
+                                             float* out, void* stream) {
+    if (!t || W < 1 || !out || !aligned16(out)) return GCE_ERR_ARG;
+    const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
+    if ((t->vals_pw > 0 && !vals) || (sparse && !idx)) return GCE_ERR_ARG;
+    if (t->ckind == GCE_KIND_POWERSGD && (!P || !Q)) return GCE_ERR_ARG;
+    if (int64_t(W) * t->dc_slots > kNoAllocBoundSlots) return GCE_ERR_WORKSPACE;
+    int32_t* bounds = noalloc_bounds_on_current_device();
+    if (!bounds) return GCE_ERR_CUDA;
+    // every bound slot a sparse layer uses is rewritten by the bounds pass, so
+    // nothing left from an earlier call needs clearing
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int sms = sm_count();
     if (sparse && t->bunits_pw > 0) {
         const int64_t units = int64_t(t->bunits_pw) * W;

@@ -232,6 +232,29 @@ GCE_API int decompress_accumulate(const gce_table* table, int32_t W, const float
                           const float* Q, float scale, float* out, void* ws, size_t ws_bytes,
                           void* stream);
 
+/*
+ * decompress_accumulate without a workspace (the pages have no counterpart:
+ * this is a deployment variant, not part of the method).  For callers that
+ * cannot allocate device memory for a workspace -- code running inside
+ * another allocator such as a caching allocator's out-of-memory hook, code
+ * whose device memory is reserved in full by its framework up front, or a
+ * latency-critical loop that must not pay cudaMalloc's implicit device-wide
+ * synchronisation.  Same arguments, results and preconditions as
+ * decompress_accumulate minus ws / ws_bytes; it allocates nothing.  Its
+ * scratch is a fixed 4 MiB array inside the library, reserved on every GPU
+ * that loads the library until the process exits, so the table and W must
+ * satisfy W x (decode tiles of 4096 elements + layers) <= 1,048,576 (the
+ * BERT-base table at W = 8 needs 214,144); larger ones return
+ * GCE_ERR_WORKSPACE.  The first call on a device looks up that device's copy
+ * of the array (cudaGetSymbolAddress), so make it before any stream capture.
+ * All calls share the one array: calls that overlap on the GPU (two streams,
+ * two threads) race and must be serialised by the caller.
+ */
+GCE_API int decompress_accumulate_noalloc(const gce_table* table, int32_t W, const float* vals,
+                                          const int32_t* idx, const int32_t* k_or_rank,
+                                          const float* P, const float* Q, float scale,
+                                          float* out, void* stream);
+
 /* Wait for `stream`, then read and clear the status word of workspace `ws`
  * (device pointer).  *status receives GCE_STATUS_* bits (0 = clean). */
 GCE_API int gce_status(void* ws, void* stream, int32_t* status);

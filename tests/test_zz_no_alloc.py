@@ -1,0 +1,78 @@
+"""decompress_accumulate_noalloc: the decoder for callers that cannot allocate.
+
+Callers that run inside another allocator, whose device memory is reserved in
+full by their framework, or that must not pay cudaMalloc's implicit device
+synchronisation cannot hand the library a workspace.  This entry point keeps
+its scratch in a fixed array inside the library instead; its output must be
+the workspace decoder's, bit for bit (the tolerance the sparse decode tests
+use), call after call -- the shared array keeps the previous call's contents.
+Collected last on purpose (file name), so a stop-at-first-failure run has
+already run every other test.
+"""
+import ctypes as C
+
+import numpy as np
+import pytest
+
+from tests.helpers import gce, need_gpu, torch
+
+pytestmark = pytest.mark.gpu
+
+
+def random_payload(table, layers, W, seed):
+    rng = np.random.default_rng(seed)
+    vals = np.zeros((W, table.vals_per_worker), np.float32)
+    idx = np.zeros((W, table.vals_per_worker), np.int32)
+    for w in range(W):
+        for l, lay in enumerate(layers):
+            o = table.info[l]["val_offset"]
+            n = lay["rows"] * lay["cols"]
+            if lay["kind"] == "dense":
+                vals[w, o:o + n] = rng.standard_normal(n)
+            else:
+                k = lay["cap"]
+                idx[w, o:o + k] = np.sort(rng.choice(n, k, replace=False))
+                vals[w, o:o + k] = rng.standard_normal(k) * 10.0 ** rng.uniform(-3, 3, k)
+    return torch.from_numpy(vals).cuda(), torch.from_numpy(idx).cuda()
+
+
+def call_noalloc(lib, table, W, vals, idx, scale, out):
+    stream = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    return lib.decompress_accumulate_noalloc(
+        table.handle, W, C.c_void_p(vals.data_ptr()), C.c_void_p(idx.data_ptr()), None, None,
+        None, C.c_float(scale), C.c_void_p(out.data_ptr()), stream)
+
+
+def test_noalloc_decode_matches_workspace_decode_twice():
+    need_gpu()
+    g = gce()
+    lib = g.lib()
+    layers = [dict(rows=50000, cols=7, kind="topk", cap=3500),
+              dict(rows=333, cols=1, kind="dense", cap=0),
+              dict(rows=4096, cols=1, kind="topk", cap=4096),
+              dict(rows=1, cols=1, kind="topk", cap=1),
+              dict(rows=300001, cols=1, kind="topk", cap=30000)]
+    W = 4
+    table = g.Table(layers)
+    ws = table.workspace(W, "decompress")
+    for call, (seed, scale) in enumerate([(1, 1.0), (2, 0.25)]):
+        vals, idx = random_payload(table, layers, W, seed)
+        want = torch.full((table.N,), float("nan"), device="cuda")
+        got = torch.full((table.N,), float("nan"), device="cuda")
+        g.decompress_accumulate(table, W, vals, idx, None, None, None, scale, want, ws)
+        assert call_noalloc(lib, table, W, vals, idx, scale, got) == 0
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int32), want.view(torch.int32)), call
+
+
+def test_noalloc_rejects_tables_beyond_its_scratch():
+    need_gpu()
+    g = gce()
+    lib = g.lib()
+    layers = [dict(rows=1 << 24, cols=1, kind="topk", cap=10)]    # 4097 bound slots per worker
+    table = g.Table(layers)
+    W = 256                                                        # 1,048,832 > 1,048,576
+    vals = torch.zeros((1, 16), device="cuda")
+    idx = torch.zeros((1, 16), dtype=torch.int32, device="cuda")
+    out = torch.zeros(16, device="cuda")
+    assert call_noalloc(lib, table, W, vals, idx, 1.0, out) == -3   # GCE_ERR_WORKSPACE
