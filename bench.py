@@ -36,7 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "gradient elements encoded+decoded per sec (GB/s vs HBM roofline); ms per step"
 UNIT = "elements/s"
 DEFAULT_WORKLOAD = "bert_base_topk1pct_w8"
-MAIN_KERNEL = "tk_main_kernel<true>"
+MAIN_KERNEL = "tk_main_kernel"
 MAIN_SOURCE = os.path.join(ROOT, "gradient_compression_error_b200", "csrc", "topk.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "tk_main_bert_base_w8_traffic.txt")
 FALLBACK_HBM_GBS = 6650.0
@@ -46,6 +46,8 @@ def workload_spec(name):
     from gradient_compression_error_b200 import workloads as wl
     if name == "bert_base_topk1pct_w8":
         return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk")
+    if name == "bert_base_topk1pct_w1":          # one replica: a profiling-sized case
+        return dict(layers=wl.bert_base_topk(), W=1, cfg=4, method="topk")
     if name == "memsgd_vector_2p20":
         return dict(layers=wl.memsgd_vector(), W=1, cfg=1, method="topk")
     if name.startswith("sweep_topk_e"):          # e.g. sweep_topk_e28_ppm10000

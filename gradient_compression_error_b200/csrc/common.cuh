@@ -144,6 +144,12 @@ __device__ __forceinline__ float4 ld_stream4(const float* p) {
     return __ldcs(reinterpret_cast<const float4*>(p));
 }
 
+// Bulk (TMA-engine) prefetch of a contiguous range into L2: one instruction
+// for `bytes` (a multiple of 16) starting at a 16-byte aligned address.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 // host entry points shared between translation units
 constexpr int kDcTileLog = 12;              // decode tile: 4096 output elements
 constexpr int kDcTile = 1 << kDcTileLog;

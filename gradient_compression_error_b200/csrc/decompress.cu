@@ -16,8 +16,11 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "scan.cuh"
 
 namespace gce {
+
+constexpr int kDcStage = 2048;  // payload entries staged in shared memory per tile
 
 size_t decompress_ws_bytes(const gce_table* t, int32_t W) {
     Carver c;
@@ -74,6 +77,10 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
     const int32_t* __restrict__ idx, const float* __restrict__ P, const float* __restrict__ Q,
     const int32_t* __restrict__ bounds, float scale, float* __restrict__ out) {
     __shared__ float acc[kDcTile];
+    __shared__ int32_t s_first[32], s_off[33];
+    __shared__ int32_t s_sidx[kDcStage];
+    __shared__ float s_sval[kDcStage];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int32_t t = blockIdx.x; t < dc_tiles; t += gridDim.x) {
         const int32_t l = dc_tile_layer[t];
         const DevLayer L = layers[l];
@@ -84,15 +91,53 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
         if (L.kind == GCE_KIND_TOPK || L.kind == GCE_KIND_RANDK) {
             const int32_t k = layer_k(L, k_or_rank, l);
             for (int i = threadIdx.x; i < cnt; i += blockDim.x) acc[i] = 0.0f;
-            for (int w = 0; w < W; ++w) {
-                __syncthreads();
-                const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base + tt;
-                const int32_t a = min(max(b[0], 0), k), e = min(max(b[1], a), k);
-                const float* v = vals + int64_t(w) * vals_pw + L.val_off;
-                const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
-                for (int32_t j = a + threadIdx.x; j < e; j += blockDim.x) {
-                    const int64_t i = int64_t(ix[j]) - start;
-                    if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], v[j]);
+            // every worker's entry range for this tile at once, then one staged
+            // load of all the entries, so the worker-order sums below touch
+            // only shared memory
+            if (W <= 32 && warp == 0) {
+                int32_t a = 0, e = 0;
+                if (lane < W) {
+                    const int32_t* b = bounds + int64_t(lane) * dc_slots + L.dc_base + tt;
+                    a = min(max(b[0], 0), k);
+                    e = min(max(b[1], a), k);
+                    s_first[lane] = a;
+                }
+                const int c = e - a;
+                const int incl = warp_inclusive_scan(c);
+                if (lane < W) s_off[lane] = incl - c;
+                if (lane == 31) s_off[32] = incl;
+            }
+            __syncthreads();
+            const bool staged = W <= 32 && s_off[32] <= kDcStage;
+            if (staged) {
+                const int total = s_off[32];
+                for (int q = threadIdx.x; q < total; q += blockDim.x) {
+                    int w = 0;
+                    while (w + 1 < W && s_off[w + 1] <= q) ++w;
+                    const int64_t j = int64_t(s_first[w]) + (q - s_off[w]);
+                    const int64_t o2 = int64_t(w) * vals_pw + L.val_off + j;
+                    s_sidx[q] = int32_t(int64_t(idx[o2]) - start);
+                    s_sval[q] = vals[o2];
+                }
+                for (int w = 0; w < W; ++w) {
+                    __syncthreads();
+                    for (int q = s_off[w] + threadIdx.x; q < s_off[w + 1 < W ? w + 1 : 32];
+                         q += blockDim.x) {
+                        const int i = s_sidx[q];
+                        if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], s_sval[q]);
+                    }
+                }
+            } else {
+                for (int w = 0; w < W; ++w) {
+                    __syncthreads();
+                    const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base + tt;
+                    const int32_t a = min(max(b[0], 0), k), e = min(max(b[1], a), k);
+                    const float* v = vals + int64_t(w) * vals_pw + L.val_off;
+                    const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
+                    for (int32_t j = a + threadIdx.x; j < e; j += blockDim.x) {
+                        const int64_t i = int64_t(ix[j]) - start;
+                        if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], v[j]);
+                    }
                 }
             }
             __syncthreads();

@@ -6,22 +6,28 @@
 // the memory keeps v except on the chosen set, where it becomes +0.
 //
 // Design (one launch per phase over every (worker, layer) of the table):
-//   setup   per-layer k, clear counters and histograms
-//   sample  read one 128-byte run of grad/mem per 2048 elements, histogram the
-//           |v| keys, and pick a lower bound lo that keeps the k-th largest
-//           key above it with a wide statistical margin
-//   main    the only full pass over HBM: v = fl(m + fl(eta*g)), mem <- v, and
-//           every element with key >= lo is appended (in index order within
-//           its 8192-element tile) to the layer's candidate list
-//   respill exact fallback: a layer whose candidate list came out shorter
-//           than k is re-listed whole from mem (rare; correctness never
-//           depends on the sample)
-//   hist1-3 three 11/11/9-bit radix levels over the candidate lists find the
-//           exact k-th largest key T and how many keys equal to T to take
+//   setup    per-layer k, clear counters and histograms
+//   sample   read one 128-byte run of grad/mem per 2048 elements, histogram
+//            the |v| keys and, interpolating inside the crossing bins, pick
+//            two bounds with a wide statistical margin: lo (the k-th largest
+//            key lies above it) and hi (almost surely chosen above it)
+//   main     the only full pass over HBM: v = fl(m + fl(eta*g)); memory <- v,
+//            or +0 when key > hi; every element with key >= lo is appended, in
+//            index order within its 8192-element tile, to the layer's
+//            candidate list (values and indices in two arrays)
+//   units    per layer: a short list (fewer than k candidates) sends the layer
+//            to the exact fallback; histogram work is cut into units
+//   restore  + respill  the fallback: memory zeroed above hi gets v back
+//            from the candidate list, then the layer is re-listed whole
+//   hist1-3  three 11/11/9-bit radix levels over the candidate values find
+//            the exact k-th largest key T and how many keys equal to T to take
 //   count / scan / emit   per-tile counts of key > T and key == T, a prefix
-//           over the tiles, and the ordered write of (v, i) plus mem[i] = +0
-// DRAM traffic is 12 B per element (read grad and mem, write mem) plus
-// about 8 B per candidate (a few % of the elements) and the payload.
+//            over the tiles, then the ordered write of (v, i); memory +0 for
+//            chosen entries at or below hi, v again for entries above hi that
+//            were not chosen
+// Results never depend on lo or hi.  DRAM traffic: 12 B per element (read
+// grad and mem, write mem) plus about 8 B per candidate (about 1.5 % of the
+// elements), the payload, and a few scattered memory writes.
 #include <cmath>
 
 #include "common.cuh"
@@ -31,10 +37,12 @@
 namespace gce {
 
 static double g_bracket_sigma = 6.0;
+double bracket_sigma() { return g_bracket_sigma; }
 
 struct TkLayout {
     int64_t S = 0, TT = 0;
-    size_t segs = 0, hists = 0, unit_start = 0, tile_dir = 0, tile_cnt = 0, spill = 0, total = 0;
+    size_t segs = 0, hists = 0, unit_start = 0, redo_list = 0, tile_dir = 0, tile_cnt = 0,
+           spill_v = 0, spill_i = 0, total = 0;
 };
 
 static TkLayout tk_layout(const gce_table* t, int32_t W) {
@@ -43,20 +51,33 @@ static TkLayout tk_layout(const gce_table* t, int32_t W) {
     o.S = (t->ckind == GCE_KIND_TOPK) ? int64_t(W) * int64_t(t->comp.size()) : 0;
     o.TT = (t->ckind == GCE_KIND_TOPK) ? int64_t(W) * t->tiles_pw : 0;
     o.segs = c.take<TkSeg>(o.S);
-    o.hists = c.take<int32_t>(o.S * 4 * kTkBins);
+    o.hists = c.take<int32_t>(o.S * (kTkSBins + 3 * kTkBins));
     o.unit_start = c.take<int32_t>(o.S + 1);
+    o.redo_list = c.take<int32_t>(o.TT + 1);
     o.tile_dir = c.take<int2>(o.TT);
     o.tile_cnt = c.take<int2>(o.TT);
-    o.spill = c.take<TkEntry>(o.S ? int64_t(W) * t->comp_N : 0);
+    o.spill_v = c.take<float>(o.S ? int64_t(W) * t->comp_N : 0);
+    o.spill_i = c.take<int32_t>(o.S ? int64_t(W) * t->comp_N : 0);
     o.total = c.off;
     return o;
 }
 
 size_t topk_ws_bytes(const gce_table* t, int32_t W) { return tk_layout(t, W).total; }
 
-// hist(level, seg): level 0 = sample, 1..3 = radix levels
+// hist(level, seg): level 0 = sample (kTkSBins bins), 1..3 = radix levels (kTkBins)
 __device__ __forceinline__ int32_t* tk_hist(int32_t* hists, int64_t S, int level, int64_t seg) {
-    return hists + (int64_t(level) * S + seg) * kTkBins;
+    if (level == 0) return hists + seg * kTkSBins;
+    return hists + S * kTkSBins + (int64_t(level - 1) * S + seg) * kTkBins;
+}
+
+// Shared-memory histogram add, combining lanes of a warp that hit the same bin
+// (candidate keys cluster in a few bins).  Call with the whole warp.
+__device__ __forceinline__ void hist_add(int32_t* h, uint32_t bin, bool take) {
+    const unsigned active = __ballot_sync(kFull, take);
+    if (take) {
+        const unsigned peers = __match_any_sync(active, bin);
+        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
+    }
 }
 
 // ---- setup -------------------------------------------------------------------
@@ -72,25 +93,43 @@ __global__ void __launch_bounds__(256) tk_setup_kernel(const DevLayer* __restric
         hists4[i] = make_int4(0, 0, 0, 0);
     for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S; s += stride) {
         const DevLayer L = layers[comp[s % ncomp]];
-        const int32_t cap = L.cap;
-        const int32_t k = k_or_rank ? k_or_rank[comp[s % ncomp]] : cap;
+        const int32_t k = k_or_rank ? k_or_rank[comp[s % ncomp]] : L.cap;
         TkSeg g{};
-        if (k >= 1 && k <= cap && int64_t(k) <= L.n) {
+        if (k >= 1 && k <= L.cap && int64_t(k) <= L.n) {
             g.k = k;
         } else {
             g.k = 0;
             set_status(status, GCE_STATUS_K_RANGE);
         }
-        g.lo = 0;  // layers too small to sample keep every element as a candidate
+        g.lo = 0;            // layers too small to sample list every element
+        g.hi = 0xFFFFFFFFu;  // and zero nothing in the main pass
         segs[s] = g;
     }
 }
 
-// ---- sample + bracket ----------------------------------------------------------
+// ---- sample + bounds ----------------------------------------------------------
 __host__ __device__ inline int64_t tk_samples_in(int64_t n) {
     const int64_t nch = (n + kTkSampleStride - 1) / kTkSampleStride;
     const int64_t last = n - (nch - 1) * kTkSampleStride;
     return (nch - 1) * kTkSampleChunk + (last < kTkSampleChunk ? last : kTkSampleChunk);
+}
+
+// Sample bins of 2^19 keys (16 per octave of |v|), counted from the top.
+// Lower bound: the bottom edge of the bin where `target` sampled keys are
+// reached.  The density of |v| falls inside a tail bin, so interpolating
+// would put this bound too high; the edge keeps the margin.  Upper bound
+// (interp): linear inside the bin, which errs towards fewer keys above it --
+// the safe side for a bound that only saves memory writes.  -1: not reached.
+// Run by one full warp.
+__device__ __forceinline__ int64_t tk_sample_key(const int32_t* h, int64_t target, bool interp) {
+    int64_t above = 0;
+    const int b = warp_find_from_top(h, kTkSBins, target, &above);
+    if (b < 0) return -1;
+    const int64_t bottom = int64_t(b) << 19;
+    if (!interp) return bottom;
+    const double f = double(target - above) / double(h[b]);
+    const int64_t key = ((int64_t(b) + 1) << 19) - int64_t(floor(f * 524288.0));
+    return key < bottom ? bottom : key;
 }
 
 __global__ void __launch_bounds__(256) tk_sample_kernel(
@@ -98,7 +137,8 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
     const int32_t* __restrict__ sunit_part, int32_t sunits_pw, int32_t W, int32_t ncomp,
     int64_t S, int64_t N, const float* __restrict__ grad, const float* __restrict__ mem,
     float eta, TkSeg* __restrict__ segs, int32_t* __restrict__ hists, double sigma) {
-    __shared__ int32_t h[kTkBins];
+    constexpr int kBatch = 16;
+    __shared__ int32_t h[kTkSBins];
     __shared__ int s_last;
     const int tid = threadIdx.x;
     const int64_t total = int64_t(sunits_pw) * W;
@@ -109,25 +149,31 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
         const int64_t seg = int64_t(w) * ncomp + L.sidx;
         const int32_t k = segs[seg].k;
         if (k == 0) continue;
-        for (int b = tid; b < kTkBins; b += blockDim.x) h[b] = 0;
+        for (int b = tid; b < kTkSBins; b += blockDim.x) h[b] = 0;
         __syncthreads();
         const int64_t p0 = int64_t(sunit_part[su]) * kTkSamplePart;
-        const int64_t pend = min(L.n, p0 + kTkSamplePart);
+        const int64_t pend = min64(L.n, p0 + kTkSamplePart);
         const int64_t nch = (pend - p0 + kTkSampleStride - 1) / kTkSampleStride;
         const int64_t ne = nch * kTkSampleChunk;
         const float* g = grad + int64_t(w) * N + L.offset;
         const float* m = mem + int64_t(w) * N + L.offset;
-#pragma unroll 4
-        for (int64_t e = tid; e < ne; e += blockDim.x) {
-            const int64_t pos = p0 + (e / kTkSampleChunk) * kTkSampleStride + (e % kTkSampleChunk);
-            if (pos < L.n) {
-                const float v = residual(m[pos], eta, __ldcs(g + pos));
-                atomicAdd(&h[abs_key(v) >> 20], 1);
+        for (int64_t e0 = 0; e0 < ne; e0 += int64_t(kBatch) * blockDim.x) {
+            float vv[kBatch];
+            bool ok[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int64_t e = e0 + int64_t(q) * blockDim.x + tid;
+                const int64_t pos = p0 + (e / kTkSampleChunk) * kTkSampleStride + (e % kTkSampleChunk);
+                ok[q] = e < ne && pos < L.n;
+                vv[q] = ok[q] ? residual(m[pos], eta, __ldcs(g + pos)) : 0.0f;
             }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q)
+                if (ok[q]) atomicAdd(&h[abs_key(vv[q]) >> 19], 1);
         }
         __syncthreads();
         int32_t* gh = tk_hist(hists, S, 0, seg);
-        for (int b = tid; b < kTkBins; b += blockDim.x)
+        for (int b = tid; b < kTkSBins; b += blockDim.x)
             if (h[b]) atomicAdd(gh + b, h[b]);
         __threadfence();
         __syncthreads();
@@ -138,36 +184,41 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
         __syncthreads();
         if (s_last) {
             __threadfence();
-            for (int b = tid; b < kTkBins; b += blockDim.x) h[b] = __ldcg(gh + b);
+            for (int b = tid; b < kTkSBins; b += blockDim.x) h[b] = __ldcg(gh + b);
             __syncthreads();
             if (tid < 32) {
                 const int64_t ns = tk_samples_in(L.n);
                 const double mu = double(k) * double(ns) / double(L.n);
-                const double tgt = mu + sigma * (sqrt(mu) + 1.0);
-                int64_t target = int64_t(ceil(tgt));
-                if (target < 1) target = 1;
-                uint32_t lo = 0;
-                if (target <= ns) {
-                    int64_t above = 0;
-                    const int b = warp_find_from_top(h, kTkBins, target, &above);
-                    if (b > 0) lo = uint32_t(b) << 20;
+                const double margin = sigma * (sqrt(mu) + 1.0);
+                int64_t t_lo = int64_t(ceil(mu + margin));
+                if (t_lo < 1) t_lo = 1;
+                const int64_t t_hi = int64_t(floor(mu - margin));
+                uint32_t lo = 0, hi = 0xFFFFFFFFu;
+                if (t_lo <= ns) {
+                    const int64_t key = tk_sample_key(h, t_lo, false);
+                    if (key > 0) lo = uint32_t(key);
                 }
-                if (tid == 0) segs[seg].lo = lo;
+                if (t_hi >= 1) {
+                    const int64_t key = tk_sample_key(h, t_hi, true);
+                    if (key >= 0) hi = uint32_t(key);
+                }
+                if (hi < lo) hi = lo;  // everything zeroed above hi must be a candidate
+                if (tid == 0) {
+                    segs[seg].lo = lo;
+                    segs[seg].hi = hi;
+                }
             }
         }
         __syncthreads();
     }
 }
 
-// ---- main pass / fallback re-listing ------------------------------------------------
-// kCompute: v = fl(m + fl(eta*g)) and mem <- v; otherwise v = mem (the fallback
-// re-lists a whole layer whose candidate list came out shorter than k).
-template <bool kCompute>
+// ---- main pass -------------------------------------------------------------------------
 __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, const float* __restrict__ grad,
     float* __restrict__ mem, float eta, TkSeg* __restrict__ segs, int2* __restrict__ tile_dir,
-    TkEntry* __restrict__ spill) {
+    float* __restrict__ spill_v, int32_t* __restrict__ spill_i) {
     constexpr int kIters = kTkPerThread / 4;           // 8 float4 per thread
     constexpr int kWarps = kTkThreads / 32;            // 8
     __shared__ int32_t s_wt[kIters * kWarps];
@@ -178,18 +229,23 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
         const DevLayer L = layers[tile_layer[lt]];
+        // keep DRAM busy through this tile's compaction: the bulk-copy engine
+        // pulls this block's next tile of grad and mem into L2 meanwhile
+        if (tid == 0 && t + gridDim.x < total) {
+            const int64_t t2 = t + gridDim.x;
+            const int lt2 = int(t2 % tiles_pw);
+            const DevLayer L2 = layers[tile_layer[lt2]];
+            const int64_t s2 = int64_t(lt2 - L2.tile0) * kTkTile;
+            const int64_t e2 = int64_t(t2 / tiles_pw) * N + L2.offset + s2;
+            if (s2 + kTkTile <= L2.n && (e2 & 3) == 0) {
+                prefetch_l2_bulk(grad + e2, kTkTile * 4);
+                prefetch_l2_bulk(mem + e2, kTkTile * 4);
+            }
+        }
         const int64_t seg = int64_t(w) * ncomp + L.sidx;
         const int32_t k = segs[seg].k;
         if (k == 0) continue;
-        uint32_t lo = 0;
-        int32_t* counter;
-        if (kCompute) {
-            lo = segs[seg].lo;
-            counter = &segs[seg].spill_main;
-        } else {
-            if (segs[seg].spill_main >= k) continue;
-            counter = &segs[seg].spill_redo;
-        }
+        const uint32_t lo = segs[seg].lo, hi = segs[seg].hi;
         const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
         const int cnt = int(min64(kTkTile, L.n - tstart));
         const int64_t ebase = int64_t(w) * N + L.offset + tstart;
@@ -198,21 +254,26 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
         float v[kTkPerThread];
         uint32_t flags = 0;
         if (cnt == kTkTile && (ebase & 3) == 0) {
+            float4 gg[kIters], mm[kIters];
 #pragma unroll
             for (int j = 0; j < kIters; ++j) {
                 const int e = j * (kTkThreads * 4) + tid * 4;
-                float4 x;
-                if (kCompute) {
-                    const float4 gg = ld_stream4(g + e);
-                    const float4 mm = ld_stream4(m + e);
-                    x.x = residual(mm.x, eta, gg.x);
-                    x.y = residual(mm.y, eta, gg.y);
-                    x.z = residual(mm.z, eta, gg.z);
-                    x.w = residual(mm.w, eta, gg.w);
-                    *reinterpret_cast<float4*>(m + e) = x;
-                } else {
-                    x = __ldcg(reinterpret_cast<const float4*>(m + e));
-                }
+                gg[j] = ld_stream4(g + e);
+                mm[j] = ld_stream4(m + e);
+            }
+#pragma unroll
+            for (int j = 0; j < kIters; ++j) {
+                const int e = j * (kTkThreads * 4) + tid * 4;
+                float4 x, o;
+                x.x = residual(mm[j].x, eta, gg[j].x);
+                x.y = residual(mm[j].y, eta, gg[j].y);
+                x.z = residual(mm[j].z, eta, gg[j].z);
+                x.w = residual(mm[j].w, eta, gg[j].w);
+                o.x = abs_key(x.x) > hi ? 0.0f : x.x;
+                o.y = abs_key(x.y) > hi ? 0.0f : x.y;
+                o.z = abs_key(x.z) > hi ? 0.0f : x.z;
+                o.w = abs_key(x.w) > hi ? 0.0f : x.w;
+                *reinterpret_cast<float4*>(m + e) = o;
                 v[4 * j + 0] = x.x;
                 v[4 * j + 1] = x.y;
                 v[4 * j + 2] = x.z;
@@ -229,12 +290,8 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
                     const int e = j * (kTkThreads * 4) + tid * 4 + q;
                     float x = 0.0f;
                     if (e < cnt) {
-                        if (kCompute) {
-                            x = residual(m[e], eta, __ldcs(g + e));
-                            m[e] = x;
-                        } else {
-                            x = __ldcg(m + e);
-                        }
+                        x = residual(m[e], eta, __ldcs(g + e));
+                        m[e] = abs_key(x) > hi ? 0.0f : x;
                         flags |= uint32_t(abs_key(x) >= lo) << (4 * j + q);
                     }
                     v[4 * j + q] = x;
@@ -261,12 +318,14 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
         __syncthreads();
         if (tid == 0) {
             const int tot = s_total;
-            const int base = tot ? atomicAdd(counter, tot) : 0;
+            const int base = tot ? atomicAdd(&segs[seg].spill_main, tot) : 0;
             s_base = base;
             tile_dir[t] = make_int2(base, tot);
         }
         __syncthreads();
-        TkEntry* out = spill + int64_t(w) * comp_N + L.sp_off + s_base;
+        const int64_t sbase = int64_t(w) * comp_N + L.sp_off + s_base;
+        float* ov = spill_v + sbase;
+        int32_t* oi = spill_i + sbase;
 #pragma unroll
         for (int j = 0; j < kIters; ++j) {
             const uint32_t f = (flags >> (4 * j)) & 0xFu;
@@ -274,10 +333,9 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 if (f & (1u << q)) {
-                    TkEntry en;
-                    en.v = v[4 * j + q];
-                    en.i = int32_t(tstart + j * (kTkThreads * 4) + tid * 4 + q);
-                    out[pos++] = en;
+                    ov[pos] = v[4 * j + q];
+                    oi[pos] = int32_t(tstart + j * (kTkThreads * 4) + tid * 4 + q);
+                    ++pos;
                 }
             }
         }
@@ -285,24 +343,40 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
     }
 }
 
-// ---- histogram units ------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) tk_units_kernel(TkSeg* __restrict__ segs, int64_t S,
+// ---- units: fallback decision, tile list of the fallback, histogram units ---------------
+__global__ void __launch_bounds__(1024) tk_units_kernel(const DevLayer* __restrict__ layers,
+                                                        const int32_t* __restrict__ comp,
+                                                        int32_t ncomp, int32_t tiles_pw,
+                                                        TkSeg* __restrict__ segs, int64_t S,
                                                         int32_t* __restrict__ unit_start,
+                                                        int32_t* __restrict__ redo_list,
                                                         int32_t* __restrict__ status) {
     __shared__ int s_warp[33];
-    __shared__ int s_carry;
-    if (threadIdx.x == 0) s_carry = 0;
+    __shared__ int s_carry, s_rcarry;
+    if (threadIdx.x == 0) {
+        s_carry = 0;
+        s_rcarry = 0;
+    }
     __syncthreads();
     for (int64_t b0 = 0; b0 < S; b0 += blockDim.x) {
         const int64_t s = b0 + threadIdx.x;
-        int units = 0;
+        int units = 0, rtiles = 0;
+        int64_t t0 = 0;
         if (s < S) {
             TkSeg& g = segs[s];
+            const DevLayer L = layers[comp[s % ncomp]];
             int32_t cnt = 0;
+            g.redo = 0;
             if (g.k > 0) {
-                const bool redo = g.spill_main < g.k;
-                cnt = redo ? g.spill_redo : g.spill_main;
-                if (redo) set_status(status, GCE_STATUS_FALLBACK);
+                if (g.spill_main < g.k) {
+                    g.redo = 1;
+                    cnt = int32_t(L.n);   // the fallback lists every element
+                    rtiles = L.ntiles;
+                    t0 = int64_t(s / ncomp) * tiles_pw + L.tile0;
+                    set_status(status, GCE_STATUS_FALLBACK);
+                } else {
+                    cnt = g.spill_main;
+                }
                 units = (cnt + kTkHUnit - 1) / kTkHUnit;
             }
             g.count = cnt;
@@ -312,14 +386,76 @@ __global__ void __launch_bounds__(1024) tk_units_kernel(TkSeg* __restrict__ segs
         int tot = 0;
         const int ex = block_exclusive_scan(units, s_warp, &tot);
         if (s < S) unit_start[s] = s_carry + ex;
+        int rtot = 0;
+        const int rex = block_exclusive_scan(rtiles, s_warp, &rtot);
+        for (int i = 0; i < rtiles; ++i) redo_list[1 + s_rcarry + rex + i] = int32_t(t0 + i);
         __syncthreads();
-        if (threadIdx.x == 0) s_carry += tot;
+        if (threadIdx.x == 0) {
+            s_carry += tot;
+            s_rcarry += rtot;
+        }
         __syncthreads();
     }
-    if (threadIdx.x == 0) unit_start[S] = s_carry;
+    if (threadIdx.x == 0) {
+        unit_start[S] = s_carry;
+        redo_list[0] = s_rcarry;
+    }
 }
 
-// ---- radix levels over the candidate lists --------------------------------------------------
+// ---- exact fallback: give v back to memory zeroed above hi, then list every element ------
+__global__ void __launch_bounds__(256) tk_restore_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
+    int32_t ncomp, int64_t N, int64_t comp_N, const TkSeg* __restrict__ segs,
+    const int32_t* __restrict__ redo_list, const int2* __restrict__ tile_dir,
+    const float* __restrict__ spill_v, const int32_t* __restrict__ spill_i,
+    float* __restrict__ mem) {
+    const int32_t n = redo_list[0];
+    for (int32_t u = blockIdx.x; u < n; u += gridDim.x) {
+        const int32_t t = redo_list[1 + u];
+        const int w = t / tiles_pw;
+        const DevLayer L = layers[tile_layer[t % tiles_pw]];
+        const uint32_t hi = segs[int64_t(w) * ncomp + L.sidx].hi;
+        const int2 d = tile_dir[t];
+        const int64_t sb = int64_t(w) * comp_N + L.sp_off + d.x;
+        float* m = mem + int64_t(w) * N + L.offset;
+        for (int j = threadIdx.x; j < d.y; j += blockDim.x) {
+            const float x = spill_v[sb + j];
+            if (abs_key(x) > hi) m[spill_i[sb + j]] = x;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) tk_respill_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
+    int32_t ncomp, int64_t N, int64_t comp_N, TkSeg* __restrict__ segs,
+    const int32_t* __restrict__ redo_list, int2* __restrict__ tile_dir,
+    const float* __restrict__ mem, float* __restrict__ spill_v, int32_t* __restrict__ spill_i) {
+    __shared__ int s_base;
+    const int32_t n = redo_list[0];
+    for (int32_t u = blockIdx.x; u < n; u += gridDim.x) {
+        const int32_t t = redo_list[1 + u];
+        const int w = t / tiles_pw;
+        const int lt = t % tiles_pw;
+        const DevLayer L = layers[tile_layer[lt]];
+        const int64_t seg = int64_t(w) * ncomp + L.sidx;
+        const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
+        const int cnt = int(min64(kTkTile, L.n - tstart));
+        if (threadIdx.x == 0) {
+            s_base = atomicAdd(&segs[seg].spill_redo, cnt);
+            tile_dir[t] = make_int2(s_base, cnt);
+        }
+        __syncthreads();
+        const float* m = mem + int64_t(w) * N + L.offset + tstart;
+        const int64_t sb = int64_t(w) * comp_N + L.sp_off + s_base;
+        for (int e = threadIdx.x; e < cnt; e += blockDim.x) {
+            spill_v[sb + e] = __ldcg(m + e);
+            spill_i[sb + e] = int32_t(tstart + e);
+        }
+        __syncthreads();
+    }
+}
+
+// ---- radix levels over the candidate values --------------------------------------------
 template <int kLevel>
 __global__ void __launch_bounds__(256) tk_hist_kernel(const DevLayer* __restrict__ layers,
                                                       const int32_t* __restrict__ comp,
@@ -327,9 +463,10 @@ __global__ void __launch_bounds__(256) tk_hist_kernel(const DevLayer* __restrict
                                                       TkSeg* __restrict__ segs,
                                                       const int32_t* __restrict__ unit_start,
                                                       int32_t* __restrict__ hists,
-                                                      const TkEntry* __restrict__ spill) {
+                                                      const float* __restrict__ spill_v) {
     constexpr int kNb = kLevel == 3 ? 512 : kTkBins;
     constexpr int kShift = kLevel == 1 ? 20 : (kLevel == 2 ? 9 : 0);
+    constexpr int kPer = 32;  // candidates per thread per load batch
     __shared__ int32_t h[kTkBins];
     __shared__ int s_last;
     const int tid = threadIdx.x;
@@ -346,16 +483,25 @@ __global__ void __launch_bounds__(256) tk_hist_kernel(const DevLayer* __restrict
         const uint32_t prefix = segs[s].prefix;
         const int32_t count = segs[s].count;
         const int64_t j0 = int64_t(u - unit_start[s]) * kTkHUnit;
-        const int64_t j1 = min64(j0 + kTkHUnit, count);
         for (int b = tid; b < kNb; b += blockDim.x) h[b] = 0;
         __syncthreads();
-        const TkEntry* e = spill + int64_t(w) * comp_N + L.sp_off;
-        for (int64_t j = j0 + tid; j < j1; j += blockDim.x) {
-            const uint32_t key = abs_key(e[j].v);
-            bool take = true;
-            if (kLevel == 2) take = (key >> 20) == (prefix >> 20);
-            if (kLevel == 3) take = (key >> 9) == (prefix >> 9);
-            if (take) atomicAdd(&h[(key >> kShift) & (kNb - 1)], 1);
+        const float* e = spill_v + int64_t(w) * comp_N + L.sp_off;
+        for (int64_t jb = j0; jb < min64(j0 + kTkHUnit, count); jb += int64_t(kPer) * 256) {
+            uint32_t key[kPer];
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int64_t j = jb + int64_t(q) * 256 + tid;
+                key[q] = j < count ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
+            }
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                bool take = key[q] != 0xFFFFFFFFu;
+                if (kLevel == 2) take = take && (key[q] >> 20) == (prefix >> 20);
+                if (kLevel == 3) take = take && (key[q] >> 9) == (prefix >> 9);
+                const uint32_t bin = (key[q] >> kShift) & (kNb - 1);
+                if (kLevel == 1) hist_add(h, bin, take);   // few, crowded bins
+                else if (take) atomicAdd(&h[bin], 1);
+            }
         }
         __syncthreads();
         int32_t* gh = tk_hist(hists, S, kLevel, s);
@@ -387,14 +533,15 @@ __global__ void __launch_bounds__(256) tk_hist_kernel(const DevLayer* __restrict
     }
 }
 
-// ---- per-tile counts, prefix over tiles, ordered emit ------------------------------------------
+// ---- per-tile counts, prefix over tiles, ordered emit --------------------------------------
 __global__ void __launch_bounds__(256) tk_count_kernel(const DevLayer* __restrict__ layers,
                                                        const int32_t* __restrict__ tile_layer,
                                                        int32_t tiles_pw, int32_t W, int32_t ncomp,
                                                        int64_t comp_N, const TkSeg* __restrict__ segs,
                                                        const int2* __restrict__ tile_dir,
                                                        int2* __restrict__ tile_cnt,
-                                                       const TkEntry* __restrict__ spill) {
+                                                       const float* __restrict__ spill_v) {
+    constexpr int kBatch = 8;
     const int lane = threadIdx.x & 31;
     const int64_t total = int64_t(tiles_pw) * W;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
@@ -408,11 +555,21 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const DevLayer* __restric
         if (k > 0) {
             const uint32_t T = segs[s].prefix;
             const int2 d = tile_dir[t];
-            const TkEntry* e = spill + int64_t(w) * comp_N + L.sp_off + d.x;
-            for (int j = lane; j < d.y; j += 32) {
-                const uint32_t key = abs_key(e[j].v);
-                gt += key > T;
-                eq += key == T;
+            const float* e = spill_v + int64_t(w) * comp_N + L.sp_off + d.x;
+            for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
+                uint32_t key[kBatch];
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    const int j = j0 + q * 32 + lane;
+                    key[q] = j < d.y ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
+                }
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    if (key[q] != 0xFFFFFFFFu) {
+                        gt += key[q] > T;
+                        eq += key[q] == T;
+                    }
+                }
             }
             gt = warp_sum(gt);
             eq = warp_sum(eq);
@@ -450,8 +607,10 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, int64_t vals_pw,
     const TkSeg* __restrict__ segs, const int2* __restrict__ tile_dir,
-    const int2* __restrict__ tile_cnt, const TkEntry* __restrict__ spill, float* __restrict__ mem,
-    float* __restrict__ vals, int32_t* __restrict__ idx) {
+    const int2* __restrict__ tile_cnt, const float* __restrict__ spill_v,
+    const int32_t* __restrict__ spill_i, float* __restrict__ mem, float* __restrict__ vals,
+    int32_t* __restrict__ idx) {
+    constexpr int kBatch = 4;
     const int lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int64_t total = int64_t(tiles_pw) * W;
@@ -465,36 +624,49 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
         if (k == 0) continue;
         const uint32_t T = segs[s].prefix;
         const int32_t need = segs[s].need;  // keys equal to T that are taken
+        // after the fallback the memory holds v everywhere (nothing was zeroed)
+        const uint32_t hi = segs[s].redo ? 0xFFFFFFFFu : segs[s].hi;
         const int2 d = tile_dir[t];
         const int2 before = tile_cnt[t];    // (key > T, key == T) in earlier tiles
         int sel_before = before.x + min(before.y, need);
         int eq_seen = before.y;
-        const TkEntry* e = spill + int64_t(w) * comp_N + L.sp_off + d.x;
+        const int64_t sb = int64_t(w) * comp_N + L.sp_off + d.x;
         float* vout = vals + int64_t(w) * vals_pw + L.val_off;
         int32_t* iout = idx + int64_t(w) * vals_pw + L.val_off;
         float* m = mem + int64_t(w) * N + L.offset;
-        for (int j0 = 0; j0 < d.y; j0 += 32) {
-            const int j = j0 + lane;
-            TkEntry en{0.0f, 0};
-            uint32_t key = 0;
-            const bool valid = j < d.y;
-            if (valid) {
-                en = e[j];
-                key = abs_key(en.v);
+        for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
+            float ev[kBatch];
+            int32_t ei[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * 32 + lane;
+                ev[q] = 0.0f;
+                ei[q] = -1;
+                if (j < d.y) {
+                    ev[q] = __ldcg(spill_v + sb + j);
+                    ei[q] = __ldcg(spill_i + sb + j);
+                }
             }
-            const bool is_eq = valid && key == T;
-            const unsigned eq_mask = __ballot_sync(kFull, is_eq);
-            const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
-            const bool sel = valid && (key > T || (is_eq && eq_rank < need));
-            const unsigned sel_mask = __ballot_sync(kFull, sel);
-            const int pos = sel_before + __popc(sel_mask & lt_mask);
-            if (sel && pos < k) {
-                vout[pos] = en.v;
-                iout[pos] = en.i;
-                m[en.i] = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const bool valid = ei[q] >= 0;
+                const uint32_t key = abs_key(ev[q]);
+                const bool is_eq = valid && key == T;
+                const unsigned eq_mask = __ballot_sync(kFull, is_eq);
+                const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+                const bool sel = valid && (key > T || (is_eq && eq_rank < need));
+                const unsigned sel_mask = __ballot_sync(kFull, sel);
+                const int pos = sel_before + __popc(sel_mask & lt_mask);
+                if (sel && pos < k) {
+                    vout[pos] = ev[q];
+                    iout[pos] = ei[q];
+                    if (key <= hi) m[ei[q]] = 0.0f;
+                } else if (valid && !sel && key > hi) {
+                    m[ei[q]] = ev[q];  // zeroed in the main pass but not chosen
+                }
+                sel_before += __popc(sel_mask);
+                eq_seen += __popc(eq_mask);
             }
-            sel_before += __popc(sel_mask);
-            eq_seen += __popc(eq_mask);
         }
     }
 }
@@ -541,10 +713,12 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         TkSeg* segs = at<TkSeg>(ws, lay.segs);
         int32_t* hists = at<int32_t>(ws, lay.hists);
         int32_t* unit_start = at<int32_t>(ws, lay.unit_start);
+        int32_t* redo_list = at<int32_t>(ws, lay.redo_list);
         int2* tile_dir = at<int2>(ws, lay.tile_dir);
         int2* tile_cnt = at<int2>(ws, lay.tile_cnt);
-        TkEntry* spill = at<TkEntry>(ws, lay.spill);
-        const int64_t n4 = lay.S * 4 * kTkBins / 4;
+        float* spill_v = at<float>(ws, lay.spill_v);
+        int32_t* spill_i = at<int32_t>(ws, lay.spill_i);
+        const int64_t n4 = lay.S * (kTkSBins + 3 * kTkBins) / 4;
 
         GCE_LAUNCH(tk_setup_kernel, grid_for((n4 + lay.S + 255) / 256, 8), 256, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, k_or_rank, segs, reinterpret_cast<int4*>(hists), n4,
@@ -553,35 +727,35 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
             GCE_LAUNCH(tk_sample_kernel, grid_for(int64_t(t->sunits_pw) * W, 8), 256, 0, st,
                        t->d_layers, t->d_sunit_layer, t->d_sunit_part, t->sunits_pw, W, ncomp,
                        lay.S, t->N, grad, mem, eta, segs, hists, g_bracket_sigma);
-        static int occ_main = occupancy(tk_main_kernel<true>, kTkThreads);
-        static int occ_redo = occupancy(tk_main_kernel<false>, kTkThreads);
-        GCE_LAUNCH(tk_main_kernel<true>, grid_for(lay.TT, occ_main), kTkThreads, 0, st, t->d_layers,
+        static int occ_main = occupancy(tk_main_kernel, kTkThreads);
+        GCE_LAUNCH(tk_main_kernel, grid_for(lay.TT, occ_main), kTkThreads, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->comp_N, grad, mem, eta, segs,
-                   tile_dir, spill);
-        GCE_LAUNCH(tk_main_kernel<false>, grid_for(lay.TT, occ_redo), kTkThreads, 0, st,
-                   t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->comp_N, grad, mem,
-                   eta, segs, tile_dir, spill);
-        GCE_LAUNCH(tk_units_kernel, 1, 1024, 0, st, segs, lay.S, unit_start, status);
+                   tile_dir, spill_v, spill_i);
+        GCE_LAUNCH(tk_units_kernel, 1, 1024, 0, st, t->d_layers, t->d_comp, ncomp, t->tiles_pw,
+                   segs, lay.S, unit_start, redo_list, status);
+        const int rgrid = grid_for(lay.TT, 4);
+        GCE_LAUNCH(tk_restore_kernel, rgrid, 256, 0, st, t->d_layers, t->d_tile_layer,
+                   t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, spill_v,
+                   spill_i, mem);
+        GCE_LAUNCH(tk_respill_kernel, rgrid, 256, 0, st, t->d_layers, t->d_tile_layer,
+                   t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, mem, spill_v,
+                   spill_i);
         const int hgrid = grid_for(lay.TT + lay.S, 8);
         GCE_LAUNCH(tk_hist_kernel<1>, hgrid, 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
-                   t->comp_N, segs, unit_start, hists, spill);
+                   t->comp_N, segs, unit_start, hists, spill_v);
         GCE_LAUNCH(tk_hist_kernel<2>, hgrid, 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
-                   t->comp_N, segs, unit_start, hists, spill);
+                   t->comp_N, segs, unit_start, hists, spill_v);
         GCE_LAUNCH(tk_hist_kernel<3>, hgrid, 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
-                   t->comp_N, segs, unit_start, hists, spill);
+                   t->comp_N, segs, unit_start, hists, spill_v);
         const int wgrid = grid_for((lay.TT + 7) / 8, 8);
         GCE_LAUNCH(tk_count_kernel, wgrid, 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw,
-                   W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill);
+                   W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
         GCE_LAUNCH(tk_scan_kernel, grid_for(lay.S, 2), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
                    lay.S, t->tiles_pw, segs, tile_cnt);
         GCE_LAUNCH(tk_emit_kernel, wgrid, 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw, W,
-                   ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt, spill, mem, vals,
-                   idx);
+                   ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt, spill_v, spill_i,
+                   mem, vals, idx);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, st);
 }
-
-namespace gce {
-double bracket_sigma() { return g_bracket_sigma; }
-}  // namespace gce
