@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
     const int32_t* __restrict__ k_or_rank, const float* __restrict__ vals,
     const int32_t* __restrict__ idx, const float* __restrict__ P, const float* __restrict__ Q,
     const int32_t* __restrict__ bounds, float scale, float* __restrict__ out) {
-    __shared__ float acc[kDcTile];
+    __shared__ __align__(16) float acc[kDcTile];
     __shared__ int32_t s_first[32], s_off[33];
     __shared__ int32_t s_sidx[kDcStage];
     __shared__ float s_sval[kDcStage];
@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
         float* o = out + L.offset + start;
         if (L.kind == GCE_KIND_TOPK || L.kind == GCE_KIND_RANDK) {
             const int32_t k = layer_k(L, k_or_rank, l);
-            for (int i = threadIdx.x; i < cnt; i += blockDim.x) acc[i] = 0.0f;
+            for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
+                reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             // every worker's entry range for this tile at once, then one staged
             // load of all the entries, so the worker-order sums below touch
             // only shared memory
@@ -141,7 +142,16 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
                 }
             }
             __syncthreads();
-            for (int i = threadIdx.x; i < cnt; i += blockDim.x) o[i] = __fmul_rn(acc[i], scale);
+            if (cnt == kDcTile && ((L.offset + start) & 3) == 0) {
+                for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x) {
+                    const float4 a = reinterpret_cast<const float4*>(acc)[i];
+                    reinterpret_cast<float4*>(o)[i] =
+                        make_float4(__fmul_rn(a.x, scale), __fmul_rn(a.y, scale),
+                                    __fmul_rn(a.z, scale), __fmul_rn(a.w, scale));
+                }
+            } else {
+                for (int i = threadIdx.x; i < cnt; i += blockDim.x) o[i] = __fmul_rn(acc[i], scale);
+            }
             __syncthreads();
         } else if (L.kind == GCE_KIND_DENSE) {
             for (int i = threadIdx.x; i < cnt; i += blockDim.x) {

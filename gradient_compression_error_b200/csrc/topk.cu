@@ -192,7 +192,9 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
                 const double margin = sigma * (sqrt(mu) + 1.0);
                 int64_t t_lo = int64_t(ceil(mu + margin));
                 if (t_lo < 1) t_lo = 1;
-                const int64_t t_hi = int64_t(floor(mu - margin));
+                // hi aims at the expected k-th key itself: a miss either way
+                // costs only a few scattered memory writes in the emit
+                const int64_t t_hi = int64_t(floor(mu));
                 uint32_t lo = 0, hi = 0xFFFFFFFFu;
                 if (t_lo <= ns) {
                     const int64_t key = tk_sample_key(h, t_lo, false);
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
     const int2* __restrict__ tile_cnt, const float* __restrict__ spill_v,
     const int32_t* __restrict__ spill_i, float* __restrict__ mem, float* __restrict__ vals,
     int32_t* __restrict__ idx) {
-    constexpr int kBatch = 4;
+    constexpr int kBatch = 8;
     const int lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int64_t total = int64_t(tiles_pw) * W;
