@@ -48,15 +48,32 @@ def workload_spec(name):
         return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk")
     if name == "bert_base_topk1pct_w1":          # one replica: a profiling-sized case
         return dict(layers=wl.bert_base_topk(), W=1, cfg=4, method="topk")
+    if name == "bert_base_randk1pct_w8":
+        return dict(layers=wl.bert_base_topk(kind="randk"), W=8, cfg=4, method="randk")
     if name == "memsgd_vector_2p20":
         return dict(layers=wl.memsgd_vector(), W=1, cfg=1, method="topk")
+    if name == "resnet18_powersgd_r2":
+        return dict(layers=wl.resnet18_powersgd(2), W=1, cfg=2, method="powersgd")
+    if name == "vgg19_accordion_powersgd":       # ranks 4 / 2 chosen by Accordion
+        return dict(layers=wl.vgg19("powersgd", 4), W=1, cfg=3, method="powersgd",
+                    accordion=(4, 2))
+    if name == "vgg19_accordion_topk":           # k 10 % / 1 % chosen by Accordion
+        return dict(layers=wl.vgg19("topk", 100000), W=1, cfg=3, method="topk",
+                    accordion=(100000, 10000))
     if name.startswith("sweep_topk_e"):          # e.g. sweep_topk_e28_ppm10000
         e, ppm = name[len("sweep_topk_e"):].split("_ppm")
         return dict(layers=wl.sweep(int(e), "topk", int(ppm)), W=1, cfg=5, method="topk")
     if name.startswith("sweep_randk_e"):
         e, ppm = name[len("sweep_randk_e"):].split("_ppm")
         return dict(layers=wl.sweep(int(e), "randk", int(ppm)), W=1, cfg=5, method="randk")
+    if name.startswith("sweep_powersgd_e"):      # e.g. sweep_powersgd_e28_r2
+        e, r = name[len("sweep_powersgd_e"):].split("_r")
+        return dict(layers=wl.sweep(int(e), "powersgd", rank=int(r)), W=1, cfg=5,
+                    method="powersgd")
     raise SystemExit("unknown workload %s" % name)
+
+
+MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel"}
 
 
 def measured_hbm_gbs():
@@ -157,12 +174,22 @@ def cpu_oracle_sample(spec, units, steps_seed):
         w, l = u
         lay = layers[l]
         gg, mm = data[u]
-        if spec["method"] == "topk":
+        out = np.zeros(gg.size, np.float32)
+        if lay["kind"] == "dense":
+            pay, m_new = oracle.dense_unit(gg, mm, wl.ETA)
+            oracle.accum_dense(out, pay)
+        elif spec["method"] == "powersgd":
+            rows, cols = lay["rows"], lay["cols"]
+            Q = oracle.powersgd_init_q(cols, lay["cap"], 1, w, l)
+            P, Qn, m_new, _ = oracle.powersgd_unit(gg.reshape(rows, cols), mm.reshape(rows, cols),
+                                                   Q, lay["cap"], wl.ETA, want_mhat=False)
+            oracle.accum_lowrank(out, P, Qn, lay["cap"])
+        elif spec["method"] == "topk":
             vals, idx, m_new = oracle.ef_topk_unit(gg, mm, lay["cap"], wl.ETA)
+            oracle.accum_sparse(out, vals, idx)
         else:
             vals, idx, m_new = oracle.ef_randk_unit(gg, mm, lay["cap"], wl.ETA, 5, w, l, 0)
-        out = np.zeros(gg.size, np.float32)
-        oracle.accum_sparse(out, vals, idx)
+            oracle.accum_sparse(out, vals, idx)
         return gg.size
 
     t0 = time.perf_counter()
@@ -252,14 +279,35 @@ def main():
     ws = table.workspace(W, spec["method"])
     ws_dc = table.workspace(W, "decompress")
     out = torch.zeros(N, dtype=torch.float32, device=dev)
-    encode = gce.ef_topk_step if spec["method"] == "topk" else None
+    method = spec["method"]
+    P = Q = None
+    if method == "powersgd":
+        P = torch.zeros((W, max(4, table.P_per_worker)), dtype=torch.float32, device=dev)
+        Q = torch.zeros((W, max(4, table.Q_per_worker)), dtype=torch.float32, device=dev)
+        gce.powersgd_init_q(table, W, 1, Q)
+    kr = None
+    if "accordion" in spec:   # Accordion picks each layer's k or rank every step
+        L = len(layers)
+        prev = torch.empty(L, dtype=torch.float64, device=dev)
+        level = torch.empty(L, dtype=torch.int32, device=dev)
+        cur = torch.zeros(L, dtype=torch.float64, device=dev)
+        kr = torch.zeros(L, dtype=torch.int32, device=dev)
+        ws_ac = table.workspace(1, "accordion")
+        gce.accordion_init(table, prev, level)
+        lvl_low, lvl_high = spec["accordion"]
 
     def step(s, grad):
-        if spec["method"] == "topk":
-            gce.ef_topk_step(table, W, grad, mem, wl.ETA, None, vals, idx, ws)
+        if kr is not None:
+            gce.accordion_select(table, grad[0], s, 10, 0.5, lvl_low, lvl_high, prev, level, cur,
+                                 kr, ws_ac)
+        if method == "topk":
+            gce.ef_topk_step(table, W, grad, mem, wl.ETA, kr, vals, idx, ws)
+        elif method == "randk":
+            gce.ef_randk_step(table, W, grad, mem, wl.ETA, kr, 5, s, vals, idx, ws)
         else:
-            gce.ef_randk_step(table, W, grad, mem, wl.ETA, None, 5, s, vals, idx, ws)
-        gce.decompress_accumulate(table, W, vals, idx, None, None, None, 1.0, out, ws_dc)
+            gce.powersgd_step(table, W, grad, mem, wl.ETA, kr, P, Q, vals, None, ws)
+        gce.decompress_accumulate(table, W, vals, idx if method != "powersgd" else None, kr, P, Q,
+                                  1.0, out, ws_dc)
 
     def barrier():
         if world > 1:
@@ -302,8 +350,8 @@ def main():
     value = world * elems_per_step * args.steps / (t_ms / 1e3)
     ms_step = t_ms / args.steps
 
-    main_ms, main_n = prof.get(MAIN_KERNEL if spec["method"] == "topk" else "rk_emit_kernel",
-                               (0.0, 0))
+    main_kernel = MAIN_KERNELS[method]
+    main_ms, main_n = prof.get(main_kernel, (0.0, 0))
     peak, peak_kind = measured_hbm_gbs()
     bytes_per_launch = 12.0 * W * (N - sum(l["rows"] * l["cols"] for l in layers
                                           if l["kind"] == "dense"))
@@ -311,12 +359,16 @@ def main():
     traffic = ncu_traffic_per_launch() if args.workload == DEFAULT_WORKLOAD else None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": (achieved / peak) if achieved else None, "traffic": traffic,
-                "kernel": MAIN_KERNEL if spec["method"] == "topk" else "rk_emit_kernel",
+                "kernel": main_kernel,
                 "peak_source": peak_kind,
                 "algorithmic_bytes_per_launch": bytes_per_launch,
                 "avg_launch_ms": main_ms / main_n if main_n else None}
-    # whole-step algorithmic traffic: W(12N + 8K) encode + 16 W K + 4N decode
-    step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total + 4.0 * N
+    # whole-step algorithmic traffic: sparse W(12N + 8K) encode + 16 W K + 4N
+    # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
+    if method == "powersgd":
+        step_bytes = W * 12.0 * N + 4.0 * N
+    else:
+        step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total + 4.0 * N
     step_gbs = step_bytes / (ms_step / 1e3) / 1e9
 
     # end to end through the public API with host buffers

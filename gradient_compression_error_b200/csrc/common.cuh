@@ -55,6 +55,9 @@ struct gce_table {
     int32_t dc_tiles = 0;                  // decode tiles over all layers
     int32_t dc_slots = 0;                  // tile-bound slots per worker (tiles + L)
     int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
+    int32_t dc_sp_n = 0, dc_ot_n = 0;      // decode tiles of sparse / other layers
+    int32_t* d_dc_sp_tiles = nullptr;      // their decode tile ids
+    int32_t* d_dc_ot_tiles = nullptr;
     int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker
     int32_t* d_bunit_layer = nullptr;
     int32_t* d_bunit_chunk = nullptr;

@@ -72,16 +72,18 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
 
 __global__ void __launch_bounds__(256) dc_accum_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
-    int32_t dc_tiles, int32_t W, int64_t vals_pw, int64_t P_pw, int64_t Q_pw, int32_t dc_slots,
-    const int32_t* __restrict__ k_or_rank, const float* __restrict__ vals,
-    const int32_t* __restrict__ idx, const float* __restrict__ P, const float* __restrict__ Q,
-    const int32_t* __restrict__ bounds, float scale, float* __restrict__ out) {
+    const int32_t* __restrict__ tile_list, int32_t dc_tiles, int32_t W, int64_t vals_pw,
+    int64_t P_pw, int64_t Q_pw, int32_t dc_slots, const int32_t* __restrict__ k_or_rank,
+    const float* __restrict__ vals, const int32_t* __restrict__ idx, const float* __restrict__ P,
+    const float* __restrict__ Q, const int32_t* __restrict__ bounds, float scale,
+    float* __restrict__ out) {
     __shared__ __align__(16) float acc[kDcTile];
     __shared__ int32_t s_first[32], s_off[33];
     __shared__ int32_t s_sidx[kDcStage];
     __shared__ float s_sval[kDcStage];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int32_t t = blockIdx.x; t < dc_tiles; t += gridDim.x) {
+    for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
+        const int32_t t = tile_list ? tile_list[u] : u;
         const int32_t l = dc_tile_layer[t];
         const DevLayer L = layers[l];
         const int32_t tt = t - L.dc_tile0;
@@ -183,6 +185,24 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
     }
 }
 
+// bounds pass plus the decode kernels for every kind the table holds
+static int launch_decode(const gce_table* t, int32_t W, const float* vals, const int32_t* idx,
+                         const int32_t* k_or_rank, const float* P, const float* Q, float scale,
+                         float* out, int32_t* bounds, cudaStream_t st) {
+    const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
+    const int sms = sm_count();
+    if (sparse && t->bunits_pw > 0) {
+        const int64_t units = int64_t(t->bunits_pw) * W;
+        GCE_LAUNCH(dc_bounds_kernel, int(min64(units, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
+                   t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
+                   k_or_rank, idx, bounds);
+    }
+    GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st,
+               t->d_layers, t->d_dc_tile_layer, nullptr, t->dc_tiles, W, t->vals_pw, t->P_pw,
+               t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q, bounds, scale, out);
+    return check_launch();
+}
+
 }  // namespace gce
 
 using namespace gce;
@@ -196,19 +216,8 @@ extern "C" int decompress_accumulate(const gce_table* t, int32_t W, const float*
     if ((t->vals_pw > 0 && !vals) || (sparse && !idx)) return GCE_ERR_ARG;
     if (t->ckind == GCE_KIND_POWERSGD && (!P || !Q)) return GCE_ERR_ARG;
     if (ws_bytes < decompress_ws_bytes(t, W)) return GCE_ERR_WORKSPACE;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    int32_t* bounds = at<int32_t>(ws, GCE_WS_HEADER_BYTES);
-    const int sms = sm_count();
-    if (sparse && t->bunits_pw > 0) {
-        const int64_t units = int64_t(t->bunits_pw) * W;
-        GCE_LAUNCH(dc_bounds_kernel, int(min64(units, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
-                   t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
-                   k_or_rank, idx, bounds);
-    }
-    GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
-               t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots,
-               k_or_rank, vals, idx, P, Q, bounds, scale, out);
-    return check_launch();
+    return launch_decode(t, W, vals, idx, k_or_rank, P, Q, scale, out,
+                         at<int32_t>(ws, GCE_WS_HEADER_BYTES), static_cast<cudaStream_t>(stream));
 }
 
 // ---- decode without a caller workspace -------------------------------------------------
@@ -253,16 +262,6 @@ extern "C" int decompress_accumulate_noalloc(const gce_table* t, int32_t W, cons
     if (!bounds) return GCE_ERR_CUDA;
     // every bound slot a sparse layer uses is rewritten by the bounds pass, so
     // nothing left from an earlier call needs clearing
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int sms = sm_count();
-    if (sparse && t->bunits_pw > 0) {
-        const int64_t units = int64_t(t->bunits_pw) * W;
-        GCE_LAUNCH(dc_bounds_kernel, int(min64(units, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
-                   t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
-                   k_or_rank, idx, bounds);
-    }
-    GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
-               t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots,
-               k_or_rank, vals, idx, P, Q, bounds, scale, out);
-    return check_launch();
+    return launch_decode(t, W, vals, idx, k_or_rank, P, Q, scale, out, bounds,
+                         static_cast<cudaStream_t>(stream));
 }
