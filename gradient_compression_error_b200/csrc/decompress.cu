@@ -165,21 +165,31 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
         } else {  // POWERSGD: P Q^T over the first r columns
             const int32_t r = layer_k(L, k_or_rank, l);
             const int cap = L.cap;
+            // neighbouring threads take neighbouring columns (coalesced Q
+            // reads and output writes); one 32-bit division per thread finds
+            // its first (row, col), then the column advances by the block size
+            const uint32_t cols = uint32_t(L.cols);
+            const uint32_t c0 = uint32_t((start + threadIdx.x) % int64_t(cols));
+            int64_t row = (start + threadIdx.x) / int64_t(cols);
+            uint32_t col = c0;
             for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
-                const int64_t e = start + i;
-                const int64_t row = e / L.cols, col = e - row * L.cols;
                 float s = 0.0f;
                 for (int w = 0; w < W; ++w) {
                     const float* p = P + int64_t(w) * P_pw + L.p_off + row * cap;
-                    const float* q = Q + int64_t(w) * Q_pw + L.q_off + col * cap;
+                    const float* qq = Q + int64_t(w) * Q_pw + L.q_off + int64_t(col) * cap;
                     float m = 0.0f;
                     if (r > 0) {
-                        m = __fmul_rn(p[0], q[0]);
-                        for (int j = 1; j < r; ++j) m = __fmaf_rn(p[j], q[j], m);
+                        m = __fmul_rn(p[0], qq[0]);
+                        for (int j = 1; j < r; ++j) m = __fmaf_rn(p[j], qq[j], m);
                     }
                     s = __fadd_rn(s, m);
                 }
                 o[i] = __fmul_rn(s, scale);
+                col += blockDim.x;
+                if (col >= cols) {
+                    row += col / cols;
+                    col %= cols;
+                }
             }
         }
     }

@@ -129,14 +129,12 @@ __global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict
         const uint64_t base = g.base;
         const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
         const int64_t e0 = tstart + int64_t(tid) * 32;
-        uint32_t keys[32];
+        const uint64_t x0 = base + uint64_t(e0 + 1) * kGamma;  // generator state of element e0
         uint32_t below = 0, inband = 0;
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-            const int64_t i = e0 + q;
-            const uint32_t key = uint32_t(mix64(base + uint64_t(i + 1) * kGamma) >> 32);
-            keys[q] = key;
-            if (i < L.n) {
+            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+            if (e0 + q < L.n) {
                 below |= uint32_t(key < lo) << q;
                 inband |= uint32_t(key >= lo && key <= hi) << q;
             }
@@ -161,9 +159,12 @@ __global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict
         wbase = __shfl_sync(kFull, wbase, 31);
         RkEntry* out = cand + int64_t(w) * comp_N + L.sp_off + wbase + (incl - nb);
         int pos = 0;
-#pragma unroll
-        for (int q = 0; q < 32; ++q)
-            if (inband & (1u << q)) out[pos++] = RkEntry{keys[q], int32_t(e0 + q)};
+        while (inband) {  // few band entries: their keys are recomputed
+            const int q = __ffs(inband) - 1;
+            inband &= inband - 1;
+            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+            out[pos++] = RkEntry{key, int32_t(e0 + q)};
+        }
     }
 }
 
@@ -334,6 +335,18 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
         const DevLayer L = layers[tile_layer[lt]];
+        // the bulk-copy engine pulls this block's next tile into L2 meanwhile
+        if (tid == 0 && t + gridDim.x < total) {
+            const int64_t t2 = t + gridDim.x;
+            const int lt2 = int(t2 % tiles_pw);
+            const DevLayer L2 = layers[tile_layer[lt2]];
+            const int64_t s2 = int64_t(lt2 - L2.tile0) * kTkTile;
+            const int64_t e2 = int64_t(t2 / tiles_pw) * N + L2.offset + s2;
+            if (s2 + kTkTile <= L2.n && (e2 & 3) == 0) {
+                prefetch_l2_bulk(grad + e2, kTkTile * 4);
+                prefetch_l2_bulk(mem + e2, kTkTile * 4);
+            }
+        }
         const int64_t s = int64_t(w) * ncomp + L.sidx;
         const int32_t k = segs[s].k;
         if (k == 0) continue;
