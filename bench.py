@@ -76,6 +76,23 @@ def workload_spec(name):
 MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel"}
 
 
+def max_over_ranks_of(x, world, device):
+    """The largest of the ranks' values (each rank times its own device)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, elems_per_step, steps, t_ms_max):
+    """Whole-job elements per second: every rank's elements over the slowest
+    rank's time (each rank runs its own replica of the workload)."""
+    return world * elems_per_step * steps / (t_ms_max / 1e3)
+
+
 def measured_hbm_gbs():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -314,11 +331,7 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks_of(x, world, dev)
 
     for s in range(args.warmup):
         step(s, grads[s % 2])
@@ -347,7 +360,7 @@ def main():
     fallback_seen = bool(gce.status(ws) & gce.STATUS_FALLBACK)
 
     elems_per_step = W * N
-    value = world * elems_per_step * args.steps / (t_ms / 1e3)
+    value = job_throughput(world, elems_per_step, args.steps, t_ms)
     ms_step = t_ms / args.steps
 
     main_kernel = MAIN_KERNELS[method]

@@ -55,9 +55,8 @@ struct gce_table {
     int32_t dc_tiles = 0;                  // decode tiles over all layers
     int32_t dc_slots = 0;                  // tile-bound slots per worker (tiles + L)
     int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
-    int32_t dc_sp_n = 0, dc_ot_n = 0;      // decode tiles of sparse / other layers
-    int32_t* d_dc_sp_tiles = nullptr;      // their decode tile ids
-    int32_t* d_dc_ot_tiles = nullptr;
+    int32_t dc_nl_n = 0;                   // decode tiles of sparse and DENSE layers
+    int32_t* d_dc_nl_tiles = nullptr;      // their decode tile ids
     int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker
     int32_t* d_bunit_layer = nullptr;
     int32_t* d_bunit_chunk = nullptr;
@@ -72,6 +71,8 @@ struct gce_table {
     int32_t* d_ps_layers = nullptr;        // POWERSGD layer ids
     int32_t nps = 0;
     int64_t ppart_pw = 0, pd_pw = 0, qpart_pw = 0;  // workspace floats / doubles per worker
+    int32_t ps_ntall = 0, ps_tall_parts = 0, ps_tall_cap = 0, ps_tall_nunits = 0;
+    int2* d_ps_tall_units = nullptr;       // (layer, row chunk) of tall P matrices
     // Accordion plan (built by gce::accordion_plan)
     int2* d_ac_tiles = nullptr;            // (layer, chunk) of the norm reduction
     int32_t ac_ntiles = 0;
@@ -160,6 +161,9 @@ constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
 
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
                         float eta, float* vals, cudaStream_t st);
+bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_rank,
+                           const float* P, const float* Q, float scale, float* out,
+                           cudaStream_t st);
 int powersgd_plan(gce_table* t);   // called once by gce_table_create
 void powersgd_plan_free(gce_table* t);
 int accordion_plan(gce_table* t);  // called once by gce_table_create

@@ -207,6 +207,15 @@ static int launch_decode(const gce_table* t, int32_t W, const float* vals, const
                    t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
                    k_or_rank, idx, bounds);
     }
+    if (t->nps > 0 && launch_lowrank_decode(t, W, k_or_rank, P, Q, scale, out, st)) {
+        // PowerSGD layers done by their own tiled kernel; the rest here
+        if (t->dc_nl_n > 0)
+            GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_nl_n, int64_t(sms) * 8)), 256, 0, st,
+                       t->d_layers, t->d_dc_tile_layer, t->d_dc_nl_tiles, t->dc_nl_n, W,
+                       t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q,
+                       bounds, scale, out);
+        return check_launch();
+    }
     GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st,
                t->d_layers, t->d_dc_tile_layer, nullptr, t->dc_tiles, W, t->vals_pw, t->P_pw,
                t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q, bounds, scale, out);

@@ -38,21 +38,39 @@ constexpr int kPsCB = 1024;   // columns per chunk (256 threads x 4)
 constexpr int kPsRB3 = 64;    // rows per M^T P tile
 constexpr int kPsQB = 256;    // columns per Q-reduction tile
 
+constexpr int64_t kPsTallRows = 8192;  // taller P: Gram-Schmidt spread over many blocks
+constexpr int kPsOrthChunk = 1024;     // rows per block in that case
+
 struct PsLayer {
     int64_t ppart_off;  // floats: nch1 x rows x cap partial P
     int64_t pd_off;     // doubles: rows x cap
     int64_t qpart_off;  // floats: nrb3 x cols x cap partial Q
     int32_t nch1, nrb3;
+    int32_t tall;       // index among the tall layers, -1 otherwise
+    int32_t part_off;   // first partial-sum slot of a tall layer
+    int32_t nchunk;     // row chunks of a tall layer
+    int32_t pad;
 };
 
 int powersgd_plan(gce_table* t) {
     std::vector<PsLayer> ps(t->L);
     std::vector<int4> t1, t3, tq;
+    std::vector<int2> tall_units;
     std::vector<int32_t> ids;
     int64_t pp = 0, pd = 0, qp = 0;
+    int32_t ntall = 0, nparts = 0, tall_cap = 0;
     for (int32_t l = 0; l < t->L; ++l) {
         const DevLayer& L = t->layers[l];
         PsLayer x{};
+        x.tall = -1;
+        if (L.kind == GCE_KIND_POWERSGD && L.rows > kPsTallRows) {
+            x.tall = ntall++;
+            x.nchunk = int32_t((L.rows + kPsOrthChunk - 1) / kPsOrthChunk);
+            x.part_off = nparts;
+            nparts += x.nchunk;
+            tall_cap = std::max(tall_cap, L.cap);
+            for (int32_t c = 0; c < x.nchunk; ++c) tall_units.push_back(make_int2(l, c));
+        }
         if (L.kind == GCE_KIND_POWERSGD) {
             x.nch1 = int32_t((L.cols + kPsCB - 1) / kPsCB);
             x.nrb3 = int32_t((L.rows + kPsRB3 - 1) / kPsRB3);
@@ -79,6 +97,10 @@ int powersgd_plan(gce_table* t) {
     t->ps3_ntiles = int32_t(t3.size());
     t->psq_ntiles = int32_t(tq.size());
     t->nps = int32_t(ids.size());
+    t->ps_ntall = ntall;
+    t->ps_tall_parts = nparts;
+    t->ps_tall_cap = tall_cap;
+    t->ps_tall_nunits = int32_t(tall_units.size());
     auto up = [](void** dst, const void* src, size_t bytes) -> int {
         *dst = nullptr;
         if (bytes == 0) return GCE_OK;
@@ -91,10 +113,14 @@ int powersgd_plan(gce_table* t) {
     if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_ps3_tiles), t3.data(), t3.size() * sizeof(int4));
     if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_psq_tiles), tq.data(), tq.size() * sizeof(int4));
     if (rc == GCE_OK) rc = up(reinterpret_cast<void**>(&t->d_ps_layers), ids.data(), ids.size() * sizeof(int32_t));
+    if (rc == GCE_OK)
+        rc = up(reinterpret_cast<void**>(&t->d_ps_tall_units), tall_units.data(),
+                tall_units.size() * sizeof(int2));
     return rc;
 }
 
 void powersgd_plan_free(gce_table* t) {
+    cudaFree(t->d_ps_tall_units);
     cudaFree(t->d_ps);
     cudaFree(t->d_ps1_tiles);
     cudaFree(t->d_ps3_tiles);
@@ -103,7 +129,7 @@ void powersgd_plan_free(gce_table* t) {
 }
 
 struct PsWs {
-    size_t ppart = 0, pd = 0, qpart = 0, total = 0;
+    size_t ppart = 0, pd = 0, qpart = 0, tparts = 0, tscal = 0, tdone = 0, total = 0;
 };
 
 static PsWs ps_layout(const gce_table* t, int32_t W) {
@@ -112,6 +138,9 @@ static PsWs ps_layout(const gce_table* t, int32_t W) {
     o.ppart = c.take<float>(int64_t(W) * t->ppart_pw);
     o.pd = c.take<double>(int64_t(W) * t->pd_pw);
     o.qpart = c.take<float>(int64_t(W) * t->qpart_pw);
+    o.tparts = c.take<double>(int64_t(W) * t->ps_tall_parts);
+    o.tscal = c.take<double>(int64_t(W) * t->ps_ntall);
+    o.tdone = c.take<int32_t>(int64_t(W) * t->ps_ntall);
     o.total = c.off;
     return o;
 }
@@ -232,7 +261,8 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W, int64_t P_pw, int64_t ppart_pw,
     int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ ppart,
-    double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status) {
+    double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status,
+    int32_t ntall, int32_t* __restrict__ tdone) {
     __shared__ double s_red[32];
     for (int64_t u = blockIdx.x; u < int64_t(nps) * W; u += gridDim.x) {
         const int w = int(u / nps);
@@ -242,6 +272,10 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         const int r = ps_rank(L, k_or_rank, l);
         if (r == 0) {
             if (threadIdx.x == 0) set_status(status, GCE_STATUS_K_RANGE);
+            continue;
+        }
+        if (X.tall >= 0) {  // orthonormalised by the multi-block kernel below
+            if (threadIdx.x == 0) tdone[int64_t(w) * ntall + X.tall] = 0;
             continue;
         }
         const int cap = L.cap;
@@ -282,6 +316,123 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         }
         __syncthreads();
     }
+}
+
+// ---- orthonormalise tall P over many blocks ---------------------------------------------
+// The same modified Gram-Schmidt, one launch per step: a launch first applies
+// the previous step's update to its 1024-row chunk (p_j -= d p_i, or
+// p_j /= ||p_j||), then forms its chunk's part of the next dot product; the
+// last block to finish adds the parts in chunk order (fixed, so the result is
+// deterministic) and leaves the scalar for the next launch.
+struct PsOrthOp {
+    int8_t init;        // first launch: sum the partial P into fp64
+    int8_t apply;       // 0 none, 1 subtract, 2 scale
+    int8_t ai, aj;      // apply: p_aj -= d * p_ai, or p_aj /= sqrt(nn)
+    int8_t reduce;      // 1: form p_ri . p_rj
+    int8_t ri, rj;
+    int8_t final_;      // last launch: write P in fp32
+};
+
+__global__ void __launch_bounds__(256) ps_orth_tall_kernel(
+    PsOrthOp op, const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
+    const int2* __restrict__ units, int32_t nunits, int32_t W, int64_t P_pw, int64_t ppart_pw,
+    int64_t pd_pw, int32_t ntall, int32_t nparts, const int32_t* __restrict__ k_or_rank,
+    const float* __restrict__ ppart, double* __restrict__ pdw, double* __restrict__ tparts,
+    double* __restrict__ tscal, int32_t* __restrict__ tdone, float* __restrict__ P) {
+    __shared__ double s_red[8];
+    __shared__ int s_last;
+    for (int64_t u = blockIdx.x; u < int64_t(nunits) * W; u += gridDim.x) {
+        const int w = int(u / nunits);
+        const int2 d = units[u % nunits];
+        const DevLayer L = layers[d.x];
+        const PsLayer X = ps[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        if (r == 0) continue;
+        const int cap = L.cap;
+        const int64_t R = L.rows;
+        const int64_t r0 = int64_t(d.y) * kPsOrthChunk;
+        const int64_t r1 = min64(r0 + kPsOrthChunk, R);
+        double* pd = pdw + int64_t(w) * pd_pw + X.pd_off;
+        double* scal = tscal + int64_t(w) * ntall + X.tall;
+        if (op.init) {
+            const float* pp = ppart + int64_t(w) * ppart_pw + X.ppart_off;
+            for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
+                for (int j = 0; j < r; ++j) {
+                    double s = 0.0;
+                    for (int ch = 0; ch < X.nch1; ++ch) s += double(pp[(int64_t(ch) * R + row) * cap + j]);
+                    pd[row * cap + j] = s;
+                }
+        }
+        if (op.apply && op.aj < r) {
+            const double sv = *scal;
+            if (op.apply == 1) {
+                for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
+                    pd[row * cap + op.aj] -= sv * pd[row * cap + op.ai];
+            } else {
+                const double nu = sqrt(sv);
+                for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
+                    pd[row * cap + op.aj] = nu > 0.0 ? pd[row * cap + op.aj] / nu : 0.0;
+            }
+        }
+        if (op.reduce && op.rj < r) {
+            double part = 0.0;
+            for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
+                part += pd[row * cap + op.ri] * pd[row * cap + op.rj];
+            part = warp_sum(part);
+            if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = part;
+            __syncthreads();
+            double* parts = tparts + int64_t(w) * nparts + X.part_off;
+            if (threadIdx.x == 0) {
+                double tsum = 0.0;
+                for (int i = 0; i < int(blockDim.x >> 5); ++i) tsum += s_red[i];
+                parts[d.y] = tsum;
+                __threadfence();
+                s_last = atomicAdd(&tdone[int64_t(w) * ntall + X.tall], 1) == X.nchunk - 1;
+            }
+            __syncthreads();
+            if (s_last && threadIdx.x == 0) {
+                __threadfence();
+                double s = 0.0;
+                for (int c = 0; c < X.nchunk; ++c) s += __ldcg(parts + c);
+                *scal = s;
+                tdone[int64_t(w) * ntall + X.tall] = 0;  // ready for the next launch
+            }
+        }
+        if (op.final_) {
+            float* p = P + int64_t(w) * P_pw + L.p_off;
+            for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
+                for (int j = 0; j < r; ++j) p[row * cap + j] = float(pd[row * cap + j]);
+        }
+        __syncthreads();
+    }
+}
+
+// the launch sequence for P with up to `cap` columns
+static std::vector<PsOrthOp> ps_orth_ops(int cap) {
+    std::vector<PsOrthOp> ops;
+    PsOrthOp cur{};
+    cur.init = 1;
+    auto push_reduce = [&](int i, int j) {
+        cur.reduce = 1;
+        cur.ri = int8_t(i);
+        cur.rj = int8_t(j);
+        ops.push_back(cur);
+        cur = PsOrthOp{};
+    };
+    for (int j = 0; j < cap; ++j) {
+        for (int i = 0; i < j; ++i) {
+            push_reduce(i, j);
+            cur.apply = 1;
+            cur.ai = int8_t(i);
+            cur.aj = int8_t(j);
+        }
+        push_reduce(j, j);
+        cur.apply = 2;
+        cur.ai = cur.aj = int8_t(j);
+    }
+    cur.final_ = 1;
+    ops.push_back(cur);
+    return ops;
 }
 
 // ---- phase 3: partial Q = M^T P over 64-row blocks ---------------------------------------
@@ -431,6 +582,79 @@ static int grid_of(int64_t work, int per_sm) {
     return int(max64(1, min64(work, int64_t(sm_count()) * per_sm)));
 }
 
+// ---- decode of PowerSGD payloads: out = scale * sum_w P_w Q_w^T ---------------------------
+// Per (16-row, 1024-column) tile, in 256-column quarters: the quarter's Q
+// columns and the tile's P rows of every worker sit in shared memory, each
+// thread owns one column and walks the 16 rows, so the output is written in
+// full 128-byte lines.  Each entry is formed exactly as the element-wise
+// decoder forms it (product, then fused multiply-adds in column order, then
+// the workers summed in order from +0), so both give the same bits.
+constexpr int kDcLrMaxW = 8;
+
+__global__ void __launch_bounds__(256) ps_decode_kernel(
+    const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles,
+    int32_t W, int64_t P_pw, int64_t Q_pw, const int32_t* __restrict__ k_or_rank,
+    const float* __restrict__ P, const float* __restrict__ Q, float scale,
+    float* __restrict__ out) {
+    __shared__ float qs[kDcLrMaxW][kMaxRank][256];
+    __shared__ float prow[kDcLrMaxW][kPsRB][kMaxRank];
+    const int tid = threadIdx.x;
+    for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
+        const int4 d = tiles[u];
+        const DevLayer L = layers[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        const int cap = L.cap;
+        const int64_t C = L.cols;
+        const int64_t r0 = int64_t(d.y) * kPsRB;
+        const int rh = int(min64(kPsRB, L.rows - r0));
+        const int64_t c0 = int64_t(d.z) * kPsCB;
+        const int cw = int(min64(kPsCB, C - c0));
+        for (int i = tid; i < W * kPsRB * kMaxRank; i += blockDim.x) {
+            const int w = i / (kPsRB * kMaxRank), rr = (i / kMaxRank) % kPsRB, j = i % kMaxRank;
+            prow[w][rr][j] = (rr < rh && j < r) ? P[int64_t(w) * P_pw + L.p_off + (r0 + rr) * cap + j]
+                                                : 0.0f;
+        }
+        for (int qb = 0; qb < cw; qb += 256) {
+            __syncthreads();
+            for (int i = tid; i < W * kMaxRank * 256; i += blockDim.x) {
+                const int w = i / (kMaxRank * 256), j = (i / 256) % kMaxRank, c = i % 256;
+                qs[w][j][c] = (j < r && qb + c < cw)
+                                  ? Q[int64_t(w) * Q_pw + L.q_off + (c0 + qb + c) * cap + j]
+                                  : 0.0f;
+            }
+            __syncthreads();
+            const int c = qb + tid;
+            if (c < cw) {
+                float* o = out + L.offset + r0 * C + c0 + c;
+                for (int rr = 0; rr < rh; ++rr) {
+                    float s = 0.0f;
+                    for (int w = 0; w < W; ++w) {
+                        float m = 0.0f;
+                        if (r > 0) {
+                            m = __fmul_rn(prow[w][rr][0], qs[w][0][tid]);
+                            for (int j = 1; j < r; ++j) m = __fmaf_rn(prow[w][rr][j], qs[w][j][tid], m);
+                        }
+                        s = __fadd_rn(s, m);
+                    }
+                    o[int64_t(rr) * C] = __fmul_rn(s, scale);
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// PowerSGD layers of the decode; false: W too large, use the element-wise path
+bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_rank, const float* P,
+                           const float* Q, float scale, float* out, cudaStream_t st) {
+    if (W > kDcLrMaxW) return false;
+    if (t->ps1_ntiles > 0)
+        GCE_LAUNCH(ps_decode_kernel, grid_of(t->ps1_ntiles, 4), 256, 0, st, t->d_layers,
+                   t->d_ps1_tiles, t->ps1_ntiles, W, t->P_pw, t->Q_pw, k_or_rank, P, Q, scale,
+                   out);
+    return true;
+}
+
 }  // namespace gce
 
 using namespace gce;
@@ -467,9 +691,18 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         GCE_LAUNCH(ps_mq_kernel, grid_of(int64_t(t->ps1_ntiles) * W, 8), 256, 0, st, t->d_layers,
                    ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw, t->ppart_pw, grad, mem,
                    eta, k_or_rank, Q, ppart);
+        int32_t* tdone = at<int32_t>(ws, lay.tdone);
         GCE_LAUNCH(ps_orth_kernel, grid_of(int64_t(t->nps) * W, 8), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
-                   pd, P, status);
+                   pd, P, status, t->ps_ntall, tdone);
+        if (t->ps_ntall > 0) {
+            for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
+                GCE_LAUNCH(ps_orth_tall_kernel, grid_of(int64_t(t->ps_tall_nunits) * W, 8), 256, 0,
+                           st, op, t->d_layers, ps, t->d_ps_tall_units, t->ps_tall_nunits, W,
+                           t->P_pw, t->ppart_pw, t->pd_pw, t->ps_ntall, t->ps_tall_parts,
+                           k_or_rank, ppart, pd, at<double>(ws, lay.tparts),
+                           at<double>(ws, lay.tscal), tdone, P);
+        }
         GCE_LAUNCH(ps_mtp_kernel, grid_of(int64_t(t->ps3_ntiles) * W, 8), 256, 0, st,
                    t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->P_pw, t->qpart_pw,
                    mem, k_or_rank, P, qpart);

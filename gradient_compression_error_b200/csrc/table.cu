@@ -123,8 +123,7 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_dtile_layer);
     cudaFree(t->d_dtile_start);
     cudaFree(t->d_dc_tile_layer);
-    cudaFree(t->d_dc_sp_tiles);
-    cudaFree(t->d_dc_ot_tiles);
+    cudaFree(t->d_dc_nl_tiles);
     cudaFree(t->d_bunit_layer);
     cudaFree(t->d_bunit_chunk);
     powersgd_plan_free(t);
@@ -150,7 +149,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     int64_t off = 0, voff = 0, poff = 0, qoff = 0, spoff = 0;
     int32_t tiles = 0;
     std::vector<int32_t> tile_layer, sunit_layer, sunit_part, dtile_layer, dtile_start;
-    std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_sp, dc_ot;
+    std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_nl;
     int32_t dc_tiles = 0, dc_slots = 0;
     for (int32_t l = 0; l < L; ++l) {
         const gce_layer_desc& d = descs[l];
@@ -218,8 +217,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
         x.dc_ntiles = int32_t((n + kDcTile - 1) / kDcTile);
         x.dc_base = dc_slots;
         for (int32_t i = 0; i < x.dc_ntiles; ++i) {
-            const bool sp = d.kind == GCE_KIND_TOPK || d.kind == GCE_KIND_RANDK;
-            (sp ? dc_sp : dc_ot).push_back(dc_tiles + i);
+            if (d.kind != GCE_KIND_POWERSGD) dc_nl.push_back(dc_tiles + i);
             dc_tile_layer.push_back(l);
         }
         dc_tiles += x.dc_ntiles;
@@ -255,10 +253,8 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_dtile_layer, dtile_layer);
     if (rc == GCE_OK) rc = upload(&t->d_dtile_start, dtile_start);
     if (rc == GCE_OK) rc = upload(&t->d_dc_tile_layer, dc_tile_layer);
-    t->dc_sp_n = int32_t(dc_sp.size());
-    t->dc_ot_n = int32_t(dc_ot.size());
-    if (rc == GCE_OK) rc = upload(&t->d_dc_sp_tiles, dc_sp);
-    if (rc == GCE_OK) rc = upload(&t->d_dc_ot_tiles, dc_ot);
+    t->dc_nl_n = int32_t(dc_nl.size());
+    if (rc == GCE_OK) rc = upload(&t->d_dc_nl_tiles, dc_nl);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_layer, bunit_layer);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_chunk, bunit_chunk);
     if (rc == GCE_OK) rc = powersgd_plan(t);

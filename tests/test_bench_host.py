@@ -1,0 +1,72 @@
+"""Host-side logic of bench.py: multi-rank timing aggregation (two gloo ranks
+on CPU, as torchrun would launch them) and the CPU reference leg."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+from tests.conftest import ROOT
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    local_ms = [12.5, 20.0][rank]
+    t = bench.max_over_ranks_of(local_ms, world, "cpu")
+    v = bench.job_throughput(world, 1000, 10, t)
+    dist.barrier()
+    dist.destroy_process_group()
+    q.put((rank, t, v))
+
+
+def test_two_gloo_ranks_take_the_slowest_time():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29511
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, t, v in out:
+        assert t == 20.0                          # max over ranks
+        assert v == pytest.approx(2 * 1000 * 10 / 0.020)
+
+
+def run_bench(args, env=None):
+    e = dict(os.environ)
+    e.update(env or {})
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], capture_output=True,
+                       text=True, env=e, timeout=600, cwd=ROOT)
+    return r
+
+
+def test_reference_leg_prints_one_json_line():
+    r = run_bench(["--impl", "reference", "--workload", "memsgd_vector_2p20", "--steps", "2",
+                   "--warmup", "3"])
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "elements/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["higher_is_better"] is True
+
+
+def test_reference_leg_is_silent_on_other_ranks():
+    r = run_bench(["--impl", "reference", "--workload", "memsgd_vector_2p20", "--steps", "2",
+                   "--warmup", "3"], env={"RANK": "1", "WORLD_SIZE": "2"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_warmup_below_three_is_refused():
+    r = run_bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
+    assert r.returncode != 0

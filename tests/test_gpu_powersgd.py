@@ -171,3 +171,14 @@ def test_rank_one_matrix_recovered():
     torch.cuda.synchronize()
     assert float((out - M).norm() / M.norm()) < 1e-5
     assert float(mem.abs().max()) < 1e-5 * float(M.abs().max())
+
+
+def test_tall_p_is_orthonormalised_over_many_blocks():
+    """P taller than 8192 rows takes the multi-block Gram-Schmidt; ranks vary."""
+    need_gpu()
+    layers = [dict(rows=20000, cols=96, kind="powersgd", cap=4, sigma=0.1),
+              dict(rows=16384, cols=1024, kind="powersgd", cap=2, sigma=0.03),
+              dict(rows=300, cols=40, kind="powersgd", cap=4, sigma=0.2)]
+    run = PsRun(layers, 2, seed=11)
+    for s, ranks in enumerate([None, [2, 1, 3], [3, 2, 4]]):
+        run.step(workloads.gradients(layers, 2, 305, s), 0.05, ranks)
