@@ -565,13 +565,33 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
             float pr[kMaxRank];
 #pragma unroll
             for (int j = 0; j < kMaxRank; ++j) pr[j] = j < r ? prow[row][j] : 0.0f;
-            for (int c = lane; c < cw; c += 32) {
-                float mh = __fmul_rn(pr[0], qs[0][c]);
+            if (((e & 3) == 0) && ((cw & 3) == 0)) {  // 16-byte rows: four columns a lane
+                for (int c = lane * 4; c < cw; c += 128) {
+                    float4 mm = *reinterpret_cast<const float4*>(m + c);
+                    float mh[4];
 #pragma unroll
-                for (int j = 1; j < kMaxRank; ++j)
-                    if (j < r) mh = __fmaf_rn(pr[j], qs[j][c], mh);
-                m[c] = __fsub_rn(m[c], mh);
-                if (o) o[c] = mh;
+                    for (int q = 0; q < 4; ++q) {
+                        mh[q] = __fmul_rn(pr[0], qs[0][c + q]);
+#pragma unroll
+                        for (int j = 1; j < kMaxRank; ++j)
+                            if (j < r) mh[q] = __fmaf_rn(pr[j], qs[j][c + q], mh[q]);
+                    }
+                    mm.x = __fsub_rn(mm.x, mh[0]);
+                    mm.y = __fsub_rn(mm.y, mh[1]);
+                    mm.z = __fsub_rn(mm.z, mh[2]);
+                    mm.w = __fsub_rn(mm.w, mh[3]);
+                    *reinterpret_cast<float4*>(m + c) = mm;
+                    if (o) *reinterpret_cast<float4*>(o + c) = make_float4(mh[0], mh[1], mh[2], mh[3]);
+                }
+            } else {
+                for (int c = lane; c < cw; c += 32) {
+                    float mh = __fmul_rn(pr[0], qs[0][c]);
+#pragma unroll
+                    for (int j = 1; j < kMaxRank; ++j)
+                        if (j < r) mh = __fmaf_rn(pr[j], qs[j][c], mh);
+                    m[c] = __fsub_rn(m[c], mh);
+                    if (o) o[c] = mh;
+                }
             }
         }
         __syncthreads();
@@ -613,6 +633,39 @@ __global__ void __launch_bounds__(256) ps_decode_kernel(
             const int w = i / (kPsRB * kMaxRank), rr = (i / kMaxRank) % kPsRB, j = i % kMaxRank;
             prow[w][rr][j] = (rr < rh && j < r) ? P[int64_t(w) * P_pw + L.p_off + (r0 + rr) * cap + j]
                                                 : 0.0f;
+        }
+        const bool rows16 = ((L.offset + r0 * C + c0) & 3) == 0 && (C & 3) == 0 && (cw & 3) == 0;
+        if (W == 1 && rows16) {
+            // one worker, 16-byte rows: a thread owns four neighbouring columns,
+            // keeps their Q in registers and writes float4s down the 16 rows
+            __syncthreads();
+            const int cc = tid * 4;
+            if (cc < cw) {
+                float q[4][kMaxRank];
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+#pragma unroll
+                    for (int j = 0; j < kMaxRank; ++j)
+                        q[c][j] = j < r ? __ldg(Q + L.q_off + (c0 + cc + c) * cap + j) : 0.0f;
+                float* o = out + L.offset + r0 * C + c0 + cc;
+                for (int rr = 0; rr < rh; ++rr) {
+                    float v[4];
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        float m = 0.0f;
+                        if (r > 0) {
+                            m = __fmul_rn(prow[0][rr][0], q[c][0]);
+#pragma unroll
+                            for (int j = 1; j < kMaxRank; ++j)
+                                if (j < r) m = __fmaf_rn(prow[0][rr][j], q[c][j], m);
+                        }
+                        v[c] = __fmul_rn(__fadd_rn(0.0f, m), scale);
+                    }
+                    *reinterpret_cast<float4*>(o + int64_t(rr) * C) = make_float4(v[0], v[1], v[2], v[3]);
+                }
+            }
+            __syncthreads();
+            continue;
         }
         for (int qb = 0; qb < cw; qb += 256) {
             __syncthreads();
