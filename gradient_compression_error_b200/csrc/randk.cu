@@ -346,6 +346,7 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
                 prefetch_l2_bulk(grad + e2, kTkTile * 4);
                 prefetch_l2_bulk(mem + e2, kTkTile * 4);
             }
+            prefetch_l2_bulk(bitmask + t2 * kRkWords, kRkWords * 4);
         }
         const int64_t s = int64_t(w) * ncomp + L.sidx;
         const int32_t k = segs[s].k;
@@ -356,45 +357,46 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
         const float* g = grad + ebase;
         float* m = mem + ebase;
         const uint32_t* bm = bitmask + t * kRkWords;
-        float v[kTkPerThread];
         uint32_t flags = 0;
         const bool vec = cnt == kTkTile && (ebase & 3) == 0;
+        // every load of the tile issued up front, then the arithmetic; the
+        // memory first receives v everywhere, and the few chosen entries are
+        // read back and zeroed once their payload slots are known
+        uint32_t words[kIters];
+#pragma unroll
+        for (int j = 0; j < kIters; ++j) words[j] = __ldcg(bm + ((j * (kTkThreads * 4) + tid * 4) >> 5));
+        if (vec) {
+            float4 gv[kIters], mv[kIters];
+#pragma unroll
+            for (int j = 0; j < kIters; ++j) {
+                const int e = j * (kTkThreads * 4) + tid * 4;
+                gv[j] = ld_stream4(g + e);
+                mv[j] = ld_stream4(m + e);
+            }
+#pragma unroll
+            for (int j = 0; j < kIters; ++j) {
+                const int e = j * (kTkThreads * 4) + tid * 4;
+                float4 x;
+                x.x = residual(mv[j].x, eta, gv[j].x);
+                x.y = residual(mv[j].y, eta, gv[j].y);
+                x.z = residual(mv[j].z, eta, gv[j].z);
+                x.w = residual(mv[j].w, eta, gv[j].w);
+                *reinterpret_cast<float4*>(m + e) = x;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < kIters; ++j) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int e = j * (kTkThreads * 4) + tid * 4 + q;
+                    if (e < cnt) m[e] = residual(m[e], eta, __ldcs(g + e));
+                }
+            }
+        }
 #pragma unroll
         for (int j = 0; j < kIters; ++j) {
             const int e = j * (kTkThreads * 4) + tid * 4;
-            const uint32_t word = bm[e >> 5];
-            const uint32_t f = (word >> (e & 31)) & 0xFu;
-            float4 x;
-            if (vec) {
-                const float4 gg = ld_stream4(g + e);
-                const float4 mm = ld_stream4(m + e);
-                x.x = residual(mm.x, eta, gg.x);
-                x.y = residual(mm.y, eta, gg.y);
-                x.z = residual(mm.z, eta, gg.z);
-                x.w = residual(mm.w, eta, gg.w);
-                float4 o;
-                o.x = (f & 1u) ? 0.0f : x.x;
-                o.y = (f & 2u) ? 0.0f : x.y;
-                o.z = (f & 4u) ? 0.0f : x.z;
-                o.w = (f & 8u) ? 0.0f : x.w;
-                *reinterpret_cast<float4*>(m + e) = o;
-            } else {
-                float xs[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    xs[q] = 0.0f;
-                    if (e + q < cnt) {
-                        xs[q] = residual(m[e + q], eta, __ldcs(g + e + q));
-                        m[e + q] = (f & (1u << q)) ? 0.0f : xs[q];
-                    }
-                }
-                x = make_float4(xs[0], xs[1], xs[2], xs[3]);
-            }
-            v[4 * j + 0] = x.x;
-            v[4 * j + 1] = x.y;
-            v[4 * j + 2] = x.z;
-            v[4 * j + 3] = x.w;
-            flags |= f << (4 * j);
+            flags |= ((words[j] >> (e & 31)) & 0xFu) << (4 * j);
         }
         int incl[kIters];
 #pragma unroll
@@ -420,8 +422,10 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 if ((f & (1u << q)) && pos < k) {
-                    vout[pos] = v[4 * j + q];
-                    iout[pos] = int32_t(tstart + j * (kTkThreads * 4) + tid * 4 + q);
+                    const int e = j * (kTkThreads * 4) + tid * 4 + q;
+                    vout[pos] = m[e];
+                    iout[pos] = int32_t(tstart + e);
+                    m[e] = 0.0f;
                 }
                 pos += (f >> q) & 1u;
             }
