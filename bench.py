@@ -366,16 +366,21 @@ def main():
     main_kernel = MAIN_KERNELS[method]
     main_ms, main_n = prof.get(main_kernel, (0.0, 0))
     peak, peak_kind = measured_hbm_gbs()
-    bytes_per_launch = 12.0 * W * (N - sum(l["rows"] * l["cols"] for l in layers
-                                          if l["kind"] == "dense"))
-    achieved = bytes_per_launch / (main_ms / main_n / 1e3) / 1e9 if main_n else None
+    # the main pass covers every compressed element once per step: bytes and
+    # kernel time per step
+    bytes_per_step_main = 12.0 * W * (N - sum(l["rows"] * l["cols"] for l in layers
+                                             if l["kind"] == "dense"))
+    main_launches_per_step = main_n / args.steps
+    main_ms_per_step = main_ms / args.steps
+    achieved = (bytes_per_step_main / (main_ms_per_step / 1e3) / 1e9) if main_n else None
     traffic = ncu_traffic_per_launch() if args.workload == DEFAULT_WORKLOAD else None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                 "kernel": main_kernel,
                 "peak_source": peak_kind,
-                "algorithmic_bytes_per_launch": bytes_per_launch,
-                "avg_launch_ms": main_ms / main_n if main_n else None}
+                "algorithmic_bytes_per_step": bytes_per_step_main,
+                "launches_per_step": main_launches_per_step,
+                "kernel_ms_per_step": main_ms_per_step if main_n else None}
     # whole-step algorithmic traffic: sparse W(12N + 8K) encode + 16 W K + 4N
     # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
     if method == "powersgd":

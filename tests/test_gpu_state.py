@@ -112,7 +112,7 @@ def test_cuda_graph_replay_matches_eager():
     need_gpu()
     g = gce()
     layers = workloads.bert_base_topk()[:20]
-    W = 2
+    W = 4
     t = g.Table(workloads.table_layers(layers))
     grads = [workloads.gradients(layers, W, 403, s) for s in range(3)]
     e = topk_buffers(g, t, W)

@@ -153,6 +153,44 @@ def test_forced_fallback_is_still_exact():
         g.set_bracket_sigma(6.0)
 
 
+def test_large_table_with_fallback_in_every_layer():
+    """Ten 2.5 M-element top-k layers and a dense one over 4 workers (about
+    1.2 GB of main-pass traffic), run once on the sampled bounds and once
+    with every layer forced to the exact fallback.  Properties on every unit,
+    the oracle on four units."""
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=2500, cols=1000, kind="topk", cap=25000, sigma=1.0) for _ in range(10)]
+    layers.insert(5, dict(rows=300, cols=7, kind="dense", cap=0))
+    W = 4
+    units = [(3, 1), (0, 4), (1, 6), (2, 10)]
+    for sigma in (6.0, -60.0):
+        try:
+            g.set_bracket_sigma(sigma)
+            run = TopkRun(layers, W)
+            host_mem = {u: np.zeros(2500 * 1000, np.float32) for u in units}
+            for t in range(2):
+                grad = workloads.gradients(layers, W, 106, t)
+                mem_old = run.mem.clone()
+                run.step(grad, workloads.ETA)
+                check_topk_properties(run, grad, mem_old, workloads.ETA)
+                del mem_old
+                vals, idx = host(run.vals), host(run.idx)
+                for (w, l) in units:
+                    ls = layer_slice(run.table, l)
+                    ev, ei, m_new = oracle.ef_topk_unit(host(grad[w, ls]), host_mem[(w, l)],
+                                                        layers[l]["cap"], workloads.ETA)
+                    host_mem[(w, l)] = m_new
+                    sl = payload_slice(run.table, 0, l, layers[l]["cap"])
+                    assert np.array_equal(idx[w, sl], ei), (sigma, w, l)
+                    assert np.array_equal(bits(vals[w, sl]), bits(ev)), (sigma, w, l)
+                    assert np.array_equal(bits(host(run.mem[w, ls])), bits(m_new)), (sigma, w, l)
+            if sigma < 0:
+                assert g.status(run.ws) & g.STATUS_FALLBACK
+        finally:
+            g.set_bracket_sigma(6.0)
+
+
 def test_k_out_of_range_skips_layer_and_flags():
     need_gpu()
     g = gce()
@@ -210,6 +248,11 @@ def check_topk_properties(run, grad, mem_old, eta):
         off = t.info[l]["offset"]
         k = lay["cap"]
         vo = t.info[l]["val_offset"]
+        if lay["kind"] == "dense":     # sent whole; memory left at zero
+            dv = run.vals[:, vo:vo + n]
+            assert torch.equal(dv.view(torch.int32), v[:, off:off + n].view(torch.int32)), l
+            sent[:, off:off + n] = dv
+            continue
         ix = run.idx[:, vo:vo + k].long()
         vv = run.vals[:, vo:vo + k]
         assert bool((ix[:, 1:] > ix[:, :-1]).all()) if k > 1 else True, l
