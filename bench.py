@@ -46,6 +46,8 @@ def workload_spec(name):
     from gradient_compression_error_b200 import workloads as wl
     if name == "bert_base_topk1pct_w8":
         return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk")
+    if name == "bert_base_topk1pct_w8_apply":    # decode fused with x -= mean update, eta_t
+        return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk", apply=True)
     if name == "bert_base_topk1pct_w1":          # one replica: a profiling-sized case
         return dict(layers=wl.bert_base_topk(), W=1, cfg=4, method="topk")
     if name == "bert_base_randk1pct_w8":
@@ -313,18 +315,29 @@ def main():
         gce.accordion_init(table, prev, level)
         lvl_low, lvl_high = spec["accordion"]
 
+    apply = bool(spec.get("apply"))
+    if apply:    # the parameters the mean update is applied to, in place
+        out.normal_(generator=torch.Generator(device=dev).manual_seed(77))
+
     def step(s, grad):
+        # the Mem-SGD step size eta_t = 8 / (mu (a + t)) with mu = 1, a = 160
+        # (eta_0 = 0.05) when the update is applied; the fixed eta otherwise
+        eta = gce.memsgd_eta(s, 1.0, 160.0) if apply else wl.ETA
         if kr is not None:
             gce.accordion_select(table, grad[0], s, 10, 0.5, lvl_low, lvl_high, prev, level, cur,
                                  kr, ws_ac)
         if method == "topk":
-            gce.ef_topk_step(table, W, grad, mem, wl.ETA, kr, vals, idx, ws)
+            gce.ef_topk_step(table, W, grad, mem, eta, kr, vals, idx, ws)
         elif method == "randk":
-            gce.ef_randk_step(table, W, grad, mem, wl.ETA, kr, 5, s, vals, idx, ws)
+            gce.ef_randk_step(table, W, grad, mem, eta, kr, 5, s, vals, idx, ws)
         else:
-            gce.powersgd_step(table, W, grad, mem, wl.ETA, kr, P, Q, vals, None, ws)
-        gce.decompress_accumulate(table, W, vals, idx if method != "powersgd" else None, kr, P, Q,
-                                  1.0, out, ws_dc)
+            gce.powersgd_step(table, W, grad, mem, eta, kr, P, Q, vals, None, ws)
+        if apply:
+            gce.decompress_apply(table, W, vals, idx if method != "powersgd" else None, kr, P, Q,
+                                 1.0 / W, out, ws_dc)
+        else:
+            gce.decompress_accumulate(table, W, vals, idx if method != "powersgd" else None, kr,
+                                      P, Q, 1.0, out, ws_dc)
 
     def barrier():
         if world > 1:
@@ -384,9 +397,11 @@ def main():
     # whole-step algorithmic traffic: sparse W(12N + 8K) encode + 16 W K + 4N
     # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
     if method == "powersgd":
-        step_bytes = W * 12.0 * N + 4.0 * N
+        step_bytes = W * 12.0 * N
     else:
-        step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total + 4.0 * N
+        step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total
+    # the dense result: written (4 B), or read and written in place (8 B)
+    step_bytes += (8.0 if apply else 4.0) * N
     step_gbs = step_bytes / (ms_step / 1e3) / 1e9
 
     # end to end through the public API with host buffers
@@ -434,7 +449,9 @@ def main():
                 "data": "synthetic (seeded N(0,1) gradients, resident in HBM)",
                 "config": {"workload": args.workload, "W": W, "elements_per_worker": N,
                            "tensors": len(layers), "k_total_per_worker": K_total,
-                           "eta": wl.ETA, "parallelism": "replicas x%d" % world,
+                           "eta": "8/(1*(160+t))" if apply else wl.ETA,
+                           "update": "x -= mean of payloads (fused)" if apply else "decode only",
+                           "parallelism": "replicas x%d" % world,
                            "l2": "inputs larger than L2 (%.1f GB of grad+memory per step)"
                                  % (8.0 * W * N / 1e9),
                            "step_algorithmic_GBps": step_gbs,

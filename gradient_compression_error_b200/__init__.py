@@ -73,6 +73,9 @@ SIGNATURES = {
                                         C.c_size_t, _vp]),
     "decompress_accumulate_noalloc": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _f32, _vp,
                                                 _vp]),
+    "decompress_apply": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _f32, _vp, _vp,
+                                   C.c_size_t, _vp]),
+    "gce_memsgd_eta": (C.c_int, [_i64, _f64, _f64, C.POINTER(_f32)]),
     "gce_status": (C.c_int, [_vp, _vp, C.POINTER(_i32)]),
     "gce_launch_count": (_u64, []),
     "gce_error_string": (C.c_char_p, [C.c_int]),
@@ -230,6 +233,21 @@ def decompress_accumulate(table, W, vals, idx, k_or_rank, P, Q, scale, out, ws, 
         table.handle, int(W), _ptr(vals, _f32()), _ptr(idx, _i32()), _ptr(k_or_rank, _i32()),
         _ptr(P, _f32()), _ptr(Q, _f32()), float(scale), _ptr(out, _f32()), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def decompress_apply(table, W, vals, idx, k_or_rank, P, Q, scale, x, ws, stream=None):
+    """x -= scale * (worker-order sum of the payloads), in place (include/gce.h)."""
+    _check("decompress_apply", lib().decompress_apply(
+        table.handle, int(W), _ptr(vals, _f32()), _ptr(idx, _i32()), _ptr(k_or_rank, _i32()),
+        _ptr(P, _f32()), _ptr(Q, _f32()), float(scale), _ptr(x, _f32()), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def memsgd_eta(step, mu, a):
+    """Step size 8 / (mu (a + t)) of the Mem-SGD method, as a float."""
+    e = C.c_float()
+    _check("gce_memsgd_eta", lib().gce_memsgd_eta(int(step), float(mu), float(a), C.byref(e)))
+    return e.value
 
 
 def decompress_accumulate_noalloc(table, W, vals, idx, k_or_rank, P, Q, scale, out, stream=None):

@@ -182,11 +182,12 @@ extern "C" int accordion_select(const gce_table* t, const float* grad, int64_t s
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     double* part = at<double>(ws, GCE_WS_HEADER_BYTES);
     const int check = (step % interval) == 0;
-    const int sms = sm_count();
+    static const int r_norm = resident_blocks(ac_norm_kernel, 256);
+    static const int r_decide = resident_blocks(ac_decide_kernel, 256);
     if (check && t->ac_ntiles > 0)
-        GCE_LAUNCH(ac_norm_kernel, int(min64(t->ac_ntiles, int64_t(sms) * 8)), 256, 0, st,
+        GCE_LAUNCH(ac_norm_kernel, wave_grid(t->ac_ntiles, 8, r_norm), 256, 0, st,
                    t->d_layers, t->d_ac_tiles, t->ac_ntiles, grad, part);
-    GCE_LAUNCH(ac_decide_kernel, int(min64((t->L + 7) / 8, int64_t(sms) * 4)), 256, 0, st,
+    GCE_LAUNCH(ac_decide_kernel, wave_grid((t->L + 7) / 8, 4, r_decide), 256, 0, st,
                t->d_layers, t->d_ac_layer, t->L, part, check, threshold, lvl_low, lvl_high,
                prev_norm, level, cur_norm, k_or_rank_out);
     return check_launch();

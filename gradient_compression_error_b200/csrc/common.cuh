@@ -107,6 +107,27 @@ inline int check_launch() {
 // ---- device properties (cached per device) --------------------------------
 int sm_count();
 
+// ---- grids -------------------------------------------------------------------
+// Blocks of `kernel` (`threads` threads, no dynamic shared memory) that fit on
+// one SM at once.
+template <class K>
+inline int resident_blocks(K kernel, int threads) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1)
+        n = 1;
+    return n;
+}
+
+// Grid of a grid-stride kernel: at most `per_sm` blocks per SM and never more
+// than fit at once (`resident`), so the whole grid runs in one wave.  A block
+// of a second, partial wave would start only when a first-wave block had
+// finished all of its tiles, nearly doubling the kernel's time.
+inline int wave_grid(int64_t work, int per_sm, int resident) {
+    const int p = per_sm < resident ? per_sm : resident;
+    const int64_t cap = int64_t(sm_count()) * p;
+    return int(work < 1 ? 1 : (work < cap ? work : cap));
+}
+
 // ---- workspace carving ------------------------------------------------------
 struct Carver {
     size_t off = GCE_WS_HEADER_BYTES;
@@ -139,6 +160,26 @@ __device__ __forceinline__ float residual(float m, float eta, float g) {
     return __fadd_rn(m, __fmul_rn(eta, g));
 }
 
+// Last step of every decoder: out = fl(scale * s), or, fused with the
+// parameter update x_{t+1} = x_t - g_t (kApply), x = fl(x - fl(scale * s)).
+template <bool kApply>
+__device__ __forceinline__ float dc_final(float s, float scale, const float* o) {
+    const float u = __fmul_rn(s, scale);
+    return kApply ? __fsub_rn(*o, u) : u;
+}
+
+template <bool kApply>
+__device__ __forceinline__ float4 dc_final4(float4 s, float scale, const float4* o4) {
+    float4 u = make_float4(__fmul_rn(s.x, scale), __fmul_rn(s.y, scale), __fmul_rn(s.z, scale),
+                           __fmul_rn(s.w, scale));
+    if (kApply) {
+        const float4 x = __ldcs(o4);
+        u = make_float4(__fsub_rn(x.x, u.x), __fsub_rn(x.y, u.y), __fsub_rn(x.z, u.z),
+                        __fsub_rn(x.w, u.w));
+    }
+    return u;
+}
+
 // |v| ordering key: the float's bits with the sign cleared.
 __device__ __forceinline__ uint32_t abs_key(float v) {
     return __float_as_uint(v) & 0x7FFFFFFFu;
@@ -162,7 +203,7 @@ constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
                         float eta, float* vals, cudaStream_t st);
 bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_rank,
-                           const float* P, const float* Q, float scale, float* out,
+                           const float* P, const float* Q, float scale, float* out, bool apply,
                            cudaStream_t st);
 int powersgd_plan(gce_table* t);   // called once by gce_table_create
 void powersgd_plan_free(gce_table* t);

@@ -20,7 +20,9 @@
 
 namespace gce {
 
-constexpr int kDcStage = 2048;  // payload entries staged in shared memory per tile
+constexpr int kDcThreads = 128;                   // 4 warps per decode tile
+constexpr int kDcSpan = kDcTile / (kDcThreads / 32);  // outputs each warp owns: 1024
+constexpr int kDcStage = 960;   // entries staged per pass (9 blocks of 24 KB fit an SM)
 
 size_t decompress_ws_bytes(const gce_table* t, int32_t W) {
     Carver c;
@@ -60,17 +62,99 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
         }
         const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
         const int64_t j1 = min64(j0 + kDcBoundChunk, k);
-        for (int64_t j = j0 + threadIdx.x; j < j1; j += blockDim.x) {
-            const int32_t tj = min(max(ix[j], 0) >> kDcTileLog, nt);
-            const int32_t tp = j > 0 ? min(max(ix[j - 1], 0) >> kDcTileLog, nt) : -1;
-            for (int32_t tt = tp + 1; tt <= tj; ++tt) b[tt] = int32_t(j);
-            if (j == k - 1)
-                for (int32_t tt = tj + 1; tt <= nt; ++tt) b[tt] = k;
+        constexpr int kBatch = 8;  // loads in flight per thread
+        for (int64_t jb = j0 + threadIdx.x; jb < j1; jb += int64_t(kBatch) * blockDim.x) {
+            int32_t cur[kBatch], prev[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int64_t j = jb + int64_t(q) * blockDim.x;
+                cur[q] = j < j1 ? ix[j] : 0;
+                prev[q] = (j < j1 && j > 0) ? ix[j - 1] : 0;
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int64_t j = jb + int64_t(q) * blockDim.x;
+                if (j >= j1) continue;
+                const int32_t tj = min(max(cur[q], 0) >> kDcTileLog, nt);
+                const int32_t tp = j > 0 ? min(max(prev[q], 0) >> kDcTileLog, nt) : -1;
+                for (int32_t tt = tp + 1; tt <= tj; ++tt) b[tt] = int32_t(j);
+                if (j == k - 1)
+                    for (int32_t tt = tj + 1; tt <= nt; ++tt) b[tt] = k;
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(256) dc_accum_kernel(
+// First position in [l, r) of the sorted run s[l..r) whose value is >= key.
+__device__ __forceinline__ int lower_bound_smem(const int32_t* s, int l, int r, int key) {
+    while (l < r) {
+        const int m = (l + r) >> 1;
+        if (s[m] < key) l = m + 1;
+        else r = m;
+    }
+    return l;
+}
+
+// The staged entries (tile-relative index, value) that fall in this warp's
+// kDcSpan outputs are added to the accumulator, one worker after the other.  The
+// stage holds entries [c0, c0 + cn) of the tile's worker-ordered list, and
+// each worker's run is sorted by index, so lane w finds worker w's part of
+// the warp's range by binary search in shared memory.  Within one worker the
+// indices are distinct, so the lanes add without conflict.  Run by a full
+// warp; W <= 32.
+__device__ __forceinline__ void dc_add_staged(float* acc, const int32_t* s_sidx,
+                                              const float* s_sval, const int32_t* s_off,
+                                              int c0, int cn, int W, int warp, int cnt) {
+    const int lane = threadIdx.x & 31;
+    const int lo = warp * kDcSpan, hi = min(lo + kDcSpan, cnt);
+    int a = 0, b = 0;
+    if (lane < W) {
+        const int e = lane + 1 < W ? s_off[lane + 1] : s_off[32];
+        const int r0 = min(max(s_off[lane] - c0, 0), cn);
+        const int r1 = min(max(e - c0, r0), cn);
+        a = lower_bound_smem(s_sidx, r0, r1, lo);
+        b = lower_bound_smem(s_sidx, a, r1, hi);
+    }
+    for (int w = 0; w < W; ++w) {
+        const int aw = __shfl_sync(kFull, a, w), bw = __shfl_sync(kFull, b, w);
+        for (int j = aw + lane; j < bw; j += 32) {
+            const int i = s_sidx[j];
+            if (i >= lo && i < hi) acc[i] = __fadd_rn(acc[i], s_sval[j]);  // sorted input: always
+        }
+        __syncwarp();
+    }
+}
+
+// Write this warp's kDcSpan outputs (times scale) and zero them in the
+// accumulator for the next tile.  Run by a full warp after __syncwarp.
+// Write this warp's kDcSpan outputs and zero them in the accumulator for the
+// next tile: out = fl(scale * sum), or with kApply x = fl(x - fl(scale * sum)).
+// Run by a full warp after __syncwarp.
+template <bool kApply>
+__device__ __forceinline__ void dc_write_quarter(float* acc, float* o, int cnt, int warp,
+                                                 float scale, bool aligned) {
+    const int lane = threadIdx.x & 31;
+    const int lo = warp * kDcSpan;
+    if (aligned && lo + kDcSpan <= cnt) {
+        float4* a4 = reinterpret_cast<float4*>(acc + lo);
+        float4* o4 = reinterpret_cast<float4*>(o + lo);
+#pragma unroll
+        for (int j = 0; j < kDcSpan / 4 / 32; ++j) {
+            const float4 x = a4[lane + 32 * j];
+            __stcs(o4 + lane + 32 * j, dc_final4<kApply>(x, scale, o4 + lane + 32 * j));
+            a4[lane + 32 * j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+    } else {
+        for (int i = lo + lane; i < lo + kDcSpan; i += 32) {
+            if (i < cnt) o[i] = dc_final<kApply>(acc[i], scale, o + i);
+            acc[i] = 0.0f;
+        }
+    }
+    __syncwarp();
+}
+
+template <bool kApply>
+__global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
     const int32_t* __restrict__ tile_list, int32_t dc_tiles, int32_t W, int64_t vals_pw,
     int64_t P_pw, int64_t Q_pw, int32_t dc_slots, const int32_t* __restrict__ k_or_rank,
@@ -82,6 +166,11 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
     __shared__ int32_t s_sidx[kDcStage];
     __shared__ float s_sval[kDcStage];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // the accumulator is all zero between sparse tiles: each warp zeroes the
+    // part it writes out
+    for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
+        reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncthreads();
     for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
         const int32_t t = tile_list ? tile_list[u] : u;
         const int32_t l = dc_tile_layer[t];
@@ -92,75 +181,99 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
         float* o = out + L.offset + start;
         if (L.kind == GCE_KIND_TOPK || L.kind == GCE_KIND_RANDK) {
             const int32_t k = layer_k(L, k_or_rank, l);
+            if (W <= 32) {
+                // Warp w of the block owns outputs [w, w + 1) x kDcSpan of the
+                // tile: it adds the staged entries that fall there and writes
+                // them out, so the accumulator needs no block-wide barrier
+                // between the adds and the write.  Every worker's entry range
+                // for the tile is read at once, then the entries are staged
+                // in worker order, kDcStage at a time.
+                if (warp == 0) {
+                    int32_t a = 0, e = 0;
+                    if (lane < W) {
+                        const int32_t* b = bounds + int64_t(lane) * dc_slots + L.dc_base + tt;
+                        a = min(max(b[0], 0), k);
+                        e = min(max(b[1], a), k);
+                        s_first[lane] = a;
+                    }
+                    const int c = e - a;
+                    const int incl = warp_inclusive_scan(c);
+                    if (lane < W) s_off[lane] = incl - c;
+                    if (lane == 31) s_off[32] = incl;
+                }
+                __syncthreads();
+                const int total = s_off[32];
+                // at least one pass, so that every warp has read this tile's
+                // s_off before warp 0 writes the next tile's
+                int c0 = 0;
+                do {
+                    const int cn = min(kDcStage, total - c0);
+                    if (c0 > 0) __syncthreads();  // every warp is done with the last chunk
+                    // kSB entries per thread in flight: all loads first, then the stores
+                    constexpr int kSB = 4;
+                    for (int q0 = 0; q0 < cn; q0 += kSB * kDcThreads) {
+                        int32_t ri[kSB];
+                        float rv[kSB];
+#pragma unroll
+                        for (int e = 0; e < kSB; ++e) {
+                            const int q = q0 + e * kDcThreads + int(threadIdx.x);
+                            ri[e] = 0;
+                            rv[e] = 0.0f;
+                            if (q < cn) {
+                                const int qq = c0 + q;
+                                int w = 0;  // the last worker whose entries start at or before qq
+#pragma unroll
+                                for (int step = 16; step > 0; step >>= 1)
+                                    if (w + step < W && s_off[w + step] <= qq) w += step;
+                                const int64_t o2 = int64_t(w) * vals_pw + L.val_off + s_first[w] +
+                                                   (qq - s_off[w]);
+                                ri[e] = idx[o2];
+                                rv[e] = vals[o2];
+                            }
+                        }
+#pragma unroll
+                        for (int e = 0; e < kSB; ++e) {
+                            const int q = q0 + e * kDcThreads + int(threadIdx.x);
+                            if (q < cn) {
+                                s_sidx[q] = int32_t(int64_t(ri[e]) - start);
+                                s_sval[q] = rv[e];
+                            }
+                        }
+                    }
+                    __syncthreads();
+                    dc_add_staged(acc, s_sidx, s_sval, s_off, c0, cn, W, warp, cnt);
+                    c0 += kDcStage;
+                } while (c0 < total);
+                __syncwarp();
+                dc_write_quarter<kApply>(acc, o, cnt, warp, scale, ((L.offset + start) & 3) == 0);
+                continue;
+            }
+            // more than 32 workers: one worker at a time, straight from memory
+            for (int w = 0; w < W; ++w) {
+                __syncthreads();
+                const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base + tt;
+                const int32_t a = min(max(b[0], 0), k), e = min(max(b[1], a), k);
+                const float* v = vals + int64_t(w) * vals_pw + L.val_off;
+                const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
+                for (int32_t j = a + threadIdx.x; j < e; j += blockDim.x) {
+                    const int64_t i = int64_t(ix[j]) - start;
+                    if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], v[j]);
+                }
+            }
+            __syncthreads();
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x)
+                o[i] = dc_final<kApply>(acc[i], scale, o + i);
+            __syncthreads();
+            // leave the accumulator at zero for the next tile's staged path
             for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
                 reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            // every worker's entry range for this tile at once, then one staged
-            // load of all the entries, so the worker-order sums below touch
-            // only shared memory
-            if (W <= 32 && warp == 0) {
-                int32_t a = 0, e = 0;
-                if (lane < W) {
-                    const int32_t* b = bounds + int64_t(lane) * dc_slots + L.dc_base + tt;
-                    a = min(max(b[0], 0), k);
-                    e = min(max(b[1], a), k);
-                    s_first[lane] = a;
-                }
-                const int c = e - a;
-                const int incl = warp_inclusive_scan(c);
-                if (lane < W) s_off[lane] = incl - c;
-                if (lane == 31) s_off[32] = incl;
-            }
-            __syncthreads();
-            const bool staged = W <= 32 && s_off[32] <= kDcStage;
-            if (staged) {
-                const int total = s_off[32];
-                for (int q = threadIdx.x; q < total; q += blockDim.x) {
-                    int w = 0;
-                    while (w + 1 < W && s_off[w + 1] <= q) ++w;
-                    const int64_t j = int64_t(s_first[w]) + (q - s_off[w]);
-                    const int64_t o2 = int64_t(w) * vals_pw + L.val_off + j;
-                    s_sidx[q] = int32_t(int64_t(idx[o2]) - start);
-                    s_sval[q] = vals[o2];
-                }
-                for (int w = 0; w < W; ++w) {
-                    __syncthreads();
-                    for (int q = s_off[w] + threadIdx.x; q < s_off[w + 1 < W ? w + 1 : 32];
-                         q += blockDim.x) {
-                        const int i = s_sidx[q];
-                        if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], s_sval[q]);
-                    }
-                }
-            } else {
-                for (int w = 0; w < W; ++w) {
-                    __syncthreads();
-                    const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base + tt;
-                    const int32_t a = min(max(b[0], 0), k), e = min(max(b[1], a), k);
-                    const float* v = vals + int64_t(w) * vals_pw + L.val_off;
-                    const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
-                    for (int32_t j = a + threadIdx.x; j < e; j += blockDim.x) {
-                        const int64_t i = int64_t(ix[j]) - start;
-                        if (i >= 0 && i < cnt) acc[i] = __fadd_rn(acc[i], v[j]);
-                    }
-                }
-            }
-            __syncthreads();
-            if (cnt == kDcTile && ((L.offset + start) & 3) == 0) {
-                for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x) {
-                    const float4 a = reinterpret_cast<const float4*>(acc)[i];
-                    reinterpret_cast<float4*>(o)[i] =
-                        make_float4(__fmul_rn(a.x, scale), __fmul_rn(a.y, scale),
-                                    __fmul_rn(a.z, scale), __fmul_rn(a.w, scale));
-                }
-            } else {
-                for (int i = threadIdx.x; i < cnt; i += blockDim.x) o[i] = __fmul_rn(acc[i], scale);
-            }
             __syncthreads();
         } else if (L.kind == GCE_KIND_DENSE) {
             for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
                 float s = 0.0f;
                 for (int w = 0; w < W; ++w)
                     s = __fadd_rn(s, vals[int64_t(w) * vals_pw + L.val_off + start + i]);
-                o[i] = __fmul_rn(s, scale);
+                o[i] = dc_final<kApply>(s, scale, o + i);
             }
         } else {  // POWERSGD: P Q^T over the first r columns
             const int32_t r = layer_k(L, k_or_rank, l);
@@ -184,7 +297,7 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
                     }
                     s = __fadd_rn(s, m);
                 }
-                o[i] = __fmul_rn(s, scale);
+                o[i] = dc_final<kApply>(s, scale, o + i);
                 col += blockDim.x;
                 if (col >= cols) {
                     row += col / cols;
@@ -195,31 +308,40 @@ __global__ void __launch_bounds__(256) dc_accum_kernel(
     }
 }
 
-// bounds pass plus the decode kernels for every kind the table holds
-static int launch_decode(const gce_table* t, int32_t W, const float* vals, const int32_t* idx,
-                         const int32_t* k_or_rank, const float* P, const float* Q, float scale,
-                         float* out, int32_t* bounds, cudaStream_t st) {
+// bounds pass plus the decode kernels for every kind the table holds;
+// apply: out is the parameter vector x and gets x - scale * sum
+template <bool kApply>
+static int launch_decode_t(const gce_table* t, int32_t W, const float* vals, const int32_t* idx,
+                           const int32_t* k_or_rank, const float* P, const float* Q, float scale,
+                           float* out, int32_t* bounds, cudaStream_t st) {
     const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
-    const int sms = sm_count();
+    static const int r_bounds = resident_blocks(dc_bounds_kernel, 256);
+    static const int r_accum = resident_blocks(dc_accum_kernel<kApply>, kDcThreads);
     if (sparse && t->bunits_pw > 0) {
         const int64_t units = int64_t(t->bunits_pw) * W;
-        GCE_LAUNCH(dc_bounds_kernel, int(min64(units, int64_t(sms) * 8)), 256, 0, st, t->d_layers,
+        GCE_LAUNCH(dc_bounds_kernel, wave_grid(units, 8, r_bounds), 256, 0, st, t->d_layers,
                    t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
                    k_or_rank, idx, bounds);
     }
-    if (t->nps > 0 && launch_lowrank_decode(t, W, k_or_rank, P, Q, scale, out, st)) {
+    if (t->nps > 0 && launch_lowrank_decode(t, W, k_or_rank, P, Q, scale, out, kApply, st)) {
         // PowerSGD layers done by their own tiled kernel; the rest here
         if (t->dc_nl_n > 0)
-            GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_nl_n, int64_t(sms) * 8)), 256, 0, st,
-                       t->d_layers, t->d_dc_tile_layer, t->d_dc_nl_tiles, t->dc_nl_n, W,
+            GCE_LAUNCH(dc_accum_kernel<kApply>, wave_grid(t->dc_nl_n, 16, r_accum), kDcThreads, 0,
+                       st, t->d_layers, t->d_dc_tile_layer, t->d_dc_nl_tiles, t->dc_nl_n, W,
                        t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q,
                        bounds, scale, out);
         return check_launch();
     }
-    GCE_LAUNCH(dc_accum_kernel, int(min64(t->dc_tiles, int64_t(sms) * 8)), 256, 0, st,
+    GCE_LAUNCH(dc_accum_kernel<kApply>, wave_grid(t->dc_tiles, 16, r_accum), kDcThreads, 0, st,
                t->d_layers, t->d_dc_tile_layer, nullptr, t->dc_tiles, W, t->vals_pw, t->P_pw,
                t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q, bounds, scale, out);
     return check_launch();
+}
+
+static int launch_decode(const gce_table* t, int32_t W, const float* vals, const int32_t* idx,
+                         const int32_t* k_or_rank, const float* P, const float* Q, float scale,
+                         float* out, int32_t* bounds, cudaStream_t st) {
+    return launch_decode_t<false>(t, W, vals, idx, k_or_rank, P, Q, scale, out, bounds, st);
 }
 
 }  // namespace gce
@@ -237,6 +359,28 @@ extern "C" int decompress_accumulate(const gce_table* t, int32_t W, const float*
     if (ws_bytes < decompress_ws_bytes(t, W)) return GCE_ERR_WORKSPACE;
     return launch_decode(t, W, vals, idx, k_or_rank, P, Q, scale, out,
                          at<int32_t>(ws, GCE_WS_HEADER_BYTES), static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int decompress_apply(const gce_table* t, int32_t W, const float* vals,
+                                const int32_t* idx, const int32_t* k_or_rank, const float* P,
+                                const float* Q, float scale, float* x, void* ws, size_t ws_bytes,
+                                void* stream) {
+    if (!t || W < 1 || !x || !ws || !aligned16(x) || !aligned16(ws)) return GCE_ERR_ARG;
+    const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
+    if ((t->vals_pw > 0 && !vals) || (sparse && !idx)) return GCE_ERR_ARG;
+    if (t->ckind == GCE_KIND_POWERSGD && (!P || !Q)) return GCE_ERR_ARG;
+    if (ws_bytes < decompress_ws_bytes(t, W)) return GCE_ERR_WORKSPACE;
+    return launch_decode_t<true>(t, W, vals, idx, k_or_rank, P, Q, scale, x,
+                                 at<int32_t>(ws, GCE_WS_HEADER_BYTES),
+                                 static_cast<cudaStream_t>(stream));
+}
+
+extern "C" int gce_memsgd_eta(int64_t step, double mu, double a, float* eta) {
+    if (!eta || !(mu > 0.0) || !(a + double(step) > 0.0) || step < 0) return GCE_ERR_ARG;
+    const double e = 8.0 / (mu * (a + double(step)));
+    if (!(e < 3.0e38)) return GCE_ERR_ARG;
+    *eta = float(e);
+    return GCE_OK;
 }
 
 // ---- decode without a caller workspace -------------------------------------------------

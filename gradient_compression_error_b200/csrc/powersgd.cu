@@ -598,10 +598,6 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
     }
 }
 
-static int grid_of(int64_t work, int per_sm) {
-    return int(max64(1, min64(work, int64_t(sm_count()) * per_sm)));
-}
-
 // ---- decode of PowerSGD payloads: out = scale * sum_w P_w Q_w^T ---------------------------
 // Per (16-row, 1024-column) tile, in 256-column quarters: the quarter's Q
 // columns and the tile's P rows of every worker sit in shared memory, each
@@ -611,6 +607,7 @@ static int grid_of(int64_t work, int per_sm) {
 // the workers summed in order from +0), so both give the same bits.
 constexpr int kDcLrMaxW = 8;
 
+template <bool kApply>
 __global__ void __launch_bounds__(256) ps_decode_kernel(
     const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles,
     int32_t W, int64_t P_pw, int64_t Q_pw, const int32_t* __restrict__ k_or_rank,
@@ -659,9 +656,10 @@ __global__ void __launch_bounds__(256) ps_decode_kernel(
                             for (int j = 1; j < kMaxRank; ++j)
                                 if (j < r) m = __fmaf_rn(prow[0][rr][j], q[c][j], m);
                         }
-                        v[c] = __fmul_rn(__fadd_rn(0.0f, m), scale);
+                        v[c] = __fadd_rn(0.0f, m);
                     }
-                    *reinterpret_cast<float4*>(o + int64_t(rr) * C) = make_float4(v[0], v[1], v[2], v[3]);
+                    float4* o4 = reinterpret_cast<float4*>(o + int64_t(rr) * C);
+                    *o4 = dc_final4<kApply>(make_float4(v[0], v[1], v[2], v[3]), scale, o4);
                 }
             }
             __syncthreads();
@@ -689,7 +687,7 @@ __global__ void __launch_bounds__(256) ps_decode_kernel(
                         }
                         s = __fadd_rn(s, m);
                     }
-                    o[int64_t(rr) * C] = __fmul_rn(s, scale);
+                    o[int64_t(rr) * C] = dc_final<kApply>(s, scale, o + int64_t(rr) * C);
                 }
             }
         }
@@ -699,12 +697,18 @@ __global__ void __launch_bounds__(256) ps_decode_kernel(
 
 // PowerSGD layers of the decode; false: W too large, use the element-wise path
 bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_rank, const float* P,
-                           const float* Q, float scale, float* out, cudaStream_t st) {
+                           const float* Q, float scale, float* out, bool apply, cudaStream_t st) {
     if (W > kDcLrMaxW) return false;
-    if (t->ps1_ntiles > 0)
-        GCE_LAUNCH(ps_decode_kernel, grid_of(t->ps1_ntiles, 4), 256, 0, st, t->d_layers,
-                   t->d_ps1_tiles, t->ps1_ntiles, W, t->P_pw, t->Q_pw, k_or_rank, P, Q, scale,
-                   out);
+    static const int r_dec = resident_blocks(ps_decode_kernel<false>, 256);
+    static const int r_dec_apply = resident_blocks(ps_decode_kernel<true>, 256);
+    if (t->ps1_ntiles > 0 && !apply)
+        GCE_LAUNCH(ps_decode_kernel<false>, wave_grid(t->ps1_ntiles, 4, r_dec), 256, 0, st,
+                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->P_pw, t->Q_pw, k_or_rank, P,
+                   Q, scale, out);
+    if (t->ps1_ntiles > 0 && apply)
+        GCE_LAUNCH(ps_decode_kernel<true>, wave_grid(t->ps1_ntiles, 4, r_dec_apply), 256, 0, st,
+                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->P_pw, t->Q_pw, k_or_rank, P,
+                   Q, scale, out);
     return true;
 }
 
@@ -718,7 +722,8 @@ extern "C" int powersgd_init_q(const gce_table* t, int32_t W, uint64_t seed, flo
     if (t->nps == 0) return GCE_OK;
     if (!Q || !aligned16(Q)) return GCE_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    GCE_LAUNCH(ps_init_q_kernel, grid_of(int64_t(t->nps) * W, 4), 256, 0, st, t->d_layers,
+    static const int r_init = resident_blocks(ps_init_q_kernel, 256);
+    GCE_LAUNCH(ps_init_q_kernel, wave_grid(int64_t(t->nps) * W, 4, r_init), 256, 0, st, t->d_layers,
                t->d_ps_layers, t->nps, W, t->Q_pw, seed, Q);
     return check_launch();
 }
@@ -741,28 +746,34 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         double* pd = at<double>(ws, lay.pd);
         float* qpart = at<float>(ws, lay.qpart);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        GCE_LAUNCH(ps_mq_kernel, grid_of(int64_t(t->ps1_ntiles) * W, 8), 256, 0, st, t->d_layers,
+        static const int r_mq = resident_blocks(ps_mq_kernel, 256);
+        static const int r_orth = resident_blocks(ps_orth_kernel, 256);
+        static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
+        static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
+        static const int r_qred = resident_blocks(ps_qred_kernel, 256);
+        static const int r_resid = resident_blocks(ps_resid_kernel, 256);
+        GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st, t->d_layers,
                    ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw, t->ppart_pw, grad, mem,
                    eta, k_or_rank, Q, ppart);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
-        GCE_LAUNCH(ps_orth_kernel, grid_of(int64_t(t->nps) * W, 8), 256, 0, st, t->d_layers, ps,
+        GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
                    pd, P, status, t->ps_ntall, tdone);
         if (t->ps_ntall > 0) {
             for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
-                GCE_LAUNCH(ps_orth_tall_kernel, grid_of(int64_t(t->ps_tall_nunits) * W, 8), 256, 0,
+                GCE_LAUNCH(ps_orth_tall_kernel, wave_grid(int64_t(t->ps_tall_nunits) * W, 8, r_tall), 256, 0,
                            st, op, t->d_layers, ps, t->d_ps_tall_units, t->ps_tall_nunits, W,
                            t->P_pw, t->ppart_pw, t->pd_pw, t->ps_ntall, t->ps_tall_parts,
                            k_or_rank, ppart, pd, at<double>(ws, lay.tparts),
                            at<double>(ws, lay.tscal), tdone, P);
         }
-        GCE_LAUNCH(ps_mtp_kernel, grid_of(int64_t(t->ps3_ntiles) * W, 8), 256, 0, st,
+        GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
                    t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->P_pw, t->qpart_pw,
                    mem, k_or_rank, P, qpart);
-        GCE_LAUNCH(ps_qred_kernel, grid_of(int64_t(t->psq_ntiles) * W, 8), 256, 0, st,
+        GCE_LAUNCH(ps_qred_kernel, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0, st,
                    t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
                    k_or_rank, qpart, Q);
-        GCE_LAUNCH(ps_resid_kernel, grid_of(int64_t(t->ps1_ntiles) * W, 8), 256, 0, st,
+        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
                    t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
                    k_or_rank, P, Q, mem, dense_out);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;

@@ -434,19 +434,6 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
     }
 }
 
-template <class K>
-static int occupancy_of(K kernel, int threads) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1)
-        n = 1;
-    return n;
-}
-
-static int grid_cap(int64_t work, int per_sm) {
-    const int64_t cap = int64_t(sm_count()) * per_sm;
-    return int(max64(1, min64(work, cap)));
-}
-
 }  // namespace gce
 
 using namespace gce;
@@ -470,24 +457,30 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
         int32_t* tile_cnt = at<int32_t>(ws, lay.tile_cnt);
         uint32_t* bitmask = at<uint32_t>(ws, lay.bitmask);
         RkEntry* cand = at<RkEntry>(ws, lay.cand);
-        static int occ_emit = occupancy_of(rk_emit_kernel, kTkThreads);
-        GCE_LAUNCH(rk_setup_kernel, grid_cap((lay.S + 255) / 256, 4), 256, 0, st, t->d_layers,
+        static const int r_setup = resident_blocks(rk_setup_kernel, 256);
+        static const int r_keys0 = resident_blocks(rk_keys_kernel<false>, 256);
+        static const int r_keys1 = resident_blocks(rk_keys_kernel<true>, 256);
+        static const int r_res0 = resident_blocks(rk_resolve_kernel<false>, 1024);
+        static const int r_res1 = resident_blocks(rk_resolve_kernel<true>, 1024);
+        static const int r_scan = resident_blocks(rk_scan_kernel, 1024);
+        static const int r_emit = resident_blocks(rk_emit_kernel, kTkThreads);
+        GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, k_or_rank, seed, step, bracket_sigma(), segs, status);
-        GCE_LAUNCH(rk_keys_kernel<false>, grid_cap(lay.TT, 8), 256, 0, st, t->d_layers,
+        GCE_LAUNCH(rk_keys_kernel<false>, wave_grid(lay.TT, 8, r_keys0), 256, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs, tile_cnt, bitmask,
                    cand);
-        GCE_LAUNCH(rk_resolve_kernel<false>, grid_cap(lay.S, 2), 1024, 0, st, t->d_layers,
+        GCE_LAUNCH(rk_resolve_kernel<false>, wave_grid(lay.S, 2, r_res0), 1024, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, bitmask, cand,
                    status);
-        GCE_LAUNCH(rk_keys_kernel<true>, grid_cap(lay.TT, 8), 256, 0, st, t->d_layers,
+        GCE_LAUNCH(rk_keys_kernel<true>, wave_grid(lay.TT, 8, r_keys1), 256, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs, tile_cnt, bitmask,
                    cand);
-        GCE_LAUNCH(rk_resolve_kernel<true>, grid_cap(lay.S, 2), 1024, 0, st, t->d_layers,
+        GCE_LAUNCH(rk_resolve_kernel<true>, wave_grid(lay.S, 2, r_res1), 1024, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, bitmask, cand,
                    status);
-        GCE_LAUNCH(rk_scan_kernel, grid_cap(lay.S, 2), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
+        GCE_LAUNCH(rk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
                    lay.S, t->tiles_pw, segs, tile_cnt);
-        GCE_LAUNCH(rk_emit_kernel, grid_cap(lay.TT, occ_emit), kTkThreads, 0, st, t->d_layers,
+        GCE_LAUNCH(rk_emit_kernel, wave_grid(lay.TT, r_emit, r_emit), kTkThreads, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw, grad, mem, eta, segs,
                    tile_cnt, bitmask, vals, idx);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;

@@ -102,7 +102,8 @@ int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float*
     if (t->dtiles_pw == 0) return GCE_OK;
     if (!vals) return GCE_ERR_ARG;
     int64_t total = int64_t(t->dtiles_pw) * W;
-    int grid = int(min64(total, int64_t(sm_count()) * 8));
+    static const int r_dense = resident_blocks(dense_kernel, 256);
+    const int grid = wave_grid(total, 8, r_dense);
     GCE_LAUNCH(dense_kernel, grid, 256, 0, st, t->d_layers, t->d_dtile_layer, t->d_dtile_start,
                t->dtiles_pw, W, t->N, t->vals_pw, grad, mem, eta, vals);
     return check_launch();
@@ -204,12 +205,10 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
                 x.ntiles = int32_t((n + kTkTile - 1) / kTkTile);
                 for (int32_t i = 0; i < x.ntiles; ++i) tile_layer.push_back(l);
                 tiles += x.ntiles;
-                if (n >= kTkSampleMinN) {
-                    int32_t parts = int32_t((n + kTkSamplePart - 1) / kTkSamplePart);
-                    for (int32_t p = 0; p < parts; ++p) {
-                        sunit_layer.push_back(l);
-                        sunit_part.push_back(p);
-                    }
+                const int32_t parts = int32_t((n + kTkSamplePart - 1) / kTkSamplePart);
+                for (int32_t p = 0; p < parts; ++p) {
+                    sunit_layer.push_back(l);
+                    sunit_part.push_back(p);
                 }
             }
         }

@@ -10,7 +10,9 @@
 //   sample   read one 128-byte run of grad/mem per 2048 elements, histogram
 //            the |v| keys and, interpolating inside the crossing bins, pick
 //            two bounds with a wide statistical margin: lo (the k-th largest
-//            key lies above it) and hi (almost surely chosen above it)
+//            key lies above it) and hi (almost surely chosen above it);
+//            layers under 65536 elements are histogrammed whole and get
+//            exact bounds (the edges of the bin holding the k-th key)
 //   main     the only full pass over HBM: v = fl(m + fl(eta*g)); memory <- v,
 //            or +0 when key > hi; every element with key >= lo is appended, in
 //            index order within its 8192-element tile, to the layer's
@@ -101,8 +103,8 @@ __global__ void __launch_bounds__(256) tk_setup_kernel(const DevLayer* __restric
             g.k = 0;
             set_status(status, GCE_STATUS_K_RANGE);
         }
-        g.lo = 0;            // layers too small to sample list every element
-        g.hi = 0xFFFFFFFFu;  // and zero nothing in the main pass
+        g.lo = 0;            // until the sample pass sets them: list every
+        g.hi = 0xFFFFFFFFu;  // element and zero nothing in the main pass
         segs[s] = g;
     }
 }
@@ -151,10 +153,13 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
         if (k == 0) continue;
         for (int b = tid; b < kTkSBins; b += blockDim.x) h[b] = 0;
         __syncthreads();
+        // a layer below kTkSampleMinN elements is histogrammed whole: its
+        // bounds come from exact counts
+        const bool exact = L.n < kTkSampleMinN;
         const int64_t p0 = int64_t(sunit_part[su]) * kTkSamplePart;
         const int64_t pend = min64(L.n, p0 + kTkSamplePart);
         const int64_t nch = (pend - p0 + kTkSampleStride - 1) / kTkSampleStride;
-        const int64_t ne = nch * kTkSampleChunk;
+        const int64_t ne = exact ? L.n : nch * kTkSampleChunk;
         const float* g = grad + int64_t(w) * N + L.offset;
         const float* m = mem + int64_t(w) * N + L.offset;
         for (int64_t e0 = 0; e0 < ne; e0 += int64_t(kBatch) * blockDim.x) {
@@ -163,7 +168,8 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
                 const int64_t e = e0 + int64_t(q) * blockDim.x + tid;
-                const int64_t pos = p0 + (e / kTkSampleChunk) * kTkSampleStride + (e % kTkSampleChunk);
+                const int64_t pos =
+                    exact ? e : p0 + (e / kTkSampleChunk) * kTkSampleStride + (e % kTkSampleChunk);
                 ok[q] = e < ne && pos < L.n;
                 vv[q] = ok[q] ? residual(m[pos], eta, __ldcs(g + pos)) : 0.0f;
             }
@@ -186,7 +192,17 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
             __threadfence();
             for (int b = tid; b < kTkSBins; b += blockDim.x) h[b] = __ldcg(gh + b);
             __syncthreads();
-            if (tid < 32) {
+            if (tid < 32 && exact) {
+                // b: the bin where the count from the top reaches k.  Fewer
+                // than k keys lie above it (all chosen), at least k at or
+                // above its bottom edge.
+                int64_t above = 0;
+                const int b = warp_find_from_top(h, kTkSBins, k, &above);
+                if (tid == 0 && b >= 0) {
+                    segs[seg].lo = uint32_t(b) << 19;
+                    segs[seg].hi = ((uint32_t(b) + 1u) << 19) - 1u;
+                }
+            } else if (tid < 32) {
                 const int64_t ns = tk_samples_in(L.n);
                 const double mu = double(k) * double(ns) / double(L.n);
                 const double margin = sigma * (sqrt(mu) + 1.0);
@@ -674,18 +690,6 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
 }
 
 // ---- host ------------------------------------------------------------------------------------
-template <class K>
-static int occupancy(K kernel, int threads) {
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1)
-        n = 1;
-    return n;
-}
-
-static int grid_for(int64_t work, int per_sm) {
-    const int64_t cap = int64_t(sm_count()) * per_sm;
-    return int(max64(1, min64(work, cap)));
-}
 
 }  // namespace gce
 
@@ -722,39 +726,48 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         int32_t* spill_i = at<int32_t>(ws, lay.spill_i);
         const int64_t n4 = lay.S * (kTkSBins + 3 * kTkBins) / 4;
 
-        GCE_LAUNCH(tk_setup_kernel, grid_for((n4 + lay.S + 255) / 256, 8), 256, 0, st, t->d_layers,
+        static const int r_setup = resident_blocks(tk_setup_kernel, 256);
+        static const int r_sample = resident_blocks(tk_sample_kernel, 256);
+        static const int r_main = resident_blocks(tk_main_kernel, kTkThreads);
+        static const int r_restore = resident_blocks(tk_restore_kernel, 256);
+        static const int r_respill = resident_blocks(tk_respill_kernel, 256);
+        static const int r_h1 = resident_blocks(tk_hist_kernel<1>, 256);
+        static const int r_h2 = resident_blocks(tk_hist_kernel<2>, 256);
+        static const int r_h3 = resident_blocks(tk_hist_kernel<3>, 256);
+        static const int r_count = resident_blocks(tk_count_kernel, 256);
+        static const int r_scan = resident_blocks(tk_scan_kernel, 1024);
+        static const int r_emit = resident_blocks(tk_emit_kernel, 256);
+        GCE_LAUNCH(tk_setup_kernel, wave_grid((n4 + lay.S + 255) / 256, 8, r_setup), 256, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, k_or_rank, segs, reinterpret_cast<int4*>(hists), n4,
                    status);
         if (t->sunits_pw > 0)
-            GCE_LAUNCH(tk_sample_kernel, grid_for(int64_t(t->sunits_pw) * W, 8), 256, 0, st,
+            GCE_LAUNCH(tk_sample_kernel, wave_grid(int64_t(t->sunits_pw) * W, 8, r_sample), 256, 0, st,
                        t->d_layers, t->d_sunit_layer, t->d_sunit_part, t->sunits_pw, W, ncomp,
                        lay.S, t->N, grad, mem, eta, segs, hists, g_bracket_sigma);
-        static int occ_main = occupancy(tk_main_kernel, kTkThreads);
-        GCE_LAUNCH(tk_main_kernel, grid_for(lay.TT, occ_main), kTkThreads, 0, st, t->d_layers,
+        GCE_LAUNCH(tk_main_kernel, wave_grid(lay.TT, r_main, r_main), kTkThreads, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->comp_N, grad, mem, eta, segs,
                    tile_dir, spill_v, spill_i);
         GCE_LAUNCH(tk_units_kernel, 1, 1024, 0, st, t->d_layers, t->d_comp, ncomp, t->tiles_pw,
                    segs, lay.S, unit_start, redo_list, status);
-        const int rgrid = grid_for(lay.TT, 4);
-        GCE_LAUNCH(tk_restore_kernel, rgrid, 256, 0, st, t->d_layers, t->d_tile_layer,
+        GCE_LAUNCH(tk_restore_kernel, wave_grid(lay.TT, 4, r_restore), 256, 0, st, t->d_layers, t->d_tile_layer,
                    t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, spill_v,
                    spill_i, mem);
-        GCE_LAUNCH(tk_respill_kernel, rgrid, 256, 0, st, t->d_layers, t->d_tile_layer,
+        GCE_LAUNCH(tk_respill_kernel, wave_grid(lay.TT, 4, r_respill), 256, 0, st, t->d_layers, t->d_tile_layer,
                    t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, mem, spill_v,
                    spill_i);
-        const int hgrid = grid_for(lay.TT + lay.S, 8);
-        GCE_LAUNCH(tk_hist_kernel<1>, hgrid, 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
+        const int64_t hwork = lay.TT + lay.S;
+        GCE_LAUNCH(tk_hist_kernel<1>, wave_grid(hwork, 8, r_h1), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
                    t->comp_N, segs, unit_start, hists, spill_v);
-        GCE_LAUNCH(tk_hist_kernel<2>, hgrid, 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
+        GCE_LAUNCH(tk_hist_kernel<2>, wave_grid(hwork, 8, r_h2), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
                    t->comp_N, segs, unit_start, hists, spill_v);
-        GCE_LAUNCH(tk_hist_kernel<3>, hgrid, 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
+        GCE_LAUNCH(tk_hist_kernel<3>, wave_grid(hwork, 8, r_h3), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
                    t->comp_N, segs, unit_start, hists, spill_v);
-        const int wgrid = grid_for((lay.TT + 7) / 8, 8);
-        GCE_LAUNCH(tk_count_kernel, wgrid, 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw,
+        const int64_t wwork = (lay.TT + 7) / 8;  // a warp per tile
+        GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw,
                    W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
-        GCE_LAUNCH(tk_scan_kernel, grid_for(lay.S, 2), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
+        GCE_LAUNCH(tk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
                    lay.S, t->tiles_pw, segs, tile_cnt);
-        GCE_LAUNCH(tk_emit_kernel, wgrid, 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw, W,
+        GCE_LAUNCH(tk_emit_kernel, wave_grid(wwork, 8, r_emit), 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw, W,
                    ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt, spill_v, spill_i,
                    mem, vals, idx);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;

@@ -13,7 +13,7 @@ constexpr int kTkSBins = 4096;                     // sample bins: 2^19 keys, 16
 constexpr int kTkSampleChunk = 32;                 // sampled run length (one 128-B line)
 constexpr int kTkSampleStride = 2048;              // one run per 2048 elements
 constexpr int64_t kTkSamplePart = int64_t(1) << 20; // elements covered by one sample unit
-constexpr int64_t kTkSampleMinN = 65536;           // smaller layers list every element
+constexpr int64_t kTkSampleMinN = 65536;           // smaller layers: exact histogram of all
 constexpr int kTkHUnit = 32768;                    // candidates per histogram unit
 
 // Per (worker, layer) state of one top-k step.

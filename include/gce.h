@@ -233,6 +233,29 @@ GCE_API int decompress_accumulate(const gce_table* table, int32_t W, const float
                           void* stream);
 
 /*
+ * Aggregate fused with the parameter update of [MEM] Method (x_{t+1} = x_t -
+ * g_t, the workers' compressed updates summed): with S the worker-order sum
+ * that decompress_accumulate forms,
+ *   x[j] = fl(x[j] - fl(scale * S[j]))   for every j in [0, N),
+ * bit for bit what decompress_accumulate into a scratch buffer followed by
+ * x -= scratch would give, without the scratch buffer's write and read.
+ * x: device fp32 [N], 16-byte aligned, read and written in place.  Other
+ * arguments, preconditions, workspace and errors as decompress_accumulate.
+ */
+GCE_API int decompress_apply(const gce_table* table, int32_t W, const float* vals,
+                             const int32_t* idx, const int32_t* k_or_rank, const float* P,
+                             const float* Q, float scale, float* x, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/*
+ * The step size of [MEM] Method for step t: eta_t = 8 / (mu (a + t)),
+ * computed in double and rounded once to float into *eta (host memory).
+ * GCE_ERR_ARG if eta is NULL, t < 0, mu <= 0, a + t <= 0 or the value
+ * overflows float.
+ */
+GCE_API int gce_memsgd_eta(int64_t step, double mu, double a, float* eta);
+
+/*
  * decompress_accumulate without a workspace (the pages have no counterpart:
  * this is a deployment variant, not part of the method).  For callers that
  * cannot allocate device memory for a workspace -- code running inside

@@ -176,3 +176,18 @@ def decompress(layers, W, payload, scale_factor, rank_per_layer=None, k_per_laye
                 accum_sparse(view, vals[:k], idx[:k])
     scale(out, scale_factor)
     return out
+
+
+def apply_update(layers, W, payload, scale_factor, x, rank_per_layer=None, k_per_layer=None):
+    """Parameter update of "Sparsified SGD with Memory", Method: x_{t+1} =
+    x_t - g_t, with the W workers' updates combined as `decompress` combines
+    them: x - fl(scale * S), one fp32 round-to-nearest subtraction per
+    element.  Returns the new x (float32)."""
+    u = decompress(layers, W, payload, scale_factor, rank_per_layer, k_per_layer)
+    return np.subtract(np.asarray(x, np.float32), u, dtype=np.float32)
+
+
+def memsgd_eta(t, mu, a):
+    """Step size eta_t = 8 / (mu (a + t)) of "Sparsified SGD with Memory",
+    Method, in fp64, rounded once to fp32."""
+    return np.float32(8.0 / (float(mu) * (float(a) + float(t))))

@@ -5,6 +5,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 
 from tests.conftest import ROOT
@@ -56,6 +57,13 @@ def test_null_arguments_are_rejected_on_the_host():
     assert L.decompress_accumulate(None, 1, None, None, None, None, None, 1.0, None, None, 0,
                                    None) == -1
     assert L.gce_set_bracket_sigma(C.c_double(float("nan"))) == -1
+    assert L.decompress_apply(None, 1, None, None, None, None, None, 1.0, None, None, 0,
+                              None) == -1
+    e = C.c_float()
+    assert L.gce_memsgd_eta(0, 0.0, 1.0, C.byref(e)) == -1        # mu <= 0
+    assert L.gce_memsgd_eta(3, 1.0, -3.0, C.byref(e)) == -1       # a + t <= 0
+    assert L.gce_memsgd_eta(-1, 1.0, 5.0, C.byref(e)) == -1       # t < 0
+    assert L.gce_memsgd_eta(0, 1.0, 1.0, None) == -1
     assert L.gce_error_string(-3) == b"workspace missing or too small"
 
 
@@ -75,3 +83,11 @@ def test_missing_library_fails_loudly(tmp_path, monkeypatch):
     monkeypatch.setattr(gce, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError):
         gce.lib()
+
+
+def test_memsgd_eta_matches_the_oracle():
+    """The step-size helper is host code: checked here against the oracle."""
+    import gradient_compression_error_b200 as gce
+    from oracle import steps
+    for t, mu, a in [(0, 1.0, 8.0), (7, 0.01, 1000.0), (123456, 3.5, 0.25), (1, 1e-3, 1.0)]:
+        assert np.float32(gce.memsgd_eta(t, mu, a)) == steps.memsgd_eta(t, mu, a)
