@@ -35,6 +35,8 @@ def lib():
             "or_dense": (C.c_int, [i64, f32, vp, vp, vp]),
             "or_powersgd_init_q": (C.c_int, [i64, i64, u64, u64, u64, vp]),
             "or_powersgd": (C.c_int, [i64, i64, i64, i64, f32, vp, vp, vp, vp, vp]),
+            "or_powersgd_dp": (C.c_int, [i64, i64, i64, i64, i64, f32, vp, vp, vp, vp]),
+            "or_dense_dp": (C.c_int, [i64, i64, f32, vp, vp, vp]),
             "or_layer_norm": (f64, [i64, vp]),
             "or_accordion_decide": (i32, [f64, f64, f64]),
             "or_accum_sparse": (None, [i64, vp, vp, vp]),
@@ -140,6 +142,35 @@ def powersgd_unit(g, m, Q, r, eta, want_mhat=True):
                              _ptr(m), _ptr(Q), _ptr(P),
                              _ptr(Mhat) if want_mhat else None), "powersgd")
     return P, Q, m, Mhat
+
+
+def powersgd_dp_unit(g, m, Q, r, eta):
+    """Data-parallel PowerSGD step on one matrix over W workers.
+
+    g, m: (W, rows, cols) float32; Q: (cols, r_max) shared warm start.
+    Returns (P (rows, r_max), Q_new (cols, r_max), m_new (W, rows, cols));
+    columns >= r of P are zero and of Q_new are copied from Q.
+    """
+    g = _f32(g)
+    W, rows, cols = g.shape
+    m = _f32(m).copy()
+    Q = _f32(Q).copy()
+    r_max = Q.shape[1]
+    P = np.zeros((rows, r_max), np.float32)
+    _check(lib().or_powersgd_dp(W, rows, cols, int(r), r_max, float(np.float32(eta)), _ptr(g),
+                                _ptr(m), _ptr(Q), _ptr(P)), "powersgd_dp")
+    return P, Q, m
+
+
+def dense_dp_unit(g, m, eta):
+    """Data-parallel DENSE layer: g, m (W, n).  Returns (mean payload, m_new)."""
+    g = _f32(g)
+    W, n = g.shape
+    m = _f32(m).copy()
+    out = np.empty(n, np.float32)
+    _check(lib().or_dense_dp(W, n, float(np.float32(eta)), _ptr(g), _ptr(m), _ptr(out)),
+           "dense_dp")
+    return out, m
 
 
 def layer_norm(g):

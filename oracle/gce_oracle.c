@@ -51,6 +51,11 @@
  *     missing previous norm (prev < 0) means "critical", rel change >= the
  *     threshold means "critical" (level LOW = l_low), else HIGH = l_high;
  *   - k from a fraction in parts per million: k = max(1, floor(n*ppm/1e6)).
+ *   - data-parallel PowerSGD (or_powersgd_dp): the all-reduces are sums over
+ *     the workers -- P = sum_w M_w Q before orthonormalising, Q = the mean of
+ *     the workers' Q_w = M_w^T P -- and each worker keeps its own error
+ *     m_w = M_w - P Q_w^T; a DENSE layer sends the workers' mean residual
+ *     (fp32 sum in worker order, then times fl32(1/W)).
  *
  * Parity unpinned (nothing on the pages fixes it):
  *   or_randk_base / the stream composition of the rand-k and Q-init hashes
@@ -323,6 +328,112 @@ int or_powersgd(int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
     free(M);
     free(Pd);
     free(Qd);
+    return OR_OK;
+}
+
+/*
+ * Data-parallel PowerSGD step for one matrix over W workers ([UTIL] Key
+ * results: PowerSGD is all-reduce compatible; the all-reduces are sums over
+ * the workers).  Every worker shares the warm start Q and the orthonormal P:
+ *   M_w = fl32(m_w + fl32(eta*g_w))                 (the Mem-SGD residual)
+ *   P   = sum_w M_w Q                               (all-reduce of P)
+ *   P  <- modified Gram-Schmidt in column order
+ *   Q_w = M_w^T P;  m_w <- M_w - P Q_w^T            (each worker's own error)
+ *   Q   = (1/W) sum_w Q_w                           (all-reduce mean of Q)
+ * so that P Q^T is the mean of the workers' decompressed updates.
+ *   g, m   W x rows x cols fp32 (worker-major); m overwritten
+ *   Q      cols x r_max shared warm start; columns 0..r-1 overwritten
+ *   P      rows x r_max; columns 0..r-1 receive the orthonormal P
+ * Arithmetic after the M_w are formed runs in double; P, Q and m are stored
+ * as fp32.
+ */
+int or_powersgd_dp(int64_t W, int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
+                   const float* g, float* m, float* Q, float* P)
+{
+    if (W < 1 || rows < 1 || cols < 1 || r < 1 || r > r_max || r > rows || r > cols)
+        return OR_ERR_ARG;
+    int64_t n = rows * cols;
+    double* M = (double*)malloc((size_t)(W * n) * sizeof(double));
+    double* Pd = (double*)calloc((size_t)(rows * r), sizeof(double));
+    double* Qw = (double*)malloc((size_t)(cols * r) * sizeof(double));
+    double* Qsum = (double*)calloc((size_t)(cols * r), sizeof(double));
+    if (!M || !Pd || !Qw || !Qsum) { free(M); free(Pd); free(Qw); free(Qsum); return OR_ERR_NOMEM; }
+
+    for (int64_t w = 0; w < W; ++w)
+        for (int64_t i = 0; i < n; ++i)
+            M[w * n + i] = (double)or_residual(m[w * n + i], eta, g[w * n + i]);
+
+    /* P = sum over workers of M_w Q */
+    for (int64_t w = 0; w < W; ++w)
+        for (int64_t a = 0; a < rows; ++a)
+            for (int64_t j = 0; j < r; ++j) {
+                double s = 0.0;
+                for (int64_t c = 0; c < cols; ++c)
+                    s += M[w * n + a * cols + c] * (double)Q[c * r_max + j];
+                Pd[a * r + j] += s;
+            }
+
+    /* modified Gram-Schmidt over the columns of P, in order 0..r-1 */
+    for (int64_t j = 0; j < r; ++j) {
+        for (int64_t i = 0; i < j; ++i) {
+            double d = 0.0;
+            for (int64_t a = 0; a < rows; ++a) d += Pd[a * r + i] * Pd[a * r + j];
+            for (int64_t a = 0; a < rows; ++a) Pd[a * r + j] -= d * Pd[a * r + i];
+        }
+        double nn = 0.0;
+        for (int64_t a = 0; a < rows; ++a) nn += Pd[a * r + j] * Pd[a * r + j];
+        double nu = sqrt(nn);
+        for (int64_t a = 0; a < rows; ++a) Pd[a * r + j] = nu > 0.0 ? Pd[a * r + j] / nu : 0.0;
+    }
+
+    /* each worker: Q_w = M_w^T P, its residual, and the running sum of Q_w */
+    for (int64_t w = 0; w < W; ++w) {
+        const double* Mw = M + w * n;
+        for (int64_t c = 0; c < cols; ++c)
+            for (int64_t j = 0; j < r; ++j) {
+                double s = 0.0;
+                for (int64_t a = 0; a < rows; ++a) s += Mw[a * cols + c] * Pd[a * r + j];
+                Qw[c * r + j] = s;
+                Qsum[c * r + j] += s;
+            }
+        for (int64_t a = 0; a < rows; ++a)
+            for (int64_t c = 0; c < cols; ++c) {
+                double s = 0.0;
+                for (int64_t j = 0; j < r; ++j) s += Pd[a * r + j] * Qw[c * r + j];
+                m[w * n + a * cols + c] = (float)(Mw[a * cols + c] - s);
+            }
+    }
+
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t j = 0; j < r; ++j) P[a * r_max + j] = (float)Pd[a * r + j];
+    for (int64_t c = 0; c < cols; ++c)
+        for (int64_t j = 0; j < r; ++j) Q[c * r_max + j] = (float)(Qsum[c * r + j] / (double)W);
+
+    free(M);
+    free(Pd);
+    free(Qw);
+    free(Qsum);
+    return OR_OK;
+}
+
+/*
+ * Data-parallel uncompressed (DENSE) layer: the all-reduce mean of the
+ * workers' residuals, payload = fl32(fl32(sum_w v_w) * fl32(1/W)) with the
+ * sum in worker order from +0.0; every worker's memory becomes +0.0.
+ *   g, m  W x n (worker-major); out n.
+ */
+int or_dense_dp(int64_t W, int64_t n, float eta, const float* g, float* m, float* out)
+{
+    if (W < 1 || n < 0) return OR_ERR_ARG;
+    float inv = 1.0f / (float)W;
+    for (int64_t i = 0; i < n; ++i) {
+        float s = 0.0f;
+        for (int64_t w = 0; w < W; ++w) {
+            s = s + or_residual(m[w * n + i], eta, g[w * n + i]);
+            m[w * n + i] = 0.0f;
+        }
+        out[i] = s * inv;
+    }
     return OR_OK;
 }
 

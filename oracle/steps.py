@@ -11,8 +11,8 @@ from concurrent.futures import ThreadPoolExecutor
 import numpy as np
 
 from . import (accordion_decide, accum_dense, accum_lowrank, accum_sparse,
-               dense_unit, ef_randk_unit, ef_topk_unit, k_from_ppm, layer_norm,
-               powersgd_init_q, powersgd_unit, scale)
+               dense_dp_unit, dense_unit, ef_randk_unit, ef_topk_unit, k_from_ppm, layer_norm,
+               powersgd_dp_unit, powersgd_init_q, powersgd_unit, scale)
 
 
 def layer_offsets(layers):
@@ -109,6 +109,43 @@ def powersgd_step(layers, grad, mem, eta, rank_per_layer, Qs, units=None, thread
         else:
             Qs[u] = Qn
             out[u] = (a, Mhat)
+    return out
+
+
+def powersgd_dp_step(layers, grad, mem, eta, rank_per_layer, Qs, units=None, threads=1):
+    """Data-parallel PowerSGD step over all W workers of grad / mem (W, N):
+    P summed over the workers, one orthonormal P, each worker's own Q_w and
+    residual, Q the workers' mean ("On the Utility of Gradient Compression",
+    Key results: PowerSGD is all-reduce compatible).  Qs {l: Q} (shared per
+    layer) is updated in place; mem is updated in place.
+
+    Returns {l: P} for PowerSGD layers and {l: mean payload} for dense ones.
+    units: the layer ids to run (default all).
+    """
+    offs, N = layer_offsets(layers)
+    W = grad.shape[0]
+    if units is None:
+        units = list(range(len(layers)))
+
+    def one(l):
+        lay = layers[l]
+        rows, cols = lay["rows"], lay["cols"]
+        sl = slice(offs[l], offs[l] + rows * cols)
+        if lay["kind"] == "dense":
+            pay, m_new = dense_dp_unit(grad[:, sl], mem[:, sl], eta)
+            return l, pay, None, m_new
+        P, Qn, m_new = powersgd_dp_unit(grad[:, sl].reshape(W, rows, cols),
+                                        mem[:, sl].reshape(W, rows, cols), Qs[l],
+                                        int(rank_per_layer[l]), eta)
+        return l, P, Qn, m_new.reshape(W, -1)
+
+    out = {}
+    for l, a, Qn, m_new in _run(units, one, threads):
+        lay = layers[l]
+        mem[:, offs[l]:offs[l] + lay["rows"] * lay["cols"]] = m_new
+        if Qn is not None:
+            Qs[l] = Qn
+        out[l] = a
     return out
 
 
