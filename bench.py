@@ -56,6 +56,8 @@ def workload_spec(name):
         return dict(layers=wl.memsgd_vector(), W=1, cfg=1, method="topk")
     if name == "resnet18_powersgd_r2":
         return dict(layers=wl.resnet18_powersgd(2), W=1, cfg=2, method="powersgd")
+    if name == "resnet18_powersgd_r2_w8_dp":     # data-parallel: shared P and Q over 8 workers
+        return dict(layers=wl.resnet18_powersgd(2), W=8, cfg=2, method="powersgd_dp")
     if name == "vgg19_accordion_powersgd":       # ranks 4 / 2 chosen by Accordion
         return dict(layers=wl.vgg19("powersgd", 4), W=1, cfg=3, method="powersgd",
                     accordion=(4, 2))
@@ -75,7 +77,8 @@ def workload_spec(name):
     raise SystemExit("unknown workload %s" % name)
 
 
-MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel"}
+MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel",
+                "powersgd_dp": "ps_mq_kernel"}
 
 
 def max_over_ranks_of(x, world, device):
@@ -181,20 +184,35 @@ def cpu_oracle_sample(spec, units, steps_seed):
         offs.append(o)
         o += l["rows"] * l["cols"]
     threads = os.cpu_count() or 1
+    dp = spec["method"] == "powersgd_dp"   # a unit is one layer of every worker
     data = {}
     for (w, l) in units:
         n = layers[l]["rows"] * layers[l]["cols"]
-        g = torch.Generator()
-        g.manual_seed(wl.seed_for(spec["cfg"], w, steps_seed) + l)
-        data[(w, l)] = (torch.randn(n, generator=g).numpy().astype(np.float32),
-                        np.zeros(n, np.float32))
+        gs = []
+        for ww in (range(spec["W"]) if dp else [w]):
+            g = torch.Generator()
+            g.manual_seed(wl.seed_for(spec["cfg"], ww, steps_seed) + l)
+            gs.append(torch.randn(n, generator=g).numpy().astype(np.float32))
+        data[(w, l)] = (np.stack(gs) if dp else gs[0],
+                        np.zeros((len(gs), n) if dp else n, np.float32))
 
     def one(u):
         w, l = u
         lay = layers[l]
         gg, mm = data[u]
-        out = np.zeros(gg.size, np.float32)
-        if lay["kind"] == "dense":
+        out = np.zeros(gg.shape[-1], np.float32)
+        if dp:
+            if lay["kind"] == "dense":
+                pay, m_new = oracle.dense_dp_unit(gg, mm, wl.ETA)
+                oracle.accum_dense(out, pay)
+            else:
+                rows, cols = lay["rows"], lay["cols"]
+                Q = oracle.powersgd_init_q(cols, lay["cap"], 1, 0, l)
+                P, Qn, m_new = oracle.powersgd_dp_unit(gg.reshape(-1, rows, cols),
+                                                       mm.reshape(-1, rows, cols), Q, lay["cap"],
+                                                       wl.ETA)
+                oracle.accum_lowrank(out, P, Qn, lay["cap"])
+        elif lay["kind"] == "dense":
             pay, m_new = oracle.dense_unit(gg, mm, wl.ETA)
             oracle.accum_dense(out, pay)
         elif spec["method"] == "powersgd":
@@ -229,8 +247,9 @@ def run_reference(args, rank, world):
     for s in range(args.warmup + args.steps):
         w = s % spec["W"]
         units, tot = [], 0
+        per_unit = spec["W"] if spec["method"] == "powersgd_dp" else 1
         for l in sorted(range(L), key=lambda l: -(spec["layers"][l]["rows"] * spec["layers"][l]["cols"])):
-            n = spec["layers"][l]["rows"] * spec["layers"][l]["cols"]
+            n = spec["layers"][l]["rows"] * spec["layers"][l]["cols"] * per_unit
             if tot + n <= 6_000_000 or not units:
                 units.append((w, l))
                 tot += n
@@ -249,8 +268,10 @@ def run_reference(args, rank, world):
             "data": "synthetic (seeded N(0,1) gradients)",
             "config": {"workload": args.workload, "W": spec["W"]},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": "per step: the largest tensors of one worker (rotating), "
-                                       "about 6 M elements, encode (top-k) + decode"},
+                             "sample": "per step: the largest tensors of one worker (rotating; "
+                                       "for the data-parallel PowerSGD workload, of every "
+                                       "worker), about 6 M elements, %s encode + decode"
+                                       % spec["method"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -304,6 +325,11 @@ def main():
         P = torch.zeros((W, max(4, table.P_per_worker)), dtype=torch.float32, device=dev)
         Q = torch.zeros((W, max(4, table.Q_per_worker)), dtype=torch.float32, device=dev)
         gce.powersgd_init_q(table, W, 1, Q)
+    if method == "powersgd_dp":      # one shared P, Q and dense payload for all workers
+        P = torch.zeros(max(4, table.P_per_worker), dtype=torch.float32, device=dev)
+        Q = torch.zeros(max(4, table.Q_per_worker), dtype=torch.float32, device=dev)
+        vals = torch.zeros(max(4, table.vals_per_worker), dtype=torch.float32, device=dev)
+        gce.powersgd_init_q(table, 1, 1, Q)
     kr = None
     if "accordion" in spec:   # Accordion picks each layer's k or rank every step
         L = len(layers)
@@ -330,6 +356,11 @@ def main():
             gce.ef_topk_step(table, W, grad, mem, eta, kr, vals, idx, ws)
         elif method == "randk":
             gce.ef_randk_step(table, W, grad, mem, eta, kr, 5, s, vals, idx, ws)
+        elif method == "powersgd_dp":
+            gce.powersgd_dp_step(table, W, grad, mem, eta, kr, P, Q, vals, ws)
+            # the shared payload is already the workers' mean: one decode
+            gce.decompress_accumulate(table, 1, vals, None, kr, P, Q, 1.0, out, ws_dc)
+            return
         else:
             gce.powersgd_step(table, W, grad, mem, eta, kr, P, Q, vals, None, ws)
         if apply:
@@ -396,7 +427,7 @@ def main():
                 "kernel_ms_per_step": main_ms_per_step if main_n else None}
     # whole-step algorithmic traffic: sparse W(12N + 8K) encode + 16 W K + 4N
     # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
-    if method == "powersgd":
+    if method in ("powersgd", "powersgd_dp"):
         step_bytes = W * 12.0 * N
     else:
         step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total

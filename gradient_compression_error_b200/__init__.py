@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgce.so")
 
 KIND = {"topk": 0, "randk": 1, "powersgd": 2, "dense": 3}
 KIND_NAME = {v: k for k, v in KIND.items()}
-OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4}
+OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4, "powersgd_dp": 5}
 STATUS_K_RANGE = 1
 STATUS_FALLBACK = 2
 LEVEL_LOW, LEVEL_HIGH = 0, 1
@@ -66,6 +66,8 @@ SIGNATURES = {
     "powersgd_init_q": (C.c_int, [_vp, _i32, _u64, _vp, _vp]),
     "powersgd_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
                                 C.c_size_t, _vp]),
+    "powersgd_dp_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
+                                   C.c_size_t, _vp]),
     "accordion_init": (C.c_int, [_vp, _vp, _vp, _vp]),
     "accordion_select": (C.c_int, [_vp, _vp, _i64, _i32, _f64, _i32, _i32, _vp, _vp, _vp, _vp,
                                    _vp, C.c_size_t, _vp]),
@@ -210,6 +212,15 @@ def powersgd_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, dense_out, ws
         table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
         _ptr(k_or_rank, _i32()), _ptr(P, _f32()), _ptr(Q, _f32()), _ptr(vals, _f32()),
         _ptr(dense_out, _f32()), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def powersgd_dp_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, ws, stream=None):
+    """Data-parallel PowerSGD over the W workers: shared P and Q (the mean),
+    per-worker memory (include/gce.h)."""
+    _check("powersgd_dp_step", lib().powersgd_dp_step(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), _ptr(P, _f32()), _ptr(Q, _f32()), _ptr(vals, _f32()),
+        _ptr(ws), ws.numel(), _stream(stream)))
 
 
 def accordion_init(table, prev_norm, level, stream=None):

@@ -199,6 +199,7 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 constexpr int kDcTileLog = 12;              // decode tile: 4096 output elements
 constexpr int kDcTile = 1 << kDcTileLog;
 constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
+constexpr int kDenseTile = 4096;            // elements per tile of a DENSE layer
 
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
                         float eta, float* vals, cudaStream_t st);

@@ -323,18 +323,23 @@ static int launch_decode_t(const gce_table* t, int32_t W, const float* vals, con
                    t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
                    k_or_rank, idx, bounds);
     }
-    if (t->nps > 0 && launch_lowrank_decode(t, W, k_or_rank, P, Q, scale, out, kApply, st)) {
-        // PowerSGD layers done by their own tiled kernel; the rest here
-        if (t->dc_nl_n > 0)
-            GCE_LAUNCH(dc_accum_kernel<kApply>, wave_grid(t->dc_nl_n, 16, r_accum), kDcThreads, 0,
-                       st, t->d_layers, t->d_dc_tile_layer, t->d_dc_nl_tiles, t->dc_nl_n, W,
-                       t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q,
-                       bounds, scale, out);
-        return check_launch();
+    // PowerSGD layers by their own tiled kernel when it takes them (then the
+    // element-wise kernel covers only the other layers' tiles)
+    const bool lowrank = t->nps > 0 &&
+                         launch_lowrank_decode(t, W, k_or_rank, P, Q, scale, out, kApply, st);
+    const int32_t ntiles = lowrank ? t->dc_nl_n : t->dc_tiles;
+    const int32_t* list = lowrank ? t->d_dc_nl_tiles : nullptr;
+    if (ntiles > 0) {
+        const int grid = wave_grid(ntiles, 16, r_accum);
+        if (kApply)
+            GCE_LAUNCH(dc_accum_kernel<true>, grid, kDcThreads, 0, st, t->d_layers,
+                       t->d_dc_tile_layer, list, ntiles, W, t->vals_pw, t->P_pw, t->Q_pw,
+                       t->dc_slots, k_or_rank, vals, idx, P, Q, bounds, scale, out);
+        else
+            GCE_LAUNCH(dc_accum_kernel<false>, grid, kDcThreads, 0, st, t->d_layers,
+                       t->d_dc_tile_layer, list, ntiles, W, t->vals_pw, t->P_pw, t->Q_pw,
+                       t->dc_slots, k_or_rank, vals, idx, P, Q, bounds, scale, out);
     }
-    GCE_LAUNCH(dc_accum_kernel<kApply>, wave_grid(t->dc_tiles, 16, r_accum), kDcThreads, 0, st,
-               t->d_layers, t->d_dc_tile_layer, nullptr, t->dc_tiles, W, t->vals_pw, t->P_pw,
-               t->Q_pw, t->dc_slots, k_or_rank, vals, idx, P, Q, bounds, scale, out);
     return check_launch();
 }
 

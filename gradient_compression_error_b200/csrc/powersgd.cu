@@ -129,7 +129,7 @@ void powersgd_plan_free(gce_table* t) {
 }
 
 struct PsWs {
-    size_t ppart = 0, pd = 0, qpart = 0, tparts = 0, tscal = 0, tdone = 0, total = 0;
+    size_t ppart = 0, pd = 0, qpart = 0, qloc = 0, tparts = 0, tscal = 0, tdone = 0, total = 0;
 };
 
 static PsWs ps_layout(const gce_table* t, int32_t W) {
@@ -146,6 +146,24 @@ static PsWs ps_layout(const gce_table* t, int32_t W) {
 }
 
 size_t powersgd_ws_bytes(const gce_table* t, int32_t W) { return ps_layout(t, W).total; }
+
+// The data-parallel step: partials per worker, one orthonormal P per layer,
+// and every worker's Q_w kept for its residual.
+static PsWs ps_dp_layout(const gce_table* t, int32_t W) {
+    PsWs o;
+    Carver c;
+    o.ppart = c.take<float>(int64_t(W) * t->ppart_pw);
+    o.pd = c.take<double>(t->pd_pw);
+    o.qpart = c.take<float>(int64_t(W) * t->qpart_pw);
+    o.qloc = c.take<float>(int64_t(W) * t->Q_pw);
+    o.tparts = c.take<double>(t->ps_tall_parts);
+    o.tscal = c.take<double>(t->ps_ntall);
+    o.tdone = c.take<int32_t>(t->ps_ntall);
+    o.total = c.off;
+    return o;
+}
+
+size_t powersgd_dp_ws_bytes(const gce_table* t, int32_t W) { return ps_dp_layout(t, W).total; }
 
 __device__ __forceinline__ int32_t ps_rank(const DevLayer& L, const int32_t* k_or_rank, int32_t l) {
     const int32_t r = k_or_rank ? k_or_rank[l] : L.cap;
@@ -257,9 +275,13 @@ __device__ __forceinline__ double block_sum_d(double x, double* s_red) {
     return t;
 }
 
+// W outputs (one P per output); output w sums the partial P of workers
+// w*nsum ... w*nsum + nsum - 1 in worker order (nsum = 1: independent
+// replicas; W = 1, nsum = all workers: the data-parallel step).
 __global__ void __launch_bounds__(256) ps_orth_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
-    const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W, int64_t P_pw, int64_t ppart_pw,
+    const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W, int32_t nsum, int64_t P_pw,
+    int64_t ppart_pw,
     int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ ppart,
     double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status,
     int32_t ntall, int32_t* __restrict__ tdone) {
@@ -280,13 +302,15 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         }
         const int cap = L.cap;
         const int64_t R = L.rows;
-        const float* pp = ppart + int64_t(w) * ppart_pw + X.ppart_off;
+        const float* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
         double* pd = pdw + int64_t(w) * pd_pw + X.pd_off;
         for (int64_t i = threadIdx.x; i < R * r; i += blockDim.x) {
             const int64_t row = i / r;
             const int j = int(i - row * r);
             double s = 0.0;
-            for (int ch = 0; ch < X.nch1; ++ch) s += double(pp[(int64_t(ch) * R + row) * cap + j]);
+            for (int ws = 0; ws < nsum; ++ws)
+                for (int ch = 0; ch < X.nch1; ++ch)
+                    s += double(pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j]);
             pd[row * cap + j] = s;
         }
         __syncthreads();
@@ -335,8 +359,9 @@ struct PsOrthOp {
 
 __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
     PsOrthOp op, const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
-    const int2* __restrict__ units, int32_t nunits, int32_t W, int64_t P_pw, int64_t ppart_pw,
-    int64_t pd_pw, int32_t ntall, int32_t nparts, const int32_t* __restrict__ k_or_rank,
+    const int2* __restrict__ units, int32_t nunits, int32_t W, int32_t nsum, int64_t P_pw,
+    int64_t ppart_pw, int64_t pd_pw, int32_t ntall, int32_t nparts,
+    const int32_t* __restrict__ k_or_rank,
     const float* __restrict__ ppart, double* __restrict__ pdw, double* __restrict__ tparts,
     double* __restrict__ tscal, int32_t* __restrict__ tdone, float* __restrict__ P) {
     __shared__ double s_red[8];
@@ -355,11 +380,13 @@ __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
         double* pd = pdw + int64_t(w) * pd_pw + X.pd_off;
         double* scal = tscal + int64_t(w) * ntall + X.tall;
         if (op.init) {
-            const float* pp = ppart + int64_t(w) * ppart_pw + X.ppart_off;
+            const float* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
             for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
                 for (int j = 0; j < r; ++j) {
                     double s = 0.0;
-                    for (int ch = 0; ch < X.nch1; ++ch) s += double(pp[(int64_t(ch) * R + row) * cap + j]);
+                    for (int ws = 0; ws < nsum; ++ws)
+                        for (int ch = 0; ch < X.nch1; ++ch)
+                            s += double(pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j]);
                     pd[row * cap + j] = s;
                 }
         }
@@ -499,12 +526,18 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
 }
 
 // ---- Q = sum of the row-block partials (fp64, block order) ----------------------------------
+// kMean (the data-parallel step): every worker's Q_w goes to Q (stride
+// Q_pw) and their mean -- fp32 sum in worker order from +0, times inv_w --
+// to qmean, one tile per block for all W workers.
+template <bool kMean>
 __global__ void __launch_bounds__(256) ps_qred_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t Q_pw, int64_t qpart_pw,
-    const int32_t* __restrict__ k_or_rank, const float* __restrict__ qpart, float* __restrict__ Q) {
-    for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
-        const int w = int(u / ntiles);
+    const int32_t* __restrict__ k_or_rank, const float* __restrict__ qpart, float* __restrict__ Q,
+    float* __restrict__ qmean, float inv_w) {
+    const int64_t nunits = kMean ? int64_t(ntiles) : int64_t(ntiles) * W;
+    for (int64_t u = blockIdx.x; u < nunits; u += gridDim.x) {
+        const int w = kMean ? 0 : int(u / ntiles);
         const int4 d = tiles[u % ntiles];
         const DevLayer L = layers[d.x];
         const PsLayer X = ps[d.x];
@@ -514,14 +547,42 @@ __global__ void __launch_bounds__(256) ps_qred_kernel(
         const int64_t C = L.cols;
         const int64_t c0 = int64_t(d.y) * kPsQB;
         const int cw = int(min64(kPsQB, C - c0));
-        const float* qp = qpart + int64_t(w) * qpart_pw + X.qpart_off;
-        float* q = Q + int64_t(w) * Q_pw + L.q_off;
         for (int i = threadIdx.x; i < cw * r; i += blockDim.x) {
             const int64_t c = c0 + i / r;
             const int j = i % r;
-            double s = 0.0;
-            for (int rb = 0; rb < X.nrb3; ++rb) s += double(qp[(int64_t(rb) * C + c) * cap + j]);
-            q[c * cap + j] = float(s);
+            float mean = 0.0f;
+            for (int wi = 0; wi < (kMean ? W : 1); ++wi) {
+                const int ww = kMean ? wi : w;
+                const float* qp = qpart + int64_t(ww) * qpart_pw + X.qpart_off;
+                double s = 0.0;
+                for (int rb = 0; rb < X.nrb3; ++rb) s += double(qp[(int64_t(rb) * C + c) * cap + j]);
+                const float qv = float(s);
+                Q[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = qv;
+                if (kMean) mean = __fadd_rn(mean, qv);
+            }
+            if (kMean) qmean[L.q_off + c * cap + j] = __fmul_rn(mean, inv_w);
+        }
+    }
+}
+
+// ---- data-parallel DENSE layers: payload = mean of the workers' residuals ------------------
+__global__ void __launch_bounds__(256) ps_dense_mean_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ dtile_layer,
+    const int32_t* __restrict__ dtile_start, int32_t ntiles, int32_t W, int64_t N,
+    const float* __restrict__ grad, float* __restrict__ mem, float eta, float inv_w,
+    float* __restrict__ vals) {
+    for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
+        const DevLayer L = layers[dtile_layer[u]];
+        const int64_t s0 = dtile_start[u];
+        const int64_t cnt = min64(int64_t(kDenseTile), L.n - s0);
+        for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+            float s = 0.0f;
+            for (int w = 0; w < W; ++w) {
+                const int64_t e = int64_t(w) * N + L.offset + s0 + i;
+                s = __fadd_rn(s, residual(mem[e], eta, __ldcs(grad + e)));
+                mem[e] = 0.0f;
+            }
+            vals[L.val_off + s0 + i] = __fmul_rn(s, inv_w);
         }
     }
 }
@@ -750,19 +811,19 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
-        static const int r_qred = resident_blocks(ps_qred_kernel, 256);
+        static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
         static const int r_resid = resident_blocks(ps_resid_kernel, 256);
         GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st, t->d_layers,
                    ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw, t->ppart_pw, grad, mem,
                    eta, k_or_rank, Q, ppart);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
-                   t->d_ps_layers, t->nps, W, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
+                   t->d_ps_layers, t->nps, W, 1, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
                    pd, P, status, t->ps_ntall, tdone);
         if (t->ps_ntall > 0) {
             for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
                 GCE_LAUNCH(ps_orth_tall_kernel, wave_grid(int64_t(t->ps_tall_nunits) * W, 8, r_tall), 256, 0,
-                           st, op, t->d_layers, ps, t->d_ps_tall_units, t->ps_tall_nunits, W,
+                           st, op, t->d_layers, ps, t->d_ps_tall_units, t->ps_tall_nunits, W, 1,
                            t->P_pw, t->ppart_pw, t->pd_pw, t->ps_ntall, t->ps_tall_parts,
                            k_or_rank, ppart, pd, at<double>(ws, lay.tparts),
                            at<double>(ws, lay.tscal), tdone, P);
@@ -770,13 +831,79 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
                    t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->P_pw, t->qpart_pw,
                    mem, k_or_rank, P, qpart);
-        GCE_LAUNCH(ps_qred_kernel, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0, st,
-                   t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
-                   k_or_rank, qpart, Q);
+        GCE_LAUNCH(ps_qred_kernel<false>, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0,
+                   st, t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
+                   k_or_rank, qpart, Q, nullptr, 1.0f);
         GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
                    t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
                    k_or_rank, P, Q, mem, dense_out);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+}
+
+extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad, float* mem,
+                                float eta, const int32_t* k_or_rank, float* P, float* Q,
+                                float* vals, void* ws, size_t ws_bytes, void* stream) {
+    if (!t || W < 1 || !grad || !mem || !ws) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    if (!aligned16(grad) || !aligned16(mem) || !aligned16(ws)) return GCE_ERR_ARG;
+    if (t->nps > 0 && (!P || !Q || !aligned16(P) || !aligned16(Q))) return GCE_ERR_ARG;
+    if (t->dtiles_pw > 0 && !vals) return GCE_ERR_ARG;
+    if (k_or_rank && (reinterpret_cast<uintptr_t>(k_or_rank) & 3)) return GCE_ERR_ARG;
+    const PsWs lay = ps_dp_layout(t, W);
+    if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(ws);
+    const float inv_w = 1.0f / float(W);
+    if (t->nps > 0) {
+        float* ppart = at<float>(ws, lay.ppart);
+        double* pd = at<double>(ws, lay.pd);
+        float* qpart = at<float>(ws, lay.qpart);
+        float* qloc = at<float>(ws, lay.qloc);
+        int32_t* tdone = at<int32_t>(ws, lay.tdone);
+        const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
+        static const int r_mq = resident_blocks(ps_mq_kernel, 256);
+        static const int r_orth = resident_blocks(ps_orth_kernel, 256);
+        static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
+        static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
+        static const int r_qred = resident_blocks(ps_qred_kernel<true>, 256);
+        static const int r_resid = resident_blocks(ps_resid_kernel, 256);
+        // every worker reads the shared warm start Q (stride 0)
+        GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
+                   t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0),
+                   t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart);
+        // one P per layer from the partials of all W workers
+        GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
+                   t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank,
+                   ppart, pd, P, status, t->ps_ntall, tdone);
+        if (t->ps_ntall > 0) {
+            for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
+                GCE_LAUNCH(ps_orth_tall_kernel, wave_grid(t->ps_tall_nunits, 8, r_tall), 256, 0,
+                           st, op, t->d_layers, ps, t->d_ps_tall_units, t->ps_tall_nunits, 1, W,
+                           int64_t(0), t->ppart_pw, t->pd_pw, t->ps_ntall, t->ps_tall_parts,
+                           k_or_rank, ppart, pd, at<double>(ws, lay.tparts),
+                           at<double>(ws, lay.tscal), tdone, P);
+        }
+        // Q_w = M_w^T P for every worker with the shared P (stride 0)
+        GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
+                   t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, int64_t(0),
+                   t->qpart_pw, mem, k_or_rank, P, qpart);
+        GCE_LAUNCH(ps_qred_kernel<true>, wave_grid(t->psq_ntiles, 8, r_qred), 256, 0, st,
+                   t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
+                   k_or_rank, qpart, qloc, Q, inv_w);
+        // each worker's error against its own Q_w
+        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
+                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->Q_pw,
+                   k_or_rank, P, qloc, mem, nullptr);
+        if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+    }
+    if (t->dtiles_pw > 0) {
+        static const int r_dm = resident_blocks(ps_dense_mean_kernel, 256);
+        GCE_LAUNCH(ps_dense_mean_kernel, wave_grid(t->dtiles_pw, 8, r_dm), 256, 0, st,
+                   t->d_layers, t->d_dtile_layer, t->d_dtile_start, t->dtiles_pw, W, t->N, grad,
+                   mem, eta, inv_w, vals);
+        if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+    }
+    return GCE_OK;
 }

@@ -71,7 +71,6 @@ int sm_count() {
 }
 
 // ---- DENSE layers: payload = fl32(m + fl32(eta*g)), memory -> +0 ----------
-constexpr int kDenseTile = 4096;
 
 __global__ void __launch_bounds__(256) dense_kernel(const DevLayer* __restrict__ layers,
                                                     const int32_t* __restrict__ dtile_layer,
@@ -302,6 +301,7 @@ namespace gce {
 size_t topk_ws_bytes(const gce_table* t, int32_t W);
 size_t randk_ws_bytes(const gce_table* t, int32_t W);
 size_t powersgd_ws_bytes(const gce_table* t, int32_t W);
+size_t powersgd_dp_ws_bytes(const gce_table* t, int32_t W);
 size_t accordion_ws_bytes(const gce_table* t);
 size_t decompress_ws_bytes(const gce_table* t, int32_t W);
 }  // namespace gce
@@ -314,6 +314,7 @@ extern "C" int gce_workspace_bytes(const gce_table* t, int32_t W, int32_t op, si
         case GCE_OP_POWERSGD: *bytes = powersgd_ws_bytes(t, W); break;
         case GCE_OP_ACCORDION: *bytes = accordion_ws_bytes(t); break;
         case GCE_OP_DECOMPRESS: *bytes = decompress_ws_bytes(t, W); break;
+        case GCE_OP_POWERSGD_DP: *bytes = powersgd_dp_ws_bytes(t, W); break;
         default: return GCE_ERR_ARG;
     }
     return GCE_OK;

@@ -84,6 +84,7 @@ extern "C" {
 #define GCE_OP_POWERSGD 2
 #define GCE_OP_ACCORDION 3
 #define GCE_OP_DECOMPRESS 4
+#define GCE_OP_POWERSGD_DP 5
 
 /* Accordion levels [ACC] */
 #define GCE_LEVEL_LOW 0  /* l_low: less compression (critical regime) */
@@ -190,6 +191,26 @@ GCE_API int powersgd_init_q(const gce_table* table, int32_t W, uint64_t seed, fl
 GCE_API int powersgd_step(const gce_table* table, int32_t W, const float* grad, float* mem,
                   float eta, const int32_t* k_or_rank, float* P, float* Q, float* vals,
                   float* dense_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Data-parallel PowerSGD step ([UTIL] Key results: PowerSGD is all-reduce
+ * compatible) over the W workers of one GPU: the two all-reduces become sums
+ * over the workers in worker order, the orthonormal P and the warm start Q
+ * are shared, and each worker keeps its own error:
+ *   M_w = fl32(mem_w + fl32(eta*grad_w));  P = sum_w M_w Q;
+ *   P <- orthonormal columns (modified Gram-Schmidt, column order, fp64);
+ *   Q_w = M_w^T P;  mem_w <- M_w - P Q_w^T;
+ *   Q <- fl32(fl32(sum_w Q_w) * fl32(1/W))   (the workers' mean);
+ * DENSE layers: vals <- fl32(fl32(sum_w M_w) * fl32(1/W)), every mem_w -> 0.
+ * P Q^T (decompress_accumulate with W = 1 on P, Q, vals) is the mean of the
+ * workers' decompressed updates.  grad, mem: [W][N]; P: [P_per_worker]
+ * written; Q: [Q_per_worker] read and written; vals: [vals_per_worker]
+ * (NULL allowed without DENSE layers).  k_or_rank as for powersgd_step.
+ * ws: gce_workspace_bytes(GCE_OP_POWERSGD_DP).
+ */
+GCE_API int powersgd_dp_step(const gce_table* table, int32_t W, const float* grad, float* mem,
+                             float eta, const int32_t* k_or_rank, float* P, float* Q,
+                             float* vals, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Accordion select [ACC] over every compressed layer of the table.
