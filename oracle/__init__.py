@@ -37,6 +37,9 @@ def lib():
             "or_powersgd": (C.c_int, [i64, i64, i64, i64, f32, vp, vp, vp, vp, vp]),
             "or_powersgd_dp": (C.c_int, [i64, i64, i64, i64, i64, f32, vp, vp, vp, vp]),
             "or_dense_dp": (C.c_int, [i64, i64, f32, vp, vp, vp]),
+            "or_ef_sign": (C.c_int, [i64, f32, vp, vp, vp, vp]),
+            "or_accum_sign": (None, [i64, f32, vp, vp]),
+            "or_vote_sign": (None, [i64, i64, i64, vp, f32, vp]),
             "or_layer_norm": (f64, [i64, vp]),
             "or_accordion_decide": (i32, [f64, f64, f64]),
             "or_accum_sparse": (None, [i64, vp, vp, vp]),
@@ -171,6 +174,37 @@ def dense_dp_unit(g, m, eta):
     _check(lib().or_dense_dp(W, n, float(np.float32(eta)), _ptr(g), _ptr(m), _ptr(out)),
            "dense_dp")
     return out, m
+
+
+def ef_sign_unit(g, m, eta):
+    """signSGD with error feedback on one unit.  Returns (scale, words
+    (uint32, ceil(n/32)), m_new)."""
+    g = _f32(g)
+    m = _f32(m).copy()
+    n = g.size
+    words = np.zeros((n + 31) // 32, np.uint32)
+    sc = np.zeros(1, np.float32)
+    _check(lib().or_ef_sign(n, float(np.float32(eta)), _ptr(g), _ptr(m), _ptr(sc), _ptr(words)),
+           "ef_sign")
+    return sc[0], words, m
+
+
+def accum_sign(out, scale, words):
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    assert out.dtype == np.float32 and out.flags.c_contiguous
+    assert words.size >= (out.size + 31) // 32
+    lib().or_accum_sign(out.size, float(np.float32(scale)), _ptr(words), _ptr(out))
+
+
+def vote_sign(words, n, out_scale):
+    """words: (W, words_per_worker) uint32.  Returns the majority-vote
+    update (n,) float32."""
+    words = np.ascontiguousarray(words, dtype=np.uint32)
+    W, wpw = words.shape
+    assert wpw >= (n + 31) // 32
+    out = np.empty(n, np.float32)
+    lib().or_vote_sign(W, n, wpw, _ptr(words), float(np.float32(out_scale)), _ptr(out))
+    return out
 
 
 def layer_norm(g):

@@ -51,6 +51,10 @@
  *     missing previous norm (prev < 0) means "critical", rel change >= the
  *     threshold means "critical" (level LOW = l_low), else HIGH = l_high;
  *   - k from a fraction in parts per million: k = max(1, floor(n*ppm/1e6)).
+ *   - signSGD with error feedback (or_ef_sign): the 1-bit payload is the
+ *     float's sign bit, scaled by the layer's mean |p| (fp64 sum in index
+ *     order, one rounding), so that the memory keeps p - s sign(p); the
+ *     aggregate is the worker-order fp32 sum, or sign SGD's majority vote;
  *   - data-parallel PowerSGD (or_powersgd_dp): the all-reduces are sums over
  *     the workers -- P = sum_w M_w Q before orthonormalising, Q = the mean of
  *     the workers' Q_w = M_w^T P -- and each worker keeps its own error
@@ -435,6 +439,58 @@ int or_dense_dp(int64_t W, int64_t n, float eta, const float* g, float* m, float
         out[i] = s * inv;
     }
     return OR_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* signSGD with error feedback ([UTIL] Method / Key results evaluate sign
+ * SGD, whose 1-bit payload cannot be all-reduced and is gathered; [MEM]
+ * Method gives the memory).  One worker's layer of n elements:
+ *   p_i   = fl32(m_i + fl32(eta * g_i))              (the Mem-SGD residual)
+ *   s     = fl32( (sum_i |p_i|, in double, index order) / n )
+ *   b_i   = sign bit of p_i (1 for negative, -0 included)
+ *   g_i   = s with b_i's sign;  m_i <- fl32(p_i - g_i)
+ * words: ceil(n/32) uint32, bit (i mod 32) of word i/32 is b_i; the unused
+ * high bits of the last word are 0.  *scale receives s. */
+int or_ef_sign(int64_t n, float eta, const float* g, float* m, float* scale, uint32_t* words)
+{
+    if (n < 1) return OR_ERR_ARG;
+    double l1 = 0.0;
+    for (int64_t i = 0; i < n; ++i) {
+        float p = or_residual(m[i], eta, g[i]);
+        l1 += fabs((double)p);
+    }
+    float sc = (float)(l1 / (double)n);
+    for (int64_t j = 0; j < (n + 31) / 32; ++j) words[j] = 0u;
+    for (int64_t i = 0; i < n; ++i) {
+        float p = or_residual(m[i], eta, g[i]);
+        int neg = signbit(p) ? 1 : 0;
+        if (neg) words[i / 32] |= 1u << (i % 32);
+        m[i] = neg ? p + sc : p - sc;
+    }
+    *scale = sc;
+    return OR_OK;
+}
+
+/* out[i] += (bit i set ? -scale : scale) for one worker's sign payload. */
+void or_accum_sign(int64_t n, float scale, const uint32_t* words, float* out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        int neg = (words[i / 32] >> (i % 32)) & 1u;
+        out[i] = out[i] + (neg ? -scale : scale);
+    }
+}
+
+/* Majority vote over W workers' sign payloads (sign SGD's aggregation):
+ * out[i] = out_scale * sign(#positive - #negative), 0 on a tie. */
+void or_vote_sign(int64_t W, int64_t n, int64_t words_per_worker, const uint32_t* words,
+                  float out_scale, float* out)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        int64_t c = 0;
+        for (int64_t w = 0; w < W; ++w)
+            c += ((words[w * words_per_worker + i / 32] >> (i % 32)) & 1u) ? -1 : 1;
+        out[i] = c > 0 ? out_scale : (c < 0 ? -out_scale : 0.0f);
+    }
 }
 
 /* ------------------------------------------------------------------ */

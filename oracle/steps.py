@@ -10,9 +10,9 @@ from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
 
-from . import (accordion_decide, accum_dense, accum_lowrank, accum_sparse,
-               dense_dp_unit, dense_unit, ef_randk_unit, ef_topk_unit, k_from_ppm, layer_norm,
-               powersgd_dp_unit, powersgd_init_q, powersgd_unit, scale)
+from . import (accordion_decide, accum_dense, accum_lowrank, accum_sign, accum_sparse,
+               dense_dp_unit, dense_unit, ef_randk_unit, ef_sign_unit, ef_topk_unit, k_from_ppm,
+               layer_norm, powersgd_dp_unit, powersgd_init_q, powersgd_unit, scale, vote_sign)
 
 
 def layer_offsets(layers):
@@ -32,11 +32,14 @@ def _run(units, fn, threads):
 
 def sparse_step(layers, grad, mem, eta, k_per_layer, method="topk", seed=0, step=0,
                 units=None, threads=1):
-    """Mem-SGD top-k / rand-k step (Sparsified SGD with Memory, Method).
+    """Mem-SGD top-k / rand-k step (Sparsified SGD with Memory, Method), or
+    with method="sign" signSGD with the same memory (On the Utility of
+    Gradient Compression, Method: sign SGD).
 
     grad, mem: (W, N) float32; mem is updated in place.  Layers whose kind is
-    'dense' are sent whole.  Returns {(w, l): (vals, idx)} for compressed
-    layers and {(w, l): payload} for dense ones.
+    'dense' are sent whole.  Returns {(w, l): (vals, idx)} for top-k / rand-k
+    layers, {(w, l): (scale, words)} for sign layers and {(w, l): payload}
+    for dense ones.  k_per_layer is unused for sign.
     """
     offs, N = layer_offsets(layers)
     W = grad.shape[0]
@@ -51,6 +54,9 @@ def sparse_step(layers, grad, mem, eta, k_per_layer, method="topk", seed=0, step
         if lay["kind"] == "dense":
             pay, m_new = dense_unit(grad[w, sl], mem[w, sl], eta)
             return u, pay, None, m_new
+        if method == "sign":
+            sc, words, m_new = ef_sign_unit(grad[w, sl], mem[w, sl], eta)
+            return u, sc, words, m_new
         k = int(k_per_layer[l])
         if method == "topk":
             vals, idx, m_new = ef_topk_unit(grad[w, sl], mem[w, sl], k, eta)
@@ -207,6 +213,9 @@ def decompress(layers, W, payload, scale_factor, rank_per_layer=None, k_per_laye
             elif lay["kind"] == "powersgd":
                 P, Q = p
                 accum_lowrank(view, P, Q, int(rank_per_layer[l]))
+            elif lay["kind"] == "sign":
+                sc, words = p
+                accum_sign(view, sc, words)
             else:
                 vals, idx = p
                 k = int(k_per_layer[l]) if k_per_layer is not None else len(vals)
@@ -228,3 +237,23 @@ def memsgd_eta(t, mu, a):
     """Step size eta_t = 8 / (mu (a + t)) of "Sparsified SGD with Memory",
     Method, in fp64, rounded once to fp32."""
     return np.float32(8.0 / (float(mu) * (float(a) + float(t))))
+
+
+def vote(layers, W, payload, scale_factor):
+    """Majority-vote aggregate of sign payloads (sign SGD's aggregation, On
+    the Utility of Gradient Compression, Method): per element scale *
+    sign(#positive - #negative) over the workers, 0 on a tie; dense layers
+    are summed as `decompress` sums them."""
+    offs, N = layer_offsets(layers)
+    out = np.zeros(N, np.float32)
+    for l, lay in enumerate(layers):
+        n = lay["rows"] * lay["cols"]
+        view = out[offs[l]:offs[l] + n]
+        if lay["kind"] == "dense":
+            for w in range(W):
+                accum_dense(view, payload[(w, l)])
+            scale(view, scale_factor)
+        else:
+            words = np.stack([payload[(w, l)][1] for w in range(W)])
+            view[:] = vote_sign(words, n, scale_factor)
+    return out
