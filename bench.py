@@ -48,6 +48,8 @@ def workload_spec(name):
         return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk")
     if name == "bert_base_topk1pct_w8_apply":    # decode fused with x -= mean update, eta_t
         return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk", apply=True)
+    if name == "bert_base_sign_w8":              # signSGD with memory, 1 bit per element
+        return dict(layers=wl.bert_base_topk(kind="sign"), W=8, cfg=4, method="sign")
     if name == "bert_base_topk1pct_w1":          # one replica: a profiling-sized case
         return dict(layers=wl.bert_base_topk(), W=1, cfg=4, method="topk")
     if name == "bert_base_randk1pct_w8":
@@ -78,7 +80,7 @@ def workload_spec(name):
 
 
 MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel",
-                "powersgd_dp": "ps_mq_kernel"}
+                "powersgd_dp": "ps_mq_kernel", "sign": "sg_emit_kernel"}
 
 
 def max_over_ranks_of(x, world, device):
@@ -224,6 +226,9 @@ def cpu_oracle_sample(spec, units, steps_seed):
         elif spec["method"] == "topk":
             vals, idx, m_new = oracle.ef_topk_unit(gg, mm, lay["cap"], wl.ETA)
             oracle.accum_sparse(out, vals, idx)
+        elif spec["method"] == "sign":
+            sc, words, m_new = oracle.ef_sign_unit(gg, mm, wl.ETA)
+            oracle.accum_sign(out, sc, words)
         else:
             vals, idx, m_new = oracle.ef_randk_unit(gg, mm, lay["cap"], wl.ETA, 5, w, l, 0)
             oracle.accum_sparse(out, vals, idx)
@@ -356,6 +361,8 @@ def main():
             gce.ef_topk_step(table, W, grad, mem, eta, kr, vals, idx, ws)
         elif method == "randk":
             gce.ef_randk_step(table, W, grad, mem, eta, kr, 5, s, vals, idx, ws)
+        elif method == "sign":
+            gce.ef_sign_step(table, W, grad, mem, eta, vals, ws)
         elif method == "powersgd_dp":
             gce.powersgd_dp_step(table, W, grad, mem, eta, kr, P, Q, vals, ws)
             # the shared payload is already the workers' mean: one decode
@@ -429,6 +436,9 @@ def main():
     # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
     if method in ("powersgd", "powersgd_dp"):
         step_bytes = W * 12.0 * N
+    elif method == "sign":
+        # norm pass 8 B/el, emit pass 12 B/el + words; decode reads the words
+        step_bytes = W * (20.0 * N + N / 8.0) + W * N / 8.0
     else:
         step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total
     # the dense result: written (4 B), or read and written in place (8 B)

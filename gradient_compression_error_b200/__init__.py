@@ -17,9 +17,10 @@ import os
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgce.so")
 
-KIND = {"topk": 0, "randk": 1, "powersgd": 2, "dense": 3}
+KIND = {"topk": 0, "randk": 1, "powersgd": 2, "dense": 3, "sign": 4}
 KIND_NAME = {v: k for k, v in KIND.items()}
-OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4, "powersgd_dp": 5}
+OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4, "powersgd_dp": 5,
+      "sign": 6}
 STATUS_K_RANGE = 1
 STATUS_FALLBACK = 2
 LEVEL_LOW, LEVEL_HIGH = 0, 1
@@ -68,6 +69,8 @@ SIGNATURES = {
                                 C.c_size_t, _vp]),
     "powersgd_dp_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
                                    C.c_size_t, _vp]),
+    "ef_sign_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, C.c_size_t, _vp]),
+    "decompress_vote": (C.c_int, [_vp, _i32, _vp, _f32, _vp, _vp]),
     "accordion_init": (C.c_int, [_vp, _vp, _vp, _vp]),
     "accordion_select": (C.c_int, [_vp, _vp, _i64, _i32, _f64, _i32, _i32, _vp, _vp, _vp, _vp,
                                    _vp, C.c_size_t, _vp]),
@@ -221,6 +224,20 @@ def powersgd_dp_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, ws, stream
         table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
         _ptr(k_or_rank, _i32()), _ptr(P, _f32()), _ptr(Q, _f32()), _ptr(vals, _f32()),
         _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def ef_sign_step(table, W, grad, mem, eta, vals, ws, stream=None):
+    """signSGD with error feedback; vals holds each SIGN layer's scale (slot
+    0) and sign words (slots 4..., uint32 bit patterns) (include/gce.h)."""
+    _check("ef_sign_step", lib().ef_sign_step(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(vals), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def decompress_vote(table, W, vals, scale, out, stream=None):
+    """sign SGD's majority vote over the workers' sign payloads."""
+    _check("decompress_vote", lib().decompress_vote(
+        table.handle, int(W), _ptr(vals), float(scale), _ptr(out, _f32()), _stream(stream)))
 
 
 def accordion_init(table, prev_norm, level, stream=None):

@@ -102,6 +102,7 @@ __device__ __forceinline__ int32_t ac_param(const DevLayer& L, int32_t level, in
                                             int32_t lvl_high) {
     const int32_t p = level == GCE_LEVEL_LOW ? lvl_low : lvl_high;
     if (L.kind == GCE_KIND_POWERSGD) return p;
+    if (L.kind == GCE_KIND_SIGN) return 0;  // one fixed level: nothing to choose
     const int64_t k = (L.n * int64_t(p)) / 1000000;
     return int32_t(k < 1 ? 1 : k);
 }

@@ -308,6 +308,100 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     }
 }
 
+// Decode of a SIGN table (SIGN and DENSE layers), one 4096-output tile per
+// block.  The tile's sign words of up to 32 workers at a time are staged in
+// shared memory (128 words a worker) with their scales; each thread then forms
+// its 32 outputs (four neighbouring ones in each of 8 rounds) as the
+// worker-order sum of +-s.
+template <bool kApply>
+__global__ void __launch_bounds__(kDcThreads) dc_sign_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
+    int32_t dc_tiles, int32_t W, int64_t vals_pw, const float* __restrict__ vals, float scale,
+    float* __restrict__ out) {
+    constexpr int kWordsPerTile = kDcTile / 32;           // 128
+    constexpr int kRounds = kDcTile / (4 * kDcThreads);   // 8
+    __shared__ uint32_t sw[32 * kWordsPerTile];
+    __shared__ float s_sc[32];
+    for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
+        const int32_t l = dc_tile_layer[u];
+        const DevLayer L = layers[l];
+        const int64_t start = int64_t(u - L.dc_tile0) << kDcTileLog;
+        const int cnt = int(min64(kDcTile, L.n - start));
+        float* o = out + L.offset + start;
+        if (L.kind == GCE_KIND_DENSE) {
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+                float s = 0.0f;
+                for (int w = 0; w < W; ++w)
+                    s = __fadd_rn(s, vals[int64_t(w) * vals_pw + L.val_off + start + i]);
+                o[i] = dc_final<kApply>(s, scale, o + i);
+            }
+            continue;
+        }
+        if (L.kind != GCE_KIND_SIGN) continue;
+        const int nwords = (cnt + 31) >> 5;
+        const int64_t word0 = start >> 5;
+        float a[kRounds][4];
+#pragma unroll
+        for (int it = 0; it < kRounds; ++it)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) a[it][j] = 0.0f;
+        for (int wc = 0; wc < W; wc += 32) {
+            const int wn = min(32, W - wc);
+            __syncthreads();  // the previous words are consumed
+            // kB loads a thread in flight, then their stores
+            constexpr int kB = 8;
+            for (int q0 = 0; q0 < wn * nwords; q0 += kB * kDcThreads) {
+                uint32_t v[kB];
+#pragma unroll
+                for (int e = 0; e < kB; ++e) {
+                    const int q = q0 + e * kDcThreads + int(threadIdx.x);
+                    v[e] = 0u;
+                    if (q < wn * nwords) {
+                        const int wq = q / nwords, j = q - wq * nwords;
+                        v[e] = reinterpret_cast<const uint32_t*>(
+                            vals + int64_t(wc + wq) * vals_pw + L.val_off + 4)[word0 + j];
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < kB; ++e) {
+                    const int q = q0 + e * kDcThreads + int(threadIdx.x);
+                    if (q < wn * nwords) {
+                        const int wq = q / nwords;
+                        sw[wq * kWordsPerTile + (q - wq * nwords)] = v[e];
+                    }
+                }
+            }
+            if (int(threadIdx.x) < wn)
+                s_sc[threadIdx.x] = vals[int64_t(wc + threadIdx.x) * vals_pw + L.val_off];
+            __syncthreads();
+            for (int wq = 0; wq < wn; ++wq) {
+                const float sc = s_sc[wq];
+#pragma unroll
+                for (int it = 0; it < kRounds; ++it) {
+                    const int i = 4 * int(threadIdx.x) + 4 * kDcThreads * it;
+                    const uint32_t nib = sw[wq * kWordsPerTile + (i >> 5)] >> (i & 31);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        a[it][j] = __fadd_rn(a[it][j], ((nib >> j) & 1u) ? -sc : sc);
+                }
+            }
+        }
+        const bool al = ((L.offset + start) & 3) == 0;
+#pragma unroll
+        for (int it = 0; it < kRounds; ++it) {
+            const int i = 4 * int(threadIdx.x) + 4 * kDcThreads * it;
+            if (al && i + 4 <= cnt) {
+                float4* o4 = reinterpret_cast<float4*>(o + i);
+                __stcs(o4, dc_final4<kApply>(make_float4(a[it][0], a[it][1], a[it][2], a[it][3]),
+                                             scale, o4));
+            } else {
+                for (int j = 0; j < 4; ++j)
+                    if (i + j < cnt) o[i + j] = dc_final<kApply>(a[it][j], scale, o + i + j);
+            }
+        }
+    }
+}
+
 // bounds pass plus the decode kernels for every kind the table holds;
 // apply: out is the parameter vector x and gets x - scale * sum
 template <bool kApply>
@@ -317,6 +411,17 @@ static int launch_decode_t(const gce_table* t, int32_t W, const float* vals, con
     const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
     static const int r_bounds = resident_blocks(dc_bounds_kernel, 256);
     static const int r_accum = resident_blocks(dc_accum_kernel<kApply>, kDcThreads);
+    if (t->ckind == GCE_KIND_SIGN) {
+        static const int r_sign = resident_blocks(dc_sign_kernel<kApply>, kDcThreads);
+        const int grid = wave_grid(t->dc_tiles, 16, r_sign);
+        if (kApply)
+            GCE_LAUNCH(dc_sign_kernel<true>, grid, kDcThreads, 0, st, t->d_layers,
+                       t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, vals, scale, out);
+        else
+            GCE_LAUNCH(dc_sign_kernel<false>, grid, kDcThreads, 0, st, t->d_layers,
+                       t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, vals, scale, out);
+        return check_launch();
+    }
     if (sparse && t->bunits_pw > 0) {
         const int64_t units = int64_t(t->bunits_pw) * W;
         GCE_LAUNCH(dc_bounds_kernel, wave_grid(units, 8, r_bounds), 256, 0, st, t->d_layers,

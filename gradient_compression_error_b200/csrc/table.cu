@@ -154,7 +154,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     for (int32_t l = 0; l < L; ++l) {
         const gce_layer_desc& d = descs[l];
         const int64_t n = d.rows * d.cols;
-        if (d.rows < 1 || d.cols < 1 || n > INT32_MAX || d.kind < 0 || d.kind > GCE_KIND_DENSE) {
+        if (d.rows < 1 || d.cols < 1 || n > INT32_MAX || d.kind < 0 || d.kind > GCE_KIND_SIGN) {
             delete t;
             return GCE_ERR_ARG;
         }
@@ -181,6 +181,10 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
             x.q_off = qoff;
             poff += (d.rows * d.cap + 3) & ~int64_t(3);
             qoff += (d.cols * d.cap + 3) & ~int64_t(3);
+        } else if (d.kind == GCE_KIND_SIGN) {
+            // slot 0: the scale, slots 1-3: zero, then the sign words
+            x.val_off = voff;
+            voff += 4 + ((((n + 31) / 32) + 3) & ~int64_t(3));
         } else {  // DENSE
             x.val_off = voff;
             voff += (n + 3) & ~int64_t(3);
@@ -302,6 +306,7 @@ size_t topk_ws_bytes(const gce_table* t, int32_t W);
 size_t randk_ws_bytes(const gce_table* t, int32_t W);
 size_t powersgd_ws_bytes(const gce_table* t, int32_t W);
 size_t powersgd_dp_ws_bytes(const gce_table* t, int32_t W);
+size_t sign_ws_bytes(const gce_table* t, int32_t W);
 size_t accordion_ws_bytes(const gce_table* t);
 size_t decompress_ws_bytes(const gce_table* t, int32_t W);
 }  // namespace gce
@@ -315,6 +320,7 @@ extern "C" int gce_workspace_bytes(const gce_table* t, int32_t W, int32_t op, si
         case GCE_OP_ACCORDION: *bytes = accordion_ws_bytes(t); break;
         case GCE_OP_DECOMPRESS: *bytes = decompress_ws_bytes(t, W); break;
         case GCE_OP_POWERSGD_DP: *bytes = powersgd_dp_ws_bytes(t, W); break;
+        case GCE_OP_SIGN: *bytes = sign_ws_bytes(t, W); break;
         default: return GCE_ERR_ARG;
     }
     return GCE_OK;

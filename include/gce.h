@@ -77,6 +77,7 @@ extern "C" {
 #define GCE_KIND_RANDK 1
 #define GCE_KIND_POWERSGD 2
 #define GCE_KIND_DENSE 3 /* sent uncompressed: payload = m + eta*grad, memory -> 0 */
+#define GCE_KIND_SIGN 4  /* 1 bit per element plus one scale (signSGD with memory) */
 
 /* operations, for gce_workspace_bytes */
 #define GCE_OP_TOPK 0
@@ -85,6 +86,7 @@ extern "C" {
 #define GCE_OP_ACCORDION 3
 #define GCE_OP_DECOMPRESS 4
 #define GCE_OP_POWERSGD_DP 5
+#define GCE_OP_SIGN 6
 
 /* Accordion levels [ACC] */
 #define GCE_LEVEL_LOW 0  /* l_low: less compression (critical regime) */
@@ -94,7 +96,10 @@ typedef struct gce_table gce_table;
 
 /* One layer as the caller describes it.  cap: for TOPK / RANDK the largest k
  * any step will use (payload slots, 1 <= cap <= rows*cols); for POWERSGD the
- * largest rank r_max (1..4, <= min(rows, cols)); ignored for DENSE. */
+ * largest rank r_max (1..4, <= min(rows, cols)); ignored for DENSE and SIGN.
+ * A SIGN layer's payload takes 4 + ceil(n/32) slots (rounded up to a multiple
+ * of 4): slot 0 the fp32 scale, slots 1-3 zero, then the packed sign words
+ * (uint32 bit patterns; bit i mod 32 of word i/32 is element i's sign). */
 typedef struct gce_layer_desc {
     int64_t rows;
     int64_t cols; /* 1 for a 1-D layer */
@@ -213,6 +218,32 @@ GCE_API int powersgd_dp_step(const gce_table* table, int32_t W, const float* gra
                              float* vals, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * signSGD with error feedback for every (worker, SIGN layer) ([UTIL]
+ * Method / Key results: sign SGD, one bit per element; [MEM] Method: the
+ * memory), plus DENSE layers (payload to vals, memory -> 0):
+ *   p = fl32(mem + fl32(eta*grad));  s = fl32(sum_i |p_i| / n) with the sum
+ *   in fp64;  payload: s and the sign bits of p (-0 counts as negative);
+ *   mem <- fl32(p - s) where p's sign bit is 0, fl32(p + s) where it is 1.
+ * vals: [W][vals_per_worker] 32-bit slots laid out as gce_layer_desc states.
+ * The sign bits and, for a given s, the memory are exact; s may differ from
+ * a sequential fp64 sum by one fp32 rounding in rare cases (the fp64 sum's
+ * order is the library's own, fixed).  ws: gce_workspace_bytes(GCE_OP_SIGN).
+ */
+GCE_API int ef_sign_step(const gce_table* table, int32_t W, const float* grad, float* mem,
+                         float eta, float* vals, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * sign SGD's majority-vote aggregate ([UTIL] Method: sign SGD is gathered,
+ * not all-reduced): for every element of a SIGN layer
+ *   out = scale * sign(#workers with sign bit 0 - #workers with sign bit 1),
+ * 0 on a tie (the workers' scales are not used); DENSE layers are summed in
+ * worker order and scaled as decompress_accumulate does.  vals as written by
+ * ef_sign_step.  No workspace.
+ */
+GCE_API int decompress_vote(const gce_table* table, int32_t W, const float* vals, float scale,
+                            float* out, void* stream);
+
+/*
  * Accordion select [ACC] over every compressed layer of the table.
  * Sets prev_norm[l] = -1 (no earlier check) and level[l] = LOW.
  */
@@ -226,7 +257,7 @@ GCE_API int accordion_init(const gce_table* table, double* prev_norm, int32_t* l
  * Every step: k_or_rank_out[l] = the level's parameter -- for POWERSGD
  * layers the rank lvl_low / lvl_high, for TOPK / RANDK layers
  * k = max(1, floor(n * ppm / 1e6)) with ppm = lvl_low / lvl_high (parts per
- * million of the layer); DENSE layers get 0.  lvl_low / lvl_high are host
+ * million of the layer); DENSE and SIGN layers get 0.  lvl_low / lvl_high are host
  * values.  prev_norm, cur_norm: device double[L]; level, k_or_rank_out:
  * device int32[L].
  */
