@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
     const int32_t* __restrict__ sunit_part, int32_t sunits_pw, int32_t W, int32_t ncomp,
     int64_t S, int64_t N, const float* __restrict__ grad, const float* __restrict__ mem,
     float eta, TkSeg* __restrict__ segs, int32_t* __restrict__ hists, double sigma) {
-    constexpr int kBatch = 16;
+    constexpr int kBatch = 8;
     __shared__ int32_t h[kTkSBins];
     __shared__ int s_last;
     const int tid = threadIdx.x;

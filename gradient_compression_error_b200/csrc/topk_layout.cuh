@@ -14,7 +14,7 @@ constexpr int kTkSampleChunk = 32;                 // sampled run length (one 12
 constexpr int kTkSampleStride = 2048;              // one run per 2048 elements
 constexpr int64_t kTkSamplePart = int64_t(1) << 20; // elements covered by one sample unit
 constexpr int64_t kTkSampleMinN = 65536;           // smaller layers: exact histogram of all
-constexpr int kTkHUnit = 32768;                    // candidates per histogram unit
+constexpr int kTkHUnit = 16384;                    // candidates per histogram unit
 
 // Per (worker, layer) state of one top-k step.
 struct TkSeg {
