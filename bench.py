@@ -415,7 +415,10 @@ def main():
     ms_step = t_ms / args.steps
 
     main_kernel = MAIN_KERNELS[method]
-    main_ms, main_n = prof.get(main_kernel, (0.0, 0))
+    # the main pass, whichever template instance ran (rand-k's may carry the
+    # next step's key pass)
+    hits = [v for name, v in prof.items() if name == main_kernel or name.startswith(main_kernel + "<")]
+    main_ms, main_n = sum(v[0] for v in hits), sum(v[1] for v in hits)
     peak, peak_kind = measured_hbm_gbs()
     # the main pass covers every compressed element once per step: bytes and
     # kernel time per step

@@ -85,6 +85,7 @@ SIGNATURES = {
     "gce_launch_count": (_u64, []),
     "gce_error_string": (C.c_char_p, [C.c_int]),
     "gce_set_bracket_sigma": (C.c_int, [_f64]),
+    "gce_set_randk_ahead": (C.c_int, [C.c_int32]),
     "gce_profile_start": (C.c_int, []),
     "gce_profile_stop": (C.c_int, []),
     "gce_profile_count": (C.c_int, []),
@@ -315,3 +316,8 @@ def profile_stop():
 
 def set_bracket_sigma(sigma):
     _check("gce_set_bracket_sigma", lib().gce_set_bracket_sigma(float(sigma)))
+
+
+def set_randk_ahead(on):
+    """Run the next rand-k step's key pass inside this one (include/gce.h)."""
+    _check("gce_set_randk_ahead", lib().gce_set_randk_ahead(1 if on else 0))

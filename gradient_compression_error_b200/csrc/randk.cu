@@ -31,6 +31,8 @@ namespace gce {
 
 extern double bracket_sigma();
 
+static bool g_randk_ahead = true;  // run the next step's key pass ahead (see gce.h)
+
 struct RkSeg {
     int32_t k;       // 0: layer skipped
     uint32_t lo, hi; // band of candidate keys
@@ -63,7 +65,7 @@ static RkLayout rk_layout(const gce_table* t, int32_t W) {
     const bool on = t->ckind == GCE_KIND_RANDK;
     o.S = on ? int64_t(W) * int64_t(t->comp.size()) : 0;
     o.TT = on ? int64_t(W) * t->tiles_pw : 0;
-    o.segs = c.take<RkSeg>(o.S);
+    o.segs = c.take<RkSeg>(2 * o.S);  // two sets: this step's and the next one's
     o.tile_cnt = c.take<int32_t>(o.TT);
     o.bitmask = c.take<uint32_t>(o.TT * kRkWords);
     o.cand = c.take<RkEntry>(o.S ? int64_t(W) * t->comp_N : 0);
@@ -73,39 +75,112 @@ static RkLayout rk_layout(const gce_table* t, int32_t W) {
 
 size_t randk_ws_bytes(const gce_table* t, int32_t W) { return rk_layout(t, W).total; }
 
+// State of (worker, layer) segment s for `step`: k (0 when out of range),
+// the band [lo, hi] of +-(sigma * binomial sd + sigma) keys around the
+// expected k-th smallest key, the generator state, counters at zero.
+__device__ __forceinline__ void rk_setup_seg(int64_t s, const DevLayer* __restrict__ layers,
+                                             const int32_t* __restrict__ comp, int32_t ncomp,
+                                             const int32_t* __restrict__ k_or_rank, uint64_t seed,
+                                             uint64_t step, double sigma, RkSeg* __restrict__ segs,
+                                             int32_t* __restrict__ status) {
+    const int32_t l = comp[s % ncomp];
+    const DevLayer L = layers[l];
+    const int32_t k = k_or_rank ? k_or_rank[l] : L.cap;
+    RkSeg g{};
+    if (k >= 1 && k <= L.cap && int64_t(k) <= L.n) {
+        g.k = k;
+    } else {
+        g.k = 0;
+        if (status) set_status(status, GCE_STATUS_K_RANGE);
+    }
+    const double n = double(L.n), p = double(k) / n;
+    const double d = sigma * (sqrt(n * p * (1.0 - p)) + 1.0);
+    const double scale = 4294967296.0 / n;
+    const double lo = (double(k) - d) * scale, hi = (double(k) + d) * scale;
+    g.lo = lo <= 0.0 ? 0u : (lo >= 4294967295.0 ? 0xFFFFFFFFu : uint32_t(lo));
+    g.hi = hi >= 4294967295.0 ? 0xFFFFFFFFu : (hi <= 0.0 ? 0u : uint32_t(hi));
+    if (g.hi < g.lo) g.hi = g.lo;
+    g.base = hash_base(seed, 0, uint64_t(s / ncomp), uint64_t(l), step);
+    segs[s] = g;
+}
+
+// tag: where the workspace records which step's key pass it holds; block 0
+// writes tag_value there (0: none).
 __global__ void __launch_bounds__(256) rk_setup_kernel(const DevLayer* __restrict__ layers,
                                                        const int32_t* __restrict__ comp,
                                                        int32_t ncomp, int64_t S,
                                                        const int32_t* __restrict__ k_or_rank,
                                                        uint64_t seed, uint64_t step, double sigma,
                                                        RkSeg* __restrict__ segs,
-                                                       int32_t* __restrict__ status) {
+                                                       int32_t* __restrict__ status,
+                                                       uint64_t* __restrict__ tag,
+                                                       uint64_t tag_value) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tag = tag_value;
     for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
-         s += int64_t(gridDim.x) * blockDim.x) {
-        const int32_t l = comp[s % ncomp];
-        const DevLayer L = layers[l];
-        const int32_t k = k_or_rank ? k_or_rank[l] : L.cap;
-        RkSeg g{};
-        if (k >= 1 && k <= L.cap && int64_t(k) <= L.n) {
-            g.k = k;
-        } else {
-            g.k = 0;
-            set_status(status, GCE_STATUS_K_RANGE);
+         s += int64_t(gridDim.x) * blockDim.x)
+        rk_setup_seg(s, layers, comp, ncomp, k_or_rank, seed, step, sigma, segs, status);
+}
+
+// Key pass over one tile t (worker w, layer L): the bitmask words of key < lo,
+// the tile's count below lo and the band entries [lo, hi] appended to the
+// layer's list.  kRedo: re-list a failed layer whole (band = every key,
+// nothing below it).  Run by the whole block; g.k != 0.
+template <bool kRedo>
+__device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const DevLayer& L,
+                                             RkSeg& g, int64_t comp_N, int32_t* tile_cnt,
+                                             uint32_t* bitmask, RkEntry* cand, int* s_red) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const uint32_t lo = kRedo ? 0u : g.lo, hi = kRedo ? 0xFFFFFFFFu : g.hi;
+    const uint64_t base = g.base;
+    const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
+    const int64_t e0 = tstart + int64_t(tid) * 32;
+    const uint64_t x0 = base + uint64_t(e0 + 1) * kGamma;  // generator state of element e0
+    uint32_t below = 0, inband = 0;
+    if (e0 + 32 <= L.n) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+            below |= uint32_t(key < lo) << q;
+            inband |= uint32_t(key >= lo && key <= hi) << q;
         }
-        // band: k -+ (sigma * binomial sd + sigma) keys around the expected position
-        const double n = double(L.n), p = double(k) / n;
-        const double d = sigma * (sqrt(n * p * (1.0 - p)) + 1.0);
-        const double scale = 4294967296.0 / n;
-        const double lo = (double(k) - d) * scale, hi = (double(k) + d) * scale;
-        g.lo = lo <= 0.0 ? 0u : (lo >= 4294967295.0 ? 0xFFFFFFFFu : uint32_t(lo));
-        g.hi = hi >= 4294967295.0 ? 0xFFFFFFFFu : (hi <= 0.0 ? 0u : uint32_t(hi));
-        if (g.hi < g.lo) g.hi = g.lo;
-        g.base = hash_base(seed, 0, uint64_t(s / ncomp), uint64_t(l), step);
-        segs[s] = g;
+    } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+            if (e0 + q < L.n) {
+                below |= uint32_t(key < lo) << q;
+                inband |= uint32_t(key >= lo && key <= hi) << q;
+            }
+        }
+    }
+    bitmask[t * kRkWords + tid] = below;
+    // tile count of keys below the band
+    const int c = warp_sum(__popc(below));
+    if (lane == 0) s_red[warp] = c;
+    __syncthreads();
+    if (tid == 0) {
+        int tot = 0;
+        for (int i = 0; i < 8; ++i) tot += s_red[i];
+        tile_cnt[t] = tot;
+        if (tot) atomicAdd(&g.c_lo, tot);
+    }
+    __syncthreads();
+    // band entries: order does not matter, the resolve sorts them out
+    const int nb = __popc(inband);
+    const int incl = warp_inclusive_scan(nb);
+    int wbase = 0;
+    if (lane == 31 && incl) wbase = atomicAdd(kRedo ? &g.cand_redo : &g.cand, incl);
+    wbase = __shfl_sync(kFull, wbase, 31);
+    RkEntry* out = cand + int64_t(w) * comp_N + L.sp_off + wbase + (incl - nb);
+    int pos = 0;
+    while (inband) {  // few band entries: their keys are recomputed
+        const int q = __ffs(inband) - 1;
+        inband &= inband - 1;
+        const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+        out[pos++] = RkEntry{key, int32_t(e0 + q)};
     }
 }
 
-// kRedo: re-list a failed layer whole (band = every key, nothing below it).
 template <bool kRedo>
 __global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict__ layers,
                                                       const int32_t* __restrict__ tile_layer,
@@ -115,55 +190,48 @@ __global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict
                                                       uint32_t* __restrict__ bitmask,
                                                       RkEntry* __restrict__ cand) {
     __shared__ int s_red[8];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t total = int64_t(tiles_pw) * W;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
         const DevLayer L = layers[tile_layer[lt]];
-        const int64_t s = int64_t(w) * ncomp + L.sidx;
-        RkSeg& g = segs[s];
+        RkSeg& g = segs[int64_t(w) * ncomp + L.sidx];
         if (g.k == 0) continue;
         if (kRedo && !g.fail) continue;
-        const uint32_t lo = kRedo ? 0u : g.lo, hi = kRedo ? 0xFFFFFFFFu : g.hi;
-        const uint64_t base = g.base;
-        const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
-        const int64_t e0 = tstart + int64_t(tid) * 32;
-        const uint64_t x0 = base + uint64_t(e0 + 1) * kGamma;  // generator state of element e0
-        uint32_t below = 0, inband = 0;
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
-            if (e0 + q < L.n) {
-                below |= uint32_t(key < lo) << q;
-                inband |= uint32_t(key >= lo && key <= hi) << q;
-            }
+        rk_keys_tile<kRedo>(t, w, lt, L, g, comp_N, tile_cnt, bitmask, cand, s_red);
+    }
+}
+
+// The k of every (worker, layer) read again for this step (the key pass run
+// ahead used the k of the step before, which only sized its band: a band
+// that misses the new k-th key sends the layer to the exact fallback).  If
+// the workspace does not hold the expected step's key pass (its tag
+// differs), every segment is set up afresh and sent to the exact fallback.
+__global__ void __launch_bounds__(256) rk_refresh_k_kernel(const DevLayer* __restrict__ layers,
+                                                           const int32_t* __restrict__ comp,
+                                                           int32_t ncomp, int64_t S,
+                                                           const int32_t* __restrict__ k_or_rank,
+                                                           uint64_t seed, uint64_t step,
+                                                           double sigma, RkSeg* __restrict__ segs,
+                                                           int32_t* __restrict__ status,
+                                                           const uint64_t* __restrict__ tag,
+                                                           uint64_t tag_value) {
+    const bool held = *tag == tag_value;
+    for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
+         s += int64_t(gridDim.x) * blockDim.x) {
+        if (!held) {
+            rk_setup_seg(s, layers, comp, ncomp, k_or_rank, seed, step, sigma, segs, status);
+            segs[s].fail = 1;
+            continue;
         }
-        bitmask[t * kRkWords + tid] = below;
-        // tile count of keys below the band
-        int c = warp_sum(__popc(below));
-        if (lane == 0) s_red[warp] = c;
-        __syncthreads();
-        if (tid == 0) {
-            int tot = 0;
-            for (int i = 0; i < 8; ++i) tot += s_red[i];
-            tile_cnt[t] = tot;
-            if (tot) atomicAdd(&g.c_lo, tot);
-        }
-        __syncthreads();
-        // band entries: order does not matter, the resolve sorts them out
-        const int nb = __popc(inband);
-        const int incl = warp_inclusive_scan(nb);
-        int wbase = 0;
-        if (lane == 31 && incl) wbase = atomicAdd(kRedo ? &g.cand_redo : &g.cand, incl);
-        wbase = __shfl_sync(kFull, wbase, 31);
-        RkEntry* out = cand + int64_t(w) * comp_N + L.sp_off + wbase + (incl - nb);
-        int pos = 0;
-        while (inband) {  // few band entries: their keys are recomputed
-            const int q = __ffs(inband) - 1;
-            inband &= inband - 1;
-            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
-            out[pos++] = RkEntry{key, int32_t(e0 + q)};
+        const int32_t l = comp[s % ncomp];
+        const DevLayer L = layers[l];
+        const int32_t k = k_or_rank ? k_or_rank[l] : L.cap;
+        if (k >= 1 && k <= L.cap && int64_t(k) <= L.n) {
+            segs[s].k = k;
+        } else {
+            segs[s].k = 0;
+            set_status(status, GCE_STATUS_K_RANGE);
         }
     }
 }
@@ -320,15 +388,23 @@ __global__ void __launch_bounds__(1024) rk_scan_kernel(const DevLayer* __restric
     }
 }
 
+// kNext: once a tile's memory pass is done, the block also runs the next
+// step's key pass over the same tile (segs_next): ALU work that overlaps the
+// other blocks' memory traffic.  The tile's bitmask words and offset are read
+// before the block's barriers and rewritten after them, by the same block.
+template <bool kNext>
 __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
-    int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, const float* __restrict__ grad,
-    float* __restrict__ mem, float eta, const RkSeg* __restrict__ segs,
-    const int32_t* __restrict__ tile_off, const uint32_t* __restrict__ bitmask,
-    float* __restrict__ vals, int32_t* __restrict__ idx) {
+    int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, int64_t comp_N,
+    const float* __restrict__ grad, float* __restrict__ mem, float eta,
+    const RkSeg* __restrict__ segs, RkSeg* __restrict__ segs_next, int32_t* tile_off,
+    uint32_t* bitmask, RkEntry* __restrict__ cand, float* __restrict__ vals,
+    int32_t* __restrict__ idx) {
     constexpr int kIters = kTkPerThread / 4;
     constexpr int kWarps = kTkThreads / 32;
     __shared__ int32_t s_wt[kIters * kWarps];
+    __shared__ int s_red[8];
+    __shared__ int32_t s_toff;  // this tile's first payload slot
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t total = int64_t(tiles_pw) * W;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
@@ -350,87 +426,96 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
         }
         const int64_t s = int64_t(w) * ncomp + L.sidx;
         const int32_t k = segs[s].k;
-        if (k == 0) continue;
+        const bool next = kNext && segs_next[s].k != 0;
+        if (k == 0 && !next) continue;
         const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
         const int cnt = int(min64(kTkTile, L.n - tstart));
         const int64_t ebase = int64_t(w) * N + L.offset + tstart;
         const float* g = grad + ebase;
         float* m = mem + ebase;
         const uint32_t* bm = bitmask + t * kRkWords;
-        uint32_t flags = 0;
         const bool vec = cnt == kTkTile && (ebase & 3) == 0;
-        // every load of the tile issued up front, then the arithmetic; the
-        // memory first receives v everywhere, and the few chosen entries are
-        // read back and zeroed once their payload slots are known
-        uint32_t words[kIters];
+        if (k != 0) {
+            // every load of the tile issued up front, then the arithmetic; the
+            // memory first receives v everywhere, and the few chosen entries
+            // are read back and zeroed once their payload slots are known
+            uint32_t words[kIters];
 #pragma unroll
-        for (int j = 0; j < kIters; ++j) words[j] = __ldcg(bm + ((j * (kTkThreads * 4) + tid * 4) >> 5));
-        if (vec) {
-            float4 gv[kIters], mv[kIters];
+            for (int j = 0; j < kIters; ++j)
+                words[j] = __ldcg(bm + ((j * (kTkThreads * 4) + tid * 4) >> 5));
+            if (tid == 0) s_toff = tile_off[t];
+            if (vec) {
+                float4 gv[kIters], mv[kIters];
+#pragma unroll
+                for (int j = 0; j < kIters; ++j) {
+                    const int e = j * (kTkThreads * 4) + tid * 4;
+                    gv[j] = ld_stream4(g + e);
+                    mv[j] = ld_stream4(m + e);
+                }
+#pragma unroll
+                for (int j = 0; j < kIters; ++j) {
+                    const int e = j * (kTkThreads * 4) + tid * 4;
+                    float4 x;
+                    x.x = residual(mv[j].x, eta, gv[j].x);
+                    x.y = residual(mv[j].y, eta, gv[j].y);
+                    x.z = residual(mv[j].z, eta, gv[j].z);
+                    x.w = residual(mv[j].w, eta, gv[j].w);
+                    *reinterpret_cast<float4*>(m + e) = x;
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < kIters; ++j) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int e = j * (kTkThreads * 4) + tid * 4 + q;
+                        if (e < cnt) m[e] = residual(m[e], eta, __ldcs(g + e));
+                    }
+                }
+            }
+            uint32_t flags = 0;
 #pragma unroll
             for (int j = 0; j < kIters; ++j) {
                 const int e = j * (kTkThreads * 4) + tid * 4;
-                gv[j] = ld_stream4(g + e);
-                mv[j] = ld_stream4(m + e);
+                flags |= ((words[j] >> (e & 31)) & 0xFu) << (4 * j);
             }
+            int incl[kIters];
 #pragma unroll
             for (int j = 0; j < kIters; ++j) {
-                const int e = j * (kTkThreads * 4) + tid * 4;
-                float4 x;
-                x.x = residual(mv[j].x, eta, gv[j].x);
-                x.y = residual(mv[j].y, eta, gv[j].y);
-                x.z = residual(mv[j].z, eta, gv[j].z);
-                x.w = residual(mv[j].w, eta, gv[j].w);
-                *reinterpret_cast<float4*>(m + e) = x;
+                incl[j] = warp_inclusive_scan(__popc((flags >> (4 * j)) & 0xFu));
+                if (lane == 31) s_wt[j * kWarps + warp] = incl[j];
             }
-        } else {
+            __syncthreads();
+            if (warp == 0) {
+                const int a = s_wt[2 * lane], b = s_wt[2 * lane + 1];
+                const int x = warp_inclusive_scan(a + b);
+                s_wt[2 * lane] = x - a - b;
+                s_wt[2 * lane + 1] = x - b;
+            }
+            __syncthreads();
+            const int base = s_toff;
+            float* vout = vals + int64_t(w) * vals_pw + L.val_off;
+            int32_t* iout = idx + int64_t(w) * vals_pw + L.val_off;
 #pragma unroll
             for (int j = 0; j < kIters; ++j) {
+                const uint32_t f = (flags >> (4 * j)) & 0xFu;
+                int pos = base + s_wt[j * kWarps + warp] + incl[j] - __popc(f);
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const int e = j * (kTkThreads * 4) + tid * 4 + q;
-                    if (e < cnt) m[e] = residual(m[e], eta, __ldcs(g + e));
+                    if ((f & (1u << q)) && pos < k) {
+                        const int e = j * (kTkThreads * 4) + tid * 4 + q;
+                        vout[pos] = m[e];
+                        iout[pos] = int32_t(tstart + e);
+                        m[e] = 0.0f;
+                    }
+                    pos += (f >> q) & 1u;
                 }
             }
+            __syncthreads();  // words, s_wt and s_toff are consumed
         }
-#pragma unroll
-        for (int j = 0; j < kIters; ++j) {
-            const int e = j * (kTkThreads * 4) + tid * 4;
-            flags |= ((words[j] >> (e & 31)) & 0xFu) << (4 * j);
-        }
-        int incl[kIters];
-#pragma unroll
-        for (int j = 0; j < kIters; ++j) {
-            incl[j] = warp_inclusive_scan(__popc((flags >> (4 * j)) & 0xFu));
-            if (lane == 31) s_wt[j * kWarps + warp] = incl[j];
-        }
-        __syncthreads();
-        if (warp == 0) {
-            const int a = s_wt[2 * lane], b = s_wt[2 * lane + 1];
-            const int x = warp_inclusive_scan(a + b);
-            s_wt[2 * lane] = x - a - b;
-            s_wt[2 * lane + 1] = x - b;
-        }
-        __syncthreads();
-        const int base = tile_off[t];
-        float* vout = vals + int64_t(w) * vals_pw + L.val_off;
-        int32_t* iout = idx + int64_t(w) * vals_pw + L.val_off;
-#pragma unroll
-        for (int j = 0; j < kIters; ++j) {
-            const uint32_t f = (flags >> (4 * j)) & 0xFu;
-            int pos = base + s_wt[j * kWarps + warp] + incl[j] - __popc(f);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                if ((f & (1u << q)) && pos < k) {
-                    const int e = j * (kTkThreads * 4) + tid * 4 + q;
-                    vout[pos] = m[e];
-                    iout[pos] = int32_t(tstart + e);
-                    m[e] = 0.0f;
-                }
-                pos += (f >> q) & 1u;
-            }
-        }
-        __syncthreads();
+        // the next step's key pass over the same tile: ALU work while the
+        // other resident blocks stream memory
+        if (next)
+            rk_keys_tile<false>(t, w, lt, L, segs_next[s], comp_N, tile_off, bitmask, cand, s_red);
     }
 }
 
@@ -453,22 +538,52 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
     int32_t* status = static_cast<int32_t*>(ws);
     if (lay.S > 0) {
         const int32_t ncomp = int32_t(t->comp.size());
-        RkSeg* segs = at<RkSeg>(ws, lay.segs);
         int32_t* tile_cnt = at<int32_t>(ws, lay.tile_cnt);
         uint32_t* bitmask = at<uint32_t>(ws, lay.bitmask);
         RkEntry* cand = at<RkEntry>(ws, lay.cand);
+        // Run the next step's key pass inside this step's memory pass unless
+        // the stream is being captured (a graph would replay one step number).
+        cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+        if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GCE_ERR_CUDA;
+        const bool pipe = g_randk_ahead && cs == cudaStreamCaptureStatusNone &&
+                          step != ~uint64_t(0);
+        bool have = false;
+        {
+            std::lock_guard<std::mutex> lk(t->rk_mu);
+            have = pipe && t->rk_valid && t->rk_ws == ws && t->rk_seed == seed &&
+                   t->rk_step == step && t->rk_W == W;
+            t->rk_valid = false;
+        }
+        // which step's key pass the workspace holds (header bytes 64-71)
+        uint64_t* tag = at<uint64_t>(ws, 64);
+        auto tag_of = [&](uint64_t sv) {
+            const uint64_t h = mix64(mix64(mix64(seed + kGamma) + sv) + uint64_t(W)) ^
+                               reinterpret_cast<uintptr_t>(t);
+            return h ? h : 1u;
+        };
+        RkSeg* segs = at<RkSeg>(ws, lay.segs) + (step & 1) * lay.S;
+        RkSeg* segs_next = at<RkSeg>(ws, lay.segs) + ((step + 1) & 1) * lay.S;
         static const int r_setup = resident_blocks(rk_setup_kernel, 256);
+        static const int r_refresh = resident_blocks(rk_refresh_k_kernel, 256);
         static const int r_keys0 = resident_blocks(rk_keys_kernel<false>, 256);
         static const int r_keys1 = resident_blocks(rk_keys_kernel<true>, 256);
         static const int r_res0 = resident_blocks(rk_resolve_kernel<false>, 1024);
         static const int r_res1 = resident_blocks(rk_resolve_kernel<true>, 1024);
         static const int r_scan = resident_blocks(rk_scan_kernel, 1024);
-        static const int r_emit = resident_blocks(rk_emit_kernel, kTkThreads);
-        GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st, t->d_layers,
-                   t->d_comp, ncomp, lay.S, k_or_rank, seed, step, bracket_sigma(), segs, status);
-        GCE_LAUNCH(rk_keys_kernel<false>, wave_grid(lay.TT, 8, r_keys0), 256, 0, st, t->d_layers,
-                   t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs, tile_cnt, bitmask,
-                   cand);
+        static const int r_emit0 = resident_blocks(rk_emit_kernel<false>, kTkThreads);
+        static const int r_emit1 = resident_blocks(rk_emit_kernel<true>, kTkThreads);
+        if (have) {
+            GCE_LAUNCH(rk_refresh_k_kernel, wave_grid((lay.S + 255) / 256, 4, r_refresh), 256, 0,
+                       st, t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed, step,
+                       bracket_sigma(), segs, status, tag, tag_of(step));
+        } else {
+            GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st,
+                       t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed, step,
+                       bracket_sigma(), segs, status, tag, uint64_t(0));
+            GCE_LAUNCH(rk_keys_kernel<false>, wave_grid(lay.TT, 8, r_keys0), 256, 0, st,
+                       t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs,
+                       tile_cnt, bitmask, cand);
+        }
         GCE_LAUNCH(rk_resolve_kernel<false>, wave_grid(lay.S, 2, r_res0), 1024, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, bitmask, cand,
                    status);
@@ -478,12 +593,39 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
         GCE_LAUNCH(rk_resolve_kernel<true>, wave_grid(lay.S, 2, r_res1), 1024, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, bitmask, cand,
                    status);
-        GCE_LAUNCH(rk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
-                   lay.S, t->tiles_pw, segs, tile_cnt);
-        GCE_LAUNCH(rk_emit_kernel, wave_grid(lay.TT, r_emit, r_emit), kTkThreads, 0, st, t->d_layers,
-                   t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw, grad, mem, eta, segs,
-                   tile_cnt, bitmask, vals, idx);
+        GCE_LAUNCH(rk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp,
+                   ncomp, lay.S, t->tiles_pw, segs, tile_cnt);
+        if (pipe) {
+            // the next step's band from this step's k (a guess: the exact
+            // resolve of that step re-reads k and repairs any miss)
+            GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st,
+                       t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed, step + 1,
+                       bracket_sigma(), segs_next, nullptr, tag, tag_of(step + 1));
+            GCE_LAUNCH(rk_emit_kernel<true>, wave_grid(lay.TT, r_emit1, r_emit1), kTkThreads, 0, st,
+                       t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
+                       t->comp_N, grad, mem, eta, segs, segs_next, tile_cnt, bitmask, cand, vals,
+                       idx);
+        } else {
+            GCE_LAUNCH(rk_emit_kernel<false>, wave_grid(lay.TT, r_emit0, r_emit0), kTkThreads, 0,
+                       st, t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
+                       t->comp_N, grad, mem, eta, segs, nullptr, tile_cnt, bitmask, cand, vals,
+                       idx);
+        }
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+        if (pipe) {
+            std::lock_guard<std::mutex> lk(t->rk_mu);
+            t->rk_ws = ws;
+            t->rk_seed = seed;
+            t->rk_step = step + 1;
+            t->rk_W = W;
+            t->rk_valid = true;
+        }
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+}
+
+extern "C" int gce_set_randk_ahead(int32_t on) {
+    if (on != 0 && on != 1) return GCE_ERR_ARG;
+    g_randk_ahead = on != 0;
+    return GCE_OK;
 }

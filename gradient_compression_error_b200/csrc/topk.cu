@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(256) tk_respill_kernel(
 
 // ---- radix levels over the candidate values --------------------------------------------
 template <int kLevel>
-__global__ void __launch_bounds__(256) tk_hist_kernel(const DevLayer* __restrict__ layers,
+__global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restrict__ layers,
                                                       const int32_t* __restrict__ comp,
                                                       int32_t ncomp, int64_t S, int64_t comp_N,
                                                       TkSeg* __restrict__ segs,
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(256) tk_hist_kernel(const DevLayer* __restrict
                                                       const float* __restrict__ spill_v) {
     constexpr int kNb = kLevel == 3 ? 512 : kTkBins;
     constexpr int kShift = kLevel == 1 ? 20 : (kLevel == 2 ? 9 : 0);
-    constexpr int kPer = 32;  // candidates per thread per load batch
+    constexpr int kPer = 16;  // candidates per thread per load batch
     __shared__ int32_t h[kTkBins];
     __shared__ int s_last;
     const int tid = threadIdx.x;

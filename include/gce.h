@@ -174,6 +174,21 @@ GCE_API int ef_randk_step(const gce_table* table, int32_t W, const float* grad, 
                   float* vals, int32_t* idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * rand-k look-ahead (on by default; the pages have no counterpart: it only
+ * moves work).  The chosen set does not depend on the data, so while a step's
+ * memory pass streams grad and mem, ef_randk_step also hashes the next step's
+ * keys (step + 1, same seed, W and table, with this step's k sizing the
+ * band) into its workspace.  The next call with the same table, workspace,
+ * seed, W and step + 1 skips its own key pass.  Results never depend on it:
+ * that call re-reads k, repairs a band the new k misses exactly, and checks a
+ * tag in the workspace header, recomputing everything if another step's pass
+ * is there.  Between the two calls nothing else may write the workspace.
+ * Off while the stream is being captured into a graph.  on: 1 or 0; other
+ * values give GCE_ERR_ARG.
+ */
+GCE_API int gce_set_randk_ahead(int32_t on);
+
+/*
  * Initial (warm-start) Q for every (worker, POWERSGD layer): entries
  * (h >> 40) * 2^-23 - 1 in [-1, 1), h the SplitMix64 output c*r_max + j + 1
  * from the state of (seed, stream 1, worker, layer, step 0).  Q: [W][Q_per_worker].

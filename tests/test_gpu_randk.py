@@ -15,7 +15,9 @@ from tests.helpers import bits, gce, host, layer_slice, need_gpu, payload_slice,
 pytestmark = pytest.mark.gpu
 
 
-def run_randk(layers, W, T, seed, make_grad, eta=0.05, k_fn=None):
+def run_randk(layers, W, T, seed, make_grad, eta=0.05, k_fn=None, steps=None, between=None):
+    """T steps (or the given step numbers) against the oracle; between(ws)
+    runs after every step."""
     g = gce()
     t = g.Table(workloads.table_layers(layers))
     mem = torch.zeros((W, t.N), device="cuda")
@@ -23,7 +25,7 @@ def run_randk(layers, W, T, seed, make_grad, eta=0.05, k_fn=None):
     idx = torch.zeros((W, max(4, t.vals_per_worker)), dtype=torch.int32, device="cuda")
     ws = t.workspace(W, "randk")
     hmem = np.zeros((W, t.N), np.float32)
-    for step in range(T):
+    for step in (range(T) if steps is None else steps):
         grad = make_grad(step)
         ks = [l["cap"] for l in layers] if k_fn is None else k_fn(step)
         kt = None if k_fn is None else torch.tensor(ks, dtype=torch.int32, device="cuda")
@@ -41,6 +43,8 @@ def run_randk(layers, W, T, seed, make_grad, eta=0.05, k_fn=None):
                 assert np.array_equal(bits(hv[w, sl]), bits(e[0])), ("vals", step, w, l)
             ls = layer_slice(t, l)
             assert np.array_equal(bits(hm[w, ls]), bits(hmem[w, ls])), ("mem", step, w, l)
+        if between is not None:
+            between(ws)
     return g, ws
 
 
@@ -63,6 +67,39 @@ def test_k_changes_between_steps():
     ks = [[10000], [1000], [1]]
     run_randk(layers, 1, 3, 7, lambda s: workloads.gradients(layers, 1, 202, s),
               k_fn=lambda s: ks[s])
+
+
+def test_look_ahead_on_and_off_and_skipped_steps():
+    """The next step's key pass run inside this step's memory pass gives the
+    same bits as running it in its own step: consecutive steps use it, a
+    jump in the step number or a different seed does not."""
+    need_gpu()
+    g = gce()
+    mk = lambda s: workloads.gradients(LAYERS, 2, 204, s)
+    run_randk(LAYERS, 2, 0, 31, mk, steps=[0, 1, 2, 5, 6, 9])
+    try:
+        g.set_randk_ahead(False)
+        run_randk(LAYERS, 2, 0, 31, mk, steps=[0, 1, 2, 5, 6, 9])
+    finally:
+        g.set_randk_ahead(True)
+
+
+def test_look_ahead_survives_a_cleared_workspace():
+    """A workspace wiped between two consecutive steps (as a fresh allocation at
+    the same address would be) no longer holds the key pass: the tag check
+    sends every layer to the exact fallback and the result stays exact."""
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=300017, cols=1, kind="randk", cap=3000, sigma=1.0),
+              dict(rows=70000, cols=1, kind="randk", cap=700, sigma=1.0)]
+    seen = []
+
+    def wipe(ws):
+        seen.append(g.status(ws))
+        ws.zero_()
+
+    run_randk(layers, 2, 3, 77, lambda s: workloads.gradients(layers, 2, 205, s), between=wipe)
+    assert seen[1] & g.STATUS_FALLBACK and seen[2] & g.STATUS_FALLBACK
 
 
 def test_forced_fallback_is_still_exact():
