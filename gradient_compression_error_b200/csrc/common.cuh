@@ -228,6 +228,23 @@ __host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
     return z ^ (z >> 31);
 }
 
+// The high 32 bits of mix64(z), forming only the high word of the last
+// product (the same value: the final xor-shift moves bit 63 into bit 32
+// and leaves the high word otherwise as it is).
+__host__ __device__ __forceinline__ uint32_t mix64_hi(uint64_t z) {
+    const uint64_t y0 = z ^ (z >> 30);
+    const uint64_t z1 = y0 * 0xBF58476D1CE4E5B9ull;
+    const uint64_t y1 = z1 ^ (z1 >> 27);
+    const uint32_t lo = uint32_t(y1), hi = uint32_t(y1 >> 32);
+    constexpr uint32_t c_lo = 0x133111EBu, c_hi = 0x94D049BBu;
+#ifdef __CUDA_ARCH__
+    const uint32_t h = __umulhi(lo, c_lo) + lo * c_hi + hi * c_lo;
+#else
+    const uint32_t h = uint32_t((uint64_t(lo) * c_lo) >> 32) + lo * c_hi + hi * c_lo;
+#endif
+    return h ^ (h >> 31);
+}
+
 // state of (seed, stream, worker, layer, step): each field folded in as the
 // first SplitMix64 output from (previous + (field + 1) * gamma)
 __host__ __device__ __forceinline__ uint64_t hash_base(uint64_t seed, uint64_t stream,

@@ -131,6 +131,7 @@ __device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const Dev
                                              uint32_t* bitmask, RkEntry* cand, int* s_red) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const uint32_t lo = kRedo ? 0u : g.lo, hi = kRedo ? 0xFFFFFFFFu : g.hi;
+    const uint32_t span = hi - lo;  // lo <= key <= hi  iff  key - lo <= hi - lo (unsigned)
     const uint64_t base = g.base;
     const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
     const int64_t e0 = tstart + int64_t(tid) * 32;
@@ -139,17 +140,17 @@ __device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const Dev
     if (e0 + 32 <= L.n) {
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+            const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
             below |= uint32_t(key < lo) << q;
-            inband |= uint32_t(key >= lo && key <= hi) << q;
+            inband |= uint32_t(key - lo <= span) << q;
         }
     } else {
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-            const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+            const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
             if (e0 + q < L.n) {
                 below |= uint32_t(key < lo) << q;
-                inband |= uint32_t(key >= lo && key <= hi) << q;
+                inband |= uint32_t(key - lo <= span) << q;
             }
         }
     }
@@ -176,7 +177,7 @@ __device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const Dev
     while (inband) {  // few band entries: their keys are recomputed
         const int q = __ffs(inband) - 1;
         inband &= inband - 1;
-        const uint32_t key = uint32_t(mix64(x0 + uint64_t(q) * kGamma) >> 32);
+        const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
         out[pos++] = RkEntry{key, int32_t(e0 + q)};
     }
 }
