@@ -291,6 +291,9 @@ def main():
     ap.add_argument("--profile", action="store_true", help="per-kernel table on stderr")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step as a CUDA graph (workloads whose step takes no "
+                         "per-step host values: top-k, sign, PowerSGD without Accordion)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -390,6 +393,24 @@ def main():
     if gce.status(ws) & gce.STATUS_K_RANGE:
         raise SystemExit("device status reports an out-of-range k")
 
+    # CUDA-graph replay: one graph per gradient buffer, captured after the
+    # warm-up; the kernels and their arguments are those of the eager step
+    graphs, launches_per_step = None, None
+    if args.graph:
+        if method == "randk" or kr is not None or apply:
+            raise SystemExit("--graph: this workload's step takes per-step host values")
+        graphs = []
+        for b in range(2):
+            gr = torch.cuda.CUDAGraph()
+            l_before = gce.launch_count()
+            with torch.cuda.graph(gr):
+                step(0, grads[b])
+            launches_per_step = gce.launch_count() - l_before
+            graphs.append(gr)
+        for s in range(3):
+            graphs[s % 2].replay()
+        torch.cuda.synchronize()
+
     clocks = ClockSampler(torch.cuda.current_device())
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -397,14 +418,30 @@ def main():
     clocks.start()
     time.sleep(0.2)
     l0 = gce.launch_count()
+    # events around the main pass only (every kernel with --profile)
+    gce.profile_only(None if args.profile else MAIN_KERNELS[method])
     gce.profile_start()
     ev0.record()
     for s in range(args.steps):
-        step(args.warmup + s, grads[s % 2])
+        if graphs:
+            graphs[s % 2].replay()
+        else:
+            step(args.warmup + s, grads[s % 2])
     ev1.record()
     torch.cuda.synchronize()
     prof = gce.profile_stop()
     launches = gce.launch_count() - l0
+    if graphs:
+        # replays launch nothing from the host: the captured kernels per step;
+        # the main-pass time comes from a short eager pass right after
+        launches = launches_per_step * args.steps
+        gce.profile_start()
+        for s in range(min(args.steps, 20)):
+            step(args.warmup + s, grads[s % 2])
+        torch.cuda.synchronize()
+        prof = gce.profile_stop()
+        prof = {k: (v[0] * args.steps / min(args.steps, 20), v[1] * args.steps // min(args.steps, 20))
+                for k, v in prof.items()}
     barrier()
     clk = clocks.stop()
     t_ms = max_over_ranks(ev0.elapsed_time(ev1))
@@ -496,6 +533,8 @@ def main():
                            "eta": "8/(1*(160+t))" if apply else wl.ETA,
                            "update": "x -= mean of payloads (fused)" if apply else "decode only",
                            "parallelism": "replicas x%d" % world,
+                           "launch": ("CUDA graph replay (main-pass time from 20 eager steps)"
+                                      if graphs else "eager"),
                            "l2": "inputs larger than L2 (%.1f GB of grad+memory per step)"
                                  % (8.0 * W * N / 1e9),
                            "step_algorithmic_GBps": step_gbs,

@@ -88,6 +88,7 @@ SIGNATURES = {
     "gce_set_randk_ahead": (C.c_int, [C.c_int32]),
     "gce_profile_start": (C.c_int, []),
     "gce_profile_stop": (C.c_int, []),
+    "gce_profile_only": (C.c_int, [C.c_char_p]),
     "gce_profile_count": (C.c_int, []),
     "gce_profile_get": (C.c_int, [_i32, C.c_char_p, _i32, C.POINTER(_f64), C.POINTER(_i64)]),
 }
@@ -300,6 +301,12 @@ def launch_count():
 
 def profile_start():
     _check("gce_profile_start", lib().gce_profile_start())
+
+
+def profile_only(name_prefix=None):
+    """Record only kernels whose name starts with name_prefix (None: all)."""
+    _check("gce_profile_only", lib().gce_profile_only(
+        None if name_prefix is None else name_prefix.encode()))
 
 
 def profile_stop():

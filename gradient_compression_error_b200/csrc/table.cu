@@ -29,6 +29,7 @@ struct ProfAgg {
     int64_t n;
 };
 std::vector<ProfAgg> g_prof_agg;
+std::string g_prof_only;  // record only kernels whose name starts with this (empty: all)
 
 cudaEvent_t prof_event() {
     if (g_prof_used < g_prof_pool.size()) return g_prof_pool[g_prof_used++];
@@ -43,6 +44,8 @@ cudaEvent_t prof_event() {
 void prof_before(const char* name, cudaStream_t st) {
     std::lock_guard<std::mutex> lk(g_prof_mu);
     if (g_prof_recs.size() >= kProfMax) return;
+    if (!g_prof_only.empty() && std::strncmp(name, g_prof_only.c_str(), g_prof_only.size()) != 0)
+        return;
     ProfRec r{name, prof_event(), nullptr};
     if (!r.a) return;
     cudaEventRecord(r.a, st);
@@ -346,6 +349,12 @@ extern "C" int gce_profile_start(void) {
     g_prof_agg.clear();
     g_prof_used = 0;
     g_prof_on.store(true);
+    return GCE_OK;
+}
+
+extern "C" int gce_profile_only(const char* name_prefix) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof_only = name_prefix ? name_prefix : "";
     return GCE_OK;
 }
 

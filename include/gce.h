@@ -360,6 +360,10 @@ GCE_API uint64_t gce_launch_count(void);
  * bookkeeping only; the kernels themselves are unchanged. */
 GCE_API int gce_profile_start(void);
 GCE_API int gce_profile_stop(void);
+/* Restrict the recording to launches whose kernel name starts with
+ * name_prefix (host string, copied); NULL or "" records every launch.  Fewer
+ * events in the timed stream when only one kernel's time is wanted. */
+GCE_API int gce_profile_only(const char* name_prefix);
 GCE_API int gce_profile_count(void);
 GCE_API int gce_profile_get(int32_t i, char* name, int32_t name_len, double* total_ms,
                             int64_t* launches);
