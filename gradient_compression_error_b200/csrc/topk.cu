@@ -43,7 +43,8 @@ double bracket_sigma() { return g_bracket_sigma; }
 
 struct TkLayout {
     int64_t S = 0, TT = 0;
-    size_t segs = 0, hists = 0, unit_start = 0, redo_list = 0, tile_dir = 0, tile_cnt = 0,
+    size_t segs = 0, hists = 0, unit_start = 0, unit_seg = 0, redo_list = 0, tile_dir = 0,
+           tile_cnt = 0,
            spill_v = 0, spill_i = 0, total = 0;
 };
 
@@ -55,6 +56,9 @@ static TkLayout tk_layout(const gce_table* t, int32_t W) {
     o.segs = c.take<TkSeg>(o.S);
     o.hists = c.take<int32_t>(o.S * (kTkSBins + 3 * kTkBins));
     o.unit_start = c.take<int32_t>(o.S + 1);
+    // (segment, unit within it) of every histogram unit; a segment of n
+    // candidates has ceil(n / kTkHUnit) units and n is at most the layer size
+    o.unit_seg = c.take<int2>(o.S ? int64_t(W) * (t->comp_N / kTkHUnit + int64_t(t->comp.size())) : 0);
     o.redo_list = c.take<int32_t>(o.TT + 1);
     o.tile_dir = c.take<int2>(o.TT);
     o.tile_cnt = c.take<int2>(o.TT);
@@ -367,6 +371,7 @@ __global__ void __launch_bounds__(1024) tk_units_kernel(const DevLayer* __restri
                                                         int32_t ncomp, int32_t tiles_pw,
                                                         TkSeg* __restrict__ segs, int64_t S,
                                                         int32_t* __restrict__ unit_start,
+                                                        int2* __restrict__ unit_seg,
                                                         int32_t* __restrict__ redo_list,
                                                         int32_t* __restrict__ status) {
     __shared__ int s_warp[33];
@@ -404,6 +409,7 @@ __global__ void __launch_bounds__(1024) tk_units_kernel(const DevLayer* __restri
         int tot = 0;
         const int ex = block_exclusive_scan(units, s_warp, &tot);
         if (s < S) unit_start[s] = s_carry + ex;
+        for (int i = 0; i < units; ++i) unit_seg[s_carry + ex + i] = make_int2(int32_t(s), i);
         int rtot = 0;
         const int rex = block_exclusive_scan(rtiles, s_warp, &rtot);
         for (int i = 0; i < rtiles; ++i) redo_list[1 + s_rcarry + rex + i] = int32_t(t0 + i);
@@ -480,6 +486,7 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
                                                       int32_t ncomp, int64_t S, int64_t comp_N,
                                                       TkSeg* __restrict__ segs,
                                                       const int32_t* __restrict__ unit_start,
+                                                      const int2* __restrict__ unit_seg,
                                                       int32_t* __restrict__ hists,
                                                       const float* __restrict__ spill_v) {
     constexpr int kNb = kLevel == 3 ? 512 : kTkBins;
@@ -490,17 +497,13 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
     const int tid = threadIdx.x;
     const int32_t total = unit_start[S];
     for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
-        int64_t lo_ = 0, hi_ = S;
-        while (hi_ - lo_ > 1) {
-            const int64_t mid = (lo_ + hi_) >> 1;
-            if (unit_start[mid] <= u) lo_ = mid; else hi_ = mid;
-        }
-        const int64_t s = lo_;
+        const int2 us = unit_seg[u];
+        const int64_t s = us.x;
         const int w = int(s / ncomp);
         const DevLayer L = layers[comp[s % ncomp]];
         const uint32_t prefix = segs[s].prefix;
         const int32_t count = segs[s].count;
-        const int64_t j0 = int64_t(u - unit_start[s]) * kTkHUnit;
+        const int64_t j0 = int64_t(us.y) * kTkHUnit;
         for (int b = tid; b < kNb; b += blockDim.x) h[b] = 0;
         __syncthreads();
         const float* e = spill_v + int64_t(w) * comp_N + L.sp_off;
@@ -719,6 +722,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         TkSeg* segs = at<TkSeg>(ws, lay.segs);
         int32_t* hists = at<int32_t>(ws, lay.hists);
         int32_t* unit_start = at<int32_t>(ws, lay.unit_start);
+        int2* unit_seg = at<int2>(ws, lay.unit_seg);
         int32_t* redo_list = at<int32_t>(ws, lay.redo_list);
         int2* tile_dir = at<int2>(ws, lay.tile_dir);
         int2* tile_cnt = at<int2>(ws, lay.tile_cnt);
@@ -748,7 +752,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->comp_N, grad, mem, eta, segs,
                    tile_dir, spill_v, spill_i);
         GCE_LAUNCH(tk_units_kernel, 1, 1024, 0, st, t->d_layers, t->d_comp, ncomp, t->tiles_pw,
-                   segs, lay.S, unit_start, redo_list, status);
+                   segs, lay.S, unit_start, unit_seg, redo_list, status);
         GCE_LAUNCH(tk_restore_kernel, wave_grid(lay.TT, 4, r_restore), 256, 0, st, t->d_layers, t->d_tile_layer,
                    t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, spill_v,
                    spill_i, mem);
@@ -757,11 +761,11 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
                    spill_i);
         const int64_t hwork = lay.TT + lay.S;
         GCE_LAUNCH(tk_hist_kernel<1>, wave_grid(hwork, 8, r_h1), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
-                   t->comp_N, segs, unit_start, hists, spill_v);
+                   t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
         GCE_LAUNCH(tk_hist_kernel<2>, wave_grid(hwork, 8, r_h2), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
-                   t->comp_N, segs, unit_start, hists, spill_v);
+                   t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
         GCE_LAUNCH(tk_hist_kernel<3>, wave_grid(hwork, 8, r_h3), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
-                   t->comp_N, segs, unit_start, hists, spill_v);
+                   t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
         const int64_t wwork = (lay.TT + 7) / 8;  // a warp per tile
         GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw,
                    W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
