@@ -30,6 +30,16 @@ struct DevLayer {
     int32_t dc_base;        // first slot of this layer's ntiles+1 tile bounds
 };
 
+// One main tile's layer fields, for kernels whose per-tile work is short:
+// one 32-byte load instead of tile -> layer id -> layer record.
+struct alignas(16) TileInfo {
+    int64_t offset;   // first element of the tile's layer in a worker's buffer
+    int64_t sp_off;   // the layer's first candidate slot
+    int64_t val_off;  // the layer's first payload slot
+    int32_t sidx;     // index among the compressed layers
+    int32_t tstart;   // first element of the tile within its layer
+};
+
 }  // namespace gce
 
 struct gce_table {
@@ -47,6 +57,7 @@ struct gce_table {
     int64_t max_comp_n = 0;
     int32_t tiles_pw = 0;                  // main tiles (compressed layers) per worker
     int32_t* d_tile_layer = nullptr;       // [tiles_pw] layer of each main tile
+    gce::TileInfo* d_tile_info = nullptr;  // [tiles_pw] the same tiles' layer fields
     int32_t sunits_pw = 0;                 // top-k sample units per worker
     int32_t* d_sunit_layer = nullptr;      // [sunits_pw] layer of each sample unit
     int32_t* d_sunit_part = nullptr;       // [sunits_pw] part index within the layer

@@ -121,6 +121,7 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_comp);
     cudaFree(t->d_dense);
     cudaFree(t->d_tile_layer);
+    cudaFree(t->d_tile_info);
     cudaFree(t->d_sunit_layer);
     cudaFree(t->d_sunit_part);
     cudaFree(t->d_dtile_layer);
@@ -152,6 +153,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     int64_t off = 0, voff = 0, poff = 0, qoff = 0, spoff = 0;
     int32_t tiles = 0;
     std::vector<int32_t> tile_layer, sunit_layer, sunit_part, dtile_layer, dtile_start;
+    std::vector<TileInfo> tile_info;
     std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_nl;
     int32_t dc_tiles = 0, dc_slots = 0;
     for (int32_t l = 0; l < L; ++l) {
@@ -209,7 +211,11 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
             if (d.kind != GCE_KIND_POWERSGD) {
                 x.tile0 = tiles;
                 x.ntiles = int32_t((n + kTkTile - 1) / kTkTile);
-                for (int32_t i = 0; i < x.ntiles; ++i) tile_layer.push_back(l);
+                for (int32_t i = 0; i < x.ntiles; ++i) {
+                    tile_layer.push_back(l);
+                    tile_info.push_back(TileInfo{x.offset, x.sp_off, x.val_off, x.sidx,
+                                                 int32_t(int64_t(i) * kTkTile)});
+                }
                 tiles += x.ntiles;
                 const int32_t parts = int32_t((n + kTkSamplePart - 1) / kTkSamplePart);
                 for (int32_t p = 0; p < parts; ++p) {
@@ -253,6 +259,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_comp, t->comp);
     if (rc == GCE_OK) rc = upload(&t->d_dense, t->dense);
     if (rc == GCE_OK) rc = upload(&t->d_tile_layer, tile_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_tile_info, tile_info);
     if (rc == GCE_OK) rc = upload(&t->d_sunit_layer, sunit_layer);
     if (rc == GCE_OK) rc = upload(&t->d_sunit_part, sunit_part);
     if (rc == GCE_OK) rc = upload(&t->d_dtile_layer, dtile_layer);

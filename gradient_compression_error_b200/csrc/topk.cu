@@ -555,8 +555,7 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
 }
 
 // ---- per-tile counts, prefix over tiles, ordered emit --------------------------------------
-__global__ void __launch_bounds__(256) tk_count_kernel(const DevLayer* __restrict__ layers,
-                                                       const int32_t* __restrict__ tile_layer,
+__global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restrict__ tile_info,
                                                        int32_t tiles_pw, int32_t W, int32_t ncomp,
                                                        int64_t comp_N, const TkSeg* __restrict__ segs,
                                                        const int2* __restrict__ tile_dir,
@@ -569,14 +568,14 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const DevLayer* __restric
     for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
-        const DevLayer L = layers[tile_layer[lt]];
-        const int64_t s = int64_t(w) * ncomp + L.sidx;
+        const TileInfo ti = tile_info[lt];
+        const int2 d = tile_dir[t];
+        const int64_t s = int64_t(w) * ncomp + ti.sidx;
         const int32_t k = segs[s].k;
         int gt = 0, eq = 0;
         if (k > 0) {
             const uint32_t T = segs[s].prefix;
-            const int2 d = tile_dir[t];
-            const float* e = spill_v + int64_t(w) * comp_N + L.sp_off + d.x;
+            const float* e = spill_v + int64_t(w) * comp_N + ti.sp_off + d.x;
             for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
                 uint32_t key[kBatch];
 #pragma unroll
@@ -625,7 +624,7 @@ __global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restric
 }
 
 __global__ void __launch_bounds__(256) tk_emit_kernel(
-    const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
+    const TileInfo* __restrict__ tile_info, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, int64_t vals_pw,
     const TkSeg* __restrict__ segs, const int2* __restrict__ tile_dir,
     const int2* __restrict__ tile_cnt, const float* __restrict__ spill_v,
@@ -639,22 +638,22 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
     for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
-        const DevLayer L = layers[tile_layer[lt]];
-        const int64_t s = int64_t(w) * ncomp + L.sidx;
+        const TileInfo ti = tile_info[lt];
+        const int2 d = tile_dir[t];
+        const int2 before = tile_cnt[t];    // (key > T, key == T) in earlier tiles
+        const int64_t s = int64_t(w) * ncomp + ti.sidx;
         const int32_t k = segs[s].k;
         if (k == 0) continue;
         const uint32_t T = segs[s].prefix;
         const int32_t need = segs[s].need;  // keys equal to T that are taken
         // after the fallback the memory holds v everywhere (nothing was zeroed)
         const uint32_t hi = segs[s].redo ? 0xFFFFFFFFu : segs[s].hi;
-        const int2 d = tile_dir[t];
-        const int2 before = tile_cnt[t];    // (key > T, key == T) in earlier tiles
         int sel_before = before.x + min(before.y, need);
         int eq_seen = before.y;
-        const int64_t sb = int64_t(w) * comp_N + L.sp_off + d.x;
-        float* vout = vals + int64_t(w) * vals_pw + L.val_off;
-        int32_t* iout = idx + int64_t(w) * vals_pw + L.val_off;
-        float* m = mem + int64_t(w) * N + L.offset;
+        const int64_t sb = int64_t(w) * comp_N + ti.sp_off + d.x;
+        float* vout = vals + int64_t(w) * vals_pw + ti.val_off;
+        int32_t* iout = idx + int64_t(w) * vals_pw + ti.val_off;
+        float* m = mem + int64_t(w) * N + ti.offset;
         for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
             float ev[kBatch];
             int32_t ei[kBatch];
@@ -767,13 +766,13 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         GCE_LAUNCH(tk_hist_kernel<3>, wave_grid(hwork, 8, r_h3), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
                    t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
         const int64_t wwork = (lay.TT + 7) / 8;  // a warp per tile
-        GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw,
-                   W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
+        GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_tile_info,
+                   t->tiles_pw, W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
         GCE_LAUNCH(tk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
                    lay.S, t->tiles_pw, segs, tile_cnt);
-        GCE_LAUNCH(tk_emit_kernel, wave_grid(wwork, 8, r_emit), 256, 0, st, t->d_layers, t->d_tile_layer, t->tiles_pw, W,
-                   ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt, spill_v, spill_i,
-                   mem, vals, idx);
+        GCE_LAUNCH(tk_emit_kernel, wave_grid(wwork, 8, r_emit), 256, 0, st, t->d_tile_info,
+                   t->tiles_pw, W, ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt,
+                   spill_v, spill_i, mem, vals, idx);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, st);
