@@ -585,10 +585,8 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
                 }
 #pragma unroll
                 for (int q = 0; q < kBatch; ++q) {
-                    if (key[q] != 0xFFFFFFFFu) {
-                        gt += key[q] > T;
-                        eq += key[q] == T;
-                    }
+                    gt += key[q] != 0xFFFFFFFFu && key[q] > T;
+                    eq += key[q] == T;
                 }
             }
             gt = warp_sum(gt);
@@ -669,6 +667,7 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
             }
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
+                if (j0 + q * 32 >= d.y) break;  // the warp's remaining slots are empty
                 const bool valid = ei[q] >= 0;
                 const uint32_t key = abs_key(ev[q]);
                 const bool is_eq = valid && key == T;
