@@ -641,8 +641,8 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
                     mm.y = __fsub_rn(mm.y, mh[1]);
                     mm.z = __fsub_rn(mm.z, mh[2]);
                     mm.w = __fsub_rn(mm.w, mh[3]);
-                    *reinterpret_cast<float4*>(m + c) = mm;
-                    if (o) *reinterpret_cast<float4*>(o + c) = make_float4(mh[0], mh[1], mh[2], mh[3]);
+                    __stcs(reinterpret_cast<float4*>(m + c), mm);
+                    if (o) __stcs(reinterpret_cast<float4*>(o + c), make_float4(mh[0], mh[1], mh[2], mh[3]));
                 }
             } else {
                 for (int c = lane; c < cw; c += 32) {

@@ -461,7 +461,7 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
                     x.y = residual(mv[j].y, eta, gv[j].y);
                     x.z = residual(mv[j].z, eta, gv[j].z);
                     x.w = residual(mv[j].w, eta, gv[j].w);
-                    *reinterpret_cast<float4*>(m + e) = x;
+                    __stcs(reinterpret_cast<float4*>(m + e), x);
                 }
             } else {
 #pragma unroll

@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(256) sg_emit_kernel(
                 r.y = sg_update(residual(m[q].y, eta, g[q].y), s, n1);
                 r.z = sg_update(residual(m[q].z, eta, g[q].z), s, n2);
                 r.w = sg_update(residual(m[q].w, eta, g[q].w), s, n3);
-                *reinterpret_cast<float4*>(mem + base + e) = r;
+                __stcs(reinterpret_cast<float4*>(mem + base + e), r);
                 // eight lanes hold one word's 32 bits, four each
                 uint32_t v = (n0 | (n1 << 1) | (n2 << 2) | (n3 << 3)) << (4 * (lane & 7));
                 v |= __shfl_xor_sync(kFull, v, 1);

@@ -295,7 +295,9 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
                 o.y = abs_key(x.y) > hi ? 0.0f : x.y;
                 o.z = abs_key(x.z) > hi ? 0.0f : x.z;
                 o.w = abs_key(x.w) > hi ? 0.0f : x.w;
-                *reinterpret_cast<float4*>(m + e) = o;
+                // evict-first: the memory is not read again in this step, and
+                // keeping it out of L2 leaves room for the prefetched next tile
+                __stcs(reinterpret_cast<float4*>(m + e), o);
                 v[4 * j + 0] = x.x;
                 v[4 * j + 1] = x.y;
                 v[4 * j + 2] = x.z;
