@@ -141,7 +141,7 @@ __device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const Dev
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
             const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
-            below |= uint32_t(key < lo) << q;
+            below |= uint32_t(!kRedo && key < lo) << q;  // the redo lists every key
             inband |= uint32_t(key - lo <= span) << q;
         }
     } else {
@@ -149,7 +149,7 @@ __device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const Dev
         for (int q = 0; q < 32; ++q) {
             const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
             if (e0 + q < L.n) {
-                below |= uint32_t(key < lo) << q;
+                below |= uint32_t(!kRedo && key < lo) << q;  // the redo lists every key
                 inband |= uint32_t(key - lo <= span) << q;
             }
         }
