@@ -7,7 +7,7 @@
 //
 // Design (one launch per phase over every (worker, layer) of the table):
 //   setup    per-layer k, clear counters and histograms
-//   sample   read one 128-byte run of grad/mem per 2048 elements, histogram
+//   sample   read one 128-byte run of grad/mem per 4096 elements, histogram
 //            the |v| keys and, interpolating inside the crossing bins, pick
 //            two bounds with a wide statistical margin: lo (the k-th largest
 //            key lies above it) and hi (almost surely chosen above it);

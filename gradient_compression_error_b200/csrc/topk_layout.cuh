@@ -11,7 +11,7 @@ constexpr int kTkTile = kTkThreads * kTkPerThread;  // 8192 elements per main ti
 constexpr int kTkBins = 2048;                      // radix bins per level (11 bits)
 constexpr int kTkSBins = 4096;                     // sample bins: 2^19 keys, 16 per octave
 constexpr int kTkSampleChunk = 32;                 // sampled run length (one 128-B line)
-constexpr int kTkSampleStride = 2048;              // one run per 2048 elements
+constexpr int kTkSampleStride = 4096;              // one run per 4096 elements
 constexpr int64_t kTkSamplePart = int64_t(1) << 20; // elements covered by one sample unit
 constexpr int64_t kTkSampleMinN = 65536;           // smaller layers: exact histogram of all
 constexpr int kTkHUnit = 16384;                    // candidates per histogram unit
