@@ -23,6 +23,7 @@ OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4, "po
       "sign": 6}
 STATUS_K_RANGE = 1
 STATUS_FALLBACK = 2
+STATUS_NONFINITE = 4
 LEVEL_LOW, LEVEL_HIGH = 0, 1
 WS_HEADER_BYTES = 256
 

@@ -199,6 +199,16 @@ __device__ __forceinline__ float4 dc_final4(float4 s, float scale, const float4*
     return u;
 }
 
+// Keys at or above this one (sign cleared) belong to +-Inf and NaN.
+constexpr uint32_t kNonFiniteKey = 0x7F800000u;
+
+// Sets GCE_STATUS_NONFINITE if any lane saw a non-finite value.  Call with
+// the whole warp.
+__device__ __forceinline__ void flag_nonfinite(bool bad, int32_t* status) {
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0)
+        atomicOr(status, GCE_STATUS_NONFINITE);
+}
+
 // |v| ordering key: the float's bits with the sign cleared.
 __device__ __forceinline__ uint32_t abs_key(float v) {
     return __float_as_uint(v) & 0x7FFFFFFFu;
@@ -221,7 +231,7 @@ constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
 constexpr int kDenseTile = 4096;            // elements per tile of a DENSE layer
 
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
-                        float eta, float* vals, cudaStream_t st);
+                        float eta, float* vals, int32_t* status, cudaStream_t st);
 bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_rank,
                            const float* P, const float* Q, float scale, float* out, bool apply,
                            cudaStream_t st);

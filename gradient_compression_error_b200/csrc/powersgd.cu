@@ -193,7 +193,8 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t Q_pw,
     int64_t ppart_pw, const float* __restrict__ grad, float* __restrict__ mem, float eta,
-    const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, float* __restrict__ ppart) {
+    const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, float* __restrict__ ppart,
+    int32_t* __restrict__ status) {
     __shared__ float qs[kMaxRank][kPsCB];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
@@ -249,6 +250,8 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
                         if (j < r) acc[j] = fmaf(x, qs[j][c], acc[j]);
                 }
             }
+            // a NaN or infinite M makes its row's products non-finite
+            flag_nonfinite(!(fabsf(acc[0]) <= 3.4e38f), status);
 #pragma unroll
             for (int j = 0; j < kMaxRank; ++j) acc[j] = warp_sum(acc[j]);
             if (lane < r) {
@@ -570,7 +573,8 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dtile_layer,
     const int32_t* __restrict__ dtile_start, int32_t ntiles, int32_t W, int64_t N,
     const float* __restrict__ grad, float* __restrict__ mem, float eta, float inv_w,
-    float* __restrict__ vals) {
+    float* __restrict__ vals, int32_t* __restrict__ status) {
+    bool bad = false;
     for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
         const DevLayer L = layers[dtile_layer[u]];
         const int64_t s0 = dtile_start[u];
@@ -582,9 +586,11 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
                 s = __fadd_rn(s, residual(mem[e], eta, __ldcs(grad + e)));
                 mem[e] = 0.0f;
             }
+            bad |= abs_key(s) >= kNonFiniteKey;
             vals[L.val_off + s0 + i] = __fmul_rn(s, inv_w);
         }
     }
+    flag_nonfinite(bad, status);
 }
 
 // ---- residual: m <- M - P Q^T, dense_out <- P Q^T ---------------------------------------------
@@ -815,7 +821,7 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         static const int r_resid = resident_blocks(ps_resid_kernel, 256);
         GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st, t->d_layers,
                    ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw, t->ppart_pw, grad, mem,
-                   eta, k_or_rank, Q, ppart);
+                   eta, k_or_rank, Q, ppart, status);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, 1, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
@@ -839,7 +845,7 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
                    k_or_rank, P, Q, mem, dense_out);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
-    return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+    return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
 }
 
 extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad, float* mem,
@@ -872,7 +878,7 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         // every worker reads the shared warm start Q (stride 0)
         GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
                    t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0),
-                   t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart);
+                   t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status);
         // one P per layer from the partials of all W workers
         GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank,
@@ -902,7 +908,7 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         static const int r_dm = resident_blocks(ps_dense_mean_kernel, 256);
         GCE_LAUNCH(ps_dense_mean_kernel, wave_grid(t->dtiles_pw, 8, r_dm), 256, 0, st,
                    t->d_layers, t->d_dtile_layer, t->d_dtile_start, t->dtiles_pw, W, t->N, grad,
-                   mem, eta, inv_w, vals);
+                   mem, eta, inv_w, vals, status);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return GCE_OK;

@@ -400,7 +400,7 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
     const float* __restrict__ grad, float* __restrict__ mem, float eta,
     const RkSeg* __restrict__ segs, RkSeg* __restrict__ segs_next, int32_t* tile_off,
     uint32_t* bitmask, RkEntry* __restrict__ cand, float* __restrict__ vals,
-    int32_t* __restrict__ idx) {
+    int32_t* __restrict__ idx, int32_t* __restrict__ status) {
     constexpr int kIters = kTkPerThread / 4;
     constexpr int kWarps = kTkThreads / 32;
     __shared__ int32_t s_wt[kIters * kWarps];
@@ -453,6 +453,7 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
                     gv[j] = ld_stream4(g + e);
                     mv[j] = ld_stream4(m + e);
                 }
+                bool bad = false;
 #pragma unroll
                 for (int j = 0; j < kIters; ++j) {
                     const int e = j * (kTkThreads * 4) + tid * 4;
@@ -461,17 +462,26 @@ __global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
                     x.y = residual(mv[j].y, eta, gv[j].y);
                     x.z = residual(mv[j].z, eta, gv[j].z);
                     x.w = residual(mv[j].w, eta, gv[j].w);
+                    bad |= (abs_key(x.x) >= kNonFiniteKey) | (abs_key(x.y) >= kNonFiniteKey) |
+                           (abs_key(x.z) >= kNonFiniteKey) | (abs_key(x.w) >= kNonFiniteKey);
                     __stcs(reinterpret_cast<float4*>(m + e), x);
                 }
+                flag_nonfinite(bad, status);
             } else {
+                bool bad = false;
 #pragma unroll
                 for (int j = 0; j < kIters; ++j) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int e = j * (kTkThreads * 4) + tid * 4 + q;
-                        if (e < cnt) m[e] = residual(m[e], eta, __ldcs(g + e));
+                        if (e < cnt) {
+                            const float x = residual(m[e], eta, __ldcs(g + e));
+                            bad |= abs_key(x) >= kNonFiniteKey;
+                            m[e] = x;
+                        }
                     }
                 }
+                flag_nonfinite(bad, status);
             }
             uint32_t flags = 0;
 #pragma unroll
@@ -605,12 +615,12 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
             GCE_LAUNCH(rk_emit_kernel<true>, wave_grid(lay.TT, r_emit1, r_emit1), kTkThreads, 0, st,
                        t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
                        t->comp_N, grad, mem, eta, segs, segs_next, tile_cnt, bitmask, cand, vals,
-                       idx);
+                       idx, status);
         } else {
             GCE_LAUNCH(rk_emit_kernel<false>, wave_grid(lay.TT, r_emit0, r_emit0), kTkThreads, 0,
                        st, t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
                        t->comp_N, grad, mem, eta, segs, nullptr, tile_cnt, bitmask, cand, vals,
-                       idx);
+                       idx, status);
         }
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
         if (pipe) {
@@ -622,7 +632,7 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
             t->rk_valid = true;
         }
     }
-    return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+    return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
 }
 
 extern "C" int gce_set_randk_ahead(int32_t on) {

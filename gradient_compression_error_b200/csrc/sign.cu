@@ -57,7 +57,8 @@ __global__ void __launch_bounds__(256) sg_norm_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, const float* __restrict__ grad,
     const float* __restrict__ mem, float eta, double* __restrict__ partials,
-    int32_t* __restrict__ done, float* __restrict__ scales, float* __restrict__ vals) {
+    int32_t* __restrict__ done, float* __restrict__ scales, float* __restrict__ vals,
+    int32_t* __restrict__ status) {
     __shared__ double s_red[8];
     __shared__ int s_last;
     const int tid = threadIdx.x;
@@ -82,6 +83,8 @@ __global__ void __launch_bounds__(256) sg_norm_kernel(
             for (int e = tid; e < cnt; e += 256)
                 acc += fabs(double(residual(mem[base + e], eta, grad[base + e])));
         }
+        // a NaN or infinite p makes the sum non-finite
+        flag_nonfinite(!(fabs(acc) < 1.0e308), status);
         acc = block_sum_fixed(acc, s_red);
         if (tid == 0) {
             partials[t] = acc;
@@ -228,6 +231,7 @@ extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, fl
     const SgLayout lay = sg_layout(t, W);
     if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(ws);
     if (t->ckind == GCE_KIND_SIGN && t->tiles_pw > 0) {
         const int32_t ncomp = int32_t(t->comp.size());
         int32_t* done = at<int32_t>(ws, lay.done);
@@ -238,13 +242,14 @@ extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, fl
         const int64_t tiles = int64_t(t->tiles_pw) * W;
         GCE_LAUNCH(sg_norm_kernel, wave_grid(tiles, 8, r_norm), 256, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw, grad, mem, eta,
-                   at<double>(ws, lay.partials), done, at<float>(ws, lay.scales), vals);
+                   at<double>(ws, lay.partials), done, at<float>(ws, lay.scales), vals,
+                   status);
         GCE_LAUNCH(sg_emit_kernel, wave_grid(tiles, 8, r_emit), 256, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw, grad, mem, eta,
                    at<float>(ws, lay.scales), vals);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
-    return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+    return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
 }
 
 extern "C" int decompress_vote(const gce_table* t, int32_t W, const float* vals, float scale,

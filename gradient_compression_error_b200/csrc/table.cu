@@ -81,8 +81,10 @@ __global__ void __launch_bounds__(256) dense_kernel(const DevLayer* __restrict__
                                                     int32_t dtiles_pw, int32_t W, int64_t N,
                                                     int64_t vals_pw, const float* __restrict__ grad,
                                                     float* __restrict__ mem, float eta,
-                                                    float* __restrict__ vals) {
+                                                    float* __restrict__ vals,
+                                                    int32_t* __restrict__ status) {
     const int64_t total = int64_t(dtiles_pw) * W;
+    bool bad = false;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
         const int w = int(t / dtiles_pw);
         const int lt = int(t % dtiles_pw);
@@ -93,21 +95,24 @@ __global__ void __launch_bounds__(256) dense_kernel(const DevLayer* __restrict__
         float* m = mem + int64_t(w) * N + L.offset + start;
         float* out = vals + int64_t(w) * vals_pw + L.val_off + start;
         for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
-            out[i] = residual(m[i], eta, __ldcs(g + i));
+            const float v = residual(m[i], eta, __ldcs(g + i));
+            bad |= abs_key(v) >= kNonFiniteKey;
+            out[i] = v;
             m[i] = 0.0f;
         }
     }
+    flag_nonfinite(bad, status);
 }
 
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
-                        float* vals, cudaStream_t st) {
+                        float* vals, int32_t* status, cudaStream_t st) {
     if (t->dtiles_pw == 0) return GCE_OK;
     if (!vals) return GCE_ERR_ARG;
     int64_t total = int64_t(t->dtiles_pw) * W;
     static const int r_dense = resident_blocks(dense_kernel, 256);
     const int grid = wave_grid(total, 8, r_dense);
     GCE_LAUNCH(dense_kernel, grid, 256, 0, st, t->d_layers, t->d_dtile_layer, t->d_dtile_start,
-               t->dtiles_pw, W, t->N, t->vals_pw, grad, mem, eta, vals);
+               t->dtiles_pw, W, t->N, t->vals_pw, grad, mem, eta, vals, status);
     return check_launch();
 }
 

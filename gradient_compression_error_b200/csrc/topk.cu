@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, const float* __restrict__ grad,
     float* __restrict__ mem, float eta, TkSeg* __restrict__ segs, int2* __restrict__ tile_dir,
-    float* __restrict__ spill_v, int32_t* __restrict__ spill_i) {
+    float* __restrict__ spill_v, int32_t* __restrict__ spill_i, int32_t* __restrict__ status) {
     constexpr int kIters = kTkPerThread / 4;           // 8 float4 per thread
     constexpr int kWarps = kTkThreads / 32;            // 8
     __shared__ int32_t s_wt[kIters * kWarps];
@@ -322,6 +322,10 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
                 }
             }
         }
+        bool bad = false;
+#pragma unroll
+        for (int q = 0; q < kTkPerThread; ++q) bad |= abs_key(v[q]) >= kNonFiniteKey;
+        flag_nonfinite(bad, status);
         // ordered compaction: element order is (j, warp, lane, q)
         int incl[kIters];
 #pragma unroll
@@ -750,7 +754,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
                        lay.S, t->N, grad, mem, eta, segs, hists, g_bracket_sigma);
         GCE_LAUNCH(tk_main_kernel, wave_grid(lay.TT, r_main, r_main), kTkThreads, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->comp_N, grad, mem, eta, segs,
-                   tile_dir, spill_v, spill_i);
+                   tile_dir, spill_v, spill_i, status);
         GCE_LAUNCH(tk_units_kernel, 1, 1024, 0, st, t->d_layers, t->d_comp, ncomp, t->tiles_pw,
                    segs, lay.S, unit_start, unit_seg, redo_list, status);
         GCE_LAUNCH(tk_restore_kernel, wave_grid(lay.TT, 4, r_restore), 256, 0, st, t->d_layers, t->d_tile_layer,
@@ -776,5 +780,5 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
                    spill_v, spill_i, mem, vals, idx);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
-    return launch_dense_layers(t, W, grad, mem, eta, vals, st);
+    return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
 }

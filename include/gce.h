@@ -71,6 +71,9 @@ extern "C" {
 /* device status bits, read with gce_status */
 #define GCE_STATUS_K_RANGE 1    /* a per-layer k / rank was out of range: layer skipped   */
 #define GCE_STATUS_FALLBACK 2   /* informational: an exact fallback path ran              */
+#define GCE_STATUS_NONFINITE 4  /* a residual m + eta*grad was NaN or +-Inf (inputs must be
+                                   finite; the step still completes, ordering such keys by
+                                   their bits)                                            */
 
 /* layer kinds */
 #define GCE_KIND_TOPK 0
