@@ -94,6 +94,25 @@ def max_over_ranks_of(x, world, device):
     return float(t.item())
 
 
+def payload_bytes_per_worker(layers, method):
+    """Bytes one worker sends per step (what its exchange would carry): sparse
+    (value, index) pairs, a sign layer's words and scale, PowerSGD's P and Q,
+    a dense layer's floats.  For the data-parallel PowerSGD step, a worker's
+    share of the two all-reduces."""
+    total = 0
+    for l in layers:
+        n = l["rows"] * l["cols"]
+        if l["kind"] == "dense":
+            total += 4 * n
+        elif l["kind"] in ("topk", "randk"):
+            total += 8 * l["cap"]
+        elif l["kind"] == "sign":
+            total += 4 * ((n + 31) // 32) + 4
+        else:
+            total += 4 * l["cap"] * (l["rows"] + l["cols"])
+    return total
+
+
 def job_throughput(world, elems_per_step, steps, t_ms_max):
     """Whole-job elements per second: every rank's elements over the slowest
     rank's time (each rank runs its own replica of the workload)."""
@@ -537,6 +556,8 @@ def main():
                                       if graphs else "eager"),
                            "l2": "inputs larger than L2 (%.1f GB of grad+memory per step)"
                                  % (8.0 * W * N / 1e9),
+                           "payload_bytes_per_worker": payload_bytes_per_worker(layers, method),
+                           "compression_ratio": 4.0 * N / payload_bytes_per_worker(layers, method),
                            "step_algorithmic_GBps": step_gbs,
                            "step_frac_of_hbm": step_gbs / peak,
                            "fallback_seen": fallback_seen},

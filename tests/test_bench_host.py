@@ -70,3 +70,19 @@ def test_reference_leg_is_silent_on_other_ranks():
 def test_warmup_below_three_is_refused():
     r = run_bench(["--impl", "reference", "--steps", "1", "--warmup", "2"])
     assert r.returncode != 0
+
+
+def test_payload_bytes_per_worker():
+    sys.path.insert(0, ROOT)
+    import bench
+    from gradient_compression_error_b200 import workloads as wl
+    layers = [dict(rows=1000, cols=1, kind="topk", cap=10), dict(rows=7, cols=1, kind="dense")]
+    assert bench.payload_bytes_per_worker(layers, "topk") == 80 + 28
+    assert bench.payload_bytes_per_worker([dict(rows=33, cols=1, kind="sign")], "sign") == 12
+    assert bench.payload_bytes_per_worker([dict(rows=64, cols=576, kind="powersgd", cap=2)],
+                                          "powersgd") == 4 * 2 * (64 + 576)
+    # BERT-base top-k 1 %: K = 1,094,775 pairs of 8 bytes against 437.9 MB of fp32
+    bert = wl.bert_base_topk()
+    b = bench.payload_bytes_per_worker(bert, "topk")
+    assert b == 8 * 1094775
+    assert 49 < 4 * 109482240 / b < 51
