@@ -35,7 +35,7 @@
  *   reused (warm-started) Q: P = M Q, orthonormalise P, Q' = M^T P,
  *   decompress P Q'^T, residual into memory.
  *
- * Readings where the pages are silent (each listed in the design doc):
+ * Readings where the pages are silent:
  *   - residual rounding: v = fl32(m + fl32(eta * g)), two separate roundings,
  *     no fused multiply-add;
  *   - top-k order: key = |v| taken as the float's bits with the sign cleared;
@@ -61,7 +61,7 @@
  *     m_w = M_w - P Q_w^T; a DENSE layer sends the workers' mean residual
  *     (fp32 sum in worker order, then times fl32(1/W)).
  *
- * Parity unpinned (nothing on the pages fixes it; see DESIGN.md):
+ * Parity unpinned (nothing on the pages fixes it):
  *   or_randk_base / the stream composition of the rand-k and Q-init hashes
  *   (the SplitMix64 step itself is pinned by its published outputs);
  *   or_powersgd_init_q's mapping of hash bits to [-1, 1).
