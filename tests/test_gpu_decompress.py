@@ -227,3 +227,20 @@ def test_apply_lowrank_matches_decode(W):
     expect = osteps.apply_update(layers, W, pay, 0.5, x0, rank_per_layer=ranks)
     err = np.abs(host(x).astype(np.float64) - expect) - np.abs(np.spacing(expect))
     assert float(err.max()) <= 1e-6 * float(np.abs(agg).max())
+
+
+def test_apply_reads_the_k_prefix():
+    """With per-layer k, the fused update adds only the first k entries of
+    every payload, like the decode."""
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=50000, cols=1, kind="topk", cap=5000), dict(rows=33, cols=1, kind="dense", cap=0)]
+    t = g.Table(layers)
+    pay = sparse_payloads(layers, 3, 6)
+    vals, idx = upload(t, layers, 3, pay)
+    k = torch.tensor([777, 0], dtype=torch.int32, device="cuda")
+    x0 = np.random.default_rng(8).standard_normal(t.N).astype(np.float32)
+    x = torch.from_numpy(x0.copy()).cuda()
+    g.decompress_apply(t, 3, vals, idx, k, None, None, 1.0 / 3.0, x, t.workspace(3, "decompress"))
+    expect = osteps.apply_update(layers, 3, pay, 1.0 / 3.0, x0, k_per_layer=[777, 0])
+    assert np.array_equal(bits(host(x)), bits(expect))

@@ -178,3 +178,27 @@ def test_bert_base_w8_full_size():
                 host_mem[(w, l)] = host(run.mem[w, ls])
         del grad
     torch.cuda.empty_cache()
+
+
+def test_thirty_three_workers_sum_vote_and_noalloc():
+    """33 workers: the sum decode stages the sign words of 32 workers at a
+    time (two chunks here); the vote counts all 33; the decode without a
+    workspace gives the same bits as the one with."""
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=5000, cols=3, kind="sign", cap=0), dict(rows=9, cols=1, kind="dense", cap=0),
+              dict(rows=4097, cols=1, kind="sign", cap=0)]
+    W = 33
+    run = SignRun(layers, W)
+    pay = run.step(workloads.gradients(layers, W, 702, 0), 0.05)
+    t = run.t
+    out = torch.full((t.N,), float("nan"), device="cuda")
+    g.decompress_accumulate(t, W, run.vals, None, None, None, None, 0.75, out,
+                            t.workspace(W, "decompress"))
+    assert np.array_equal(bits(host(out)), bits(osteps.decompress(layers, W, pay, 0.75)))
+    out2 = torch.full((t.N,), float("nan"), device="cuda")
+    g.decompress_accumulate_noalloc(t, W, run.vals, None, None, None, None, 0.75, out2)
+    assert torch.equal(out.view(torch.int32), out2.view(torch.int32))
+    vote = torch.full((t.N,), float("nan"), device="cuda")
+    g.decompress_vote(t, W, run.vals, 2.0, vote)
+    assert np.array_equal(bits(host(vote)), bits(osteps.vote(layers, W, pay, 2.0)))
