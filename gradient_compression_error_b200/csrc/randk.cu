@@ -393,8 +393,11 @@ __global__ void __launch_bounds__(1024) rk_scan_kernel(const DevLayer* __restric
 // step's key pass over the same tile (segs_next): ALU work that overlaps the
 // other blocks' memory traffic.  The tile's bitmask words and offset are read
 // before the block's barriers and rewritten after them, by the same block.
+// Four blocks per SM (64 registers): the fifth register bank the look-ahead
+// variant would otherwise take costs a resident block and 3 % of the step,
+// more than the one value it spills.
 template <bool kNext>
-__global__ void __launch_bounds__(kTkThreads) rk_emit_kernel(
+__global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, int64_t comp_N,
     const float* __restrict__ grad, float* __restrict__ mem, float eta,
