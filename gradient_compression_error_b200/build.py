@@ -57,7 +57,7 @@ def build(force=False, verbose=False, extra_flags=()):
     procs = []
     for src in _sources():
         obj = os.path.join(BUILD_DIR, os.path.basename(src)[:-3] + ".o")
-        cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-dc" if False else "-c",
+        cmd = [nvcc, *NVCC_FLAGS, *extra_flags, "-I", INCLUDE, "-c",
                src, "-o", obj]
         if verbose:
             print(" ".join(cmd))
