@@ -80,7 +80,7 @@ def workload_spec(name):
 
 
 MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel",
-                "powersgd_dp": "ps_mq_kernel", "sign": "sg_emit_kernel"}
+                "powersgd_dp": "ps_mq_kernel", "sign": "sg_fused_kernel"}
 
 
 def max_over_ranks_of(x, world, device):
@@ -496,8 +496,9 @@ def main():
     if method in ("powersgd", "powersgd_dp"):
         step_bytes = W * 12.0 * N
     elif method == "sign":
-        # norm pass 8 B/el, emit pass 12 B/el + words; decode reads the words
-        step_bytes = W * (20.0 * N + N / 8.0) + W * N / 8.0
+        # grad and memory read once, memory written, words written (the
+        # pipelined kernel's second visit reads L2); decode reads the words
+        step_bytes = W * (12.0 * N + N / 8.0) + W * N / 8.0
     else:
         step_bytes = W * (12.0 * N + 8.0 * K_total) + 16.0 * W * K_total
     # the dense result: written (4 B), or read and written in place (8 B)

@@ -24,6 +24,7 @@ OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4, "po
 STATUS_K_RANGE = 1
 STATUS_FALLBACK = 2
 STATUS_NONFINITE = 4
+STATUS_WAIT_TIMEOUT = 8
 LEVEL_LOW, LEVEL_HIGH = 0, 1
 WS_HEADER_BYTES = 256
 
@@ -87,6 +88,8 @@ SIGNATURES = {
     "gce_error_string": (C.c_char_p, [C.c_int]),
     "gce_set_bracket_sigma": (C.c_int, [_f64]),
     "gce_set_randk_ahead": (C.c_int, [C.c_int32]),
+    "gce_set_sign_ahead": (C.c_int, [C.c_int32]),
+    "gce_set_sign_emit_first": (C.c_int, [C.c_int32]),
     "gce_profile_start": (C.c_int, []),
     "gce_profile_stop": (C.c_int, []),
     "gce_profile_only": (C.c_int, [C.c_char_p]),
@@ -329,3 +332,15 @@ def set_bracket_sigma(sigma):
 def set_randk_ahead(on):
     """Run the next rand-k step's key pass inside this one (include/gce.h)."""
     _check("gce_set_randk_ahead", lib().gce_set_randk_ahead(1 if on else 0))
+
+
+def set_sign_ahead(tiles):
+    """signSGD schedule: the norm runs `tiles` 8192-element tiles ahead of the
+    memory update in one launch; 0 runs two passes (include/gce.h)."""
+    _check("gce_set_sign_ahead", lib().gce_set_sign_ahead(int(tiles)))
+
+
+def set_sign_emit_first(on):
+    """Test of the bounded wait: every memory-update tile before every norm
+    tile, so the waits run out and GCE_STATUS_WAIT_TIMEOUT is set."""
+    _check("gce_set_sign_emit_first", lib().gce_set_sign_emit_first(1 if on else 0))

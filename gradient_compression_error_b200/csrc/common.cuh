@@ -40,6 +40,14 @@ struct alignas(16) TileInfo {
     int32_t tstart;   // first element of the tile within its layer
 };
 
+// A pipelined signSGD schedule uploaded for one (W, ahead): nphase runs
+// (the last a sentinel) covering nitems work items.
+struct SgPlan {
+    int32_t W, ahead, nphase;
+    int64_t nitems;
+    void* d_phases;
+};
+
 }  // namespace gce
 
 struct gce_table {
@@ -96,6 +104,10 @@ struct gce_table {
     mutable uint64_t rk_seed = 0, rk_step = 0;
     mutable int32_t rk_W = 0;
     mutable bool rk_valid = false;
+    // signSGD: pipelined schedules by (W, ahead), kept until the table is
+    // destroyed; guarded by sg_mu
+    mutable std::mutex sg_mu;
+    mutable std::vector<gce::SgPlan> sg_plans;
 };
 
 namespace gce {
@@ -230,6 +242,7 @@ constexpr int kDcTile = 1 << kDcTileLog;
 constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
 constexpr int kDenseTile = 4096;            // elements per tile of a DENSE layer
 
+void sign_plan_free(gce_table* t);
 int launch_dense_layers(const gce_table* t, int32_t W, const float* grad, float* mem,
                         float eta, float* vals, int32_t* status, cudaStream_t st);
 bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_rank,

@@ -137,6 +137,7 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_bunit_chunk);
     powersgd_plan_free(t);
     accordion_plan_free(t);
+    sign_plan_free(t);
     delete t;
 }
 

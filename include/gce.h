@@ -74,6 +74,9 @@ extern "C" {
 #define GCE_STATUS_NONFINITE 4  /* a residual m + eta*grad was NaN or +-Inf (inputs must be
                                    finite; the step still completes, ordering such keys by
                                    their bits)                                            */
+#define GCE_STATUS_WAIT_TIMEOUT 8  /* a bounded wait inside a kernel gave up (a scale that
+                                      was never published): that call's results are not
+                                      valid                                                 */
 
 /* layer kinds */
 #define GCE_KIND_TOPK 0
@@ -260,6 +263,29 @@ GCE_API int ef_sign_step(const gce_table* table, int32_t W, const float* grad, f
  */
 GCE_API int decompress_vote(const gce_table* table, int32_t W, const float* vals, float scale,
                             float* out, void* stream);
+
+/*
+ * How ef_sign_step schedules its two visits of every element.  tiles > 0:
+ * one launch in which the norm of the layer scale runs at most `tiles`
+ * 8192-element tiles ahead of the memory update, so the update reads grad
+ * and memory back from L2 rather than HBM (the schedule is built and cached
+ * per table and W on first use, outside stream capture: that first call
+ * allocates a small device array (cudaMalloc, with its implicit
+ * synchronisation) kept until gce_table_destroy; while capturing before
+ * that, the two passes run).  0: two passes over the whole set.  Both give
+ * the same bits.  Default 768.  tiles outside [0, 2^20] gives GCE_ERR_ARG.
+ */
+GCE_API int gce_set_sign_ahead(int32_t tiles);
+
+/*
+ * Test of the bounded wait in the pipelined signSGD kernel.  on = 1 places
+ * every memory-update tile before every norm tile and runs the kernel as one
+ * block, so each update's wait for its layer scale runs out (about a second
+ * per tile) and sets GCE_STATUS_WAIT_TIMEOUT;
+ * that call's results are not valid.  Nothing faults or hangs.  0 (the
+ * default) restores the normal order.  Other values give GCE_ERR_ARG.
+ */
+GCE_API int gce_set_sign_emit_first(int32_t on);
 
 /*
  * Accordion select [ACC] over every compressed layer of the table.

@@ -202,3 +202,68 @@ def test_thirty_three_workers_sum_vote_and_noalloc():
     vote = torch.full((t.N,), float("nan"), device="cuda")
     g.decompress_vote(t, W, run.vals, 2.0, vote)
     assert np.array_equal(bits(host(vote)), bits(osteps.vote(layers, W, pay, 2.0)))
+
+
+PIPE_LAYERS = [dict(rows=190000, cols=1, kind="sign", cap=0, sigma=1.0),
+               dict(rows=33, cols=1, kind="dense", cap=0, sigma=1.0),
+               dict(rows=5000, cols=3, kind="sign", cap=0, sigma=0.5),
+               dict(rows=8192, cols=1, kind="sign", cap=0, sigma=2.0),
+               dict(rows=300000, cols=1, kind="sign", cap=0, sigma=1.0),
+               dict(rows=1, cols=1, kind="sign", cap=0, sigma=1.0)]
+
+
+def _sign_steps(g, t, W, grad_seeds, ahead):
+    """Two steps from the same memory under one schedule; (mem, vals, status)."""
+    g.set_sign_ahead(ahead)
+    mem = 0.1 * workloads.gradients(PIPE_LAYERS, W, 951, 0)
+    vals = torch.zeros((W, max(4, t.vals_per_worker)), device="cuda")
+    ws = t.workspace(W, "sign")
+    for s in grad_seeds:
+        g.ef_sign_step(t, W, workloads.gradients(PIPE_LAYERS, W, 950, s), mem, 0.05, vals, ws)
+    return mem, vals, g.status(ws)
+
+
+@pytest.mark.parametrize("ahead", [1, 64, 300, 100000])
+def test_pipelined_schedule_gives_the_two_pass_bits(ahead):
+    """The one-launch schedule (norm tiles `ahead` tiles in front of the memory
+    update) and the two passes give the same memory, scales and words: the
+    partials, their order and the scale do not depend on the schedule.  The
+    default schedule is checked against the oracle by the tests above."""
+    need_gpu()
+    g = gce()
+    W = 3
+    t = g.Table(workloads.table_layers(PIPE_LAYERS))
+    try:
+        m0, v0, st0 = _sign_steps(g, t, W, [0, 1], 0)
+        m1, v1, st1 = _sign_steps(g, t, W, [0, 1], ahead)
+    finally:
+        g.set_sign_ahead(768)
+    assert st0 == 0 and st1 == 0
+    assert torch.equal(m0.view(torch.int32), m1.view(torch.int32))
+    assert torch.equal(v0.view(torch.int32), v1.view(torch.int32))
+
+
+def test_wait_that_runs_out_sets_the_status():
+    """Failure detection without a fault: with every memory-update tile placed
+    before every norm tile, each update's wait for its layer scale runs out
+    (about a second), the kernel sets GCE_STATUS_WAIT_TIMEOUT and returns; the
+    context stays usable and the next step, in the normal order, is clean and
+    matches the oracle.  One tile, one block: a single wait runs out."""
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=8192, cols=1, kind="sign", cap=0, sigma=1.0)]
+    t = g.Table(workloads.table_layers(layers))
+    mem = torch.zeros((1, t.N), device="cuda")
+    vals = torch.zeros((1, max(4, t.vals_per_worker)), device="cuda")
+    ws = t.workspace(1, "sign")
+    grad = workloads.gradients(layers, 1, 952, 0)
+    try:
+        g.set_sign_emit_first(True)
+        g.ef_sign_step(t, 1, grad, mem, 0.05, vals, ws)
+        st = g.status(ws)
+    finally:
+        g.set_sign_emit_first(False)
+    assert st & g.STATUS_WAIT_TIMEOUT
+    run = SignRun(layers, 1)
+    run.step(grad, np.float32(0.05))
+    assert g.status(run.ws) == 0
