@@ -19,7 +19,9 @@
 //   pipelined (sg_fused_kernel, one launch): norm tiles run a bounded
 //          distance ahead of emit tiles, so an emit tile's grad and memory
 //          are still in L2 and HBM sees them once (8 B/element read, 4 B
-//          written, plus 1/8 B of sign words);
+//          written, plus 1/8 B of sign words).  The norm reads with an L2
+//          evict-last policy and the emit re-reads with evict-first, so
+//          the lines wait in L2 for their second visit and leave after it;
 //   two passes (sg_norm_kernel, then sg_emit_kernel): 8 B/element, then
 //          12 B/element; used while a stream is being captured before the
 //          pipelined schedule exists, or when it is switched off.
@@ -76,6 +78,26 @@ __device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
     asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ float4 ld_hint4(const float* p, uint64_t pol) {
+    float4 v;
+    asm volatile("ld.global.L2::cache_hint.v4.f32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+                 : "l"(p), "l"(pol));
+    return v;
+}
+
 // Where tile t (worker-major over the compressed layers) lies.
 struct SgTile {
     DevLayer L;
@@ -99,8 +121,8 @@ __device__ __forceinline__ SgTile sg_tile(const DevLayer* layers, const int32_t*
 // ---- norm of one tile ---------------------------------------------------------------
 // The tile's fp64 partial of |p|; the block that completes the layer adds
 // the layer's partials in a fixed order, writes s (scales and the payload
-// slot) and, when `ready` is given, publishes it.  kKeep: plain L2 loads, so
-// the lines stay for the emit that follows; otherwise grad is read
+// slot) and, when `ready` is given, publishes it.  kKeep: L2 evict-last
+// loads, so the lines stay for the emit that follows; otherwise grad is read
 // evict-first.  Ends with the block synchronised.
 template <bool kKeep>
 __device__ __forceinline__ void sg_norm_tile(const SgTile& x, int64_t t, int32_t tiles_pw,
@@ -113,12 +135,13 @@ __device__ __forceinline__ void sg_norm_tile(const SgTile& x, int64_t t, int32_t
     const int tid = threadIdx.x;
     double acc = 0.0;
     if ((x.base & 3) == 0 && x.cnt == kTkTile) {
+        const uint64_t pol = kKeep ? l2_evict_last_policy() : 0;
 #pragma unroll
         for (int q = 0; q < kTkTile / 4 / 256; ++q) {
             const int e = 4 * (q * 256 + tid);
-            const float4 g = kKeep ? __ldcg(reinterpret_cast<const float4*>(grad + x.base + e))
+            const float4 g = kKeep ? ld_hint4(grad + x.base + e, pol)
                                    : ld_stream4(grad + x.base + e);
-            const float4 m = kKeep ? __ldcg(reinterpret_cast<const float4*>(mem + x.base + e))
+            const float4 m = kKeep ? ld_hint4(mem + x.base + e, pol)
                                    : *reinterpret_cast<const float4*>(mem + x.base + e);
             acc += fabs(double(residual(m.x, eta, g.x))) + fabs(double(residual(m.y, eta, g.y))) +
                    fabs(double(residual(m.z, eta, g.z))) + fabs(double(residual(m.w, eta, g.w)));
@@ -171,6 +194,9 @@ __device__ __forceinline__ uint32_t* sg_words(float* vals, int64_t vals_pw, int 
 }
 
 // words: the tile's first sign word; base: its first element in grad / mem.
+// kHint: the second visit of the pipelined kernel, whose loads mark the lines
+// evict-first (their last use).
+template <bool kHint>
 __device__ __forceinline__ void sg_emit_tile(int64_t base, int cnt, uint32_t* words, float s,
                                              const float* __restrict__ grad,
                                              float* __restrict__ mem, float eta) {
@@ -179,11 +205,13 @@ __device__ __forceinline__ void sg_emit_tile(int64_t base, int cnt, uint32_t* wo
     if ((base & 3) == 0 && cnt == kTkTile) {
         // all loads of the warp's 1024 elements first, then the updates
         float4 g[8], m[8];
+        const uint64_t pol = kHint ? l2_evict_first_policy() : 0;
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int e = e0 + 128 * q + 4 * lane;
-            g[q] = ld_stream4(grad + base + e);
-            m[q] = *reinterpret_cast<const float4*>(mem + base + e);
+            g[q] = kHint ? ld_hint4(grad + base + e, pol) : ld_stream4(grad + base + e);
+            m[q] = kHint ? ld_hint4(mem + base + e, pol)
+                         : *reinterpret_cast<const float4*>(mem + base + e);
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
@@ -241,7 +269,7 @@ __global__ void __launch_bounds__(256) sg_emit_kernel(
         const int lt = int(t % tiles_pw);
         const DevLayer L = layers[tile_layer[lt]];
         const int64_t s0 = int64_t(lt - L.tile0) * kTkTile;
-        sg_emit_tile(int64_t(w) * N + L.offset + s0, int(min64(kTkTile, L.n - s0)),
+        sg_emit_tile<false>(int64_t(w) * N + L.offset + s0, int(min64(kTkTile, L.n - s0)),
                      sg_words(vals, vals_pw, w, L.val_off, s0), scales[int64_t(w) * ncomp + L.sidx],
                      grad, mem, eta);
     }
@@ -307,7 +335,7 @@ __global__ void __launch_bounds__(256, 4) sg_fused_kernel(
                 s_scale = __ldcg(scales + x.seg);
             }
             __syncthreads();
-            sg_emit_tile(x.base, x.cnt, sg_words(vals, vals_pw, x.w, x.L.val_off, x.s0), s_scale,
+            sg_emit_tile<true>(x.base, x.cnt, sg_words(vals, vals_pw, x.w, x.L.val_off, x.s0), s_scale,
                          grad, mem, eta);
         }
         __syncthreads();  // s_item, s_ph and s_scale are rewritten next
