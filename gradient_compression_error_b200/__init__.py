@@ -66,6 +66,8 @@ SIGNATURES = {
     "ef_topk_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, C.c_size_t, _vp]),
     "ef_randk_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _u64, _u64, _vp, _vp, _vp,
                                 C.c_size_t, _vp]),
+    "ef_randk_step_at": (C.c_int, [_vp, C.c_int64, _i32, _vp, _vp, _f32, _vp, _u64, _u64, _vp,
+                                   _vp, _vp, C.c_size_t, _vp]),
     "powersgd_init_q": (C.c_int, [_vp, _i32, _u64, _vp, _vp]),
     "powersgd_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
                                 C.c_size_t, _vp]),
@@ -207,6 +209,15 @@ def ef_topk_step(table, W, grad, mem, eta, k_or_rank, vals, idx, ws, stream=None
 def ef_randk_step(table, W, grad, mem, eta, k_or_rank, seed, step, vals, idx, ws, stream=None):
     _check("ef_randk_step", lib().ef_randk_step(
         table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), int(seed), int(step), _ptr(vals, _f32()), _ptr(idx, _i32()),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def ef_randk_step_at(table, worker0, W, grad, mem, eta, k_or_rank, seed, step, vals, idx, ws,
+                     stream=None):
+    """ef_randk_step for job-wide workers worker0 .. worker0+W-1 (include/gce.h)."""
+    _check("ef_randk_step_at", lib().ef_randk_step_at(
+        table.handle, int(worker0), int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
         _ptr(k_or_rank, _i32()), int(seed), int(step), _ptr(vals, _f32()), _ptr(idx, _i32()),
         _ptr(ws), ws.numel(), _stream(stream)))
 

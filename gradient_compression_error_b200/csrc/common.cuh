@@ -98,11 +98,13 @@ struct gce_table {
     int32_t ac_ntiles = 0;
     int2* d_ac_layer = nullptr;            // per layer: (first norm tile, tile count)
     // rand-k: the key pass the last ef_randk_step ran ahead for the next step
-    // (step rk_step, seed rk_seed, W rk_W) in workspace rk_ws; guarded by rk_mu
+    // (step rk_step, seed rk_seed, W rk_W workers from rk_worker0) in workspace
+    // rk_ws; guarded by rk_mu
     mutable std::mutex rk_mu;
     mutable const void* rk_ws = nullptr;
     mutable uint64_t rk_seed = 0, rk_step = 0;
     mutable int32_t rk_W = 0;
+    mutable int64_t rk_worker0 = 0;
     mutable bool rk_valid = false;
     // signSGD: pipelined schedules by (W, ahead), kept until the table is
     // destroyed; guarded by sg_mu

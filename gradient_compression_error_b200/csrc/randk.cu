@@ -77,11 +77,13 @@ size_t randk_ws_bytes(const gce_table* t, int32_t W) { return rk_layout(t, W).to
 
 // State of (worker, layer) segment s for `step`: k (0 when out of range),
 // the band [lo, hi] of +-(sigma * binomial sd + sigma) keys around the
-// expected k-th smallest key, the generator state, counters at zero.
+// expected k-th smallest key, the generator state, counters at zero.  The
+// generator takes the job-wide worker index worker0 + s / ncomp.
 __device__ __forceinline__ void rk_setup_seg(int64_t s, const DevLayer* __restrict__ layers,
                                              const int32_t* __restrict__ comp, int32_t ncomp,
                                              const int32_t* __restrict__ k_or_rank, uint64_t seed,
-                                             uint64_t step, double sigma, RkSeg* __restrict__ segs,
+                                             uint64_t worker0, uint64_t step, double sigma,
+                                             RkSeg* __restrict__ segs,
                                              int32_t* __restrict__ status) {
     const int32_t l = comp[s % ncomp];
     const DevLayer L = layers[l];
@@ -100,7 +102,7 @@ __device__ __forceinline__ void rk_setup_seg(int64_t s, const DevLayer* __restri
     g.lo = lo <= 0.0 ? 0u : (lo >= 4294967295.0 ? 0xFFFFFFFFu : uint32_t(lo));
     g.hi = hi >= 4294967295.0 ? 0xFFFFFFFFu : (hi <= 0.0 ? 0u : uint32_t(hi));
     if (g.hi < g.lo) g.hi = g.lo;
-    g.base = hash_base(seed, 0, uint64_t(s / ncomp), uint64_t(l), step);
+    g.base = hash_base(seed, 0, worker0 + uint64_t(s / ncomp), uint64_t(l), step);
     segs[s] = g;
 }
 
@@ -110,7 +112,8 @@ __global__ void __launch_bounds__(256) rk_setup_kernel(const DevLayer* __restric
                                                        const int32_t* __restrict__ comp,
                                                        int32_t ncomp, int64_t S,
                                                        const int32_t* __restrict__ k_or_rank,
-                                                       uint64_t seed, uint64_t step, double sigma,
+                                                       uint64_t seed, uint64_t worker0,
+                                                       uint64_t step, double sigma,
                                                        RkSeg* __restrict__ segs,
                                                        int32_t* __restrict__ status,
                                                        uint64_t* __restrict__ tag,
@@ -118,7 +121,8 @@ __global__ void __launch_bounds__(256) rk_setup_kernel(const DevLayer* __restric
     if (blockIdx.x == 0 && threadIdx.x == 0) *tag = tag_value;
     for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
          s += int64_t(gridDim.x) * blockDim.x)
-        rk_setup_seg(s, layers, comp, ncomp, k_or_rank, seed, step, sigma, segs, status);
+        rk_setup_seg(s, layers, comp, ncomp, k_or_rank, seed, worker0, step, sigma, segs,
+                     status);
 }
 
 // Key pass over one tile t (worker w, layer L): the bitmask words of key < lo,
@@ -212,7 +216,8 @@ __global__ void __launch_bounds__(256) rk_refresh_k_kernel(const DevLayer* __res
                                                            const int32_t* __restrict__ comp,
                                                            int32_t ncomp, int64_t S,
                                                            const int32_t* __restrict__ k_or_rank,
-                                                           uint64_t seed, uint64_t step,
+                                                           uint64_t seed, uint64_t worker0,
+                                                           uint64_t step,
                                                            double sigma, RkSeg* __restrict__ segs,
                                                            int32_t* __restrict__ status,
                                                            const uint64_t* __restrict__ tag,
@@ -221,7 +226,8 @@ __global__ void __launch_bounds__(256) rk_refresh_k_kernel(const DevLayer* __res
     for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
          s += int64_t(gridDim.x) * blockDim.x) {
         if (!held) {
-            rk_setup_seg(s, layers, comp, ncomp, k_or_rank, seed, step, sigma, segs, status);
+            rk_setup_seg(s, layers, comp, ncomp, k_or_rank, seed, worker0, step, sigma, segs,
+                         status);
             segs[s].fail = 1;
             continue;
         }
@@ -537,10 +543,11 @@ __global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
 
 using namespace gce;
 
-extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
-                             const int32_t* k_or_rank, uint64_t seed, uint64_t step, float* vals,
-                             int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
-    if (!t || W < 1 || !grad || !mem || !ws) return GCE_ERR_ARG;
+static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const float* grad,
+                      float* mem, float eta, const int32_t* k_or_rank, uint64_t seed,
+                      uint64_t step, float* vals, int32_t* idx, void* ws, size_t ws_bytes,
+                      void* stream) {
+    if (!t || W < 1 || worker0 < 0 || !grad || !mem || !ws) return GCE_ERR_ARG;
     if (t->ckind != GCE_KIND_RANDK && t->ckind != -1) return GCE_ERR_KIND;
     if (!aligned16(grad) || !aligned16(mem) || !aligned16(ws)) return GCE_ERR_ARG;
     if ((t->vals_pw > 0) && (!vals || !aligned16(vals))) return GCE_ERR_ARG;
@@ -565,13 +572,14 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
         {
             std::lock_guard<std::mutex> lk(t->rk_mu);
             have = pipe && t->rk_valid && t->rk_ws == ws && t->rk_seed == seed &&
-                   t->rk_step == step && t->rk_W == W;
+                   t->rk_step == step && t->rk_W == W && t->rk_worker0 == worker0;
             t->rk_valid = false;
         }
         // which step's key pass the workspace holds (header bytes 64-71)
         uint64_t* tag = at<uint64_t>(ws, 64);
         auto tag_of = [&](uint64_t sv) {
-            const uint64_t h = mix64(mix64(mix64(seed + kGamma) + sv) + uint64_t(W)) ^
+            const uint64_t h = mix64(mix64(mix64(mix64(seed + kGamma) + sv) + uint64_t(W)) +
+                                     uint64_t(worker0)) ^
                                reinterpret_cast<uintptr_t>(t);
             return h ? h : 1u;
         };
@@ -588,12 +596,14 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
         static const int r_emit1 = resident_blocks(rk_emit_kernel<true>, kTkThreads);
         if (have) {
             GCE_LAUNCH(rk_refresh_k_kernel, wave_grid((lay.S + 255) / 256, 4, r_refresh), 256, 0,
-                       st, t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed, step,
-                       bracket_sigma(), segs, status, tag, tag_of(step));
+                       st, t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
+                       uint64_t(worker0), step, bracket_sigma(), segs, status, tag,
+                       tag_of(step));
         } else {
             GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st,
-                       t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed, step,
-                       bracket_sigma(), segs, status, tag, uint64_t(0));
+                       t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
+                       uint64_t(worker0), step, bracket_sigma(), segs, status, tag,
+                       uint64_t(0));
             GCE_LAUNCH(rk_keys_kernel<false>, wave_grid(lay.TT, 8, r_keys0), 256, 0, st,
                        t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs,
                        tile_cnt, bitmask, cand);
@@ -613,8 +623,9 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
             // the next step's band from this step's k (a guess: the exact
             // resolve of that step re-reads k and repairs any miss)
             GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st,
-                       t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed, step + 1,
-                       bracket_sigma(), segs_next, nullptr, tag, tag_of(step + 1));
+                       t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
+                       uint64_t(worker0), step + 1, bracket_sigma(), segs_next, nullptr, tag,
+                       tag_of(step + 1));
             GCE_LAUNCH(rk_emit_kernel<true>, wave_grid(lay.TT, r_emit1, r_emit1), kTkThreads, 0, st,
                        t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
                        t->comp_N, grad, mem, eta, segs, segs_next, tile_cnt, bitmask, cand, vals,
@@ -632,10 +643,26 @@ extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, f
             t->rk_seed = seed;
             t->rk_step = step + 1;
             t->rk_W = W;
+            t->rk_worker0 = worker0;
             t->rk_valid = true;
         }
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
+}
+
+extern "C" int ef_randk_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
+                             const int32_t* k_or_rank, uint64_t seed, uint64_t step, float* vals,
+                             int32_t* idx, void* ws, size_t ws_bytes, void* stream) {
+    return randk_step(t, W, 0, grad, mem, eta, k_or_rank, seed, step, vals, idx, ws, ws_bytes,
+                      stream);
+}
+
+extern "C" int ef_randk_step_at(const gce_table* t, int64_t worker0, int32_t W, const float* grad,
+                                float* mem, float eta, const int32_t* k_or_rank, uint64_t seed,
+                                uint64_t step, float* vals, int32_t* idx, void* ws,
+                                size_t ws_bytes, void* stream) {
+    return randk_step(t, W, worker0, grad, mem, eta, k_or_rank, seed, step, vals, idx, ws,
+                      ws_bytes, stream);
 }
 
 extern "C" int gce_set_randk_ahead(int32_t on) {

@@ -21,16 +21,15 @@ arithmetic of the method runs in the native library.  The ranks must agree on
 the table and on k: with Accordion's per-layer levels, every rank passes the
 same k tensor.
 
-Payload kinds: top-k, signSGD and dense layers.  Not exchanged here:
-- rand-k, whose key stream folds the worker index in: a one-worker step on
-  every rank would draw worker 0's coordinates everywhere;
-- PowerSGD, whose data-parallel form sums P and Q over the workers inside the
-  step, between its contractions.
+Payload kinds: top-k, rand-k, signSGD and dense layers.  rand-k's generator
+takes the worker index, so rank r encodes as job-wide worker r
+(ef_randk_step_at).  Not exchanged here: PowerSGD, whose data-parallel form
+sums P and Q over the workers inside the step, between its contractions.
 """
 import torch
 import torch.distributed as dist
 
-METHODS = ("topk", "sign")
+METHODS = ("topk", "randk", "sign")
 
 
 class PayloadExchange:
@@ -77,8 +76,9 @@ class PayloadExchange:
 class DataParallelStep:
     """One data-parallel step over the ranks of ``group``, one worker per rank.
 
-    ``encode`` runs this rank's one-worker step (ef_topk_step or ef_sign_step,
-    W = 1) on grad / mem [1, N]; ``exchange`` gathers every rank's payload;
+    ``encode`` runs this rank's one-worker step (ef_topk_step, ef_randk_step_at
+    as worker ``rank`` or ef_sign_step; W = 1) on grad / mem [1, N];
+    ``exchange`` gathers every rank's payload;
     ``decode`` writes the aggregate of the gathered payloads.  ``__call__``
     runs the three in order.  The native calls run on the current CUDA stream,
     and torch.distributed orders its collectives after that stream's work.
@@ -87,8 +87,8 @@ class DataParallelStep:
     def __init__(self, table, method, group=None, device="cuda"):
         import gradient_compression_error_b200 as g
         if method not in METHODS:
-            raise ValueError("method must be one of %s (rand-k and PowerSGD are not "
-                             "exchanged here)" % (METHODS,))
+            raise ValueError("method must be one of %s (PowerSGD is not exchanged here)"
+                             % (METHODS,))
         ck = table.compressed_kind
         if ck not in (-1, g.KIND[method]):
             raise ValueError("table of kind %s cannot take a %s step"
@@ -96,20 +96,25 @@ class DataParallelStep:
         self.g = g
         self.table = table
         self.method = method
-        self.ex = PayloadExchange(table.vals_per_worker, method == "topk", device, group)
+        sparse = method in ("topk", "randk")
+        self.ex = PayloadExchange(table.vals_per_worker, sparse, device, group)
         self.world = self.ex.world
         n = self.ex.n
         self.vals_row = torch.zeros((1, n), dtype=torch.float32, device=device)
         self.idx_row = (torch.zeros((1, n), dtype=torch.int32, device=device)
-                        if method == "topk" else None)
+                        if sparse else None)
         self.ws_step = table.workspace(1, method, device)
         self.ws_dec = table.workspace(self.world, "decompress", device)
 
-    def encode(self, grad, mem, eta, k=None):
+    def encode(self, grad, mem, eta, k=None, seed=0, step=0):
+        """seed, step: rand-k's generator (the same on every rank)."""
         g = self.g
         if self.method == "topk":
             g.ef_topk_step(self.table, 1, grad, mem, eta, k, self.vals_row, self.idx_row,
                            self.ws_step)
+        elif self.method == "randk":
+            g.ef_randk_step_at(self.table, self.ex.rank, 1, grad, mem, eta, k, seed, step,
+                               self.vals_row, self.idx_row, self.ws_step)
         else:
             g.ef_sign_step(self.table, 1, grad, mem, eta, self.vals_row, self.ws_step)
 
@@ -133,9 +138,10 @@ class DataParallelStep:
             g.decompress_accumulate(self.table, self.world, vals, idx, k, None, None, scale, out,
                                     self.ws_dec)
 
-    def __call__(self, grad, mem, eta, out, scale=None, k=None, apply=False, vote=False):
+    def __call__(self, grad, mem, eta, out, scale=None, k=None, apply=False, vote=False,
+                 seed=0, step=0):
         """One step; scale defaults to 1/world (the mean)."""
-        self.encode(grad, mem, eta, k)
+        self.encode(grad, mem, eta, k, seed, step)
         self.exchange()
         self.decode(out, 1.0 / self.world if scale is None else scale, k, apply, vote)
         return out

@@ -180,12 +180,25 @@ GCE_API int ef_randk_step(const gce_table* table, int32_t W, const float* grad, 
                   float* vals, int32_t* idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * ef_randk_step for workers worker0 .. worker0+W-1 of a larger job (one
+ * rank's share of a data-parallel job): row w of grad, mem, vals and idx
+ * belongs to job-wide worker worker0 + w, whose index the generator takes,
+ * so the rows are bit for bit those of an ef_randk_step over the whole job.
+ * worker0 < 0 gives GCE_ERR_ARG.  ef_randk_step is this call with worker0 0.
+ */
+GCE_API int ef_randk_step_at(const gce_table* table, int64_t worker0, int32_t W,
+                             const float* grad, float* mem, float eta,
+                             const int32_t* k_or_rank, uint64_t seed, uint64_t step,
+                             float* vals, int32_t* idx, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/*
  * rand-k look-ahead (on by default; the pages have no counterpart: it only
  * moves work).  The chosen set does not depend on the data, so while a step's
  * memory pass streams grad and mem, ef_randk_step also hashes the next step's
- * keys (step + 1, same seed, W and table, with this step's k sizing the
- * band) into its workspace.  The next call with the same table, workspace,
- * seed, W and step + 1 skips its own key pass.  Results never depend on it:
+ * keys (step + 1, same seed, W, worker0 and table, with this step's k sizing
+ * the band) into its workspace.  The next call with the same table,
+ * workspace, seed, W, worker0 and step + 1 skips its own key pass.  Results never depend on it:
  * that call re-reads k, repairs a band the new k misses exactly, and checks a
  * tag in the workspace header, recomputing everything if another step's pass
  * is there.  Between the two calls nothing else may write the workspace.
@@ -249,6 +262,8 @@ GCE_API int powersgd_dp_step(const gce_table* table, int32_t W, const float* gra
  * The sign bits and, for a given s, the memory are exact; s may differ from
  * a sequential fp64 sum by one fp32 rounding in rare cases (the fp64 sum's
  * order is the library's own, fixed).  ws: gce_workspace_bytes(GCE_OP_SIGN).
+ * The two visits of every element (the layer scale, then the update) are
+ * scheduled as gce_set_sign_ahead sets; every schedule gives the same bits.
  */
 GCE_API int ef_sign_step(const gce_table* table, int32_t W, const float* grad, float* mem,
                          float eta, float* vals, void* ws, size_t ws_bytes, void* stream);

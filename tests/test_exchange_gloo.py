@@ -1,8 +1,8 @@
 """Payload exchange between data-parallel ranks (gradient_compression_error_b200.exchange),
 run as gloo ranks on CPU.
 
-Each rank encodes its own worker's gradient with the oracle as a one-worker
-step, packs the payload into one row, and gathers the rows through
+Each rank encodes its own worker's gradient with the oracle (that worker's
+units alone), packs the payload into one row, and gathers the rows through
 PayloadExchange.  The gathered payloads must equal, bit for bit, those of the
 oracle's W-worker step on one process, and so must their sum and (signSGD)
 majority-vote aggregates.  This pins the claim the exchange rests on: one
@@ -23,11 +23,15 @@ LAYERS = {
     "topk": [dict(rows=300, cols=41, kind="topk", cap=123, sigma=1.0),
              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
              dict(rows=5000, cols=1, kind="topk", cap=50, sigma=0.5)],
+    "randk": [dict(rows=300, cols=41, kind="randk", cap=123, sigma=1.0),
+              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
+              dict(rows=5000, cols=1, kind="randk", cap=50, sigma=0.5)],
     "sign": [dict(rows=40, cols=100, kind="sign", cap=0, sigma=1.0),
              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
              dict(rows=1000, cols=1, kind="sign", cap=0, sigma=2.0)],
 }
 ETA = np.float32(0.05)
+SEED, STEP = 41, 3
 
 
 def _slots(lay):
@@ -102,26 +106,29 @@ def _rank(rank, world, port, method, q):
         layers = LAYERS[method]
         k = [l["cap"] for l in layers]
         grad, mem = _inputs(layers, world)
-        # this rank: worker `rank` alone, as a one-worker step
-        m1 = mem[rank:rank + 1].copy()
-        pay1 = osteps.sparse_step(layers, grad[rank:rank + 1], m1, ETA, k, method=method)
-        v, i = _pack(layers, pay1, 0)
-        ex = PayloadExchange(len(v), method == "topk", "cpu")
+        # this rank: worker `rank` alone (its units only; rand-k's generator
+        # takes the job-wide worker index)
+        m1 = mem.copy()
+        pay1 = osteps.sparse_step(layers, grad, m1, ETA, k, method=method, seed=SEED, step=STEP,
+                                  units=[(rank, l) for l in range(len(layers))])
+        v, i = _pack(layers, pay1, rank)
+        sparse = method != "sign"
+        ex = PayloadExchange(len(v), sparse, "cpu")
         # a row of the wrong size is refused on every rank before any collective
         try:
             ex.gather(torch.zeros(len(v) + 1), torch.zeros(len(v) + 1, dtype=torch.int32))
             refused = False
         except ValueError:
             refused = True
-        gv, gi = ex.gather(torch.from_numpy(v), torch.from_numpy(i) if method == "topk" else None)
+        gv, gi = ex.gather(torch.from_numpy(v), torch.from_numpy(i) if sparse else None)
         gathered = {}
         for w in range(world):
             _unpack(layers, gv[w].numpy(), gi[w].numpy() if gi is not None else None, w, gathered)
         # the same W workers on one process
         mW = mem.copy()
-        payW = osteps.sparse_step(layers, grad, mW, ETA, k, method=method)
+        payW = osteps.sparse_step(layers, grad, mW, ETA, k, method=method, seed=SEED, step=STEP)
         same_payload = all(_same_bits(gathered[u], payW[u]) for u in payW)
-        same_mem = np.array_equal(m1[0].view(np.uint32), mW[rank].view(np.uint32))
+        same_mem = np.array_equal(m1[rank].view(np.uint32), mW[rank].view(np.uint32))
         scale = np.float32(1.0 / world)
         s1 = osteps.decompress(layers, world, gathered, scale).view(np.uint32)
         sW = osteps.decompress(layers, world, payW, scale).view(np.uint32)
@@ -154,7 +161,8 @@ def _run(method, world, port):
     return out
 
 
-@pytest.mark.parametrize("method,world,port", [("topk", 2, 29521), ("sign", 3, 29522)])
+@pytest.mark.parametrize("method,world,port", [("topk", 2, 29521), ("sign", 3, 29522),
+                                               ("randk", 2, 29523)])
 def test_one_worker_per_rank_gathers_the_w_worker_step(method, world, port):
     out = _run(method, world, port)
     assert sorted(out) == list(range(world))

@@ -25,11 +25,15 @@ LAYERS = {
     "topk": [dict(rows=300, cols=41, kind="topk", cap=123, sigma=1.0),
              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
              dict(rows=70000, cols=1, kind="topk", cap=700, sigma=0.5)],
+    "randk": [dict(rows=300, cols=41, kind="randk", cap=123, sigma=1.0),
+              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
+              dict(rows=70000, cols=1, kind="randk", cap=700, sigma=0.5)],
     "sign": [dict(rows=40, cols=100, kind="sign", cap=0, sigma=1.0),
              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
              dict(rows=9000, cols=1, kind="sign", cap=0, sigma=2.0)],
 }
 ETA = 0.05
+SEED = 23
 
 
 def _bits(a):
@@ -63,8 +67,8 @@ def _rank(port, method, q):
         for s in range(2):
             grad = workloads.gradients(layers, 1, 940, s)
             pay = osteps.sparse_step(layers, grad.cpu().numpy(), mem_h, np.float32(ETA), k,
-                                     method=method)
-            step(grad, mem, ETA, out)                          # scale 1/world = 1
+                                     method=method, seed=SEED, step=s)
+            step(grad, mem, ETA, out, seed=SEED, step=s)       # scale 1/world = 1
             torch.cuda.synchronize()
             res["sum%d" % s] = np.array_equal(
                 _bits(out.cpu().numpy()), _bits(osteps.decompress(layers, 1, pay, np.float32(1.0))))
@@ -79,14 +83,15 @@ def _rank(port, method, q):
                 res["vote%d" % s] = np.array_equal(
                     _bits(out.cpu().numpy()), _bits(osteps.vote(layers, 1, pay, np.float32(2.0))))
         res["status_clear"] = g.status(step.ws_step) == 0
-        # rand-k payloads are not exchanged: refused on the host before any call
+        # PowerSGD is not exchanged, and a table takes only its own kind's step:
+        # both refused on the host before any call
         rk = g.Table(workloads.table_layers([dict(rows=1000, cols=1, kind="randk", cap=10,
                                                   sigma=1.0)]))
         try:
-            DataParallelStep(rk, "randk")
-            res["randk_refused"] = False
+            DataParallelStep(rk, "powersgd")
+            res["powersgd_refused"] = False
         except ValueError:
-            res["randk_refused"] = True
+            res["powersgd_refused"] = True
         try:
             DataParallelStep(rk, "topk")
             res["kind_mismatch_refused"] = False
@@ -100,7 +105,7 @@ def _rank(port, method, q):
         q.put(res)
 
 
-@pytest.mark.parametrize("method,port", [("topk", 29531), ("sign", 29532)])
+@pytest.mark.parametrize("method,port", [("topk", 29531), ("sign", 29532), ("randk", 29533)])
 def test_one_rank_nccl_step_matches_the_oracle(method, port):
     need_gpu()
     ctx = mp.get_context("spawn")

@@ -138,3 +138,46 @@ def test_bert_base_w8_sampled_units():
         assert np.array_equal(hi[w, sl], ei)
         assert np.array_equal(bits(hv[w, sl]), bits(ev))
         assert np.array_equal(bits(host(mem[w, ls])), bits(em))
+
+
+def test_worker_offset_rows_equal_the_whole_job():
+    """ef_randk_step_at: workers worker0 .. worker0+W-1 of a larger job give,
+    row for row and bit for bit, what one ef_randk_step over the whole job
+    gives those workers (the generator takes the job-wide worker index).
+    Three steps, so the look-ahead record, keyed by worker0 too, is reused."""
+    need_gpu()
+    g = gce()
+    layers = [dict(rows=300, cols=41, kind="randk", cap=123, sigma=1.0),
+              dict(rows=77, cols=1, kind="dense", cap=0, sigma=1.0),
+              dict(rows=70000, cols=1, kind="randk", cap=700, sigma=0.5)]
+    W = 4
+    t = g.Table(workloads.table_layers(layers))
+
+    def run(worker0, w_count, rows):
+        mem = torch.zeros((w_count, t.N), device="cuda")
+        vals = torch.zeros((w_count, max(4, t.vals_per_worker)), device="cuda")
+        idx = torch.zeros((w_count, max(4, t.vals_per_worker)), dtype=torch.int32, device="cuda")
+        ws = t.workspace(w_count, "randk")
+        out = []
+        for s in range(3):
+            grad = workloads.gradients(layers, W, 960, s)[rows].clone()  # 16-byte aligned
+            g.ef_randk_step_at(t, worker0, w_count, grad, mem, 0.05, None, 17, s, vals, idx, ws)
+            out.append((mem.clone(), vals.clone(), idx.clone()))
+        assert g.status(ws) & g.STATUS_K_RANGE == 0
+        return out
+
+    whole = run(0, W, slice(0, W))
+    for worker0, w_count in [(1, 1), (3, 1), (1, 2)]:
+        part = run(worker0, w_count, slice(worker0, worker0 + w_count))
+        for (m, v, i), (mw, vw, iw) in zip(part, whole):
+            rows = slice(worker0, worker0 + w_count)
+            assert torch.equal(m.view(torch.int32), mw[rows].view(torch.int32)), worker0
+            assert torch.equal(v.view(torch.int32), vw[rows].view(torch.int32)), worker0
+            assert torch.equal(i, iw[rows]), worker0
+    with pytest.raises(g.GceError):
+        g.ef_randk_step_at(t, -1, 1, torch.zeros((1, t.N), device="cuda"),
+                           torch.zeros((1, t.N), device="cuda"), 0.05, None, 17, 0,
+                           torch.zeros((1, max(4, t.vals_per_worker)), device="cuda"),
+                           torch.zeros((1, max(4, t.vals_per_worker)), dtype=torch.int32,
+                                       device="cuda"),
+                           t.workspace(1, "randk"))
