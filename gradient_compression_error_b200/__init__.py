@@ -8,9 +8,12 @@ torch CUDA tensors into device pointers and the current CUDA stream into a
 first call raises -- there is no fallback.
 
 The entry points keep the C names: ef_topk_step, ef_randk_step,
-powersgd_init_q, powersgd_step, accordion_init, accordion_select,
-decompress_accumulate, plus the Table wrapper of gce_table_* and the
-workspace / status helpers.
+ef_randk_step_at, ef_sign_step, powersgd_init_q, powersgd_step,
+powersgd_dp_step, accordion_init, accordion_select, decompress_accumulate,
+decompress_apply, decompress_accumulate_noalloc, decompress_vote, plus the
+Table wrapper of gce_table_* and the workspace, status, schedule and profiling
+helpers.  The exchange of payloads between data-parallel ranks sits on top of
+these, in the ``exchange`` module.
 """
 import ctypes as C
 import os
