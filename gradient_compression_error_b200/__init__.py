@@ -95,6 +95,7 @@ SIGNATURES = {
     "gce_set_randk_ahead": (C.c_int, [C.c_int32]),
     "gce_set_sign_ahead": (C.c_int, [C.c_int32]),
     "gce_set_sign_emit_first": (C.c_int, [C.c_int32]),
+    "gce_sign_schedule": (C.c_int, [_vp, _i32, _i32, _i32, _vp, _i64, C.POINTER(_i64)]),
     "gce_profile_start": (C.c_int, []),
     "gce_profile_stop": (C.c_int, []),
     "gce_profile_only": (C.c_int, [C.c_char_p]),
@@ -352,6 +353,20 @@ def set_sign_ahead(tiles):
     """signSGD schedule: the norm runs `tiles` 8192-element tiles ahead of the
     memory update in one launch; 0 runs two passes (include/gce.h)."""
     _check("gce_set_sign_ahead", lib().gce_set_sign_ahead(int(tiles)))
+
+
+def sign_schedule(layer_tiles, W, ahead):
+    """The pipelined signSGD kernel's work-item order (host only): a list of
+    runs (first item, first tile, kind), kind 0 norm, 1 update, -1 the
+    closing sentinel whose first item is the item count (include/gce.h)."""
+    tiles = (C.c_int32 * len(layer_tiles))(*[int(x) for x in layer_tiles])
+    n = _i64()
+    _check("gce_sign_schedule", lib().gce_sign_schedule(tiles, len(layer_tiles), int(W),
+                                                        int(ahead), None, 0, C.byref(n)))
+    runs = (C.c_int64 * (3 * n.value))()
+    _check("gce_sign_schedule", lib().gce_sign_schedule(tiles, len(layer_tiles), int(W),
+                                                        int(ahead), runs, n.value, C.byref(n)))
+    return [(runs[3 * i], runs[3 * i + 1], runs[3 * i + 2]) for i in range(n.value)]
 
 
 def set_sign_emit_first(on):

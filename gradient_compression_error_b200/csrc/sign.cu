@@ -398,9 +398,9 @@ static std::atomic<int32_t> g_sign_emit_first{0};  // test of the bounded wait
 // while the norm is fewer than `ahead` tiles in front, else a run of emit
 // tiles, never past the first layer whose norm tiles are not all placed.
 // ahead < 0 (the wait test): every emit run first, then every norm run.
-static std::vector<SgPhase> sg_schedule(const gce_table* t, int32_t W, int32_t ahead,
-                                        int64_t* nitems) {
-    const int64_t T = int64_t(W) * t->tiles_pw;
+// starts: the first tile of every (worker, layer), ascending; T tiles in all.
+static std::vector<SgPhase> sg_schedule_of(const std::vector<int64_t>& starts, int64_t T,
+                                           int32_t ahead, int64_t* nitems) {
     if (ahead < 0) {
         std::vector<SgPhase> ph;
         int64_t item = 0;
@@ -413,11 +413,6 @@ static std::vector<SgPhase> sg_schedule(const gce_table* t, int32_t W, int32_t a
         *nitems = item;
         return ph;
     }
-    std::vector<int64_t> starts;  // first tile of every (worker, layer), ascending
-    starts.reserve(size_t(W) * t->comp.size());
-    for (int32_t w = 0; w < W; ++w)
-        for (int32_t l : t->comp) starts.push_back(int64_t(w) * t->tiles_pw + t->layers[l].tile0);
-    std::sort(starts.begin(), starts.end());
     std::vector<SgPhase> ph;
     int64_t np = 0, ep = 0, item = 0;  // next norm tile, next emit tile
     while (ep < T) {
@@ -443,6 +438,16 @@ static std::vector<SgPhase> sg_schedule(const gce_table* t, int32_t W, int32_t a
     ph.push_back(SgPhase{item, T, -1, 0});
     *nitems = item;
     return ph;
+}
+
+static std::vector<SgPhase> sg_schedule(const gce_table* t, int32_t W, int32_t ahead,
+                                        int64_t* nitems) {
+    std::vector<int64_t> starts;
+    starts.reserve(size_t(W) * t->comp.size());
+    for (int32_t w = 0; w < W; ++w)
+        for (int32_t l : t->comp) starts.push_back(int64_t(w) * t->tiles_pw + t->layers[l].tile0);
+    std::sort(starts.begin(), starts.end());
+    return sg_schedule_of(starts, int64_t(W) * t->tiles_pw, ahead, nitems);
 }
 
 // The cached schedule of (W, ahead), built and uploaded on first use.  None
@@ -492,6 +497,34 @@ using namespace gce;
 extern "C" int gce_set_sign_ahead(int32_t tiles) {
     if (tiles < 0 || tiles > (1 << 20)) return GCE_ERR_ARG;
     g_sign_ahead.store(tiles);
+    return GCE_OK;
+}
+
+extern "C" int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int32_t W,
+                                 int32_t ahead, int64_t* runs, int64_t cap, int64_t* nruns) {
+    if (!layer_tiles || ncomp < 1 || W < 1 || ahead < -1 || ahead > (1 << 20) || !nruns ||
+        cap < 0 || (cap > 0 && !runs))
+        return GCE_ERR_ARG;
+    int64_t tiles_pw = 0;
+    std::vector<int64_t> tile0(size_t(ncomp), 0);
+    for (int32_t l = 0; l < ncomp; ++l) {
+        if (layer_tiles[l] < 1) return GCE_ERR_ARG;
+        tile0[l] = tiles_pw;
+        tiles_pw += layer_tiles[l];
+    }
+    std::vector<int64_t> starts;
+    starts.reserve(size_t(W) * size_t(ncomp));
+    for (int32_t w = 0; w < W; ++w)
+        for (int32_t l = 0; l < ncomp; ++l) starts.push_back(int64_t(w) * tiles_pw + tile0[l]);
+    int64_t nitems = 0;
+    const std::vector<SgPhase> ph =
+        sg_schedule_of(starts, int64_t(W) * tiles_pw, ahead == -1 ? -1 : ahead, &nitems);
+    *nruns = int64_t(ph.size());
+    for (int64_t i = 0; i < std::min<int64_t>(cap, int64_t(ph.size())); ++i) {
+        runs[3 * i] = ph[size_t(i)].item0;
+        runs[3 * i + 1] = ph[size_t(i)].t0;
+        runs[3 * i + 2] = ph[size_t(i)].kind;
+    }
     return GCE_OK;
 }
 

@@ -303,6 +303,20 @@ GCE_API int gce_set_sign_ahead(int32_t tiles);
 GCE_API int gce_set_sign_emit_first(int32_t on);
 
 /*
+ * The work-item order of the pipelined signSGD kernel, host only (no device
+ * call; for inspection and tests).  For W workers over ncomp SIGN layers of
+ * layer_tiles[l] >= 1 tiles each (8192 elements a tile, layers numbered
+ * consecutively, worker-major), with the norm at most `ahead` tiles in front
+ * (1 .. 2^20), or ahead = -1 for the wait test's order (every update first).
+ * Writes up to cap runs to runs[3 * i ..]: (first item, first tile, kind:
+ * 0 norm, 1 update, -1 the closing sentinel, whose first item is the item
+ * count); *nruns = the number of runs, sentinel included.  Bad arguments
+ * give GCE_ERR_ARG.
+ */
+GCE_API int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int32_t W, int32_t ahead,
+                              int64_t* runs, int64_t cap, int64_t* nruns);
+
+/*
  * Accordion select [ACC] over every compressed layer of the table.
  * Sets prev_norm[l] = -1 (no earlier check) and level[l] = LOW.
  */
