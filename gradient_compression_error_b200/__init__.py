@@ -351,7 +351,8 @@ def set_randk_ahead(on):
 
 def set_sign_ahead(tiles):
     """signSGD schedule: the norm runs `tiles` 8192-element tiles ahead of the
-    memory update in one launch; 0 runs two passes (include/gce.h)."""
+    memory update in one launch; 0 runs two passes; -1 (the default) sizes the
+    look-ahead from the device's L2 (include/gce.h)."""
     _check("gce_set_sign_ahead", lib().gce_set_sign_ahead(int(tiles)))
 
 

@@ -29,6 +29,7 @@
 // same.  The aggregates live in decompress.cu (worker-order sum) and here
 // (the majority vote).
 #include <algorithm>
+#include <cmath>
 
 #include "common.cuh"
 #include "scan.cuh"
@@ -390,8 +391,8 @@ __global__ void __launch_bounds__(128) sg_vote_kernel(
 
 // ---- host: the pipelined schedule, built once per (table, W, ahead) -------------------
 constexpr int64_t kSgRun = 64;             // tiles per run of the schedule
-constexpr int32_t kSgDefaultAhead = 768;   // norm tiles in front of the emit (48 MB of grad+mem)
-static std::atomic<int32_t> g_sign_ahead{kSgDefaultAhead};
+constexpr int32_t kSgAuto = -1;            // look-ahead from the device's L2 size
+static std::atomic<int32_t> g_sign_ahead{kSgAuto};
 static std::atomic<int32_t> g_sign_emit_first{0};  // test of the bounded wait
 
 // The order of the pipelined kernel's work items: runs of kSgRun norm tiles
@@ -450,6 +451,25 @@ static std::vector<SgPhase> sg_schedule(const gce_table* t, int32_t W, int32_t a
     return sg_schedule_of(starts, int64_t(W) * t->tiles_pw, ahead, nitems);
 }
 
+// The look-ahead in tiles: the setting, or by default the tiles (grad and
+// memory, 64 KB each) in 3/8 of the device's L2, rounded to whole runs.  The
+// live window is about twice the look-ahead (norm tiles waiting for their
+// update, plus the tiles in flight), which must stay in L2: on B200 (126 MB)
+// this is 768 tiles, the best of the look-aheads measured there.
+static int32_t sign_ahead_now() {
+    const int32_t a = g_sign_ahead.load();
+    if (a != kSgAuto) return a;
+    int dev = 0, l2 = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev) != cudaSuccess || l2 <= 0) {
+        cudaGetLastError();
+        return 768;
+    }
+    const double tiles = double(l2) * 3.0 / 8.0 / double(kTkTile * 8);
+    const int64_t r = std::llround(tiles / double(kSgRun)) * kSgRun;
+    return int32_t(std::min<int64_t>(std::max<int64_t>(r, kSgRun), int64_t(1) << 20));
+}
+
 // The cached schedule of (W, ahead), built and uploaded on first use.  None
 // while the stream is being captured (no synchronous copy then), or if the
 // item counter could overflow: the caller then runs the two passes.
@@ -495,7 +515,7 @@ void sign_plan_free(gce_table* t) {
 using namespace gce;
 
 extern "C" int gce_set_sign_ahead(int32_t tiles) {
-    if (tiles < 0 || tiles > (1 << 20)) return GCE_ERR_ARG;
+    if (tiles < kSgAuto || tiles > (1 << 20)) return GCE_ERR_ARG;
     g_sign_ahead.store(tiles);
     return GCE_OK;
 }
@@ -553,7 +573,7 @@ extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, fl
         if (cudaMemsetAsync(done, 0, sizeof(int32_t) * size_t(2 * segs + 1), st) != cudaSuccess)
             return GCE_ERR_CUDA;
         const int64_t tiles = int64_t(t->tiles_pw) * W;
-        const int32_t ahead = g_sign_emit_first.load() ? -1 : g_sign_ahead.load();
+        const int32_t ahead = g_sign_emit_first.load() ? -1 : sign_ahead_now();
         SgPlan plan;
         if (ahead != 0 && sg_plan(t, W, ahead, st, &plan)) {
             static const int r_fused = resident_blocks(sg_fused_kernel, 256);

@@ -287,8 +287,10 @@ GCE_API int decompress_vote(const gce_table* table, int32_t W, const float* vals
  * per table and W on first use, outside stream capture: that first call
  * allocates a small device array (cudaMalloc, with its implicit
  * synchronisation) kept until gce_table_destroy; while capturing before
- * that, the two passes run).  0: two passes over the whole set.  Both give
- * the same bits.  Default 768.  tiles outside [0, 2^20] gives GCE_ERR_ARG.
+ * that, the two passes run).  0: two passes over the whole set.  -1 (the
+ * default): the tiles of grad and memory that fill 3/8 of the device's L2,
+ * rounded to a multiple of 64 (768 on B200).  Every setting gives the same
+ * bits.  tiles outside [-1, 2^20] gives GCE_ERR_ARG.
  */
 GCE_API int gce_set_sign_ahead(int32_t tiles);
 

@@ -63,8 +63,8 @@ def test_null_arguments_are_rejected_on_the_host():
                               None) == -1
     assert L.ef_sign_step(None, 1, None, None, 0.1, None, None, 0, None) == -1
     assert L.gce_set_randk_ahead(2) == -1
-    assert L.gce_set_sign_ahead(-1) == -1 and L.gce_set_sign_ahead((1 << 20) + 1) == -1
-    assert L.gce_set_sign_ahead(768) == 0                          # the default, unchanged
+    assert L.gce_set_sign_ahead(-2) == -1 and L.gce_set_sign_ahead((1 << 20) + 1) == -1
+    assert L.gce_set_sign_ahead(-1) == 0                           # back to the default
     assert L.gce_set_sign_emit_first(2) == -1 and L.gce_set_sign_emit_first(0) == 0
     assert L.decompress_vote(None, 1, None, 1.0, None, None) == -1
     e = C.c_float()
