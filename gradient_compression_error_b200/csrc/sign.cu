@@ -394,6 +394,7 @@ constexpr int64_t kSgRun = 64;             // tiles per run of the schedule
 constexpr int32_t kSgAuto = -1;            // look-ahead from the device's L2 size
 static std::atomic<int32_t> g_sign_ahead{kSgAuto};
 static std::atomic<int32_t> g_sign_emit_first{0};  // test of the bounded wait
+constexpr int64_t kSgWaitTestTiles = 8;             // largest table (tiles) it runs on
 
 // The order of the pipelined kernel's work items: runs of kSgRun norm tiles
 // while the norm is fewer than `ahead` tiles in front, else a run of emit
@@ -537,8 +538,7 @@ extern "C" int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int3
     for (int32_t w = 0; w < W; ++w)
         for (int32_t l = 0; l < ncomp; ++l) starts.push_back(int64_t(w) * tiles_pw + tile0[l]);
     int64_t nitems = 0;
-    const std::vector<SgPhase> ph =
-        sg_schedule_of(starts, int64_t(W) * tiles_pw, ahead == -1 ? -1 : ahead, &nitems);
+    const std::vector<SgPhase> ph = sg_schedule_of(starts, int64_t(W) * tiles_pw, ahead, &nitems);
     *nruns = int64_t(ph.size());
     for (int64_t i = 0; i < std::min<int64_t>(cap, int64_t(ph.size())); ++i) {
         runs[3 * i] = ph[size_t(i)].item0;
@@ -567,13 +567,17 @@ extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, fl
     if (t->ckind == GCE_KIND_SIGN && t->tiles_pw > 0) {
         const int32_t ncomp = int32_t(t->comp.size());
         const int64_t segs = int64_t(W) * ncomp;
+        const int64_t tiles = int64_t(t->tiles_pw) * W;
+        const bool emit_first = g_sign_emit_first.load() != 0;
+        // the wait test: every update's wait runs out, one block after another,
+        // so it is refused beyond a few tiles
+        if (emit_first && tiles > kSgWaitTestTiles) return GCE_ERR_ARG;
         int32_t* done = at<int32_t>(ws, lay.sync);
         int32_t* ready = done + segs;
         uint32_t* counter = reinterpret_cast<uint32_t*>(done + 2 * segs);
         if (cudaMemsetAsync(done, 0, sizeof(int32_t) * size_t(2 * segs + 1), st) != cudaSuccess)
             return GCE_ERR_CUDA;
-        const int64_t tiles = int64_t(t->tiles_pw) * W;
-        const int32_t ahead = g_sign_emit_first.load() ? -1 : sign_ahead_now();
+        const int32_t ahead = emit_first ? -1 : sign_ahead_now();
         SgPlan plan;
         if (ahead != 0 && sg_plan(t, W, ahead, st, &plan)) {
             static const int r_fused = resident_blocks(sg_fused_kernel, 256);

@@ -298,9 +298,11 @@ GCE_API int gce_set_sign_ahead(int32_t tiles);
  * Test of the bounded wait in the pipelined signSGD kernel.  on = 1 places
  * every memory-update tile before every norm tile and runs the kernel as one
  * block, so each update's wait for its layer scale runs out (about a second
- * per tile) and sets GCE_STATUS_WAIT_TIMEOUT;
- * that call's results are not valid.  Nothing faults or hangs.  0 (the
- * default) restores the normal order.  Other values give GCE_ERR_ARG.
+ * per tile) and sets GCE_STATUS_WAIT_TIMEOUT; that call's results are not
+ * valid.  Nothing faults or hangs.  While it is on, ef_sign_step refuses
+ * (GCE_ERR_ARG) tables of more than 8 tiles of SIGN layers over all
+ * workers.  0 (the default) restores the normal order.  Other values give
+ * GCE_ERR_ARG.
  */
 GCE_API int gce_set_sign_emit_first(int32_t on);
 

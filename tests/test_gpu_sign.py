@@ -257,10 +257,17 @@ def test_wait_that_runs_out_sets_the_status():
     vals = torch.zeros((1, max(4, t.vals_per_worker)), device="cuda")
     ws = t.workspace(1, "sign")
     grad = workloads.gradients(layers, 1, 952, 0)
+    big = g.Table(workloads.table_layers([dict(rows=9 * 8192, cols=1, kind="sign", cap=0)]))
     try:
         g.set_sign_emit_first(True)
         g.ef_sign_step(t, 1, grad, mem, 0.05, vals, ws)
         st = g.status(ws)
+        # more than 8 tiles: refused on the host, nothing launched
+        with pytest.raises(g.GceError):
+            g.ef_sign_step(big, 1, torch.zeros((1, big.N), device="cuda"),
+                           torch.zeros((1, big.N), device="cuda"), 0.05,
+                           torch.zeros((1, max(4, big.vals_per_worker)), device="cuda"),
+                           big.workspace(1, "sign"))
     finally:
         g.set_sign_emit_first(False)
     assert st & g.STATUS_WAIT_TIMEOUT
