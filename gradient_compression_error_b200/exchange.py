@@ -12,10 +12,9 @@ GPU.
 
 Rank r's row lands where worker r's row sits in the one-GPU layout
 ([W, vals_per_worker] floats, and the same for the int32 indices of top-k and
-rand-k), so
-the decode is bit for bit the decode of W replicas whose worker r holds rank
-r's gradient and memory: each (worker, layer) encode is independent of the
-other workers, and the decode adds the workers in index order.
+rand-k), so the decode is bit for bit the decode of W replicas whose worker r
+holds rank r's gradient and memory: each (worker, layer) encode is independent
+of the other workers, and the decode adds the workers in index order.
 
 Only torch.distributed moves bytes here (NCCL between GPUs, gloo on CPU); the
 arithmetic of the method runs in the native library.  The ranks must agree on
