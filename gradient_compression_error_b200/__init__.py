@@ -24,6 +24,7 @@ KIND = {"topk": 0, "randk": 1, "powersgd": 2, "dense": 3, "sign": 4}
 KIND_NAME = {v: k for k, v in KIND.items()}
 OP = {"topk": 0, "randk": 1, "powersgd": 2, "accordion": 3, "decompress": 4, "powersgd_dp": 5,
       "sign": 6}
+OPT = {"bracket_sigma": 0, "randk_ahead": 1, "sign_ahead": 2, "sign_emit_first": 3}
 STATUS_K_RANGE = 1
 STATUS_FALLBACK = 2
 STATUS_NONFINITE = 4
@@ -92,6 +93,9 @@ SIGNATURES = {
     "gce_launch_count": (_u64, []),
     "gce_error_string": (C.c_char_p, [C.c_int]),
     "gce_set_bracket_sigma": (C.c_int, [_f64]),
+    "gce_table_set_option": (C.c_int, [_vp, _i32, _f64]),
+    "gce_table_reset_option": (C.c_int, [_vp, _i32]),
+    "gce_table_get_option": (C.c_int, [_vp, _i32, C.POINTER(_f64)]),
     "gce_set_randk_ahead": (C.c_int, [C.c_int32]),
     "gce_set_sign_ahead": (C.c_int, [C.c_int32]),
     "gce_set_sign_emit_first": (C.c_int, [C.c_int32]),
@@ -179,6 +183,22 @@ class Table:
             self.close()
         except Exception:
             pass
+
+    def set_option(self, name, value):
+        """This table's own value of a setting (include/gce.h, GCE_OPT_*)."""
+        _check("gce_table_set_option", lib().gce_table_set_option(self.handle, OPT[name],
+                                                                  float(value)))
+
+    def reset_option(self, name):
+        """Follow the process-wide value of a setting again."""
+        _check("gce_table_reset_option", lib().gce_table_reset_option(self.handle, OPT[name]))
+
+    def option(self, name):
+        """The value of a setting that a call on this table uses now."""
+        v = C.c_double()
+        _check("gce_table_get_option", lib().gce_table_get_option(self.handle, OPT[name],
+                                                                  C.byref(v)))
+        return v.value
 
     def workspace_bytes(self, W, op):
         n = C.c_size_t()

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstddef>
 #include <cstdint>
 #include <mutex>
@@ -110,6 +111,9 @@ struct gce_table {
     // destroyed; guarded by sg_mu
     mutable std::mutex sg_mu;
     mutable std::vector<gce::SgPlan> sg_plans;
+    // settings of this table (gce_table_set_option), one per GCE_OPT_*; NaN:
+    // follow the process-wide setting
+    std::atomic<double> opt[4] = {NAN, NAN, NAN, NAN};
 };
 
 namespace gce {
@@ -136,6 +140,11 @@ void prof_after(cudaStream_t st);
 inline int check_launch() {
     return cudaGetLastError() == cudaSuccess ? GCE_OK : GCE_ERR_CUDA;
 }
+
+// ---- settings that move work or test a wait ------------------------------------
+// The value a call on table t uses for option `opt` (GCE_OPT_*): the table's
+// own, else the process-wide one.  Read once per call.
+double option_of(const gce_table* t, int opt);
 
 // ---- device properties (cached per device) --------------------------------
 int sm_count();

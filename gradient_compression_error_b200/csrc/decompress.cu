@@ -125,8 +125,6 @@ __device__ __forceinline__ void dc_add_staged(float* acc, const int32_t* s_sidx,
     }
 }
 
-// Write this warp's kDcSpan outputs (times scale) and zero them in the
-// accumulator for the next tile.  Run by a full warp after __syncwarp.
 // Write this warp's kDcSpan outputs and zero them in the accumulator for the
 // next tile: out = fl(scale * sum), or with kApply x = fl(x - fl(scale * sum)).
 // Run by a full warp after __syncwarp.
@@ -162,7 +160,12 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     const float* __restrict__ Q, const int32_t* __restrict__ bounds, float scale,
     float* __restrict__ out) {
     __shared__ __align__(16) float acc[kDcTile];
-    __shared__ int32_t s_first[32], s_off[33];
+    // per-worker entry ranges of the tile, double-buffered by sparse-tile
+    // parity: warp 0 fills the next tile's copy while a slower warp may still
+    // be reading this tile's in dc_add_staged (no barrier lies between the
+    // two); the copy is reused only after the next tile's barrier, which every
+    // warp reaches after it has finished with this tile
+    __shared__ int32_t s_first2[2][32], s_off2[2][33];
     __shared__ int32_t s_sidx[kDcStage];
     __shared__ float s_sval[kDcStage];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -171,6 +174,7 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
         reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
+    int par = 0;  // parity of the staged sparse tiles this block has taken
     for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
         const int32_t t = tile_list ? tile_list[u] : u;
         const int32_t l = dc_tile_layer[t];
@@ -188,6 +192,9 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
                 // between the adds and the write.  Every worker's entry range
                 // for the tile is read at once, then the entries are staged
                 // in worker order, kDcStage at a time.
+                int32_t* s_first = s_first2[par];
+                int32_t* s_off = s_off2[par];
+                par ^= 1;
                 if (warp == 0) {
                     int32_t a = 0, e = 0;
                     if (lane < W) {
@@ -203,8 +210,6 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
                 }
                 __syncthreads();
                 const int total = s_off[32];
-                // at least one pass, so that every warp has read this tile's
-                // s_off before warp 0 writes the next tile's
                 int c0 = 0;
                 do {
                     const int cn = min(kDcStage, total - c0);
@@ -506,17 +511,34 @@ extern "C" int gce_memsgd_eta(int64_t step, double mu, double a, float* eta) {
 constexpr int64_t kNoAllocBoundSlots = int64_t(1) << 20;
 static __device__ __align__(256) int32_t g_noalloc_bounds[kNoAllocBoundSlots];
 
-// Device address of g_noalloc_bounds on the current device, looked up once per
-// device (host code cannot use the symbol itself as a device address).
-static int32_t* noalloc_bounds_on_current_device() {
+// Device address of g_noalloc_bounds on the current device (host code cannot
+// use the symbol itself as a device address).  Looked up again on every call
+// made outside stream capture, so a context re-created after cudaDeviceReset
+// gets its own array's address; during capture the address of the last call
+// outside capture on that device is used (the first call on a device must not
+// be captured).  A failed look-up clears the runtime's error state so that it
+// does not surface in a later, unrelated call.
+static int32_t* noalloc_bounds_on_current_device(cudaStream_t st) {
     static std::mutex mu;
     static int32_t* addr[64] = {};
     int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
     std::lock_guard<std::mutex> lk(mu);
-    if (!addr[dev]) {
+    if (cs == cudaStreamCaptureStatusNone || !addr[dev]) {
+        if (cs != cudaStreamCaptureStatusNone) return nullptr;  // never looked up outside capture
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_bounds) != cudaSuccess || !p) return nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_bounds) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return nullptr;
+        }
         addr[dev] = static_cast<int32_t*>(p);
     }
     return addr[dev];
@@ -531,10 +553,10 @@ extern "C" int decompress_accumulate_noalloc(const gce_table* t, int32_t W, cons
     if ((t->vals_pw > 0 && !vals) || (sparse && !idx)) return GCE_ERR_ARG;
     if (t->ckind == GCE_KIND_POWERSGD && (!P || !Q)) return GCE_ERR_ARG;
     if (int64_t(W) * t->dc_slots > kNoAllocBoundSlots) return GCE_ERR_WORKSPACE;
-    int32_t* bounds = noalloc_bounds_on_current_device();
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* bounds = noalloc_bounds_on_current_device(st);
     if (!bounds) return GCE_ERR_CUDA;
     // every bound slot a sparse layer uses is rewritten by the bounds pass, so
     // nothing left from an earlier call needs clearing
-    return launch_decode(t, W, vals, idx, k_or_rank, P, Q, scale, out, bounds,
-                         static_cast<cudaStream_t>(stream));
+    return launch_decode(t, W, vals, idx, k_or_rank, P, Q, scale, out, bounds, st);
 }

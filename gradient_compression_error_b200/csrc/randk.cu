@@ -29,9 +29,7 @@
 
 namespace gce {
 
-extern double bracket_sigma();
 
-static bool g_randk_ahead = true;  // run the next step's key pass ahead (see gce.h)
 
 struct RkSeg {
     int32_t k;       // 0: layer skipped
@@ -566,7 +564,9 @@ static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const floa
         // the stream is being captured (a graph would replay one step number).
         cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
         if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return GCE_ERR_CUDA;
-        const bool pipe = g_randk_ahead && cs == cudaStreamCaptureStatusNone &&
+        const double sigma = option_of(t, GCE_OPT_BRACKET_SIGMA);
+        const bool pipe = option_of(t, GCE_OPT_RANDK_AHEAD) != 0.0 &&
+                          cs == cudaStreamCaptureStatusNone &&
                           step != ~uint64_t(0);
         bool have = false;
         {
@@ -597,12 +597,12 @@ static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const floa
         if (have) {
             GCE_LAUNCH(rk_refresh_k_kernel, wave_grid((lay.S + 255) / 256, 4, r_refresh), 256, 0,
                        st, t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
-                       uint64_t(worker0), step, bracket_sigma(), segs, status, tag,
+                       uint64_t(worker0), step, sigma, segs, status, tag,
                        tag_of(step));
         } else {
             GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st,
                        t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
-                       uint64_t(worker0), step, bracket_sigma(), segs, status, tag,
+                       uint64_t(worker0), step, sigma, segs, status, tag,
                        uint64_t(0));
             GCE_LAUNCH(rk_keys_kernel<false>, wave_grid(lay.TT, 8, r_keys0), 256, 0, st,
                        t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->comp_N, segs,
@@ -624,7 +624,7 @@ static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const floa
             // resolve of that step re-reads k and repairs any miss)
             GCE_LAUNCH(rk_setup_kernel, wave_grid((lay.S + 255) / 256, 4, r_setup), 256, 0, st,
                        t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
-                       uint64_t(worker0), step + 1, bracket_sigma(), segs_next, nullptr, tag,
+                       uint64_t(worker0), step + 1, sigma, segs_next, nullptr, tag,
                        tag_of(step + 1));
             GCE_LAUNCH(rk_emit_kernel<true>, wave_grid(lay.TT, r_emit1, r_emit1), kTkThreads, 0, st,
                        t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
@@ -663,10 +663,4 @@ extern "C" int ef_randk_step_at(const gce_table* t, int64_t worker0, int32_t W, 
                                 size_t ws_bytes, void* stream) {
     return randk_step(t, W, worker0, grad, mem, eta, k_or_rank, seed, step, vals, idx, ws,
                       ws_bytes, stream);
-}
-
-extern "C" int gce_set_randk_ahead(int32_t on) {
-    if (on != 0 && on != 1) return GCE_ERR_ARG;
-    g_randk_ahead = on != 0;
-    return GCE_OK;
 }

@@ -392,8 +392,6 @@ __global__ void __launch_bounds__(128) sg_vote_kernel(
 // ---- host: the pipelined schedule, built once per (table, W, ahead) -------------------
 constexpr int64_t kSgRun = 64;             // tiles per run of the schedule
 constexpr int32_t kSgAuto = -1;            // look-ahead from the device's L2 size
-static std::atomic<int32_t> g_sign_ahead{kSgAuto};
-static std::atomic<int32_t> g_sign_emit_first{0};  // test of the bounded wait
 constexpr int64_t kSgWaitTestTiles = 8;             // largest table (tiles) it runs on
 
 // The order of the pipelined kernel's work items: runs of kSgRun norm tiles
@@ -457,8 +455,8 @@ static std::vector<SgPhase> sg_schedule(const gce_table* t, int32_t W, int32_t a
 // live window is about twice the look-ahead (norm tiles waiting for their
 // update, plus the tiles in flight), which must stay in L2: on B200 (126 MB)
 // this is 768 tiles, the best of the look-aheads measured there.
-static int32_t sign_ahead_now() {
-    const int32_t a = g_sign_ahead.load();
+static int32_t sign_ahead_now(const gce_table* t) {
+    const int32_t a = int32_t(option_of(t, GCE_OPT_SIGN_AHEAD));
     if (a != kSgAuto) return a;
     int dev = 0, l2 = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -515,12 +513,6 @@ void sign_plan_free(gce_table* t) {
 
 using namespace gce;
 
-extern "C" int gce_set_sign_ahead(int32_t tiles) {
-    if (tiles < kSgAuto || tiles > (1 << 20)) return GCE_ERR_ARG;
-    g_sign_ahead.store(tiles);
-    return GCE_OK;
-}
-
 extern "C" int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int32_t W,
                                  int32_t ahead, int64_t* runs, int64_t cap, int64_t* nruns) {
     if (!layer_tiles || ncomp < 1 || W < 1 || ahead < -1 || ahead > (1 << 20) || !nruns ||
@@ -548,12 +540,6 @@ extern "C" int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int3
     return GCE_OK;
 }
 
-extern "C" int gce_set_sign_emit_first(int32_t on) {
-    if (on != 0 && on != 1) return GCE_ERR_ARG;
-    g_sign_emit_first.store(on);
-    return GCE_OK;
-}
-
 extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, float* mem,
                             float eta, float* vals, void* ws, size_t ws_bytes, void* stream) {
     if (!t || W < 1 || !grad || !mem || !ws) return GCE_ERR_ARG;
@@ -568,7 +554,7 @@ extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, fl
         const int32_t ncomp = int32_t(t->comp.size());
         const int64_t segs = int64_t(W) * ncomp;
         const int64_t tiles = int64_t(t->tiles_pw) * W;
-        const bool emit_first = g_sign_emit_first.load() != 0;
+        const bool emit_first = option_of(t, GCE_OPT_SIGN_EMIT_FIRST) != 0.0;
         // the wait test: every update's wait runs out, one block after another,
         // so it is refused beyond a few tiles
         if (emit_first && tiles > kSgWaitTestTiles) return GCE_ERR_ARG;
@@ -577,7 +563,7 @@ extern "C" int ef_sign_step(const gce_table* t, int32_t W, const float* grad, fl
         uint32_t* counter = reinterpret_cast<uint32_t*>(done + 2 * segs);
         if (cudaMemsetAsync(done, 0, sizeof(int32_t) * size_t(2 * segs + 1), st) != cudaSuccess)
             return GCE_ERR_CUDA;
-        const int32_t ahead = emit_first ? -1 : sign_ahead_now();
+        const int32_t ahead = emit_first ? -1 : sign_ahead_now(t);
         SgPlan plan;
         if (ahead != 0 && sg_plan(t, W, ahead, st, &plan)) {
             static const int r_fused = resident_blocks(sg_fused_kernel, 256);

@@ -1,5 +1,6 @@
 // table.cu -- layer table, workspace queries, status word, launch counter,
 // and the kernel for uncompressed (DENSE) layers shared by every step.
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -58,6 +59,35 @@ void prof_after(cudaStream_t st) {
     ProfRec& r = g_prof_recs.back();
     r.b = prof_event();
     if (r.b) cudaEventRecord(r.b, st);
+}
+
+// ---- settings: process-wide values and each table's own -------------------------
+namespace {
+// defaults: bracket margin 6 sigma, rand-k look-ahead on, signSGD look-ahead
+// from L2 (-1), wait test off
+std::atomic<double> g_opt[4] = {6.0, 1.0, -1.0, 0.0};
+
+bool option_valid(int opt, double v) {
+    switch (opt) {
+        case GCE_OPT_BRACKET_SIGMA: return v > -100.0 && v < 100.0;
+        case GCE_OPT_RANDK_AHEAD:
+        case GCE_OPT_SIGN_EMIT_FIRST: return v == 0.0 || v == 1.0;
+        case GCE_OPT_SIGN_AHEAD:
+            return v >= -1.0 && v <= double(1 << 20) && v == std::floor(v);
+        default: return false;
+    }
+}
+
+int set_process_option(int opt, double v) {
+    if (!option_valid(opt, v)) return GCE_ERR_ARG;
+    g_opt[opt].store(v);
+    return GCE_OK;
+}
+}  // namespace
+
+double option_of(const gce_table* t, int opt) {
+    const double v = t ? t->opt[opt].load(std::memory_order_relaxed) : NAN;
+    return std::isnan(v) ? g_opt[opt].load(std::memory_order_relaxed) : v;
 }
 
 int sm_count() {
@@ -422,4 +452,38 @@ extern "C" const char* gce_error_string(int code) {
         case GCE_ERR_KIND: return "layer kinds do not fit this call";
         default: return "unknown error";
     }
+}
+
+extern "C" int gce_set_bracket_sigma(double sigma) {
+    return set_process_option(GCE_OPT_BRACKET_SIGMA, sigma);
+}
+
+extern "C" int gce_set_randk_ahead(int32_t on) {
+    return set_process_option(GCE_OPT_RANDK_AHEAD, double(on));
+}
+
+extern "C" int gce_set_sign_ahead(int32_t tiles) {
+    return set_process_option(GCE_OPT_SIGN_AHEAD, double(tiles));
+}
+
+extern "C" int gce_set_sign_emit_first(int32_t on) {
+    return set_process_option(GCE_OPT_SIGN_EMIT_FIRST, double(on));
+}
+
+extern "C" int gce_table_set_option(gce_table* t, int32_t option, double value) {
+    if (!t || option < 0 || option > 3 || !option_valid(option, value)) return GCE_ERR_ARG;
+    t->opt[option].store(value);
+    return GCE_OK;
+}
+
+extern "C" int gce_table_reset_option(gce_table* t, int32_t option) {
+    if (!t || option < 0 || option > 3) return GCE_ERR_ARG;
+    t->opt[option].store(NAN);
+    return GCE_OK;
+}
+
+extern "C" int gce_table_get_option(const gce_table* t, int32_t option, double* value) {
+    if (!t || option < 0 || option > 3 || !value) return GCE_ERR_ARG;
+    *value = option_of(t, option);
+    return GCE_OK;
 }

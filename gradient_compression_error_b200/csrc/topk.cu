@@ -38,9 +38,6 @@
 
 namespace gce {
 
-static double g_bracket_sigma = 6.0;
-double bracket_sigma() { return g_bracket_sigma; }
-
 struct TkLayout {
     int64_t S = 0, TT = 0;
     size_t segs = 0, hists = 0, unit_start = 0, unit_seg = 0, redo_list = 0, tile_dir = 0,
@@ -702,12 +699,6 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
 
 using namespace gce;
 
-extern "C" int gce_set_bracket_sigma(double sigma) {
-    if (!(sigma > -100.0 && sigma < 100.0)) return GCE_ERR_ARG;
-    g_bracket_sigma = sigma;
-    return GCE_OK;
-}
-
 extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
                             const int32_t* k_or_rank, float* vals, int32_t* idx, void* ws,
                             size_t ws_bytes, void* stream) {
@@ -751,7 +742,8 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         if (t->sunits_pw > 0)
             GCE_LAUNCH(tk_sample_kernel, wave_grid(int64_t(t->sunits_pw) * W, 8, r_sample), 256, 0, st,
                        t->d_layers, t->d_sunit_layer, t->d_sunit_part, t->sunits_pw, W, ncomp,
-                       lay.S, t->N, grad, mem, eta, segs, hists, g_bracket_sigma);
+                       lay.S, t->N, grad, mem, eta, segs, hists,
+                       option_of(t, GCE_OPT_BRACKET_SIGMA));
         GCE_LAUNCH(tk_main_kernel, wave_grid(lay.TT, r_main, r_main), kTkThreads, 0, st, t->d_layers,
                    t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->comp_N, grad, mem, eta, segs,
                    tile_dir, spill_v, spill_i, status);

@@ -397,10 +397,15 @@ GCE_API int gce_memsgd_eta(int64_t step, double mu, double a, float* eta);
  * that loads the library until the process exits, so the table and W must
  * satisfy W x (decode tiles of 4096 elements + layers) <= 1,048,576 (the
  * BERT-base table at W = 8 needs 214,144); larger ones return
- * GCE_ERR_WORKSPACE.  The first call on a device looks up that device's copy
- * of the array (cudaGetSymbolAddress), so make it before any stream capture.
- * All calls share the one array: calls that overlap on the GPU (two streams,
- * two threads) race and must be serialised by the caller.
+ * GCE_ERR_WORKSPACE.  Every call made outside stream capture looks up the
+ * current device's copy of the array (cudaGetSymbolAddress); a call made
+ * while its stream is being captured reuses the address of the last call
+ * outside capture on that device, so make the first call on a device before
+ * any capture (a captured first call returns GCE_ERR_CUDA).  A device reset
+ * (cudaDeviceReset) gives the device a new array: graphs captured before it
+ * must not be replayed after it.  All calls share the one array: calls that
+ * overlap on the GPU (two streams, two threads) race and must be serialised
+ * by the caller.
  */
 GCE_API int decompress_accumulate_noalloc(const gce_table* table, int32_t W, const float* vals,
                                           const int32_t* idx, const int32_t* k_or_rank,
@@ -435,8 +440,36 @@ GCE_API const char* gce_error_string(int code);
 
 /* Tuning knob for the approximate pre-selection of top-k / rand-k: the safety
  * margin in standard deviations (default 6).  Results never depend on it;
- * small values only make the exact fallback run more often. */
+ * small values only make the exact fallback run more often.  Values outside
+ * (-100, 100) give GCE_ERR_ARG. */
 GCE_API int gce_set_bracket_sigma(double sigma);
+
+/*
+ * Per-table settings.  gce_set_bracket_sigma, gce_set_randk_ahead,
+ * gce_set_sign_ahead and gce_set_sign_emit_first set process-wide values
+ * (atomically; a call reads them once, when it is made).  A table follows
+ * them until one of its own options is set here; from then on calls on that
+ * table use the table's value, whatever the process-wide one, so two tables
+ * driven from two threads can hold different settings without sharing state.
+ * Options and their values (as the process-wide setters check them):
+ *   GCE_OPT_BRACKET_SIGMA    margin in standard deviations, in (-100, 100)
+ *   GCE_OPT_RANDK_AHEAD      0 or 1
+ *   GCE_OPT_SIGN_AHEAD       an integer in [-1, 2^20] (tiles; -1 = from L2)
+ *   GCE_OPT_SIGN_EMIT_FIRST  0 or 1 (the bounded-wait test)
+ * None of them changes any result.  A bad table, option or value gives
+ * GCE_ERR_ARG.  gce_table_reset_option makes the table follow the
+ * process-wide value again; gce_table_get_option writes the value a call on
+ * the table would use now into *value (host memory).  Setting an option while
+ * another thread runs a step on the same table is allowed; that step uses
+ * either the old or the new value.
+ */
+#define GCE_OPT_BRACKET_SIGMA 0
+#define GCE_OPT_RANDK_AHEAD 1
+#define GCE_OPT_SIGN_AHEAD 2
+#define GCE_OPT_SIGN_EMIT_FIRST 3
+GCE_API int gce_table_set_option(gce_table* table, int32_t option, double value);
+GCE_API int gce_table_reset_option(gce_table* table, int32_t option);
+GCE_API int gce_table_get_option(const gce_table* table, int32_t option, double* value);
 
 #ifdef __cplusplus
 }

@@ -34,6 +34,7 @@ def lib():
             "or_ef_randk": (C.c_int, [i64, i64, f32, vp, vp, vp, vp, u64, u64, u64, u64]),
             "or_dense": (C.c_int, [i64, f32, vp, vp, vp]),
             "or_powersgd_init_q": (C.c_int, [i64, i64, u64, u64, u64, vp]),
+            "or_q_entry": (f32, [u64]),
             "or_powersgd": (C.c_int, [i64, i64, i64, i64, f32, vp, vp, vp, vp, vp]),
             "or_powersgd_dp": (C.c_int, [i64, i64, i64, i64, i64, f32, vp, vp, vp, vp]),
             "or_dense_dp": (C.c_int, [i64, i64, f32, vp, vp, vp]),
@@ -118,6 +119,11 @@ def dense_unit(g, m, eta):
     _check(lib().or_dense(g.size, float(np.float32(eta)), _ptr(g), _ptr(m), _ptr(out)),
            "dense")
     return out, m
+
+
+def q_entry(h):
+    """The warm-start Q entry in [-1, 1) of one 64-bit generator output."""
+    return np.float32(lib().or_q_entry(int(h) & (2**64 - 1)))
 
 
 def powersgd_init_q(cols, r_max, seed, worker, layer):

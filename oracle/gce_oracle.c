@@ -61,10 +61,16 @@
  *     m_w = M_w - P Q_w^T; a DENSE layer sends the workers' mean residual
  *     (fp32 sum in worker order, then times fl32(1/W)).
  *
- * Parity unpinned (nothing on the pages fixes it):
- *   or_randk_base / the stream composition of the rand-k and Q-init hashes
- *   (the SplitMix64 step itself is pinned by its published outputs);
- *   or_powersgd_init_q's mapping of hash bits to [-1, 1).
+ * Pins of the generator readings (nothing on the pages fixes them; they
+ * are pinned against their stated definitions by hand-worked values):
+ *   or_splitmix64_output: the published SplitMix64 outputs;
+ *   or_randk_base: its first fold is a published output (seed as the state,
+ *   stream + 1 as the counter), the later folds a hand-worked chain
+ *   (tests/golden/randk_base_hand.txt);
+ *   or_q_entry: hand-worked values of the [-1, 1) mapping on published
+ *   outputs (tests/golden/powersgd_init_q_hand.txt).
+ * Parity unpinned: the rand-k subset distribution beyond uniformity (checked
+ * statistically only).
  */
 #include <math.h>
 #include <stdint.h>
@@ -245,19 +251,27 @@ int or_dense(int64_t n, float eta, const float* g, float* m, float* payload)
 }
 
 /* ------------------------------------------------------------------ */
+/* One warm-start Q entry from a 64-bit generator output h: its top 24 bits,
+ * read as an integer t in [0, 2^24), give x = t * 2^-23 - 1 in [-1, 1).
+ * Both operations are exact in fp32 (t has 24 bits; the difference is a
+ * multiple of 2^-23 below 1 in magnitude). */
+float or_q_entry(uint64_t h)
+{
+    return (float)(h >> 40) * (1.0f / 8388608.0f) - 1.0f;
+}
+
 /* PowerSGD warm-start Q: entries uniform in [-1, 1) drawn from the hash with
- * stream 1; x = (h >> 40) * 2^-23 - 1, exact in fp32.  Q is cols x r_max,
- * row-major; element (c, j) uses counter c*r_max + j. */
+ * stream 1 (or_q_entry of each output).  Q is cols x r_max, row-major;
+ * element (c, j) uses counter c*r_max + j. */
 int or_powersgd_init_q(int64_t cols, int64_t r_max, uint64_t seed, uint64_t worker,
                        uint64_t layer, float* Q)
 {
     if (cols < 1 || r_max < 1) return OR_ERR_ARG;
     uint64_t base = or_randk_base(seed, 1, worker, layer, 0);
     for (int64_t c = 0; c < cols; ++c)
-        for (int64_t j = 0; j < r_max; ++j) {
-            uint64_t h = or_splitmix64_output(base, (uint64_t)(c * r_max + j) + 1);
-            Q[c * r_max + j] = (float)(h >> 40) * (1.0f / 8388608.0f) - 1.0f;
-        }
+        for (int64_t j = 0; j < r_max; ++j)
+            Q[c * r_max + j] =
+                or_q_entry(or_splitmix64_output(base, (uint64_t)(c * r_max + j) + 1));
     return OR_OK;
 }
 

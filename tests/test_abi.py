@@ -67,6 +67,12 @@ def test_null_arguments_are_rejected_on_the_host():
     assert L.gce_set_sign_ahead(-1) == 0                           # back to the default
     assert L.gce_set_sign_emit_first(2) == -1 and L.gce_set_sign_emit_first(0) == 0
     assert L.decompress_vote(None, 1, None, 1.0, None, None) == -1
+    v = C.c_double()
+    assert L.gce_table_set_option(None, 0, 1.0) == -1
+    assert L.gce_table_reset_option(None, 0) == -1
+    assert L.gce_table_get_option(None, 0, C.byref(v)) == -1
+    assert L.gce_set_bracket_sigma(C.c_double(100.0)) == -1
+    assert L.gce_set_bracket_sigma(C.c_double(6.0)) == 0          # back to the default
     e = C.c_float()
     assert L.gce_memsgd_eta(0, 0.0, 1.0, C.byref(e)) == -1        # mu <= 0
     assert L.gce_memsgd_eta(3, 1.0, -3.0, C.byref(e)) == -1       # a + t <= 0

@@ -7,8 +7,13 @@ Systems", Method / Key results: sign SGD, one bit per element, gathered;
 bit-exact.  The scale is an fp64 sum rounded once to fp32; the library adds
 in its own fixed order, the oracle in index order, so the two may differ by
 one fp32 step (never seen in practice): the test asserts equality within one
-step and, where the scales are equal, the memory bit for bit.  Both
-aggregates, run on the library's own payload, are bit-exact.
+step and, where the scales are equal, the memory bit for bit.  The oracle
+always follows its own trajectory and never takes the library's state.  Where
+the scales differ, the memories of that step may differ by at most the scale
+difference plus one rounding of the memory, and the two trajectories part:
+from then on that unit is checked step by step against a separate oracle call
+on the inputs the library's step had (its previous memory), with the same
+rules.  Both aggregates, run on the library's own payload, are bit-exact.
 """
 import numpy as np
 import pytest
@@ -46,9 +51,11 @@ class SignRun:
         self.vals = torch.zeros((W, max(4, t.vals_per_worker)), device="cuda")
         self.ws = t.workspace(W, "sign")
         self.hmem = np.zeros((W, t.N), np.float32)
+        self.parted = set()   # units whose trajectories parted at a scale difference
 
     def step(self, grad, eta, check=True):
         hg = host(grad)
+        gmem_old = host(self.mem) if check and self.parted else None
         expect = osteps.sparse_step(self.layers, hg, self.hmem, eta, None, method="sign",
                                     threads=8) if check else None
         self.g.ef_sign_step(self.t, self.W, grad, self.mem, eta, self.vals, self.ws)
@@ -64,15 +71,32 @@ class SignRun:
                 assert np.array_equal(bits(pay[(w, l)]), bits(e)), (w, l)
                 assert np.array_equal(bits(hm[w, ls]), bits(self.hmem[w, ls])), (w, l)
                 continue
-            sc, words = pay[(w, l)]
-            e_sc, e_words = e
-            assert np.array_equal(words, e_words), ("bits", w, l)
-            assert abs(int(bits(sc)) - int(bits(e_sc))) <= 1, ("scale", w, l, sc, e_sc)
-            if sc == e_sc:
-                assert np.array_equal(bits(hm[w, ls]), bits(self.hmem[w, ls])), ("mem", w, l)
-            else:   # keep following the library's trajectory
-                self.hmem[w, ls] = hm[w, ls]
+            m_ref = self.hmem[w, ls]
+            if (w, l) in self.parted:
+                # single-step parity from the inputs this step had on the GPU
+                m_ref = gmem_old[w, ls].copy()
+                e = oracle.ef_sign_unit(hg[w, ls], m_ref, eta)
+                e, m_ref = (e[0], e[1]), e[2]
+            if not same_step(pay[(w, l)], hm[w, ls], e, m_ref, (w, l)):
+                self.parted.add((w, l))
         return pay
+
+
+def same_step(got, m_gpu, e, m_ref, unit):
+    """Sign bits equal, scales within one fp32 step, memory bit for bit when
+    the scales agree and within their difference plus one rounding when not.
+    Returns whether the scales agreed."""
+    sc, words = got
+    e_sc, e_words = e
+    assert np.array_equal(words, e_words), ("bits", unit)
+    assert abs(int(bits(sc)) - int(bits(e_sc))) <= 1, ("scale", unit, sc, e_sc)
+    if sc == e_sc:
+        assert np.array_equal(bits(m_gpu), bits(m_ref)), ("mem", unit)
+        return True
+    mg, mr = m_gpu.astype(np.float64), m_ref.astype(np.float64)
+    slack = np.spacing(np.maximum(np.abs(m_gpu), np.abs(m_ref)))
+    assert np.all(np.abs(mg - mr) <= abs(float(sc) - float(e_sc)) + slack), ("mem", unit)
+    return False
 
 
 RAGGED = [dict(rows=1, cols=1, kind="sign", cap=0),

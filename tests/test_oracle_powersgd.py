@@ -13,6 +13,7 @@ import numpy as np
 import pytest
 
 import oracle
+from tests.conftest import read_golden_rows
 
 
 def rel(a, b):
@@ -129,14 +130,32 @@ def test_zero_matrix_gives_zero_columns():
     assert not np.any(P) and not np.any(Qn[:, :2]) and not np.any(Mhat) and not np.any(m_new)
 
 
-def test_init_q_range_and_mapping():
+def test_q_entry_hand_worked_values():
+    """The [-1, 1) mapping of a generator output, against values worked by
+    hand on the published SplitMix64 outputs and the two extreme words
+    (tests/golden/powersgd_init_q_hand.txt)."""
+    from fractions import Fraction
+    rows = read_golden_rows("powersgd_init_q_hand.txt")
+    assert len(rows) == 5
+    for h, t, x in rows:
+        h, t = int(h), int(t)
+        assert h >> 40 == t
+        assert Fraction(oracle.q_entry(h).item()) == Fraction(x)
+
+
+def test_init_q_range_and_counter_order():
     Q = oracle.powersgd_init_q(1000, 4, 123, 0, 5)
     assert Q.min() >= -1.0 and Q.max() < 1.0
     assert abs(float(Q.mean())) < 0.05
-    # entry (c, j) is (h >> 40) * 2^-23 - 1 with h the (c*4+j+1)-th output
+    # entry (c, j) comes from output c*r_max + j + 1 of the stream-1 base
     base = oracle.randk_base(123, 1, 0, 5, 0)
-    h = oracle.splitmix64_output(base, 3 * 4 + 2 + 1)
-    assert Q[3, 2] == np.float32((h >> 40) / 2.0 ** 23 - 1.0)
+    for c, j in [(0, 0), (0, 3), (3, 2), (999, 3)]:
+        h = oracle.splitmix64_output(base, c * 4 + j + 1)
+        assert Q[c, j] == oracle.q_entry(h)
+    # and the base of seed 0, worker 0, layer 0 is the hand-worked case B
+    golden = {r[0]: [int(x) for x in r[1:]] for r in read_golden_rows("randk_base_hand.txt")}
+    Q0 = oracle.powersgd_init_q(2, 2, 0, 0, 0)
+    assert Q0[1, 0] == oracle.q_entry(oracle.splitmix64_output(golden["B"][-1], 3))
 
 
 def test_bad_rank_is_rejected():

@@ -4,8 +4,9 @@ Source: "Sparsified SGD with Memory", Abstract / Motivation / Research
 questions: rand-k keeps k randomly chosen coordinates; Method: comp_k is a
 k-contraction, so the chosen values are sent unscaled.  The generator is
 SplitMix64 (Steele, Lea, Flood 2014), pinned by its published outputs; the
-way (seed, worker, layer, step) are folded into its state is this library's
-reading and stays unpinned beyond the statistical checks here.
+way (seed, stream, worker, layer, step) are folded into its state is this
+library's reading, pinned by a chain worked by hand whose first fold is a
+published output.
 """
 import math
 
@@ -20,6 +21,25 @@ def test_splitmix64_published_outputs():
     for row in read_golden_rows("splitmix64_published.txt"):
         state, *outs = (int(x) for x in row)
         assert [oracle.splitmix64_output(state, j) for j in (1, 2, 3)] == outs
+
+
+def test_base_fold_chain_hand_worked():
+    """The state of (seed, stream, worker, layer, step) against a chain worked
+    by hand (tests/golden/randk_base_hand.txt): the first fold of each case is
+    a published SplitMix64 output, which fixes the seed as the state and
+    stream + 1 as the counter; the later folds fix the field order and the
+    +1 offsets."""
+    pub = {int(r[0]): [int(x) for x in r[1:]] for r in read_golden_rows("splitmix64_published.txt")}
+    cases = read_golden_rows("randk_base_hand.txt")
+    assert [c[0] for c in cases] == ["A", "B"]
+    for name, *vals in cases:
+        seed, stream, worker, layer, step, f1, f2, f3, f4 = (int(v) for v in vals)
+        assert f1 == pub[seed][stream]          # output stream+1 of the seed state
+        assert oracle.splitmix64_output(seed, stream + 1) == f1
+        assert oracle.splitmix64_output(f1, worker + 1) == f2
+        assert oracle.splitmix64_output(f2, layer + 1) == f3
+        assert oracle.splitmix64_output(f3, step + 1) == f4
+        assert oracle.randk_base(seed, stream, worker, layer, step) == f4, name
 
 
 def test_key_is_high_half_of_output():
