@@ -191,9 +191,22 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def cpu_oracle_sample(spec, units, steps_seed):
+def cpu_model():
+    """The host CPU's model name (from /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return None
+
+
+def cpu_oracle_sample(spec, units, steps_seed, threads=None):
     """Run the oracle on `units` of the workload (host arrays from seeded
-    device gradients of worker w); returns (elements, seconds, threads)."""
+    gradients of worker w) on `threads` host threads (default: all cores);
+    returns (elements, seconds, threads)."""
     import numpy as np
     from concurrent.futures import ThreadPoolExecutor
     import oracle
@@ -204,7 +217,7 @@ def cpu_oracle_sample(spec, units, steps_seed):
     for l in layers:
         offs.append(o)
         o += l["rows"] * l["cols"]
-    threads = os.cpu_count() or 1
+    threads = threads or os.cpu_count() or 1
     dp = spec["method"] == "powersgd_dp"   # a unit is one layer of every worker
     data = {}
     for (w, l) in units:
@@ -260,6 +273,29 @@ def cpu_oracle_sample(spec, units, steps_seed):
     return elems, dt, threads
 
 
+# One step of every workload of the method's configurations, for the oracle
+# timing table: the 2^20 vector, ResNet-18 PowerSGD, VGG-19 with Accordion's
+# two levels (PowerSGD and top-k), one BERT-base worker, and the sweep (one
+# step at 2^27, the largest point the oracle finishes in about a minute).
+ORACLE_TABLE = ["memsgd_vector_2p20", "resnet18_powersgd_r2", "vgg19_accordion_powersgd",
+                "vgg19_accordion_topk", "bert_base_topk1pct_w8", "sweep_topk_e27_ppm10000",
+                "sweep_powersgd_e27_r2"]
+
+
+def oracle_timing(threads_all):
+    """{workload: (elements, s at 1 thread, s on all cores)} for one step of
+    worker 0 of each workload in ORACLE_TABLE (encode + decode)."""
+    rows = []
+    for name in ORACLE_TABLE:
+        spec = workload_spec(name)
+        units = [(0, l) for l in range(len(spec["layers"]))]
+        e1, t1, _ = cpu_oracle_sample(spec, units, 0, threads=1)
+        en, tn, n = cpu_oracle_sample(spec, units, 0, threads=threads_all)
+        rows.append({"workload": name, "elements": e1, "s_1thread": t1, "s_all": tn,
+                     "threads": n})
+    return rows
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -292,6 +328,7 @@ def run_reference(args, rank, world):
             "data": "synthetic (seeded N(0,1) gradients)",
             "config": {"workload": args.workload, "W": spec["W"]},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "cpu_model": cpu_model(),
                              "sample": "per step: the largest tensors of one worker (rotating; "
                                        "for the data-parallel PowerSGD workload, of every "
                                        "worker), about 6 M elements, %s encode + decode"
@@ -300,45 +337,26 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--profile", action="store_true", help="per-kernel table on stderr")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--graph", action="store_true",
-                    help="replay each step as a CUDA graph (workloads whose step takes no "
-                         "per-step host values: top-k, sign, PowerSGD without Accordion)")
-    args = ap.parse_args()
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
+SECONDARY = ["sweep_powersgd_e30_r2", "bert_base_randk1pct_w8", "bert_base_sign_w8",
+             "resnet18_powersgd_r2"]
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference":
-        return run_reference(args, rank, world)
 
+def run_workload(name, args, world, rank, dev, primary):
+    """Time `name` (args.steps steps after args.warmup warm-up steps) and
+    return its measurement fields.  Inputs that fit twice in L2 are timed
+    cold (L2 flushed between steps, each step between its own events) and
+    hot (one event pair around the steps); larger ones with one event pair
+    around the steps, the inputs themselves evicting L2."""
     import torch
     import torch.distributed as dist
-    torch.cuda.set_device(local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-
     import gradient_compression_error_b200 as gce
     from gradient_compression_error_b200 import workloads as wl
 
-    spec = workload_spec(args.workload)
+    spec = workload_spec(name)
     layers, W = spec["layers"], spec["W"]
     table = gce.Table(wl.table_layers(layers))
     N = table.N
     K_total = sum(l["cap"] for l in layers)
-    dev = "cuda"
     grads = [wl.gradients(layers, W, spec["cfg"], s) for s in range(2)]
     mem = torch.zeros((W, N), dtype=torch.float32, device=dev)
     vals = torch.zeros((W, table.vals_per_worker), dtype=torch.float32, device=dev)
@@ -415,7 +433,7 @@ def main():
     # CUDA-graph replay: one graph per gradient buffer, captured after the
     # warm-up; the kernels and their arguments are those of the eager step
     graphs, launches_per_step = None, None
-    if args.graph:
+    if args.graph and primary:
         if method == "randk" or kr is not None or apply:
             raise SystemExit("--graph: this workload's step takes per-step host values")
         graphs = []
@@ -430,26 +448,55 @@ def main():
             graphs[s % 2].replay()
         torch.cuda.synchronize()
 
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    input_bytes = 8 * W * N      # gradient and memory a step reads
+    cold = input_bytes < 2 * l2_bytes
+    flush = torch.empty(2 * l2_bytes // 4, dtype=torch.float32, device=dev) if cold else None
+
+    def run_steps(k0, count, flushed):
+        """count steps; returns their device time in ms (flushed: each step
+        between its own events, L2 rewritten between steps)."""
+        if not flushed:
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record()
+            for s in range(count):
+                if graphs:
+                    graphs[s % 2].replay()
+                else:
+                    step(k0 + s, grads[s % 2])
+            ev1.record()
+            torch.cuda.synchronize()
+            return ev0.elapsed_time(ev1)
+        evs = []
+        for s in range(count):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            if graphs:
+                graphs[s % 2].replay()
+            else:
+                step(k0 + s, grads[s % 2])
+            b.record()
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
     clocks = ClockSampler(torch.cuda.current_device())
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.2)
     l0 = gce.launch_count()
+    main_kernel = MAIN_KERNELS[method]
     # events around the main pass only (every kernel with --profile)
-    gce.profile_only(None if args.profile else MAIN_KERNELS[method])
+    gce.profile_only(None if args.profile else main_kernel)
     gce.profile_start()
-    ev0.record()
-    for s in range(args.steps):
-        if graphs:
-            graphs[s % 2].replay()
-        else:
-            step(args.warmup + s, grads[s % 2])
-    ev1.record()
-    torch.cuda.synchronize()
+    t_local = run_steps(args.warmup, args.steps, cold)
     prof = gce.profile_stop()
     launches = gce.launch_count() - l0
+    hot_ms = None
+    if cold:   # the same steps with L2 left warm between them
+        hot_ms = run_steps(args.warmup + args.steps, args.steps, False) / args.steps
     if graphs:
         # replays launch nothing from the host: the captured kernels per step;
         # the main-pass time comes from a short eager pass right after
@@ -463,33 +510,31 @@ def main():
                 for k, v in prof.items()}
     barrier()
     clk = clocks.stop()
-    t_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    t_ms = max_over_ranks(t_local)
     fallback_seen = bool(gce.status(ws) & gce.STATUS_FALLBACK)
 
     elems_per_step = W * N
     value = job_throughput(world, elems_per_step, args.steps, t_ms)
     ms_step = t_ms / args.steps
 
-    main_kernel = MAIN_KERNELS[method]
     # the main pass, whichever template instance ran (rand-k's may carry the
     # next step's key pass)
-    hits = [v for name, v in prof.items() if name == main_kernel or name.startswith(main_kernel + "<")]
+    hits = [v for n, v in prof.items() if n == main_kernel or n.startswith(main_kernel + "<")]
     main_ms, main_n = sum(v[0] for v in hits), sum(v[1] for v in hits)
     peak, peak_kind = measured_hbm_gbs()
     # the main pass covers every compressed element once per step: bytes and
     # kernel time per step
     bytes_per_step_main = 12.0 * W * (N - sum(l["rows"] * l["cols"] for l in layers
                                              if l["kind"] == "dense"))
-    main_launches_per_step = main_n / args.steps
     main_ms_per_step = main_ms / args.steps
     achieved = (bytes_per_step_main / (main_ms_per_step / 1e3) / 1e9) if main_n else None
-    traffic = ncu_traffic_per_launch() if args.workload == DEFAULT_WORKLOAD else None
+    traffic = ncu_traffic_per_launch() if name == DEFAULT_WORKLOAD else None
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                 "frac": (achieved / peak) if achieved else None, "traffic": traffic,
                 "kernel": main_kernel,
                 "peak_source": peak_kind,
                 "algorithmic_bytes_per_step": bytes_per_step_main,
-                "launches_per_step": main_launches_per_step,
+                "launches_per_step": main_n / args.steps,
                 "kernel_ms_per_step": main_ms_per_step if main_n else None}
     # whole-step algorithmic traffic: sparse W(12N + 8K) encode + 16 W K + 4N
     # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
@@ -507,7 +552,7 @@ def main():
 
     # end to end through the public API with host buffers
     e2e = None
-    if not args.no_e2e:
+    if primary and not args.no_e2e:
         hgrad = torch.empty((W, N), dtype=torch.float32, pin_memory=True)
         hgrad.copy_(grads[0])
         hout = torch.empty(N, dtype=torch.float32, pin_memory=True)
@@ -529,41 +574,132 @@ def main():
                "h2d_bytes_per_step": W * N * 4, "d2h_bytes_per_step": N * 4, "steps": ke}
         del hgrad, hout
 
+    if args.profile and rank == 0:
+        tot = sum(v[0] for v in prof.values())
+        for kname, (ms, n) in sorted(prof.items(), key=lambda x: -x[1][0]):
+            print("%-32s %8d launches %10.3f ms %6.1f%%" % (kname, n, ms, 100 * ms / tot),
+                  file=sys.stderr)
+
+    l2_note = ("L2 flushed before every step (a %d MB write outside the step's events); "
+               "hot (L2 warm) %.4f ms per step" % (2 * l2_bytes >> 20, hot_ms) if cold else
+               "inputs larger than L2 (%.1f GB of grad+memory per step)" % (input_bytes / 1e9))
+    return dict(spec=spec, layers=layers, W=W, N=N, K_total=K_total, apply=apply, value=value,
+                ms_step=ms_step, hot_ms=hot_ms, cold=cold, roofline=roofline, step_gbs=step_gbs,
+                peak=peak, launches=launches, clocks=clk, e2e=e2e, graphs=bool(graphs),
+                fallback_seen=fallback_seen, l2_note=l2_note, method=method)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--profile", action="store_true", help="per-kernel table on stderr")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the other workloads' short measurements")
+    ap.add_argument("--oracle-timing", action="store_true",
+                    help="time the CPU oracle on one step of every workload at 1 thread and "
+                         "on all cores, print one JSON line, and exit")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step as a CUDA graph (workloads whose step takes no "
+                         "per-step host values: top-k, sign, PowerSGD without Accordion)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if args.oracle_timing:
+        if rank == 0:
+            print(json.dumps({"oracle_timing": oracle_timing(os.cpu_count() or 1),
+                              "cpu_model": cpu_model(), "cores": os.cpu_count()}), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = "cuda"
+
+    r = run_workload(args.workload, args, world, rank, dev, primary=True)
+    spec, layers, W, N, method = r["spec"], r["layers"], r["W"], r["N"], r["method"]
+    torch.cuda.empty_cache()
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu:
         units = [(0, l) for l in range(len(layers))]
         elems, dt, threads = cpu_oracle_sample(spec, units, 0)
+        # the same sample on one thread, bounded to the largest tensors that
+        # fit about 6 M elements (at one thread the full set takes minutes)
+        sub, tot = [], 0
+        for l in sorted(range(len(layers)), key=lambda l: -(layers[l]["rows"] * layers[l]["cols"])):
+            n = layers[l]["rows"] * layers[l]["cols"]
+            if tot + n <= 6_000_000 or not sub:
+                sub.append((0, l))
+                tot += n
+        e1, t1, _ = cpu_oracle_sample(spec, sub, 0, threads=1)
         cpu = {"value": elems / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
                "sample": "worker 0: all %d tensors (%d elements), encode + decode, one step"
-                         % (len(layers), elems), "seconds": dt}
+                         % (len(layers), elems), "seconds": dt,
+               "value_1thread": e1 / t1,
+               "sample_1thread": "worker 0: its largest tensors up to about 6 M elements "
+                                 "(%d elements), encode + decode, one step, one thread" % e1,
+               "cpu_model": cpu_model()}
 
-    if args.profile and rank == 0:
-        tot = sum(v[0] for v in prof.values())
-        for name, (ms, n) in sorted(prof.items(), key=lambda x: -x[1][0]):
-            print("%-32s %8d launches %10.3f ms %6.1f%%" % (name, n, ms, 100 * ms / tot),
-                  file=sys.stderr)
+    secondary = None
+    if world == 1 and not args.no_secondary and args.workload == DEFAULT_WORKLOAD:
+        import copy
+        sargs = copy.copy(args)
+        sargs.steps, sargs.warmup, sargs.graph, sargs.profile = min(args.steps, 30), 3, False, False
+        secondary = []
+        for name in SECONDARY:
+            x = run_workload(name, sargs, world, rank, dev, primary=False)
+            secondary.append({"workload": name, "value": x["value"], "unit": UNIT,
+                              "ms_per_step": x["ms_step"], "steps": sargs.steps,
+                              "warmup": sargs.warmup,
+                              "timing": "cold (L2 flushed before every step)" if x["cold"]
+                                        else "inputs larger than L2",
+                              "ms_per_step_hot": x["hot_ms"],
+                              "step_algorithmic_GBps": x["step_gbs"],
+                              "step_frac_of_hbm": x["step_gbs"] / x["peak"],
+                              "roofline": {k: x["roofline"][k] for k in
+                                           ("kernel", "achieved", "frac", "kernel_ms_per_step")},
+                              "gpu_launches": x["launches"], "clocks": x["clocks"]})
+            del x
+            torch.cuda.empty_cache()
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+        K_total = r["K_total"]
+        line = {"metric": METRIC, "value": r["value"], "unit": UNIT, "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms_step"],
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
                 "data": "synthetic (seeded N(0,1) gradients, resident in HBM)",
                 "config": {"workload": args.workload, "W": W, "elements_per_worker": N,
                            "tensors": len(layers), "k_total_per_worker": K_total,
-                           "eta": "8/(1*(160+t))" if apply else wl.ETA,
-                           "update": "x -= mean of payloads (fused)" if apply else "decode only",
+                           "eta": "8/(1*(160+t))" if r["apply"] else 0.05,
+                           "update": "x -= mean of payloads (fused)" if r["apply"] else "decode only",
                            "parallelism": "replicas x%d" % world,
                            "launch": ("CUDA graph replay (main-pass time from 20 eager steps)"
-                                      if graphs else "eager"),
-                           "l2": "inputs larger than L2 (%.1f GB of grad+memory per step)"
-                                 % (8.0 * W * N / 1e9),
+                                      if r["graphs"] else "eager"),
+                           "l2": r["l2_note"],
                            "payload_bytes_per_worker": payload_bytes_per_worker(layers, method),
                            "compression_ratio": 4.0 * N / payload_bytes_per_worker(layers, method),
-                           "step_algorithmic_GBps": step_gbs,
-                           "step_frac_of_hbm": step_gbs / peak,
-                           "fallback_seen": fallback_seen},
-                "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-                "gpu_launches": launches, "clocks": clk}
+                           "step_algorithmic_GBps": r["step_gbs"],
+                           "step_frac_of_hbm": r["step_gbs"] / r["peak"],
+                           "fallback_seen": r["fallback_seen"]},
+                "roofline": r["roofline"], "cpu_baseline": cpu, "e2e": r["e2e"],
+                "gpu_launches": r["launches"], "clocks": r["clocks"]}
+        if secondary is not None:
+            line["secondary"] = secondary
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()

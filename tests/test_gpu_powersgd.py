@@ -49,7 +49,10 @@ class PsRun:
             o = t.info[l]["q_offset"]
             assert np.array_equal(bits(hq[w, o:o + q.size]), bits(q.reshape(-1))), "Q init"
 
-    def step(self, grad, eta, ranks=None):
+    def step(self, grad, eta, ranks=None, full=True):
+        """One step on both sides; the oracle keeps its own trajectory.  P, Q
+        and DENSE payloads are compared every step; the memory and P Q^T
+        (whole-layer arrays) when `full`."""
         kt = None if ranks is None else torch.tensor(ranks, dtype=torch.int32, device="cuda")
         r = [l["cap"] for l in self.layers] if ranks is None else ranks
         expect = osteps.powersgd_step(self.layers, host(grad), self.hmem, eta, r, self.hQ,
@@ -58,8 +61,8 @@ class PsRun:
         self.g.powersgd_step(self.t, self.W, grad, self.mem, eta, kt, self.P, self.Q, self.vals,
                              self.out, self.ws)
         torch.cuda.synchronize()
-        hP, hQ, hm, ho, hv = (host(self.P), host(self.Q), host(self.mem), host(self.out),
-                              host(self.vals))
+        hP, hQ, hv = host(self.P), host(self.Q), host(self.vals)
+        hm, ho = (host(self.mem), host(self.out)) if full else (None, None)
         worst = 0.0
         for (w, l), e in expect.items():
             lay = self.layers[l]
@@ -68,7 +71,8 @@ class PsRun:
             if lay["kind"] == "dense":
                 n = info["n"]
                 assert np.array_equal(bits(hv[w, info["val_offset"]:info["val_offset"] + n]), bits(e))
-                assert np.array_equal(bits(hm[w, ls]), bits(self.hmem[w, ls]))
+                if full:
+                    assert np.array_equal(bits(hm[w, ls]), bits(self.hmem[w, ls]))
                 continue
             rows, cols, cap = lay["rows"], lay["cols"], lay["cap"]
             rr = r[l]
@@ -78,9 +82,10 @@ class PsRun:
             P_gpu = hP[w, info["p_offset"]:info["p_offset"] + rows * cap].reshape(rows, cap)
             Q_gpu = hQ[w, info["q_offset"]:info["q_offset"] + cols * cap].reshape(cols, cap)
             errs = [relerr(P_gpu[:, :rr], P_ref[:, :rr], 0.0),
-                    relerr(Q_gpu[:, :rr], Q_ref[:, :rr], Mfull),
-                    relerr(ho[w, ls], Mhat_ref.reshape(-1), Mfull),
-                    relerr(hm[w, ls], self.hmem[w, ls], Mfull)]
+                    relerr(Q_gpu[:, :rr], Q_ref[:, :rr], Mfull)]
+            if full:
+                errs += [relerr(ho[w, ls], Mhat_ref.reshape(-1), Mfull),
+                         relerr(hm[w, ls], self.hmem[w, ls], Mfull)]
             assert max(errs) <= TOL, (w, l, errs)
             worst = max(worst, max(errs))
             # columns >= r are left as they were (the GPU's own previous values)

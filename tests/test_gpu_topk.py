@@ -232,21 +232,28 @@ def test_memsgd_vector_20_steps():
     run_and_compare(layers, 1, 20, randn_grad(layers, 1, 1))
 
 
-def check_topk_properties(run, grad, mem_old, eta):
+def check_topk_properties(run, grad, mem_old, eta, ks=None):
     """Properties that fix the top-k result at any size, checked with torch on
     the device: exactly k ascending unique indices per unit; sent values are
     v's bits; new memory + sent == v bit for bit; every sent |v| beats every
-    kept one, ties going to the lower index."""
+    kept one, ties going to the lower index.  ks: k per layer (default the
+    caps).
+
+    v = fl(m + fl(eta * g)) is formed by two separate torch kernels: the
+    product is written to memory as an fp32 tensor before the sum reads it,
+    so nothing can contract the two roundings into one FMA."""
     t = run.table
     W = run.W
-    v = mem_old + grad * torch.tensor(eta, dtype=torch.float32, device="cuda")
+    prod = grad * torch.tensor(eta, dtype=torch.float32, device="cuda")
+    v = mem_old + prod
+    del prod
     mem = run.mem
     sent = torch.zeros_like(mem)
     sel = torch.zeros(mem.shape, dtype=torch.bool, device="cuda")
     for l, lay in enumerate(run.layers):
         n = lay["rows"] * lay["cols"]
         off = t.info[l]["offset"]
-        k = lay["cap"]
+        k = lay["cap"] if ks is None else int(ks[l])
         vo = t.info[l]["val_offset"]
         if lay["kind"] == "dense":     # sent whole; memory left at zero
             dv = run.vals[:, vo:vo + n]
