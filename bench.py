@@ -72,14 +72,16 @@ def workload_spec(name):
     if name.startswith("sweep_randk_e"):
         e, ppm = name[len("sweep_randk_e"):].split("_ppm")
         return dict(layers=wl.sweep(int(e), "randk", int(ppm)), W=1, cfg=5, method="randk")
-    if name.startswith("sweep_powersgd_e"):      # e.g. sweep_powersgd_e28_r2
-        e, r = name[len("sweep_powersgd_e"):].split("_r")
+    if name.startswith("sweep_powersgd_e"):      # e.g. sweep_powersgd_e28_r2[_lazy]
+        lazy = name.endswith("_lazy")
+        e, r = name[len("sweep_powersgd_e"):].replace("_lazy", "").split("_r")
         return dict(layers=wl.sweep(int(e), "powersgd", rank=int(r)), W=1, cfg=5,
-                    method="powersgd")
+                    method="powersgd_lazy" if lazy else "powersgd")
     raise SystemExit("unknown workload %s" % name)
 
 
 MAIN_KERNELS = {"topk": "tk_main_kernel", "randk": "rk_emit_kernel", "powersgd": "ps_mq_kernel",
+                "powersgd_lazy": "ps_mq_kernel",
                 "powersgd_dp": "ps_mq_kernel", "sign": "sg_fused_kernel"}
 
 
@@ -249,7 +251,7 @@ def cpu_oracle_sample(spec, units, steps_seed, threads=None):
         elif lay["kind"] == "dense":
             pay, m_new = oracle.dense_unit(gg, mm, wl.ETA)
             oracle.accum_dense(out, pay)
-        elif spec["method"] == "powersgd":
+        elif spec["method"] in ("powersgd", "powersgd_lazy"):
             rows, cols = lay["rows"], lay["cols"]
             Q = oracle.powersgd_init_q(cols, lay["cap"], 1, w, l)
             P, Qn, m_new, _ = oracle.powersgd_unit(gg.reshape(rows, cols), mm.reshape(rows, cols),
@@ -337,8 +339,8 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-SECONDARY = ["sweep_powersgd_e30_r2", "bert_base_randk1pct_w8", "bert_base_sign_w8",
-             "resnet18_powersgd_r2"]
+SECONDARY = ["sweep_powersgd_e30_r2", "sweep_powersgd_e30_r2_lazy", "bert_base_randk1pct_w8",
+             "bert_base_sign_w8", "resnet18_powersgd_r2"]
 
 
 def run_workload(name, args, world, rank, dev, primary):
@@ -365,8 +367,10 @@ def run_workload(name, args, world, rank, dev, primary):
     ws_dc = table.workspace(W, "decompress")
     out = torch.zeros(N, dtype=torch.float32, device=dev)
     method = spec["method"]
-    P = Q = None
-    if method == "powersgd":
+    P = Q = lazy_rank = None
+    if method == "powersgd_lazy":
+        lazy_rank = torch.zeros((W, table.L), dtype=torch.int32, device=dev)
+    if method in ("powersgd", "powersgd_lazy"):
         P = torch.zeros((W, max(4, table.P_per_worker)), dtype=torch.float32, device=dev)
         Q = torch.zeros((W, max(4, table.Q_per_worker)), dtype=torch.float32, device=dev)
         gce.powersgd_init_q(table, W, 1, Q)
@@ -408,14 +412,17 @@ def run_workload(name, args, world, rank, dev, primary):
             # the shared payload is already the workers' mean: one decode
             gce.decompress_accumulate(table, 1, vals, None, kr, P, Q, 1.0, out, ws_dc)
             return
+        elif method == "powersgd_lazy":
+            gce.powersgd_step_lazy(table, W, grad, mem, eta, kr, P, Q, vals, lazy_rank, ws)
         else:
             gce.powersgd_step(table, W, grad, mem, eta, kr, P, Q, vals, None, ws)
+        sparse = method in ("topk", "randk")
         if apply:
-            gce.decompress_apply(table, W, vals, idx if method != "powersgd" else None, kr, P, Q,
-                                 1.0 / W, out, ws_dc)
+            gce.decompress_apply(table, W, vals, idx if sparse else None, kr, P, Q, 1.0 / W, out,
+                                 ws_dc)
         else:
-            gce.decompress_accumulate(table, W, vals, idx if method != "powersgd" else None, kr,
-                                      P, Q, 1.0, out, ws_dc)
+            gce.decompress_accumulate(table, W, vals, idx if sparse else None, kr, P, Q, 1.0,
+                                      out, ws_dc)
 
     def barrier():
         if world > 1:
@@ -538,7 +545,7 @@ def run_workload(name, args, world, rank, dev, primary):
                 "kernel_ms_per_step": main_ms_per_step if main_n else None}
     # whole-step algorithmic traffic: sparse W(12N + 8K) encode + 16 W K + 4N
     # decode; PowerSGD W * 12N encode + 4N decode (P and Q are negligible)
-    if method in ("powersgd", "powersgd_dp"):
+    if method in ("powersgd", "powersgd_dp", "powersgd_lazy"):
         step_bytes = W * 12.0 * N
     elif method == "sign":
         # grad and memory read once, memory written, words written (the

@@ -9,7 +9,7 @@ first call raises -- there is no fallback.
 
 The entry points keep the C names: ef_topk_step, ef_randk_step,
 ef_randk_step_at, ef_sign_step, powersgd_init_q, powersgd_step,
-powersgd_dp_step, accordion_init, accordion_select, decompress_accumulate,
+powersgd_step_lazy (with materialize_memory), powersgd_dp_step, accordion_init, accordion_select, decompress_accumulate,
 decompress_apply, decompress_accumulate_noalloc, decompress_vote, plus the
 Table wrapper of gce_table_* and the workspace, status, schedule and profiling
 helpers.  The exchange of payloads between data-parallel ranks sits on top of
@@ -77,6 +77,9 @@ SIGNATURES = {
                                 C.c_size_t, _vp]),
     "powersgd_dp_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
                                    C.c_size_t, _vp]),
+    "powersgd_step_lazy": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
+                                     C.c_size_t, _vp]),
+    "gce_materialize_memory": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp]),
     "ef_sign_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, C.c_size_t, _vp]),
     "decompress_vote": (C.c_int, [_vp, _i32, _vp, _f32, _vp, _vp]),
     "accordion_init": (C.c_int, [_vp, _vp, _vp, _vp]),
@@ -256,6 +259,23 @@ def powersgd_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, dense_out, ws
         table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
         _ptr(k_or_rank, _i32()), _ptr(P, _f32()), _ptr(Q, _f32()), _ptr(vals, _f32()),
         _ptr(dense_out, _f32()), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def powersgd_step_lazy(table, W, grad, mem, eta, k_or_rank, P, Q, vals, lazy_rank, ws,
+                       stream=None):
+    """powersgd_step leaving M in the memory; lazy_rank (int32 [W, L]) records
+    the factors to take off (include/gce.h)."""
+    _check("powersgd_step_lazy", lib().powersgd_step_lazy(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), _ptr(P, _f32()), _ptr(Q, _f32()), _ptr(vals, _f32()),
+        _ptr(lazy_rank, _i32()), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def materialize_memory(table, W, mem, P, Q, lazy_rank, stream=None):
+    """mem <- M - P Q^T where a lazy step left M; lazy_rank -> 0."""
+    _check("gce_materialize_memory", lib().gce_materialize_memory(
+        table.handle, int(W), _ptr(mem, _f32()), _ptr(P, _f32()), _ptr(Q, _f32()),
+        _ptr(lazy_rank, _i32()), _stream(stream)))
 
 
 def powersgd_dp_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, ws, stream=None):

@@ -67,6 +67,8 @@ struct gce_table {
     int32_t tiles_pw = 0;                  // main tiles (compressed layers) per worker
     int32_t* d_tile_layer = nullptr;       // [tiles_pw] layer of each main tile
     gce::TileInfo* d_tile_info = nullptr;  // [tiles_pw] the same tiles' layer fields
+    int32_t tk_groups_pw = 0;              // top-k emit items (kTkGroup tiles) per worker
+    int2* d_tk_groups = nullptr;           // [tk_groups_pw] (first tile, tiles), small layers first
     int32_t sunits_pw = 0;                 // top-k sample units per worker
     int32_t* d_sunit_layer = nullptr;      // [sunits_pw] layer of each sample unit
     int32_t* d_sunit_part = nullptr;       // [sunits_pw] part index within the layer
@@ -239,6 +241,28 @@ __device__ __forceinline__ uint32_t abs_key(float v) {
 
 __device__ __forceinline__ float4 ld_stream4(const float* p) {
     return __ldcs(reinterpret_cast<const float4*>(p));
+}
+
+// Acquire / release accesses at GPU scope, for flags that one block publishes
+// and blocks of the same launch wait on.
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+    int32_t v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint64_t ld_acquire_gpu_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.acquire.gpu.global.b64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu_u64(uint64_t* p, uint64_t v) {
+    asm volatile("st.release.gpu.global.b64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // Bulk (TMA-engine) prefetch of a contiguous range into L2: one instruction

@@ -188,14 +188,34 @@ __global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
     }
 }
 
+// m = M - P Q^T for one entry, formed exactly as the residual pass and the
+// decoder form it: the product of column 0, then fused multiply-adds in
+// column order, then one rounded subtraction.
+__device__ __forceinline__ float ps_unproject(float M, const float* pr, const float (*qs)[kPsCB],
+                                              int c, int r) {
+    float mh = __fmul_rn(pr[0], qs[0][c]);
+#pragma unroll
+    for (int j = 1; j < kMaxRank; ++j)
+        if (j < r) mh = __fmaf_rn(pr[j], qs[j][c], mh);
+    return __fsub_rn(M, mh);
+}
+
 // ---- phase 1: M = m + eta*g (written back), partial P = M Q -------------------------------
+// kLazy: the memory holds the previous step's M, and P / Q that step's
+// orthonormal P and Q' over lazy_rank[w][l] columns (0: the memory holds the
+// residual itself); the residual m = M - P Q'^T is formed on the fly, entry by
+// entry as the residual pass would have formed it, so the results are the
+// eager step's bit for bit without that pass's read and write of M.
+template <bool kLazy>
 __global__ void __launch_bounds__(256) ps_mq_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t Q_pw,
     int64_t ppart_pw, const float* __restrict__ grad, float* __restrict__ mem, float eta,
     const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, float* __restrict__ ppart,
-    int32_t* __restrict__ status) {
+    int32_t* __restrict__ status, const float* __restrict__ P, int64_t P_pw, int32_t L_all,
+    const int32_t* __restrict__ lazy_rank) {
     __shared__ float qs[kMaxRank][kPsCB];
+    __shared__ float prow[kPsRB][kMaxRank];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
         const int w = int(u / ntiles);
@@ -205,26 +225,51 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
         const int r = ps_rank(L, k_or_rank, d.x);
         if (r == 0) continue;
         const int cap = L.cap;
+        // columns of the previous step's factors to take off (lazy only)
+        int rp = 0;
+        if (kLazy) {
+            rp = lazy_rank[int64_t(w) * L_all + d.x];
+            rp = (rp >= 1 && rp <= cap) ? rp : 0;
+        }
+        const int rq = r > rp ? r : rp;  // Q columns staged
         const int64_t C = L.cols, R = L.rows;
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
         const int64_t r0 = int64_t(d.y) * kPsRB;
         const int rh = int(min64(kPsRB, R - r0));
         const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
-        for (int i = tid; i < cw * r; i += blockDim.x) {
-            const int c = i / r, j = i - c * r;
+        for (int i = tid; i < cw * rq; i += blockDim.x) {
+            const int c = i / rq, j = i - c * rq;
             qs[j][c] = q[int64_t(c) * cap + j];
+        }
+        if (kLazy && rp > 0) {
+            const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+            for (int i = tid; i < rh * rp; i += blockDim.x) {
+                const int row = i / rp, j = i - row * rp;
+                prow[row][j] = p[int64_t(row) * cap + j];
+            }
         }
         __syncthreads();
         for (int row = warp; row < rh; row += blockDim.x >> 5) {
             const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
             const float* g = grad + e;
             float* m = mem + e;
+            float pr[kMaxRank] = {0.f, 0.f, 0.f, 0.f};
+            if (kLazy && rp > 0) {
+#pragma unroll
+                for (int j = 0; j < kMaxRank; ++j) pr[j] = j < rp ? prow[row][j] : 0.0f;
+            }
             float acc[kMaxRank] = {0.f, 0.f, 0.f, 0.f};
             if (((e & 3) == 0) && ((cw & 3) == 0)) {
                 for (int c = lane * 4; c < cw; c += 128) {
                     const float4 gg = ld_stream4(g + c);
-                    const float4 mm = *reinterpret_cast<const float4*>(m + c);
+                    float4 mm = *reinterpret_cast<const float4*>(m + c);
+                    if (kLazy && rp > 0) {
+                        mm.x = ps_unproject(mm.x, pr, qs, c, rp);
+                        mm.y = ps_unproject(mm.y, pr, qs, c + 1, rp);
+                        mm.z = ps_unproject(mm.z, pr, qs, c + 2, rp);
+                        mm.w = ps_unproject(mm.w, pr, qs, c + 3, rp);
+                    }
                     float4 x;
                     x.x = residual(mm.x, eta, gg.x);
                     x.y = residual(mm.y, eta, gg.y);
@@ -243,7 +288,9 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
                 }
             } else {
                 for (int c = lane; c < cw; c += 32) {
-                    const float x = residual(m[c], eta, __ldcs(g + c));
+                    float mv = m[c];
+                    if (kLazy && rp > 0) mv = ps_unproject(mv, pr, qs, c, rp);
+                    const float x = residual(mv, eta, __ldcs(g + c));
                     m[c] = x;
 #pragma unroll
                     for (int j = 0; j < kMaxRank; ++j)
@@ -287,7 +334,7 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
     int64_t ppart_pw,
     int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ ppart,
     double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status,
-    int32_t ntall, int32_t* __restrict__ tdone) {
+    int32_t ntall, int32_t* __restrict__ tdone, int32_t L_all, int32_t* __restrict__ lazy_rank) {
     __shared__ double s_red[32];
     for (int64_t u = blockIdx.x; u < int64_t(nps) * W; u += gridDim.x) {
         const int w = int(u / nps);
@@ -296,9 +343,13 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         const PsLayer X = ps[l];
         const int r = ps_rank(L, k_or_rank, l);
         if (r == 0) {
+            // a skipped layer keeps its memory, and in the lazy step its record
             if (threadIdx.x == 0) set_status(status, GCE_STATUS_K_RANGE);
             continue;
         }
+        // the lazy step: the memory will hold M, P and Q this step's factors
+        // (every M Q tile has read the previous record by now)
+        if (lazy_rank && threadIdx.x == 0) lazy_rank[int64_t(w) * L_all + l] = r;
         if (X.tall >= 0) {  // orthonormalised by the multi-block kernel below
             if (threadIdx.x == 0) tdone[int64_t(w) * ntall + X.tall] = 0;
             continue;
@@ -594,11 +645,13 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
 }
 
 // ---- residual: m <- M - P Q^T, dense_out <- P Q^T ---------------------------------------------
+// rank_wl (nullable): per (worker, layer) ranks [W][L_all] instead of
+// k_or_rank -- the lazy step's record, for gce_materialize_memory.
 __global__ void __launch_bounds__(256) ps_resid_kernel(
     const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles, int32_t W,
     int64_t N, int64_t P_pw, int64_t Q_pw, const int32_t* __restrict__ k_or_rank,
     const float* __restrict__ P, const float* __restrict__ Q, float* __restrict__ mem,
-    float* __restrict__ dense_out) {
+    float* __restrict__ dense_out, const int32_t* __restrict__ rank_wl, int32_t L_all) {
     __shared__ float qs[kMaxRank][kPsCB];
     __shared__ float prow[kPsRB][kMaxRank];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -606,7 +659,13 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
         const int w = int(u / ntiles);
         const int4 d = tiles[u % ntiles];
         const DevLayer L = layers[d.x];
-        const int r = ps_rank(L, k_or_rank, d.x);
+        int r = 0;
+        if (rank_wl) {
+            r = rank_wl[int64_t(w) * L_all + d.x];
+            r = (r >= 1 && r <= L.cap) ? r : 0;
+        } else {
+            r = ps_rank(L, k_or_rank, d.x);
+        }
         if (r == 0) continue;
         const int cap = L.cap;
         const int64_t C = L.cols, R = L.rows;
@@ -795,9 +854,9 @@ extern "C" int powersgd_init_q(const gce_table* t, int32_t W, uint64_t seed, flo
     return check_launch();
 }
 
-extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
-                             const int32_t* k_or_rank, float* P, float* Q, float* vals,
-                             float* dense_out, void* ws, size_t ws_bytes, void* stream) {
+static int ps_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
+                   const int32_t* k_or_rank, float* P, float* Q, float* vals, float* dense_out,
+                   int32_t* lazy_rank, void* ws, size_t ws_bytes, void* stream) {
     if (!t || W < 1 || !grad || !mem || !ws) return GCE_ERR_ARG;
     if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
     if (!aligned16(grad) || !aligned16(mem) || !aligned16(ws)) return GCE_ERR_ARG;
@@ -813,19 +872,27 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         double* pd = at<double>(ws, lay.pd);
         float* qpart = at<float>(ws, lay.qpart);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_mq = resident_blocks(ps_mq_kernel, 256);
+        static const int r_mq = resident_blocks(ps_mq_kernel<false>, 256);
+        static const int r_mql = resident_blocks(ps_mq_kernel<true>, 256);
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
         static const int r_resid = resident_blocks(ps_resid_kernel, 256);
-        GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st, t->d_layers,
-                   ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw, t->ppart_pw, grad, mem,
-                   eta, k_or_rank, Q, ppart, status);
+        if (lazy_rank)
+            GCE_LAUNCH(ps_mq_kernel<true>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mql), 256, 0, st,
+                       t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw,
+                       t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, P, t->P_pw, t->L,
+                       lazy_rank);
+        else
+            GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
+                       t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw,
+                       t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, nullptr,
+                       int64_t(0), t->L, nullptr);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, 1, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
-                   pd, P, status, t->ps_ntall, tdone);
+                   pd, P, status, t->ps_ntall, tdone, t->L, lazy_rank);
         if (t->ps_ntall > 0) {
             for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
                 GCE_LAUNCH(ps_orth_tall_kernel, wave_grid(int64_t(t->ps_tall_nunits) * W, 8, r_tall), 256, 0,
@@ -840,12 +907,53 @@ extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, f
         GCE_LAUNCH(ps_qred_kernel<false>, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0,
                    st, t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
                    k_or_rank, qpart, Q, nullptr, 1.0f);
-        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
-                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
-                   k_or_rank, P, Q, mem, dense_out);
+        // the lazy step leaves M in the memory: the next step (or
+        // gce_materialize_memory) takes P Q^T off
+        if (!lazy_rank)
+            GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
+                       t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
+                       k_or_rank, P, Q, mem, dense_out, nullptr, t->L);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
+}
+
+extern "C" int powersgd_step(const gce_table* t, int32_t W, const float* grad, float* mem, float eta,
+                             const int32_t* k_or_rank, float* P, float* Q, float* vals,
+                             float* dense_out, void* ws, size_t ws_bytes, void* stream) {
+    return ps_step(t, W, grad, mem, eta, k_or_rank, P, Q, vals, dense_out, nullptr, ws, ws_bytes,
+                   stream);
+}
+
+extern "C" int powersgd_step_lazy(const gce_table* t, int32_t W, const float* grad, float* mem,
+                                  float eta, const int32_t* k_or_rank, float* P, float* Q,
+                                  float* vals, int32_t* lazy_rank, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    if (!lazy_rank || (reinterpret_cast<uintptr_t>(lazy_rank) & 3)) return GCE_ERR_ARG;
+    return ps_step(t, W, grad, mem, eta, k_or_rank, P, Q, vals, nullptr, lazy_rank, ws, ws_bytes,
+                   stream);
+}
+
+extern "C" int gce_materialize_memory(const gce_table* t, int32_t W, float* mem, const float* P,
+                                      const float* Q, int32_t* lazy_rank, void* stream) {
+    if (!t || W < 1 || !mem || !lazy_rank || !aligned16(mem)) return GCE_ERR_ARG;
+    if (reinterpret_cast<uintptr_t>(lazy_rank) & 3) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (t->nps > 0) {
+        if (!P || !Q || !aligned16(P) || !aligned16(Q)) return GCE_ERR_ARG;
+        static const int r_resid = resident_blocks(ps_resid_kernel, 256);
+        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
+                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
+                   nullptr, P, Q, mem, nullptr, lazy_rank, t->L);
+        if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+    }
+    if (cudaMemsetAsync(lazy_rank, 0, sizeof(int32_t) * size_t(W) * size_t(t->L), st) !=
+        cudaSuccess) {
+        cudaGetLastError();
+        return GCE_ERR_CUDA;
+    }
+    return GCE_OK;
 }
 
 extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad, float* mem,
@@ -869,20 +977,21 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         float* qloc = at<float>(ws, lay.qloc);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_mq = resident_blocks(ps_mq_kernel, 256);
+        static const int r_mq = resident_blocks(ps_mq_kernel<false>, 256);
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<true>, 256);
         static const int r_resid = resident_blocks(ps_resid_kernel, 256);
         // every worker reads the shared warm start Q (stride 0)
-        GCE_LAUNCH(ps_mq_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
+        GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
                    t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0),
-                   t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status);
+                   t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, nullptr, int64_t(0),
+                   t->L, nullptr);
         // one P per layer from the partials of all W workers
         GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank,
-                   ppart, pd, P, status, t->ps_ntall, tdone);
+                   ppart, pd, P, status, t->ps_ntall, tdone, t->L, nullptr);
         if (t->ps_ntall > 0) {
             for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
                 GCE_LAUNCH(ps_orth_tall_kernel, wave_grid(t->ps_tall_nunits, 8, r_tall), 256, 0,
@@ -901,7 +1010,7 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         // each worker's error against its own Q_w
         GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
                    t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->Q_pw,
-                   k_or_rank, P, qloc, mem, nullptr);
+                   k_or_rank, P, qloc, mem, nullptr, nullptr, t->L);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     if (t->dtiles_pw > 0) {

@@ -69,16 +69,6 @@ __device__ __forceinline__ double block_sum_fixed(double x, double* s_red) {
     return t;
 }
 
-__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
-    int32_t v;
-    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-__device__ __forceinline__ void st_release_gpu(int32_t* p, int32_t v) {
-    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
-}
-
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
     uint64_t p;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));

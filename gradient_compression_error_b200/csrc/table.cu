@@ -1,5 +1,6 @@
 // table.cu -- layer table, workspace queries, status word, launch counter,
 // and the kernel for uncompressed (DENSE) layers shared by every step.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -157,6 +158,7 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_dense);
     cudaFree(t->d_tile_layer);
     cudaFree(t->d_tile_info);
+    cudaFree(t->d_tk_groups);
     cudaFree(t->d_sunit_layer);
     cudaFree(t->d_sunit_part);
     cudaFree(t->d_dtile_layer);
@@ -285,6 +287,22 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     t->Q_pw = qoff;
     t->comp_N = spoff;
     t->tiles_pw = tiles;
+    // top-k emit items: runs of up to kTkGroup consecutive tiles of one layer,
+    // layers in ascending size (their selections finish first), each layer's
+    // runs in tile order
+    std::vector<int2> tk_groups;
+    if (t->ckind == GCE_KIND_TOPK) {
+        std::vector<int32_t> order(t->comp);
+        std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
+            return t->layers[a].n < t->layers[b].n;
+        });
+        for (int32_t l : order) {
+            const DevLayer& x = t->layers[l];
+            for (int32_t i = 0; i < x.ntiles; i += kTkGroup)
+                tk_groups.push_back(make_int2(x.tile0 + i, std::min(kTkGroup, x.ntiles - i)));
+        }
+    }
+    t->tk_groups_pw = int32_t(tk_groups.size());
     t->sunits_pw = int32_t(sunit_layer.size());
     t->dtiles_pw = int32_t(dtile_layer.size());
     t->dc_tiles = dc_tiles;
@@ -296,6 +314,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_dense, t->dense);
     if (rc == GCE_OK) rc = upload(&t->d_tile_layer, tile_layer);
     if (rc == GCE_OK) rc = upload(&t->d_tile_info, tile_info);
+    if (rc == GCE_OK) rc = upload(&t->d_tk_groups, tk_groups);
     if (rc == GCE_OK) rc = upload(&t->d_sunit_layer, sunit_layer);
     if (rc == GCE_OK) rc = upload(&t->d_sunit_part, sunit_part);
     if (rc == GCE_OK) rc = upload(&t->d_dtile_layer, dtile_layer);
