@@ -363,7 +363,7 @@ def run_workload(name, args, world, rank, dev, primary):
     mem = torch.zeros((W, N), dtype=torch.float32, device=dev)
     vals = torch.zeros((W, table.vals_per_worker), dtype=torch.float32, device=dev)
     idx = torch.zeros((W, table.vals_per_worker), dtype=torch.int32, device=dev)
-    ws = table.workspace(W, spec["method"])
+    ws = table.workspace(W, "powersgd" if spec["method"] == "powersgd_lazy" else spec["method"])
     ws_dc = table.workspace(W, "decompress")
     out = torch.zeros(N, dtype=torch.float32, device=dev)
     method = spec["method"]

@@ -79,7 +79,7 @@ SIGNATURES = {
                                    C.c_size_t, _vp]),
     "powersgd_step_lazy": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
                                      C.c_size_t, _vp]),
-    "gce_materialize_memory": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "gce_materialize_memory": (C.c_int, [_vp, _i32, _vp, _vp, _vp, C.c_size_t, _vp]),
     "ef_sign_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, C.c_size_t, _vp]),
     "decompress_vote": (C.c_int, [_vp, _i32, _vp, _f32, _vp, _vp]),
     "accordion_init": (C.c_int, [_vp, _vp, _vp, _vp]),
@@ -271,11 +271,12 @@ def powersgd_step_lazy(table, W, grad, mem, eta, k_or_rank, P, Q, vals, lazy_ran
         _ptr(lazy_rank, _i32()), _ptr(ws), ws.numel(), _stream(stream)))
 
 
-def materialize_memory(table, W, mem, P, Q, lazy_rank, stream=None):
-    """mem <- M - P Q^T where a lazy step left M; lazy_rank -> 0."""
+def materialize_memory(table, W, mem, lazy_rank, ws, stream=None):
+    """mem <- M - P Q^T where lazy steps left M (their workspace ws holds the
+    factors); lazy_rank -> 0."""
     _check("gce_materialize_memory", lib().gce_materialize_memory(
-        table.handle, int(W), _ptr(mem, _f32()), _ptr(P, _f32()), _ptr(Q, _f32()),
-        _ptr(lazy_rank, _i32()), _stream(stream)))
+        table.handle, int(W), _ptr(mem, _f32()), _ptr(lazy_rank, _i32()), _ptr(ws), ws.numel(),
+        _stream(stream)))
 
 
 def powersgd_dp_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, ws, stream=None):

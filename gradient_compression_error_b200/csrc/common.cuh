@@ -162,6 +162,22 @@ inline int resident_blocks(K kernel, int threads) {
     return n;
 }
 
+// The same for a kernel with `smem` bytes of dynamic shared memory; allows the
+// kernel that much (above the 48 KB default) on the current device first.
+template <class K>
+inline int resident_blocks_smem(K kernel, int threads, size_t smem) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess)
+        cudaGetLastError();
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
+        n < 1) {
+        cudaGetLastError();
+        n = 1;
+    }
+    return n;
+}
+
 // Grid of a grid-stride kernel: at most `per_sm` blocks per SM and never more
 // than fit at once (`resident`), so the whole grid runs in one wave.  A block
 // of a second, partial wave would start only when a first-wave block had

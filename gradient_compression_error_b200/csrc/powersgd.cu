@@ -129,15 +129,19 @@ void powersgd_plan_free(gce_table* t) {
 }
 
 struct PsWs {
-    size_t ppart = 0, pd = 0, qpart = 0, qloc = 0, tparts = 0, tscal = 0, tdone = 0, total = 0;
+    size_t ppart = 0, pd = 0, qpart = 0, qd = 0, qloc = 0, tparts = 0, tscal = 0, tdone = 0,
+           total = 0;
 };
 
+// pd and qd hold the last step's fp64 orthonormal P and Q' (the lazy step
+// takes its residual from them); the partial sums are fp64 too.
 static PsWs ps_layout(const gce_table* t, int32_t W) {
     PsWs o;
     Carver c;
-    o.ppart = c.take<float>(int64_t(W) * t->ppart_pw);
+    o.ppart = c.take<double>(int64_t(W) * t->ppart_pw);
     o.pd = c.take<double>(int64_t(W) * t->pd_pw);
-    o.qpart = c.take<float>(int64_t(W) * t->qpart_pw);
+    o.qpart = c.take<double>(int64_t(W) * t->qpart_pw);
+    o.qd = c.take<double>(int64_t(W) * t->Q_pw);
     o.tparts = c.take<double>(int64_t(W) * t->ps_tall_parts);
     o.tscal = c.take<double>(int64_t(W) * t->ps_ntall);
     o.tdone = c.take<int32_t>(int64_t(W) * t->ps_ntall);
@@ -148,13 +152,14 @@ static PsWs ps_layout(const gce_table* t, int32_t W) {
 size_t powersgd_ws_bytes(const gce_table* t, int32_t W) { return ps_layout(t, W).total; }
 
 // The data-parallel step: partials per worker, one orthonormal P per layer,
-// and every worker's Q_w kept for its residual.
+// and every worker's Q_w (fp32 for the mean, fp64 for its residual).
 static PsWs ps_dp_layout(const gce_table* t, int32_t W) {
     PsWs o;
     Carver c;
-    o.ppart = c.take<float>(int64_t(W) * t->ppart_pw);
+    o.ppart = c.take<double>(int64_t(W) * t->ppart_pw);
     o.pd = c.take<double>(t->pd_pw);
-    o.qpart = c.take<float>(int64_t(W) * t->qpart_pw);
+    o.qpart = c.take<double>(int64_t(W) * t->qpart_pw);
+    o.qd = c.take<double>(int64_t(W) * t->Q_pw);
     o.qloc = c.take<float>(int64_t(W) * t->Q_pw);
     o.tparts = c.take<double>(t->ps_tall_parts);
     o.tscal = c.take<double>(t->ps_ntall);
@@ -188,34 +193,48 @@ __global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
     }
 }
 
-// m = M - P Q^T for one entry, formed exactly as the residual pass and the
-// decoder form it: the product of column 0, then fused multiply-adds in
-// column order, then one rounded subtraction.
-__device__ __forceinline__ float ps_unproject(float M, const float* pr, const float (*qs)[kPsCB],
-                                              int c, int r) {
-    float mh = __fmul_rn(pr[0], qs[0][c]);
+// The residual of one entry: m = fl32(M - sum_j P_j Q'_j), the sum in fp64
+// (products of column 0, then fused multiply-adds in column order) from the
+// fp64 orthonormal P and fp64 Q' -- the residual pass and the lazy step's
+// first pass form it identically.
+__device__ __forceinline__ float ps_unproject(float M, const double* pr,
+                                              const double (*qd)[kPsCB], int c, int r) {
+    double mh = __dmul_rn(pr[0], qd[0][c]);
 #pragma unroll
     for (int j = 1; j < kMaxRank; ++j)
-        if (j < r) mh = __fmaf_rn(pr[j], qs[j][c], mh);
-    return __fsub_rn(M, mh);
+        if (j < r) mh = __fma_rn(pr[j], qd[j][c], mh);
+    return __double2float_rn(__dsub_rn(double(M), mh));
 }
 
+constexpr size_t ps_mq_smem(bool lazy) {
+    return lazy ? sizeof(double) * (2 * kMaxRank * kPsCB + kPsRB * kMaxRank)
+                : sizeof(double) * kMaxRank * kPsCB;
+}
+constexpr size_t kPsResidSmem = sizeof(double) * (kMaxRank * kPsCB + kPsRB * kMaxRank) +
+                                sizeof(float) * (kMaxRank * kPsCB + kPsRB * kMaxRank);
+
 // ---- phase 1: M = m + eta*g (written back), partial P = M Q -------------------------------
-// kLazy: the memory holds the previous step's M, and P / Q that step's
-// orthonormal P and Q' over lazy_rank[w][l] columns (0: the memory holds the
-// residual itself); the residual m = M - P Q'^T is formed on the fly, entry by
-// entry as the residual pass would have formed it, so the results are the
-// eager step's bit for bit without that pass's read and write of M.
+// Products and row sums in fp64 (the contraction is bandwidth-bound; fp64
+// keeps it within rounding-order distance of an fp64 reference).
+// kLazy: the memory holds the previous step's M, the workspace that step's
+// fp64 orthonormal P and Q' over lazy_rank[w][l] columns (0: the memory holds
+// the residual itself); the residual m is formed on the fly, entry by entry
+// as the residual pass would have formed it, so the results are the eager
+// step's bit for bit without that pass's read and write of M.
 template <bool kLazy>
 __global__ void __launch_bounds__(256) ps_mq_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t Q_pw,
     int64_t ppart_pw, const float* __restrict__ grad, float* __restrict__ mem, float eta,
-    const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, float* __restrict__ ppart,
-    int32_t* __restrict__ status, const float* __restrict__ P, int64_t P_pw, int32_t L_all,
-    const int32_t* __restrict__ lazy_rank) {
-    __shared__ float qs[kMaxRank][kPsCB];
-    __shared__ float prow[kPsRB][kMaxRank];
+    const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, double* __restrict__ ppart,
+    int32_t* __restrict__ status, const double* __restrict__ pdw, int64_t pd_pw,
+    const double* __restrict__ qdw, int32_t L_all, const int32_t* __restrict__ lazy_rank) {
+    // dynamic shared memory (ps_mq_smem bytes): the warm start Q, then (lazy)
+    // the previous Q' and the previous P rows, all fp64
+    extern __shared__ __align__(16) double ps_dyn[];
+    double (*qs)[kPsCB] = reinterpret_cast<double (*)[kPsCB]>(ps_dyn);
+    double (*qdp)[kPsCB] = qs + kMaxRank;
+    double (*prow)[kMaxRank] = reinterpret_cast<double (*)[kMaxRank]>(ps_dyn + 2 * kMaxRank * kPsCB);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
         const int w = int(u / ntiles);
@@ -231,44 +250,52 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
             rp = lazy_rank[int64_t(w) * L_all + d.x];
             rp = (rp >= 1 && rp <= cap) ? rp : 0;
         }
-        const int rq = r > rp ? r : rp;  // Q columns staged
         const int64_t C = L.cols, R = L.rows;
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
         const int64_t r0 = int64_t(d.y) * kPsRB;
         const int rh = int(min64(kPsRB, R - r0));
         const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
-        for (int i = tid; i < cw * rq; i += blockDim.x) {
-            const int c = i / rq, j = i - c * rq;
-            qs[j][c] = q[int64_t(c) * cap + j];
+        for (int i = tid; i < cw * r; i += blockDim.x) {
+            const int c = i / r, j = i - c * r;
+            qs[j][c] = double(q[int64_t(c) * cap + j]);
         }
-        if (kLazy && rp > 0) {
-            const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+        if constexpr (kLazy) {
+          if (rp > 0) {
+            const double* qp = qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap;
+            for (int i = tid; i < cw * rp; i += blockDim.x) {
+                const int c = i / rp, j = i - c * rp;
+                qdp[j][c] = qp[int64_t(c) * cap + j];
+            }
+            const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
             for (int i = tid; i < rh * rp; i += blockDim.x) {
                 const int row = i / rp, j = i - row * rp;
                 prow[row][j] = p[int64_t(row) * cap + j];
             }
+          }
         }
         __syncthreads();
         for (int row = warp; row < rh; row += blockDim.x >> 5) {
             const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
             const float* g = grad + e;
             float* m = mem + e;
-            float pr[kMaxRank] = {0.f, 0.f, 0.f, 0.f};
+            double pr[kMaxRank] = {0.0, 0.0, 0.0, 0.0};
             if (kLazy && rp > 0) {
 #pragma unroll
-                for (int j = 0; j < kMaxRank; ++j) pr[j] = j < rp ? prow[row][j] : 0.0f;
+                for (int j = 0; j < kMaxRank; ++j) pr[j] = j < rp ? prow[row][j] : 0.0;
             }
-            float acc[kMaxRank] = {0.f, 0.f, 0.f, 0.f};
+            double acc[kMaxRank] = {0.0, 0.0, 0.0, 0.0};
             if (((e & 3) == 0) && ((cw & 3) == 0)) {
                 for (int c = lane * 4; c < cw; c += 128) {
                     const float4 gg = ld_stream4(g + c);
                     float4 mm = *reinterpret_cast<const float4*>(m + c);
-                    if (kLazy && rp > 0) {
-                        mm.x = ps_unproject(mm.x, pr, qs, c, rp);
-                        mm.y = ps_unproject(mm.y, pr, qs, c + 1, rp);
-                        mm.z = ps_unproject(mm.z, pr, qs, c + 2, rp);
-                        mm.w = ps_unproject(mm.w, pr, qs, c + 3, rp);
+                    if constexpr (kLazy) {
+                        if (rp > 0) {
+                            mm.x = ps_unproject(mm.x, pr, qdp, c, rp);
+                            mm.y = ps_unproject(mm.y, pr, qdp, c + 1, rp);
+                            mm.z = ps_unproject(mm.z, pr, qdp, c + 2, rp);
+                            mm.w = ps_unproject(mm.w, pr, qdp, c + 3, rp);
+                        }
                     }
                     float4 x;
                     x.x = residual(mm.x, eta, gg.x);
@@ -279,30 +306,32 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
 #pragma unroll
                     for (int j = 0; j < kMaxRank; ++j) {
                         if (j < r) {
-                            acc[j] = fmaf(x.x, qs[j][c], acc[j]);
-                            acc[j] = fmaf(x.y, qs[j][c + 1], acc[j]);
-                            acc[j] = fmaf(x.z, qs[j][c + 2], acc[j]);
-                            acc[j] = fmaf(x.w, qs[j][c + 3], acc[j]);
+                            acc[j] = __fma_rn(double(x.x), qs[j][c], acc[j]);
+                            acc[j] = __fma_rn(double(x.y), qs[j][c + 1], acc[j]);
+                            acc[j] = __fma_rn(double(x.z), qs[j][c + 2], acc[j]);
+                            acc[j] = __fma_rn(double(x.w), qs[j][c + 3], acc[j]);
                         }
                     }
                 }
             } else {
                 for (int c = lane; c < cw; c += 32) {
                     float mv = m[c];
-                    if (kLazy && rp > 0) mv = ps_unproject(mv, pr, qs, c, rp);
+                    if constexpr (kLazy) {
+                        if (rp > 0) mv = ps_unproject(mv, pr, qdp, c, rp);
+                    }
                     const float x = residual(mv, eta, __ldcs(g + c));
                     m[c] = x;
 #pragma unroll
                     for (int j = 0; j < kMaxRank; ++j)
-                        if (j < r) acc[j] = fmaf(x, qs[j][c], acc[j]);
+                        if (j < r) acc[j] = __fma_rn(double(x), qs[j][c], acc[j]);
                 }
             }
             // a NaN or infinite M makes its row's products non-finite
-            flag_nonfinite(!(fabsf(acc[0]) <= 3.4e38f), status);
+            flag_nonfinite(!(fabs(acc[0]) <= 1.0e300), status);
 #pragma unroll
             for (int j = 0; j < kMaxRank; ++j) acc[j] = warp_sum(acc[j]);
             if (lane < r) {
-                float a = acc[0];
+                double a = acc[0];
                 if (lane == 1) a = acc[1];
                 if (lane == 2) a = acc[2];
                 if (lane == 3) a = acc[3];
@@ -332,7 +361,7 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W, int32_t nsum, int64_t P_pw,
     int64_t ppart_pw,
-    int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ ppart,
+    int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const double* __restrict__ ppart,
     double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status,
     int32_t ntall, int32_t* __restrict__ tdone, int32_t L_all, int32_t* __restrict__ lazy_rank) {
     __shared__ double s_red[32];
@@ -356,7 +385,7 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         }
         const int cap = L.cap;
         const int64_t R = L.rows;
-        const float* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
+        const double* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
         double* pd = pdw + int64_t(w) * pd_pw + X.pd_off;
         for (int64_t i = threadIdx.x; i < R * r; i += blockDim.x) {
             const int64_t row = i / r;
@@ -364,7 +393,7 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
             double s = 0.0;
             for (int ws = 0; ws < nsum; ++ws)
                 for (int ch = 0; ch < X.nch1; ++ch)
-                    s += double(pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j]);
+                    s += pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j];
             pd[row * cap + j] = s;
         }
         __syncthreads();
@@ -416,7 +445,7 @@ __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
     const int2* __restrict__ units, int32_t nunits, int32_t W, int32_t nsum, int64_t P_pw,
     int64_t ppart_pw, int64_t pd_pw, int32_t ntall, int32_t nparts,
     const int32_t* __restrict__ k_or_rank,
-    const float* __restrict__ ppart, double* __restrict__ pdw, double* __restrict__ tparts,
+    const double* __restrict__ ppart, double* __restrict__ pdw, double* __restrict__ tparts,
     double* __restrict__ tscal, int32_t* __restrict__ tdone, float* __restrict__ P) {
     __shared__ double s_red[8];
     __shared__ int s_last;
@@ -434,13 +463,13 @@ __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
         double* pd = pdw + int64_t(w) * pd_pw + X.pd_off;
         double* scal = tscal + int64_t(w) * ntall + X.tall;
         if (op.init) {
-            const float* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
+            const double* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
             for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
                 for (int j = 0; j < r; ++j) {
                     double s = 0.0;
                     for (int ws = 0; ws < nsum; ++ws)
                         for (int ch = 0; ch < X.nch1; ++ch)
-                            s += double(pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j]);
+                            s += pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j];
                     pd[row * cap + j] = s;
                 }
         }
@@ -517,12 +546,13 @@ static std::vector<PsOrthOp> ps_orth_ops(int cap) {
 }
 
 // ---- phase 3: partial Q = M^T P over 64-row blocks ---------------------------------------
+// From the fp64 orthonormal P (the workspace copy), products and sums in fp64.
 __global__ void __launch_bounds__(256) ps_mtp_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
-    const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t P_pw,
+    const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t pd_pw,
     int64_t qpart_pw, const float* __restrict__ mem, const int32_t* __restrict__ k_or_rank,
-    const float* __restrict__ P, float* __restrict__ qpart) {
-    __shared__ float prow[kPsRB3][kMaxRank];
+    const double* __restrict__ pdw, double* __restrict__ qpart) {
+    __shared__ double prow[kPsRB3][kMaxRank];
     const int tid = threadIdx.x;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
         const int w = int(u / ntiles);
@@ -537,18 +567,18 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
         const int rh = int(min64(kPsRB3, L.rows - r0));
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
-        const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+        const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
         for (int i = tid; i < rh * kMaxRank; i += blockDim.x) {
             const int row = i / kMaxRank, j = i % kMaxRank;
-            prow[row][j] = j < r ? p[int64_t(row) * cap + j] : 0.0f;
+            prow[row][j] = j < r ? p[int64_t(row) * cap + j] : 0.0;
         }
         __syncthreads();
         const int cc = tid * 4;
-        float acc[4][kMaxRank];
+        double acc[4][kMaxRank];
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-            for (int j = 0; j < kMaxRank; ++j) acc[q][j] = 0.0f;
+            for (int j = 0; j < kMaxRank; ++j) acc[q][j] = 0.0;
         const int64_t ebase = int64_t(w) * N + L.offset + r0 * C + c0;
         const bool vec = ((ebase & 3) == 0) && ((C & 3) == 0) && (cc + 3 < cw);
         if (cc < cw) {
@@ -565,9 +595,10 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
 #pragma unroll
-                    for (int j = 0; j < kMaxRank; ++j) acc[q][j] = fmaf(x[q], prow[row][j], acc[q][j]);
+                    for (int j = 0; j < kMaxRank; ++j)
+                        if (j < r) acc[q][j] = __fma_rn(double(x[q]), prow[row][j], acc[q][j]);
             }
-            float* out = qpart + int64_t(w) * qpart_pw + X.qpart_off + (int64_t(d.y) * C + c0 + cc) * cap;
+            double* out = qpart + int64_t(w) * qpart_pw + X.qpart_off + (int64_t(d.y) * C + c0 + cc) * cap;
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 if (cc + q < cw)
@@ -580,15 +611,17 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
 }
 
 // ---- Q = sum of the row-block partials (fp64, block order) ----------------------------------
+// Q' in fp64 to qd (stride Q_pw per worker) and rounded to fp32 to Q.
 // kMean (the data-parallel step): every worker's Q_w goes to Q (stride
-// Q_pw) and their mean -- fp32 sum in worker order from +0, times inv_w --
-// to qmean, one tile per block for all W workers.
+// Q_pw, fp32) and qd (fp64), and their mean -- fp32 sum of the rounded Q_w in
+// worker order from +0, times inv_w -- to qmean, one tile per block for all W
+// workers.
 template <bool kMean>
 __global__ void __launch_bounds__(256) ps_qred_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t Q_pw, int64_t qpart_pw,
-    const int32_t* __restrict__ k_or_rank, const float* __restrict__ qpart, float* __restrict__ Q,
-    float* __restrict__ qmean, float inv_w) {
+    const int32_t* __restrict__ k_or_rank, const double* __restrict__ qpart,
+    float* __restrict__ Q, double* __restrict__ qd, float* __restrict__ qmean, float inv_w) {
     const int64_t nunits = kMean ? int64_t(ntiles) : int64_t(ntiles) * W;
     for (int64_t u = blockIdx.x; u < nunits; u += gridDim.x) {
         const int w = kMean ? 0 : int(u / ntiles);
@@ -607,11 +640,12 @@ __global__ void __launch_bounds__(256) ps_qred_kernel(
             float mean = 0.0f;
             for (int wi = 0; wi < (kMean ? W : 1); ++wi) {
                 const int ww = kMean ? wi : w;
-                const float* qp = qpart + int64_t(ww) * qpart_pw + X.qpart_off;
+                const double* qp = qpart + int64_t(ww) * qpart_pw + X.qpart_off;
                 double s = 0.0;
-                for (int rb = 0; rb < X.nrb3; ++rb) s += double(qp[(int64_t(rb) * C + c) * cap + j]);
+                for (int rb = 0; rb < X.nrb3; ++rb) s += qp[(int64_t(rb) * C + c) * cap + j];
                 const float qv = float(s);
                 Q[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = qv;
+                qd[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = s;
                 if (kMean) mean = __fadd_rn(mean, qv);
             }
             if (kMean) qmean[L.q_off + c * cap + j] = __fmul_rn(mean, inv_w);
@@ -645,20 +679,32 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
 }
 
 // ---- residual: m <- M - P Q^T, dense_out <- P Q^T ---------------------------------------------
+// The memory from the fp64 factors (ps_unproject); dense_out from the fp32
+// P and Q the payload carries, formed as the decoder forms it (product, then
+// fp32 fused multiply-adds in column order), so dense_out is the decode.
 // rank_wl (nullable): per (worker, layer) ranks [W][L_all] instead of
 // k_or_rank -- the lazy step's record, for gce_materialize_memory.
 __global__ void __launch_bounds__(256) ps_resid_kernel(
-    const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles, int32_t W,
-    int64_t N, int64_t P_pw, int64_t Q_pw, const int32_t* __restrict__ k_or_rank,
-    const float* __restrict__ P, const float* __restrict__ Q, float* __restrict__ mem,
-    float* __restrict__ dense_out, const int32_t* __restrict__ rank_wl, int32_t L_all) {
-    __shared__ float qs[kMaxRank][kPsCB];
-    __shared__ float prow[kPsRB][kMaxRank];
+    const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
+    const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t P_pw,
+    int64_t Q_pw, int64_t pd_pw, const int32_t* __restrict__ k_or_rank,
+    const float* __restrict__ P, const float* __restrict__ Q, const double* __restrict__ pdw,
+    const double* __restrict__ qdw, float* __restrict__ mem, float* __restrict__ dense_out,
+    const int32_t* __restrict__ rank_wl, int32_t L_all) {
+    // dynamic shared memory (kPsResidSmem bytes)
+    extern __shared__ __align__(16) double ps_dyn[];
+    double (*qd)[kPsCB] = reinterpret_cast<double (*)[kPsCB]>(ps_dyn);
+    double (*prow)[kMaxRank] = reinterpret_cast<double (*)[kMaxRank]>(ps_dyn + kMaxRank * kPsCB);
+    float (*qs)[kPsCB] =
+        reinterpret_cast<float (*)[kPsCB]>(ps_dyn + kMaxRank * kPsCB + kPsRB * kMaxRank);
+    float (*prow32)[kMaxRank] = reinterpret_cast<float (*)[kMaxRank]>(
+        reinterpret_cast<float*>(qs) + kMaxRank * kPsCB);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
         const int w = int(u / ntiles);
         const int4 d = tiles[u % ntiles];
         const DevLayer L = layers[d.x];
+        const PsLayer X = ps[d.x];
         int r = 0;
         if (rank_wl) {
             r = rank_wl[int64_t(w) * L_all + d.x];
@@ -673,50 +719,63 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
         const int cw = int(min64(kPsCB, C - c0));
         const int64_t r0 = int64_t(d.y) * kPsRB;
         const int rh = int(min64(kPsRB, R - r0));
-        const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
+        const double* qp = qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap;
         for (int i = tid; i < cw * r; i += blockDim.x) {
             const int c = i / r, j = i - c * r;
-            qs[j][c] = q[int64_t(c) * cap + j];
+            qd[j][c] = qp[int64_t(c) * cap + j];
         }
-        const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+        const double* pp = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
         for (int i = tid; i < rh * r; i += blockDim.x) {
             const int row = i / r, j = i - row * r;
-            prow[row][j] = p[int64_t(row) * cap + j];
+            prow[row][j] = pp[int64_t(row) * cap + j];
+        }
+        if (dense_out) {
+            const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
+            for (int i = tid; i < cw * r; i += blockDim.x) {
+                const int c = i / r, j = i - c * r;
+                qs[j][c] = q[int64_t(c) * cap + j];
+            }
+            const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
+            for (int i = tid; i < rh * r; i += blockDim.x) {
+                const int row = i / r, j = i - row * r;
+                prow32[row][j] = p[int64_t(row) * cap + j];
+            }
         }
         __syncthreads();
         for (int row = warp; row < rh; row += blockDim.x >> 5) {
             const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
             float* m = mem + e;
             float* o = dense_out ? dense_out + e : nullptr;
-            float pr[kMaxRank];
+            double pr[kMaxRank];
+            float pr32[kMaxRank];
 #pragma unroll
-            for (int j = 0; j < kMaxRank; ++j) pr[j] = j < r ? prow[row][j] : 0.0f;
+            for (int j = 0; j < kMaxRank; ++j) {
+                pr[j] = j < r ? prow[row][j] : 0.0;
+                pr32[j] = (o && j < r) ? prow32[row][j] : 0.0f;
+            }
+            auto decoded = [&](int c) {
+                float mh = __fmul_rn(pr32[0], qs[0][c]);
+#pragma unroll
+                for (int j = 1; j < kMaxRank; ++j)
+                    if (j < r) mh = __fmaf_rn(pr32[j], qs[j][c], mh);
+                return mh;
+            };
             if (((e & 3) == 0) && ((cw & 3) == 0)) {  // 16-byte rows: four columns a lane
                 for (int c = lane * 4; c < cw; c += 128) {
                     float4 mm = *reinterpret_cast<const float4*>(m + c);
-                    float mh[4];
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        mh[q] = __fmul_rn(pr[0], qs[0][c + q]);
-#pragma unroll
-                        for (int j = 1; j < kMaxRank; ++j)
-                            if (j < r) mh[q] = __fmaf_rn(pr[j], qs[j][c + q], mh[q]);
-                    }
-                    mm.x = __fsub_rn(mm.x, mh[0]);
-                    mm.y = __fsub_rn(mm.y, mh[1]);
-                    mm.z = __fsub_rn(mm.z, mh[2]);
-                    mm.w = __fsub_rn(mm.w, mh[3]);
+                    mm.x = ps_unproject(mm.x, pr, qd, c, r);
+                    mm.y = ps_unproject(mm.y, pr, qd, c + 1, r);
+                    mm.z = ps_unproject(mm.z, pr, qd, c + 2, r);
+                    mm.w = ps_unproject(mm.w, pr, qd, c + 3, r);
                     __stcs(reinterpret_cast<float4*>(m + c), mm);
-                    if (o) __stcs(reinterpret_cast<float4*>(o + c), make_float4(mh[0], mh[1], mh[2], mh[3]));
+                    if (o)
+                        __stcs(reinterpret_cast<float4*>(o + c),
+                               make_float4(decoded(c), decoded(c + 1), decoded(c + 2), decoded(c + 3)));
                 }
             } else {
                 for (int c = lane; c < cw; c += 32) {
-                    float mh = __fmul_rn(pr[0], qs[0][c]);
-#pragma unroll
-                    for (int j = 1; j < kMaxRank; ++j)
-                        if (j < r) mh = __fmaf_rn(pr[j], qs[j][c], mh);
-                    m[c] = __fsub_rn(m[c], mh);
-                    if (o) o[c] = mh;
+                    m[c] = ps_unproject(m[c], pr, qd, c, r);
+                    if (o) o[c] = decoded(c);
                 }
             }
         }
@@ -868,27 +927,30 @@ static int ps_step(const gce_table* t, int32_t W, const float* grad, float* mem,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t* status = static_cast<int32_t*>(ws);
     if (t->nps > 0) {
-        float* ppart = at<float>(ws, lay.ppart);
+        double* ppart = at<double>(ws, lay.ppart);
         double* pd = at<double>(ws, lay.pd);
-        float* qpart = at<float>(ws, lay.qpart);
+        double* qpart = at<double>(ws, lay.qpart);
+        double* qd = at<double>(ws, lay.qd);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_mq = resident_blocks(ps_mq_kernel<false>, 256);
-        static const int r_mql = resident_blocks(ps_mq_kernel<true>, 256);
+        static const int r_mq = resident_blocks_smem(ps_mq_kernel<false>, 256, ps_mq_smem(false));
+        static const int r_mql = resident_blocks_smem(ps_mq_kernel<true>, 256, ps_mq_smem(true));
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
-        static const int r_resid = resident_blocks(ps_resid_kernel, 256);
+        static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
         if (lazy_rank)
-            GCE_LAUNCH(ps_mq_kernel<true>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mql), 256, 0, st,
+            GCE_LAUNCH(ps_mq_kernel<true>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mql), 256,
+                       ps_mq_smem(true), st,
                        t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw,
-                       t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, P, t->P_pw, t->L,
-                       lazy_rank);
+                       t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, pd, t->pd_pw, qd,
+                       t->L, lazy_rank);
         else
-            GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
+            GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256,
+                       ps_mq_smem(false), st,
                        t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw,
                        t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, nullptr,
-                       int64_t(0), t->L, nullptr);
+                       int64_t(0), nullptr, t->L, nullptr);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, 1, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
@@ -902,17 +964,18 @@ static int ps_step(const gce_table* t, int32_t W, const float* grad, float* mem,
                            at<double>(ws, lay.tscal), tdone, P);
         }
         GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
-                   t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->P_pw, t->qpart_pw,
-                   mem, k_or_rank, P, qpart);
+                   t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->pd_pw, t->qpart_pw,
+                   mem, k_or_rank, pd, qpart);
         GCE_LAUNCH(ps_qred_kernel<false>, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0,
                    st, t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
-                   k_or_rank, qpart, Q, nullptr, 1.0f);
+                   k_or_rank, qpart, Q, qd, nullptr, 1.0f);
         // the lazy step leaves M in the memory: the next step (or
         // gce_materialize_memory) takes P Q^T off
         if (!lazy_rank)
-            GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
-                       t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
-                       k_or_rank, P, Q, mem, dense_out, nullptr, t->L);
+            GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
+                       kPsResidSmem, st,
+                       t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
+                       t->pd_pw, k_or_rank, P, Q, pd, qd, mem, dense_out, nullptr, t->L);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
@@ -934,18 +997,23 @@ extern "C" int powersgd_step_lazy(const gce_table* t, int32_t W, const float* gr
                    stream);
 }
 
-extern "C" int gce_materialize_memory(const gce_table* t, int32_t W, float* mem, const float* P,
-                                      const float* Q, int32_t* lazy_rank, void* stream) {
-    if (!t || W < 1 || !mem || !lazy_rank || !aligned16(mem)) return GCE_ERR_ARG;
+extern "C" int gce_materialize_memory(const gce_table* t, int32_t W, float* mem,
+                                      int32_t* lazy_rank, void* ws, size_t ws_bytes,
+                                      void* stream) {
+    if (!t || W < 1 || !mem || !lazy_rank || !ws || !aligned16(mem) || !aligned16(ws))
+        return GCE_ERR_ARG;
     if (reinterpret_cast<uintptr_t>(lazy_rank) & 3) return GCE_ERR_ARG;
     if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    const PsWs lay = ps_layout(t, W);
+    if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (t->nps > 0) {
-        if (!P || !Q || !aligned16(P) || !aligned16(Q)) return GCE_ERR_ARG;
-        static const int r_resid = resident_blocks(ps_resid_kernel, 256);
-        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
-                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
-                   nullptr, P, Q, mem, nullptr, lazy_rank, t->L);
+        static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
+        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
+                       kPsResidSmem, st,
+                   t->d_layers, static_cast<const PsLayer*>(t->d_ps), t->d_ps1_tiles,
+                   t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw, t->pd_pw, nullptr, nullptr, nullptr,
+                   at<double>(ws, lay.pd), at<double>(ws, lay.qd), mem, nullptr, lazy_rank, t->L);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     if (cudaMemsetAsync(lazy_rank, 0, sizeof(int32_t) * size_t(W) * size_t(t->L), st) !=
@@ -971,23 +1039,25 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
     int32_t* status = static_cast<int32_t*>(ws);
     const float inv_w = 1.0f / float(W);
     if (t->nps > 0) {
-        float* ppart = at<float>(ws, lay.ppart);
+        double* ppart = at<double>(ws, lay.ppart);
         double* pd = at<double>(ws, lay.pd);
-        float* qpart = at<float>(ws, lay.qpart);
+        double* qpart = at<double>(ws, lay.qpart);
+        double* qd = at<double>(ws, lay.qd);
         float* qloc = at<float>(ws, lay.qloc);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_mq = resident_blocks(ps_mq_kernel<false>, 256);
+        static const int r_mq = resident_blocks_smem(ps_mq_kernel<false>, 256, ps_mq_smem(false));
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<true>, 256);
-        static const int r_resid = resident_blocks(ps_resid_kernel, 256);
+        static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
         // every worker reads the shared warm start Q (stride 0)
-        GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256, 0, st,
+        GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256,
+                   ps_mq_smem(false), st,
                    t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0),
                    t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, nullptr, int64_t(0),
-                   t->L, nullptr);
+                   nullptr, t->L, nullptr);
         // one P per layer from the partials of all W workers
         GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank,
@@ -1003,14 +1073,15 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         // Q_w = M_w^T P for every worker with the shared P (stride 0)
         GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
                    t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, int64_t(0),
-                   t->qpart_pw, mem, k_or_rank, P, qpart);
+                   t->qpart_pw, mem, k_or_rank, pd, qpart);
         GCE_LAUNCH(ps_qred_kernel<true>, wave_grid(t->psq_ntiles, 8, r_qred), 256, 0, st,
                    t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
-                   k_or_rank, qpart, qloc, Q, inv_w);
-        // each worker's error against its own Q_w
-        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256, 0, st,
-                   t->d_layers, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->Q_pw,
-                   k_or_rank, P, qloc, mem, nullptr, nullptr, t->L);
+                   k_or_rank, qpart, qloc, qd, Q, inv_w);
+        // each worker's error against its own Q_w (the shared fp64 P, stride 0)
+        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
+                       kPsResidSmem, st,
+                   t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->Q_pw,
+                   int64_t(0), k_or_rank, P, qloc, pd, qd, mem, nullptr, nullptr, t->L);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     if (t->dtiles_pw > 0) {

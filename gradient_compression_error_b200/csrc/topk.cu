@@ -179,9 +179,10 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
                 ok[q] = e < ne && pos < L.n;
                 vv[q] = ok[q] ? residual(m[pos], eta, __ldcs(g + pos)) : 0.0f;
             }
+            // most samples fall in a few bins near the bulk of |v|: one
+            // shared-memory atomic per distinct bin of the warp
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q)
-                if (ok[q]) atomicAdd(&h[abs_key(vv[q]) >> 19], 1);
+            for (int q = 0; q < kBatch; ++q) hist_add(h, abs_key(vv[q]) >> 19, ok[q]);
         }
         __syncthreads();
         int32_t* gh = tk_hist(hists, S, 0, seg);
@@ -677,39 +678,52 @@ __device__ __forceinline__ void tk_emit_item(
         sh.cnt_eq[warp] = eq;
     }
     __syncthreads();
-    if (tid == 0) {
-        int64_t ggt = 0, geq = 0;
+    if (warp == 0) {
+        int64_t ggt = 0, geq = 0;  // this item's counts
         for (int i = 0; i < kTkGroup; ++i) {
-            sh.base_gt[i] = int32_t(ggt);
-            sh.base_eq[i] = int32_t(geq);
             ggt += sh.cnt_gt[i];
             geq += sh.cnt_eq[i];
         }
-        int64_t pgt = 0, peq = 0;  // counts of the segment's earlier items
-        if (tile_info[gr.x].tstart == 0) {
-            st_release_gpu_u64(gstate + e, kTkInc | tk_pack(ggt, geq));
-        } else {
-            st_release_gpu_u64(gstate + e, kTkAgg | tk_pack(ggt, geq));
-            // the same segment's previous items sit W entries apart
-            for (int64_t j = e - W;; j -= W) {
-                uint64_t v = ld_acquire_gpu_u64(gstate + j);
+        // items of the layer before this one (its first item has none)
+        const int64_t before = int64_t(tile_info[gr.x].tstart / kTkTile) / kTkGroup;
+        if (lane == 0) st_release_gpu_u64(gstate + e, (before ? kTkAgg : kTkInc) | tk_pack(ggt, geq));
+        // look back a warp at a time: lane i reads the item i + 1 back (W
+        // entries apart), until one has published its running counts
+        int64_t pgt = 0, peq = 0;
+        for (int64_t back = 1; back <= before; back += 32) {
+            const int64_t jj = back + lane;
+            const bool have = jj <= before;
+            uint64_t v = 0;
+            if (have) {
+                const uint64_t* src = gstate + (e - jj * W);
+                v = ld_acquire_gpu_u64(src);
                 for (uint32_t n = 0; (v >> 62) == 0 && n < kTkSpinLimit; ++n) {
                     __nanosleep(32);
-                    v = ld_acquire_gpu_u64(gstate + j);
+                    v = ld_acquire_gpu_u64(src);
                 }
-                if ((v >> 62) == 0) {
+                if ((v >> 62) == 0) {  // never published: counted as empty and final
                     atomicOr(status, GCE_STATUS_WAIT_TIMEOUT);
-                    break;
+                    v = kTkInc;
                 }
-                pgt += int64_t((v >> 31) & 0x7FFFFFFFull);
-                peq += int64_t(v & 0x7FFFFFFFull);
-                if ((v >> 62) == 2) break;
             }
-            st_release_gpu_u64(gstate + e, kTkInc | tk_pack(pgt + ggt, peq + geq));
+            const unsigned inc = __ballot_sync(kFull, have && (v >> 62) == 2);
+            const int stop = inc ? __ffs(inc) - 1 : 31;
+            const bool take = have && lane <= stop;
+            const int64_t vg = take ? int64_t((v >> 31) & 0x7FFFFFFFull) : 0;
+            const int64_t ve = take ? int64_t(v & 0x7FFFFFFFull) : 0;
+            pgt += warp_sum(vg);
+            peq += warp_sum(ve);
+            if (inc) break;
         }
-        for (int i = 0; i < kTkGroup; ++i) {
-            sh.base_gt[i] += int32_t(pgt);
-            sh.base_eq[i] += int32_t(peq);
+        if (lane == 0) {
+            if (before) st_release_gpu_u64(gstate + e, kTkInc | tk_pack(pgt + ggt, peq + geq));
+            int64_t bgt = pgt, beq = peq;
+            for (int i = 0; i < kTkGroup; ++i) {
+                sh.base_gt[i] = int32_t(bgt);
+                sh.base_eq[i] = int32_t(beq);
+                bgt += sh.cnt_gt[i];
+                beq += sh.cnt_eq[i];
+            }
         }
     }
     __syncthreads();
@@ -757,7 +771,7 @@ __device__ __forceinline__ void tk_emit_item(
     }
 }
 
-__global__ void __launch_bounds__(256, 4) tk_select_kernel(
+__global__ void __launch_bounds__(256, 5) tk_select_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ comp, int32_t ncomp,
     int64_t S, int32_t W, int32_t tiles_pw, int64_t N, int64_t comp_N, int64_t vals_pw,
     const TileInfo* __restrict__ tile_info, const int2* __restrict__ groups, int32_t groups_pw,

@@ -240,17 +240,18 @@ GCE_API int powersgd_step(const gce_table* table, int32_t W, const float* grad, 
  *   unused), owned by the caller, zero before the first call (or after
  *   gce_materialize_memory).  Entry (w, l) = 0: mem holds the residual m, as
  *   powersgd_step leaves it.  Entry r > 0: mem holds the M of the last lazy
- *   step, and P / Q (columns 0..r-1) that step's orthonormal P and Q', so that
- *   the residual is m = M - P Q'^T (each entry formed as the decoder forms
- *   it).
+ *   step, and the workspace that step's fp64 orthonormal P and Q' over
+ *   columns 0..r-1, so that the residual is m = M - P Q'^T, each entry formed
+ *   as powersgd_step forms it.
  * The step forms m on the fly while it reads mem for M = m + eta*grad, writes
- * M (not M - P Q'^T) back to mem, and sets entry (w, l) to this step's rank (a
- * layer skipped for an out-of-range rank keeps its memory and its entry).
- * Memory traffic per element: grad read, memory read and written, M read once
- * more for Q' = M^T P (16 B, against 24 B for powersgd_step on layers that do
- * not stay in L2).  Other arguments, the workspace (GCE_OP_POWERSGD) and errors
- * as powersgd_step, without dense_out.  Between lazy steps the memory must be
- * left as it is; to read it, call gce_materialize_memory.
+ * M back to mem, and sets entry (w, l) to this step's rank (a layer skipped
+ * for an out-of-range rank keeps its memory and its entry).  Memory traffic
+ * per element: grad read, memory read and written, M read once more for
+ * Q' = M^T P (16 B, against 24 B for powersgd_step on layers that do not stay
+ * in L2).  Other arguments, the workspace (GCE_OP_POWERSGD) and errors as
+ * powersgd_step, without dense_out.  Between lazy steps the memory, lazy_rank
+ * and the workspace must be left as they are (the workspace carries the
+ * factors); to read the memory, call gce_materialize_memory.
  */
 GCE_API int powersgd_step_lazy(const gce_table* table, int32_t W, const float* grad, float* mem,
                                float eta, const int32_t* k_or_rank, float* P, float* Q,
@@ -258,13 +259,15 @@ GCE_API int powersgd_step_lazy(const gce_table* table, int32_t W, const float* g
                                void* stream);
 
 /*
- * Turns the memory a lazy step left into the residual: for every (w, l) with
- * lazy_rank entry r > 0, mem <- M - P Q^T over columns 0..r-1 (the residual
- * powersgd_step would have written, bit for bit); then every entry -> 0.
- * mem [W][N], P, Q, lazy_rank as powersgd_step_lazy.  No workspace.
+ * Turns the memory that lazy steps left into the residual: for every (w, l)
+ * with lazy_rank entry r > 0, mem <- M - P Q'^T over columns 0..r-1, from the
+ * fp64 factors in ws (the workspace of those lazy steps) -- the residual
+ * powersgd_step would have written, bit for bit; then every entry -> 0.
+ * mem [W][N], lazy_rank as powersgd_step_lazy.  GCE_ERR_WORKSPACE if ws_bytes
+ * is below gce_workspace_bytes(GCE_OP_POWERSGD).
  */
-GCE_API int gce_materialize_memory(const gce_table* table, int32_t W, float* mem, const float* P,
-                                   const float* Q, int32_t* lazy_rank, void* stream);
+GCE_API int gce_materialize_memory(const gce_table* table, int32_t W, float* mem,
+                                   int32_t* lazy_rank, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Data-parallel PowerSGD step ([UTIL] Key results: PowerSGD is all-reduce

@@ -55,7 +55,7 @@ class Pair:
 
     def materialize_and_compare(self):
         z = self.bufs["lazy"]
-        self.g.materialize_memory(self.t, self.W, z["mem"], z["P"], z["Q"], self.lazy_rank)
+        self.g.materialize_memory(self.t, self.W, z["mem"], self.lazy_rank, z["ws"])
         torch.cuda.synchronize()
         assert torch.equal(self.bufs["eager"]["mem"].view(torch.int32), z["mem"].view(torch.int32))
         assert not torch.any(self.lazy_rank)
@@ -119,7 +119,7 @@ def test_lazy_payload_follows_the_oracle():
             Qg = hQg[w, info["q_offset"]:info["q_offset"] + cols * cap].reshape(cols, cap)
             assert relerr(Pg, P_ref, 0.0) <= 1e-4, (s, l)
             assert relerr(Qg, hQ[(w, l)], Mn) <= 1e-4, (s, l)
-    g.materialize_memory(t, W, mem, P, Q, lazy)
+    g.materialize_memory(t, W, mem, lazy, ws)
     torch.cuda.synchronize()
     hm = host(mem)
     for l, lay in enumerate(layers):
