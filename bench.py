@@ -129,11 +129,21 @@ def measured_hbm_gbs():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def main_kernel_source_hash():
+    """sha256 of the main kernel's source text (its definition in topk.cu),
+    which is what the committed traffic capture was taken of."""
+    src = open(MAIN_SOURCE).read()
+    head = "tk_main_kernel("
+    a = src.index("__global__ void __launch_bounds__(kTkThreads) " + head)
+    b = src.index("\n}\n", a) + 3
+    return hashlib.sha256(src[a:b].encode()).hexdigest()
+
+
 def ncu_traffic_per_launch():
     """Per-launch DRAM bytes of the main kernel from the committed ncu summary,
-    or None when the kernel source changed since the capture."""
+    or None when the kernel's source changed since the capture."""
     try:
-        src_hash = hashlib.sha256(open(MAIN_SOURCE, "rb").read()).hexdigest()
+        src_hash = main_kernel_source_hash()
         fields = {}
         with open(TRAFFIC_FILE) as f:
             for line in f:

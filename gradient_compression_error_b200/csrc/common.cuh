@@ -41,6 +41,20 @@ struct alignas(16) TileInfo {
     int32_t tstart;   // first element of the tile within its layer
 };
 
+// One decode tile's fields (kDcTile outputs of one layer), so that a decoder
+// reaches them with one 48-byte load instead of tile -> layer -> record.
+struct alignas(16) DcTile {
+    int64_t out_off;  // first output element: the layer's offset + tile start
+    int64_t val_off;  // the layer's first payload slot
+    int32_t l;        // layer
+    int32_t tt;       // tile index within the layer
+    int32_t cnt;      // outputs in this tile
+    int32_t kind;
+    int32_t dc_base;  // the layer's first tile-bound slot
+    int32_t cap;
+    int32_t pad[2];
+};
+
 // A pipelined signSGD schedule uploaded for one (W, ahead): nphase runs
 // (the last a sentinel) covering nitems work items.
 struct SgPlan {
@@ -78,6 +92,7 @@ struct gce_table {
     int32_t dc_tiles = 0;                  // decode tiles over all layers
     int32_t dc_slots = 0;                  // tile-bound slots per worker (tiles + L)
     int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
+    gce::DcTile* d_dc_tiles = nullptr;     // [dc_tiles] the same tiles' fields
     int32_t dc_nl_n = 0;                   // decode tiles of sparse and DENSE layers
     int32_t* d_dc_nl_tiles = nullptr;      // their decode tile ids
     int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker

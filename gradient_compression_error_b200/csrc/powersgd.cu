@@ -27,6 +27,7 @@
 // element (read grad, read mem, write mem once); otherwise mtp and resid
 // re-read M (+8 B) and resid writes it (+4 B; +4 B for dense_out).
 #include <cmath>
+#include <type_traits>
 
 #include "common.cuh"
 #include "scan.cuh"
@@ -193,17 +194,100 @@ __global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
     }
 }
 
-// The residual of one entry: m = fl32(M - sum_j P_j Q'_j), the sum in fp64
-// (products of column 0, then fused multiply-adds in column order) from the
-// fp64 orthonormal P and fp64 Q' -- the residual pass and the lazy step's
-// first pass form it identically.
-__device__ __forceinline__ float ps_unproject(float M, const double* pr,
-                                              const double (*qd)[kPsCB], int c, int r) {
-    double mh = __dmul_rn(pr[0], qd[0][c]);
+// Precision of a layer's products.  Layers of at most kPsExactMax elements
+// form M Q, M^T P and the residual in fp64, from the fp64 orthonormal P and
+// Q' (the oracle's arithmetic up to the order of fp64 sums).  B200's CUDA
+// cores run fp64 at about 1/32 of the fp32 rate, which would make a larger,
+// bandwidth-bound layer ALU-bound; larger layers form the products in fp32
+// (per lane, from the fp32-rounded P and Q' the payload carries) and every
+// sum across lanes, chunks and row blocks in fp64.
+constexpr int64_t kPsExactMax = int64_t(1) << 22;
+
+// The residual of one entry: m = fl32(M - sum_j P_j Q'_j), the sum formed
+// as a product of column 0 then fused multiply-adds in column order -- in
+// fp64 from the fp64 factors (T = double), or in fp32 from their fp32
+// roundings, which are the P and Q the payload carries (T = float).  The
+// residual pass and the lazy step's first pass form it identically.
+template <class T>
+__device__ __forceinline__ float ps_unproject(float M, const T* pr, const T (*qd)[kPsCB], int c,
+                                              int r) {
+    if constexpr (std::is_same<T, double>::value) {
+        double mh = __dmul_rn(pr[0], qd[0][c]);
 #pragma unroll
-    for (int j = 1; j < kMaxRank; ++j)
-        if (j < r) mh = __fma_rn(pr[j], qd[j][c], mh);
-    return __double2float_rn(__dsub_rn(double(M), mh));
+        for (int j = 1; j < kMaxRank; ++j)
+            if (j < r) mh = __fma_rn(pr[j], qd[j][c], mh);
+        return __double2float_rn(__dsub_rn(double(M), mh));
+    } else {
+        float mh = __fmul_rn(pr[0], qd[0][c]);
+#pragma unroll
+        for (int j = 1; j < kMaxRank; ++j)
+            if (j < r) mh = __fmaf_rn(pr[j], qd[j][c], mh);
+        return __fsub_rn(M, mh);
+    }
+}
+
+// One row of a M Q tile (cw columns from c0 of one 16-row block): M formed,
+// optionally from the lazy residual, and written back; returns the row's
+// partial P over the columns in acc (this lane's share, fp64).  The products
+// in T (double or float); qs / qdp / pr hold the factors in T.  Full warp.
+template <bool kLazy, class T>
+__device__ __forceinline__ void ps_mq_row(const float* __restrict__ g, float* __restrict__ m,
+                                          bool vec, int cw, float eta, int r, int rp,
+                                          const T* pr, const T (*qs)[kPsCB],
+                                          const T (*qdp)[kPsCB], double* acc) {
+    const int lane = threadIdx.x & 31;
+    T a[kMaxRank] = {T(0), T(0), T(0), T(0)};
+    auto take = [&](float x, int c) {
+#pragma unroll
+        for (int j = 0; j < kMaxRank; ++j)
+            if (j < r) {
+                if constexpr (std::is_same<T, double>::value) a[j] = __fma_rn(double(x), qs[j][c], a[j]);
+                else a[j] = __fmaf_rn(x, qs[j][c], a[j]);
+            }
+    };
+    if (vec) {
+        for (int c = lane * 4; c < cw; c += 128) {
+            const float4 gg = ld_stream4(g + c);
+            float4 mm = *reinterpret_cast<const float4*>(m + c);
+            if (kLazy && rp > 0) {
+                mm.x = ps_unproject<T>(mm.x, pr, qdp, c, rp);
+                mm.y = ps_unproject<T>(mm.y, pr, qdp, c + 1, rp);
+                mm.z = ps_unproject<T>(mm.z, pr, qdp, c + 2, rp);
+                mm.w = ps_unproject<T>(mm.w, pr, qdp, c + 3, rp);
+            }
+            float4 x;
+            x.x = residual(mm.x, eta, gg.x);
+            x.y = residual(mm.y, eta, gg.y);
+            x.z = residual(mm.z, eta, gg.z);
+            x.w = residual(mm.w, eta, gg.w);
+            *reinterpret_cast<float4*>(m + c) = x;
+            take(x.x, c);
+            take(x.y, c + 1);
+            take(x.z, c + 2);
+            take(x.w, c + 3);
+        }
+    } else {
+        for (int c = lane; c < cw; c += 32) {
+            float mv = m[c];
+            if (kLazy && rp > 0) mv = ps_unproject<T>(mv, pr, qdp, c, rp);
+            const float x = residual(mv, eta, __ldcs(g + c));
+            m[c] = x;
+            take(x, c);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxRank; ++j) acc[j] = double(a[j]);
+}
+
+// Stage n entries of a rows x cap (row stride cap) factor, columns 0..rc-1,
+// into dst[j][i] as T (double from fp64, or its fp32 rounding).
+template <class T>
+__device__ __forceinline__ void ps_stage(T (*dst)[kPsCB], const double* src, int n, int rc,
+                                         int cap) {
+    for (int i = threadIdx.x; i < n * rc; i += blockDim.x) {
+        const int c = i / rc, j = i - c * rc;
+        dst[j][c] = T(src[int64_t(c) * cap + j]);
+    }
 }
 
 constexpr size_t ps_mq_smem(bool lazy) {
@@ -214,8 +298,8 @@ constexpr size_t kPsResidSmem = sizeof(double) * (kMaxRank * kPsCB + kPsRB * kMa
                                 sizeof(float) * (kMaxRank * kPsCB + kPsRB * kMaxRank);
 
 // ---- phase 1: M = m + eta*g (written back), partial P = M Q -------------------------------
-// Products and row sums in fp64 (the contraction is bandwidth-bound; fp64
-// keeps it within rounding-order distance of an fp64 reference).
+// Products in the layer's precision (kPsExactMax), sums across lanes and
+// chunks in fp64.
 // kLazy: the memory holds the previous step's M, the workspace that step's
 // fp64 orthonormal P and Q' over lazy_rank[w][l] columns (0: the memory holds
 // the residual itself); the residual m is formed on the fly, entry by entry
@@ -229,12 +313,8 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
     const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, double* __restrict__ ppart,
     int32_t* __restrict__ status, const double* __restrict__ pdw, int64_t pd_pw,
     const double* __restrict__ qdw, int32_t L_all, const int32_t* __restrict__ lazy_rank) {
-    // dynamic shared memory (ps_mq_smem bytes): the warm start Q, then (lazy)
-    // the previous Q' and the previous P rows, all fp64
+    // dynamic shared memory (ps_mq_smem bytes)
     extern __shared__ __align__(16) double ps_dyn[];
-    double (*qs)[kPsCB] = reinterpret_cast<double (*)[kPsCB]>(ps_dyn);
-    double (*qdp)[kPsCB] = qs + kMaxRank;
-    double (*prow)[kMaxRank] = reinterpret_cast<double (*)[kMaxRank]>(ps_dyn + 2 * kMaxRank * kPsCB);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
         const int w = int(u / ntiles);
@@ -255,89 +335,53 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
         const int cw = int(min64(kPsCB, C - c0));
         const int64_t r0 = int64_t(d.y) * kPsRB;
         const int rh = int(min64(kPsRB, R - r0));
+        const bool exact = L.n <= kPsExactMax;
         const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
-        for (int i = tid; i < cw * r; i += blockDim.x) {
-            const int c = i / r, j = i - c * r;
-            qs[j][c] = double(q[int64_t(c) * cap + j]);
-        }
-        if constexpr (kLazy) {
-          if (rp > 0) {
-            const double* qp = qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap;
-            for (int i = tid; i < cw * rp; i += blockDim.x) {
-                const int c = i / rp, j = i - c * rp;
-                qdp[j][c] = qp[int64_t(c) * cap + j];
+        // shared memory: the warm start Q, then (lazy) the previous Q' and
+        // the previous P rows, in the layer's precision
+        auto tile = [&](auto zero) {
+            using T = decltype(zero);
+            T (*qs)[kPsCB] = reinterpret_cast<T (*)[kPsCB]>(ps_dyn);
+            T (*qdp)[kPsCB] = qs + kMaxRank;
+            T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(qdp + kMaxRank);
+            for (int i = tid; i < cw * r; i += blockDim.x) {
+                const int c = i / r, j = i - c * r;
+                qs[j][c] = T(q[int64_t(c) * cap + j]);
             }
-            const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
-            for (int i = tid; i < rh * rp; i += blockDim.x) {
-                const int row = i / rp, j = i - row * rp;
-                prow[row][j] = p[int64_t(row) * cap + j];
-            }
-          }
-        }
-        __syncthreads();
-        for (int row = warp; row < rh; row += blockDim.x >> 5) {
-            const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
-            const float* g = grad + e;
-            float* m = mem + e;
-            double pr[kMaxRank] = {0.0, 0.0, 0.0, 0.0};
             if (kLazy && rp > 0) {
-#pragma unroll
-                for (int j = 0; j < kMaxRank; ++j) pr[j] = j < rp ? prow[row][j] : 0.0;
-            }
-            double acc[kMaxRank] = {0.0, 0.0, 0.0, 0.0};
-            if (((e & 3) == 0) && ((cw & 3) == 0)) {
-                for (int c = lane * 4; c < cw; c += 128) {
-                    const float4 gg = ld_stream4(g + c);
-                    float4 mm = *reinterpret_cast<const float4*>(m + c);
-                    if constexpr (kLazy) {
-                        if (rp > 0) {
-                            mm.x = ps_unproject(mm.x, pr, qdp, c, rp);
-                            mm.y = ps_unproject(mm.y, pr, qdp, c + 1, rp);
-                            mm.z = ps_unproject(mm.z, pr, qdp, c + 2, rp);
-                            mm.w = ps_unproject(mm.w, pr, qdp, c + 3, rp);
-                        }
-                    }
-                    float4 x;
-                    x.x = residual(mm.x, eta, gg.x);
-                    x.y = residual(mm.y, eta, gg.y);
-                    x.z = residual(mm.z, eta, gg.z);
-                    x.w = residual(mm.w, eta, gg.w);
-                    *reinterpret_cast<float4*>(m + c) = x;
-#pragma unroll
-                    for (int j = 0; j < kMaxRank; ++j) {
-                        if (j < r) {
-                            acc[j] = __fma_rn(double(x.x), qs[j][c], acc[j]);
-                            acc[j] = __fma_rn(double(x.y), qs[j][c + 1], acc[j]);
-                            acc[j] = __fma_rn(double(x.z), qs[j][c + 2], acc[j]);
-                            acc[j] = __fma_rn(double(x.w), qs[j][c + 3], acc[j]);
-                        }
-                    }
-                }
-            } else {
-                for (int c = lane; c < cw; c += 32) {
-                    float mv = m[c];
-                    if constexpr (kLazy) {
-                        if (rp > 0) mv = ps_unproject(mv, pr, qdp, c, rp);
-                    }
-                    const float x = residual(mv, eta, __ldcs(g + c));
-                    m[c] = x;
-#pragma unroll
-                    for (int j = 0; j < kMaxRank; ++j)
-                        if (j < r) acc[j] = __fma_rn(double(x), qs[j][c], acc[j]);
+                ps_stage<T>(qdp, qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap, cw, rp, cap);
+                const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
+                for (int i = tid; i < rh * rp; i += blockDim.x) {
+                    const int row = i / rp, j = i - row * rp;
+                    prow[row][j] = T(p[int64_t(row) * cap + j]);
                 }
             }
-            // a NaN or infinite M makes its row's products non-finite
-            flag_nonfinite(!(fabs(acc[0]) <= 1.0e300), status);
+            __syncthreads();
+            for (int row = warp; row < rh; row += blockDim.x >> 5) {
+                const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
+                T pr[kMaxRank] = {T(0), T(0), T(0), T(0)};
+                if (kLazy && rp > 0) {
 #pragma unroll
-            for (int j = 0; j < kMaxRank; ++j) acc[j] = warp_sum(acc[j]);
-            if (lane < r) {
-                double a = acc[0];
-                if (lane == 1) a = acc[1];
-                if (lane == 2) a = acc[2];
-                if (lane == 3) a = acc[3];
-                ppart[int64_t(w) * ppart_pw + X.ppart_off + (int64_t(d.z) * R + r0 + row) * cap + lane] = a;
+                    for (int j = 0; j < kMaxRank; ++j) pr[j] = j < rp ? prow[row][j] : T(0);
+                }
+                double acc[kMaxRank];
+                ps_mq_row<kLazy, T>(grad + e, mem + e, ((e & 3) == 0) && ((cw & 3) == 0), cw, eta,
+                                    r, rp, pr, qs, qdp, acc);
+                // a NaN or infinite M makes its row's products non-finite
+                flag_nonfinite(!(fabs(acc[0]) <= 1.0e300), status);
+#pragma unroll
+                for (int j = 0; j < kMaxRank; ++j) acc[j] = warp_sum(acc[j]);
+                if (lane < r) {
+                    double a = acc[0];
+                    if (lane == 1) a = acc[1];
+                    if (lane == 2) a = acc[2];
+                    if (lane == 3) a = acc[3];
+                    ppart[int64_t(w) * ppart_pw + X.ppart_off + (int64_t(d.z) * R + r0 + row) * cap + lane] = a;
+                }
             }
-        }
+        };
+        if (exact) tile(0.0);
+        else tile(0.0f);
         __syncthreads();
     }
 }
@@ -546,13 +590,15 @@ static std::vector<PsOrthOp> ps_orth_ops(int cap) {
 }
 
 // ---- phase 3: partial Q = M^T P over 64-row blocks ---------------------------------------
-// From the fp64 orthonormal P (the workspace copy), products and sums in fp64.
+// From the orthonormal P of the workspace: products in the layer's
+// precision (fp64, or fp32 from the P the payload carries), the partial of
+// each 64-row block stored in fp64.
 __global__ void __launch_bounds__(256) ps_mtp_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t pd_pw,
     int64_t qpart_pw, const float* __restrict__ mem, const int32_t* __restrict__ k_or_rank,
     const double* __restrict__ pdw, double* __restrict__ qpart) {
-    __shared__ double prow[kPsRB3][kMaxRank];
+    __shared__ double prow_d[kPsRB3][kMaxRank];
     const int tid = threadIdx.x;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
         const int w = int(u / ntiles);
@@ -568,44 +614,55 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
         const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
-        for (int i = tid; i < rh * kMaxRank; i += blockDim.x) {
-            const int row = i / kMaxRank, j = i % kMaxRank;
-            prow[row][j] = j < r ? p[int64_t(row) * cap + j] : 0.0;
-        }
-        __syncthreads();
         const int cc = tid * 4;
-        double acc[4][kMaxRank];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int j = 0; j < kMaxRank; ++j) acc[q][j] = 0.0;
         const int64_t ebase = int64_t(w) * N + L.offset + r0 * C + c0;
         const bool vec = ((ebase & 3) == 0) && ((C & 3) == 0) && (cc + 3 < cw);
-        if (cc < cw) {
-            for (int row = 0; row < rh; ++row) {
-                const float* m = mem + ebase + int64_t(row) * C + cc;
-                float x[4];
-                if (vec) {
-                    const float4 mm = *reinterpret_cast<const float4*>(m);
-                    x[0] = mm.x; x[1] = mm.y; x[2] = mm.z; x[3] = mm.w;
-                } else {
+        double* out = qpart + int64_t(w) * qpart_pw + X.qpart_off + (int64_t(d.y) * C + c0 + cc) * cap;
+        auto tile = [&](auto zero) {
+            using T = decltype(zero);
+            T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(&prow_d[0][0]);
+            for (int i = tid; i < rh * kMaxRank; i += blockDim.x) {
+                const int row = i / kMaxRank, j = i % kMaxRank;
+                prow[row][j] = j < r ? T(p[int64_t(row) * cap + j]) : T(0);
+            }
+            __syncthreads();
+            T acc[4][kMaxRank];
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) x[q] = (cc + q < cw) ? m[q] : 0.0f;
+            for (int q = 0; q < 4; ++q)
+#pragma unroll
+                for (int j = 0; j < kMaxRank; ++j) acc[q][j] = T(0);
+            if (cc < cw) {
+                for (int row = 0; row < rh; ++row) {
+                    const float* m = mem + ebase + int64_t(row) * C + cc;
+                    float x[4];
+                    if (vec) {
+                        const float4 mm = *reinterpret_cast<const float4*>(m);
+                        x[0] = mm.x; x[1] = mm.y; x[2] = mm.z; x[3] = mm.w;
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) x[q] = (cc + q < cw) ? m[q] : 0.0f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+#pragma unroll
+                        for (int j = 0; j < kMaxRank; ++j)
+                            if (j < r) {
+                                if constexpr (std::is_same<T, double>::value)
+                                    acc[q][j] = __fma_rn(double(x[q]), prow[row][j], acc[q][j]);
+                                else
+                                    acc[q][j] = __fmaf_rn(x[q], prow[row][j], acc[q][j]);
+                            }
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
+                    if (cc + q < cw)
 #pragma unroll
-                    for (int j = 0; j < kMaxRank; ++j)
-                        if (j < r) acc[q][j] = __fma_rn(double(x[q]), prow[row][j], acc[q][j]);
+                        for (int j = 0; j < kMaxRank; ++j)
+                            if (j < r) out[q * cap + j] = double(acc[q][j]);
             }
-            double* out = qpart + int64_t(w) * qpart_pw + X.qpart_off + (int64_t(d.y) * C + c0 + cc) * cap;
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (cc + q < cw)
-#pragma unroll
-                    for (int j = 0; j < kMaxRank; ++j)
-                        if (j < r) out[q * cap + j] = acc[q][j];
-        }
+        };
+        if (L.n <= kPsExactMax) tile(0.0);
+        else tile(0.0f);
         __syncthreads();
     }
 }
@@ -679,9 +736,10 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
 }
 
 // ---- residual: m <- M - P Q^T, dense_out <- P Q^T ---------------------------------------------
-// The memory from the fp64 factors (ps_unproject); dense_out from the fp32
-// P and Q the payload carries, formed as the decoder forms it (product, then
-// fp32 fused multiply-adds in column order), so dense_out is the decode.
+// The memory from the workspace's factors in the layer's precision
+// (ps_unproject); dense_out from the fp32 P and Q the payload carries, formed
+// as the decoder forms it (product, then fp32 fused multiply-adds in column
+// order), so dense_out is the decode.
 // rank_wl (nullable): per (worker, layer) ranks [W][L_all] instead of
 // k_or_rank -- the lazy step's record, for gce_materialize_memory.
 __global__ void __launch_bounds__(256) ps_resid_kernel(
@@ -693,8 +751,6 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
     const int32_t* __restrict__ rank_wl, int32_t L_all) {
     // dynamic shared memory (kPsResidSmem bytes)
     extern __shared__ __align__(16) double ps_dyn[];
-    double (*qd)[kPsCB] = reinterpret_cast<double (*)[kPsCB]>(ps_dyn);
-    double (*prow)[kMaxRank] = reinterpret_cast<double (*)[kMaxRank]>(ps_dyn + kMaxRank * kPsCB);
     float (*qs)[kPsCB] =
         reinterpret_cast<float (*)[kPsCB]>(ps_dyn + kMaxRank * kPsCB + kPsRB * kMaxRank);
     float (*prow32)[kMaxRank] = reinterpret_cast<float (*)[kMaxRank]>(
@@ -719,16 +775,6 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
         const int cw = int(min64(kPsCB, C - c0));
         const int64_t r0 = int64_t(d.y) * kPsRB;
         const int rh = int(min64(kPsRB, R - r0));
-        const double* qp = qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap;
-        for (int i = tid; i < cw * r; i += blockDim.x) {
-            const int c = i / r, j = i - c * r;
-            qd[j][c] = qp[int64_t(c) * cap + j];
-        }
-        const double* pp = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
-        for (int i = tid; i < rh * r; i += blockDim.x) {
-            const int row = i / r, j = i - row * r;
-            prow[row][j] = pp[int64_t(row) * cap + j];
-        }
         if (dense_out) {
             const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
             for (int i = tid; i < cw * r; i += blockDim.x) {
@@ -741,44 +787,58 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
                 prow32[row][j] = p[int64_t(row) * cap + j];
             }
         }
-        __syncthreads();
-        for (int row = warp; row < rh; row += blockDim.x >> 5) {
-            const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
-            float* m = mem + e;
-            float* o = dense_out ? dense_out + e : nullptr;
-            double pr[kMaxRank];
-            float pr32[kMaxRank];
-#pragma unroll
-            for (int j = 0; j < kMaxRank; ++j) {
-                pr[j] = j < r ? prow[row][j] : 0.0;
-                pr32[j] = (o && j < r) ? prow32[row][j] : 0.0f;
+        auto tile = [&](auto zero) {
+            using T = decltype(zero);
+            T (*qd)[kPsCB] = reinterpret_cast<T (*)[kPsCB]>(ps_dyn);
+            T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(ps_dyn + kMaxRank * kPsCB);
+            ps_stage<T>(qd, qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap, cw, r, cap);
+            const double* pp = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
+            for (int i = tid; i < rh * r; i += blockDim.x) {
+                const int row = i / r, j = i - row * r;
+                prow[row][j] = T(pp[int64_t(row) * cap + j]);
             }
-            auto decoded = [&](int c) {
-                float mh = __fmul_rn(pr32[0], qs[0][c]);
+            __syncthreads();
+            for (int row = warp; row < rh; row += blockDim.x >> 5) {
+                const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
+                float* m = mem + e;
+                float* o = dense_out ? dense_out + e : nullptr;
+                T pr[kMaxRank];
+                float pr32[kMaxRank];
 #pragma unroll
-                for (int j = 1; j < kMaxRank; ++j)
-                    if (j < r) mh = __fmaf_rn(pr32[j], qs[j][c], mh);
-                return mh;
-            };
-            if (((e & 3) == 0) && ((cw & 3) == 0)) {  // 16-byte rows: four columns a lane
-                for (int c = lane * 4; c < cw; c += 128) {
-                    float4 mm = *reinterpret_cast<const float4*>(m + c);
-                    mm.x = ps_unproject(mm.x, pr, qd, c, r);
-                    mm.y = ps_unproject(mm.y, pr, qd, c + 1, r);
-                    mm.z = ps_unproject(mm.z, pr, qd, c + 2, r);
-                    mm.w = ps_unproject(mm.w, pr, qd, c + 3, r);
-                    __stcs(reinterpret_cast<float4*>(m + c), mm);
-                    if (o)
-                        __stcs(reinterpret_cast<float4*>(o + c),
-                               make_float4(decoded(c), decoded(c + 1), decoded(c + 2), decoded(c + 3)));
+                for (int j = 0; j < kMaxRank; ++j) {
+                    pr[j] = j < r ? prow[row][j] : T(0);
+                    pr32[j] = (o && j < r) ? prow32[row][j] : 0.0f;
                 }
-            } else {
-                for (int c = lane; c < cw; c += 32) {
-                    m[c] = ps_unproject(m[c], pr, qd, c, r);
-                    if (o) o[c] = decoded(c);
+                auto decoded = [&](int c) {
+                    float mh = __fmul_rn(pr32[0], qs[0][c]);
+#pragma unroll
+                    for (int j = 1; j < kMaxRank; ++j)
+                        if (j < r) mh = __fmaf_rn(pr32[j], qs[j][c], mh);
+                    return mh;
+                };
+                if (((e & 3) == 0) && ((cw & 3) == 0)) {  // 16-byte rows: four columns a lane
+                    for (int c = lane * 4; c < cw; c += 128) {
+                        float4 mm = *reinterpret_cast<const float4*>(m + c);
+                        mm.x = ps_unproject<T>(mm.x, pr, qd, c, r);
+                        mm.y = ps_unproject<T>(mm.y, pr, qd, c + 1, r);
+                        mm.z = ps_unproject<T>(mm.z, pr, qd, c + 2, r);
+                        mm.w = ps_unproject<T>(mm.w, pr, qd, c + 3, r);
+                        __stcs(reinterpret_cast<float4*>(m + c), mm);
+                        if (o)
+                            __stcs(reinterpret_cast<float4*>(o + c),
+                                   make_float4(decoded(c), decoded(c + 1), decoded(c + 2),
+                                               decoded(c + 3)));
+                    }
+                } else {
+                    for (int c = lane; c < cw; c += 32) {
+                        m[c] = ps_unproject<T>(m[c], pr, qd, c, r);
+                        if (o) o[c] = decoded(c);
+                    }
                 }
             }
-        }
+        };
+        if (L.n <= kPsExactMax) tile(0.0);
+        else tile(0.0f);
         __syncthreads();
     }
 }

@@ -164,6 +164,7 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_dtile_layer);
     cudaFree(t->d_dtile_start);
     cudaFree(t->d_dc_tile_layer);
+    cudaFree(t->d_dc_tiles);
     cudaFree(t->d_dc_nl_tiles);
     cudaFree(t->d_bunit_layer);
     cudaFree(t->d_bunit_chunk);
@@ -193,6 +194,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     std::vector<int32_t> tile_layer, sunit_layer, sunit_part, dtile_layer, dtile_start;
     std::vector<TileInfo> tile_info;
     std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_nl;
+    std::vector<DcTile> dc_tile_info;
     int32_t dc_tiles = 0, dc_slots = 0;
     for (int32_t l = 0; l < L; ++l) {
         const gce_layer_desc& d = descs[l];
@@ -268,6 +270,17 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
         for (int32_t i = 0; i < x.dc_ntiles; ++i) {
             if (d.kind != GCE_KIND_POWERSGD) dc_nl.push_back(dc_tiles + i);
             dc_tile_layer.push_back(l);
+            const int64_t start = int64_t(i) << kDcTileLog;
+            DcTile dt{};
+            dt.out_off = x.offset + start;
+            dt.val_off = x.val_off;
+            dt.l = l;
+            dt.tt = i;
+            dt.cnt = int32_t(std::min<int64_t>(kDcTile, n - start));
+            dt.kind = d.kind;
+            dt.dc_base = x.dc_base;
+            dt.cap = d.cap;
+            dc_tile_info.push_back(dt);
         }
         dc_tiles += x.dc_ntiles;
         dc_slots += x.dc_ntiles + 1;
@@ -320,6 +333,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_dtile_layer, dtile_layer);
     if (rc == GCE_OK) rc = upload(&t->d_dtile_start, dtile_start);
     if (rc == GCE_OK) rc = upload(&t->d_dc_tile_layer, dc_tile_layer);
+    if (rc == GCE_OK) rc = upload(&t->d_dc_tiles, dc_tile_info);
     t->dc_nl_n = int32_t(dc_nl.size());
     if (rc == GCE_OK) rc = upload(&t->d_dc_nl_tiles, dc_nl);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_layer, bunit_layer);

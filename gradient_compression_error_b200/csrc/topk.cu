@@ -179,10 +179,9 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
                 ok[q] = e < ne && pos < L.n;
                 vv[q] = ok[q] ? residual(m[pos], eta, __ldcs(g + pos)) : 0.0f;
             }
-            // most samples fall in a few bins near the bulk of |v|: one
-            // shared-memory atomic per distinct bin of the warp
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) hist_add(h, abs_key(vv[q]) >> 19, ok[q]);
+            for (int q = 0; q < kBatch; ++q)
+                if (ok[q]) atomicAdd(&h[abs_key(vv[q]) >> 19], 1);
         }
         __syncthreads();
         int32_t* gh = tk_hist(hists, S, 0, seg);
@@ -614,23 +613,27 @@ __device__ __forceinline__ void tk_hist_unit(int32_t u, const DevLayer* __restri
 }
 
 // One emit item: up to kTkGroup consecutive main tiles of one (worker, layer),
-// a warp per tile.  Counts keys > T and == T per tile, takes the segment's
-// running counts before the item (look-back), then writes the chosen (v, i)
-// in index order, memory +0 for chosen entries at or below hi and v again for
-// entries above hi that were not chosen.  Whole block.
+// kTkWarpTiles consecutive tiles per warp.  Counts keys > T and == T per tile,
+// takes the segment's running counts before the item (look-back), then writes
+// the chosen (v, i) in index order, memory +0 for chosen entries at or below
+// hi and v again for entries above hi that were not chosen.  Whole block.
+constexpr int kTkSelThreads = 128;
+constexpr int kTkWarpTiles = kTkGroup / (kTkSelThreads / 32);  // 2
+
 __device__ __forceinline__ void tk_emit_item(
     int64_t e, int32_t W, int32_t ncomp, int32_t tiles_pw, int64_t N, int64_t comp_N,
     int64_t vals_pw, const TileInfo* __restrict__ tile_info, const int2* __restrict__ groups,
     TkSeg* segs, const int2* __restrict__ tile_dir, const float* __restrict__ spill_v,
     const int32_t* __restrict__ spill_i, uint64_t* gstate, float* __restrict__ mem,
     float* __restrict__ vals, int32_t* __restrict__ idx, int32_t* status, TkSelShared& sh) {
-    constexpr int kBatch = 8;
+    constexpr int kBatch = 4;  // candidates per lane per tile in flight
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lt_mask = (1u << lane) - 1u;
     const int64_t gi = e / W;
     const int w = int(e - gi * W);
     const int2 gr = groups[gi];
-    const int64_t s = int64_t(w) * ncomp + tile_info[gr.x].sidx;
+    const TileInfo ti0 = tile_info[gr.x];
+    const int64_t s = int64_t(w) * ncomp + ti0.sidx;
     if (tid == 0) {
         sh.k = segs[s].k;
         sh.ok = sh.k > 0 && tk_wait_level(&segs[s].level, 3, status);
@@ -642,40 +645,43 @@ __device__ __forceinline__ void tk_emit_item(
         // after the fallback the memory holds v everywhere (nothing was zeroed)
         sh.hi = segs[s].redo ? 0xFFFFFFFFu : segs[s].hi;
     }
+    // this warp's tiles and their candidate ranges, loaded while thread 0 waits
+    int2 d[kTkWarpTiles];
+    int64_t sb[kTkWarpTiles];
+#pragma unroll
+    for (int i = 0; i < kTkWarpTiles; ++i) {
+        const int slot = warp * kTkWarpTiles + i;
+        d[i] = make_int2(0, 0);
+        if (slot < gr.y) d[i] = tile_dir[int64_t(w) * tiles_pw + gr.x + slot];
+        sb[i] = int64_t(w) * comp_N + ti0.sp_off + d[i].x;  // one layer: one candidate region
+    }
     __syncthreads();
     if (!sh.ok) return;
     const uint32_t T = sh.T;
     const int32_t k = sh.k, need = sh.need;
-    const bool mine = warp < gr.y;
-    const int lt = gr.x + warp;
-    const int64_t t = int64_t(w) * tiles_pw + lt;
-    TileInfo ti{};
-    int2 d = make_int2(0, 0);
-    if (mine) {
-        ti = tile_info[lt];
-        d = tile_dir[t];
-    }
-    const int64_t sb = int64_t(w) * comp_N + ti.sp_off + d.x;
-    // counts of this warp's tile
-    int gt = 0, eq = 0;
-    for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
-        uint32_t key[kBatch];
+    // counts of this warp's tiles
 #pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int j = j0 + q * 32 + lane;
-            key[q] = j < d.y ? abs_key(__ldcg(spill_v + sb + j)) : 0xFFFFFFFFu;
-        }
+    for (int i = 0; i < kTkWarpTiles; ++i) {
+        int gt = 0, eq = 0;
+        for (int j0 = 0; j0 < d[i].y; j0 += 32 * kBatch) {
+            uint32_t key[kBatch];
 #pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            gt += key[q] != 0xFFFFFFFFu && key[q] > T;
-            eq += key[q] == T;
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * 32 + lane;
+                key[q] = j < d[i].y ? abs_key(__ldcg(spill_v + sb[i] + j)) : 0xFFFFFFFFu;
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                gt += key[q] != 0xFFFFFFFFu && key[q] > T;
+                eq += key[q] == T;
+            }
         }
-    }
-    gt = warp_sum(gt);
-    eq = warp_sum(eq);
-    if (lane == 0) {
-        sh.cnt_gt[warp] = gt;
-        sh.cnt_eq[warp] = eq;
+        gt = warp_sum(gt);
+        eq = warp_sum(eq);
+        if (lane == 0) {
+            sh.cnt_gt[warp * kTkWarpTiles + i] = gt;
+            sh.cnt_eq[warp * kTkWarpTiles + i] = eq;
+        }
     }
     __syncthreads();
     if (warp == 0) {
@@ -685,7 +691,7 @@ __device__ __forceinline__ void tk_emit_item(
             geq += sh.cnt_eq[i];
         }
         // items of the layer before this one (its first item has none)
-        const int64_t before = int64_t(tile_info[gr.x].tstart / kTkTile) / kTkGroup;
+        const int64_t before = int64_t(ti0.tstart / kTkTile) / kTkGroup;
         if (lane == 0) st_release_gpu_u64(gstate + e, (before ? kTkAgg : kTkInc) | tk_pack(ggt, geq));
         // look back a warp at a time: lane i reads the item i + 1 back (W
         // entries apart), until one has published its running counts
@@ -727,51 +733,54 @@ __device__ __forceinline__ void tk_emit_item(
         }
     }
     __syncthreads();
-    if (!mine) return;
     const uint32_t hi = sh.hi;
-    int sel_before = sh.base_gt[warp] + min(sh.base_eq[warp], need);
-    int eq_seen = sh.base_eq[warp];
-    float* vout = vals + int64_t(w) * vals_pw + ti.val_off;
-    int32_t* iout = idx + int64_t(w) * vals_pw + ti.val_off;
-    float* m = mem + int64_t(w) * N + ti.offset;
-    for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
-        float ev[kBatch];
-        int32_t ei[kBatch];
+    float* vout = vals + int64_t(w) * vals_pw + ti0.val_off;
+    int32_t* iout = idx + int64_t(w) * vals_pw + ti0.val_off;
+    float* m = mem + int64_t(w) * N + ti0.offset;
 #pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            const int j = j0 + q * 32 + lane;
-            ev[q] = 0.0f;
-            ei[q] = -1;
-            if (j < d.y) {
-                ev[q] = __ldcg(spill_v + sb + j);
-                ei[q] = __ldcg(spill_i + sb + j);
-            }
-        }
+    for (int i = 0; i < kTkWarpTiles; ++i) {
+        const int slot = warp * kTkWarpTiles + i;
+        int sel_before = sh.base_gt[slot] + min(sh.base_eq[slot], need);
+        int eq_seen = sh.base_eq[slot];
+        for (int j0 = 0; j0 < d[i].y; j0 += 32 * kBatch) {
+            float ev[kBatch];
+            int32_t ei[kBatch];
 #pragma unroll
-        for (int q = 0; q < kBatch; ++q) {
-            if (j0 + q * 32 >= d.y) break;  // the warp's remaining slots are empty
-            const bool valid = ei[q] >= 0;
-            const uint32_t key = abs_key(ev[q]);
-            const bool is_eq = valid && key == T;
-            const unsigned eq_mask = __ballot_sync(kFull, is_eq);
-            const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
-            const bool sel = valid && (key > T || (is_eq && eq_rank < need));
-            const unsigned sel_mask = __ballot_sync(kFull, sel);
-            const int pos = sel_before + __popc(sel_mask & lt_mask);
-            if (sel && pos < k) {
-                vout[pos] = ev[q];
-                iout[pos] = ei[q];
-                if (key <= hi) m[ei[q]] = 0.0f;
-            } else if (valid && !sel && key > hi) {
-                m[ei[q]] = ev[q];  // zeroed in the main pass but not chosen
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * 32 + lane;
+                ev[q] = 0.0f;
+                ei[q] = -1;
+                if (j < d[i].y) {
+                    ev[q] = __ldcg(spill_v + sb[i] + j);
+                    ei[q] = __ldcg(spill_i + sb[i] + j);
+                }
             }
-            sel_before += __popc(sel_mask);
-            eq_seen += __popc(eq_mask);
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                if (j0 + q * 32 >= d[i].y) break;  // the warp's remaining slots are empty
+                const bool valid = ei[q] >= 0;
+                const uint32_t key = abs_key(ev[q]);
+                const bool is_eq = valid && key == T;
+                const unsigned eq_mask = __ballot_sync(kFull, is_eq);
+                const int eq_rank = eq_seen + __popc(eq_mask & lt_mask);
+                const bool sel = valid && (key > T || (is_eq && eq_rank < need));
+                const unsigned sel_mask = __ballot_sync(kFull, sel);
+                const int pos = sel_before + __popc(sel_mask & lt_mask);
+                if (sel && pos < k) {
+                    vout[pos] = ev[q];
+                    iout[pos] = ei[q];
+                    if (key <= hi) m[ei[q]] = 0.0f;
+                } else if (valid && !sel && key > hi) {
+                    m[ei[q]] = ev[q];  // zeroed in the main pass but not chosen
+                }
+                sel_before += __popc(sel_mask);
+                eq_seen += __popc(eq_mask);
+            }
         }
     }
 }
 
-__global__ void __launch_bounds__(256, 5) tk_select_kernel(
+__global__ void __launch_bounds__(kTkSelThreads) tk_select_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ comp, int32_t ncomp,
     int64_t S, int32_t W, int32_t tiles_pw, int64_t N, int64_t comp_N, int64_t vals_pw,
     const TileInfo* __restrict__ tile_info, const int2* __restrict__ groups, int32_t groups_pw,
@@ -783,8 +792,16 @@ __global__ void __launch_bounds__(256, 5) tk_select_kernel(
     __shared__ TkSelShared sh;
     const int64_t U = unit_start[S];
     const int64_t nitems = 3 * U + int64_t(groups_pw) * W;
+    // thread 0 takes the next item while the block works on the current one
+    // (a block holds at most one item it has not started, taken after every
+    // item it has finished, so the earliest unfinished item is always running)
+    uint32_t next = 0;
+    if (threadIdx.x == 0) next = atomicAdd(counter, 1u);
     for (;;) {
-        if (threadIdx.x == 0) sh.item = int64_t(atomicAdd(counter, 1u));
+        if (threadIdx.x == 0) {
+            sh.item = int64_t(next);
+            if (int64_t(next) < nitems) next = atomicAdd(counter, 1u);
+        }
         __syncthreads();
         const int64_t it = sh.item;
         if (it >= nitems) break;
@@ -841,7 +858,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         static const int r_main = resident_blocks(tk_main_kernel, kTkThreads);
         static const int r_restore = resident_blocks(tk_restore_kernel, 256);
         static const int r_respill = resident_blocks(tk_respill_kernel, 256);
-        static const int r_select = resident_blocks(tk_select_kernel, 256);
+        static const int r_select = resident_blocks(tk_select_kernel, kTkSelThreads);
         GCE_LAUNCH(tk_setup_kernel, wave_grid((n4 + lay.S + 255) / 256, 8, r_setup), 256, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, k_or_rank, segs, reinterpret_cast<int4*>(hists), n4,
                    status);
@@ -862,7 +879,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
                    t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, mem, spill_v,
                    spill_i);
         // every resident block takes items until none are left
-        GCE_LAUNCH(tk_select_kernel, wave_grid(lay.TT + lay.S, r_select, r_select), 256, 0, st,
+        GCE_LAUNCH(tk_select_kernel, wave_grid(lay.TT + lay.S, r_select, r_select), kTkSelThreads, 0, st,
                    t->d_layers, t->d_comp, ncomp, lay.S, W, t->tiles_pw, t->N, t->comp_N,
                    t->vals_pw, t->d_tile_info, t->d_tk_groups, t->tk_groups_pw, segs, unit_start,
                    unit_seg, hists, tile_dir, spill_v, spill_i, at<uint64_t>(ws, lay.gstate),

@@ -38,6 +38,9 @@ def lib():
             "or_powersgd": (C.c_int, [i64, i64, i64, i64, f32, vp, vp, vp, vp, vp]),
             "or_powersgd_dp": (C.c_int, [i64, i64, i64, i64, i64, f32, vp, vp, vp, vp]),
             "or_dense_dp": (C.c_int, [i64, i64, f32, vp, vp, vp]),
+            "or_powersgd_dp_p": (C.c_int, [i64, i64, i64, i64, f32, vp, vp, vp, vp]),
+            "or_mgs": (None, [i64, i64, vp]),
+            "or_powersgd_dp_q": (C.c_int, [i64, i64, i64, vp, vp, vp]),
             "or_ef_sign": (C.c_int, [i64, f32, vp, vp, vp, vp]),
             "or_accum_sign": (None, [i64, f32, vp, vp]),
             "or_vote_sign": (None, [i64, i64, i64, vp, f32, vp]),
@@ -169,6 +172,38 @@ def powersgd_dp_unit(g, m, Q, r, eta):
     _check(lib().or_powersgd_dp(W, rows, cols, int(r), r_max, float(np.float32(eta)), _ptr(g),
                                 _ptr(m), _ptr(Q), _ptr(P)), "powersgd_dp")
     return P, Q, m
+
+
+def powersgd_dp_p_unit(g, m, Q, r, eta):
+    """Phase 1 of the data-parallel step for one worker's matrix: returns
+    (M_w (rows, cols) float32, P_w = M_w Q (rows, r) float64)."""
+    g = _f32(g)
+    rows, cols = g.shape
+    m = _f32(m).copy()
+    Q = _f32(Q)
+    Pw = np.zeros((rows, int(r)), np.float64)
+    _check(lib().or_powersgd_dp_p(rows, cols, int(r), Q.shape[1], float(np.float32(eta)),
+                                  _ptr(g), _ptr(m), _ptr(Q), _ptr(Pw)), "powersgd_dp_p")
+    return m, Pw
+
+
+def mgs(P):
+    """Modified Gram-Schmidt of the columns of P (rows, r) float64, in order."""
+    P = np.ascontiguousarray(P, np.float64).copy()
+    lib().or_mgs(P.shape[0], P.shape[1], _ptr(P))
+    return P
+
+
+def powersgd_dp_q_unit(Pd, M):
+    """Phase 2 for one worker: (Q_w = M^T P (cols, r) float64, residual
+    M - P Q_w^T (rows, cols) float32)."""
+    Pd = np.ascontiguousarray(Pd, np.float64)
+    m = _f32(M).copy()
+    rows, cols = m.shape
+    Qw = np.zeros((cols, Pd.shape[1]), np.float64)
+    _check(lib().or_powersgd_dp_q(rows, cols, Pd.shape[1], _ptr(Pd), _ptr(m), _ptr(Qw)),
+           "powersgd_dp_q")
+    return Qw, m
 
 
 def dense_dp_unit(g, m, eta):

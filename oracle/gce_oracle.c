@@ -365,33 +365,32 @@ int or_powersgd(int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
  * Arithmetic after the M_w are formed runs in double; P, Q and m are stored
  * as fp32.
  */
-int or_powersgd_dp(int64_t W, int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
-                   const float* g, float* m, float* Q, float* P)
+/* The data-parallel step in the order its two all-reduces cut it into:
+ *   phase 1, each worker:  M_w = m_w + eta*grad_w (stored back in m_w, exact
+ *                          in fp32), P_w = M_w Q  (fp64, rows x r);
+ *   all-reduce:            P = sum_w P_w  (fp64, worker order from 0);
+ *   orthonormalise P       (modified Gram-Schmidt, as or_powersgd);
+ *   phase 2, each worker:  Q_w = M_w^T P (fp64), m_w = M_w - P Q_w^T;
+ *   all-reduce:            Q = (float)(sum_w Q_w / W)  (fp64, worker order). */
+int or_powersgd_dp_p(int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
+                     const float* g, float* m, const float* Q, double* Pw)
 {
-    if (W < 1 || rows < 1 || cols < 1 || r < 1 || r > r_max || r > rows || r > cols)
-        return OR_ERR_ARG;
+    if (rows < 1 || cols < 1 || r < 1 || r > r_max || r > rows || r > cols) return OR_ERR_ARG;
     int64_t n = rows * cols;
-    double* M = (double*)malloc((size_t)(W * n) * sizeof(double));
-    double* Pd = (double*)calloc((size_t)(rows * r), sizeof(double));
-    double* Qw = (double*)malloc((size_t)(cols * r) * sizeof(double));
-    double* Qsum = (double*)calloc((size_t)(cols * r), sizeof(double));
-    if (!M || !Pd || !Qw || !Qsum) { free(M); free(Pd); free(Qw); free(Qsum); return OR_ERR_NOMEM; }
+    for (int64_t i = 0; i < n; ++i) m[i] = or_residual(m[i], eta, g[i]);
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t j = 0; j < r; ++j) {
+            double s = 0.0;
+            for (int64_t c = 0; c < cols; ++c) s += (double)m[a * cols + c] * (double)Q[c * r_max + j];
+            Pw[a * r + j] = s;
+        }
+    return OR_OK;
+}
 
-    for (int64_t w = 0; w < W; ++w)
-        for (int64_t i = 0; i < n; ++i)
-            M[w * n + i] = (double)or_residual(m[w * n + i], eta, g[w * n + i]);
-
-    /* P = sum over workers of M_w Q */
-    for (int64_t w = 0; w < W; ++w)
-        for (int64_t a = 0; a < rows; ++a)
-            for (int64_t j = 0; j < r; ++j) {
-                double s = 0.0;
-                for (int64_t c = 0; c < cols; ++c)
-                    s += M[w * n + a * cols + c] * (double)Q[c * r_max + j];
-                Pd[a * r + j] += s;
-            }
-
-    /* modified Gram-Schmidt over the columns of P, in order 0..r-1 */
+/* Modified Gram-Schmidt over the r columns of P (rows x r, fp64) in place,
+ * in column order; a zero column stays zero. */
+void or_mgs(int64_t rows, int64_t r, double* Pd)
+{
     for (int64_t j = 0; j < r; ++j) {
         for (int64_t i = 0; i < j; ++i) {
             double d = 0.0;
@@ -403,23 +402,52 @@ int or_powersgd_dp(int64_t W, int64_t rows, int64_t cols, int64_t r, int64_t r_m
         double nu = sqrt(nn);
         for (int64_t a = 0; a < rows; ++a) Pd[a * r + j] = nu > 0.0 ? Pd[a * r + j] / nu : 0.0;
     }
+}
+
+/* phase 2 of one worker: m holds M_w on entry and the residual on return;
+ * Qw (cols x r, fp64) receives M_w^T P. */
+int or_powersgd_dp_q(int64_t rows, int64_t cols, int64_t r, const double* Pd, float* m,
+                     double* Qw)
+{
+    if (rows < 1 || cols < 1 || r < 1 || r > rows || r > cols) return OR_ERR_ARG;
+    for (int64_t c = 0; c < cols; ++c)
+        for (int64_t j = 0; j < r; ++j) {
+            double s = 0.0;
+            for (int64_t a = 0; a < rows; ++a) s += (double)m[a * cols + c] * Pd[a * r + j];
+            Qw[c * r + j] = s;
+        }
+    for (int64_t a = 0; a < rows; ++a)
+        for (int64_t c = 0; c < cols; ++c) {
+            double s = 0.0;
+            for (int64_t j = 0; j < r; ++j) s += Pd[a * r + j] * Qw[c * r + j];
+            m[a * cols + c] = (float)((double)m[a * cols + c] - s);
+        }
+    return OR_OK;
+}
+
+int or_powersgd_dp(int64_t W, int64_t rows, int64_t cols, int64_t r, int64_t r_max, float eta,
+                   const float* g, float* m, float* Q, float* P)
+{
+    if (W < 1 || rows < 1 || cols < 1 || r < 1 || r > r_max || r > rows || r > cols)
+        return OR_ERR_ARG;
+    int64_t n = rows * cols;
+    double* Pd = (double*)calloc((size_t)(rows * r), sizeof(double));
+    double* Pw = (double*)malloc((size_t)(rows * r) * sizeof(double));
+    double* Qw = (double*)malloc((size_t)(cols * r) * sizeof(double));
+    double* Qsum = (double*)calloc((size_t)(cols * r), sizeof(double));
+    if (!Pd || !Pw || !Qw || !Qsum) { free(Pd); free(Pw); free(Qw); free(Qsum); return OR_ERR_NOMEM; }
+
+    /* P = sum over workers of M_w Q */
+    for (int64_t w = 0; w < W; ++w) {
+        or_powersgd_dp_p(rows, cols, r, r_max, eta, g + w * n, m + w * n, Q, Pw);
+        for (int64_t i = 0; i < rows * r; ++i) Pd[i] += Pw[i];
+    }
+    or_mgs(rows, r, Pd);
 
     /* each worker: Q_w = M_w^T P, its residual, and the running sum of Q_w */
     for (int64_t w = 0; w < W; ++w) {
-        const double* Mw = M + w * n;
-        for (int64_t c = 0; c < cols; ++c)
-            for (int64_t j = 0; j < r; ++j) {
-                double s = 0.0;
-                for (int64_t a = 0; a < rows; ++a) s += Mw[a * cols + c] * Pd[a * r + j];
-                Qw[c * r + j] = s;
-                Qsum[c * r + j] += s;
-            }
-        for (int64_t a = 0; a < rows; ++a)
-            for (int64_t c = 0; c < cols; ++c) {
-                double s = 0.0;
-                for (int64_t j = 0; j < r; ++j) s += Pd[a * r + j] * Qw[c * r + j];
-                m[w * n + a * cols + c] = (float)(Mw[a * cols + c] - s);
-            }
+        or_powersgd_dp_q(rows, cols, r, Pd, m + w * n, Qw);
+        for (int64_t i = 0; i < cols * r; ++i) Qsum[i] += Qw[i];
     }
 
     for (int64_t a = 0; a < rows; ++a)
@@ -427,8 +455,8 @@ int or_powersgd_dp(int64_t W, int64_t rows, int64_t cols, int64_t r, int64_t r_m
     for (int64_t c = 0; c < cols; ++c)
         for (int64_t j = 0; j < r; ++j) Q[c * r_max + j] = (float)(Qsum[c * r + j] / (double)W);
 
-    free(M);
     free(Pd);
+    free(Pw);
     free(Qw);
     free(Qsum);
     return OR_OK;

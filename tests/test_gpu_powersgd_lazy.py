@@ -129,3 +129,17 @@ def test_lazy_payload_follows_the_oracle():
             assert np.array_equal(bits(hm[0, sl]), bits(hmem[0, sl]))
         else:
             assert relerr(hm[0, sl], hmem[0, sl], np.linalg.norm(hmem[0, sl])) <= 1e-4, l
+
+
+def test_lazy_equals_eager_on_a_large_layer():
+    """A layer above 4 Mi elements (products in fp32 from the payload's
+    factors, sums in fp64) next to a small one (fp64 products): the lazy
+    step is the eager step bit for bit in both precisions."""
+    need_gpu()
+    layers = [dict(rows=4200, cols=1024, kind="powersgd", cap=4, sigma=0.03),
+              dict(rows=64, cols=576, kind="powersgd", cap=2, sigma=0.04)]
+    W = 1
+    pair = Pair(layers, W)
+    for s, ranks in enumerate([[4, 2], [2, 2], [3, 1]]):
+        pair.step(workloads.gradients(layers, W, 332, s), ranks)
+    pair.materialize_and_compare()

@@ -118,3 +118,31 @@ def test_dense_dp_sums_in_worker_order():
         m = np.array(order, np.float32).reshape(3, 1)
         out, _ = oracle.dense_dp_unit(g, m, 0.05)
         assert out[0] == np.float32(want) * np.float32(1.0 / 3.0)
+
+
+def test_phases_compose_to_the_step():
+    """The data-parallel step cut at its two all-reduces: per-worker P_w,
+    their sum in worker order, Gram-Schmidt, per-worker Q_w and residual, the
+    mean of Q_w -- bit for bit the one-call step (the cut an exchange between
+    ranks makes), and P against numpy's QR of the summed P."""
+    rng = np.random.default_rng(31)
+    W, rows, cols, r = 3, 17, 23, 2
+    g = rng.standard_normal((W, rows, cols)).astype(np.float32)
+    m = rng.standard_normal((W, rows, cols)).astype(np.float32)
+    Q = oracle.powersgd_init_q(cols, 4, 2, 0, 0)
+    P_ref, Q_ref, m_ref = oracle.powersgd_dp_unit(g, m, Q, r, 0.05)
+    Ms, Psum = [], np.zeros((rows, r))
+    for w in range(W):
+        M, Pw = oracle.powersgd_dp_p_unit(g[w], m[w], Q, r, 0.05)
+        Ms.append(M)
+        Psum = Psum + Pw
+    Pd = oracle.mgs(Psum)
+    q, rr = np.linalg.qr(Psum)
+    assert np.allclose(Pd, q * np.sign(np.diag(rr)), atol=1e-12)
+    Qsum = np.zeros((cols, r))
+    for w in range(W):
+        Qw, res = oracle.powersgd_dp_q_unit(Pd, Ms[w])
+        Qsum = Qsum + Qw
+        assert np.array_equal(res.view(np.uint32), m_ref[w].view(np.uint32))
+    assert np.array_equal(Pd.astype(np.float32), P_ref[:, :r])
+    assert np.array_equal((Qsum / W).astype(np.float32), Q_ref[:, :r])
