@@ -9,7 +9,8 @@ first call raises -- there is no fallback.
 
 The entry points keep the C names: ef_topk_step, ef_randk_step,
 ef_randk_step_at, ef_sign_step, powersgd_init_q, powersgd_step,
-powersgd_step_lazy (with materialize_memory), powersgd_dp_step, accordion_init, accordion_select, decompress_accumulate,
+powersgd_step_lazy (with materialize_memory), powersgd_dp_step and its four parts
+for ranks (powersgd_dp_encode / _orthogonalize / _project / _mean), accordion_init, accordion_select, decompress_accumulate,
 decompress_apply, decompress_accumulate_noalloc, decompress_vote, plus the
 Table wrapper of gce_table_* and the workspace, status, schedule and profiling
 helpers.  The exchange of payloads between data-parallel ranks sits on top of
@@ -80,6 +81,15 @@ SIGNATURES = {
     "powersgd_step_lazy": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp,
                                      C.c_size_t, _vp]),
     "gce_materialize_memory": (C.c_int, [_vp, _i32, _vp, _vp, _vp, C.c_size_t, _vp]),
+    "gce_powersgd_dp_partials": (C.c_int, [_vp, C.POINTER(_i64)]),
+    "accordion_sumsq": (C.c_int, [_vp, _vp, _vp, _vp, C.c_size_t, _vp]),
+    "accordion_decide": (C.c_int, [_vp, _vp, _i64, _i32, _f64, _i32, _i32, _vp, _vp, _vp, _vp,
+                                   _vp]),
+    "powersgd_dp_encode": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp,
+                                     C.c_size_t, _vp]),
+    "powersgd_dp_orthogonalize": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, C.c_size_t, _vp]),
+    "powersgd_dp_project": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, C.c_size_t, _vp]),
+    "powersgd_dp_mean": (C.c_int, [_vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp]),
     "ef_sign_step": (C.c_int, [_vp, _i32, _vp, _vp, _f32, _vp, _vp, C.c_size_t, _vp]),
     "decompress_vote": (C.c_int, [_vp, _i32, _vp, _f32, _vp, _vp]),
     "accordion_init": (C.c_int, [_vp, _vp, _vp, _vp]),
@@ -288,6 +298,45 @@ def powersgd_dp_step(table, W, grad, mem, eta, k_or_rank, P, Q, vals, ws, stream
         _ptr(ws), ws.numel(), _stream(stream)))
 
 
+def powersgd_dp_partials(table):
+    """fp64 partial products per worker that powersgd_dp_encode writes."""
+    n = _i64()
+    _check("gce_powersgd_dp_partials", lib().gce_powersgd_dp_partials(table.handle, C.byref(n)))
+    return n.value
+
+
+def powersgd_dp_encode(table, W, grad, mem, eta, k_or_rank, Q, Ppart, vals, ws, stream=None):
+    """Data-parallel PowerSGD, first part: M into mem, partial M Q per worker
+    (float64 [W, partials]), DENSE residual rows into vals (include/gce.h)."""
+    import torch
+    _check("powersgd_dp_encode", lib().powersgd_dp_encode(
+        table.handle, int(W), _ptr(grad, _f32()), _ptr(mem, _f32()), float(eta),
+        _ptr(k_or_rank, _i32()), _ptr(Q, _f32()), _ptr(Ppart, torch.float64),
+        _ptr(vals, _f32()), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def powersgd_dp_orthogonalize(table, W, k_or_rank, Ppart, P, ws, stream=None):
+    """P from the gathered partials of all W workers."""
+    import torch
+    _check("powersgd_dp_orthogonalize", lib().powersgd_dp_orthogonalize(
+        table.handle, int(W), _ptr(k_or_rank, _i32()), _ptr(Ppart, torch.float64),
+        _ptr(P, _f32()), _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def powersgd_dp_project(table, W, mem, k_or_rank, Qw, ws, stream=None):
+    """Q_w = M_w^T P per worker into Qw, each worker's residual into mem."""
+    _check("powersgd_dp_project", lib().powersgd_dp_project(
+        table.handle, int(W), _ptr(mem, _f32()), _ptr(k_or_rank, _i32()), _ptr(Qw, _f32()),
+        _ptr(ws), ws.numel(), _stream(stream)))
+
+
+def powersgd_dp_mean(table, W, k_or_rank, Qw, Q, vals_all, vals, stream=None):
+    """The workers' mean Q and DENSE payloads from the gathered rows."""
+    _check("powersgd_dp_mean", lib().powersgd_dp_mean(
+        table.handle, int(W), _ptr(k_or_rank, _i32()), _ptr(Qw, _f32()), _ptr(Q, _f32()),
+        _ptr(vals_all, _f32()), _ptr(vals, _f32()), _stream(stream)))
+
+
 def ef_sign_step(table, W, grad, mem, eta, vals, ws, stream=None):
     """signSGD with error feedback; vals holds each SIGN layer's scale (slot
     0) and sign words (slots 4..., uint32 bit patterns) (include/gce.h)."""
@@ -316,6 +365,24 @@ def accordion_select(table, grad, step, interval, threshold, lvl_low, lvl_high, 
         int(lvl_low), int(lvl_high), _ptr(prev_norm, torch.float64), _ptr(level, _i32()),
         _ptr(cur_norm, torch.float64), _ptr(k_or_rank_out, _i32()), _ptr(ws), ws.numel(),
         _stream(stream)))
+
+
+def accordion_sumsq(table, grad, sumsq, ws, stream=None):
+    """Per-layer sum of squares of grad (float64 [L]); see accordion_decide."""
+    import torch
+    _check("accordion_sumsq", lib().accordion_sumsq(
+        table.handle, _ptr(grad, _f32()), _ptr(sumsq, torch.float64), _ptr(ws), ws.numel(),
+        _stream(stream)))
+
+
+def accordion_decide(table, sumsq, step, interval, threshold, lvl_low, lvl_high, prev_norm, level,
+                     cur_norm, k_or_rank_out, stream=None):
+    """accordion_select's decision from given per-layer sums of squares."""
+    import torch
+    _check("accordion_decide", lib().accordion_decide(
+        table.handle, _ptr(sumsq, torch.float64), int(step), int(interval), float(threshold),
+        int(lvl_low), int(lvl_high), _ptr(prev_norm, torch.float64), _ptr(level, _i32()),
+        _ptr(cur_norm, torch.float64), _ptr(k_or_rank_out, _i32()), _stream(stream)))
 
 
 def decompress_accumulate(table, W, vals, idx, k_or_rank, P, Q, scale, out, ws, stream=None):

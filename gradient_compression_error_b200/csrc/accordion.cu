@@ -107,12 +107,36 @@ __device__ __forceinline__ int32_t ac_param(const DevLayer& L, int32_t level, in
     return int32_t(k < 1 ? 1 : k);
 }
 
-// one warp per layer
+// A layer's sum of squares from its tile partials, in a fixed order: lane i
+// adds tiles i, i + 32, ... in order, then the lanes' sums by warp_sum.  Run by
+// a full warp.
+__device__ __forceinline__ double ac_layer_sumsq(const int2 pl, const double* __restrict__ part) {
+    const int lane = threadIdx.x & 31;
+    double s = 0.0;
+    for (int i = lane; i < pl.y; i += 32) s += part[pl.x + i];
+    return warp_sum(s);
+}
+
+// one warp per layer: sumsq[l] (0 for DENSE layers)
+__global__ void __launch_bounds__(256) ac_sumsq_kernel(const DevLayer* __restrict__ layers,
+                                                       const int2* __restrict__ ac_layer, int32_t L,
+                                                       const double* __restrict__ part,
+                                                       double* __restrict__ sumsq) {
+    const int lane = threadIdx.x & 31;
+    const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t l = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); l < L; l += wstride) {
+        const double s = layers[l].kind == GCE_KIND_DENSE ? 0.0 : ac_layer_sumsq(ac_layer[l], part);
+        if (lane == 0) sumsq[l] = s;
+    }
+}
+
+// one warp per layer; the sums of squares from the tile partials, or (sumsq
+// non-null) given per layer
 __global__ void __launch_bounds__(256) ac_decide_kernel(
     const DevLayer* __restrict__ layers, const int2* __restrict__ ac_layer, int32_t L,
-    const double* __restrict__ part, int32_t check, double threshold, int32_t lvl_low,
-    int32_t lvl_high, double* __restrict__ prev_norm, int32_t* __restrict__ level,
-    double* __restrict__ cur_norm, int32_t* __restrict__ k_or_rank) {
+    const double* __restrict__ part, const double* __restrict__ sumsq, int32_t check,
+    double threshold, int32_t lvl_low, int32_t lvl_high, double* __restrict__ prev_norm,
+    int32_t* __restrict__ level, double* __restrict__ cur_norm, int32_t* __restrict__ k_or_rank) {
     const int lane = threadIdx.x & 31;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t l = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); l < L; l += wstride) {
@@ -123,10 +147,7 @@ __global__ void __launch_bounds__(256) ac_decide_kernel(
         }
         int32_t lv = level[l];
         if (check) {
-            const int2 pl = ac_layer[l];
-            double s = 0.0;
-            for (int i = lane; i < pl.y; i += 32) s += part[pl.x + i];
-            s = warp_sum(s);
+            const double s = sumsq ? sumsq[l] : ac_layer_sumsq(ac_layer[l], part);
             const double cur = sqrt(s);
             const double prev = prev_norm[l];
             double rel;
@@ -189,7 +210,44 @@ extern "C" int accordion_select(const gce_table* t, const float* grad, int64_t s
         GCE_LAUNCH(ac_norm_kernel, wave_grid(t->ac_ntiles, 8, r_norm), 256, 0, st,
                    t->d_layers, t->d_ac_tiles, t->ac_ntiles, grad, part);
     GCE_LAUNCH(ac_decide_kernel, wave_grid((t->L + 7) / 8, 4, r_decide), 256, 0, st,
-               t->d_layers, t->d_ac_layer, t->L, part, check, threshold, lvl_low, lvl_high,
-               prev_norm, level, cur_norm, k_or_rank_out);
+               t->d_layers, t->d_ac_layer, t->L, part, nullptr, check, threshold, lvl_low,
+               lvl_high, prev_norm, level, cur_norm, k_or_rank_out);
+    return check_launch();
+}
+
+extern "C" int accordion_sumsq(const gce_table* t, const float* grad, double* sumsq, void* ws,
+                               size_t ws_bytes, void* stream) {
+    if (!t || !grad || !sumsq || !ws || !aligned16(grad) || !aligned16(ws)) return GCE_ERR_ARG;
+    if (ws_bytes < accordion_ws_bytes(t)) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    double* part = at<double>(ws, GCE_WS_HEADER_BYTES);
+    static const int r_norm = resident_blocks(ac_norm_kernel, 256);
+    static const int r_sum = resident_blocks(ac_sumsq_kernel, 256);
+    if (t->ac_ntiles > 0)
+        GCE_LAUNCH(ac_norm_kernel, wave_grid(t->ac_ntiles, 8, r_norm), 256, 0, st,
+                   t->d_layers, t->d_ac_tiles, t->ac_ntiles, grad, part);
+    GCE_LAUNCH(ac_sumsq_kernel, wave_grid((t->L + 7) / 8, 4, r_sum), 256, 0, st, t->d_layers,
+               t->d_ac_layer, t->L, part, sumsq);
+    return check_launch();
+}
+
+extern "C" int accordion_decide(const gce_table* t, const double* sumsq, int64_t step,
+                                int32_t interval, double threshold, int32_t lvl_low,
+                                int32_t lvl_high, double* prev_norm, int32_t* level,
+                                double* cur_norm, int32_t* k_or_rank_out, void* stream) {
+    if (!t || !prev_norm || !level || !k_or_rank_out) return GCE_ERR_ARG;
+    if (interval < 1 || step < 0 || !(threshold >= 0.0)) return GCE_ERR_ARG;
+    if (t->ckind == GCE_KIND_POWERSGD) {
+        if (lvl_low < 1 || lvl_low > kMaxRank || lvl_high < 1 || lvl_high > kMaxRank) return GCE_ERR_ARG;
+    } else if (lvl_low < 1 || lvl_low > 1000000 || lvl_high < 1 || lvl_high > 1000000) {
+        return GCE_ERR_ARG;
+    }
+    const int check = (step % interval) == 0;
+    if (check && !sumsq) return GCE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    static const int r_decide = resident_blocks(ac_decide_kernel, 256);
+    GCE_LAUNCH(ac_decide_kernel, wave_grid((t->L + 7) / 8, 4, r_decide), 256, 0, st,
+               t->d_layers, t->d_ac_layer, t->L, nullptr, sumsq, check, threshold, lvl_low,
+               lvl_high, prev_norm, level, cur_norm, k_or_rank_out);
     return check_launch();
 }

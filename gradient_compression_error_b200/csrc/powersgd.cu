@@ -154,17 +154,20 @@ size_t powersgd_ws_bytes(const gce_table* t, int32_t W) { return ps_layout(t, W)
 
 // The data-parallel step: partials per worker, one orthonormal P per layer,
 // and every worker's Q_w (fp32 for the mean, fp64 for its residual).
+// The parts that do not grow with W come first, so that the orthonormalisation
+// of a step split between ranks finds them at the same place whatever W the
+// workspace was sized for.
 static PsWs ps_dp_layout(const gce_table* t, int32_t W) {
     PsWs o;
     Carver c;
-    o.ppart = c.take<double>(int64_t(W) * t->ppart_pw);
     o.pd = c.take<double>(t->pd_pw);
-    o.qpart = c.take<double>(int64_t(W) * t->qpart_pw);
-    o.qd = c.take<double>(int64_t(W) * t->Q_pw);
-    o.qloc = c.take<float>(int64_t(W) * t->Q_pw);
     o.tparts = c.take<double>(t->ps_tall_parts);
     o.tscal = c.take<double>(t->ps_ntall);
     o.tdone = c.take<int32_t>(t->ps_ntall);
+    o.ppart = c.take<double>(int64_t(W) * t->ppart_pw);
+    o.qpart = c.take<double>(int64_t(W) * t->qpart_pw);
+    o.qd = c.take<double>(int64_t(W) * t->Q_pw);
+    o.qloc = c.take<float>(int64_t(W) * t->Q_pw);
     o.total = c.off;
     return o;
 }
@@ -735,6 +738,48 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
     flag_nonfinite(bad, status);
 }
 
+// ---- the workers' means after an exchange between ranks ------------------------------------
+// Q = fl(fl(sum_w Q_w) * inv_w) over W gathered rows of Q_w (worker order from
+// +0, fp32), as the one-GPU data-parallel step forms its warm start.
+__global__ void __launch_bounds__(256) ps_qmean_kernel(
+    const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles,
+    int32_t W, int64_t Q_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ Qw,
+    float* __restrict__ Q, float inv_w) {
+    for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
+        const int4 d = tiles[u];
+        const DevLayer L = layers[d.x];
+        const int r = ps_rank(L, k_or_rank, d.x);
+        if (r == 0) continue;
+        const int cap = L.cap;
+        const int64_t c0 = int64_t(d.y) * kPsQB;
+        const int cw = int(min64(kPsQB, L.cols - c0));
+        for (int i = threadIdx.x; i < cw * r; i += blockDim.x) {
+            const int64_t o = L.q_off + (c0 + i / r) * cap + i % r;
+            float sum = 0.0f;
+            for (int w = 0; w < W; ++w) sum = __fadd_rn(sum, Qw[int64_t(w) * Q_pw + o]);
+            Q[o] = __fmul_rn(sum, inv_w);
+        }
+    }
+}
+
+// DENSE layers: mean = fl(fl(sum_w v_w) * inv_w) over W gathered payload rows.
+__global__ void __launch_bounds__(256) ps_vmean_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ dtile_layer,
+    const int32_t* __restrict__ dtile_start, int32_t ntiles, int32_t W, int64_t vals_pw,
+    const float* __restrict__ vals_all, float* __restrict__ vals, float inv_w) {
+    for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
+        const DevLayer L = layers[dtile_layer[u]];
+        const int64_t s0 = dtile_start[u];
+        const int64_t cnt = min64(int64_t(kDenseTile), L.n - s0);
+        for (int64_t i = threadIdx.x; i < cnt; i += blockDim.x) {
+            float sum = 0.0f;
+            for (int w = 0; w < W; ++w)
+                sum = __fadd_rn(sum, vals_all[int64_t(w) * vals_pw + L.val_off + s0 + i]);
+            vals[L.val_off + s0 + i] = __fmul_rn(sum, inv_w);
+        }
+    }
+}
+
 // ---- residual: m <- M - P Q^T, dense_out <- P Q^T ---------------------------------------------
 // The memory from the workspace's factors in the layer's precision
 // (ps_unproject); dense_out from the fp32 P and Q the payload carries, formed
@@ -1152,4 +1197,133 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return GCE_OK;
+}
+
+// ---- data-parallel PowerSGD between ranks: the step cut at its two sums ------------------
+static int ps_dp_check(const gce_table* t, const int32_t* k_or_rank, void* ws) {
+    if (!t || !ws || !aligned16(ws)) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    if (k_or_rank && (reinterpret_cast<uintptr_t>(k_or_rank) & 3)) return GCE_ERR_ARG;
+    return GCE_OK;
+}
+
+extern "C" int gce_powersgd_dp_partials(const gce_table* t, int64_t* doubles_per_worker) {
+    if (!t || !doubles_per_worker) return GCE_ERR_ARG;
+    *doubles_per_worker = t->ppart_pw;
+    return GCE_OK;
+}
+
+extern "C" int powersgd_dp_encode(const gce_table* t, int32_t W, const float* grad, float* mem,
+                                  float eta, const int32_t* k_or_rank, const float* Q,
+                                  double* Ppart, float* vals, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    int rc = ps_dp_check(t, k_or_rank, ws);
+    if (rc != GCE_OK) return rc;
+    if (W < 1 || !grad || !mem || !aligned16(grad) || !aligned16(mem)) return GCE_ERR_ARG;
+    if (t->nps > 0 && (!Q || !Ppart || !aligned16(Q) || !aligned16(Ppart))) return GCE_ERR_ARG;
+    if (t->dtiles_pw > 0 && (!vals || !aligned16(vals))) return GCE_ERR_ARG;
+    if (ws_bytes < ps_dp_layout(t, W).total) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(ws);
+    if (t->nps > 0) {
+        static const int r_mq = resident_blocks_smem(ps_mq_kernel<false>, 256, ps_mq_smem(false));
+        // every worker reads the shared warm start Q (stride 0)
+        GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256,
+                   ps_mq_smem(false), st, t->d_layers, static_cast<const PsLayer*>(t->d_ps),
+                   t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->ppart_pw, grad, mem,
+                   eta, k_or_rank, Q, Ppart, status, nullptr, int64_t(0), nullptr, t->L, nullptr);
+        if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
+    }
+    // DENSE layers: each worker's residual as its payload row, memory -> 0
+    return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
+}
+
+extern "C" int powersgd_dp_orthogonalize(const gce_table* t, int32_t W, const int32_t* k_or_rank,
+                                         const double* Ppart, float* P, void* ws, size_t ws_bytes,
+                                         void* stream) {
+    int rc = ps_dp_check(t, k_or_rank, ws);
+    if (rc != GCE_OK) return rc;
+    if (W < 1) return GCE_ERR_ARG;
+    if (t->nps == 0) return GCE_OK;
+    if (!Ppart || !P || !aligned16(Ppart) || !aligned16(P)) return GCE_ERR_ARG;
+    // the W-independent head of the workspace (any W it was sized for)
+    const PsWs lay = ps_dp_layout(t, 1);
+    if (ws_bytes < lay.ppart) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int32_t* status = static_cast<int32_t*>(ws);
+    const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
+    double* pd = at<double>(ws, lay.pd);
+    int32_t* tdone = at<int32_t>(ws, lay.tdone);
+    static const int r_orth = resident_blocks(ps_orth_kernel, 256);
+    static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
+    // one P per layer from the partials of all W workers, in worker order
+    GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
+               t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank, Ppart,
+               pd, P, status, t->ps_ntall, tdone, t->L, nullptr);
+    if (t->ps_ntall > 0) {
+        for (const PsOrthOp& op : ps_orth_ops(t->ps_tall_cap))
+            GCE_LAUNCH(ps_orth_tall_kernel, wave_grid(t->ps_tall_nunits, 8, r_tall), 256, 0, st,
+                       op, t->d_layers, ps, t->d_ps_tall_units, t->ps_tall_nunits, 1, W,
+                       int64_t(0), t->ppart_pw, t->pd_pw, t->ps_ntall, t->ps_tall_parts,
+                       k_or_rank, Ppart, pd, at<double>(ws, lay.tparts),
+                       at<double>(ws, lay.tscal), tdone, P);
+    }
+    return check_launch();
+}
+
+extern "C" int powersgd_dp_project(const gce_table* t, int32_t W, float* mem,
+                                   const int32_t* k_or_rank, float* Qw, void* ws,
+                                   size_t ws_bytes, void* stream) {
+    int rc = ps_dp_check(t, k_or_rank, ws);
+    if (rc != GCE_OK) return rc;
+    if (W < 1 || !mem || !aligned16(mem)) return GCE_ERR_ARG;
+    if (t->nps == 0) return GCE_OK;
+    if (!Qw || !aligned16(Qw)) return GCE_ERR_ARG;
+    const PsWs lay = ps_dp_layout(t, W);
+    if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
+    double* pd = at<double>(ws, lay.pd);
+    double* qpart = at<double>(ws, lay.qpart);
+    double* qd = at<double>(ws, lay.qd);
+    static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
+    static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
+    static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
+    // Q_w = M_w^T P for this rank's workers with the shared P (stride 0)
+    GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
+               t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, int64_t(0), t->qpart_pw,
+               mem, k_or_rank, pd, qpart);
+    GCE_LAUNCH(ps_qred_kernel<false>, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0,
+               st, t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
+               k_or_rank, qpart, Qw, qd, nullptr, 1.0f);
+    // each worker's error against its own Q_w
+    GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
+               kPsResidSmem, st, t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N,
+               int64_t(0), t->Q_pw, int64_t(0), k_or_rank, nullptr, nullptr, pd, qd, mem,
+               nullptr, nullptr, t->L);
+    return check_launch();
+}
+
+extern "C" int powersgd_dp_mean(const gce_table* t, int32_t W, const int32_t* k_or_rank,
+                                const float* Qw, float* Q, const float* vals_all, float* vals,
+                                void* stream) {
+    if (!t || W < 1) return GCE_ERR_ARG;
+    if (t->ckind != GCE_KIND_POWERSGD && t->ckind != -1) return GCE_ERR_KIND;
+    if (k_or_rank && (reinterpret_cast<uintptr_t>(k_or_rank) & 3)) return GCE_ERR_ARG;
+    if (t->nps > 0 && (!Qw || !Q)) return GCE_ERR_ARG;
+    if (t->dtiles_pw > 0 && (!vals_all || !vals)) return GCE_ERR_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const float inv_w = 1.0f / float(W);
+    if (t->nps > 0) {
+        static const int r_qm = resident_blocks(ps_qmean_kernel, 256);
+        GCE_LAUNCH(ps_qmean_kernel, wave_grid(t->psq_ntiles, 8, r_qm), 256, 0, st, t->d_layers,
+                   t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, k_or_rank, Qw, Q, inv_w);
+    }
+    if (t->dtiles_pw > 0) {
+        static const int r_vm = resident_blocks(ps_vmean_kernel, 256);
+        GCE_LAUNCH(ps_vmean_kernel, wave_grid(t->dtiles_pw, 8, r_vm), 256, 0, st, t->d_layers,
+                   t->d_dtile_layer, t->d_dtile_start, t->dtiles_pw, W, t->vals_pw, vals_all, vals,
+                   inv_w);
+    }
+    return check_launch();
 }

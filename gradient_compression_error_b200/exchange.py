@@ -23,13 +23,39 @@ same k tensor.
 
 Payload kinds: top-k, rand-k, signSGD and dense layers.  rand-k's generator
 takes the worker index, so rank r encodes as job-wide worker r
-(ef_randk_step_at).  Not exchanged here: PowerSGD, whose data-parallel form
-sums P and Q over the workers inside the step, between its contractions.
+(ef_randk_step_at).
+
+PowerSGD's data-parallel form sums P and Q over the workers between its
+contractions (On the Utility of Gradient Compression, Key results: PowerSGD is
+all-reduce compatible).  PowerSgdDataParallelStep runs it between ranks cut at
+those two sums: each rank gathers the other ranks' rows (partial products of
+M_w Q, then Q_w) and sums them in worker order itself, so every rank holds the
+same P and Q and the step is bit for bit powersgd_dp_step over all workers.
+AccordionAcrossRanks all-reduces the per-layer sums of squares, so every rank
+takes Accordion's decision from the norm of all ranks' gradients.
 """
 import torch
 import torch.distributed as dist
 
 METHODS = ("topk", "randk", "sign")
+
+
+def gather_rows(out, row, group=None):
+    """Row r of ``out`` [world, n] <- rank r's ``row`` (n elements of out's
+    dtype and device), on every rank; every rank must call it, in the same
+    order.  NCCL gathers into the buffer; gloo into a list of its row views."""
+    if row is None or row.numel() != out.shape[1] or row.dtype != out.dtype \
+            or row.device != out.device:
+        raise ValueError("row must be %d %s elements on %s" % (out.shape[1], out.dtype,
+                                                                out.device))
+    row = row.reshape(-1)
+    if not row.is_contiguous():
+        raise ValueError("row must be contiguous")
+    if dist.get_backend(group) == "nccl":
+        dist.all_gather_into_tensor(out, row, group=group)
+    else:
+        dist.all_gather(list(out.unbind(0)), row, group=group)
+    return out
 
 
 class PayloadExchange:
@@ -48,22 +74,9 @@ class PayloadExchange:
         self.vals = torch.zeros((self.world, self.n), dtype=torch.float32, device=device)
         self.idx = (torch.zeros((self.world, self.n), dtype=torch.int32, device=device)
                     if with_idx else None)
-        # NCCL gathers straight into the [world, n] buffer; gloo takes a list
-        # of its rows (views, written in place)
-        self._into = dist.get_backend(group) == "nccl"
 
     def _gather(self, out, row):
-        if row is None or row.numel() != self.n or row.dtype != out.dtype \
-                or row.device != out.device:
-            raise ValueError("payload row must be %d %s elements on %s"
-                             % (self.n, out.dtype, out.device))
-        row = row.reshape(-1)
-        if not row.is_contiguous():
-            raise ValueError("payload row must be contiguous")
-        if self._into:
-            dist.all_gather_into_tensor(out, row, group=self.group)
-        else:
-            dist.all_gather(list(out.unbind(0)), row, group=self.group)
+        gather_rows(out, row, self.group)
 
     def gather(self, vals_row, idx_row=None):
         """All ranks' rows, in rank order: (vals, idx); idx is None without indices."""
@@ -87,7 +100,7 @@ class DataParallelStep:
     def __init__(self, table, method, group=None, device="cuda"):
         import gradient_compression_error_b200 as g
         if method not in METHODS:
-            raise ValueError("method must be one of %s (PowerSGD is not exchanged here)"
+            raise ValueError("method must be one of %s (PowerSGD: PowerSgdDataParallelStep)"
                              % (METHODS,))
         ck = table.compressed_kind
         if ck not in (-1, g.KIND[method]):
@@ -145,3 +158,92 @@ class DataParallelStep:
         self.exchange()
         self.decode(out, 1.0 / self.world if scale is None else scale, k, apply, vote)
         return out
+
+
+class PowerSgdDataParallelStep:
+    """Data-parallel PowerSGD over the ranks of ``group``, one worker per rank,
+    cut at its two sums (include/gce.h, powersgd_dp_encode ... _mean).
+
+    Every rank starts from the same warm start Q (``seed``) and ends each step
+    with the same P, Q and DENSE mean; ``decode`` writes P Q^T plus the DENSE
+    means (the workers' mean update) into a dense buffer.
+    """
+
+    def __init__(self, table, group=None, device="cuda", seed=0):
+        import gradient_compression_error_b200 as g
+        if table.compressed_kind not in (-1, g.KIND["powersgd"]):
+            raise ValueError("PowerSgdDataParallelStep needs a PowerSGD table")
+        self.g = g
+        self.table = table
+        self.group = group
+        self.world = dist.get_world_size(group)
+        f32, f64 = torch.float32, torch.float64
+        npart = max(2, g.powersgd_dp_partials(table))
+        nq, nv = max(4, table.Q_per_worker), max(4, table.vals_per_worker)
+        self.P = torch.zeros(max(4, table.P_per_worker), dtype=f32, device=device)
+        self.Q = torch.zeros(nq, dtype=f32, device=device)
+        g.powersgd_init_q(table, 1, seed, self.Q)
+        self.ppart_row = torch.zeros((1, npart), dtype=f64, device=device)
+        self.ppart_all = torch.zeros((self.world, npart), dtype=f64, device=device)
+        self.qw_row = torch.zeros((1, nq), dtype=f32, device=device)
+        self.qw_all = torch.zeros((self.world, nq), dtype=f32, device=device)
+        self.vals_row = torch.zeros((1, nv), dtype=f32, device=device)
+        self.vals_all = torch.zeros((self.world, nv), dtype=f32, device=device)
+        self.vals = torch.zeros(nv, dtype=f32, device=device)
+        self.ws = table.workspace(1, "powersgd_dp", device)
+        self.ws_dec = table.workspace(1, "decompress", device)
+
+    def __call__(self, grad, mem, eta, k=None):
+        """One step on this rank's gradient and memory [1, N]; returns (P, Q,
+        DENSE means), the same on every rank."""
+        g, t = self.g, self.table
+        g.powersgd_dp_encode(t, 1, grad, mem, eta, k, self.Q, self.ppart_row, self.vals_row,
+                             self.ws)
+        gather_rows(self.ppart_all, self.ppart_row, self.group)
+        gather_rows(self.vals_all, self.vals_row, self.group)
+        g.powersgd_dp_orthogonalize(t, self.world, k, self.ppart_all, self.P, self.ws)
+        g.powersgd_dp_project(t, 1, mem, k, self.qw_row, self.ws)
+        gather_rows(self.qw_all, self.qw_row, self.group)
+        g.powersgd_dp_mean(t, self.world, k, self.qw_all, self.Q, self.vals_all, self.vals)
+        return self.P, self.Q, self.vals
+
+    def decode(self, out, k=None, apply=False, scale=1.0):
+        """out = P Q^T + DENSE means (scale times that); with ``apply``,
+        out -= it instead."""
+        fn = self.g.decompress_apply if apply else self.g.decompress_accumulate
+        fn(self.table, 1, self.vals, None, k, self.P, self.Q, scale, out, self.ws_dec)
+
+
+class AccordionAcrossRanks:
+    """Accordion's per-layer level switch taken from the gradients of every
+    rank of ``group``: on check steps the per-layer sums of squares are
+    all-reduced before the decision, so all ranks hold the same levels and
+    k / ranks (include/gce.h, accordion_sumsq / accordion_decide)."""
+
+    def __init__(self, table, interval, threshold, lvl_low, lvl_high, group=None,
+                 device="cuda"):
+        import gradient_compression_error_b200 as g
+        self.g = g
+        self.table = table
+        self.group = group
+        self.args = (int(interval), float(threshold), int(lvl_low), int(lvl_high))
+        L = table.L
+        self.sumsq = torch.zeros(L, dtype=torch.float64, device=device)
+        self.prev = torch.empty(L, dtype=torch.float64, device=device)
+        self.level = torch.empty(L, dtype=torch.int32, device=device)
+        self.cur = torch.zeros(L, dtype=torch.float64, device=device)
+        self.k = torch.zeros(L, dtype=torch.int32, device=device)
+        self.ws = table.workspace(1, "accordion", device)
+        g.accordion_init(table, self.prev, self.level)
+
+    def __call__(self, grad, step):
+        """k (or rank) per layer for this step, from this rank's gradient [N]."""
+        g = self.g
+        interval, threshold, lo, hi = self.args
+        if step % interval == 0:
+            g.accordion_sumsq(self.table, grad, self.sumsq, self.ws)
+            dist.all_reduce(self.sumsq, op=dist.ReduceOp.SUM, group=self.group)
+        g.accordion_decide(self.table, self.sumsq, step, interval, threshold, lo, hi, self.prev,
+                           self.level, self.cur, self.k)
+        return self.k
+

@@ -290,6 +290,45 @@ GCE_API int powersgd_dp_step(const gce_table* table, int32_t W, const float* gra
                              float* vals, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * The data-parallel PowerSGD step cut at its two sums, for data-parallel
+ * ranks that each hold some of the W workers ([UTIL] Key results: PowerSGD is
+ * all-reduce compatible).  Run in this order, with the rows of every rank
+ * gathered in worker order where marked; the result is powersgd_dp_step over
+ * all W workers, bit for bit (the sums run over the gathered rows in worker
+ * order, as that step sums them):
+ *   powersgd_dp_encode(Wl workers): M_w = fl32(mem_w + fl32(eta*grad_w)) into
+ *     mem; Ppart [Wl][gce_powersgd_dp_partials doubles] the fp64 partial
+ *     products M_w Q of each worker (Q: the shared warm start); DENSE layers:
+ *     vals [Wl][vals_per_worker] each worker's residual, memory -> 0.
+ *   -- gather Ppart rows of all W workers (and the vals rows) --
+ *   powersgd_dp_orthogonalize(W): P <- the orthonormal columns (modified
+ *     Gram-Schmidt, fp64) of sum_w M_w Q from the W gathered Ppart rows;
+ *     P [P_per_worker] fp32, and its fp64 copy kept in ws.
+ *   powersgd_dp_project(Wl): Qw [Wl][Q_per_worker] <- Q_w = M_w^T P (fp32),
+ *     mem_w <- M_w - P Q_w^T; reads P from ws (the same ws as
+ *     powersgd_dp_orthogonalize).
+ *   -- gather Qw rows of all W workers --
+ *   powersgd_dp_mean(W): Q <- fl32(fl32(sum_w Q_w) * fl32(1/W)); DENSE:
+ *     vals <- fl32(fl32(sum_w vals_all_w) * fl32(1/W)) from the gathered rows.
+ * ws: gce_workspace_bytes(GCE_OP_POWERSGD_DP) for this rank's Wl workers, the
+ * same workspace for the four calls of a step.  k_or_rank as powersgd_step
+ * (the same on every rank).  Errors as powersgd_dp_step.
+ */
+GCE_API int gce_powersgd_dp_partials(const gce_table* table, int64_t* doubles_per_worker);
+GCE_API int powersgd_dp_encode(const gce_table* table, int32_t W, const float* grad, float* mem,
+                               float eta, const int32_t* k_or_rank, const float* Q, double* Ppart,
+                               float* vals, void* ws, size_t ws_bytes, void* stream);
+GCE_API int powersgd_dp_orthogonalize(const gce_table* table, int32_t W,
+                                      const int32_t* k_or_rank, const double* Ppart, float* P,
+                                      void* ws, size_t ws_bytes, void* stream);
+GCE_API int powersgd_dp_project(const gce_table* table, int32_t W, float* mem,
+                                const int32_t* k_or_rank, float* Qw, void* ws, size_t ws_bytes,
+                                void* stream);
+GCE_API int powersgd_dp_mean(const gce_table* table, int32_t W, const int32_t* k_or_rank,
+                             const float* Qw, float* Q, const float* vals_all, float* vals,
+                             void* stream);
+
+/*
  * signSGD with error feedback for every (worker, SIGN layer) ([UTIL]
  * Method / Key results: sign SGD, one bit per element; [MEM] Method: the
  * memory), plus DENSE layers (payload to vals, memory -> 0):
@@ -380,6 +419,28 @@ GCE_API int accordion_select(const gce_table* table, const float* grad, int64_t 
                      int32_t interval, double threshold, int32_t lvl_low, int32_t lvl_high,
                      double* prev_norm, int32_t* level, double* cur_norm,
                      int32_t* k_or_rank_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * accordion_select cut in two, for data-parallel ranks that must take the
+ * same decision from the norms of all their gradients ([ACC] Method: the
+ * gradient norm; [UTIL] Key results: the all-reduce):
+ *   accordion_sumsq: sumsq[l] = sum of grad_i^2 over each compressed layer
+ *     (fp64, the fixed order accordion_select uses; 0 for DENSE layers).
+ *     sumsq: device double[L].  ws as accordion_select.
+ *   -- all-reduce (sum) sumsq over the ranks: the squared norm of the layer's
+ *      gradients of every rank --
+ *   accordion_decide: accordion_select's decision and k / rank output from
+ *     s_l = sqrt(sumsq[l]) (sumsq may be NULL on steps that are not check
+ *     steps).  Other arguments as accordion_select.
+ * accordion_sumsq then accordion_decide on one gradient is accordion_select,
+ * bit for bit.
+ */
+GCE_API int accordion_sumsq(const gce_table* table, const float* grad, double* sumsq, void* ws,
+                            size_t ws_bytes, void* stream);
+GCE_API int accordion_decide(const gce_table* table, const double* sumsq, int64_t step,
+                             int32_t interval, double threshold, int32_t lvl_low,
+                             int32_t lvl_high, double* prev_norm, int32_t* level,
+                             double* cur_norm, int32_t* k_or_rank_out, void* stream);
 
 /*
  * Aggregate [UTIL] of the W workers' payloads into a dense fp32 out [N]:

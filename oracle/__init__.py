@@ -45,6 +45,7 @@ def lib():
             "or_accum_sign": (None, [i64, f32, vp, vp]),
             "or_vote_sign": (None, [i64, i64, i64, vp, f32, vp]),
             "or_layer_norm": (f64, [i64, vp]),
+            "or_layer_sumsq": (f64, [i64, vp]),
             "or_accordion_decide": (i32, [f64, f64, f64]),
             "or_accum_sparse": (None, [i64, vp, vp, vp]),
             "or_accum_dense": (None, [i64, vp, vp]),
@@ -251,6 +252,11 @@ def vote_sign(words, n, out_scale):
 def layer_norm(g):
     g = _f32(g)
     return float(lib().or_layer_norm(g.size, _ptr(g)))
+
+
+def layer_sumsq(g):
+    g = _f32(g)
+    return float(lib().or_layer_sumsq(g.size, _ptr(g)))
 
 
 def accordion_decide(s_prev, s_cur, threshold):

@@ -538,11 +538,18 @@ void or_vote_sign(int64_t W, int64_t n, int64_t words_per_worker, const uint32_t
 /* ------------------------------------------------------------------ */
 /* Accordion [ACC]: L2 norm of one layer's raw gradient, summed in index
  * order in double. */
-double or_layer_norm(int64_t n, const float* g)
+/* A layer's sum of squares, fp64 in index order; its square root is the
+ * layer's gradient norm [ACC]. */
+double or_layer_sumsq(int64_t n, const float* g)
 {
     double s = 0.0;
     for (int64_t i = 0; i < n; ++i) s += (double)g[i] * (double)g[i];
-    return sqrt(s);
+    return s;
+}
+
+double or_layer_norm(int64_t n, const float* g)
+{
+    return sqrt(or_layer_sumsq(n, g));
 }
 
 /*
