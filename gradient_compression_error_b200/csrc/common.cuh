@@ -41,20 +41,6 @@ struct alignas(16) TileInfo {
     int32_t tstart;   // first element of the tile within its layer
 };
 
-// One decode tile's fields (kDcTile outputs of one layer), so that a decoder
-// reaches them with one 48-byte load instead of tile -> layer -> record.
-struct alignas(16) DcTile {
-    int64_t out_off;  // first output element: the layer's offset + tile start
-    int64_t val_off;  // the layer's first payload slot
-    int32_t l;        // layer
-    int32_t tt;       // tile index within the layer
-    int32_t cnt;      // outputs in this tile
-    int32_t kind;
-    int32_t dc_base;  // the layer's first tile-bound slot
-    int32_t cap;
-    int32_t pad[2];
-};
-
 // A pipelined signSGD schedule uploaded for one (W, ahead): nphase runs
 // (the last a sentinel) covering nitems work items.
 struct SgPlan {
@@ -81,8 +67,6 @@ struct gce_table {
     int32_t tiles_pw = 0;                  // main tiles (compressed layers) per worker
     int32_t* d_tile_layer = nullptr;       // [tiles_pw] layer of each main tile
     gce::TileInfo* d_tile_info = nullptr;  // [tiles_pw] the same tiles' layer fields
-    int32_t tk_groups_pw = 0;              // top-k emit items (kTkGroup tiles) per worker
-    int2* d_tk_groups = nullptr;           // [tk_groups_pw] (first tile, tiles), small layers first
     int32_t sunits_pw = 0;                 // top-k sample units per worker
     int32_t* d_sunit_layer = nullptr;      // [sunits_pw] layer of each sample unit
     int32_t* d_sunit_part = nullptr;       // [sunits_pw] part index within the layer
@@ -92,7 +76,6 @@ struct gce_table {
     int32_t dc_tiles = 0;                  // decode tiles over all layers
     int32_t dc_slots = 0;                  // tile-bound slots per worker (tiles + L)
     int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
-    gce::DcTile* d_dc_tiles = nullptr;     // [dc_tiles] the same tiles' fields
     int32_t dc_nl_n = 0;                   // decode tiles of sparse and DENSE layers
     int32_t* d_dc_nl_tiles = nullptr;      // their decode tile ids
     int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker
@@ -102,8 +85,10 @@ struct gce_table {
     void* d_ps = nullptr;                  // PsLayer[L]
     int4* d_ps1_tiles = nullptr;           // (layer, row block, column chunk) of M Q and residual
     int32_t ps1_ntiles = 0;
+    int32_t ps1_nexact = 0;                // the first ps1_nexact of them: fp64-product layers
     int4* d_ps3_tiles = nullptr;           // (layer, row block, column chunk) of M^T P
     int32_t ps3_ntiles = 0;
+    int32_t ps3_nexact = 0;
     int4* d_psq_tiles = nullptr;           // (layer, column block) of the Q reduction
     int32_t psq_ntiles = 0;
     int32_t* d_ps_layers = nullptr;        // POWERSGD layer ids
@@ -150,6 +135,18 @@ void prof_after(cudaStream_t st);
         ::gce::count_launch();                                                   \
         const bool gce_prof_ = ::gce::g_prof_on.load(std::memory_order_relaxed); \
         if (gce_prof_) ::gce::prof_before(#kern, (stream));                      \
+        kern<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+        if (gce_prof_) ::gce::prof_after((stream));                              \
+    } while (0)
+
+// The same with the name recorded for the profile given as a string, for a
+// kernel whose template arguments hold a comma (written with GCE_COMMA).
+#define GCE_COMMA ,
+#define GCE_LAUNCH_AS(name, kern, grid, block, smem, stream, ...)               \
+    do {                                                                         \
+        ::gce::count_launch();                                                   \
+        const bool gce_prof_ = ::gce::g_prof_on.load(std::memory_order_relaxed); \
+        if (gce_prof_) ::gce::prof_before((name), (stream));                     \
         kern<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
         if (gce_prof_) ::gce::prof_after((stream));                              \
     } while (0)

@@ -313,136 +313,6 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     }
 }
 
-// ---- decode of a sparse table (top-k / rand-k and DENSE layers), W <= 32 ------------------
-// The same sums as dc_accum_kernel's staged path, with the next tile fetched
-// while the current one is added: four warps own a 1024-output span of the
-// tile each (stage its entries, add them in worker order, write it out), and
-// a fifth warp meanwhile loads the block's next tile record, its k and every
-// worker's entry range for it into the other half of a double buffer.  The
-// chain of dependent loads in front of each tile leaves the critical path.
-constexpr int kDsWarps = 4;                         // warps that add and write
-constexpr int kDsThreads = 32 * (kDsWarps + 1);     // plus the fetching warp
-
-struct DsMeta {
-    int64_t out_off, val_off;
-    int32_t kind, tt, cnt, k, total;
-};
-
-// named barrier among the adding warps only
-__device__ __forceinline__ void ds_bar() {
-    asm volatile("bar.sync 1, %0;" ::"n"(32 * kDsWarps) : "memory");
-}
-
-template <bool kApply>
-__global__ void __launch_bounds__(kDsThreads, 9) dc_sparse_kernel(
-    const DcTile* __restrict__ tiles, int32_t dc_tiles, int32_t W, int64_t vals_pw,
-    int32_t dc_slots, const int32_t* __restrict__ k_or_rank, const float* __restrict__ vals,
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ bounds, float scale,
-    float* __restrict__ out) {
-    __shared__ __align__(16) float acc[kDcTile];
-    __shared__ int32_t s_first[2][32], s_off[2][33];
-    __shared__ DsMeta s_meta[2];
-    __shared__ int32_t s_sidx[kDcStage];
-    __shared__ float s_sval[kDcStage];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // the fetching warp: tile u's record, k and entry ranges into buffer b
-    auto fetch = [&](int32_t u, int b) {
-        const DcTile d = tiles[u];
-        const bool sparse = d.kind == GCE_KIND_TOPK || d.kind == GCE_KIND_RANDK;
-        int32_t k = 0;
-        if (sparse) {
-            k = k_or_rank ? k_or_rank[d.l] : d.cap;
-            k = (k >= 1 && k <= d.cap) ? k : 0;
-        }
-        int32_t a = 0, e = 0;
-        if (sparse && lane < W) {
-            const int32_t* bb = bounds + int64_t(lane) * dc_slots + d.dc_base + d.tt;
-            a = min(max(bb[0], 0), k);
-            e = min(max(bb[1], a), k);
-            s_first[b][lane] = a;
-        }
-        const int c = e - a;
-        const int incl = warp_inclusive_scan(c);
-        if (lane < W) s_off[b][lane] = incl - c;
-        if (lane == 31) {
-            s_off[b][32] = incl;
-            s_meta[b] = DsMeta{d.out_off, d.val_off, d.kind, d.tt, d.cnt, k, incl};
-        }
-    };
-    if (warp == kDsWarps) {
-        if (int32_t(blockIdx.x) < dc_tiles) fetch(blockIdx.x, 0);
-    } else {
-        for (int i = tid; i < kDcTile / 4; i += 32 * kDsWarps)
-            reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    __syncthreads();
-    int par = 0;
-    for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
-        if (warp == kDsWarps) {
-            if (u + int32_t(gridDim.x) < dc_tiles) fetch(u + gridDim.x, par ^ 1);
-        } else {
-            const DsMeta M = s_meta[par];
-            float* o = out + M.out_off;
-            const int cnt = M.cnt;
-            if (M.kind == GCE_KIND_DENSE) {
-                for (int i = tid; i < cnt; i += 32 * kDsWarps) {
-                    float sum = 0.0f;
-                    for (int w = 0; w < W; ++w)
-                        sum = __fadd_rn(sum, vals[int64_t(w) * vals_pw + M.val_off +
-                                                  (int64_t(M.tt) << kDcTileLog) + i]);
-                    o[i] = dc_final<kApply>(sum, scale, o + i);
-                }
-            } else {
-                const int64_t start = int64_t(M.tt) << kDcTileLog;
-                const int32_t* sf = s_first[par];
-                const int32_t* so = s_off[par];
-                const int total = M.total;
-                int c0 = 0;
-                while (c0 < total) {
-                    const int cn = min(kDcStage, total - c0);
-                    if (c0 > 0) ds_bar();  // every adding warp is done with the last chunk
-                    constexpr int kSB = 8;  // loads a thread in flight, then the stores
-                    for (int q0 = 0; q0 < cn; q0 += kSB * 32 * kDsWarps) {
-                        int32_t ri[kSB];
-                        float rv[kSB];
-#pragma unroll
-                        for (int e = 0; e < kSB; ++e) {
-                            const int q = q0 + e * 32 * kDsWarps + tid;
-                            ri[e] = 0;
-                            rv[e] = 0.0f;
-                            if (q < cn) {
-                                const int qq = c0 + q;
-                                int w = 0;  // the last worker whose entries start at or before qq
-#pragma unroll
-                                for (int step = 16; step > 0; step >>= 1)
-                                    if (w + step < W && so[w + step] <= qq) w += step;
-                                const int64_t o2 = int64_t(w) * vals_pw + M.val_off + sf[w] + (qq - so[w]);
-                                ri[e] = idx[o2];
-                                rv[e] = vals[o2];
-                            }
-                        }
-#pragma unroll
-                        for (int e = 0; e < kSB; ++e) {
-                            const int q = q0 + e * 32 * kDsWarps + tid;
-                            if (q < cn) {
-                                s_sidx[q] = int32_t(int64_t(ri[e]) - start);
-                                s_sval[q] = rv[e];
-                            }
-                        }
-                    }
-                    ds_bar();
-                    dc_add_staged(acc, s_sidx, s_sval, so, c0, cn, W, warp, cnt);
-                    c0 += kDcStage;
-                }
-                __syncwarp();
-                dc_write_quarter<kApply>(acc, o, cnt, warp, scale, (M.out_off & 3) == 0);
-            }
-        }
-        __syncthreads();  // the next tile's buffer is complete; this tile's is free
-        par ^= 1;
-    }
-}
-
 // Decode of a SIGN table (SIGN and DENSE layers), one 4096-output tile per
 // block.  The tile's sign words of up to 32 workers at a time are staged in
 // shared memory (128 words a worker) with their scales; each thread then forms
@@ -562,21 +432,6 @@ static int launch_decode_t(const gce_table* t, int32_t W, const float* vals, con
         GCE_LAUNCH(dc_bounds_kernel, wave_grid(units, 8, r_bounds), 256, 0, st, t->d_layers,
                    t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
                    k_or_rank, idx, bounds);
-    }
-    if (sparse && W <= 32) {
-        static const int r_sp = resident_blocks(dc_sparse_kernel<kApply>, kDsThreads);
-        if (t->dc_tiles > 0) {
-            const int grid = wave_grid(t->dc_tiles, 16, r_sp);
-            if (kApply)
-                GCE_LAUNCH(dc_sparse_kernel<true>, grid, kDsThreads, 0, st, t->d_dc_tiles,
-                           t->dc_tiles, W, t->vals_pw, t->dc_slots, k_or_rank, vals, idx, bounds,
-                           scale, out);
-            else
-                GCE_LAUNCH(dc_sparse_kernel<false>, grid, kDsThreads, 0, st, t->d_dc_tiles,
-                           t->dc_tiles, W, t->vals_pw, t->dc_slots, k_or_rank, vals, idx, bounds,
-                           scale, out);
-        }
-        return check_launch();
     }
     // PowerSGD layers by their own tiled kernel when it takes them (then the
     // element-wise kernel covers only the other layers' tiles)

@@ -42,6 +42,16 @@ constexpr int kPsQB = 256;    // columns per Q-reduction tile
 constexpr int64_t kPsTallRows = 8192;  // taller P: Gram-Schmidt spread over many blocks
 constexpr int kPsOrthChunk = 1024;     // rows per block in that case
 
+// Precision of a layer's products.  Layers of at most kPsExactMax elements
+// form M Q, M^T P and the residual in fp64, from the fp64 orthonormal P and
+// Q' (the oracle's arithmetic up to the order of fp64 sums); their tiles come
+// first in the tile lists, and each precision has its own kernel instances.  B200's CUDA
+// cores run fp64 at about 1/32 of the fp32 rate, which would make a larger,
+// bandwidth-bound layer ALU-bound; larger layers form the products in fp32
+// (per lane, from the fp32-rounded P and Q' the payload carries) and every
+// sum across lanes, chunks and row blocks in fp64.
+constexpr int64_t kPsExactMax = int64_t(1) << 22;
+
 struct PsLayer {
     int64_t ppart_off;  // floats: nch1 x rows x cap partial P
     int64_t pd_off;     // doubles: rows x cap
@@ -55,7 +65,7 @@ struct PsLayer {
 
 int powersgd_plan(gce_table* t) {
     std::vector<PsLayer> ps(t->L);
-    std::vector<int4> t1, t3, tq;
+    std::vector<int4> t1, t3, tq, t1f, t3f;
     std::vector<int2> tall_units;
     std::vector<int32_t> ids;
     int64_t pp = 0, pd = 0, qp = 0;
@@ -81,16 +91,24 @@ int powersgd_plan(gce_table* t) {
             pp += int64_t(x.nch1) * L.rows * L.cap;
             pd += L.rows * L.cap;
             qp += int64_t(x.nrb3) * L.cols * L.cap;
+            // tiles of the fp64-product layers first, then the others
+            const bool exact = L.n <= kPsExactMax;
+            std::vector<int4>& o1 = exact ? t1 : t1f;
+            std::vector<int4>& o3 = exact ? t3 : t3f;
             for (int32_t rb = 0; rb < (L.rows + kPsRB - 1) / kPsRB; ++rb)
-                for (int32_t ch = 0; ch < x.nch1; ++ch) t1.push_back(make_int4(l, rb, ch, 0));
+                for (int32_t ch = 0; ch < x.nch1; ++ch) o1.push_back(make_int4(l, rb, ch, 0));
             for (int32_t rb = 0; rb < x.nrb3; ++rb)
-                for (int32_t ch = 0; ch < x.nch1; ++ch) t3.push_back(make_int4(l, rb, ch, 0));
+                for (int32_t ch = 0; ch < x.nch1; ++ch) o3.push_back(make_int4(l, rb, ch, 0));
             for (int32_t cb = 0; cb < (L.cols + kPsQB - 1) / kPsQB; ++cb)
                 tq.push_back(make_int4(l, cb, 0, 0));
             ids.push_back(l);
         }
         ps[l] = x;
     }
+    t->ps1_nexact = int32_t(t1.size());
+    t->ps3_nexact = int32_t(t3.size());
+    t1.insert(t1.end(), t1f.begin(), t1f.end());
+    t3.insert(t3.end(), t3f.begin(), t3f.end());
     t->ppart_pw = pp;
     t->pd_pw = pd;
     t->qpart_pw = qp;
@@ -197,14 +215,6 @@ __global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
     }
 }
 
-// Precision of a layer's products.  Layers of at most kPsExactMax elements
-// form M Q, M^T P and the residual in fp64, from the fp64 orthonormal P and
-// Q' (the oracle's arithmetic up to the order of fp64 sums).  B200's CUDA
-// cores run fp64 at about 1/32 of the fp32 rate, which would make a larger,
-// bandwidth-bound layer ALU-bound; larger layers form the products in fp32
-// (per lane, from the fp32-rounded P and Q' the payload carries) and every
-// sum across lanes, chunks and row blocks in fp64.
-constexpr int64_t kPsExactMax = int64_t(1) << 22;
 
 // The residual of one entry: m = fl32(M - sum_j P_j Q'_j), the sum formed
 // as a product of column 0 then fused multiply-adds in column order -- in
@@ -293,12 +303,18 @@ __device__ __forceinline__ void ps_stage(T (*dst)[kPsCB], const double* src, int
     }
 }
 
+template <class T>
 constexpr size_t ps_mq_smem(bool lazy) {
-    return lazy ? sizeof(double) * (2 * kMaxRank * kPsCB + kPsRB * kMaxRank)
-                : sizeof(double) * kMaxRank * kPsCB;
+    return lazy ? sizeof(T) * (2 * kMaxRank * kPsCB + kPsRB * kMaxRank)
+                : sizeof(T) * kMaxRank * kPsCB;
 }
 constexpr size_t kPsResidSmem = sizeof(double) * (kMaxRank * kPsCB + kPsRB * kMaxRank) +
                                 sizeof(float) * (kMaxRank * kPsCB + kPsRB * kMaxRank);
+
+template <class T>
+constexpr const char* ps_prec_name(const char* d, const char* f) {
+    return std::is_same<T, double>::value ? d : f;
+}
 
 // ---- phase 1: M = m + eta*g (written back), partial P = M Q -------------------------------
 // Products in the layer's precision (kPsExactMax), sums across lanes and
@@ -308,7 +324,7 @@ constexpr size_t kPsResidSmem = sizeof(double) * (kMaxRank * kPsCB + kPsRB * kMa
 // the residual itself); the residual m is formed on the fly, entry by entry
 // as the residual pass would have formed it, so the results are the eager
 // step's bit for bit without that pass's read and write of M.
-template <bool kLazy>
+template <bool kLazy, class T>
 __global__ void __launch_bounds__(256) ps_mq_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t Q_pw,
@@ -338,12 +354,10 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
         const int cw = int(min64(kPsCB, C - c0));
         const int64_t r0 = int64_t(d.y) * kPsRB;
         const int rh = int(min64(kPsRB, R - r0));
-        const bool exact = L.n <= kPsExactMax;
         const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
         // shared memory: the warm start Q, then (lazy) the previous Q' and
-        // the previous P rows, in the layer's precision
-        auto tile = [&](auto zero) {
-            using T = decltype(zero);
+        // the previous P rows, in the layer's precision T
+        {
             T (*qs)[kPsCB] = reinterpret_cast<T (*)[kPsCB]>(ps_dyn);
             T (*qdp)[kPsCB] = qs + kMaxRank;
             T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(qdp + kMaxRank);
@@ -382,9 +396,7 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
                     ppart[int64_t(w) * ppart_pw + X.ppart_off + (int64_t(d.z) * R + r0 + row) * cap + lane] = a;
                 }
             }
-        };
-        if (exact) tile(0.0);
-        else tile(0.0f);
+        }
         __syncthreads();
     }
 }
@@ -596,6 +608,7 @@ static std::vector<PsOrthOp> ps_orth_ops(int cap) {
 // From the orthonormal P of the workspace: products in the layer's
 // precision (fp64, or fp32 from the P the payload carries), the partial of
 // each 64-row block stored in fp64.
+template <class T>
 __global__ void __launch_bounds__(256) ps_mtp_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t pd_pw,
@@ -621,8 +634,7 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
         const int64_t ebase = int64_t(w) * N + L.offset + r0 * C + c0;
         const bool vec = ((ebase & 3) == 0) && ((C & 3) == 0) && (cc + 3 < cw);
         double* out = qpart + int64_t(w) * qpart_pw + X.qpart_off + (int64_t(d.y) * C + c0 + cc) * cap;
-        auto tile = [&](auto zero) {
-            using T = decltype(zero);
+        {
             T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(&prow_d[0][0]);
             for (int i = tid; i < rh * kMaxRank; i += blockDim.x) {
                 const int row = i / kMaxRank, j = i % kMaxRank;
@@ -663,9 +675,7 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
                         for (int j = 0; j < kMaxRank; ++j)
                             if (j < r) out[q * cap + j] = double(acc[q][j]);
             }
-        };
-        if (L.n <= kPsExactMax) tile(0.0);
-        else tile(0.0f);
+        }
         __syncthreads();
     }
 }
@@ -787,6 +797,7 @@ __global__ void __launch_bounds__(256) ps_vmean_kernel(
 // order), so dense_out is the decode.
 // rank_wl (nullable): per (worker, layer) ranks [W][L_all] instead of
 // k_or_rank -- the lazy step's record, for gce_materialize_memory.
+template <class T>
 __global__ void __launch_bounds__(256) ps_resid_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t P_pw,
@@ -832,8 +843,7 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
                 prow32[row][j] = p[int64_t(row) * cap + j];
             }
         }
-        auto tile = [&](auto zero) {
-            using T = decltype(zero);
+        {
             T (*qd)[kPsCB] = reinterpret_cast<T (*)[kPsCB]>(ps_dyn);
             T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(ps_dyn + kMaxRank * kPsCB);
             ps_stage<T>(qd, qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap, cw, r, cap);
@@ -881,9 +891,7 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
                     }
                 }
             }
-        };
-        if (L.n <= kPsExactMax) tile(0.0);
-        else tile(0.0f);
+        }
         __syncthreads();
     }
 }
@@ -1002,6 +1010,94 @@ bool launch_lowrank_decode(const gce_table* t, int32_t W, const int32_t* k_or_ra
     return true;
 }
 
+// ---- launches over both precisions: the fp64-product layers' tiles come first ------------
+template <bool kLazy, class T>
+static void ps_launch_mq_part(const gce_table* t, const int4* tiles, int32_t n, int32_t W,
+                              int64_t Q_pw, const float* grad, float* mem, float eta,
+                              const int32_t* k_or_rank, const float* Q, double* ppart,
+                              int32_t* status, const double* pd, int64_t pd_pw, const double* qd,
+                              const int32_t* lazy_rank, cudaStream_t st) {
+    if (n <= 0) return;
+    static const int r = resident_blocks_smem(ps_mq_kernel<kLazy GCE_COMMA T>, 256,
+                                              ps_mq_smem<T>(kLazy));
+    GCE_LAUNCH_AS(kLazy ? ps_prec_name<T>("ps_mq_kernel<lazy,f64>", "ps_mq_kernel<lazy,f32>")
+                        : ps_prec_name<T>("ps_mq_kernel<f64>", "ps_mq_kernel<f32>"),
+                  ps_mq_kernel<kLazy GCE_COMMA T>, wave_grid(int64_t(n) * W, 8, r), 256,
+                  ps_mq_smem<T>(kLazy), st, t->d_layers, static_cast<const PsLayer*>(t->d_ps),
+                  tiles, n, W, t->N, Q_pw, t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart,
+                  status, pd, pd_pw, qd, t->L, lazy_rank);
+}
+
+// M Q pass (and the memory's M) over every PowerSGD tile; Q_pw 0: one Q for
+// every worker.  lazy_rank non-null: the lazy first pass.
+static void ps_launch_mq(const gce_table* t, int32_t W, int64_t Q_pw, const float* grad,
+                         float* mem, float eta, const int32_t* k_or_rank, const float* Q,
+                         double* ppart, int32_t* status, const double* pd, int64_t pd_pw,
+                         const double* qd, const int32_t* lazy_rank, cudaStream_t st) {
+    const int32_t nx = t->ps1_nexact, nf = t->ps1_ntiles - nx;
+    const int4* tx = t->d_ps1_tiles;
+    const int4* tf = t->d_ps1_tiles + nx;
+    if (lazy_rank) {
+        ps_launch_mq_part<true, double>(t, tx, nx, W, Q_pw, grad, mem, eta, k_or_rank, Q, ppart,
+                                        status, pd, pd_pw, qd, lazy_rank, st);
+        ps_launch_mq_part<true, float>(t, tf, nf, W, Q_pw, grad, mem, eta, k_or_rank, Q, ppart,
+                                       status, pd, pd_pw, qd, lazy_rank, st);
+    } else {
+        ps_launch_mq_part<false, double>(t, tx, nx, W, Q_pw, grad, mem, eta, k_or_rank, Q,
+                                         ppart, status, pd, pd_pw, qd, lazy_rank, st);
+        ps_launch_mq_part<false, float>(t, tf, nf, W, Q_pw, grad, mem, eta, k_or_rank, Q, ppart,
+                                        status, pd, pd_pw, qd, lazy_rank, st);
+    }
+}
+
+template <class T>
+static void ps_launch_mtp_part(const gce_table* t, const int4* tiles, int32_t n, int32_t W,
+                               int64_t pd_pw, const float* mem, const int32_t* k_or_rank,
+                               const double* pd, double* qpart, cudaStream_t st) {
+    if (n <= 0) return;
+    static const int r = resident_blocks(ps_mtp_kernel<T>, 256);
+    GCE_LAUNCH_AS(ps_prec_name<T>("ps_mtp_kernel<f64>", "ps_mtp_kernel<f32>"), ps_mtp_kernel<T>,
+                  wave_grid(int64_t(n) * W, 8, r), 256, 0, st, t->d_layers,
+                  static_cast<const PsLayer*>(t->d_ps), tiles, n, W, t->N, pd_pw, t->qpart_pw,
+                  mem, k_or_rank, pd, qpart);
+}
+
+// partial Q = M^T P over every PowerSGD tile; pd_pw 0: one P for every worker
+static void ps_launch_mtp(const gce_table* t, int32_t W, int64_t pd_pw, const float* mem,
+                          const int32_t* k_or_rank, const double* pd, double* qpart,
+                          cudaStream_t st) {
+    const int32_t nx = t->ps3_nexact;
+    ps_launch_mtp_part<double>(t, t->d_ps3_tiles, nx, W, pd_pw, mem, k_or_rank, pd, qpart, st);
+    ps_launch_mtp_part<float>(t, t->d_ps3_tiles + nx, t->ps3_ntiles - nx, W, pd_pw, mem,
+                              k_or_rank, pd, qpart, st);
+}
+
+template <class T>
+static void ps_launch_resid_part(const gce_table* t, const int4* tiles, int32_t n, int32_t W,
+                                 int64_t P_pw, int64_t Q_pw, int64_t pd_pw,
+                                 const int32_t* k_or_rank, const float* P, const float* Q,
+                                 const double* pd, const double* qd, float* mem,
+                                 float* dense_out, const int32_t* rank_wl, cudaStream_t st) {
+    if (n <= 0) return;
+    static const int r = resident_blocks_smem(ps_resid_kernel<T>, 256, kPsResidSmem);
+    GCE_LAUNCH_AS(ps_prec_name<T>("ps_resid_kernel<f64>", "ps_resid_kernel<f32>"),
+                  ps_resid_kernel<T>, wave_grid(int64_t(n) * W, 8, r), 256, kPsResidSmem, st,
+                  t->d_layers, static_cast<const PsLayer*>(t->d_ps), tiles, n, W, t->N, P_pw,
+                  Q_pw, pd_pw, k_or_rank, P, Q, pd, qd, mem, dense_out, rank_wl, t->L);
+}
+
+// m <- M - P Q^T over every PowerSGD tile (rank_wl: the lazy record)
+static void ps_launch_resid(const gce_table* t, int32_t W, int64_t P_pw, int64_t Q_pw,
+                            int64_t pd_pw, const int32_t* k_or_rank, const float* P,
+                            const float* Q, const double* pd, const double* qd, float* mem,
+                            float* dense_out, const int32_t* rank_wl, cudaStream_t st) {
+    const int32_t nx = t->ps1_nexact;
+    ps_launch_resid_part<double>(t, t->d_ps1_tiles, nx, W, P_pw, Q_pw, pd_pw, k_or_rank, P, Q,
+                                 pd, qd, mem, dense_out, rank_wl, st);
+    ps_launch_resid_part<float>(t, t->d_ps1_tiles + nx, t->ps1_ntiles - nx, W, P_pw, Q_pw,
+                                pd_pw, k_or_rank, P, Q, pd, qd, mem, dense_out, rank_wl, st);
+}
+
 }  // namespace gce
 
 using namespace gce;
@@ -1037,25 +1133,11 @@ static int ps_step(const gce_table* t, int32_t W, const float* grad, float* mem,
         double* qpart = at<double>(ws, lay.qpart);
         double* qd = at<double>(ws, lay.qd);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_mq = resident_blocks_smem(ps_mq_kernel<false>, 256, ps_mq_smem(false));
-        static const int r_mql = resident_blocks_smem(ps_mq_kernel<true>, 256, ps_mq_smem(true));
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
-        static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
-        static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
-        if (lazy_rank)
-            GCE_LAUNCH(ps_mq_kernel<true>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mql), 256,
-                       ps_mq_smem(true), st,
-                       t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw,
-                       t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, pd, t->pd_pw, qd,
-                       t->L, lazy_rank);
-        else
-            GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256,
-                       ps_mq_smem(false), st,
-                       t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->Q_pw,
-                       t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, nullptr,
-                       int64_t(0), nullptr, t->L, nullptr);
+        ps_launch_mq(t, W, t->Q_pw, grad, mem, eta, k_or_rank, Q, ppart, status, pd, t->pd_pw, qd,
+                     lazy_rank, st);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, 1, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
@@ -1068,19 +1150,15 @@ static int ps_step(const gce_table* t, int32_t W, const float* grad, float* mem,
                            k_or_rank, ppart, pd, at<double>(ws, lay.tparts),
                            at<double>(ws, lay.tscal), tdone, P);
         }
-        GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
-                   t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, t->pd_pw, t->qpart_pw,
-                   mem, k_or_rank, pd, qpart);
+        ps_launch_mtp(t, W, t->pd_pw, mem, k_or_rank, pd, qpart, st);
         GCE_LAUNCH(ps_qred_kernel<false>, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0,
                    st, t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
                    k_or_rank, qpart, Q, qd, nullptr, 1.0f);
         // the lazy step leaves M in the memory: the next step (or
         // gce_materialize_memory) takes P Q^T off
         if (!lazy_rank)
-            GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
-                       kPsResidSmem, st,
-                       t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw,
-                       t->pd_pw, k_or_rank, P, Q, pd, qd, mem, dense_out, nullptr, t->L);
+            ps_launch_resid(t, W, t->P_pw, t->Q_pw, t->pd_pw, k_or_rank, P, Q, pd, qd, mem,
+                            dense_out, nullptr, st);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);
@@ -1113,12 +1191,9 @@ extern "C" int gce_materialize_memory(const gce_table* t, int32_t W, float* mem,
     if (ws_bytes < lay.total) return GCE_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (t->nps > 0) {
-        static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
-        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
-                       kPsResidSmem, st,
-                   t->d_layers, static_cast<const PsLayer*>(t->d_ps), t->d_ps1_tiles,
-                   t->ps1_ntiles, W, t->N, t->P_pw, t->Q_pw, t->pd_pw, nullptr, nullptr, nullptr,
-                   at<double>(ws, lay.pd), at<double>(ws, lay.qd), mem, nullptr, lazy_rank, t->L);
+        ps_launch_resid(t, W, t->P_pw, t->Q_pw, t->pd_pw, nullptr, nullptr, nullptr,
+                        at<double>(ws, lay.pd), at<double>(ws, lay.qd), mem, nullptr, lazy_rank,
+                        st);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     if (cudaMemsetAsync(lazy_rank, 0, sizeof(int32_t) * size_t(W) * size_t(t->L), st) !=
@@ -1151,18 +1226,12 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         float* qloc = at<float>(ws, lay.qloc);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_mq = resident_blocks_smem(ps_mq_kernel<false>, 256, ps_mq_smem(false));
         static const int r_orth = resident_blocks(ps_orth_kernel, 256);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
-        static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<true>, 256);
-        static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
         // every worker reads the shared warm start Q (stride 0)
-        GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256,
-                   ps_mq_smem(false), st,
-                   t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0),
-                   t->ppart_pw, grad, mem, eta, k_or_rank, Q, ppart, status, nullptr, int64_t(0),
-                   nullptr, t->L, nullptr);
+        ps_launch_mq(t, W, int64_t(0), grad, mem, eta, k_or_rank, Q, ppart, status, nullptr,
+                     int64_t(0), nullptr, nullptr, st);
         // one P per layer from the partials of all W workers
         GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank,
@@ -1176,17 +1245,13 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
                            at<double>(ws, lay.tscal), tdone, P);
         }
         // Q_w = M_w^T P for every worker with the shared P (stride 0)
-        GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
-                   t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, int64_t(0),
-                   t->qpart_pw, mem, k_or_rank, pd, qpart);
+        ps_launch_mtp(t, W, int64_t(0), mem, k_or_rank, pd, qpart, st);
         GCE_LAUNCH(ps_qred_kernel<true>, wave_grid(t->psq_ntiles, 8, r_qred), 256, 0, st,
                    t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
                    k_or_rank, qpart, qloc, qd, Q, inv_w);
         // each worker's error against its own Q_w (the shared fp64 P, stride 0)
-        GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
-                       kPsResidSmem, st,
-                   t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->Q_pw,
-                   int64_t(0), k_or_rank, P, qloc, pd, qd, mem, nullptr, nullptr, t->L);
+        ps_launch_resid(t, W, int64_t(0), t->Q_pw, int64_t(0), k_or_rank, P, qloc, pd, qd, mem,
+                        nullptr, nullptr, st);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     if (t->dtiles_pw > 0) {
@@ -1226,12 +1291,9 @@ extern "C" int powersgd_dp_encode(const gce_table* t, int32_t W, const float* gr
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int32_t* status = static_cast<int32_t*>(ws);
     if (t->nps > 0) {
-        static const int r_mq = resident_blocks_smem(ps_mq_kernel<false>, 256, ps_mq_smem(false));
         // every worker reads the shared warm start Q (stride 0)
-        GCE_LAUNCH(ps_mq_kernel<false>, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_mq), 256,
-                   ps_mq_smem(false), st, t->d_layers, static_cast<const PsLayer*>(t->d_ps),
-                   t->d_ps1_tiles, t->ps1_ntiles, W, t->N, int64_t(0), t->ppart_pw, grad, mem,
-                   eta, k_or_rank, Q, Ppart, status, nullptr, int64_t(0), nullptr, t->L, nullptr);
+        ps_launch_mq(t, W, int64_t(0), grad, mem, eta, k_or_rank, Q, Ppart, status, nullptr,
+                     int64_t(0), nullptr, nullptr, st);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     // DENSE layers: each worker's residual as its payload row, memory -> 0
@@ -1286,21 +1348,15 @@ extern "C" int powersgd_dp_project(const gce_table* t, int32_t W, float* mem,
     double* pd = at<double>(ws, lay.pd);
     double* qpart = at<double>(ws, lay.qpart);
     double* qd = at<double>(ws, lay.qd);
-    static const int r_mtp = resident_blocks(ps_mtp_kernel, 256);
     static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
-    static const int r_resid = resident_blocks_smem(ps_resid_kernel, 256, kPsResidSmem);
     // Q_w = M_w^T P for this rank's workers with the shared P (stride 0)
-    GCE_LAUNCH(ps_mtp_kernel, wave_grid(int64_t(t->ps3_ntiles) * W, 8, r_mtp), 256, 0, st,
-               t->d_layers, ps, t->d_ps3_tiles, t->ps3_ntiles, W, t->N, int64_t(0), t->qpart_pw,
-               mem, k_or_rank, pd, qpart);
+    ps_launch_mtp(t, W, int64_t(0), mem, k_or_rank, pd, qpart, st);
     GCE_LAUNCH(ps_qred_kernel<false>, wave_grid(int64_t(t->psq_ntiles) * W, 8, r_qred), 256, 0,
                st, t->d_layers, ps, t->d_psq_tiles, t->psq_ntiles, W, t->Q_pw, t->qpart_pw,
                k_or_rank, qpart, Qw, qd, nullptr, 1.0f);
     // each worker's error against its own Q_w
-    GCE_LAUNCH(ps_resid_kernel, wave_grid(int64_t(t->ps1_ntiles) * W, 8, r_resid), 256,
-               kPsResidSmem, st, t->d_layers, ps, t->d_ps1_tiles, t->ps1_ntiles, W, t->N,
-               int64_t(0), t->Q_pw, int64_t(0), k_or_rank, nullptr, nullptr, pd, qd, mem,
-               nullptr, nullptr, t->L);
+    ps_launch_resid(t, W, int64_t(0), t->Q_pw, int64_t(0), k_or_rank, nullptr, nullptr, pd, qd,
+                    mem, nullptr, nullptr, st);
     return check_launch();
 }
 

@@ -158,13 +158,11 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_dense);
     cudaFree(t->d_tile_layer);
     cudaFree(t->d_tile_info);
-    cudaFree(t->d_tk_groups);
     cudaFree(t->d_sunit_layer);
     cudaFree(t->d_sunit_part);
     cudaFree(t->d_dtile_layer);
     cudaFree(t->d_dtile_start);
     cudaFree(t->d_dc_tile_layer);
-    cudaFree(t->d_dc_tiles);
     cudaFree(t->d_dc_nl_tiles);
     cudaFree(t->d_bunit_layer);
     cudaFree(t->d_bunit_chunk);
@@ -194,7 +192,6 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     std::vector<int32_t> tile_layer, sunit_layer, sunit_part, dtile_layer, dtile_start;
     std::vector<TileInfo> tile_info;
     std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_nl;
-    std::vector<DcTile> dc_tile_info;
     int32_t dc_tiles = 0, dc_slots = 0;
     for (int32_t l = 0; l < L; ++l) {
         const gce_layer_desc& d = descs[l];
@@ -270,17 +267,6 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
         for (int32_t i = 0; i < x.dc_ntiles; ++i) {
             if (d.kind != GCE_KIND_POWERSGD) dc_nl.push_back(dc_tiles + i);
             dc_tile_layer.push_back(l);
-            const int64_t start = int64_t(i) << kDcTileLog;
-            DcTile dt{};
-            dt.out_off = x.offset + start;
-            dt.val_off = x.val_off;
-            dt.l = l;
-            dt.tt = i;
-            dt.cnt = int32_t(std::min<int64_t>(kDcTile, n - start));
-            dt.kind = d.kind;
-            dt.dc_base = x.dc_base;
-            dt.cap = d.cap;
-            dc_tile_info.push_back(dt);
         }
         dc_tiles += x.dc_ntiles;
         dc_slots += x.dc_ntiles + 1;
@@ -300,22 +286,6 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     t->Q_pw = qoff;
     t->comp_N = spoff;
     t->tiles_pw = tiles;
-    // top-k emit items: runs of up to kTkGroup consecutive tiles of one layer,
-    // layers in ascending size (their selections finish first), each layer's
-    // runs in tile order
-    std::vector<int2> tk_groups;
-    if (t->ckind == GCE_KIND_TOPK) {
-        std::vector<int32_t> order(t->comp);
-        std::stable_sort(order.begin(), order.end(), [&](int32_t a, int32_t b) {
-            return t->layers[a].n < t->layers[b].n;
-        });
-        for (int32_t l : order) {
-            const DevLayer& x = t->layers[l];
-            for (int32_t i = 0; i < x.ntiles; i += kTkGroup)
-                tk_groups.push_back(make_int2(x.tile0 + i, std::min(kTkGroup, x.ntiles - i)));
-        }
-    }
-    t->tk_groups_pw = int32_t(tk_groups.size());
     t->sunits_pw = int32_t(sunit_layer.size());
     t->dtiles_pw = int32_t(dtile_layer.size());
     t->dc_tiles = dc_tiles;
@@ -327,13 +297,11 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_dense, t->dense);
     if (rc == GCE_OK) rc = upload(&t->d_tile_layer, tile_layer);
     if (rc == GCE_OK) rc = upload(&t->d_tile_info, tile_info);
-    if (rc == GCE_OK) rc = upload(&t->d_tk_groups, tk_groups);
     if (rc == GCE_OK) rc = upload(&t->d_sunit_layer, sunit_layer);
     if (rc == GCE_OK) rc = upload(&t->d_sunit_part, sunit_part);
     if (rc == GCE_OK) rc = upload(&t->d_dtile_layer, dtile_layer);
     if (rc == GCE_OK) rc = upload(&t->d_dtile_start, dtile_start);
     if (rc == GCE_OK) rc = upload(&t->d_dc_tile_layer, dc_tile_layer);
-    if (rc == GCE_OK) rc = upload(&t->d_dc_tiles, dc_tile_info);
     t->dc_nl_n = int32_t(dc_nl.size());
     if (rc == GCE_OK) rc = upload(&t->d_dc_nl_tiles, dc_nl);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_layer, bunit_layer);

@@ -5,7 +5,7 @@
 // is the k largest |v| (ties -> lower index), emitted in ascending index;
 // the memory keeps v except on the chosen set, where it becomes +0.
 //
-// Design (each launch covers every (worker, layer) of the table):
+// Design (one launch per phase over every (worker, layer) of the table):
 //   setup    per-layer k, clear counters and histograms
 //   sample   read one 128-byte run of grad/mem per 4096 elements, histogram
 //            the |v| keys and, interpolating inside the crossing bins, pick
@@ -21,14 +21,12 @@
 //            to the exact fallback; histogram work is cut into units
 //   restore  + respill  the fallback: memory zeroed above hi gets v back
 //            from the candidate list, then the layer is re-listed whole
-//   select   one launch whose blocks take work items from a queue: three
-//            11/11/9-bit radix levels over the candidate values find the exact
-//            k-th largest key T and how many keys equal to T to take (each
-//            level's units wait only for their own layer's previous level),
-//            then emit items count key > T and key == T per tile, chain the
-//            counts along the layer (decoupled look-back) and write (v, i) in
-//            index order; memory +0 for chosen entries at or below hi, v again
-//            for entries above hi that were not chosen
+//   hist1-3  three 11/11/9-bit radix levels over the candidate values find
+//            the exact k-th largest key T and how many keys equal to T to take
+//   count / scan / emit   per-tile counts of key > T and key == T, a prefix
+//            over the tiles, then the ordered write of (v, i); memory +0 for
+//            chosen entries at or below hi, v again for entries above hi that
+//            were not chosen
 // Results never depend on lo or hi.  DRAM traffic: 12 B per element (read
 // grad and mem, write mem) plus about 8 B per candidate (about 1.5 % of the
 // elements), the payload, and a few scattered memory writes.
@@ -42,8 +40,9 @@ namespace gce {
 
 struct TkLayout {
     int64_t S = 0, TT = 0;
-    size_t segs = 0, hists = 0, gstate = 0, counter = 0, zero_end = 0, unit_start = 0,
-           unit_seg = 0, redo_list = 0, tile_dir = 0, spill_v = 0, spill_i = 0, total = 0;
+    size_t segs = 0, hists = 0, unit_start = 0, unit_seg = 0, redo_list = 0, tile_dir = 0,
+           tile_cnt = 0,
+           spill_v = 0, spill_i = 0, total = 0;
 };
 
 static TkLayout tk_layout(const gce_table* t, int32_t W) {
@@ -53,17 +52,13 @@ static TkLayout tk_layout(const gce_table* t, int32_t W) {
     o.TT = (t->ckind == GCE_KIND_TOPK) ? int64_t(W) * t->tiles_pw : 0;
     o.segs = c.take<TkSeg>(o.S);
     o.hists = c.take<int32_t>(o.S * (kTkSBins + 3 * kTkBins));
-    // the emit items' look-back words and the work counter of the select
-    // kernel, cleared together with the histograms
-    o.gstate = c.take<uint64_t>(o.S ? int64_t(W) * t->tk_groups_pw : 0);
-    o.counter = c.take<uint32_t>(o.S ? 1 : 0);
-    o.zero_end = c.off;
     o.unit_start = c.take<int32_t>(o.S + 1);
     // (segment, unit within it) of every histogram unit; a segment of n
     // candidates has ceil(n / kTkHUnit) units and n is at most the layer size
     o.unit_seg = c.take<int2>(o.S ? int64_t(W) * (t->comp_N / kTkHUnit + int64_t(t->comp.size())) : 0);
     o.redo_list = c.take<int32_t>(o.TT + 1);
     o.tile_dir = c.take<int2>(o.TT);
+    o.tile_cnt = c.take<int2>(o.TT);
     o.spill_v = c.take<float>(o.S ? int64_t(W) * t->comp_N : 0);
     o.spill_i = c.take<int32_t>(o.S ? int64_t(W) * t->comp_N : 0);
     o.total = c.off;
@@ -487,262 +482,180 @@ __global__ void __launch_bounds__(256) tk_respill_kernel(
     }
 }
 
-// ---- selection and ordered emit: one launch ---------------------------------------------
-// Blocks take work items from a counter in a fixed order: every histogram
-// unit of radix level 1, then every unit of level 2, then of level 3, then
-// every emit item (kTkGroup consecutive main tiles of one layer of one worker;
-// the smallest layers first, each layer's items in tile order, the workers of
-// one item next to each other).  An item waits only on items before it: a
-// level-L unit on its segment's level L-1 (published by that level's last
-// unit), an emit item on its segment's level 3 and on the running count of the
-// segment's previous emit item (a decoupled look-back).  Items go to running
-// blocks only, so the earliest unfinished item never waits and every wait
-// ends.  Past kTkSpinLimit polls (about a second) a wait sets
-// GCE_STATUS_WAIT_TIMEOUT and the block goes on; that call's results are not
-// valid.
-constexpr uint32_t kTkSpinLimit = 1u << 21;
-
-// Look-back word of an emit item: bits 62-63 the state (1: this item's own
-// counts, 2: the counts of every item of the segment up to and including it),
-// bits 31-61 the count of keys > T, bits 0-30 the count of keys == T.
-constexpr uint64_t kTkAgg = uint64_t(1) << 62, kTkInc = uint64_t(2) << 62;
-__device__ __forceinline__ uint64_t tk_pack(int64_t gt, int64_t eq) {
-    return (uint64_t(gt) << 31) | uint64_t(eq);
-}
-
-// thread 0: poll *p with acquire loads until it is >= v
-__device__ __forceinline__ bool tk_wait_level(const int32_t* p, int32_t v, int32_t* status) {
-    int32_t x = ld_acquire_gpu(p);
-    for (uint32_t n = 0; x < v && n < kTkSpinLimit; ++n) {
-        __nanosleep(64);
-        x = ld_acquire_gpu(p);
-    }
-    if (x >= v) return true;
-    atomicOr(status, GCE_STATUS_WAIT_TIMEOUT);
-    return false;
-}
-
-struct TkSelShared {
-    int32_t h[kTkBins];
-    int64_t item;
-    int32_t ok, last;
-    uint32_t prefix, T, hi;
-    int32_t count, need, k, nunits;
-    int32_t cnt_gt[kTkGroup], cnt_eq[kTkGroup];
-    int32_t base_gt[kTkGroup], base_eq[kTkGroup];
-};
-
-// One histogram unit of radix level kLevel (11 / 11 / 9 key bits) over a
-// segment's candidate values; the level's last unit picks the bin where the
-// count from the top reaches `need` and publishes the level.  Whole block.
+// ---- radix levels over the candidate values --------------------------------------------
 template <int kLevel>
-__device__ __forceinline__ void tk_hist_unit(int32_t u, const DevLayer* __restrict__ layers,
-                                             const int32_t* __restrict__ comp, int32_t ncomp,
-                                             int64_t S, int64_t comp_N, TkSeg* segs,
-                                             const int32_t* __restrict__ unit_start,
-                                             const int2* __restrict__ unit_seg, int32_t* hists,
-                                             const float* __restrict__ spill_v,
-                                             int32_t* status, TkSelShared& sh) {
+__global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restrict__ layers,
+                                                      const int32_t* __restrict__ comp,
+                                                      int32_t ncomp, int64_t S, int64_t comp_N,
+                                                      TkSeg* __restrict__ segs,
+                                                      const int32_t* __restrict__ unit_start,
+                                                      const int2* __restrict__ unit_seg,
+                                                      int32_t* __restrict__ hists,
+                                                      const float* __restrict__ spill_v) {
     constexpr int kNb = kLevel == 3 ? 512 : kTkBins;
     constexpr int kShift = kLevel == 1 ? 20 : (kLevel == 2 ? 9 : 0);
     constexpr int kPer = 16;  // candidates per thread per load batch
+    __shared__ int32_t h[kTkBins];
+    __shared__ int s_last;
     const int tid = threadIdx.x;
-    const int2 us = unit_seg[u];
-    const int64_t s = us.x;
-    if (tid == 0) {
-        sh.ok = kLevel == 1 || tk_wait_level(&segs[s].level, kLevel - 1, status);
-        sh.prefix = segs[s].prefix;
-        sh.count = segs[s].count;
-        sh.nunits = unit_start[s + 1] - unit_start[s];
-    }
-    for (int b = tid; b < kNb; b += blockDim.x) sh.h[b] = 0;
-    __syncthreads();
-    // a wait that ran out still counts the unit as done (adding nothing), so
-    // the level is published and nothing after it waits in vain
-    const int w = int(s / ncomp);
-    const DevLayer L = layers[comp[s % ncomp]];
-    const uint32_t prefix = sh.prefix;
-    const int32_t count = sh.count;
-    const int64_t j0 = int64_t(us.y) * kTkHUnit;
-    const int64_t j1 = sh.ok ? min64(j0 + kTkHUnit, count) : j0;
-    const float* e = spill_v + int64_t(w) * comp_N + L.sp_off;
-    for (int64_t jb = j0; jb < j1; jb += int64_t(kPer) * blockDim.x) {
-        uint32_t key[kPer];
+    const int32_t total = unit_start[S];
+    for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
+        const int2 us = unit_seg[u];
+        const int64_t s = us.x;
+        const int w = int(s / ncomp);
+        const DevLayer L = layers[comp[s % ncomp]];
+        const uint32_t prefix = segs[s].prefix;
+        const int32_t count = segs[s].count;
+        const int64_t j0 = int64_t(us.y) * kTkHUnit;
+        for (int b = tid; b < kNb; b += blockDim.x) h[b] = 0;
+        __syncthreads();
+        const float* e = spill_v + int64_t(w) * comp_N + L.sp_off;
+        for (int64_t jb = j0; jb < min64(j0 + kTkHUnit, count); jb += int64_t(kPer) * 256) {
+            uint32_t key[kPer];
 #pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            const int64_t j = jb + int64_t(q) * blockDim.x + tid;
-            key[q] = j < count ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
-        }
-#pragma unroll
-        for (int q = 0; q < kPer; ++q) {
-            bool take = key[q] != 0xFFFFFFFFu;
-            if (kLevel == 2) take = take && (key[q] >> 20) == (prefix >> 20);
-            if (kLevel == 3) take = take && (key[q] >> 9) == (prefix >> 9);
-            const uint32_t bin = (key[q] >> kShift) & (kNb - 1);
-            if (kLevel == 1) hist_add(sh.h, bin, take);   // few, crowded bins
-            else if (take) atomicAdd(&sh.h[bin], 1);
-        }
-    }
-    __syncthreads();
-    int32_t* gh = tk_hist(hists, S, kLevel, s);
-    for (int b = tid; b < kNb; b += blockDim.x)
-        if (sh.h[b]) atomicAdd(gh + b, sh.h[b]);
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        int32_t* done = kLevel == 1 ? &segs[s].done_1 : (kLevel == 2 ? &segs[s].done_2 : &segs[s].done_3);
-        sh.last = (atomicAdd(done, 1) == sh.nunits - 1);
-        if (sh.last) sh.need = segs[s].need;
-    }
-    __syncthreads();
-    if (!sh.last) return;
-    __threadfence();
-    for (int b = tid; b < kNb; b += blockDim.x) sh.h[b] = __ldcg(gh + b);
-    __syncthreads();
-    if (tid < 32) {
-        int64_t above = 0;
-        const int b = warp_find_from_top(sh.h, kNb, sh.need, &above);
-        if (tid == 0) {
-            if (b >= 0) {
-                segs[s].prefix = prefix | (uint32_t(b) << kShift);
-                segs[s].need = sh.need - int32_t(above);
+            for (int q = 0; q < kPer; ++q) {
+                const int64_t j = jb + int64_t(q) * 256 + tid;
+                key[q] = j < count ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
             }
-            st_release_gpu(&segs[s].level, kLevel);  // after the two stores above
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                bool take = key[q] != 0xFFFFFFFFu;
+                if (kLevel == 2) take = take && (key[q] >> 20) == (prefix >> 20);
+                if (kLevel == 3) take = take && (key[q] >> 9) == (prefix >> 9);
+                const uint32_t bin = (key[q] >> kShift) & (kNb - 1);
+                if (kLevel == 1) hist_add(h, bin, take);   // few, crowded bins
+                else if (take) atomicAdd(&h[bin], 1);
+            }
+        }
+        __syncthreads();
+        int32_t* gh = tk_hist(hists, S, kLevel, s);
+        for (int b = tid; b < kNb; b += blockDim.x)
+            if (h[b]) atomicAdd(gh + b, h[b]);
+        __threadfence();
+        __syncthreads();
+        if (tid == 0) {
+            int32_t* done = kLevel == 1 ? &segs[s].done_1 : (kLevel == 2 ? &segs[s].done_2 : &segs[s].done_3);
+            const int32_t nunits = unit_start[s + 1] - unit_start[s];
+            s_last = (atomicAdd(done, 1) == nunits - 1);
+        }
+        __syncthreads();
+        if (s_last) {
+            __threadfence();
+            for (int b = tid; b < kNb; b += blockDim.x) h[b] = __ldcg(gh + b);
+            __syncthreads();
+            if (tid < 32) {
+                int64_t above = 0;
+                const int32_t need = segs[s].need;
+                const int b = warp_find_from_top(h, kNb, need, &above);
+                if (tid == 0 && b >= 0) {
+                    segs[s].prefix = prefix | (uint32_t(b) << kShift);
+                    segs[s].need = need - int32_t(above);
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---- per-tile counts, prefix over tiles, ordered emit --------------------------------------
+__global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restrict__ tile_info,
+                                                       int32_t tiles_pw, int32_t W, int32_t ncomp,
+                                                       int64_t comp_N, const TkSeg* __restrict__ segs,
+                                                       const int2* __restrict__ tile_dir,
+                                                       int2* __restrict__ tile_cnt,
+                                                       const float* __restrict__ spill_v) {
+    constexpr int kBatch = 8;
+    const int lane = threadIdx.x & 31;
+    const int64_t total = int64_t(tiles_pw) * W;
+    const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
+        const int w = int(t / tiles_pw);
+        const int lt = int(t % tiles_pw);
+        const TileInfo ti = tile_info[lt];
+        const int2 d = tile_dir[t];
+        const int64_t s = int64_t(w) * ncomp + ti.sidx;
+        const int32_t k = segs[s].k;
+        int gt = 0, eq = 0;
+        if (k > 0) {
+            const uint32_t T = segs[s].prefix;
+            const float* e = spill_v + int64_t(w) * comp_N + ti.sp_off + d.x;
+            for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
+                uint32_t key[kBatch];
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    const int j = j0 + q * 32 + lane;
+                    key[q] = j < d.y ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
+                }
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    gt += key[q] != 0xFFFFFFFFu && key[q] > T;
+                    eq += key[q] == T;
+                }
+            }
+            gt = warp_sum(gt);
+            eq = warp_sum(eq);
+        }
+        if (lane == 0) tile_cnt[t] = make_int2(gt, eq);
+    }
+}
+
+__global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restrict__ layers,
+                                                       const int32_t* __restrict__ comp,
+                                                       int32_t ncomp, int64_t S, int32_t tiles_pw,
+                                                       const TkSeg* __restrict__ segs,
+                                                       int2* __restrict__ tile_cnt) {
+    __shared__ int s_warp[33];
+    for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
+        if (segs[s].k == 0) continue;
+        const int w = int(s / ncomp);
+        const DevLayer L = layers[comp[s % ncomp]];
+        int2* tc = tile_cnt + int64_t(w) * tiles_pw + L.tile0;
+        int carry_gt = 0, carry_eq = 0;
+        for (int b0 = 0; b0 < L.ntiles; b0 += blockDim.x) {
+            const int i = b0 + threadIdx.x;
+            const int2 x = i < L.ntiles ? tc[i] : make_int2(0, 0);
+            int tg = 0, te = 0;
+            const int eg = block_exclusive_scan(x.x, s_warp, &tg);
+            const int ee = block_exclusive_scan(x.y, s_warp, &te);
+            if (i < L.ntiles) tc[i] = make_int2(carry_gt + eg, carry_eq + ee);
+            carry_gt += tg;
+            carry_eq += te;
         }
     }
 }
 
-// One emit item: up to kTkGroup consecutive main tiles of one (worker, layer),
-// kTkWarpTiles consecutive tiles per warp.  Counts keys > T and == T per tile,
-// takes the segment's running counts before the item (look-back), then writes
-// the chosen (v, i) in index order, memory +0 for chosen entries at or below
-// hi and v again for entries above hi that were not chosen.  Whole block.
-constexpr int kTkSelThreads = 128;
-constexpr int kTkWarpTiles = kTkGroup / (kTkSelThreads / 32);  // 2
-
-__device__ __forceinline__ void tk_emit_item(
-    int64_t e, int32_t W, int32_t ncomp, int32_t tiles_pw, int64_t N, int64_t comp_N,
-    int64_t vals_pw, const TileInfo* __restrict__ tile_info, const int2* __restrict__ groups,
-    TkSeg* segs, const int2* __restrict__ tile_dir, const float* __restrict__ spill_v,
-    const int32_t* __restrict__ spill_i, uint64_t* gstate, float* __restrict__ mem,
-    float* __restrict__ vals, int32_t* __restrict__ idx, int32_t* status, TkSelShared& sh) {
-    constexpr int kBatch = 4;  // candidates per lane per tile in flight
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__global__ void __launch_bounds__(256) tk_emit_kernel(
+    const TileInfo* __restrict__ tile_info, int32_t tiles_pw,
+    int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, int64_t vals_pw,
+    const TkSeg* __restrict__ segs, const int2* __restrict__ tile_dir,
+    const int2* __restrict__ tile_cnt, const float* __restrict__ spill_v,
+    const int32_t* __restrict__ spill_i, float* __restrict__ mem, float* __restrict__ vals,
+    int32_t* __restrict__ idx) {
+    constexpr int kBatch = 8;
+    const int lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
-    const int64_t gi = e / W;
-    const int w = int(e - gi * W);
-    const int2 gr = groups[gi];
-    const TileInfo ti0 = tile_info[gr.x];
-    const int64_t s = int64_t(w) * ncomp + ti0.sidx;
-    if (tid == 0) {
-        sh.k = segs[s].k;
-        sh.ok = sh.k > 0 && tk_wait_level(&segs[s].level, 3, status);
-        // a wait that ran out: publish empty counts so that the segment's
-        // later items do not wait in vain (the status already marks the call)
-        if (sh.k > 0 && !sh.ok) st_release_gpu_u64(gstate + e, kTkInc);
-        sh.T = segs[s].prefix;
-        sh.need = segs[s].need;
+    const int64_t total = int64_t(tiles_pw) * W;
+    const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
+    for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
+        const int w = int(t / tiles_pw);
+        const int lt = int(t % tiles_pw);
+        const TileInfo ti = tile_info[lt];
+        const int2 d = tile_dir[t];
+        const int2 before = tile_cnt[t];    // (key > T, key == T) in earlier tiles
+        const int64_t s = int64_t(w) * ncomp + ti.sidx;
+        const int32_t k = segs[s].k;
+        if (k == 0) continue;
+        const uint32_t T = segs[s].prefix;
+        const int32_t need = segs[s].need;  // keys equal to T that are taken
         // after the fallback the memory holds v everywhere (nothing was zeroed)
-        sh.hi = segs[s].redo ? 0xFFFFFFFFu : segs[s].hi;
-    }
-    // this warp's tiles and their candidate ranges, loaded while thread 0 waits
-    int2 d[kTkWarpTiles];
-    int64_t sb[kTkWarpTiles];
-#pragma unroll
-    for (int i = 0; i < kTkWarpTiles; ++i) {
-        const int slot = warp * kTkWarpTiles + i;
-        d[i] = make_int2(0, 0);
-        if (slot < gr.y) d[i] = tile_dir[int64_t(w) * tiles_pw + gr.x + slot];
-        sb[i] = int64_t(w) * comp_N + ti0.sp_off + d[i].x;  // one layer: one candidate region
-    }
-    __syncthreads();
-    if (!sh.ok) return;
-    const uint32_t T = sh.T;
-    const int32_t k = sh.k, need = sh.need;
-    // counts of this warp's tiles
-#pragma unroll
-    for (int i = 0; i < kTkWarpTiles; ++i) {
-        int gt = 0, eq = 0;
-        for (int j0 = 0; j0 < d[i].y; j0 += 32 * kBatch) {
-            uint32_t key[kBatch];
-#pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int j = j0 + q * 32 + lane;
-                key[q] = j < d[i].y ? abs_key(__ldcg(spill_v + sb[i] + j)) : 0xFFFFFFFFu;
-            }
-#pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                gt += key[q] != 0xFFFFFFFFu && key[q] > T;
-                eq += key[q] == T;
-            }
-        }
-        gt = warp_sum(gt);
-        eq = warp_sum(eq);
-        if (lane == 0) {
-            sh.cnt_gt[warp * kTkWarpTiles + i] = gt;
-            sh.cnt_eq[warp * kTkWarpTiles + i] = eq;
-        }
-    }
-    __syncthreads();
-    if (warp == 0) {
-        int64_t ggt = 0, geq = 0;  // this item's counts
-        for (int i = 0; i < kTkGroup; ++i) {
-            ggt += sh.cnt_gt[i];
-            geq += sh.cnt_eq[i];
-        }
-        // items of the layer before this one (its first item has none)
-        const int64_t before = int64_t(ti0.tstart / kTkTile) / kTkGroup;
-        if (lane == 0) st_release_gpu_u64(gstate + e, (before ? kTkAgg : kTkInc) | tk_pack(ggt, geq));
-        // look back a warp at a time: lane i reads the item i + 1 back (W
-        // entries apart), until one has published its running counts
-        int64_t pgt = 0, peq = 0;
-        for (int64_t back = 1; back <= before; back += 32) {
-            const int64_t jj = back + lane;
-            const bool have = jj <= before;
-            uint64_t v = 0;
-            if (have) {
-                const uint64_t* src = gstate + (e - jj * W);
-                v = ld_acquire_gpu_u64(src);
-                for (uint32_t n = 0; (v >> 62) == 0 && n < kTkSpinLimit; ++n) {
-                    __nanosleep(32);
-                    v = ld_acquire_gpu_u64(src);
-                }
-                if ((v >> 62) == 0) {  // never published: counted as empty and final
-                    atomicOr(status, GCE_STATUS_WAIT_TIMEOUT);
-                    v = kTkInc;
-                }
-            }
-            const unsigned inc = __ballot_sync(kFull, have && (v >> 62) == 2);
-            const int stop = inc ? __ffs(inc) - 1 : 31;
-            const bool take = have && lane <= stop;
-            const int64_t vg = take ? int64_t((v >> 31) & 0x7FFFFFFFull) : 0;
-            const int64_t ve = take ? int64_t(v & 0x7FFFFFFFull) : 0;
-            pgt += warp_sum(vg);
-            peq += warp_sum(ve);
-            if (inc) break;
-        }
-        if (lane == 0) {
-            if (before) st_release_gpu_u64(gstate + e, kTkInc | tk_pack(pgt + ggt, peq + geq));
-            int64_t bgt = pgt, beq = peq;
-            for (int i = 0; i < kTkGroup; ++i) {
-                sh.base_gt[i] = int32_t(bgt);
-                sh.base_eq[i] = int32_t(beq);
-                bgt += sh.cnt_gt[i];
-                beq += sh.cnt_eq[i];
-            }
-        }
-    }
-    __syncthreads();
-    const uint32_t hi = sh.hi;
-    float* vout = vals + int64_t(w) * vals_pw + ti0.val_off;
-    int32_t* iout = idx + int64_t(w) * vals_pw + ti0.val_off;
-    float* m = mem + int64_t(w) * N + ti0.offset;
-#pragma unroll
-    for (int i = 0; i < kTkWarpTiles; ++i) {
-        const int slot = warp * kTkWarpTiles + i;
-        int sel_before = sh.base_gt[slot] + min(sh.base_eq[slot], need);
-        int eq_seen = sh.base_eq[slot];
-        for (int j0 = 0; j0 < d[i].y; j0 += 32 * kBatch) {
+        const uint32_t hi = segs[s].redo ? 0xFFFFFFFFu : segs[s].hi;
+        int sel_before = before.x + min(before.y, need);
+        int eq_seen = before.y;
+        const int64_t sb = int64_t(w) * comp_N + ti.sp_off + d.x;
+        float* vout = vals + int64_t(w) * vals_pw + ti.val_off;
+        int32_t* iout = idx + int64_t(w) * vals_pw + ti.val_off;
+        float* m = mem + int64_t(w) * N + ti.offset;
+        for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
             float ev[kBatch];
             int32_t ei[kBatch];
 #pragma unroll
@@ -750,14 +663,14 @@ __device__ __forceinline__ void tk_emit_item(
                 const int j = j0 + q * 32 + lane;
                 ev[q] = 0.0f;
                 ei[q] = -1;
-                if (j < d[i].y) {
-                    ev[q] = __ldcg(spill_v + sb[i] + j);
-                    ei[q] = __ldcg(spill_i + sb[i] + j);
+                if (j < d.y) {
+                    ev[q] = __ldcg(spill_v + sb + j);
+                    ei[q] = __ldcg(spill_i + sb + j);
                 }
             }
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
-                if (j0 + q * 32 >= d[i].y) break;  // the warp's remaining slots are empty
+                if (j0 + q * 32 >= d.y) break;  // the warp's remaining slots are empty
                 const bool valid = ei[q] >= 0;
                 const uint32_t key = abs_key(ev[q]);
                 const bool is_eq = valid && key == T;
@@ -777,47 +690,6 @@ __device__ __forceinline__ void tk_emit_item(
                 eq_seen += __popc(eq_mask);
             }
         }
-    }
-}
-
-__global__ void __launch_bounds__(kTkSelThreads) tk_select_kernel(
-    const DevLayer* __restrict__ layers, const int32_t* __restrict__ comp, int32_t ncomp,
-    int64_t S, int32_t W, int32_t tiles_pw, int64_t N, int64_t comp_N, int64_t vals_pw,
-    const TileInfo* __restrict__ tile_info, const int2* __restrict__ groups, int32_t groups_pw,
-    TkSeg* segs, const int32_t* __restrict__ unit_start, const int2* __restrict__ unit_seg,
-    int32_t* hists, const int2* __restrict__ tile_dir, const float* __restrict__ spill_v,
-    const int32_t* __restrict__ spill_i, uint64_t* gstate, uint32_t* counter,
-    float* __restrict__ mem, float* __restrict__ vals, int32_t* __restrict__ idx,
-    int32_t* status) {
-    __shared__ TkSelShared sh;
-    const int64_t U = unit_start[S];
-    const int64_t nitems = 3 * U + int64_t(groups_pw) * W;
-    // thread 0 takes the next item while the block works on the current one
-    // (a block holds at most one item it has not started, taken after every
-    // item it has finished, so the earliest unfinished item is always running)
-    uint32_t next = 0;
-    if (threadIdx.x == 0) next = atomicAdd(counter, 1u);
-    for (;;) {
-        if (threadIdx.x == 0) {
-            sh.item = int64_t(next);
-            if (int64_t(next) < nitems) next = atomicAdd(counter, 1u);
-        }
-        __syncthreads();
-        const int64_t it = sh.item;
-        if (it >= nitems) break;
-        if (it < U)
-            tk_hist_unit<1>(int32_t(it), layers, comp, ncomp, S, comp_N, segs, unit_start,
-                            unit_seg, hists, spill_v, status, sh);
-        else if (it < 2 * U)
-            tk_hist_unit<2>(int32_t(it - U), layers, comp, ncomp, S, comp_N, segs, unit_start,
-                            unit_seg, hists, spill_v, status, sh);
-        else if (it < 3 * U)
-            tk_hist_unit<3>(int32_t(it - 2 * U), layers, comp, ncomp, S, comp_N, segs,
-                            unit_start, unit_seg, hists, spill_v, status, sh);
-        else
-            tk_emit_item(it - 3 * U, W, ncomp, tiles_pw, N, comp_N, vals_pw, tile_info, groups,
-                         segs, tile_dir, spill_v, spill_i, gstate, mem, vals, idx, status, sh);
-        __syncthreads();  // the shared record is rewritten by the next item
     }
 }
 
@@ -848,17 +720,22 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         int2* unit_seg = at<int2>(ws, lay.unit_seg);
         int32_t* redo_list = at<int32_t>(ws, lay.redo_list);
         int2* tile_dir = at<int2>(ws, lay.tile_dir);
+        int2* tile_cnt = at<int2>(ws, lay.tile_cnt);
         float* spill_v = at<float>(ws, lay.spill_v);
         int32_t* spill_i = at<int32_t>(ws, lay.spill_i);
-        // histograms, look-back words and the work counter: one zero fill
-        const int64_t n4 = int64_t(lay.zero_end - lay.hists) / 16;
+        const int64_t n4 = lay.S * (kTkSBins + 3 * kTkBins) / 4;
 
         static const int r_setup = resident_blocks(tk_setup_kernel, 256);
         static const int r_sample = resident_blocks(tk_sample_kernel, 256);
         static const int r_main = resident_blocks(tk_main_kernel, kTkThreads);
         static const int r_restore = resident_blocks(tk_restore_kernel, 256);
         static const int r_respill = resident_blocks(tk_respill_kernel, 256);
-        static const int r_select = resident_blocks(tk_select_kernel, kTkSelThreads);
+        static const int r_h1 = resident_blocks(tk_hist_kernel<1>, 256);
+        static const int r_h2 = resident_blocks(tk_hist_kernel<2>, 256);
+        static const int r_h3 = resident_blocks(tk_hist_kernel<3>, 256);
+        static const int r_count = resident_blocks(tk_count_kernel, 256);
+        static const int r_scan = resident_blocks(tk_scan_kernel, 1024);
+        static const int r_emit = resident_blocks(tk_emit_kernel, 256);
         GCE_LAUNCH(tk_setup_kernel, wave_grid((n4 + lay.S + 255) / 256, 8, r_setup), 256, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, k_or_rank, segs, reinterpret_cast<int4*>(hists), n4,
                    status);
@@ -878,12 +755,21 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         GCE_LAUNCH(tk_respill_kernel, wave_grid(lay.TT, 4, r_respill), 256, 0, st, t->d_layers, t->d_tile_layer,
                    t->tiles_pw, ncomp, t->N, t->comp_N, segs, redo_list, tile_dir, mem, spill_v,
                    spill_i);
-        // every resident block takes items until none are left
-        GCE_LAUNCH(tk_select_kernel, wave_grid(lay.TT + lay.S, r_select, r_select), kTkSelThreads, 0, st,
-                   t->d_layers, t->d_comp, ncomp, lay.S, W, t->tiles_pw, t->N, t->comp_N,
-                   t->vals_pw, t->d_tile_info, t->d_tk_groups, t->tk_groups_pw, segs, unit_start,
-                   unit_seg, hists, tile_dir, spill_v, spill_i, at<uint64_t>(ws, lay.gstate),
-                   at<uint32_t>(ws, lay.counter), mem, vals, idx, status);
+        const int64_t hwork = lay.TT + lay.S;
+        GCE_LAUNCH(tk_hist_kernel<1>, wave_grid(hwork, 8, r_h1), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
+                   t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
+        GCE_LAUNCH(tk_hist_kernel<2>, wave_grid(hwork, 8, r_h2), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
+                   t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
+        GCE_LAUNCH(tk_hist_kernel<3>, wave_grid(hwork, 8, r_h3), 256, 0, st, t->d_layers, t->d_comp, ncomp, lay.S,
+                   t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
+        const int64_t wwork = (lay.TT + 7) / 8;  // a warp per tile
+        GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_tile_info,
+                   t->tiles_pw, W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
+        GCE_LAUNCH(tk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
+                   lay.S, t->tiles_pw, segs, tile_cnt);
+        GCE_LAUNCH(tk_emit_kernel, wave_grid(wwork, 8, r_emit), 256, 0, st, t->d_tile_info,
+                   t->tiles_pw, W, ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt,
+                   spill_v, spill_i, mem, vals, idx);
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
     }
     return launch_dense_layers(t, W, grad, mem, eta, vals, status, st);

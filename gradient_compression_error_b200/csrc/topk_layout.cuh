@@ -15,7 +15,6 @@ constexpr int kTkSampleStride = 4096;              // one run per 4096 elements
 constexpr int64_t kTkSamplePart = int64_t(1) << 20; // elements covered by one sample unit
 constexpr int64_t kTkSampleMinN = 65536;           // smaller layers: exact histogram of all
 constexpr int kTkHUnit = 16384;                    // candidates per histogram unit
-constexpr int kTkGroup = 8;                        // main tiles per emit item (a warp each)
 
 // Per (worker, layer) state of one top-k step.
 struct TkSeg {
@@ -30,8 +29,7 @@ struct TkSeg {
     uint32_t prefix;     // key bits fixed so far by the radix selection (T after level 3)
     int32_t need;        // rank still to find below the prefix; after level 3:
                          // how many keys equal to T are taken
-    int32_t level;       // radix levels finished (published with a release store)
-    int32_t pad[2];
+    int32_t pad[3];
 };
 static_assert(sizeof(TkSeg) == 64, "TkSeg is one 64-byte record");
 

@@ -147,8 +147,9 @@ def test_powersgd_split_at_its_two_sums_is_the_dp_step():
     v_a = torch.zeros(max(4, t.vals_per_worker), **f)
     ws_a = t.workspace(R, "powersgd_dp")
     g.powersgd_init_q(t, 1, 3, Q_a)
-    # the cut step: one workspace, memory row and P/Q copy per rank
-    mem_b = torch.zeros((R, t.N), **f)
+    # the cut step: one workspace, memory, P and Q per rank (a rank's buffers
+    # are its own allocations, 16-byte aligned as the calls require)
+    mem_b = [torch.zeros((1, t.N), **f) for _ in range(R)]
     Ps = [torch.zeros(max(4, t.P_per_worker), **f) for _ in range(R)]
     Qs = [Q_a.clone() for _ in range(R)]
     wss = [t.workspace(1, "powersgd_dp") for _ in range(R)]
@@ -160,13 +161,13 @@ def test_powersgd_split_at_its_two_sums_is_the_dp_step():
         prow = [torch.zeros((1, npart), dtype=torch.float64, **f) for _ in range(R)]
         vrow = [torch.zeros((1, max(4, t.vals_per_worker)), **f) for _ in range(R)]
         for r in range(R):
-            g.powersgd_dp_encode(t, 1, grad[r:r + 1], mem_b[r:r + 1], workloads.ETA, kr, Qs[r],
+            g.powersgd_dp_encode(t, 1, grad[r:r + 1].clone(), mem_b[r], workloads.ETA, kr, Qs[r],
                                  prow[r], vrow[r], wss[r])
         pall, vall = torch.cat(prow), torch.cat(vrow)          # the gathers
         qrow = [torch.zeros((1, max(4, t.Q_per_worker)), **f) for _ in range(R)]
         for r in range(R):
             g.powersgd_dp_orthogonalize(t, R, kr, pall, Ps[r], wss[r])
-            g.powersgd_dp_project(t, 1, mem_b[r:r + 1], kr, qrow[r], wss[r])
+            g.powersgd_dp_project(t, 1, mem_b[r], kr, qrow[r], wss[r])
         qall = torch.cat(qrow)
         for r in range(R):
             g.powersgd_dp_mean(t, R, kr, qall, Qs[r], vall, vals_b)
@@ -174,7 +175,7 @@ def test_powersgd_split_at_its_two_sums_is_the_dp_step():
         for r in range(R):
             assert torch.equal(Ps[r].view(torch.int32), P_a.view(torch.int32)), (s, r)
             assert torch.equal(Qs[r].view(torch.int32), Q_a.view(torch.int32)), (s, r)
-        assert torch.equal(mem_b.view(torch.int32), mem_a.view(torch.int32)), s
+        assert torch.equal(torch.cat(mem_b).view(torch.int32), mem_a.view(torch.int32)), s
         assert torch.equal(vals_b.view(torch.int32), v_a.view(torch.int32)), s
 
 
