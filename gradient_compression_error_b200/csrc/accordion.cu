@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(256) ac_norm_kernel(const DevLayer* __restrict
                                                       const int2* __restrict__ tiles, int32_t ntiles,
                                                       const float* __restrict__ grad,
                                                       double* __restrict__ part) {
+    grid_dependency_sync();
     __shared__ double s_red[8];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
@@ -122,6 +123,7 @@ __global__ void __launch_bounds__(256) ac_sumsq_kernel(const DevLayer* __restric
                                                        const int2* __restrict__ ac_layer, int32_t L,
                                                        const double* __restrict__ part,
                                                        double* __restrict__ sumsq) {
+    grid_dependency_sync();
     const int lane = threadIdx.x & 31;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t l = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); l < L; l += wstride) {
@@ -137,6 +139,7 @@ __global__ void __launch_bounds__(256) ac_decide_kernel(
     const double* __restrict__ part, const double* __restrict__ sumsq, int32_t check,
     double threshold, int32_t lvl_low, int32_t lvl_high, double* __restrict__ prev_norm,
     int32_t* __restrict__ level, double* __restrict__ cur_norm, int32_t* __restrict__ k_or_rank) {
+    grid_dependency_sync();
     const int lane = threadIdx.x & 31;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t l = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); l < L; l += wstride) {
@@ -170,6 +173,7 @@ __global__ void __launch_bounds__(256) ac_decide_kernel(
 }
 
 __global__ void ac_init_kernel(int32_t L, double* __restrict__ prev_norm, int32_t* __restrict__ level) {
+    grid_dependency_sync();
     for (int32_t l = blockIdx.x * blockDim.x + threadIdx.x; l < L; l += gridDim.x * blockDim.x) {
         prev_norm[l] = -1.0;
         level[l] = GCE_LEVEL_LOW;

@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <utility>
 #include <cstddef>
 #include <cstdint>
 #include <mutex>
@@ -130,12 +131,37 @@ extern std::atomic<bool> g_prof_on;
 void prof_before(const char* name, cudaStream_t st);
 void prof_after(cudaStream_t st);
 
+// Every kernel of the library is launched with programmatic stream
+// serialisation allowed: its blocks may be scheduled while the kernel before
+// it in the stream drains, and each kernel's first statement,
+// grid_dependency_sync(), holds them until that kernel has completed and its
+// writes are visible.  The setting is read once from the environment
+// (GCE_PROGRAMMATIC_LAUNCH=0 turns it off); results do not depend on it.
+bool programmatic_launch();
+
+template <class... KArgs, class... Args>
+inline void launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args&&... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = programmatic_launch() ? 1 : 0;
+    // a failed launch is reported by the caller's check_launch()
+    (void)cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 #define GCE_LAUNCH(kern, grid, block, smem, stream, ...)                        \
     do {                                                                         \
         ::gce::count_launch();                                                   \
         const bool gce_prof_ = ::gce::g_prof_on.load(std::memory_order_relaxed); \
         if (gce_prof_) ::gce::prof_before(#kern, (stream));                      \
-        kern<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+        ::gce::launch_kernel(kern, (grid), (block), (smem), (stream), __VA_ARGS__); \
         if (gce_prof_) ::gce::prof_after((stream));                              \
     } while (0)
 
@@ -147,9 +173,19 @@ void prof_after(cudaStream_t st);
         ::gce::count_launch();                                                   \
         const bool gce_prof_ = ::gce::g_prof_on.load(std::memory_order_relaxed); \
         if (gce_prof_) ::gce::prof_before((name), (stream));                     \
-        kern<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+        ::gce::launch_kernel(kern, (grid), (block), (smem), (stream), __VA_ARGS__); \
         if (gce_prof_) ::gce::prof_after((stream));                              \
     } while (0)
+
+// First statement of every kernel: wait until the kernel this launch depends
+// on in its stream has completed and its writes are visible (immediate when
+// the launch was not programmatic), then let the next launch in the stream
+// be scheduled.  Blocks of that launch wait in their own first statement, so
+// no kernel reads or writes memory while its predecessor still runs.
+__device__ __forceinline__ void grid_dependency_sync() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 inline int check_launch() {
     return cudaGetLastError() == cudaSuccess ? GCE_OK : GCE_ERR_CUDA;

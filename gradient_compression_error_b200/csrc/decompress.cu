@@ -45,6 +45,7 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
                                                         const int32_t* __restrict__ k_or_rank,
                                                         const int32_t* __restrict__ idx,
                                                         int32_t* __restrict__ bounds) {
+    grid_dependency_sync();
     const int64_t total = int64_t(bunits_pw) * W;
     for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
         const int w = int(u / bunits_pw);
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     const float* __restrict__ vals, const int32_t* __restrict__ idx, const float* __restrict__ P,
     const float* __restrict__ Q, const int32_t* __restrict__ bounds, float scale,
     float* __restrict__ out) {
+    grid_dependency_sync();
     __shared__ __align__(16) float acc[kDcTile];
     // per-worker entry ranges of the tile, double-buffered by sparse-tile
     // parity: warp 0 fills the next tile's copy while a slower warp may still
@@ -323,6 +325,7 @@ __global__ void __launch_bounds__(kDcThreads) dc_sign_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
     int32_t dc_tiles, int32_t W, int64_t vals_pw, const float* __restrict__ vals, float scale,
     float* __restrict__ out) {
+    grid_dependency_sync();
     constexpr int kWordsPerTile = kDcTile / 32;           // 128
     constexpr int kRounds = kDcTile / (4 * kDcThreads);   // 8
     __shared__ uint32_t sw[32 * kWordsPerTile];

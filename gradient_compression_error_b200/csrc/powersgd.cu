@@ -15,12 +15,14 @@
 // element of M: far below the tensor-core ridge and below the CUDA-core one,
 // so the kernels are plain register-blocked FMA loops shaped for bandwidth:
 //   mq      one pass over grad and mem: M written back to mem, and per
-//           (16-row block, 1024-column chunk) tile each warp reduces its rows
-//           against the Q chunk staged in shared memory -> partial P
+//           (row block, 1024-column chunk) tile each warp reduces its rows
+//           against the Q chunk staged in shared memory -> partial P; row
+//           blocks of 64 rows in layers of at least 2^24 elements, 16 below
 //   orth    one CTA per matrix: partial P summed in fp64 in chunk order,
 //           then Gram-Schmidt with fp64 block reductions in a fixed order
-//   mtp     per (64-row block, 1024-column chunk): each thread owns 4
-//           columns and accumulates M^T P over the block's rows -> partials
+//   mtp     per (row block, 1024-column chunk): each thread owns 4
+//           columns and accumulates M^T P over the block's rows -> partials;
+//           256-row blocks in layers of at least 2^24 elements, 64 below
 //   qred    the row-block partials summed in fp64 in block order -> Q
 //   resid   m <- M - P Q^T with the same product order as the decoder
 // DRAM traffic for matrices that stay in L2 between the passes: 12 B per
@@ -34,9 +36,12 @@
 
 namespace gce {
 
-constexpr int kPsRB = 16;     // rows per M Q / residual tile
+constexpr int kPsRB = 64;     // most rows per M Q / residual / decode tile
+constexpr int kPsRBSmall = 16;                     // rows per such tile of a layer
+constexpr int64_t kPsTallTileMin = int64_t(1) << 24;  // smaller than this many elements
 constexpr int kPsCB = 1024;   // columns per chunk (256 threads x 4)
-constexpr int kPsRB3 = 64;    // rows per M^T P tile
+constexpr int kPsRB3 = 256;   // most rows per M^T P tile (its partial's row block)
+constexpr int kPsRB3Small = 64;  // rows per such block of a layer under kPsTallTileMin elements
 constexpr int kPsQB = 256;    // columns per Q-reduction tile
 
 constexpr int64_t kPsTallRows = 8192;  // taller P: Gram-Schmidt spread over many blocks
@@ -60,7 +65,7 @@ struct PsLayer {
     int32_t tall;       // index among the tall layers, -1 otherwise
     int32_t part_off;   // first partial-sum slot of a tall layer
     int32_t nchunk;     // row chunks of a tall layer
-    int32_t pad;
+    int32_t rb3;        // rows per M^T P block
 };
 
 int powersgd_plan(gce_table* t) {
@@ -84,7 +89,8 @@ int powersgd_plan(gce_table* t) {
         }
         if (L.kind == GCE_KIND_POWERSGD) {
             x.nch1 = int32_t((L.cols + kPsCB - 1) / kPsCB);
-            x.nrb3 = int32_t((L.rows + kPsRB3 - 1) / kPsRB3);
+            x.rb3 = L.n >= kPsTallTileMin ? kPsRB3 : kPsRB3Small;
+            x.nrb3 = int32_t((L.rows + x.rb3 - 1) / x.rb3);
             x.ppart_off = pp;
             x.pd_off = pd;
             x.qpart_off = qp;
@@ -95,8 +101,12 @@ int powersgd_plan(gce_table* t) {
             const bool exact = L.n <= kPsExactMax;
             std::vector<int4>& o1 = exact ? t1 : t1f;
             std::vector<int4>& o3 = exact ? t3 : t3f;
-            for (int32_t rb = 0; rb < (L.rows + kPsRB - 1) / kPsRB; ++rb)
-                for (int32_t ch = 0; ch < x.nch1; ++ch) o1.push_back(make_int4(l, rb, ch, 0));
+            // (layer, first row, column chunk, rows): large layers in taller
+            // tiles, which stage their factors once for more rows
+            const int64_t rbh = L.n >= kPsTallTileMin ? kPsRB : kPsRBSmall;
+            for (int64_t r0 = 0; r0 < L.rows; r0 += rbh)
+                for (int32_t ch = 0; ch < x.nch1; ++ch)
+                    o1.push_back(make_int4(l, int32_t(r0), ch, int32_t(std::min(rbh, L.rows - r0))));
             for (int32_t rb = 0; rb < x.nrb3; ++rb)
                 for (int32_t ch = 0; ch < x.nch1; ++ch) o3.push_back(make_int4(l, rb, ch, 0));
             for (int32_t cb = 0; cb < (L.cols + kPsQB - 1) / kPsQB; ++cb)
@@ -201,6 +211,7 @@ __device__ __forceinline__ int32_t ps_rank(const DevLayer& L, const int32_t* k_o
 __global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
                                  const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W,
                                  int64_t Q_pw, uint64_t seed, float* __restrict__ Q) {
+    grid_dependency_sync();
     for (int64_t u = blockIdx.x; u < int64_t(nps) * W; u += gridDim.x) {
         const int w = int(u / nps);
         const int32_t l = ps_layers[u % nps];
@@ -221,21 +232,44 @@ __global__ void ps_init_q_kernel(const DevLayer* __restrict__ layers,
 // fp64 from the fp64 factors (T = double), or in fp32 from their fp32
 // roundings, which are the P and Q the payload carries (T = float).  The
 // residual pass and the lazy step's first pass form it identically.
+// qv[j]: the factor Q' at this entry's column.
+template <class T>
+__device__ __forceinline__ float ps_unproject_v(float M, const T* pr, const T* qv, int r) {
+    if constexpr (std::is_same<T, double>::value) {
+        double mh = __dmul_rn(pr[0], qv[0]);
+#pragma unroll
+        for (int j = 1; j < kMaxRank; ++j)
+            if (j < r) mh = __fma_rn(pr[j], qv[j], mh);
+        return __double2float_rn(__dsub_rn(double(M), mh));
+    } else {
+        float mh = __fmul_rn(pr[0], qv[0]);
+#pragma unroll
+        for (int j = 1; j < kMaxRank; ++j)
+            if (j < r) mh = __fmaf_rn(pr[j], qv[j], mh);
+        return __fsub_rn(M, mh);
+    }
+}
+
 template <class T>
 __device__ __forceinline__ float ps_unproject(float M, const T* pr, const T (*qd)[kPsCB], int c,
                                               int r) {
+    T qv[kMaxRank];
+#pragma unroll
+    for (int j = 0; j < kMaxRank; ++j) qv[j] = j < r ? qd[j][c] : T(0);
+    return ps_unproject_v<T>(M, pr, qv, r);
+}
+
+// Four neighbouring shared-memory entries p[0..3] (16-byte aligned for
+// float, 32-byte for double) in vector loads.
+template <class T>
+__device__ __forceinline__ void lds4(const T* p, T (&o)[4]) {
     if constexpr (std::is_same<T, double>::value) {
-        double mh = __dmul_rn(pr[0], qd[0][c]);
-#pragma unroll
-        for (int j = 1; j < kMaxRank; ++j)
-            if (j < r) mh = __fma_rn(pr[j], qd[j][c], mh);
-        return __double2float_rn(__dsub_rn(double(M), mh));
+        const double2 a = *reinterpret_cast<const double2*>(p);
+        const double2 b = *reinterpret_cast<const double2*>(p + 2);
+        o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
     } else {
-        float mh = __fmul_rn(pr[0], qd[0][c]);
-#pragma unroll
-        for (int j = 1; j < kMaxRank; ++j)
-            if (j < r) mh = __fmaf_rn(pr[j], qd[j][c], mh);
-        return __fsub_rn(M, mh);
+        const float4 a = *reinterpret_cast<const float4*>(p);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
     }
 }
 
@@ -263,10 +297,18 @@ __device__ __forceinline__ void ps_mq_row(const float* __restrict__ g, float* __
             const float4 gg = ld_stream4(g + c);
             float4 mm = *reinterpret_cast<const float4*>(m + c);
             if (kLazy && rp > 0) {
-                mm.x = ps_unproject<T>(mm.x, pr, qdp, c, rp);
-                mm.y = ps_unproject<T>(mm.y, pr, qdp, c + 1, rp);
-                mm.z = ps_unproject<T>(mm.z, pr, qdp, c + 2, rp);
-                mm.w = ps_unproject<T>(mm.w, pr, qdp, c + 3, rp);
+                T qv[4][kMaxRank];  // qv[column][j], from vector loads of each factor column
+#pragma unroll
+                for (int j = 0; j < kMaxRank; ++j) {
+                    T t4[4] = {T(0), T(0), T(0), T(0)};
+                    if (j < rp) lds4<T>(&qdp[j][c], t4);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) qv[i][j] = t4[i];
+                }
+                mm.x = ps_unproject_v<T>(mm.x, pr, qv[0], rp);
+                mm.y = ps_unproject_v<T>(mm.y, pr, qv[1], rp);
+                mm.z = ps_unproject_v<T>(mm.z, pr, qv[2], rp);
+                mm.w = ps_unproject_v<T>(mm.w, pr, qv[3], rp);
             }
             float4 x;
             x.x = residual(mm.x, eta, gg.x);
@@ -274,10 +316,23 @@ __device__ __forceinline__ void ps_mq_row(const float* __restrict__ g, float* __
             x.z = residual(mm.z, eta, gg.z);
             x.w = residual(mm.w, eta, gg.w);
             *reinterpret_cast<float4*>(m + c) = x;
-            take(x.x, c);
-            take(x.y, c + 1);
-            take(x.z, c + 2);
-            take(x.w, c + 3);
+#pragma unroll
+            for (int j = 0; j < kMaxRank; ++j)
+                if (j < r) {
+                    T q4[4];
+                    lds4<T>(&qs[j][c], q4);
+                    if constexpr (std::is_same<T, double>::value) {
+                        a[j] = __fma_rn(double(x.x), q4[0], a[j]);
+                        a[j] = __fma_rn(double(x.y), q4[1], a[j]);
+                        a[j] = __fma_rn(double(x.z), q4[2], a[j]);
+                        a[j] = __fma_rn(double(x.w), q4[3], a[j]);
+                    } else {
+                        a[j] = __fmaf_rn(x.x, q4[0], a[j]);
+                        a[j] = __fmaf_rn(x.y, q4[1], a[j]);
+                        a[j] = __fmaf_rn(x.z, q4[2], a[j]);
+                        a[j] = __fmaf_rn(x.w, q4[3], a[j]);
+                    }
+                }
         }
     } else {
         for (int c = lane; c < cw; c += 32) {
@@ -294,12 +349,26 @@ __device__ __forceinline__ void ps_mq_row(const float* __restrict__ g, float* __
 
 // Stage n entries of a rows x cap (row stride cap) factor, columns 0..rc-1,
 // into dst[j][i] as T (double from fp64, or its fp32 rounding).
-template <class T>
-__device__ __forceinline__ void ps_stage(T (*dst)[kPsCB], const double* src, int n, int rc,
+template <class T, class S>
+__device__ __forceinline__ void ps_stage(T (*dst)[kPsCB], const S* src, int n, int rc,
                                          int cap) {
-    for (int i = threadIdx.x; i < n * rc; i += blockDim.x) {
-        const int c = i / rc, j = i - c * rc;
-        dst[j][c] = T(src[int64_t(c) * cap + j]);
+    for (int c = threadIdx.x; c < n; c += blockDim.x) {
+        const S* x = src + int64_t(c) * cap;
+#pragma unroll
+        for (int j = 0; j < kMaxRank; ++j)
+            if (j < rc) dst[j][c] = T(x[j]);
+    }
+}
+
+// Rows x rc entries (row stride cap) into dst[row][j] as T.
+template <class T, class S>
+__device__ __forceinline__ void ps_stage_rows(T (*dst)[kMaxRank], const S* src, int rows, int rc,
+                                              int cap) {
+    for (int row = threadIdx.x; row < rows; row += blockDim.x) {
+        const S* x = src + int64_t(row) * cap;
+#pragma unroll
+        for (int j = 0; j < kMaxRank; ++j)
+            if (j < rc) dst[row][j] = T(x[j]);
     }
 }
 
@@ -332,6 +401,7 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
     const int32_t* __restrict__ k_or_rank, const float* __restrict__ Q, double* __restrict__ ppart,
     int32_t* __restrict__ status, const double* __restrict__ pdw, int64_t pd_pw,
     const double* __restrict__ qdw, int32_t L_all, const int32_t* __restrict__ lazy_rank) {
+    grid_dependency_sync();
     // dynamic shared memory (ps_mq_smem bytes)
     extern __shared__ __align__(16) double ps_dyn[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -352,8 +422,8 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
         const int64_t C = L.cols, R = L.rows;
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
-        const int64_t r0 = int64_t(d.y) * kPsRB;
-        const int rh = int(min64(kPsRB, R - r0));
+        const int64_t r0 = d.y;
+        const int rh = d.w;
         const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
         // shared memory: the warm start Q, then (lazy) the previous Q' and
         // the previous P rows, in the layer's precision T
@@ -361,17 +431,11 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
             T (*qs)[kPsCB] = reinterpret_cast<T (*)[kPsCB]>(ps_dyn);
             T (*qdp)[kPsCB] = qs + kMaxRank;
             T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(qdp + kMaxRank);
-            for (int i = tid; i < cw * r; i += blockDim.x) {
-                const int c = i / r, j = i - c * r;
-                qs[j][c] = T(q[int64_t(c) * cap + j]);
-            }
+            ps_stage<T>(qs, q, cw, r, cap);
             if (kLazy && rp > 0) {
                 ps_stage<T>(qdp, qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap, cw, rp, cap);
-                const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
-                for (int i = tid; i < rh * rp; i += blockDim.x) {
-                    const int row = i / rp, j = i - row * rp;
-                    prow[row][j] = T(p[int64_t(row) * cap + j]);
-                }
+                ps_stage_rows<T>(prow, pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap, rh, rp,
+                                 cap);
             }
             __syncthreads();
             for (int row = warp; row < rh; row += blockDim.x >> 5) {
@@ -401,6 +465,32 @@ __global__ void __launch_bounds__(256) ps_mq_kernel(
     }
 }
 
+
+// Entry (row, j) of P: the partials of nsum workers x nch column chunks
+// added in fp64 in worker, then chunk order; kB partials are in flight
+// ahead of their adds.
+__device__ __forceinline__ double ps_sum_partials(const double* pp, int nsum, int64_t ppart_pw,
+                                                  int nch, int64_t R, int cap, int64_t row,
+                                                  int j) {
+    constexpr int kB = 8;
+    const int nt = nsum * nch;
+    auto part = [&](int i) {
+        const int ws = i / nch, ch = i - ws * nch;
+        return __ldcg(pp + int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j);
+    };
+    double s = 0.0;
+    int i = 0;
+    for (; i + kB <= nt; i += kB) {
+        double v[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b) v[b] = part(i + b);
+#pragma unroll
+        for (int b = 0; b < kB; ++b) s += v[b];
+    }
+    for (; i < nt; ++i) s += part(i);
+    return s;
+}
+
 // ---- orthonormalise P (one CTA per matrix) ----------------------------------------------
 __device__ __forceinline__ double block_sum_d(double x, double* s_red) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -423,6 +513,7 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
     int64_t pd_pw, const int32_t* __restrict__ k_or_rank, const double* __restrict__ ppart,
     double* __restrict__ pdw, float* __restrict__ P, int32_t* __restrict__ status,
     int32_t ntall, int32_t* __restrict__ tdone, int32_t L_all, int32_t* __restrict__ lazy_rank) {
+    grid_dependency_sync();
     __shared__ double s_red[32];
     for (int64_t u = blockIdx.x; u < int64_t(nps) * W; u += gridDim.x) {
         const int w = int(u / nps);
@@ -449,11 +540,7 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         for (int64_t i = threadIdx.x; i < R * r; i += blockDim.x) {
             const int64_t row = i / r;
             const int j = int(i - row * r);
-            double s = 0.0;
-            for (int ws = 0; ws < nsum; ++ws)
-                for (int ch = 0; ch < X.nch1; ++ch)
-                    s += pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j];
-            pd[row * cap + j] = s;
+            pd[row * cap + j] = ps_sum_partials(pp, nsum, ppart_pw, X.nch1, R, cap, row, j);
         }
         __syncthreads();
         for (int j = 0; j < r; ++j) {
@@ -506,6 +593,7 @@ __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
     const int32_t* __restrict__ k_or_rank,
     const double* __restrict__ ppart, double* __restrict__ pdw, double* __restrict__ tparts,
     double* __restrict__ tscal, int32_t* __restrict__ tdone, float* __restrict__ P) {
+    grid_dependency_sync();
     __shared__ double s_red[8];
     __shared__ int s_last;
     for (int64_t u = blockIdx.x; u < int64_t(nunits) * W; u += gridDim.x) {
@@ -524,13 +612,8 @@ __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
         if (op.init) {
             const double* pp = ppart + int64_t(w) * nsum * ppart_pw + X.ppart_off;
             for (int64_t row = r0 + threadIdx.x; row < r1; row += blockDim.x)
-                for (int j = 0; j < r; ++j) {
-                    double s = 0.0;
-                    for (int ws = 0; ws < nsum; ++ws)
-                        for (int ch = 0; ch < X.nch1; ++ch)
-                            s += pp[int64_t(ws) * ppart_pw + (int64_t(ch) * R + row) * cap + j];
-                    pd[row * cap + j] = s;
-                }
+                for (int j = 0; j < r; ++j)
+                    pd[row * cap + j] = ps_sum_partials(pp, nsum, ppart_pw, X.nch1, R, cap, row, j);
         }
         if (op.apply && op.aj < r) {
             const double sv = *scal;
@@ -604,16 +687,17 @@ static std::vector<PsOrthOp> ps_orth_ops(int cap) {
     return ops;
 }
 
-// ---- phase 3: partial Q = M^T P over 64-row blocks ---------------------------------------
+// ---- phase 3: partial Q = M^T P over row blocks ----------------------------------------------
 // From the orthonormal P of the workspace: products in the layer's
 // precision (fp64, or fp32 from the P the payload carries), the partial of
-// each 64-row block stored in fp64.
+// each row block (PsLayer::rb3 rows) stored in fp64.
 template <class T>
 __global__ void __launch_bounds__(256) ps_mtp_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t pd_pw,
     int64_t qpart_pw, const float* __restrict__ mem, const int32_t* __restrict__ k_or_rank,
     const double* __restrict__ pdw, double* __restrict__ qpart) {
+    grid_dependency_sync();
     __shared__ double prow_d[kPsRB3][kMaxRank];
     const int tid = threadIdx.x;
     for (int64_t u = blockIdx.x; u < int64_t(ntiles) * W; u += gridDim.x) {
@@ -625,8 +709,8 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
         if (r == 0) continue;
         const int cap = L.cap;
         const int64_t C = L.cols;
-        const int64_t r0 = int64_t(d.y) * kPsRB3;
-        const int rh = int(min64(kPsRB3, L.rows - r0));
+        const int64_t r0 = int64_t(d.y) * X.rb3;
+        const int rh = int(min64(X.rb3, L.rows - r0));
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
         const double* p = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
@@ -647,16 +731,7 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
 #pragma unroll
                 for (int j = 0; j < kMaxRank; ++j) acc[q][j] = T(0);
             if (cc < cw) {
-                for (int row = 0; row < rh; ++row) {
-                    const float* m = mem + ebase + int64_t(row) * C + cc;
-                    float x[4];
-                    if (vec) {
-                        const float4 mm = *reinterpret_cast<const float4*>(m);
-                        x[0] = mm.x; x[1] = mm.y; x[2] = mm.z; x[3] = mm.w;
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) x[q] = (cc + q < cw) ? m[q] : 0.0f;
-                    }
+                auto fma_row = [&](const float (&x)[4], int row) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
 #pragma unroll
@@ -667,6 +742,35 @@ __global__ void __launch_bounds__(256) ps_mtp_kernel(
                                 else
                                     acc[q][j] = __fmaf_rn(x[q], prow[row][j], acc[q][j]);
                             }
+                };
+                int row = 0;
+                if (vec) {
+                    // kB rows' loads in flight before their products (rows in order)
+                    constexpr int kB = 8;
+                    for (; row + kB <= rh; row += kB) {
+                        float4 mm[kB];
+#pragma unroll
+                        for (int b = 0; b < kB; ++b)
+                            mm[b] = __ldg(reinterpret_cast<const float4*>(mem + ebase +
+                                                                          int64_t(row + b) * C + cc));
+#pragma unroll
+                        for (int b = 0; b < kB; ++b) {
+                            const float x[4] = {mm[b].x, mm[b].y, mm[b].z, mm[b].w};
+                            fma_row(x, row + b);
+                        }
+                    }
+                }
+                for (; row < rh; ++row) {
+                    const float* m = mem + ebase + int64_t(row) * C + cc;
+                    float x[4];
+                    if (vec) {
+                        const float4 mm = *reinterpret_cast<const float4*>(m);
+                        x[0] = mm.x; x[1] = mm.y; x[2] = mm.z; x[3] = mm.w;
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) x[q] = (cc + q < cw) ? m[q] : 0.0f;
+                    }
+                    fma_row(x, row);
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -692,6 +796,7 @@ __global__ void __launch_bounds__(256) ps_qred_kernel(
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t Q_pw, int64_t qpart_pw,
     const int32_t* __restrict__ k_or_rank, const double* __restrict__ qpart,
     float* __restrict__ Q, double* __restrict__ qd, float* __restrict__ qmean, float inv_w) {
+    grid_dependency_sync();
     const int64_t nunits = kMean ? int64_t(ntiles) : int64_t(ntiles) * W;
     for (int64_t u = blockIdx.x; u < nunits; u += gridDim.x) {
         const int w = kMean ? 0 : int(u / ntiles);
@@ -711,8 +816,20 @@ __global__ void __launch_bounds__(256) ps_qred_kernel(
             for (int wi = 0; wi < (kMean ? W : 1); ++wi) {
                 const int ww = kMean ? wi : w;
                 const double* qp = qpart + int64_t(ww) * qpart_pw + X.qpart_off;
+                // block order; kB partials in flight ahead of their adds
+                constexpr int kB = 8;
+                const int64_t stride = C * cap;
+                const double* x = qp + c * cap + j;
                 double s = 0.0;
-                for (int rb = 0; rb < X.nrb3; ++rb) s += qp[(int64_t(rb) * C + c) * cap + j];
+                int rb = 0;
+                for (; rb + kB <= X.nrb3; rb += kB) {
+                    double v[kB];
+#pragma unroll
+                    for (int b = 0; b < kB; ++b) v[b] = __ldcg(x + int64_t(rb + b) * stride);
+#pragma unroll
+                    for (int b = 0; b < kB; ++b) s += v[b];
+                }
+                for (; rb < X.nrb3; ++rb) s += __ldcg(x + int64_t(rb) * stride);
                 const float qv = float(s);
                 Q[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = qv;
                 qd[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = s;
@@ -729,6 +846,7 @@ __global__ void __launch_bounds__(256) ps_dense_mean_kernel(
     const int32_t* __restrict__ dtile_start, int32_t ntiles, int32_t W, int64_t N,
     const float* __restrict__ grad, float* __restrict__ mem, float eta, float inv_w,
     float* __restrict__ vals, int32_t* __restrict__ status) {
+    grid_dependency_sync();
     bool bad = false;
     for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
         const DevLayer L = layers[dtile_layer[u]];
@@ -755,6 +873,7 @@ __global__ void __launch_bounds__(256) ps_qmean_kernel(
     const DevLayer* __restrict__ layers, const int4* __restrict__ tiles, int32_t ntiles,
     int32_t W, int64_t Q_pw, const int32_t* __restrict__ k_or_rank, const float* __restrict__ Qw,
     float* __restrict__ Q, float inv_w) {
+    grid_dependency_sync();
     for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
         const int4 d = tiles[u];
         const DevLayer L = layers[d.x];
@@ -777,6 +896,7 @@ __global__ void __launch_bounds__(256) ps_vmean_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dtile_layer,
     const int32_t* __restrict__ dtile_start, int32_t ntiles, int32_t W, int64_t vals_pw,
     const float* __restrict__ vals_all, float* __restrict__ vals, float inv_w) {
+    grid_dependency_sync();
     for (int32_t u = blockIdx.x; u < ntiles; u += gridDim.x) {
         const DevLayer L = layers[dtile_layer[u]];
         const int64_t s0 = dtile_start[u];
@@ -805,6 +925,7 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
     const float* __restrict__ P, const float* __restrict__ Q, const double* __restrict__ pdw,
     const double* __restrict__ qdw, float* __restrict__ mem, float* __restrict__ dense_out,
     const int32_t* __restrict__ rank_wl, int32_t L_all) {
+    grid_dependency_sync();
     // dynamic shared memory (kPsResidSmem bytes)
     extern __shared__ __align__(16) double ps_dyn[];
     float (*qs)[kPsCB] =
@@ -826,32 +947,20 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
         }
         if (r == 0) continue;
         const int cap = L.cap;
-        const int64_t C = L.cols, R = L.rows;
+        const int64_t C = L.cols;
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
-        const int64_t r0 = int64_t(d.y) * kPsRB;
-        const int rh = int(min64(kPsRB, R - r0));
+        const int64_t r0 = d.y;
+        const int rh = d.w;
         if (dense_out) {
-            const float* q = Q + int64_t(w) * Q_pw + L.q_off + c0 * cap;
-            for (int i = tid; i < cw * r; i += blockDim.x) {
-                const int c = i / r, j = i - c * r;
-                qs[j][c] = q[int64_t(c) * cap + j];
-            }
-            const float* p = P + int64_t(w) * P_pw + L.p_off + r0 * cap;
-            for (int i = tid; i < rh * r; i += blockDim.x) {
-                const int row = i / r, j = i - row * r;
-                prow32[row][j] = p[int64_t(row) * cap + j];
-            }
+            ps_stage<float>(qs, Q + int64_t(w) * Q_pw + L.q_off + c0 * cap, cw, r, cap);
+            ps_stage_rows<float>(prow32, P + int64_t(w) * P_pw + L.p_off + r0 * cap, rh, r, cap);
         }
         {
             T (*qd)[kPsCB] = reinterpret_cast<T (*)[kPsCB]>(ps_dyn);
             T (*prow)[kMaxRank] = reinterpret_cast<T (*)[kMaxRank]>(ps_dyn + kMaxRank * kPsCB);
             ps_stage<T>(qd, qdw + int64_t(w) * Q_pw + L.q_off + c0 * cap, cw, r, cap);
-            const double* pp = pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap;
-            for (int i = tid; i < rh * r; i += blockDim.x) {
-                const int row = i / r, j = i - row * r;
-                prow[row][j] = T(pp[int64_t(row) * cap + j]);
-            }
+            ps_stage_rows<T>(prow, pdw + int64_t(w) * pd_pw + X.pd_off + r0 * cap, rh, r, cap);
             __syncthreads();
             for (int row = warp; row < rh; row += blockDim.x >> 5) {
                 const int64_t e = int64_t(w) * N + L.offset + (r0 + row) * C + c0;
@@ -872,17 +981,37 @@ __global__ void __launch_bounds__(256) ps_resid_kernel(
                     return mh;
                 };
                 if (((e & 3) == 0) && ((cw & 3) == 0)) {  // 16-byte rows: four columns a lane
-                    for (int c = lane * 4; c < cw; c += 128) {
-                        float4 mm = *reinterpret_cast<const float4*>(m + c);
-                        mm.x = ps_unproject<T>(mm.x, pr, qd, c, r);
-                        mm.y = ps_unproject<T>(mm.y, pr, qd, c + 1, r);
-                        mm.z = ps_unproject<T>(mm.z, pr, qd, c + 2, r);
-                        mm.w = ps_unproject<T>(mm.w, pr, qd, c + 3, r);
-                        __stcs(reinterpret_cast<float4*>(m + c), mm);
-                        if (o)
-                            __stcs(reinterpret_cast<float4*>(o + c),
-                                   make_float4(decoded(c), decoded(c + 1), decoded(c + 2),
-                                               decoded(c + 3)));
+                    // float4 of memory in flight per lane (fewer for the fp64 products)
+                    constexpr int kU = std::is_same<T, double>::value ? 2 : 4;
+                    for (int c0 = lane * 4; c0 < cw; c0 += 128 * kU) {
+                        float4 mm[kU];
+#pragma unroll
+                        for (int u = 0; u < kU; ++u)
+                            if (c0 + 128 * u < cw)
+                                mm[u] = *reinterpret_cast<const float4*>(m + c0 + 128 * u);
+#pragma unroll
+                        for (int u = 0; u < kU; ++u) {
+                            const int c = c0 + 128 * u;
+                            if (c >= cw) break;
+                            float4 mv = mm[u];
+                            T qv[4][kMaxRank];
+#pragma unroll
+                            for (int j = 0; j < kMaxRank; ++j) {
+                                T t4[4] = {T(0), T(0), T(0), T(0)};
+                                if (j < r) lds4<T>(&qd[j][c], t4);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) qv[i][j] = t4[i];
+                            }
+                            mv.x = ps_unproject_v<T>(mv.x, pr, qv[0], r);
+                            mv.y = ps_unproject_v<T>(mv.y, pr, qv[1], r);
+                            mv.z = ps_unproject_v<T>(mv.z, pr, qv[2], r);
+                            mv.w = ps_unproject_v<T>(mv.w, pr, qv[3], r);
+                            __stcs(reinterpret_cast<float4*>(m + c), mv);
+                            if (o)
+                                __stcs(reinterpret_cast<float4*>(o + c),
+                                       make_float4(decoded(c), decoded(c + 1), decoded(c + 2),
+                                                   decoded(c + 3)));
+                        }
                     }
                 } else {
                     for (int c = lane; c < cw; c += 32) {
@@ -911,6 +1040,7 @@ __global__ void __launch_bounds__(256) ps_decode_kernel(
     int32_t W, int64_t P_pw, int64_t Q_pw, const int32_t* __restrict__ k_or_rank,
     const float* __restrict__ P, const float* __restrict__ Q, float scale,
     float* __restrict__ out) {
+    grid_dependency_sync();
     __shared__ float qs[kDcLrMaxW][kMaxRank][256];
     __shared__ float prow[kDcLrMaxW][kPsRB][kMaxRank];
     const int tid = threadIdx.x;
@@ -920,14 +1050,15 @@ __global__ void __launch_bounds__(256) ps_decode_kernel(
         const int r = ps_rank(L, k_or_rank, d.x);
         const int cap = L.cap;
         const int64_t C = L.cols;
-        const int64_t r0 = int64_t(d.y) * kPsRB;
-        const int rh = int(min64(kPsRB, L.rows - r0));
+        const int64_t r0 = d.y;
+        const int rh = d.w;
         const int64_t c0 = int64_t(d.z) * kPsCB;
         const int cw = int(min64(kPsCB, C - c0));
-        for (int i = tid; i < W * kPsRB * kMaxRank; i += blockDim.x) {
-            const int w = i / (kPsRB * kMaxRank), rr = (i / kMaxRank) % kPsRB, j = i % kMaxRank;
-            prow[w][rr][j] = (rr < rh && j < r) ? P[int64_t(w) * P_pw + L.p_off + (r0 + rr) * cap + j]
-                                                : 0.0f;
+        for (int i = tid; i < W * rh; i += blockDim.x) {
+            const int w = i / rh, rr = i - w * rh;
+            const float* p = P + int64_t(w) * P_pw + L.p_off + (r0 + rr) * cap;
+#pragma unroll
+            for (int j = 0; j < kMaxRank; ++j) prow[w][rr][j] = j < r ? p[j] : 0.0f;
         }
         const bool rows16 = ((L.offset + r0 * C + c0) & 3) == 0 && (C & 3) == 0 && (cw & 3) == 0;
         if (W == 1 && rows16) {

@@ -116,6 +116,7 @@ __global__ void __launch_bounds__(256) rk_setup_kernel(const DevLayer* __restric
                                                        int32_t* __restrict__ status,
                                                        uint64_t* __restrict__ tag,
                                                        uint64_t tag_value) {
+    grid_dependency_sync();
     if (blockIdx.x == 0 && threadIdx.x == 0) *tag = tag_value;
     for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
          s += int64_t(gridDim.x) * blockDim.x)
@@ -192,6 +193,7 @@ __global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict
                                                       int32_t* __restrict__ tile_cnt,
                                                       uint32_t* __restrict__ bitmask,
                                                       RkEntry* __restrict__ cand) {
+    grid_dependency_sync();
     __shared__ int s_red[8];
     const int64_t total = int64_t(tiles_pw) * W;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
@@ -220,6 +222,7 @@ __global__ void __launch_bounds__(256) rk_refresh_k_kernel(const DevLayer* __res
                                                            int32_t* __restrict__ status,
                                                            const uint64_t* __restrict__ tag,
                                                            uint64_t tag_value) {
+    grid_dependency_sync();
     const bool held = *tag == tag_value;
     for (int64_t s = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; s < S;
          s += int64_t(gridDim.x) * blockDim.x) {
@@ -317,6 +320,7 @@ __global__ void __launch_bounds__(1024) rk_resolve_kernel(const DevLayer* __rest
                                                           uint32_t* __restrict__ bitmask,
                                                           const RkEntry* __restrict__ cand,
                                                           int32_t* __restrict__ status) {
+    grid_dependency_sync();
     __shared__ int32_t h[2048];
     __shared__ uint32_t s_pref;
     __shared__ int32_t s_rank;
@@ -375,6 +379,7 @@ __global__ void __launch_bounds__(1024) rk_scan_kernel(const DevLayer* __restric
                                                        int32_t ncomp, int64_t S, int32_t tiles_pw,
                                                        const RkSeg* __restrict__ segs,
                                                        int32_t* __restrict__ tile_cnt) {
+    grid_dependency_sync();
     __shared__ int s_warp[33];
     for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
         if (segs[s].k == 0) continue;
@@ -408,6 +413,7 @@ __global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
     const RkSeg* __restrict__ segs, RkSeg* __restrict__ segs_next, int32_t* tile_off,
     uint32_t* bitmask, RkEntry* __restrict__ cand, float* __restrict__ vals,
     int32_t* __restrict__ idx, int32_t* __restrict__ status) {
+    grid_dependency_sync();
     constexpr int kIters = kTkPerThread / 4;
     constexpr int kWarps = kTkThreads / 32;
     __shared__ int32_t s_wt[kIters * kWarps];

@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(256) sg_norm_kernel(
     const float* __restrict__ mem, float eta, double* __restrict__ partials,
     int32_t* __restrict__ done, float* __restrict__ scales, float* __restrict__ vals,
     int32_t* __restrict__ status) {
+    grid_dependency_sync();
     __shared__ double s_red[8];
     __shared__ int s_last;
     for (int64_t t = blockIdx.x; t < int64_t(tiles_pw) * W; t += gridDim.x) {
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(256) sg_emit_kernel(
     int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, const float* __restrict__ grad,
     float* __restrict__ mem, float eta, const float* __restrict__ scales,
     float* __restrict__ vals) {
+    grid_dependency_sync();
     for (int64_t t = blockIdx.x; t < int64_t(tiles_pw) * W; t += gridDim.x) {
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
@@ -292,6 +294,7 @@ __global__ void __launch_bounds__(256, 4) sg_fused_kernel(
     int64_t nitems, uint32_t* counter, double* __restrict__ partials, int32_t* done,
     int32_t* ready, float* __restrict__ scales, float* __restrict__ vals,
     int32_t* __restrict__ status) {
+    grid_dependency_sync();
     __shared__ double s_red[8];
     __shared__ int s_last;
     __shared__ int64_t s_item;
@@ -338,6 +341,7 @@ __global__ void __launch_bounds__(128) sg_vote_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
     int32_t dc_tiles, int32_t W, int64_t vals_pw, const float* __restrict__ vals, float scale,
     float* __restrict__ out) {
+    grid_dependency_sync();
     for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
         const int32_t l = dc_tile_layer[u];
         const DevLayer L = layers[l];

@@ -2,6 +2,7 @@
 // and the kernel for uncompressed (DENSE) layers shared by every step.
 #include <algorithm>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -13,6 +14,14 @@ namespace gce {
 
 std::atomic<uint64_t> g_launches{0};
 std::atomic<bool> g_prof_on{false};
+
+bool programmatic_launch() {
+    static const bool on = [] {
+        const char* v = std::getenv("GCE_PROGRAMMATIC_LAUNCH");
+        return !(v && v[0] == '0');
+    }();
+    return on;
+}
 
 // ---- launch timing (host side) -------------------------------------------------
 namespace {
@@ -114,6 +123,7 @@ __global__ void __launch_bounds__(256) dense_kernel(const DevLayer* __restrict__
                                                     float* __restrict__ mem, float eta,
                                                     float* __restrict__ vals,
                                                     int32_t* __restrict__ status) {
+    grid_dependency_sync();
     const int64_t total = int64_t(dtiles_pw) * W;
     bool bad = false;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {

@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(256) tk_setup_kernel(const DevLayer* __restric
                                                        TkSeg* __restrict__ segs,
                                                        int4* __restrict__ hists4, int64_t n4,
                                                        int32_t* __restrict__ status) {
+    grid_dependency_sync();
     const int64_t stride = int64_t(gridDim.x) * blockDim.x;
     for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride)
         hists4[i] = make_int4(0, 0, 0, 0);
@@ -140,6 +141,7 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
     const int32_t* __restrict__ sunit_part, int32_t sunits_pw, int32_t W, int32_t ncomp,
     int64_t S, int64_t N, const float* __restrict__ grad, const float* __restrict__ mem,
     float eta, TkSeg* __restrict__ segs, int32_t* __restrict__ hists, double sigma) {
+    grid_dependency_sync();
     constexpr int kBatch = 8;
     __shared__ int32_t h[kTkSBins];
     __shared__ int s_last;
@@ -238,6 +240,7 @@ __global__ void __launch_bounds__(kTkThreads) tk_main_kernel(
     int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, const float* __restrict__ grad,
     float* __restrict__ mem, float eta, TkSeg* __restrict__ segs, int2* __restrict__ tile_dir,
     float* __restrict__ spill_v, int32_t* __restrict__ spill_i, int32_t* __restrict__ status) {
+    grid_dependency_sync();
     constexpr int kIters = kTkPerThread / 4;           // 8 float4 per thread
     constexpr int kWarps = kTkThreads / 32;            // 8
     __shared__ int32_t s_wt[kIters * kWarps];
@@ -377,6 +380,7 @@ __global__ void __launch_bounds__(1024) tk_units_kernel(const DevLayer* __restri
                                                         int2* __restrict__ unit_seg,
                                                         int32_t* __restrict__ redo_list,
                                                         int32_t* __restrict__ status) {
+    grid_dependency_sync();
     __shared__ int s_warp[33];
     __shared__ int s_carry, s_rcarry;
     if (threadIdx.x == 0) {
@@ -436,6 +440,7 @@ __global__ void __launch_bounds__(256) tk_restore_kernel(
     const int32_t* __restrict__ redo_list, const int2* __restrict__ tile_dir,
     const float* __restrict__ spill_v, const int32_t* __restrict__ spill_i,
     float* __restrict__ mem) {
+    grid_dependency_sync();
     const int32_t n = redo_list[0];
     for (int32_t u = blockIdx.x; u < n; u += gridDim.x) {
         const int32_t t = redo_list[1 + u];
@@ -457,6 +462,7 @@ __global__ void __launch_bounds__(256) tk_respill_kernel(
     int32_t ncomp, int64_t N, int64_t comp_N, TkSeg* __restrict__ segs,
     const int32_t* __restrict__ redo_list, int2* __restrict__ tile_dir,
     const float* __restrict__ mem, float* __restrict__ spill_v, int32_t* __restrict__ spill_i) {
+    grid_dependency_sync();
     __shared__ int s_base;
     const int32_t n = redo_list[0];
     for (int32_t u = blockIdx.x; u < n; u += gridDim.x) {
@@ -492,6 +498,7 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
                                                       const int2* __restrict__ unit_seg,
                                                       int32_t* __restrict__ hists,
                                                       const float* __restrict__ spill_v) {
+    grid_dependency_sync();
     constexpr int kNb = kLevel == 3 ? 512 : kTkBins;
     constexpr int kShift = kLevel == 1 ? 20 : (kLevel == 2 ? 9 : 0);
     constexpr int kPer = 16;  // candidates per thread per load batch
@@ -564,6 +571,7 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
                                                        const int2* __restrict__ tile_dir,
                                                        int2* __restrict__ tile_cnt,
                                                        const float* __restrict__ spill_v) {
+    grid_dependency_sync();
     constexpr int kBatch = 8;
     const int lane = threadIdx.x & 31;
     const int64_t total = int64_t(tiles_pw) * W;
@@ -604,6 +612,7 @@ __global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restric
                                                        int32_t ncomp, int64_t S, int32_t tiles_pw,
                                                        const TkSeg* __restrict__ segs,
                                                        int2* __restrict__ tile_cnt) {
+    grid_dependency_sync();
     __shared__ int s_warp[33];
     for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
         if (segs[s].k == 0) continue;
@@ -631,6 +640,7 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
     const int2* __restrict__ tile_cnt, const float* __restrict__ spill_v,
     const int32_t* __restrict__ spill_i, float* __restrict__ mem, float* __restrict__ vals,
     int32_t* __restrict__ idx) {
+    grid_dependency_sync();
     constexpr int kBatch = 8;
     const int lane = threadIdx.x & 31;
     const unsigned lt_mask = (1u << lane) - 1u;
