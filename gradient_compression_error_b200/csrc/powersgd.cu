@@ -42,7 +42,7 @@ constexpr int64_t kPsTallTileMin = int64_t(1) << 24;  // smaller than this many 
 constexpr int kPsCB = 1024;   // columns per chunk (256 threads x 4)
 constexpr int kPsRB3 = 256;   // most rows per M^T P tile (its partial's row block)
 constexpr int kPsRB3Small = 64;  // rows per such block of a layer under kPsTallTileMin elements
-constexpr int kPsQB = 256;    // columns per Q-reduction tile
+constexpr int kPsQB = 128;    // columns per Q-reduction tile
 
 constexpr int64_t kPsTallRows = 8192;  // taller P: Gram-Schmidt spread over many blocks
 constexpr int kPsOrthChunk = 1024;     // rows per block in that case
@@ -394,7 +394,7 @@ constexpr const char* ps_prec_name(const char* d, const char* f) {
 // as the residual pass would have formed it, so the results are the eager
 // step's bit for bit without that pass's read and write of M.
 template <bool kLazy, class T>
-__global__ void __launch_bounds__(256) ps_mq_kernel(
+__global__ void __launch_bounds__(256, std::is_same<T, float>::value ? 5 : 4) ps_mq_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t Q_pw,
     int64_t ppart_pw, const float* __restrict__ grad, float* __restrict__ mem, float eta,
@@ -692,7 +692,7 @@ static std::vector<PsOrthOp> ps_orth_ops(int cap) {
 // precision (fp64, or fp32 from the P the payload carries), the partial of
 // each row block (PsLayer::rb3 rows) stored in fp64.
 template <class T>
-__global__ void __launch_bounds__(256) ps_mtp_kernel(
+__global__ void __launch_bounds__(256, std::is_same<T, float>::value ? 6 : 4) ps_mtp_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int4* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t N, int64_t pd_pw,
     int64_t qpart_pw, const float* __restrict__ mem, const int32_t* __restrict__ k_or_rank,
