@@ -18,7 +18,8 @@
 //            whose band missed (exact fallback; results never depend on sigma)
 //   scan     per-tile output offsets
 //   emit     the only HBM pass: v = fl(m + fl(eta*g)), ordered write of the
-//            chosen (v, i), mem <- v or +0
+//            chosen (v, i), mem <- v or +0; with the look-ahead, a third of
+//            each block's warps hash the next step's keys meanwhile
 // DRAM traffic: 12 B per element + 8 B per chosen entry + 1/8 B of bitmask
 // written and read.
 #include <cmath>
@@ -57,15 +58,21 @@ struct RkLayout {
     size_t segs = 0, tile_cnt = 0, bitmask = 0, cand = 0, total = 0;
 };
 
+// Threads of the look-ahead emit block: kTkThreads stream the memory, the
+// other kRkHashThreads hash the next step's keys.
+constexpr int kRkHashThreads = 128;
+constexpr int kRkSplitThreads = kTkThreads + kRkHashThreads;
+
 static RkLayout rk_layout(const gce_table* t, int32_t W) {
     RkLayout o;
     Carver c;
     const bool on = t->ckind == GCE_KIND_RANDK;
     o.S = on ? int64_t(W) * int64_t(t->comp.size()) : 0;
     o.TT = on ? int64_t(W) * t->tiles_pw : 0;
-    o.segs = c.take<RkSeg>(2 * o.S);  // two sets: this step's and the next one's
-    o.tile_cnt = c.take<int32_t>(o.TT);
-    o.bitmask = c.take<uint32_t>(o.TT * kRkWords);
+    // two sets of each, by step parity: this step's and the next one's
+    o.segs = c.take<RkSeg>(2 * o.S);
+    o.tile_cnt = c.take<int32_t>(2 * o.TT);
+    o.bitmask = c.take<uint32_t>(2 * o.TT * kRkWords);
     o.cand = c.take<RkEntry>(o.S ? int64_t(W) * t->comp_N : 0);
     o.total = c.off;
     return o;
@@ -124,65 +131,83 @@ __global__ void __launch_bounds__(256) rk_setup_kernel(const DevLayer* __restric
                      status);
 }
 
+// Barrier over the block (kId 0) or, with a named barrier, over the kThreads
+// threads of one warp group.
+template <int kId, int kThreads>
+__device__ __forceinline__ void group_sync() {
+    if constexpr (kId == 0) __syncthreads();
+    else asm volatile("bar.sync %0, %1;" ::"r"(kId), "r"(kThreads) : "memory");
+}
+
 // Key pass over one tile t (worker w, layer L): the bitmask words of key < lo,
 // the tile's count below lo and the band entries [lo, hi] appended to the
 // layer's list.  kRedo: re-list a failed layer whole (band = every key,
-// nothing below it).  Run by the whole block; g.k != 0.
-template <bool kRedo>
+// nothing below it).  Run by a group of kThreads threads (gtid = the thread's
+// index in it) that syncs on barrier kBar; g.k != 0.
+template <bool kRedo, int kThreads = kTkThreads, int kBar = 0>
 __device__ __forceinline__ void rk_keys_tile(int64_t t, int w, int lt, const DevLayer& L,
                                              RkSeg& g, int64_t comp_N, int32_t* tile_cnt,
-                                             uint32_t* bitmask, RkEntry* cand, int* s_red) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+                                             uint32_t* bitmask, RkEntry* cand, int* s_red,
+                                             int gtid) {
+    constexpr int kChunks = kRkWords / kThreads;  // 32-element words a thread
+    static_assert(kChunks * kThreads == kRkWords, "a tile's words split evenly");
+    const int lane = gtid & 31, gwarp = gtid >> 5;
     const uint32_t lo = kRedo ? 0u : g.lo, hi = kRedo ? 0xFFFFFFFFu : g.hi;
     const uint32_t span = hi - lo;  // lo <= key <= hi  iff  key - lo <= hi - lo (unsigned)
     const uint64_t base = g.base;
     const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
-    const int64_t e0 = tstart + int64_t(tid) * 32;
-    const uint64_t x0 = base + uint64_t(e0 + 1) * kGamma;  // generator state of element e0
-    uint32_t below = 0, inband = 0;
-    if (e0 + 32 <= L.n) {
+    int nbelow = 0;
+#pragma unroll 1
+    for (int c = 0; c < kChunks; ++c) {
+        const int word = gtid + c * kThreads;
+        const int64_t e0 = tstart + int64_t(word) * 32;
+        const uint64_t x0 = base + uint64_t(e0 + 1) * kGamma;  // generator state of element e0
+        uint32_t below = 0, inband = 0;
+        if (e0 + 32 <= L.n) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
-            below |= uint32_t(!kRedo && key < lo) << q;  // the redo lists every key
-            inband |= uint32_t(key - lo <= span) << q;
-        }
-    } else {
-#pragma unroll
-        for (int q = 0; q < 32; ++q) {
-            const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
-            if (e0 + q < L.n) {
+            for (int q = 0; q < 32; ++q) {
+                const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
                 below |= uint32_t(!kRedo && key < lo) << q;  // the redo lists every key
                 inband |= uint32_t(key - lo <= span) << q;
             }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
+                if (e0 + q < L.n) {
+                    below |= uint32_t(!kRedo && key < lo) << q;  // the redo lists every key
+                    inband |= uint32_t(key - lo <= span) << q;
+                }
+            }
+        }
+        bitmask[t * kRkWords + word] = below;
+        nbelow += __popc(below);
+        // band entries: order does not matter, the resolve sorts them out
+        const int nb = __popc(inband);
+        const int incl = warp_inclusive_scan(nb);
+        int wbase = 0;
+        if (lane == 31 && incl) wbase = atomicAdd(kRedo ? &g.cand_redo : &g.cand, incl);
+        wbase = __shfl_sync(kFull, wbase, 31);
+        RkEntry* out = cand + int64_t(w) * comp_N + L.sp_off + wbase + (incl - nb);
+        int pos = 0;
+        while (inband) {  // few band entries: their keys are recomputed
+            const int q = __ffs(inband) - 1;
+            inband &= inband - 1;
+            const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
+            out[pos++] = RkEntry{key, int32_t(e0 + q)};
         }
     }
-    bitmask[t * kRkWords + tid] = below;
     // tile count of keys below the band
-    const int c = warp_sum(__popc(below));
-    if (lane == 0) s_red[warp] = c;
-    __syncthreads();
-    if (tid == 0) {
+    const int cw = warp_sum(nbelow);
+    if (lane == 0) s_red[gwarp] = cw;
+    group_sync<kBar, kThreads>();
+    if (gtid == 0) {
         int tot = 0;
-        for (int i = 0; i < 8; ++i) tot += s_red[i];
+        for (int i = 0; i < kThreads / 32; ++i) tot += s_red[i];
         tile_cnt[t] = tot;
         if (tot) atomicAdd(&g.c_lo, tot);
     }
-    __syncthreads();
-    // band entries: order does not matter, the resolve sorts them out
-    const int nb = __popc(inband);
-    const int incl = warp_inclusive_scan(nb);
-    int wbase = 0;
-    if (lane == 31 && incl) wbase = atomicAdd(kRedo ? &g.cand_redo : &g.cand, incl);
-    wbase = __shfl_sync(kFull, wbase, 31);
-    RkEntry* out = cand + int64_t(w) * comp_N + L.sp_off + wbase + (incl - nb);
-    int pos = 0;
-    while (inband) {  // few band entries: their keys are recomputed
-        const int q = __ffs(inband) - 1;
-        inband &= inband - 1;
-        const uint32_t key = mix64_hi(x0 + uint64_t(q) * kGamma);
-        out[pos++] = RkEntry{key, int32_t(e0 + q)};
-    }
+    group_sync<kBar, kThreads>();  // s_red is read before the next tile writes it
 }
 
 template <bool kRedo>
@@ -203,7 +228,7 @@ __global__ void __launch_bounds__(256) rk_keys_kernel(const DevLayer* __restrict
         RkSeg& g = segs[int64_t(w) * ncomp + L.sidx];
         if (g.k == 0) continue;
         if (kRedo && !g.fail) continue;
-        rk_keys_tile<kRedo>(t, w, lt, L, g, comp_N, tile_cnt, bitmask, cand, s_red);
+        rk_keys_tile<kRedo>(t, w, lt, L, g, comp_N, tile_cnt, bitmask, cand, s_red, threadIdx.x);
     }
 }
 
@@ -398,29 +423,45 @@ __global__ void __launch_bounds__(1024) rk_scan_kernel(const DevLayer* __restric
     }
 }
 
-// kNext: once a tile's memory pass is done, the block also runs the next
-// step's key pass over the same tile (segs_next): ALU work that overlaps the
-// other blocks' memory traffic.  The tile's bitmask words and offset are read
-// before the block's barriers and rewritten after them, by the same block.
-// Four blocks per SM (64 registers): the fifth register bank the look-ahead
-// variant would otherwise take costs a resident block and 3 % of the step,
-// more than the one value it spills.
+// kNext: the block's first kTkThreads threads run the memory pass (named
+// barrier 1) while its last kRkHashThreads threads run the next step's key
+// pass (segs_next) over the same tiles into the other parity's bitmask and
+// tile counts (named barrier 2): the two groups share no data, so the hash's
+// ALU work and the memory traffic overlap on every SM.  Without kNext the
+// block is the memory group alone.
 template <bool kNext>
-__global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
+__global__ void __launch_bounds__(kNext ? kRkSplitThreads : kTkThreads, kNext ? 2 : 4)
+rk_emit_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ tile_layer, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t vals_pw, int64_t comp_N,
     const float* __restrict__ grad, float* __restrict__ mem, float eta,
-    const RkSeg* __restrict__ segs, RkSeg* __restrict__ segs_next, int32_t* tile_off,
-    uint32_t* bitmask, RkEntry* __restrict__ cand, float* __restrict__ vals,
-    int32_t* __restrict__ idx, int32_t* __restrict__ status) {
+    const RkSeg* __restrict__ segs, RkSeg* __restrict__ segs_next, const int32_t* tile_off,
+    const uint32_t* bitmask, int32_t* tile_cnt_next, uint32_t* bitmask_next,
+    RkEntry* __restrict__ cand, float* __restrict__ vals, int32_t* __restrict__ idx,
+    int32_t* __restrict__ status) {
     grid_dependency_sync();
     constexpr int kIters = kTkPerThread / 4;
     constexpr int kWarps = kTkThreads / 32;
+    constexpr int kMemBar = kNext ? 1 : 0;
     __shared__ int32_t s_wt[kIters * kWarps];
-    __shared__ int s_red[8];
+    __shared__ int s_red[kRkHashThreads / 32];
     __shared__ int32_t s_toff;  // this tile's first payload slot
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int64_t total = int64_t(tiles_pw) * W;
+    if (kNext && threadIdx.x >= kTkThreads) {
+        // the hash group
+        const int gtid = int(threadIdx.x) - kTkThreads;
+        for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+            const int w = int(t / tiles_pw);
+            const int lt = int(t % tiles_pw);
+            const DevLayer L = layers[tile_layer[lt]];
+            RkSeg& gn = segs_next[int64_t(w) * ncomp + L.sidx];
+            if (gn.k == 0) continue;
+            rk_keys_tile<false, kRkHashThreads, 2>(t, w, lt, L, gn, comp_N, tile_cnt_next,
+                                                   bitmask_next, cand, s_red, gtid);
+        }
+        return;
+    }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
         const int w = int(t / tiles_pw);
         const int lt = int(t % tiles_pw);
@@ -440,8 +481,7 @@ __global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
         }
         const int64_t s = int64_t(w) * ncomp + L.sidx;
         const int32_t k = segs[s].k;
-        const bool next = kNext && segs_next[s].k != 0;
-        if (k == 0 && !next) continue;
+        if (k == 0) continue;
         const int64_t tstart = int64_t(lt - L.tile0) * kTkTile;
         const int cnt = int(min64(kTkTile, L.n - tstart));
         const int64_t ebase = int64_t(w) * N + L.offset + tstart;
@@ -449,7 +489,7 @@ __global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
         float* m = mem + ebase;
         const uint32_t* bm = bitmask + t * kRkWords;
         const bool vec = cnt == kTkTile && (ebase & 3) == 0;
-        if (k != 0) {
+        {
             // every load of the tile issued up front, then the arithmetic; the
             // memory first receives v everywhere, and the few chosen entries
             // are read back and zeroed once their payload slots are known
@@ -508,14 +548,14 @@ __global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
                 incl[j] = warp_inclusive_scan(__popc((flags >> (4 * j)) & 0xFu));
                 if (lane == 31) s_wt[j * kWarps + warp] = incl[j];
             }
-            __syncthreads();
+            group_sync<kMemBar, kTkThreads>();
             if (warp == 0) {
                 const int a = s_wt[2 * lane], b = s_wt[2 * lane + 1];
                 const int x = warp_inclusive_scan(a + b);
                 s_wt[2 * lane] = x - a - b;
                 s_wt[2 * lane + 1] = x - b;
             }
-            __syncthreads();
+            group_sync<kMemBar, kTkThreads>();
             const int base = s_toff;
             float* vout = vals + int64_t(w) * vals_pw + L.val_off;
             int32_t* iout = idx + int64_t(w) * vals_pw + L.val_off;
@@ -534,12 +574,8 @@ __global__ void __launch_bounds__(kTkThreads, 4) rk_emit_kernel(
                     pos += (f >> q) & 1u;
                 }
             }
-            __syncthreads();  // words, s_wt and s_toff are consumed
+            group_sync<kMemBar, kTkThreads>();  // s_wt and s_toff are consumed
         }
-        // the next step's key pass over the same tile: ALU work while the
-        // other resident blocks stream memory
-        if (next)
-            rk_keys_tile<false>(t, w, lt, L, segs_next[s], comp_N, tile_off, bitmask, cand, s_red);
     }
 }
 
@@ -563,8 +599,13 @@ static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const floa
     int32_t* status = static_cast<int32_t*>(ws);
     if (lay.S > 0) {
         const int32_t ncomp = int32_t(t->comp.size());
-        int32_t* tile_cnt = at<int32_t>(ws, lay.tile_cnt);
-        uint32_t* bitmask = at<uint32_t>(ws, lay.bitmask);
+        // this step's bitmask and tile counts, and the next step's (which the
+        // look-ahead fills), by step parity
+        int32_t* tile_cnt = at<int32_t>(ws, lay.tile_cnt) + (step & 1) * lay.TT;
+        uint32_t* bitmask = at<uint32_t>(ws, lay.bitmask) + (step & 1) * lay.TT * kRkWords;
+        int32_t* tile_cnt_next = at<int32_t>(ws, lay.tile_cnt) + ((step + 1) & 1) * lay.TT;
+        uint32_t* bitmask_next =
+            at<uint32_t>(ws, lay.bitmask) + ((step + 1) & 1) * lay.TT * kRkWords;
         RkEntry* cand = at<RkEntry>(ws, lay.cand);
         // Run the next step's key pass inside this step's memory pass unless
         // the stream is being captured (a graph would replay one step number).
@@ -599,7 +640,7 @@ static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const floa
         static const int r_res1 = resident_blocks(rk_resolve_kernel<true>, 1024);
         static const int r_scan = resident_blocks(rk_scan_kernel, 1024);
         static const int r_emit0 = resident_blocks(rk_emit_kernel<false>, kTkThreads);
-        static const int r_emit1 = resident_blocks(rk_emit_kernel<true>, kTkThreads);
+        static const int r_emit1 = resident_blocks(rk_emit_kernel<true>, kRkSplitThreads);
         if (have) {
             GCE_LAUNCH(rk_refresh_k_kernel, wave_grid((lay.S + 255) / 256, 4, r_refresh), 256, 0,
                        st, t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
@@ -632,15 +673,15 @@ static int randk_step(const gce_table* t, int32_t W, int64_t worker0, const floa
                        t->d_layers, t->d_comp, ncomp, lay.S, k_or_rank, seed,
                        uint64_t(worker0), step + 1, sigma, segs_next, nullptr, tag,
                        tag_of(step + 1));
-            GCE_LAUNCH(rk_emit_kernel<true>, wave_grid(lay.TT, r_emit1, r_emit1), kTkThreads, 0, st,
-                       t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
-                       t->comp_N, grad, mem, eta, segs, segs_next, tile_cnt, bitmask, cand, vals,
-                       idx, status);
+            GCE_LAUNCH(rk_emit_kernel<true>, wave_grid(lay.TT, r_emit1, r_emit1), kRkSplitThreads,
+                       0, st, t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N,
+                       t->vals_pw, t->comp_N, grad, mem, eta, segs, segs_next, tile_cnt, bitmask,
+                       tile_cnt_next, bitmask_next, cand, vals, idx, status);
         } else {
             GCE_LAUNCH(rk_emit_kernel<false>, wave_grid(lay.TT, r_emit0, r_emit0), kTkThreads, 0,
                        st, t->d_layers, t->d_tile_layer, t->tiles_pw, W, ncomp, t->N, t->vals_pw,
-                       t->comp_N, grad, mem, eta, segs, nullptr, tile_cnt, bitmask, cand, vals,
-                       idx, status);
+                       t->comp_N, grad, mem, eta, segs, nullptr, tile_cnt, bitmask, nullptr,
+                       nullptr, cand, vals, idx, status);
         }
         if (check_launch() != GCE_OK) return GCE_ERR_CUDA;
         if (pipe) {
