@@ -503,10 +503,67 @@ __device__ __forceinline__ double block_sum_d(double x, double* s_red) {
     return t;
 }
 
+// Column passes of the Gram-Schmidt over this thread's rows (threadIdx.x,
+// + blockDim.x, ...), in row order, with kU rows' loads issued ahead of their
+// arithmetic.  ps_col_dot: sum of p_i * p_j; ps_col_axpy: p_j -= d p_i;
+// ps_col_scale: p_j = p_j / nu (0 when nu is 0).
+constexpr int kPsOrthThreads = 1024;
+
+__device__ __forceinline__ double ps_col_dot(const double* pd, int64_t R, int cap, int i, int j) {
+    constexpr int kU = 4;
+    const int64_t B = blockDim.x;
+    double part = 0.0;
+    int64_t row = threadIdx.x;
+    for (; row + (kU - 1) * B < R; row += kU * B) {
+        double a[kU], b[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            a[u] = pd[(row + u * B) * cap + i];
+            b[u] = pd[(row + u * B) * cap + j];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) part += a[u] * b[u];
+    }
+    for (; row < R; row += B) part += pd[row * cap + i] * pd[row * cap + j];
+    return part;
+}
+
+__device__ __forceinline__ void ps_col_axpy(double* pd, int64_t R, int cap, int i, int j,
+                                            double d) {
+    constexpr int kU = 4;
+    const int64_t B = blockDim.x;
+    int64_t row = threadIdx.x;
+    for (; row + (kU - 1) * B < R; row += kU * B) {
+        double a[kU], b[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            a[u] = pd[(row + u * B) * cap + i];
+            b[u] = pd[(row + u * B) * cap + j];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) pd[(row + u * B) * cap + j] = b[u] - d * a[u];
+    }
+    for (; row < R; row += B) pd[row * cap + j] -= d * pd[row * cap + i];
+}
+
+__device__ __forceinline__ void ps_col_scale(double* pd, int64_t R, int cap, int j, double nu) {
+    constexpr int kU = 4;
+    const int64_t B = blockDim.x;
+    int64_t row = threadIdx.x;
+    for (; row + (kU - 1) * B < R; row += kU * B) {
+        double b[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) b[u] = pd[(row + u * B) * cap + j];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) pd[(row + u * B) * cap + j] = nu > 0.0 ? b[u] / nu : 0.0;
+    }
+    for (; row < R; row += B) pd[row * cap + j] = nu > 0.0 ? pd[row * cap + j] / nu : 0.0;
+}
+
 // W outputs (one P per output); output w sums the partial P of workers
 // w*nsum ... w*nsum + nsum - 1 in worker order (nsum = 1: independent
 // replicas; W = 1, nsum = all workers: the data-parallel step).
-__global__ void __launch_bounds__(256) ps_orth_kernel(
+__global__ void __launch_bounds__(kPsOrthThreads) ps_orth_kernel(
     const DevLayer* __restrict__ layers, const PsLayer* __restrict__ ps,
     const int32_t* __restrict__ ps_layers, int32_t nps, int32_t W, int32_t nsum, int64_t P_pw,
     int64_t ppart_pw,
@@ -545,20 +602,12 @@ __global__ void __launch_bounds__(256) ps_orth_kernel(
         __syncthreads();
         for (int j = 0; j < r; ++j) {
             for (int i = 0; i < j; ++i) {
-                double part = 0.0;
-                for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
-                    part += pd[row * cap + i] * pd[row * cap + j];
-                const double dot = block_sum_d(part, s_red);
-                for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
-                    pd[row * cap + j] -= dot * pd[row * cap + i];
+                const double dot = block_sum_d(ps_col_dot(pd, R, cap, i, j), s_red);
+                ps_col_axpy(pd, R, cap, i, j, dot);
                 __syncthreads();
             }
-            double part = 0.0;
-            for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
-                part += pd[row * cap + j] * pd[row * cap + j];
-            const double nu = sqrt(block_sum_d(part, s_red));
-            for (int64_t row = threadIdx.x; row < R; row += blockDim.x)
-                pd[row * cap + j] = nu > 0.0 ? pd[row * cap + j] / nu : 0.0;
+            const double nu = sqrt(block_sum_d(ps_col_dot(pd, R, cap, j, j), s_red));
+            ps_col_scale(pd, R, cap, j, nu);
             __syncthreads();
         }
         float* p = P + int64_t(w) * P_pw + L.p_off;
@@ -1264,13 +1313,13 @@ static int ps_step(const gce_table* t, int32_t W, const float* grad, float* mem,
         double* qpart = at<double>(ws, lay.qpart);
         double* qd = at<double>(ws, lay.qd);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_orth = resident_blocks(ps_orth_kernel, 256);
+        static const int r_orth = resident_blocks(ps_orth_kernel, kPsOrthThreads);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<false>, 256);
         ps_launch_mq(t, W, t->Q_pw, grad, mem, eta, k_or_rank, Q, ppart, status, pd, t->pd_pw, qd,
                      lazy_rank, st);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
-        GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), 256, 0, st, t->d_layers, ps,
+        GCE_LAUNCH(ps_orth_kernel, wave_grid(int64_t(t->nps) * W, 8, r_orth), kPsOrthThreads, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, W, 1, t->P_pw, t->ppart_pw, t->pd_pw, k_or_rank, ppart,
                    pd, P, status, t->ps_ntall, tdone, t->L, lazy_rank);
         if (t->ps_ntall > 0) {
@@ -1357,14 +1406,14 @@ extern "C" int powersgd_dp_step(const gce_table* t, int32_t W, const float* grad
         float* qloc = at<float>(ws, lay.qloc);
         int32_t* tdone = at<int32_t>(ws, lay.tdone);
         const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
-        static const int r_orth = resident_blocks(ps_orth_kernel, 256);
+        static const int r_orth = resident_blocks(ps_orth_kernel, kPsOrthThreads);
         static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
         static const int r_qred = resident_blocks(ps_qred_kernel<true>, 256);
         // every worker reads the shared warm start Q (stride 0)
         ps_launch_mq(t, W, int64_t(0), grad, mem, eta, k_or_rank, Q, ppart, status, nullptr,
                      int64_t(0), nullptr, nullptr, st);
         // one P per layer from the partials of all W workers
-        GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
+        GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), kPsOrthThreads, 0, st, t->d_layers, ps,
                    t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank,
                    ppart, pd, P, status, t->ps_ntall, tdone, t->L, nullptr);
         if (t->ps_ntall > 0) {
@@ -1447,10 +1496,10 @@ extern "C" int powersgd_dp_orthogonalize(const gce_table* t, int32_t W, const in
     const PsLayer* ps = static_cast<const PsLayer*>(t->d_ps);
     double* pd = at<double>(ws, lay.pd);
     int32_t* tdone = at<int32_t>(ws, lay.tdone);
-    static const int r_orth = resident_blocks(ps_orth_kernel, 256);
+    static const int r_orth = resident_blocks(ps_orth_kernel, kPsOrthThreads);
     static const int r_tall = resident_blocks(ps_orth_tall_kernel, 256);
     // one P per layer from the partials of all W workers, in worker order
-    GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), 256, 0, st, t->d_layers, ps,
+    GCE_LAUNCH(ps_orth_kernel, wave_grid(t->nps, 8, r_orth), kPsOrthThreads, 0, st, t->d_layers, ps,
                t->d_ps_layers, t->nps, 1, W, int64_t(0), t->ppart_pw, t->pd_pw, k_or_rank, Ppart,
                pd, P, status, t->ps_ntall, tdone, t->L, nullptr);
     if (t->ps_ntall > 0) {
