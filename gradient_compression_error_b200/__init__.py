@@ -466,16 +466,17 @@ def set_sign_ahead(tiles):
 
 def sign_schedule(layer_tiles, W, ahead):
     """The pipelined signSGD kernel's work-item order (host only): a list of
-    runs (first item, first tile, kind), kind 0 norm, 1 update, -1 the
-    closing sentinel whose first item is the item count (include/gce.h)."""
+    runs (first item, lowest tile, kind, descending), kind 0 norm, 1 update,
+    -1 the closing sentinel whose first item is the item count; descending 1:
+    the run's tiles from the highest down (include/gce.h)."""
     tiles = (C.c_int32 * len(layer_tiles))(*[int(x) for x in layer_tiles])
     n = _i64()
     _check("gce_sign_schedule", lib().gce_sign_schedule(tiles, len(layer_tiles), int(W),
                                                         int(ahead), None, 0, C.byref(n)))
-    runs = (C.c_int64 * (3 * n.value))()
+    runs = (C.c_int64 * (4 * n.value))()
     _check("gce_sign_schedule", lib().gce_sign_schedule(tiles, len(layer_tiles), int(W),
                                                         int(ahead), runs, n.value, C.byref(n)))
-    return [(runs[3 * i], runs[3 * i + 1], runs[3 * i + 2]) for i in range(n.value)]
+    return [tuple(runs[4 * i + j] for j in range(4)) for i in range(n.value)]
 
 
 def set_sign_emit_first(on):

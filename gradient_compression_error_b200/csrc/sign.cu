@@ -280,9 +280,9 @@ __global__ void __launch_bounds__(256) sg_emit_kernel(
 // on with whatever scale is there.
 struct SgPhase {
     int64_t item0;  // first item of this run
-    int64_t t0;     // its first tile
+    int64_t t0;     // its lowest tile
     int32_t kind;   // 0 norm, 1 emit, -1 end
-    int32_t pad;
+    int32_t rev;    // 1: the run's tiles in descending order (item0 takes the highest)
 };
 
 constexpr uint32_t kSgSpinLimit = 1u << 21;  // polls (a sleep and an L2 load each): ~1 s
@@ -313,7 +313,8 @@ __global__ void __launch_bounds__(256, 4) sg_fused_kernel(
         const int64_t it = s_item;
         if (it >= nitems) break;
         const SgPhase P = phases[s_ph];
-        const int64_t t = P.t0 + (it - P.item0);
+        const int64_t off = it - P.item0;
+        const int64_t t = P.rev ? P.t0 + (phases[s_ph + 1].item0 - P.item0 - 1 - off) : P.t0 + off;
         const SgTile x = sg_tile(layers, tile_layer, tiles_pw, ncomp, N, t);
         if (P.kind == 0) {
             sg_norm_tile<true>(x, t, tiles_pw, vals_pw, grad, mem, eta, partials, done, ready,
@@ -409,6 +410,12 @@ static std::vector<SgPhase> sg_schedule_of(const std::vector<int64_t>& starts, i
     }
     std::vector<SgPhase> ph;
     int64_t np = 0, ep = 0, item = 0;  // next norm tile, next emit tile
+    // [first, end) tiles of the (worker, layer) holding tile x
+    auto seg_of = [&](int64_t x, int64_t* first, int64_t* end) {
+        const auto it = std::upper_bound(starts.begin(), starts.end(), x);
+        *first = it == starts.begin() ? 0 : *(it - 1);
+        *end = it == starts.end() ? T : *it;
+    };
     while (ep < T) {
         // tiles below `limit` belong to layers whose norm tiles are all placed
         int64_t limit = T;
@@ -423,8 +430,32 @@ static std::vector<SgPhase> sg_schedule_of(const std::vector<int64_t>& starts, i
             item += e - np;
             np = e;
         } else {
-            const int64_t e = std::min(limit, ep + kSgRun);
-            ph.push_back(SgPhase{item, ep, 1, 0});
+            // A layer longer than the look-ahead is updated from its last tile
+            // down: by the time its norm is complete only its last tiles are
+            // still in L2, and they are read first.  Runs stop at the edges of
+            // such a layer.
+            int64_t first = 0, end = 0;
+            seg_of(ep, &first, &end);
+            const bool big = end - first > ahead;
+            int64_t e = std::min(limit, ep + kSgRun);
+            if (big) {
+                e = std::min(e, end);
+            } else {
+                // stop before the first reversed layer inside the run
+                for (int64_t x = end; x < e;) {
+                    int64_t f2 = 0, e2 = 0;
+                    seg_of(x, &f2, &e2);
+                    if (e2 - f2 > ahead) {
+                        e = x;
+                        break;
+                    }
+                    x = e2;
+                }
+            }
+            if (big)  // the mirror of [ep, e) inside [first, end)
+                ph.push_back(SgPhase{item, first + end - e, 1, 1});
+            else
+                ph.push_back(SgPhase{item, ep, 1, 0});
             item += e - ep;
             ep = e;
         }
@@ -527,9 +558,10 @@ extern "C" int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int3
     const std::vector<SgPhase> ph = sg_schedule_of(starts, int64_t(W) * tiles_pw, ahead, &nitems);
     *nruns = int64_t(ph.size());
     for (int64_t i = 0; i < std::min<int64_t>(cap, int64_t(ph.size())); ++i) {
-        runs[3 * i] = ph[size_t(i)].item0;
-        runs[3 * i + 1] = ph[size_t(i)].t0;
-        runs[3 * i + 2] = ph[size_t(i)].kind;
+        runs[4 * i] = ph[size_t(i)].item0;
+        runs[4 * i + 1] = ph[size_t(i)].t0;
+        runs[4 * i + 2] = ph[size_t(i)].kind;
+        runs[4 * i + 3] = ph[size_t(i)].rev;
     }
     return GCE_OK;
 }

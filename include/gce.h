@@ -389,10 +389,11 @@ GCE_API int gce_set_sign_emit_first(int32_t on);
  * layer_tiles[l] >= 1 tiles each (8192 elements a tile, layers numbered
  * consecutively, worker-major), with the norm at most `ahead` tiles in front
  * (1 .. 2^20), or ahead = -1 for the wait test's order (every update first).
- * Writes up to cap runs to runs[3 * i ..]: (first item, first tile, kind:
+ * Writes up to cap runs to runs[4 * i ..]: (first item, lowest tile, kind:
  * 0 norm, 1 update, -1 the closing sentinel, whose first item is the item
- * count); *nruns = the number of runs, sentinel included.  Bad arguments
- * give GCE_ERR_ARG.
+ * count; order: 0 ascending tiles, 1 descending -- the updates of a layer of
+ * more than `ahead` tiles run from its last tile down); *nruns = the number
+ * of runs, sentinel included.  Bad arguments give GCE_ERR_ARG.
  */
 GCE_API int gce_sign_schedule(const int32_t* layer_tiles, int32_t ncomp, int32_t W, int32_t ahead,
                               int64_t* runs, int64_t cap, int64_t* nruns);

@@ -4,9 +4,11 @@ checked on the host.
 The kernel's waits end only if every memory-update tile comes after all norm
 tiles of its (worker, layer): blocks take items in this order, an update waits
 for its layer's scale, and a norm waits on nothing.  These tests check that
-property, that each tile is normed once and updated once, that the order is
-the two ascending tile sequences interleaved, and that the norm stays within
-the look-ahead (beyond it only while a layer's norm tiles are still being
+property, that each tile is normed once and updated once, that the norm runs
+in ascending tile order and so do the updates, except that a layer of more
+tiles than the look-ahead is updated from its last tile down (its last normed
+tiles are the ones still in L2), and that the norm stays within the
+look-ahead (beyond it only while a layer's norm tiles are still being
 placed), on BERT-base-shaped and ragged tables.  The order is built by the
 same C++ function the kernel's host code calls; no GPU is needed.
 """
@@ -27,11 +29,24 @@ def expand(runs):
     """(kind, tile) of every item, in item order."""
     assert runs[-1][2] == -1
     kinds, tiles = [], []
-    for (i0, t0, k), (i1, _, _) in zip(runs, runs[1:]):
-        assert i1 > i0 and k in (0, 1)
+    for (i0, t0, k, rev), (i1, _, _, _) in zip(runs, runs[1:]):
+        assert i1 > i0 and k in (0, 1) and rev in (0, 1)
+        assert not (k == 0 and rev)                     # norms always ascend
         kinds.append(np.full(i1 - i0, k, np.int8))
-        tiles.append(np.arange(t0, t0 + i1 - i0, dtype=np.int64))
+        t = np.arange(t0, t0 + i1 - i0, dtype=np.int64)
+        tiles.append(t[::-1] if rev else t)
     return np.concatenate(kinds), np.concatenate(tiles)
+
+
+def expected_update_order(tiles_per_layer, W, ahead):
+    """Ascending tiles, each layer of more than `ahead` tiles reversed."""
+    out, t = [], 0
+    for _ in range(W):
+        for n in tiles_per_layer:
+            seg = np.arange(t, t + n, dtype=np.int64)
+            out.append(seg[::-1] if ahead >= 1 and n > ahead else seg)
+            t += n
+    return np.concatenate(out)
 
 
 def check(tiles_per_layer, W, ahead):
@@ -39,12 +54,13 @@ def check(tiles_per_layer, W, ahead):
     runs = g.sign_schedule(tiles_per_layer, W, ahead)
     tpw = sum(tiles_per_layer)
     T = W * tpw
-    assert runs[-1] == (2 * T, T, -1)
+    assert runs[-1] == (2 * T, T, -1, 0)
     kind, tile = expand(runs)
     assert len(kind) == 2 * T and tile.min() >= 0 and tile.max() < T
     norm_t, upd_t = tile[kind == 0], tile[kind == 1]
     assert np.array_equal(norm_t, np.arange(T))        # each tile normed once, in order
-    assert np.array_equal(upd_t, np.arange(T))         # and updated once, in order
+    # and updated once, long layers from the last tile down
+    assert np.array_equal(upd_t, expected_update_order(tiles_per_layer, W, ahead))
     # segment (worker, layer) of every tile
     seg_of_local = np.repeat(np.arange(len(tiles_per_layer)), tiles_per_layer)
     seg = (np.arange(T) // tpw) * len(tiles_per_layer) + seg_of_local[np.arange(T) % tpw]
@@ -80,21 +96,35 @@ def test_ragged_order(W, ahead):
 
 def test_one_tile_and_large_look_ahead():
     runs = check([1], 1, 768)
-    assert runs == [(0, 0, 0), (1, 0, 1), (2, 1, -1)]
+    assert runs == [(0, 0, 0, 0), (1, 0, 1, 0), (2, 1, -1, 0)]
+
+
+def test_layer_longer_than_the_look_ahead_is_updated_backwards():
+    """BERT-base's embedding (2862 tiles) at the default look-ahead of 768:
+    its update starts at its last tile, the one normed most recently."""
+    assert BERT[0] == 2862
+    kind, tile = expand(check(BERT, 2, 768))
+    upd = tile[kind == 1]
+    assert upd[0] == BERT[0] - 1 and upd[BERT[0] - 1] == 0
+    second = sum(BERT)                                  # worker 1's embedding
+    k = np.flatnonzero(upd == second + BERT[0] - 1)[0]
+    assert np.array_equal(upd[k:k + BERT[0]], np.arange(second + BERT[0] - 1, second - 1, -1))
 
 
 def test_look_ahead_interleaves_norm_and_update_runs():
     """With many small layers and a short look-ahead the order alternates
     (the point of the schedule): updates start long before the last norm."""
     runs = check([4] * 200, 2, 64)
-    kinds = [k for _, _, k in runs[:-1]]
+    kinds = [k for _, _, k, _ in runs[:-1]]
     first_update = kinds.index(1)
     assert first_update < 10 and 0 in kinds[first_update:]
 
 
 def test_wait_test_order_puts_every_update_first():
     T = sum(RAGGED) * 2
-    kind, tile = expand(gce().sign_schedule(RAGGED, 2, -1))
+    runs = gce().sign_schedule(RAGGED, 2, -1)
+    assert all(r[3] == 0 for r in runs)
+    kind, tile = expand(runs)
     assert np.all(kind[:T] == 1) and np.all(kind[T:] == 0)
     assert np.array_equal(tile[:T], np.arange(T)) and np.array_equal(tile[T:], np.arange(T))
 
