@@ -29,7 +29,7 @@ struct DevLayer {
     int32_t sidx;           // index among compressed layers, -1 for DENSE
     int32_t dc_tile0;       // first decode tile of this layer (all layers, per table)
     int32_t dc_ntiles;      // decode tiles of this layer
-    int32_t dc_base;        // first slot of this layer's ntiles+1 tile bounds
+    int32_t dc_base;        // first slot of this layer's nspans+1 span bounds
 };
 
 // One main tile's layer fields, for kernels whose per-tile work is short:
@@ -75,7 +75,7 @@ struct gce_table {
     int32_t* d_dtile_layer = nullptr;
     int32_t* d_dtile_start = nullptr;      // element start of each dense tile
     int32_t dc_tiles = 0;                  // decode tiles over all layers
-    int32_t dc_slots = 0;                  // tile-bound slots per worker (tiles + L)
+    int32_t dc_slots = 0;                  // span-bound slots per worker (spans + L)
     int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
     int32_t dc_nl_n = 0;                   // decode tiles of sparse and DENSE layers
     int32_t* d_dc_nl_tiles = nullptr;      // their decode tile ids
@@ -338,6 +338,8 @@ __device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) 
 // host entry points shared between translation units
 constexpr int kDcTileLog = 12;              // decode tile: 4096 output elements
 constexpr int kDcTile = 1 << kDcTileLog;
+constexpr int kDcSpanLog = 10;              // decode span: 1024 outputs, a warp's share
+constexpr int kDcSpan = 1 << kDcSpanLog;    // of a tile; payload entry bounds per span
 constexpr int kDcBoundChunk = 8192;         // payload entries per bound unit
 constexpr int kDenseTile = 4096;            // elements per tile of a DENSE layer
 

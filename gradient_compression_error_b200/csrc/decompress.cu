@@ -21,8 +21,7 @@
 namespace gce {
 
 constexpr int kDcThreads = 128;                   // 4 warps per decode tile
-constexpr int kDcSpan = kDcTile / (kDcThreads / 32);  // outputs each warp owns: 1024
-constexpr int kDcStage = 960;   // entries staged per pass (9 blocks of 24 KB fit an SM)
+static_assert(kDcSpan * (kDcThreads / 32) == kDcTile, "a warp owns one span of a tile");
 
 size_t decompress_ws_bytes(const gce_table* t, int32_t W) {
     Carver c;
@@ -35,8 +34,8 @@ __device__ __forceinline__ int32_t layer_k(const DevLayer& L, const int32_t* k_o
     return (k >= 1 && k <= L.cap) ? k : 0;  // out of range: the layer contributes nothing
 }
 
-// bounds[w][L.dc_base + tt] = first payload entry of (w, l) whose index lies in
-// decode tile tt or later; slot ntiles holds k.
+// bounds[w][L.dc_base + ss] = first payload entry of (w, l) whose index lies in
+// decode span ss (1024 outputs) or later; slot nspans holds k.
 __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restrict__ layers,
                                                         const int32_t* __restrict__ bunit_layer,
                                                         const int32_t* __restrict__ bunit_chunk,
@@ -54,7 +53,7 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
         const DevLayer L = layers[l];
         const int32_t k = layer_k(L, k_or_rank, l);
         int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base;
-        const int32_t nt = L.dc_ntiles;
+        const int32_t nt = int32_t((L.n + kDcSpan - 1) >> kDcSpanLog);  // spans of the layer
         const int64_t j0 = int64_t(bunit_chunk[bu]) * kDcBoundChunk;
         if (k == 0) {
             if (j0 == 0)
@@ -76,8 +75,8 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
             for (int q = 0; q < kBatch; ++q) {
                 const int64_t j = jb + int64_t(q) * blockDim.x;
                 if (j >= j1) continue;
-                const int32_t tj = min(max(cur[q], 0) >> kDcTileLog, nt);
-                const int32_t tp = j > 0 ? min(max(prev[q], 0) >> kDcTileLog, nt) : -1;
+                const int32_t tj = min(max(cur[q], 0) >> kDcSpanLog, nt);
+                const int32_t tp = j > 0 ? min(max(prev[q], 0) >> kDcSpanLog, nt) : -1;
                 for (int32_t tt = tp + 1; tt <= tj; ++tt) b[tt] = int32_t(j);
                 if (j == k - 1)
                     for (int32_t tt = tj + 1; tt <= nt; ++tt) b[tt] = k;
@@ -86,43 +85,47 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
     }
 }
 
-// First position in [l, r) of the sorted run s[l..r) whose value is >= key.
-__device__ __forceinline__ int lower_bound_smem(const int32_t* s, int l, int r, int key) {
-    while (l < r) {
-        const int m = (l + r) >> 1;
-        if (s[m] < key) l = m + 1;
-        else r = m;
-    }
-    return l;
-}
-
-// The staged entries (tile-relative index, value) that fall in this warp's
-// kDcSpan outputs are added to the accumulator, one worker after the other.  The
-// stage holds entries [c0, c0 + cn) of the tile's worker-ordered list, and
-// each worker's run is sorted by index, so lane w finds worker w's part of
-// the warp's range by binary search in shared memory.  Within one worker the
-// indices are distinct, so the lanes add without conflict.  Run by a full
-// warp; W <= 32.
-__device__ __forceinline__ void dc_add_staged(float* acc, const int32_t* s_sidx,
-                                              const float* s_sval, const int32_t* s_off,
-                                              int c0, int cn, int W, int warp, int cnt) {
+// The entries of every worker that fall in this warp's span (outputs [lo, lo +
+// kDcSpan) of the tile that starts at index `start`) added to the accumulator in
+// worker order.  Lane w < W holds worker w's entry range [a, a + c) of the span
+// (from the span bounds); the warp walks the W ranges one after the other, 32
+// entries a round, loading each entry's index and value into a lane, and adds a
+// round's entries worker by worker (within one worker the indices are
+// distinct, so its lanes add without conflict).  Run by a full warp; W <= 32.
+__device__ __forceinline__ void dc_add_span(float* acc, int64_t start, int W, int32_t a,
+                                            int32_t c, const float* __restrict__ vals,
+                                            const int32_t* __restrict__ idx, int64_t vals_pw,
+                                            int64_t val_off) {
     const int lane = threadIdx.x & 31;
-    const int lo = warp * kDcSpan, hi = min(lo + kDcSpan, cnt);
-    int a = 0, b = 0;
-    if (lane < W) {
-        const int e = lane + 1 < W ? s_off[lane + 1] : s_off[32];
-        const int r0 = min(max(s_off[lane] - c0, 0), cn);
-        const int r1 = min(max(e - c0, r0), cn);
-        a = lower_bound_smem(s_sidx, r0, r1, lo);
-        b = lower_bound_smem(s_sidx, a, r1, hi);
-    }
-    for (int w = 0; w < W; ++w) {
-        const int aw = __shfl_sync(kFull, a, w), bw = __shfl_sync(kFull, b, w);
-        for (int j = aw + lane; j < bw; j += 32) {
-            const int i = s_sidx[j];
-            if (i >= lo && i < hi) acc[i] = __fadd_rn(acc[i], s_sval[j]);  // sorted input: always
+    const int32_t incl = warp_inclusive_scan(c);
+    const int32_t excl = incl - c;
+    const int32_t total = __shfl_sync(kFull, incl, 31);
+    for (int32_t q0 = 0; q0 < total; q0 += 32) {
+        const int32_t q = q0 + lane;
+        // the worker of entry q: the last w < W whose range starts at or before q
+        int w = 0;
+#pragma unroll
+        for (int step = 16; step > 0; step >>= 1) {
+            const int32_t e = __shfl_sync(kFull, excl, min(w + step, 31));
+            if (w + step < W && e <= q) w += step;
         }
-        __syncwarp();
+        const int32_t aw = __shfl_sync(kFull, a, w), ew = __shfl_sync(kFull, excl, w);
+        const bool have = q < total;
+        int32_t i = 0;
+        float v = 0.0f;
+        if (have) {
+            const int64_t o = int64_t(w) * vals_pw + val_off + aw + (q - ew);
+            i = int32_t(int64_t(__ldcg(idx + o)) - start);
+            v = __ldcg(vals + o);
+        }
+        unsigned pending = __ballot_sync(kFull, have);
+        while (pending) {
+            const int wl = __shfl_sync(kFull, w, __ffs(pending) - 1);
+            const bool mine = have && w == wl;
+            if (mine) acc[i] = __fadd_rn(acc[i], v);
+            __syncwarp();
+            pending &= ~__ballot_sync(kFull, mine);
+        }
     }
 }
 
@@ -162,21 +165,12 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     float* __restrict__ out) {
     grid_dependency_sync();
     __shared__ __align__(16) float acc[kDcTile];
-    // per-worker entry ranges of the tile, double-buffered by sparse-tile
-    // parity: warp 0 fills the next tile's copy while a slower warp may still
-    // be reading this tile's in dc_add_staged (no barrier lies between the
-    // two); the copy is reused only after the next tile's barrier, which every
-    // warp reaches after it has finished with this tile
-    __shared__ int32_t s_first2[2][32], s_off2[2][33];
-    __shared__ int32_t s_sidx[kDcStage];
-    __shared__ float s_sval[kDcStage];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // the accumulator is all zero between sparse tiles: each warp zeroes the
     // part it writes out
     for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
         reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
-    int par = 0;  // parity of the staged sparse tiles this block has taken
     for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
         const int32_t t = tile_list ? tile_list[u] : u;
         const int32_t l = dc_tile_layer[t];
@@ -188,78 +182,34 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
         if (L.kind == GCE_KIND_TOPK || L.kind == GCE_KIND_RANDK) {
             const int32_t k = layer_k(L, k_or_rank, l);
             if (W <= 32) {
-                // Warp w of the block owns outputs [w, w + 1) x kDcSpan of the
-                // tile: it adds the staged entries that fall there and writes
-                // them out, so the accumulator needs no block-wide barrier
-                // between the adds and the write.  Every worker's entry range
-                // for the tile is read at once, then the entries are staged
-                // in worker order, kDcStage at a time.
-                int32_t* s_first = s_first2[par];
-                int32_t* s_off = s_off2[par];
-                par ^= 1;
-                if (warp == 0) {
-                    int32_t a = 0, e = 0;
+                // Warp `warp` owns span 4 tt + warp of the layer (tile outputs
+                // [warp, warp + 1) x kDcSpan): it reads its own entry bounds,
+                // adds its entries in worker order and writes the span out; the
+                // warps of the block never wait for one another here.
+                const int lo = warp * kDcSpan;
+                if (lo < cnt) {
+                    int32_t a = 0, c = 0;
                     if (lane < W) {
-                        const int32_t* b = bounds + int64_t(lane) * dc_slots + L.dc_base + tt;
+                        const int32_t* b = bounds + int64_t(lane) * dc_slots + L.dc_base +
+                                           (tt << (kDcTileLog - kDcSpanLog)) + warp;
                         a = min(max(b[0], 0), k);
-                        e = min(max(b[1], a), k);
-                        s_first[lane] = a;
+                        c = min(max(b[1], a), k) - a;
                     }
-                    const int c = e - a;
-                    const int incl = warp_inclusive_scan(c);
-                    if (lane < W) s_off[lane] = incl - c;
-                    if (lane == 31) s_off[32] = incl;
+                    dc_add_span(acc, start, W, a, c, vals, idx, vals_pw, L.val_off);
+                    __syncwarp();
+                    dc_write_quarter<kApply>(acc, o, cnt, warp, scale,
+                                             ((L.offset + start) & 3) == 0);
                 }
-                __syncthreads();
-                const int total = s_off[32];
-                int c0 = 0;
-                do {
-                    const int cn = min(kDcStage, total - c0);
-                    if (c0 > 0) __syncthreads();  // every warp is done with the last chunk
-                    // kSB entries per thread in flight: all loads first, then the stores
-                    constexpr int kSB = 4;
-                    for (int q0 = 0; q0 < cn; q0 += kSB * kDcThreads) {
-                        int32_t ri[kSB];
-                        float rv[kSB];
-#pragma unroll
-                        for (int e = 0; e < kSB; ++e) {
-                            const int q = q0 + e * kDcThreads + int(threadIdx.x);
-                            ri[e] = 0;
-                            rv[e] = 0.0f;
-                            if (q < cn) {
-                                const int qq = c0 + q;
-                                int w = 0;  // the last worker whose entries start at or before qq
-#pragma unroll
-                                for (int step = 16; step > 0; step >>= 1)
-                                    if (w + step < W && s_off[w + step] <= qq) w += step;
-                                const int64_t o2 = int64_t(w) * vals_pw + L.val_off + s_first[w] +
-                                                   (qq - s_off[w]);
-                                ri[e] = idx[o2];
-                                rv[e] = vals[o2];
-                            }
-                        }
-#pragma unroll
-                        for (int e = 0; e < kSB; ++e) {
-                            const int q = q0 + e * kDcThreads + int(threadIdx.x);
-                            if (q < cn) {
-                                s_sidx[q] = int32_t(int64_t(ri[e]) - start);
-                                s_sval[q] = rv[e];
-                            }
-                        }
-                    }
-                    __syncthreads();
-                    dc_add_staged(acc, s_sidx, s_sval, s_off, c0, cn, W, warp, cnt);
-                    c0 += kDcStage;
-                } while (c0 < total);
-                __syncwarp();
-                dc_write_quarter<kApply>(acc, o, cnt, warp, scale, ((L.offset + start) & 3) == 0);
                 continue;
             }
             // more than 32 workers: one worker at a time, straight from memory
             for (int w = 0; w < W; ++w) {
                 __syncthreads();
-                const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base + tt;
-                const int32_t a = min(max(b[0], 0), k), e = min(max(b[1], a), k);
+                const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base;
+                const int32_t s0 = tt << (kDcTileLog - kDcSpanLog);
+                const int32_t s1 = min(s0 + (kDcTile >> kDcSpanLog),
+                                       int32_t((L.n + kDcSpan - 1) >> kDcSpanLog));
+                const int32_t a = min(max(b[s0], 0), k), e = min(max(b[s1], a), k);
                 const float* v = vals + int64_t(w) * vals_pw + L.val_off;
                 const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
                 for (int32_t j = a + threadIdx.x; j < e; j += blockDim.x) {
@@ -509,8 +459,8 @@ extern "C" int gce_memsgd_eta(int64_t step, double mu, double a, float* eta) {
 // synchronisation.  For them, decompress_accumulate_noalloc keeps its only
 // scratch -- the per-tile entry bounds -- in the fixed array below, which the
 // module reserves on every GPU that loads this library until the process
-// exits.  4 MiB: W x (decode tiles of 4096 elements + layers) <= 1,048,576
-// bound slots (the BERT-base table at W = 8 uses 214,144).
+// exits.  4 MiB: W x (decode spans of 1024 elements + layers) <= 1,048,576
+// bound slots (the BERT-base table at W = 8 uses 856,088).
 constexpr int64_t kNoAllocBoundSlots = int64_t(1) << 20;
 static __device__ __align__(256) int32_t g_noalloc_bounds[kNoAllocBoundSlots];
 

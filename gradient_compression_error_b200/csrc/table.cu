@@ -279,7 +279,7 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
             dc_tile_layer.push_back(l);
         }
         dc_tiles += x.dc_ntiles;
-        dc_slots += x.dc_ntiles + 1;
+        dc_slots += int32_t((n + kDcSpan - 1) / kDcSpan) + 1;
         if (d.kind == GCE_KIND_TOPK || d.kind == GCE_KIND_RANDK) {
             const int32_t chunks = (d.cap + kDcBoundChunk - 1) / kDcBoundChunk;
             for (int32_t c = 0; c < chunks; ++c) {

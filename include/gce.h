@@ -495,8 +495,8 @@ GCE_API int gce_memsgd_eta(int64_t step, double mu, double a, float* eta);
  * decompress_accumulate minus ws / ws_bytes; it allocates nothing.  Its
  * scratch is a fixed 4 MiB array inside the library, reserved on every GPU
  * that loads the library until the process exits, so the table and W must
- * satisfy W x (decode tiles of 4096 elements + layers) <= 1,048,576 (the
- * BERT-base table at W = 8 needs 214,144); larger ones return
+ * satisfy W x (decode spans of 1024 elements + layers) <= 1,048,576 (the
+ * BERT-base table at W = 8 needs 856,088); larger ones return
  * GCE_ERR_WORKSPACE.  Every call made outside stream capture looks up the
  * current device's copy of the array (cudaGetSymbolAddress); a call made
  * while its stream is being captured reuses the address of the last call

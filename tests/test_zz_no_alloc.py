@@ -132,9 +132,9 @@ def test_noalloc_rejects_tables_beyond_its_scratch():
     need_gpu()
     g = gce()
     lib = g.lib()
-    layers = [dict(rows=1 << 24, cols=1, kind="topk", cap=10)]    # 4097 bound slots per worker
+    layers = [dict(rows=1 << 24, cols=1, kind="topk", cap=10)]    # 16,385 bound slots per worker
     table = g.Table(layers)
-    W = 256                                                        # 1,048,832 > 1,048,576
+    W = 64                                                         # 1,048,640 > 1,048,576
     vals = torch.zeros((1, 16), device="cuda")
     idx = torch.zeros((1, 16), dtype=torch.int32, device="cuda")
     out = torch.zeros(16, device="cuda")
