@@ -43,9 +43,11 @@ constexpr int kPsCB = 1024;   // columns per chunk (256 threads x 4)
 constexpr int kPsRB3 = 256;   // most rows per M^T P tile (its partial's row block)
 constexpr int kPsRB3Small = 64;  // rows per such block of a layer under kPsTallTileMin elements
 constexpr int kPsQB = 128;    // columns per Q-reduction tile
+constexpr int kPsQBSplit = 32; // the same for a layer whose sums are split over four lanes
+constexpr int kPsQSplit = 32; // row blocks from which four lanes share a Q entry's sum
 
 constexpr int64_t kPsTallRows = 8192;  // taller P: Gram-Schmidt spread over many blocks
-constexpr int kPsOrthChunk = 1024;     // rows per block in that case
+constexpr int kPsOrthChunk = 256;      // rows per block in that case
 
 // Precision of a layer's products.  Layers of at most kPsExactMax elements
 // form M Q, M^T P and the residual in fp64, from the fp64 orthonormal P and
@@ -109,8 +111,11 @@ int powersgd_plan(gce_table* t) {
                     o1.push_back(make_int4(l, int32_t(r0), ch, int32_t(std::min(rbh, L.rows - r0))));
             for (int32_t rb = 0; rb < x.nrb3; ++rb)
                 for (int32_t ch = 0; ch < x.nch1; ++ch) o3.push_back(make_int4(l, rb, ch, 0));
-            for (int32_t cb = 0; cb < (L.cols + kPsQB - 1) / kPsQB; ++cb)
-                tq.push_back(make_int4(l, cb, 0, 0));
+            // Q-reduction tiles (layer, first column, columns): narrower where
+            // four lanes share each entry's sum
+            const int64_t qw = x.nrb3 >= kPsQSplit ? kPsQBSplit : kPsQB;
+            for (int64_t c0 = 0; c0 < L.cols; c0 += qw)
+                tq.push_back(make_int4(l, int32_t(c0), int32_t(std::min(qw, L.cols - c0)), 0));
             ids.push_back(l);
         }
         ps[l] = x;
@@ -622,7 +627,7 @@ __global__ void __launch_bounds__(kPsOrthThreads) ps_orth_kernel(
 
 // ---- orthonormalise tall P over many blocks ---------------------------------------------
 // The same modified Gram-Schmidt, one launch per step: a launch first applies
-// the previous step's update to its 1024-row chunk (p_j -= d p_i, or
+// the previous step's update to its 256-row chunk (p_j -= d p_i, or
 // p_j /= ||p_j||), then forms its chunk's part of the next dot product; the
 // last block to finish adds the parts in chunk order (fixed, so the result is
 // deterministic) and leaves the scalar for the next launch.
@@ -693,8 +698,17 @@ __global__ void __launch_bounds__(256) ps_orth_tall_kernel(
             __syncthreads();
             if (s_last && threadIdx.x == 0) {
                 __threadfence();
+                // chunk order; eight parts in flight ahead of their adds
                 double s = 0.0;
-                for (int c = 0; c < X.nchunk; ++c) s += __ldcg(parts + c);
+                int c = 0;
+                for (; c + 8 <= X.nchunk; c += 8) {
+                    double v[8];
+#pragma unroll
+                    for (int b = 0; b < 8; ++b) v[b] = __ldcg(parts + c + b);
+#pragma unroll
+                    for (int b = 0; b < 8; ++b) s += v[b];
+                }
+                for (; c < X.nchunk; ++c) s += __ldcg(parts + c);
                 *scal = s;
                 tdone[int64_t(w) * ntall + X.tall] = 0;  // ready for the next launch
             }
@@ -834,7 +848,9 @@ __global__ void __launch_bounds__(256, std::is_same<T, float>::value ? 6 : 4) ps
 }
 
 // ---- Q = sum of the row-block partials (fp64, block order) ----------------------------------
-// Q' in fp64 to qd (stride Q_pw per worker) and rounded to fp32 to Q.
+// Q' in fp64 to qd (stride Q_pw per worker) and rounded to fp32 to Q.  A layer
+// of kPsQSplit or more row blocks sums them as four contiguous quarters, each
+// in block order, added in order (a fixed order, the same every call).
 // kMean (the data-parallel step): every worker's Q_w goes to Q (stride
 // Q_pw, fp32) and qd (fp64), and their mean -- fp32 sum of the rounded Q_w in
 // worker order from +0, times inv_w -- to qmean, one tile per block for all W
@@ -856,11 +872,20 @@ __global__ void __launch_bounds__(256) ps_qred_kernel(
         if (r == 0) continue;
         const int cap = L.cap;
         const int64_t C = L.cols;
-        const int64_t c0 = int64_t(d.y) * kPsQB;
-        const int cw = int(min64(kPsQB, C - c0));
-        for (int i = threadIdx.x; i < cw * r; i += blockDim.x) {
-            const int64_t c = c0 + i / r;
-            const int j = i % r;
+        const int64_t c0 = d.y;
+        const int cw = d.z;
+        // G lanes per entry: with many row blocks, lane g of the group sums
+        // the g-th contiguous quarter of them in block order and the group
+        // adds the quarters in order; with few, one lane sums them all
+        const int G = X.nrb3 >= kPsQSplit ? 4 : 1;
+        const int nb = (X.nrb3 + G - 1) / G;
+        const int n = cw * r * G;
+        for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+            const int i = i0 + int(threadIdx.x);
+            const bool act = i < n;
+            const int item = i / G, g = i - item * G;
+            const int64_t c = c0 + item / r;
+            const int j = item % r;
             float mean = 0.0f;
             for (int wi = 0; wi < (kMean ? W : 1); ++wi) {
                 const int ww = kMean ? wi : w;
@@ -869,22 +894,31 @@ __global__ void __launch_bounds__(256) ps_qred_kernel(
                 constexpr int kB = 8;
                 const int64_t stride = C * cap;
                 const double* x = qp + c * cap + j;
+                const int rb0 = g * nb, rb1 = act ? min(X.nrb3, rb0 + nb) : rb0;
                 double s = 0.0;
-                int rb = 0;
-                for (; rb + kB <= X.nrb3; rb += kB) {
+                int rb = rb0;
+                for (; rb + kB <= rb1; rb += kB) {
                     double v[kB];
 #pragma unroll
                     for (int b = 0; b < kB; ++b) v[b] = __ldcg(x + int64_t(rb + b) * stride);
 #pragma unroll
                     for (int b = 0; b < kB; ++b) s += v[b];
                 }
-                for (; rb < X.nrb3; ++rb) s += __ldcg(x + int64_t(rb) * stride);
-                const float qv = float(s);
-                Q[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = qv;
-                qd[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = s;
-                if (kMean) mean = __fadd_rn(mean, qv);
+                for (; rb < rb1; ++rb) s += __ldcg(x + int64_t(rb) * stride);
+                if (G == 4) {  // the group's quarters, in order, into its first lane
+                    const double s1 = __shfl_down_sync(kFull, s, 1);
+                    const double s2 = __shfl_down_sync(kFull, s, 2);
+                    const double s3 = __shfl_down_sync(kFull, s, 3);
+                    s = ((s + s1) + s2) + s3;
+                }
+                if (act && g == 0) {
+                    const float qv = float(s);
+                    Q[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = qv;
+                    qd[int64_t(ww) * Q_pw + L.q_off + c * cap + j] = s;
+                    if (kMean) mean = __fadd_rn(mean, qv);
+                }
             }
-            if (kMean) qmean[L.q_off + c * cap + j] = __fmul_rn(mean, inv_w);
+            if (kMean && act && g == 0) qmean[L.q_off + c * cap + j] = __fmul_rn(mean, inv_w);
         }
     }
 }
@@ -929,8 +963,8 @@ __global__ void __launch_bounds__(256) ps_qmean_kernel(
         const int r = ps_rank(L, k_or_rank, d.x);
         if (r == 0) continue;
         const int cap = L.cap;
-        const int64_t c0 = int64_t(d.y) * kPsQB;
-        const int cw = int(min64(kPsQB, L.cols - c0));
+        const int64_t c0 = d.y;
+        const int cw = d.z;
         for (int i = threadIdx.x; i < cw * r; i += blockDim.x) {
             const int64_t o = L.q_off + (c0 + i / r) * cap + i % r;
             float sum = 0.0f;
