@@ -453,7 +453,7 @@ def run_workload(name, args, world, rank, dev, primary):
     graphable = not (method == "randk" or kr is not None or apply)
     if args.graph and primary and not graphable:
         raise SystemExit("--graph: this workload's step takes per-step host values")
-    if primary and graphable and not args.eager and args.graph is not False:
+    if args.graph and primary:
         graphs = []
         for b in range(2):
             gr = torch.cuda.CUDAGraph()
@@ -622,12 +622,9 @@ def main():
     ap.add_argument("--oracle-timing", action="store_true",
                     help="time the CPU oracle on one step of every workload at 1 thread and "
                          "on all cores, print one JSON line, and exit")
-    ap.add_argument("--graph", action="store_true", default=None,
+    ap.add_argument("--graph", action="store_true",
                     help="replay each step as a CUDA graph (workloads whose step takes no "
-                         "per-step host values: top-k, sign, PowerSGD without Accordion); "
-                         "the default for the primary workload when it allows it")
-    ap.add_argument("--eager", action="store_true",
-                    help="launch every kernel of every step from the host (no graph)")
+                         "per-step host values: top-k, sign, PowerSGD without Accordion)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -681,7 +678,6 @@ def main():
         import copy
         sargs = copy.copy(args)
         sargs.steps, sargs.warmup, sargs.graph, sargs.profile = min(args.steps, 30), 3, False, False
-        sargs.eager = True
         secondary = []
         for name in SECONDARY:
             x = run_workload(name, sargs, world, rank, dev, primary=False)
