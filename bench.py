@@ -50,6 +50,8 @@ def workload_spec(name):
         return dict(layers=wl.bert_base_topk(), W=8, cfg=4, method="topk", apply=True)
     if name == "bert_base_sign_w8":              # signSGD with memory, 1 bit per element
         return dict(layers=wl.bert_base_topk(kind="sign"), W=8, cfg=4, method="sign")
+    if name == "bert_base_sign_w1":              # one replica: a profiling-sized case
+        return dict(layers=wl.bert_base_topk(kind="sign"), W=1, cfg=4, method="sign")
     if name == "bert_base_topk1pct_w1":          # one replica: a profiling-sized case
         return dict(layers=wl.bert_base_topk(), W=1, cfg=4, method="topk")
     if name == "bert_base_randk1pct_w8":

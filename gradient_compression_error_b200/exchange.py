@@ -23,7 +23,15 @@ same k tensor.
 
 Payload kinds: top-k, rand-k, signSGD and dense layers.  rand-k's generator
 takes the worker index, so rank r encodes as job-wide worker r
-(ef_randk_step_at).
+(ef_randk_step_at).  With shared keys every rank encodes as worker 0: all
+ranks choose the same coordinates, only the values cross (half the bytes),
+and the sum is the W-replica decode of rows that share one index row -- the
+all-reduce-compatible form of rand-k.
+
+GroupedDataParallelStep cuts the table into groups of consecutive layers and
+starts each group's gather as soon as the group is encoded, so the exchange
+of one group overlaps the encoding of the next (NCCL runs the collective on
+its own stream after the work already queued on the caller's).
 
 PowerSGD's data-parallel form sums P and Q over the workers between its
 contractions (On the Utility of Gradient Compression, Key results: PowerSGD is
@@ -40,10 +48,12 @@ import torch.distributed as dist
 METHODS = ("topk", "randk", "sign")
 
 
-def gather_rows(out, row, group=None):
+def gather_rows(out, row, group=None, async_op=False):
     """Row r of ``out`` [world, n] <- rank r's ``row`` (n elements of out's
     dtype and device), on every rank; every rank must call it, in the same
-    order.  NCCL gathers into the buffer; gloo into a list of its row views."""
+    order.  NCCL gathers into the buffer; gloo into a list of its row views.
+    async_op: return the collective's work handle (wait() before reading out)
+    instead of out."""
     if row is None or row.numel() != out.shape[1] or row.dtype != out.dtype \
             or row.device != out.device:
         raise ValueError("row must be %d %s elements on %s" % (out.shape[1], out.dtype,
@@ -52,10 +62,10 @@ def gather_rows(out, row, group=None):
     if not row.is_contiguous():
         raise ValueError("row must be contiguous")
     if dist.get_backend(group) == "nccl":
-        dist.all_gather_into_tensor(out, row, group=group)
+        work = dist.all_gather_into_tensor(out, row, group=group, async_op=async_op)
     else:
-        dist.all_gather(list(out.unbind(0)), row, group=group)
-    return out
+        work = dist.all_gather(list(out.unbind(0)), row, group=group, async_op=async_op)
+    return work if async_op else out
 
 
 class PayloadExchange:
@@ -75,29 +85,35 @@ class PayloadExchange:
         self.idx = (torch.zeros((self.world, self.n), dtype=torch.int32, device=device)
                     if with_idx else None)
 
-    def _gather(self, out, row):
-        gather_rows(out, row, self.group)
-
-    def gather(self, vals_row, idx_row=None):
-        """All ranks' rows, in rank order: (vals, idx); idx is None without indices."""
-        self._gather(self.vals, vals_row)
+    def gather(self, vals_row, idx_row=None, async_op=False, values_only=False):
+        """All ranks' rows, in rank order: (vals, idx); idx is None without
+        indices.  values_only: idx_row is the same on every rank and is copied
+        into every row locally instead of gathered.  async_op: start the
+        collectives and return their work handles (wait() each before reading
+        vals / idx)."""
+        works = [gather_rows(self.vals, vals_row, self.group, async_op)]
         if self.idx is not None:
-            self._gather(self.idx, idx_row)
-        return self.vals, self.idx
+            if values_only:
+                self.idx.copy_(idx_row.reshape(1, -1).expand_as(self.idx))
+            else:
+                works.append(gather_rows(self.idx, idx_row, self.group, async_op))
+        return works if async_op else (self.vals, self.idx)
 
 
 class DataParallelStep:
     """One data-parallel step over the ranks of ``group``, one worker per rank.
 
     ``encode`` runs this rank's one-worker step (ef_topk_step, ef_randk_step_at
-    as worker ``rank`` or ef_sign_step; W = 1) on grad / mem [1, N];
-    ``exchange`` gathers every rank's payload;
+    as worker ``rank`` -- worker 0 with ``shared_keys`` -- or ef_sign_step;
+    W = 1) on grad / mem [1, N];
+    ``exchange`` gathers every rank's payload (the values alone with
+    ``shared_keys``: every rank chose the same indices);
     ``decode`` writes the aggregate of the gathered payloads.  ``__call__``
     runs the three in order.  The native calls run on the current CUDA stream,
     and torch.distributed orders its collectives after that stream's work.
     """
 
-    def __init__(self, table, method, group=None, device="cuda"):
+    def __init__(self, table, method, group=None, device="cuda", shared_keys=False):
         import gradient_compression_error_b200 as g
         if method not in METHODS:
             raise ValueError("method must be one of %s (PowerSGD: PowerSgdDataParallelStep)"
@@ -106,9 +122,12 @@ class DataParallelStep:
         if ck not in (-1, g.KIND[method]):
             raise ValueError("table of kind %s cannot take a %s step"
                              % (g.KIND_NAME.get(ck), method))
+        if shared_keys and method != "randk":
+            raise ValueError("shared keys are a rand-k mode")
         self.g = g
         self.table = table
         self.method = method
+        self.shared_keys = bool(shared_keys)
         sparse = method in ("topk", "randk")
         self.ex = PayloadExchange(table.vals_per_worker, sparse, device, group)
         self.world = self.ex.world
@@ -126,13 +145,15 @@ class DataParallelStep:
             g.ef_topk_step(self.table, 1, grad, mem, eta, k, self.vals_row, self.idx_row,
                            self.ws_step)
         elif self.method == "randk":
-            g.ef_randk_step_at(self.table, self.ex.rank, 1, grad, mem, eta, k, seed, step,
+            worker = 0 if self.shared_keys else self.ex.rank
+            g.ef_randk_step_at(self.table, worker, 1, grad, mem, eta, k, seed, step,
                                self.vals_row, self.idx_row, self.ws_step)
         else:
             g.ef_sign_step(self.table, 1, grad, mem, eta, self.vals_row, self.ws_step)
 
-    def exchange(self):
-        return self.ex.gather(self.vals_row, self.idx_row)
+    def exchange(self, async_op=False):
+        return self.ex.gather(self.vals_row, self.idx_row, async_op=async_op,
+                              values_only=self.shared_keys)
 
     def decode(self, out, scale, k=None, apply=False, vote=False):
         """out = scale * (rank-order sum of the payloads); with ``apply``,
@@ -157,6 +178,61 @@ class DataParallelStep:
         self.encode(grad, mem, eta, k, seed, step)
         self.exchange()
         self.decode(out, 1.0 / self.world if scale is None else scale, k, apply, vote)
+        return out
+
+
+class GroupedDataParallelStep:
+    """DataParallelStep over groups of consecutive layers, with each group's
+    exchange started as soon as the group is encoded: the gather of group g
+    runs while group g + 1 encodes, and every group is decoded once all
+    gathers have landed.  Results are those of the ungrouped step bit for bit
+    (each (worker, layer) unit is encoded alone and decoded in worker order).
+
+    ``layers``: the layer descriptors of the whole table (as for Table);
+    ``cuts``: the indices of the layers that start a new group (ascending,
+    each group starting at a multiple of 4 elements, the 16-byte alignment
+    the kernels need).  top-k and signSGD (rand-k's keys depend on a layer's
+    index within its table).
+    """
+
+    def __init__(self, layers, method, cuts, group=None, device="cuda"):
+        import gradient_compression_error_b200 as g
+        if method not in ("topk", "sign"):
+            raise ValueError("grouped exchange: top-k or signSGD")
+        bounds = [0] + [int(c) for c in cuts] + [len(layers)]
+        if any(b1 <= b0 for b0, b1 in zip(bounds, bounds[1:])):
+            raise ValueError("cuts must be ascending layer indices inside the table")
+        self.g = g
+        self.parts = []
+        off = 0
+        for b0, b1 in zip(bounds, bounds[1:]):
+            if off % 4:
+                raise ValueError("group at layer %d starts at element %d, not a multiple of 4"
+                                 % (b0, off))
+            t = g.Table(layers[b0:b1])
+            self.parts.append(dict(lo=b0, hi=b1, off=off, n=t.N,
+                                   step=DataParallelStep(t, method, group, device)))
+            off += t.N
+        self.N = off
+        self.world = self.parts[0]["step"].world
+
+    def __call__(self, grad, mem, eta, out, scale=None, k=None, apply=False, vote=False):
+        """One step on this rank's grad / mem [1, N]; out [N] as in
+        DataParallelStep; k: per-layer k for the whole table (or None)."""
+        if grad.shape[-1] != self.N or mem.shape[-1] != self.N or out.numel() != self.N:
+            raise ValueError("grad, mem and out must hold the table's %d elements" % self.N)
+        scale = 1.0 / self.world if scale is None else scale
+        works = []
+        for p in self.parts:
+            sl = slice(p["off"], p["off"] + p["n"])
+            kp = None if k is None else k[p["lo"]:p["hi"]]
+            p["step"].encode(grad[:, sl], mem[:, sl], eta, kp)
+            works.append(p["step"].exchange(async_op=True))
+        for p, ws in zip(self.parts, works):
+            for w in ws:
+                w.wait()
+            kp = None if k is None else k[p["lo"]:p["hi"]]
+            p["step"].decode(out[p["off"]:p["off"] + p["n"]], scale, kp, apply, vote)
         return out
 
 

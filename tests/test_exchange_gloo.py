@@ -170,6 +170,75 @@ def test_one_worker_per_rank_gathers_the_w_worker_step(method, world, port):
         assert all(r.values()), (rank, r)
 
 
+# ---- rand-k with shared keys: the values alone cross --------------------------------------
+def _shared_rank(rank, world, port, q):
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    from gradient_compression_error_b200.exchange import PayloadExchange
+    from oracle import steps as osteps
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        layers = LAYERS["randk"]
+        k = [l["cap"] for l in layers]
+        grad, mem = _inputs(layers, world)
+
+        def as_worker0(w):
+            """Worker w's payload with worker 0's keys (its data as a one-worker step)."""
+            mw = mem[w:w + 1].copy()
+            p = osteps.sparse_step(layers, grad[w:w + 1], mw, ETA, k, method="randk", seed=SEED,
+                                   step=STEP)
+            return {l: p[(0, l)] for l in range(len(layers))}, mw[0]
+        mine, _ = as_worker0(rank)
+        v, i = _pack(layers, {(rank, l): x for l, x in mine.items()}, rank)
+        ex = PayloadExchange(len(v), True, "cpu")
+        works = ex.gather(torch.from_numpy(v), torch.from_numpy(i), async_op=True,
+                          values_only=True)
+        for w in works:
+            w.wait()
+        gathered = {}
+        for w in range(world):
+            _unpack(layers, ex.vals[w].numpy(), ex.idx[w].numpy(), w, gathered)
+        ref = {}
+        for w in range(world):
+            p, _ = as_worker0(w)
+            ref.update({(w, l): x for l, x in p.items()})
+        sparse = [l for l, lay in enumerate(layers) if lay["kind"] == "randk"]
+        same_coords = all(np.array_equal(ref[(w, l)][1], ref[(0, l)][1])
+                          for w in range(world) for l in sparse)
+        same_payload = all(_same_bits(gathered[u], ref[u]) for u in ref)
+        scale = np.float32(1.0 / world)
+        same_sum = np.array_equal(osteps.decompress(layers, world, gathered, scale).view(np.uint32),
+                                  osteps.decompress(layers, world, ref, scale).view(np.uint32))
+        dist.barrier()
+        q.put((rank, dict(same_coords=same_coords, same_payload=same_payload,
+                          same_sum=same_sum, one_collective=len(works) == 1)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_randk_shared_keys_gathers_values_alone():
+    """rand-k with every rank keyed as worker 0: all ranks choose the same
+    coordinates, so only the values are gathered (one collective, started
+    asynchronously) and every row's indices are filled locally; the payloads
+    and their worker-order sum are the one-process ones bit for bit."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    world = 3
+    procs = [ctx.Process(target=_shared_rank, args=(r, world, 29526, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert sorted(out) == list(range(world))
+    for rank, r in out.items():
+        assert all(r.values()), (rank, r)
+
+
 # ---- PowerSGD and Accordion between ranks -------------------------------------------------
 # The data-parallel PowerSGD step cut at its two sums, with the oracle's
 # phases on each rank and gather_rows moving the rows: each rank sums the

@@ -303,3 +303,112 @@ def test_one_rank_nccl_powersgd_and_accordion_between_ranks():
     p.join(timeout=60)
     assert p.exitcode == 0
     assert res.get("completed") and all(res.values()), res
+
+
+# ---- grouped exchange and rand-k with shared keys ------------------------------------------
+GROUP_LAYERS = {
+    "topk": [dict(rows=300, cols=40, kind="topk", cap=120, sigma=1.0),
+             dict(rows=76, cols=1, kind="dense", cap=0, sigma=1.0),
+             dict(rows=70000, cols=1, kind="topk", cap=700, sigma=0.5),
+             dict(rows=64, cols=64, kind="topk", cap=41, sigma=2.0),
+             dict(rows=5, cols=3, kind="dense", cap=0, sigma=1.0)],
+    "sign": [dict(rows=40, cols=100, kind="sign", cap=0, sigma=1.0),
+             dict(rows=76, cols=1, kind="dense", cap=0, sigma=1.0),
+             dict(rows=9000, cols=1, kind="sign", cap=0, sigma=2.0),
+             dict(rows=33, cols=1, kind="sign", cap=0, sigma=1.0)],
+}
+
+
+def _group_rank(port, q):
+    sys.path.insert(0, ROOT)
+    import torch
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda:0"),
+                            timeout=datetime.timedelta(seconds=60))
+    res = {}
+    try:
+        from tests.helpers import gce
+        g = gce()
+        from gradient_compression_error_b200 import workloads
+        from gradient_compression_error_b200.exchange import (DataParallelStep,
+                                                              GroupedDataParallelStep)
+        for method, layers in GROUP_LAYERS.items():
+            descs = workloads.table_layers(layers)
+            t = g.Table(descs)
+            whole = DataParallelStep(t, method)
+            grouped = GroupedDataParallelStep(descs, method, cuts=[2, 3])
+            mem_a = (0.1 * workloads.gradients(layers, 1, 951, 0)).contiguous()
+            mem_b = mem_a.clone()
+            out_a = torch.zeros(t.N, device="cuda")
+            out_b = torch.full((t.N,), 3.0, device="cuda")
+            k = None
+            if method == "topk":
+                k = torch.tensor([60, 0, 700, 20, 0], dtype=torch.int32, device="cuda")
+            for s in range(2):
+                grad = workloads.gradients(layers, 1, 950, s)
+                whole(grad, mem_a, ETA, out_a, k=k)
+                grouped(grad, mem_b, ETA, out_b, k=k)
+                torch.cuda.synchronize()
+                res["%s_out%d" % (method, s)] = torch.equal(out_a.view(torch.int32),
+                                                            out_b.view(torch.int32))
+                res["%s_mem%d" % (method, s)] = torch.equal(mem_a.view(torch.int32),
+                                                            mem_b.view(torch.int32))
+            try:   # a group must start at a multiple of 4 elements (here at element 7)
+                odd = [dict(rows=7, cols=1, kind=method, cap=2 if method == "topk" else 0),
+                       dict(rows=100, cols=1, kind=method, cap=5 if method == "topk" else 0)]
+                GroupedDataParallelStep(workloads.table_layers(odd), method, cuts=[1])
+                res["%s_misaligned_refused" % method] = False
+            except ValueError:
+                res["%s_misaligned_refused" % method] = True
+            t.close()
+        # rand-k with shared keys: worker 0's keys on every rank, values
+        # alone gathered; the same as the native one-worker step as worker 0
+        layers = LAYERS["randk"]
+        t = g.Table(workloads.table_layers(layers))
+        shared = DataParallelStep(t, "randk", shared_keys=True)
+        mem_a = (0.1 * workloads.gradients(layers, 1, 953, 0)).contiguous()
+        mem_b = mem_a.clone()
+        vals = torch.zeros((1, max(4, t.vals_per_worker)), device="cuda")
+        idx = torch.zeros((1, max(4, t.vals_per_worker)), dtype=torch.int32, device="cuda")
+        ws, wsd = t.workspace(1, "randk"), t.workspace(1, "decompress")
+        out_a = torch.zeros(t.N, device="cuda")
+        out_b = torch.zeros(t.N, device="cuda")
+        for s in range(2):
+            grad = workloads.gradients(layers, 1, 952, s)
+            shared(grad, mem_a, ETA, out_a, seed=SEED, step=s)
+            g.ef_randk_step_at(t, 0, 1, grad, mem_b, ETA, None, SEED, s, vals, idx, ws)
+            g.decompress_accumulate(t, 1, vals, idx, None, None, None, 1.0, out_b, wsd)
+            torch.cuda.synchronize()
+            res["shared_out%d" % s] = torch.equal(out_a.view(torch.int32), out_b.view(torch.int32))
+            res["shared_mem%d" % s] = torch.equal(mem_a.view(torch.int32), mem_b.view(torch.int32))
+        try:
+            DataParallelStep(g.Table(workloads.table_layers(GROUP_LAYERS["topk"])), "topk",
+                             shared_keys=True)
+            res["shared_keys_topk_refused"] = False
+        except ValueError:
+            res["shared_keys_topk_refused"] = True
+        t.close()
+        res["completed"] = True
+    finally:
+        dist.destroy_process_group()
+        q.put(res)
+
+
+def test_one_rank_nccl_grouped_exchange_and_shared_randk_keys():
+    """GroupedDataParallelStep (each layer group's gather started right after
+    the group is encoded) gives the ungrouped step's aggregate and memory bit
+    for bit, for top-k with per-layer k (one layer skipped) and for signSGD;
+    misaligned groups are refused.  rand-k with shared keys equals the native
+    step as worker 0 plus the decode ("On the Utility of Gradient
+    Compression", Method: all-reduce-compatible exchange)."""
+    need_gpu()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    p = ctx.Process(target=_group_rank, args=(29538, q))
+    p.start()
+    res = q.get(timeout=300)
+    p.join(timeout=60)
+    assert p.exitcode == 0
+    assert res.get("completed") and all(res.values()), res
