@@ -42,6 +42,20 @@ struct alignas(16) TileInfo {
     int32_t tstart;   // first element of the tile within its layer
 };
 
+// One TOPK / RANDK decode tile's fields, stored in the order the sparse decoder
+// takes the tiles: its per-span work starts from one 48-byte record instead of
+// tile -> layer id -> layer record.
+struct alignas(16) DcTileInfo {
+    int64_t out_off;  // first output of the tile (layer offset + tstart)
+    int64_t val_off;  // the layer's first payload slot
+    int32_t tstart;   // first element of the tile within its layer
+    int32_t cnt;      // outputs in the tile: kDcTile, or fewer at the layer's end
+    int32_t bslot;    // span-bound slot of the tile's first span
+    int32_t layer;    // layer id, for a per-layer k
+    int32_t cap;      // the layer's cap on k
+    int32_t pad[3];
+};
+
 // A pipelined signSGD schedule uploaded for one (W, ahead): nphase runs
 // (the last a sentinel) covering nitems work items.
 struct SgPlan {
@@ -79,6 +93,10 @@ struct gce_table {
     int32_t* d_dc_tile_layer = nullptr;    // [dc_tiles] layer of each decode tile
     int32_t dc_nl_n = 0;                   // decode tiles of sparse and DENSE layers
     int32_t* d_dc_nl_tiles = nullptr;      // their decode tile ids
+    int32_t dc_sp_n = 0;                   // decode tiles of TOPK and RANDK layers
+    gce::DcTileInfo* d_dc_sp_info = nullptr;  // their fields, in decode order
+    int32_t dc_dn_n = 0;                   // decode tiles of DENSE layers
+    int32_t* d_dc_dn_tiles = nullptr;      // their decode tile ids
     int32_t bunits_pw = 0;                 // decode bound units (sparse layers) per worker
     int32_t* d_bunit_layer = nullptr;
     int32_t* d_bunit_chunk = nullptr;

@@ -85,13 +85,17 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
     }
 }
 
-// The entries of every worker that fall in this warp's span (outputs [lo, lo +
-// kDcSpan) of the tile that starts at index `start`) added to the accumulator in
-// worker order.  Lane w < W holds worker w's entry range [a, a + c) of the span
-// (from the span bounds); the warp walks the W ranges one after the other, 32
-// entries a round, loading each entry's index and value into a lane, and adds a
-// round's entries worker by worker (within one worker the indices are
-// distinct, so its lanes add without conflict).  Run by a full warp; W <= 32.
+// The entries of every worker that fall in this warp's span (outputs [start,
+// start + kDcSpan) of a layer) added to the span's accumulator in worker order.
+// Lane w < W holds worker w's entry range [a, a + c) of the span (from the span
+// bounds); the warp walks the W ranges one after the other, 32 entries a round,
+// each entry's index and value loaded into a lane.  The loads of kDcRounds
+// rounds are issued before any of their adds (a round's lanes and addresses
+// follow from the bounds alone), then each round adds its entries worker by
+// worker (within one worker the indices are distinct, so its lanes add without
+// conflict).  Run by a full warp; W <= 32.
+constexpr int kDcRounds = 3;
+
 __device__ __forceinline__ void dc_add_span(float* acc, int64_t start, int W, int32_t a,
                                             int32_t c, const float* __restrict__ vals,
                                             const int32_t* __restrict__ idx, int64_t vals_pw,
@@ -100,46 +104,57 @@ __device__ __forceinline__ void dc_add_span(float* acc, int64_t start, int W, in
     const int32_t incl = warp_inclusive_scan(c);
     const int32_t excl = incl - c;
     const int32_t total = __shfl_sync(kFull, incl, 31);
-    for (int32_t q0 = 0; q0 < total; q0 += 32) {
-        const int32_t q = q0 + lane;
-        // the worker of entry q: the last w < W whose range starts at or before q
-        int w = 0;
+    for (int32_t q0 = 0; q0 < total; q0 += 32 * kDcRounds) {
+        int w[kDcRounds];
+        int32_t i[kDcRounds];
+        float v[kDcRounds];
 #pragma unroll
-        for (int step = 16; step > 0; step >>= 1) {
-            const int32_t e = __shfl_sync(kFull, excl, min(w + step, 31));
-            if (w + step < W && e <= q) w += step;
+        for (int r = 0; r < kDcRounds; ++r) {
+            w[r] = 0;
+            i[r] = 0;
+            v[r] = 0.0f;
+            if (q0 + 32 * r < total) {  // the same for the whole warp
+                const int32_t q = q0 + 32 * r + lane;
+                int ww = 0;
+#pragma unroll
+                for (int step = 16; step > 0; step >>= 1) {
+                    const int32_t e = __shfl_sync(kFull, excl, min(ww + step, 31));
+                    if (ww + step < W && e <= q) ww += step;
+                }
+                const int32_t aw = __shfl_sync(kFull, a, ww), ew = __shfl_sync(kFull, excl, ww);
+                w[r] = ww;
+                if (q < total) {
+                    const int64_t o = int64_t(ww) * vals_pw + val_off + aw + (q - ew);
+                    i[r] = int32_t(int64_t(__ldcg(idx + o)) - start);
+                    v[r] = __ldcg(vals + o);
+                }
+            }
         }
-        const int32_t aw = __shfl_sync(kFull, a, w), ew = __shfl_sync(kFull, excl, w);
-        const bool have = q < total;
-        int32_t i = 0;
-        float v = 0.0f;
-        if (have) {
-            const int64_t o = int64_t(w) * vals_pw + val_off + aw + (q - ew);
-            i = int32_t(int64_t(__ldcg(idx + o)) - start);
-            v = __ldcg(vals + o);
-        }
-        unsigned pending = __ballot_sync(kFull, have);
-        while (pending) {
-            const int wl = __shfl_sync(kFull, w, __ffs(pending) - 1);
-            const bool mine = have && w == wl;
-            if (mine) acc[i] = __fadd_rn(acc[i], v);
-            __syncwarp();
-            pending &= ~__ballot_sync(kFull, mine);
+#pragma unroll
+        for (int r = 0; r < kDcRounds; ++r) {
+            const bool have = q0 + 32 * r + lane < total;
+            unsigned pending = __ballot_sync(kFull, have);
+            while (pending) {
+                const int wl = __shfl_sync(kFull, w[r], __ffs(pending) - 1);
+                const bool mine = have && w[r] == wl;
+                if (mine) acc[i[r]] = __fadd_rn(acc[i[r]], v[r]);
+                __syncwarp();
+                pending &= ~__ballot_sync(kFull, mine);
+            }
         }
     }
 }
 
-// Write this warp's kDcSpan outputs and zero them in the accumulator for the
-// next tile: out = fl(scale * sum), or with kApply x = fl(x - fl(scale * sum)).
+// Write a span's `cnt` outputs from the warp's accumulator and zero it for the
+// next span: out = fl(scale * sum), or with kApply x = fl(x - fl(scale * sum)).
 // Run by a full warp after __syncwarp.
 template <bool kApply>
-__device__ __forceinline__ void dc_write_quarter(float* acc, float* o, int cnt, int warp,
-                                                 float scale, bool aligned) {
+__device__ __forceinline__ void dc_write_span(float* acc, float* o, int cnt, float scale,
+                                              bool aligned) {
     const int lane = threadIdx.x & 31;
-    const int lo = warp * kDcSpan;
-    if (aligned && lo + kDcSpan <= cnt) {
-        float4* a4 = reinterpret_cast<float4*>(acc + lo);
-        float4* o4 = reinterpret_cast<float4*>(o + lo);
+    if (aligned && cnt == kDcSpan) {
+        float4* a4 = reinterpret_cast<float4*>(acc);
+        float4* o4 = reinterpret_cast<float4*>(o);
 #pragma unroll
         for (int j = 0; j < kDcSpan / 4 / 32; ++j) {
             const float4 x = a4[lane + 32 * j];
@@ -147,12 +162,59 @@ __device__ __forceinline__ void dc_write_quarter(float* acc, float* o, int cnt, 
             a4[lane + 32 * j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
     } else {
-        for (int i = lo + lane; i < lo + kDcSpan; i += 32) {
+        for (int i = lane; i < kDcSpan; i += 32) {
             if (i < cnt) o[i] = dc_final<kApply>(acc[i], scale, o + i);
             acc[i] = 0.0f;
         }
     }
     __syncwarp();
+}
+
+// TOPK and RANDK tiles for W <= 32 workers.  Each warp owns one 1024-output span
+// at a time (four spans to a decode tile) with its own accumulator in shared
+// memory: it reads the span's entry bounds of every worker, adds the entries in
+// worker order and writes the span out.  No warp waits for another; the next
+// span's tile record is loaded while the current span is added, so a span's
+// chain of dependent loads is its bounds and then its entries.
+template <bool kApply>
+__global__ void __launch_bounds__(kDcThreads, kApply ? 9 : 10) dc_sparse_kernel(
+    const DcTileInfo* __restrict__ tiles, int32_t ntiles, int32_t W, int64_t vals_pw,
+    int32_t dc_slots, const int32_t* __restrict__ k_or_rank, const float* __restrict__ vals,
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ bounds, float scale,
+    float* __restrict__ out) {
+    grid_dependency_sync();
+    constexpr int kParts = kDcTile >> kDcSpanLog;  // spans per tile, one per warp of a block
+    __shared__ __align__(16) float acc_all[kDcTile];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    float* acc = acc_all + warp * kDcSpan;
+    for (int i = lane; i < kDcSpan / 4; i += 32)
+        reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    __syncwarp();
+    const int64_t nspans = int64_t(ntiles) * kParts;
+    const int64_t qstep = int64_t(gridDim.x) * kParts;
+    int64_t q = int64_t(blockIdx.x) * kParts + warp;
+    DcTileInfo nx{};
+    if (q < nspans) nx = tiles[q / kParts];
+    for (; q < nspans; q += qstep) {
+        const DcTileInfo T = nx;
+        if (q + qstep < nspans) nx = tiles[(q + qstep) / kParts];  // the next span's record
+        const int p = int(q % kParts);
+        const int cnt = min(kDcSpan, T.cnt - p * kDcSpan);
+        if (cnt <= 0) continue;
+        int32_t k = k_or_rank ? k_or_rank[T.layer] : T.cap;
+        k = (k >= 1 && k <= T.cap) ? k : 0;  // out of range: the layer contributes nothing
+        int32_t a = 0, c = 0;
+        if (lane < W) {
+            const int32_t* b = bounds + int64_t(lane) * dc_slots + T.bslot + p;
+            a = min(max(b[0], 0), k);
+            c = min(max(b[1], a), k) - a;
+        }
+        const int64_t span0 = int64_t(T.tstart) + p * kDcSpan;
+        dc_add_span(acc, span0, W, a, c, vals, idx, vals_pw, T.val_off);
+        __syncwarp();
+        const int64_t o = T.out_off + p * kDcSpan;
+        dc_write_span<kApply>(acc, out + o, cnt, scale, (o & 3) == 0);
+    }
 }
 
 template <bool kApply>
@@ -165,9 +227,7 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
     float* __restrict__ out) {
     grid_dependency_sync();
     __shared__ __align__(16) float acc[kDcTile];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // the accumulator is all zero between sparse tiles: each warp zeroes the
-    // part it writes out
+    // the accumulator is all zero between sparse tiles
     for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
         reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
@@ -181,28 +241,8 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
         float* o = out + L.offset + start;
         if (L.kind == GCE_KIND_TOPK || L.kind == GCE_KIND_RANDK) {
             const int32_t k = layer_k(L, k_or_rank, l);
-            if (W <= 32) {
-                // Warp `warp` owns span 4 tt + warp of the layer (tile outputs
-                // [warp, warp + 1) x kDcSpan): it reads its own entry bounds,
-                // adds its entries in worker order and writes the span out; the
-                // warps of the block never wait for one another here.
-                const int lo = warp * kDcSpan;
-                if (lo < cnt) {
-                    int32_t a = 0, c = 0;
-                    if (lane < W) {
-                        const int32_t* b = bounds + int64_t(lane) * dc_slots + L.dc_base +
-                                           (tt << (kDcTileLog - kDcSpanLog)) + warp;
-                        a = min(max(b[0], 0), k);
-                        c = min(max(b[1], a), k) - a;
-                    }
-                    dc_add_span(acc, start, W, a, c, vals, idx, vals_pw, L.val_off);
-                    __syncwarp();
-                    dc_write_quarter<kApply>(acc, o, cnt, warp, scale,
-                                             ((L.offset + start) & 3) == 0);
-                }
-                continue;
-            }
-            // more than 32 workers: one worker at a time, straight from memory
+            // more than 32 workers (dc_sparse_kernel takes the rest): one worker
+            // at a time, straight from memory
             for (int w = 0; w < W; ++w) {
                 __syncthreads();
                 const int32_t* b = bounds + int64_t(w) * dc_slots + L.dc_base;
@@ -221,7 +261,7 @@ __global__ void __launch_bounds__(kDcThreads, 9) dc_accum_kernel(
             for (int i = threadIdx.x; i < cnt; i += blockDim.x)
                 o[i] = dc_final<kApply>(acc[i], scale, o + i);
             __syncthreads();
-            // leave the accumulator at zero for the next tile's staged path
+            // leave the accumulator at zero for the next sparse tile
             for (int i = threadIdx.x; i < kDcTile / 4; i += blockDim.x)
                 reinterpret_cast<float4*>(acc)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             __syncthreads();
@@ -385,6 +425,22 @@ static int launch_decode_t(const gce_table* t, int32_t W, const float* vals, con
         GCE_LAUNCH(dc_bounds_kernel, wave_grid(units, 8, r_bounds), 256, 0, st, t->d_layers,
                    t->d_bunit_layer, t->d_bunit_chunk, t->bunits_pw, W, t->vals_pw, t->dc_slots,
                    k_or_rank, idx, bounds);
+    }
+    if (sparse && W <= 32) {
+        // sparse tiles by the warp-per-span kernel, DENSE tiles by the general one
+        static const int r_sparse = resident_blocks(dc_sparse_kernel<kApply>, kDcThreads);
+        if (t->dc_sp_n > 0)
+            GCE_LAUNCH_AS(kApply ? "dc_sparse_kernel<true>" : "dc_sparse_kernel<false>",
+                          dc_sparse_kernel<kApply>, wave_grid(t->dc_sp_n, 16, r_sparse),
+                          kDcThreads, 0, st, t->d_dc_sp_info, t->dc_sp_n, W, t->vals_pw,
+                          t->dc_slots, k_or_rank, vals, idx, bounds, scale, out);
+        if (t->dc_dn_n > 0)
+            GCE_LAUNCH_AS(kApply ? "dc_accum_kernel<true>" : "dc_accum_kernel<false>",
+                          dc_accum_kernel<kApply>, wave_grid(t->dc_dn_n, 16, r_accum),
+                          kDcThreads, 0, st, t->d_layers, t->d_dc_tile_layer, t->d_dc_dn_tiles,
+                          t->dc_dn_n, W, t->vals_pw, t->P_pw, t->Q_pw, t->dc_slots, k_or_rank,
+                          vals, idx, P, Q, bounds, scale, out);
+        return check_launch();
     }
     // PowerSGD layers by their own tiled kernel when it takes them (then the
     // element-wise kernel covers only the other layers' tiles)

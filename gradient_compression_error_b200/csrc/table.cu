@@ -174,6 +174,8 @@ static void free_table(gce_table* t) {
     cudaFree(t->d_dtile_start);
     cudaFree(t->d_dc_tile_layer);
     cudaFree(t->d_dc_nl_tiles);
+    cudaFree(t->d_dc_sp_info);
+    cudaFree(t->d_dc_dn_tiles);
     cudaFree(t->d_bunit_layer);
     cudaFree(t->d_bunit_chunk);
     powersgd_plan_free(t);
@@ -201,7 +203,8 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     int32_t tiles = 0;
     std::vector<int32_t> tile_layer, sunit_layer, sunit_part, dtile_layer, dtile_start;
     std::vector<TileInfo> tile_info;
-    std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_nl;
+    std::vector<int32_t> dc_tile_layer, bunit_layer, bunit_chunk, dc_nl, dc_dn;
+    std::vector<DcTileInfo> dc_sp;
     int32_t dc_tiles = 0, dc_slots = 0;
     for (int32_t l = 0; l < L; ++l) {
         const gce_layer_desc& d = descs[l];
@@ -276,6 +279,18 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
         x.dc_base = dc_slots;
         for (int32_t i = 0; i < x.dc_ntiles; ++i) {
             if (d.kind != GCE_KIND_POWERSGD) dc_nl.push_back(dc_tiles + i);
+            if (d.kind == GCE_KIND_TOPK || d.kind == GCE_KIND_RANDK) {
+                DcTileInfo r{};
+                r.tstart = int32_t(int64_t(i) * kDcTile);
+                r.out_off = x.offset + r.tstart;
+                r.val_off = x.val_off;
+                r.cnt = int32_t(std::min<int64_t>(kDcTile, n - r.tstart));
+                r.bslot = dc_slots + int32_t((int64_t(i) * kDcTile) >> kDcSpanLog);
+                r.layer = l;
+                r.cap = d.cap;
+                dc_sp.push_back(r);
+            }
+            if (d.kind == GCE_KIND_DENSE) dc_dn.push_back(dc_tiles + i);
             dc_tile_layer.push_back(l);
         }
         dc_tiles += x.dc_ntiles;
@@ -314,6 +329,10 @@ extern "C" int gce_table_create(const gce_layer_desc* descs, int32_t L, gce_tabl
     if (rc == GCE_OK) rc = upload(&t->d_dc_tile_layer, dc_tile_layer);
     t->dc_nl_n = int32_t(dc_nl.size());
     if (rc == GCE_OK) rc = upload(&t->d_dc_nl_tiles, dc_nl);
+    t->dc_sp_n = int32_t(dc_sp.size());
+    if (rc == GCE_OK) rc = upload(&t->d_dc_sp_info, dc_sp);
+    t->dc_dn_n = int32_t(dc_dn.size());
+    if (rc == GCE_OK) rc = upload(&t->d_dc_dn_tiles, dc_dn);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_layer, bunit_layer);
     if (rc == GCE_OK) rc = upload(&t->d_bunit_chunk, bunit_chunk);
     if (rc == GCE_OK) rc = powersgd_plan(t);
