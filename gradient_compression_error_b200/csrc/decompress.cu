@@ -35,7 +35,12 @@ __device__ __forceinline__ int32_t layer_k(const DevLayer& L, const int32_t* k_o
 }
 
 // bounds[w][L.dc_base + ss] = first payload entry of (w, l) whose index lies in
-// decode span ss (1024 outputs) or later; slot nspans holds k.
+// decode span ss (1024 outputs) or later; slot nspans holds k.  A thread takes
+// kDcBoundPer consecutive entries (two 16-byte loads when the payload slice is
+// aligned) and the entry before them, and writes the slots of the spans that
+// begin after an entry's predecessor and at or before the entry itself.
+constexpr int kDcBoundPer = 8;
+
 __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restrict__ layers,
                                                         const int32_t* __restrict__ bunit_layer,
                                                         const int32_t* __restrict__ bunit_chunk,
@@ -48,7 +53,7 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
     const int64_t total = int64_t(bunits_pw) * W;
     for (int64_t u = blockIdx.x; u < total; u += gridDim.x) {
         const int w = int(u / bunits_pw);
-        const int bu = int(u % bunits_pw);
+        const int bu = int(u - int64_t(w) * bunits_pw);
         const int32_t l = bunit_layer[bu];
         const DevLayer L = layers[l];
         const int32_t k = layer_k(L, k_or_rank, l);
@@ -62,24 +67,30 @@ __global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restri
         }
         const int32_t* ix = idx + int64_t(w) * vals_pw + L.val_off;
         const int64_t j1 = min64(j0 + kDcBoundChunk, k);
-        constexpr int kBatch = 8;  // loads in flight per thread
-        for (int64_t jb = j0 + threadIdx.x; jb < j1; jb += int64_t(kBatch) * blockDim.x) {
-            int32_t cur[kBatch], prev[kBatch];
+        const bool vec = (reinterpret_cast<uintptr_t>(ix) & 15) == 0;
+        for (int64_t jb = j0 + int64_t(kDcBoundPer) * threadIdx.x; jb < j1;
+             jb += int64_t(kDcBoundPer) * blockDim.x) {
+            int32_t cur[kDcBoundPer];
+            if (vec && jb + kDcBoundPer <= j1) {
+                const int4 x0 = __ldcg(reinterpret_cast<const int4*>(ix + jb));
+                const int4 x1 = __ldcg(reinterpret_cast<const int4*>(ix + jb) + 1);
+                cur[0] = x0.x; cur[1] = x0.y; cur[2] = x0.z; cur[3] = x0.w;
+                cur[4] = x1.x; cur[5] = x1.y; cur[6] = x1.z; cur[7] = x1.w;
+            } else {
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int64_t j = jb + int64_t(q) * blockDim.x;
-                cur[q] = j < j1 ? ix[j] : 0;
-                prev[q] = (j < j1 && j > 0) ? ix[j - 1] : 0;
+                for (int q = 0; q < kDcBoundPer; ++q) cur[q] = jb + q < j1 ? __ldcg(ix + jb + q) : 0;
             }
+            // span of the previous entry (-1 before the first)
+            int32_t tp = jb > 0 ? min(max(__ldcg(ix + jb - 1), 0) >> kDcSpanLog, nt) : -1;
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int64_t j = jb + int64_t(q) * blockDim.x;
-                if (j >= j1) continue;
+            for (int q = 0; q < kDcBoundPer; ++q) {
+                if (jb + q >= j1) break;
+                const int32_t j = int32_t(jb + q);
                 const int32_t tj = min(max(cur[q], 0) >> kDcSpanLog, nt);
-                const int32_t tp = j > 0 ? min(max(prev[q], 0) >> kDcSpanLog, nt) : -1;
-                for (int32_t tt = tp + 1; tt <= tj; ++tt) b[tt] = int32_t(j);
+                for (int32_t tt = tp + 1; tt <= tj; ++tt) b[tt] = j;
                 if (j == k - 1)
                     for (int32_t tt = tj + 1; tt <= nt; ++tt) b[tt] = k;
+                tp = tj;
             }
         }
     }
