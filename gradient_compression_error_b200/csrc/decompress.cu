@@ -411,6 +411,103 @@ __global__ void __launch_bounds__(kDcThreads) dc_sign_kernel(
     }
 }
 
+// 32 x 32 bit transpose over a warp: lane r holds row r (bit c = entry (r, c))
+// on entry and column r (bit c = entry (c, r)) on return.  Five rounds, each
+// swapping the off-diagonal blocks of half the size with the partner lane.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 16; j >= 1; j >>= 1) {
+        const uint32_t m = j == 16 ? 0x0000FFFFu
+                         : j == 8  ? 0x00FF00FFu
+                         : j == 4  ? 0x0F0F0F0Fu
+                         : j == 2  ? 0x33333333u
+                                   : 0x55555555u;  // bits whose index has bit j clear
+        const uint32_t y = __shfl_xor_sync(kFull, x, j);
+        x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
+    }
+    return x;
+}
+
+// Decode of a SIGN table (SIGN and DENSE layers) for W <= 8 workers.  An
+// output's W sign bits pick one of 2^W worker-order sums of +-s_w, so the
+// block forms that table once per layer -- each entry by the same fp32 adds
+// from +0.0 in worker order as the output's own sum, then times `scale` -- and
+// an output is one lookup.  A warp takes four sign words (128 outputs) of every
+// worker at a time: lane 8c + w holds worker w's word c, and after a 32 x 32
+// bit transpose lane b holds bit b of all 32 words, whose byte c is the W-bit
+// pattern of output 32c + b.  Each block decodes a contiguous run of tiles, so
+// the table is rebuilt only where the layer changes.
+template <bool kApply>
+__global__ void __launch_bounds__(kDcThreads) dc_sign8_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
+    int32_t dc_tiles, int32_t W, int64_t vals_pw, const float* __restrict__ vals, float scale,
+    float* __restrict__ out) {
+    grid_dependency_sync();
+    constexpr int kWarps = kDcThreads / 32;
+    constexpr int kGroups = kDcTile / 128 / kWarps;  // four-word groups a warp takes per tile
+    __shared__ float s_tab[256];
+    __shared__ float s_sc[8];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int wk = lane & 7, col = lane >> 3;
+    const int32_t u0 = int32_t(int64_t(dc_tiles) * blockIdx.x / gridDim.x);
+    const int32_t u1 = int32_t(int64_t(dc_tiles) * (blockIdx.x + 1) / gridDim.x);
+    int32_t tab_layer = -1;
+    for (int32_t u = u0; u < u1; ++u) {
+        const int32_t l = dc_tile_layer[u];
+        const DevLayer L = layers[l];
+        const int64_t start = int64_t(u - L.dc_tile0) << kDcTileLog;
+        const int cnt = int(min64(kDcTile, L.n - start));
+        float* o = out + L.offset + start;
+        if (L.kind == GCE_KIND_DENSE) {
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+                float s = 0.0f;
+                for (int w = 0; w < W; ++w)
+                    s = __fadd_rn(s, vals[int64_t(w) * vals_pw + L.val_off + start + i]);
+                o[i] = dc_final<kApply>(s, scale, o + i);
+            }
+            continue;
+        }
+        if (L.kind != GCE_KIND_SIGN) continue;
+        if (l != tab_layer) {  // the same for the whole block
+            __syncthreads();   // the last layer's table is no longer read
+            if (int(threadIdx.x) < W) s_sc[threadIdx.x] = vals[int64_t(threadIdx.x) * vals_pw + L.val_off];
+            __syncthreads();
+            for (int p = threadIdx.x; p < (1 << W); p += blockDim.x) {
+                float s = 0.0f;
+                for (int w = 0; w < W; ++w) s = __fadd_rn(s, ((p >> w) & 1) ? -s_sc[w] : s_sc[w]);
+                s_tab[p] = __fmul_rn(s, scale);
+            }
+            __syncthreads();
+            tab_layer = l;
+        }
+        const int nwords = (cnt + 31) >> 5;
+        // worker wk's sign words of this tile (a lane with wk >= W reads none)
+        const uint32_t* wp = reinterpret_cast<const uint32_t*>(
+                                 vals + int64_t(wk < W ? wk : 0) * vals_pw + L.val_off + 4) +
+                             (start >> 5);
+        uint32_t x[kGroups];
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+            const int c = (g * kWarps + warp) * 4 + col;  // word of the tile
+            x[g] = (wk < W && c < nwords) ? __ldcg(wp + c) : 0u;
+        }
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g) {
+            const uint32_t pat = warp_transpose32(x[g]);
+            const int i0 = (g * kWarps + warp) * 128 + lane;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int i = i0 + 32 * c;
+                if (i < cnt) {
+                    const float v = s_tab[(pat >> (8 * c)) & 0xFFu];
+                    o[i] = kApply ? __fsub_rn(o[i], v) : v;
+                }
+            }
+        }
+    }
+}
+
 // bounds pass plus the decode kernels for every kind the table holds;
 // apply: out is the parameter vector x and gets x - scale * sum
 template <bool kApply>
@@ -420,6 +517,14 @@ static int launch_decode_t(const gce_table* t, int32_t W, const float* vals, con
     const bool sparse = t->ckind == GCE_KIND_TOPK || t->ckind == GCE_KIND_RANDK;
     static const int r_bounds = resident_blocks(dc_bounds_kernel, 256);
     static const int r_accum = resident_blocks(dc_accum_kernel<kApply>, kDcThreads);
+    if (t->ckind == GCE_KIND_SIGN && W <= 8) {
+        static const int r_sign8 = resident_blocks(dc_sign8_kernel<kApply>, kDcThreads);
+        GCE_LAUNCH_AS(kApply ? "dc_sign8_kernel<true>" : "dc_sign8_kernel<false>",
+                      dc_sign8_kernel<kApply>, wave_grid(t->dc_tiles, 16, r_sign8), kDcThreads,
+                      0, st, t->d_layers, t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, vals,
+                      scale, out);
+        return check_launch();
+    }
     if (t->ckind == GCE_KIND_SIGN) {
         static const int r_sign = resident_blocks(dc_sign_kernel<kApply>, kDcThreads);
         const int grid = wave_grid(t->dc_tiles, 16, r_sign);

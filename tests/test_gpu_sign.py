@@ -171,9 +171,13 @@ def test_bert_base_w8_full_size():
     units = [(0, 0), (7, 4), (3, len(layers) - 1), (5, 8)]
     host_mem = {u: np.zeros(layers[u[1]]["rows"] * layers[u[1]]["cols"], np.float32)
                 for u in units}
+    parted = set()   # units whose trajectories parted at a scale difference
     for s in range(2):
         grad = workloads.gradients(layers, W, 4, s)
         mem_old = run.mem.clone()
+        # a parted unit is checked for one step from the inputs it had on the
+        # GPU; the oracle's own trajectory is never overwritten
+        gpu_in = {(w, l): host(mem_old[w, layer_slice(run.t, l)]) for (w, l) in parted}
         pay = run.step(grad, workloads.ETA, check=False)
         p = mem_old + grad * torch.tensor(workloads.ETA, dtype=torch.float32, device="cuda")
         hv = host(run.vals)
@@ -190,16 +194,12 @@ def test_bert_base_w8_full_size():
         del p, mem_old
         for (w, l) in units:
             ls = layer_slice(run.t, l)
-            sc, words, m_new = oracle.ef_sign_unit(host(grad[w, ls]), host_mem[(w, l)],
-                                                   workloads.ETA)
-            host_mem[(w, l)] = m_new
-            g_sc, g_words = pay[(w, l)]
-            assert np.array_equal(g_words, words), (w, l)
-            assert abs(int(bits(g_sc)) - int(bits(sc))) <= 1
-            if g_sc == sc:
-                assert np.array_equal(bits(host(run.mem[w, ls])), bits(m_new)), (w, l)
-            else:
-                host_mem[(w, l)] = host(run.mem[w, ls])
+            m_in = gpu_in[(w, l)] if (w, l) in parted else host_mem[(w, l)]
+            sc, words, m_new = oracle.ef_sign_unit(host(grad[w, ls]), m_in, workloads.ETA)
+            if (w, l) not in parted:
+                host_mem[(w, l)] = m_new
+            if not same_step(pay[(w, l)], host(run.mem[w, ls]), (sc, words), m_new, (w, l)):
+                parted.add((w, l))
         del grad
     torch.cuda.empty_cache()
 
