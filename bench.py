@@ -68,12 +68,21 @@ def workload_spec(name):
     if name == "vgg19_accordion_topk":           # k 10 % / 1 % chosen by Accordion
         return dict(layers=wl.vgg19("topk", 100000), W=1, cfg=3, method="topk",
                     accordion=(100000, 10000))
+    # a sweep layer, one worker unless the name ends in _w<W> (e.g. the 2^24
+    # layers at W = 8: a small case of the W = 8 decoders)
+    base, sep, wsuf = name.rpartition("_w")
+    W = int(wsuf) if name.startswith("sweep_") and sep and wsuf.isdigit() else 1
+    if W > 1:
+        name = base
     if name.startswith("sweep_topk_e"):          # e.g. sweep_topk_e28_ppm10000
         e, ppm = name[len("sweep_topk_e"):].split("_ppm")
-        return dict(layers=wl.sweep(int(e), "topk", int(ppm)), W=1, cfg=5, method="topk")
+        return dict(layers=wl.sweep(int(e), "topk", int(ppm)), W=W, cfg=5, method="topk")
     if name.startswith("sweep_randk_e"):
         e, ppm = name[len("sweep_randk_e"):].split("_ppm")
-        return dict(layers=wl.sweep(int(e), "randk", int(ppm)), W=1, cfg=5, method="randk")
+        return dict(layers=wl.sweep(int(e), "randk", int(ppm)), W=W, cfg=5, method="randk")
+    if name.startswith("sweep_sign_e"):          # e.g. sweep_sign_e24
+        e = name[len("sweep_sign_e"):]
+        return dict(layers=wl.sweep(int(e), "sign"), W=W, cfg=5, method="sign")
     if name.startswith("sweep_powersgd_e"):      # e.g. sweep_powersgd_e28_r2[_lazy]
         lazy = name.endswith("_lazy")
         e, r = name[len("sweep_powersgd_e"):].replace("_lazy", "").split("_r")

@@ -411,24 +411,6 @@ __global__ void __launch_bounds__(kDcThreads) dc_sign_kernel(
     }
 }
 
-// 32 x 32 bit transpose over a warp: lane r holds row r (bit c = entry (r, c))
-// on entry and column r (bit c = entry (c, r)) on return.  Five rounds, each
-// swapping the off-diagonal blocks of half the size with the partner lane.
-__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int j = 16; j >= 1; j >>= 1) {
-        const uint32_t m = j == 16 ? 0x0000FFFFu
-                         : j == 8  ? 0x00FF00FFu
-                         : j == 4  ? 0x0F0F0F0Fu
-                         : j == 2  ? 0x33333333u
-                                   : 0x55555555u;  // bits whose index has bit j clear
-        const uint32_t y = __shfl_xor_sync(kFull, x, j);
-        x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
-    }
-    return x;
-}
-
 // Decode of a SIGN table (SIGN and DENSE layers) for W <= 8 workers.  An
 // output's W sign bits pick one of 2^W worker-order sums of +-s_w, so the
 // block forms that table once per layer -- each entry by the same fp32 adds

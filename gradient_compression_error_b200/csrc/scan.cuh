@@ -1,4 +1,5 @@
-// scan.cuh -- warp / block prefix sums and the radix-bin crossing search.
+// scan.cuh -- warp / block prefix sums, the warp bit transpose and the
+// radix-bin crossing search.
 #pragma once
 
 #include <cstdint>
@@ -22,6 +23,24 @@ template <class T>
 __device__ __forceinline__ T warp_sum(T x) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(kFull, x, o);
+    return x;
+}
+
+// 32 x 32 bit transpose over a warp: lane r holds row r (bit c = entry (r, c))
+// on entry and column r (bit c = entry (c, r)) on return.  Five rounds, each
+// swapping the off-diagonal blocks of half the size with the partner lane.
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t x) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 16; j >= 1; j >>= 1) {
+        const uint32_t m = j == 16 ? 0x0000FFFFu
+                         : j == 8  ? 0x00FF00FFu
+                         : j == 4  ? 0x0F0F0F0Fu
+                         : j == 2  ? 0x33333333u
+                                   : 0x55555555u;  // bits whose index has bit j clear
+        const uint32_t y = __shfl_xor_sync(kFull, x, j);
+        x = (lane & j) ? ((x & ~m) | ((y >> j) & m)) : ((x & m) | ((y << j) & ~m));
+    }
     return x;
 }
 

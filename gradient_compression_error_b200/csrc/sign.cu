@@ -338,7 +338,75 @@ __global__ void __launch_bounds__(256, 4) sg_fused_kernel(
 }
 
 // ---- majority vote ---------------------------------------------------------------------
+// Majority vote of a SIGN table (SIGN and DENSE layers) for W <= 16 workers,
+// one 4096-output tile per block step.  A warp takes the words of S worker
+// slots (S the power of two at or above W) for 32 / S columns at a time: lane
+// S c + w holds worker w's word c, and after a 32 x 32 bit transpose lane b
+// holds bit b of every one of those words, the S-bit field c of which marks
+// the workers with a negative sign at output 32 c + b; its population count is
+// the vote.  A lane has kVoteBatch words in flight before their transposes,
+// and every store writes 32 consecutive outputs.
+constexpr int kVoteBatch = 8;
+
 __global__ void __launch_bounds__(128) sg_vote_kernel(
+    const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
+    int32_t dc_tiles, int32_t W, int64_t vals_pw, const float* __restrict__ vals, float scale,
+    float* __restrict__ out) {
+    grid_dependency_sync();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    int S = 1;
+    while (S < W) S <<= 1;
+    const int cols = 32 / S;                // columns a warp takes per transpose
+    const int step = nwarps * cols;         // columns a block takes per transpose
+    const int wk = lane & (S - 1), cl = lane / S;
+    const uint32_t fmask = S == 32 ? 0xFFFFFFFFu : ((1u << S) - 1u);
+    for (int32_t u = blockIdx.x; u < dc_tiles; u += gridDim.x) {
+        const int32_t l = dc_tile_layer[u];
+        const DevLayer L = layers[l];
+        const int64_t start = int64_t(u - L.dc_tile0) << kDcTileLog;
+        const int cnt = int(min64(kDcTile, L.n - start));
+        float* o = out + L.offset + start;
+        if (L.kind == GCE_KIND_SIGN) {
+            const int nwords = (cnt + 31) >> 5;
+            // worker wk's sign words of this tile (a lane with wk >= W reads none)
+            const uint32_t* wp = reinterpret_cast<const uint32_t*>(
+                                     vals + int64_t(wk < W ? wk : 0) * vals_pw + L.val_off + 4) +
+                                 (start >> 5);
+            for (int c0 = warp * cols; c0 < nwords; c0 += kVoteBatch * step) {
+                uint32_t x[kVoteBatch];
+#pragma unroll
+                for (int b = 0; b < kVoteBatch; ++b) {
+                    const int c = c0 + b * step + cl;
+                    x[b] = (wk < W && c < nwords) ? __ldcg(wp + c) : 0u;
+                }
+#pragma unroll
+                for (int b = 0; b < kVoteBatch; ++b) {
+                    const int cb = c0 + b * step;  // the same for the whole warp
+                    if (cb >= nwords) break;
+                    const uint32_t neg = warp_transpose32(x[b]);
+                    for (int cc = 0; cc < cols; ++cc) {
+                        const int i = 32 * (cb + cc) + lane;
+                        const int v = W - 2 * __popc((neg >> (S * cc)) & fmask);
+                        if (i < cnt) o[i] = v > 0 ? scale : (v < 0 ? -scale : 0.0f);
+                    }
+                }
+            }
+        } else if (L.kind == GCE_KIND_DENSE) {
+            for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+                float s = 0.0f;
+                for (int w = 0; w < W; ++w)
+                    s = __fadd_rn(s, vals[int64_t(w) * vals_pw + L.val_off + start + i]);
+                o[i] = __fmul_rn(s, scale);
+            }
+        }
+    }
+}
+
+// The same vote for more than 16 workers: four outputs a thread, each worker's
+// bits added one by one.  (With 32 worker slots a lane's word comes from its
+// own worker, so every load of the transposed form touches 32 sectors; this
+// form measured faster there.)
+__global__ void __launch_bounds__(128) sg_vote_wide_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ dc_tile_layer,
     int32_t dc_tiles, int32_t W, int64_t vals_pw, const float* __restrict__ vals, float scale,
     float* __restrict__ out) {
@@ -623,8 +691,12 @@ extern "C" int decompress_vote(const gce_table* t, int32_t W, const float* vals,
     if (t->vals_pw > 0 && !vals) return GCE_ERR_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     static const int r_vote = resident_blocks(sg_vote_kernel, 128);
-    if (t->dc_tiles > 0)
+    static const int r_vote_wide = resident_blocks(sg_vote_wide_kernel, 128);
+    if (t->dc_tiles > 0 && W <= 16)
         GCE_LAUNCH(sg_vote_kernel, wave_grid(t->dc_tiles, 16, r_vote), 128, 0, st, t->d_layers,
                    t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, vals, scale, out);
+    else if (t->dc_tiles > 0)
+        GCE_LAUNCH(sg_vote_wide_kernel, wave_grid(t->dc_tiles, 16, r_vote_wide), 128, 0, st,
+                   t->d_layers, t->d_dc_tile_layer, t->dc_tiles, W, t->vals_pw, vals, scale, out);
     return check_launch();
 }

@@ -89,7 +89,8 @@ def sweep(e, method="topk", ppm=10000, rank=2):
     if method == "powersgd":
         return [dict(rows=1 << (e // 2), cols=1 << ((e + 1) // 2), kind="powersgd", cap=rank,
                      sigma=1.0)]
-    return [dict(rows=n, cols=1, kind=method, cap=_ppm_k(n, ppm), sigma=1.0)]
+    return [dict(rows=n, cols=1, kind=method, cap=0 if method == "sign" else _ppm_k(n, ppm),
+                 sigma=1.0)]
 
 
 def total_elements(layers):

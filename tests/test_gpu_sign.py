@@ -228,6 +228,26 @@ def test_thirty_three_workers_sum_vote_and_noalloc():
     assert np.array_equal(bits(host(vote)), bits(osteps.vote(layers, W, pay, 2.0)))
 
 
+@pytest.mark.parametrize("W", [1, 8, 16, 17, 32])
+def test_vote_and_sum_at_several_worker_counts(W):
+    """Both aggregates on the ragged table, bit for bit against the oracle: one
+    worker, 8 (the sum by its table of 256 worker-order sums; the vote with four
+    words a lane group), 16 (the last transposed vote), 17 and 32 (the vote a
+    thread per four outputs)."""
+    need_gpu()
+    g = gce()
+    run = SignRun(RAGGED, W)
+    pay = run.step(workloads.gradients(RAGGED, W, 703, 0), 0.05, check=False)
+    t = run.t
+    vote = torch.full((t.N,), float("nan"), device="cuda")
+    g.decompress_vote(t, W, run.vals, 0.5, vote)
+    assert np.array_equal(bits(host(vote)), bits(osteps.vote(RAGGED, W, pay, 0.5)))
+    out = torch.full((t.N,), float("nan"), device="cuda")
+    g.decompress_accumulate(t, W, run.vals, None, None, None, None, 0.25, out,
+                            t.workspace(W, "decompress"))
+    assert np.array_equal(bits(host(out)), bits(osteps.decompress(RAGGED, W, pay, 0.25)))
+
+
 PIPE_LAYERS = [dict(rows=190000, cols=1, kind="sign", cap=0, sigma=1.0),
                dict(rows=33, cols=1, kind="dense", cap=0, sigma=1.0),
                dict(rows=5000, cols=3, kind="sign", cap=0, sigma=0.5),
