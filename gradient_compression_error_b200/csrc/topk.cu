@@ -21,8 +21,13 @@
 //            to the exact fallback; histogram work is cut into units
 //   restore  + respill  the fallback: memory zeroed above hi gets v back
 //            from the candidate list, then the layer is re-listed whole
-//   hist1-3  three 11/11/9-bit radix levels over the candidate values find
-//            the exact k-th largest key T and how many keys equal to T to take
+//   hist1-3  radix levels over the candidate keys find the exact k-th largest
+//            key T and how many keys equal to T to take.  Level 1 spends 3072
+//            of its 4096 bins on [lo, top] (top: a sampled upper bound on T with
+//            the same margin as lo) and 1024 on the keys above, so that T's bin
+//            is narrow (a few hundred keys) and level 2 (4096 bins over that
+//            bin) fixes T; level 3 has work only when T fell in a coarse bin or
+//            the layer was re-listed whole (every range then needs three levels)
 //   count / scan / emit   per-tile counts of key > T and key == T, a prefix
 //            over the tiles, then the ordered write of (v, i); memory +0 for
 //            chosen entries at or below hi, v again for entries above hi that
@@ -73,16 +78,6 @@ __device__ __forceinline__ int32_t* tk_hist(int32_t* hists, int64_t S, int level
     return hists + S * kTkSBins + (int64_t(level - 1) * S + seg) * kTkBins;
 }
 
-// Shared-memory histogram add, combining lanes of a warp that hit the same bin
-// (candidate keys cluster in a few bins).  Call with the whole warp.
-__device__ __forceinline__ void hist_add(int32_t* h, uint32_t bin, bool take) {
-    const unsigned active = __ballot_sync(kFull, take);
-    if (take) {
-        const unsigned peers = __match_any_sync(active, bin);
-        if ((threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&h[bin], __popc(peers));
-    }
-}
-
 // ---- setup -------------------------------------------------------------------
 __global__ void __launch_bounds__(256) tk_setup_kernel(const DevLayer* __restrict__ layers,
                                                        const int32_t* __restrict__ comp,
@@ -107,6 +102,7 @@ __global__ void __launch_bounds__(256) tk_setup_kernel(const DevLayer* __restric
         }
         g.lo = 0;            // until the sample pass sets them: list every
         g.hi = 0xFFFFFFFFu;  // element and zero nothing in the main pass
+        g.top = 0x7FFFFFFFu;
         segs[s] = g;
     }
 }
@@ -204,6 +200,7 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
                 if (tid == 0 && b >= 0) {
                     segs[seg].lo = uint32_t(b) << 19;
                     segs[seg].hi = ((uint32_t(b) + 1u) << 19) - 1u;
+                    segs[seg].top = ((uint32_t(b) + 1u) << 19) - 1u;
                 }
             } else if (tid < 32) {
                 const int64_t ns = tk_samples_in(L.n);
@@ -224,9 +221,24 @@ __global__ void __launch_bounds__(256) tk_sample_kernel(
                     if (key >= 0) hi = uint32_t(key);
                 }
                 if (hi < lo) hi = lo;  // everything zeroed above hi must be a candidate
+                // top: the top edge of the bin where the count from the top
+                // reaches mu - margin samples, T's upper bound with lo's margin;
+                // with fewer samples than that above T, the largest sample's bin
+                // (T lies above every sample with probability about e^-mu, and
+                // a T above top costs a third radix level, not exactness)
+                int64_t t_top = int64_t(floor(mu - margin));
+                if (t_top < 1) t_top = 1;
+                uint32_t top = 0x7FFFFFFFu;
+                {
+                    int64_t above = 0;
+                    const int b = warp_find_from_top(h, kTkSBins, t_top, &above);
+                    if (b >= 0) top = ((uint32_t(b) + 1u) << 19) - 1u;
+                }
+                if (top < lo) top = lo;
                 if (tid == 0) {
                     segs[seg].lo = lo;
                     segs[seg].hi = hi;
+                    segs[seg].top = top;
                 }
             }
         }
@@ -411,6 +423,7 @@ __global__ void __launch_bounds__(1024) tk_units_kernel(const DevLayer* __restri
             }
             g.count = cnt;
             g.prefix = 0;
+            g.width = 0;
             g.need = g.k;
         }
         int tot = 0;
@@ -488,9 +501,48 @@ __global__ void __launch_bounds__(256) tk_respill_kernel(
     }
 }
 
-// ---- radix levels over the candidate values --------------------------------------------
+// ---- radix levels over the candidate keys ------------------------------------------------
+// Smallest s with (width - 1) >> s below nb (width >= 1, nb a power of two).
+__device__ __forceinline__ int tk_shift_pow2(uint32_t width, int log2_nb) {
+    const int bits = 32 - __clz(width - 1u);
+    return bits > log2_nb ? bits - log2_nb : 0;
+}
+
+// Level 1's bins of a segment: kTkFine bins of 2^sf keys from f0 for keys below
+// f1, then kTkBins - kTkFine bins of 2^sc keys from f1 up to the largest key.
+// A re-listed layer (every element a candidate) has no fine part.
+struct TkL1Bins {
+    uint32_t f0, f1;
+    int sf, sc;
+    __device__ __forceinline__ TkL1Bins(const TkSeg& g) {
+        f0 = g.redo ? 0u : g.lo;
+        f1 = g.redo ? 0u : g.top + 1u;  // top <= 2^31 - 1
+        sf = 0;
+        if (f1 > f0) {
+            sf = tk_shift_pow2(f1 - f0, 12);
+            while (((f1 - f0 - 1u) >> sf) >= uint32_t(kTkFine)) ++sf;
+        }
+        sc = f1 < 0x80000000u ? tk_shift_pow2(0x80000000u - f1, 10) : 0;
+    }
+    // (a listed key is never below f0; the clamp keeps any key inside the bins)
+    __device__ __forceinline__ uint32_t bin(uint32_t key) const {
+        return key < f1 ? min((key - f0) >> sf, uint32_t(kTkFine - 1))
+                        : uint32_t(kTkFine) + ((key - f1) >> sc);
+    }
+    // [base, base + width) of bin b
+    __device__ __forceinline__ void range(int b, uint32_t* base, uint32_t* width) const {
+        if (b < kTkFine) {
+            *base = f0 + (uint32_t(b) << sf);
+            *width = min(f1 - *base, 1u << sf);
+        } else {
+            *base = f1 + (uint32_t(b - kTkFine) << sc);
+            *width = min(0x80000000u - *base, 1u << sc);
+        }
+    }
+};
+
 template <int kLevel>
-__global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restrict__ layers,
+__global__ void __launch_bounds__(256, 6) tk_hist_kernel(const DevLayer* __restrict__ layers,
                                                       const int32_t* __restrict__ comp,
                                                       int32_t ncomp, int64_t S, int64_t comp_N,
                                                       TkSeg* __restrict__ segs,
@@ -499,8 +551,6 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
                                                       int32_t* __restrict__ hists,
                                                       const float* __restrict__ spill_v) {
     grid_dependency_sync();
-    constexpr int kNb = kLevel == 3 ? 512 : kTkBins;
-    constexpr int kShift = kLevel == 1 ? 20 : (kLevel == 2 ? 9 : 0);
     constexpr int kPer = 16;  // candidates per thread per load batch
     __shared__ int32_t h[kTkBins];
     __shared__ int s_last;
@@ -509,34 +559,39 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
     for (int32_t u = blockIdx.x; u < total; u += gridDim.x) {
         const int2 us = unit_seg[u];
         const int64_t s = us.x;
+        const TkSeg g = segs[s];
+        // levels 2 and 3 bin the range [base, base + width) that holds T; a
+        // range of one key is T itself
+        const uint32_t base = g.prefix, width = g.width;
+        if (kLevel > 1 && width <= 1u) continue;  // the same for the whole block
+        const TkL1Bins l1(g);
+        const int shift = kLevel > 1 ? tk_shift_pow2(width, 12) : 0;
         const int w = int(s / ncomp);
         const DevLayer L = layers[comp[s % ncomp]];
-        const uint32_t prefix = segs[s].prefix;
-        const int32_t count = segs[s].count;
         const int64_t j0 = int64_t(us.y) * kTkHUnit;
-        for (int b = tid; b < kNb; b += blockDim.x) h[b] = 0;
+        for (int b = tid; b < kTkBins; b += blockDim.x) h[b] = 0;
         __syncthreads();
         const float* e = spill_v + int64_t(w) * comp_N + L.sp_off;
-        for (int64_t jb = j0; jb < min64(j0 + kTkHUnit, count); jb += int64_t(kPer) * 256) {
+        for (int64_t jb = j0; jb < min64(j0 + kTkHUnit, g.count); jb += int64_t(kPer) * 256) {
             uint32_t key[kPer];
 #pragma unroll
             for (int q = 0; q < kPer; ++q) {
                 const int64_t j = jb + int64_t(q) * 256 + tid;
-                key[q] = j < count ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
+                key[q] = j < g.count ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
             }
 #pragma unroll
             for (int q = 0; q < kPer; ++q) {
-                bool take = key[q] != 0xFFFFFFFFu;
-                if (kLevel == 2) take = take && (key[q] >> 20) == (prefix >> 20);
-                if (kLevel == 3) take = take && (key[q] >> 9) == (prefix >> 9);
-                const uint32_t bin = (key[q] >> kShift) & (kNb - 1);
-                if (kLevel == 1) hist_add(h, bin, take);   // few, crowded bins
-                else if (take) atomicAdd(&h[bin], 1);
+                if (key[q] == 0xFFFFFFFFu) continue;
+                if (kLevel == 1) {
+                    atomicAdd(&h[l1.bin(key[q])], 1);
+                } else if (key[q] - base < width) {
+                    atomicAdd(&h[(key[q] - base) >> shift], 1);
+                }
             }
         }
         __syncthreads();
         int32_t* gh = tk_hist(hists, S, kLevel, s);
-        for (int b = tid; b < kNb; b += blockDim.x)
+        for (int b = tid; b < kTkBins; b += blockDim.x)
             if (h[b]) atomicAdd(gh + b, h[b]);
         __threadfence();
         __syncthreads();
@@ -547,17 +602,35 @@ __global__ void __launch_bounds__(256, 8) tk_hist_kernel(const DevLayer* __restr
         }
         __syncthreads();
         if (s_last) {
+            // the last unit of the segment: find T's bin, narrow the range
             __threadfence();
-            for (int b = tid; b < kNb; b += blockDim.x) h[b] = __ldcg(gh + b);
+            for (int b = tid; b < kTkBins; b += blockDim.x) h[b] = __ldcg(gh + b);
             __syncthreads();
+            __shared__ uint32_t s_width;
             if (tid < 32) {
                 int64_t above = 0;
-                const int32_t need = segs[s].need;
-                const int b = warp_find_from_top(h, kNb, need, &above);
-                if (tid == 0 && b >= 0) {
-                    segs[s].prefix = prefix | (uint32_t(b) << kShift);
-                    segs[s].need = need - int32_t(above);
+                const int b = warp_find_from_top(h, kTkBins, g.need, &above);
+                uint32_t nb = base, nw = 1u;  // no crossing (cannot happen): stop here
+                if (b >= 0) {
+                    if (kLevel == 1) {
+                        l1.range(b, &nb, &nw);
+                    } else {
+                        nb = base + (uint32_t(b) << shift);
+                        nw = min(width - (uint32_t(b) << shift), 1u << shift);
+                    }
                 }
+                if (tid == 0) {
+                    segs[s].prefix = nb;
+                    segs[s].width = nw;
+                    if (b >= 0) segs[s].need = g.need - int32_t(above);
+                    s_width = nw;
+                }
+            }
+            __syncthreads();
+            // the next level's histogram of this segment starts at zero
+            if (kLevel < 3 && s_width > 1u) {
+                int32_t* nh = tk_hist(hists, S, kLevel + 1, s);
+                for (int b = tid; b < kTkBins; b += blockDim.x) nh[b] = 0;
             }
         }
         __syncthreads();
@@ -733,7 +806,9 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         int2* tile_cnt = at<int2>(ws, lay.tile_cnt);
         float* spill_v = at<float>(ws, lay.spill_v);
         int32_t* spill_i = at<int32_t>(ws, lay.spill_i);
-        const int64_t n4 = lay.S * (kTkSBins + 3 * kTkBins) / 4;
+        // the sample and level-1 histograms; a level's last block clears the
+        // next level's histogram of its segment when that level has work
+        const int64_t n4 = lay.S * (kTkSBins + kTkBins) / 4;
 
         static const int r_setup = resident_blocks(tk_setup_kernel, 256);
         static const int r_sample = resident_blocks(tk_sample_kernel, 256);

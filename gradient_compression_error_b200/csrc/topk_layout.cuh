@@ -8,7 +8,8 @@ namespace gce {
 constexpr int kTkThreads = 256;                    // main pass: 256 threads x 32 elements
 constexpr int kTkPerThread = 32;
 constexpr int kTkTile = kTkThreads * kTkPerThread;  // 8192 elements per main tile
-constexpr int kTkBins = 2048;                      // radix bins per level (11 bits)
+constexpr int kTkBins = 4096;                      // radix bins per level
+constexpr int kTkFine = 3072;                      // level-1 bins inside the sampled bracket
 constexpr int kTkSBins = 4096;                     // sample bins: 2^19 keys, 16 per octave
 constexpr int kTkSampleChunk = 32;                 // sampled run length (one 128-B line)
 constexpr int kTkSampleStride = 4096;              // one run per 4096 elements
@@ -26,10 +27,13 @@ struct TkSeg {
     int32_t count;       // candidates used for the selection
     int32_t redo;        // 1: the main list was short; the layer was re-listed whole
     int32_t done_s, done_1, done_2, done_3;  // last-block counters
-    uint32_t prefix;     // key bits fixed so far by the radix selection (T after level 3)
-    int32_t need;        // rank still to find below the prefix; after level 3:
-                         // how many keys equal to T are taken
-    int32_t pad[3];
+    uint32_t prefix;     // lowest key of the range that holds T (T once width is 1)
+    int32_t need;        // rank of T, counted from the top, inside that range; once
+                         // resolved: how many keys equal to T are taken
+    uint32_t top;        // T <= top almost surely (sample bound); level 1's fine bins
+                         // span [lo, top]
+    uint32_t width;      // keys in the range [prefix, prefix + width) that holds T
+    int32_t pad;
 };
 static_assert(sizeof(TkSeg) == 64, "TkSeg is one 64-byte record");
 

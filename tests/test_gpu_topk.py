@@ -191,6 +191,32 @@ def test_large_table_with_fallback_in_every_layer():
             g.set_bracket_sigma(6.0)
 
 
+def test_sample_blind_to_the_large_values_takes_the_coarse_levels():
+    """The sample reads the first 32 elements of every 4096; here those are a
+    thousand times smaller than the rest, so both sampled bounds come out far
+    too low: nearly every element is a candidate (no fallback) and T lies above
+    the upper bound, in one of level 1's coarse bins, so the selection takes all
+    three radix levels.  Bit-exact against the oracle over two steps."""
+    need_gpu()
+    layers = [dict(rows=300000, cols=1, kind="topk", cap=3000, sigma=1.0),
+              dict(rows=1000, cols=1000, kind="topk", cap=20000, sigma=1.0)]
+    W = 2
+
+    def mk(t):
+        grad = workloads.gradients(layers, W, 108, t)
+        pos = torch.arange(grad.shape[1], device="cuda")
+        off = 0
+        for l in layers:
+            n = l["rows"] * l["cols"]
+            seen = ((pos[off:off + n] - off) % 4096) < 32
+            grad[:, off:off + n][:, seen] *= 1e-3
+            off += n
+        return grad
+
+    run = run_and_compare(layers, W, 2, mk, eta=1.0)
+    assert not run.g.status(run.ws) & run.g.STATUS_FALLBACK
+
+
 def test_k_out_of_range_skips_layer_and_flags():
     need_gpu()
     g = gce()
