@@ -25,11 +25,15 @@
 //            key T and how many keys equal to T to take.  Level 1 spends 3072
 //            of its 4096 bins on [lo, top] (top: a sampled upper bound on T with
 //            the same margin as lo) and 1024 on the keys above, so that T's bin
-//            is narrow (a few hundred keys) and level 2 (4096 bins over that
-//            bin) fixes T; level 3 has work only when T fell in a coarse bin or
-//            the layer was re-listed whole (every range then needs three levels)
+//            is narrow (a few hundred keys); then either the count pass lists
+//            the few keys in that bin and the scan fixes T from the list (the
+//            usual case), or level 2 (4096 bins over that bin) fixes it; level
+//            3 has work only when T fell in a coarse bin or the layer was
+//            re-listed whole (every range then needs three levels)
 //   count / scan / emit   per-tile counts of key > T and key == T, a prefix
-//            over the tiles, then the ordered write of (v, i); memory +0 for
+//            over the tiles (first fixing T from the list, where there is one,
+//            and adding the listed keys to their tiles' counts), then the
+//            ordered write of (v, i); memory +0 for
 //            chosen entries at or below hi, v again for entries above hi that
 //            were not chosen
 // Results never depend on lo or hi.  DRAM traffic: 12 B per element (read
@@ -563,7 +567,8 @@ __global__ void __launch_bounds__(256, 6) tk_hist_kernel(const DevLayer* __restr
         // levels 2 and 3 bin the range [base, base + width) that holds T; a
         // range of one key is T itself
         const uint32_t base = g.prefix, width = g.width;
-        if (kLevel > 1 && width <= 1u) continue;  // the same for the whole block
+        // (the same for the whole block)
+        if (kLevel > 1 && (width <= 1u || g.list_mode)) continue;
         const TkL1Bins l1(g);
         const int shift = kLevel > 1 ? tk_shift_pow2(width, 12) : 0;
         const int w = int(s / ncomp);
@@ -619,11 +624,17 @@ __global__ void __launch_bounds__(256, 6) tk_hist_kernel(const DevLayer* __restr
                         nw = min(width - (uint32_t(b) << shift), 1u << shift);
                     }
                 }
+                // a narrow bin with few keys and room for them after the
+                // candidates: the count pass lists them and the scan fixes T
+                const bool list = kLevel == 1 && b >= 0 && !g.redo && nw > 1u &&
+                                  nw <= uint32_t(kTkBins) && h[b] <= kTkListMax &&
+                                  int64_t(g.count) + h[b] <= L.n;
                 if (tid == 0) {
                     segs[s].prefix = nb;
                     segs[s].width = nw;
+                    segs[s].list_mode = list ? 1 : 0;
                     if (b >= 0) segs[s].need = g.need - int32_t(above);
-                    s_width = nw;
+                    s_width = list ? 1u : nw;
                 }
             }
             __syncthreads();
@@ -640,13 +651,15 @@ __global__ void __launch_bounds__(256, 6) tk_hist_kernel(const DevLayer* __restr
 // ---- per-tile counts, prefix over tiles, ordered emit --------------------------------------
 __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restrict__ tile_info,
                                                        int32_t tiles_pw, int32_t W, int32_t ncomp,
-                                                       int64_t comp_N, const TkSeg* __restrict__ segs,
+                                                       int64_t comp_N, TkSeg* __restrict__ segs,
                                                        const int2* __restrict__ tile_dir,
                                                        int2* __restrict__ tile_cnt,
-                                                       const float* __restrict__ spill_v) {
+                                                       float* __restrict__ spill_v,
+                                                       int32_t* __restrict__ spill_i) {
     grid_dependency_sync();
     constexpr int kBatch = 8;
     const int lane = threadIdx.x & 31;
+    const unsigned lt_mask = (1u << lane) - 1u;
     const int64_t total = int64_t(tiles_pw) * W;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
     for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
@@ -659,7 +672,12 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
         int gt = 0, eq = 0;
         if (k > 0) {
             const uint32_t T = segs[s].prefix;
-            const float* e = spill_v + int64_t(w) * comp_N + ti.sp_off + d.x;
+            // list mode: T lies in [T, T + width); keys at or above its top are
+            // counted as greater and the keys inside are listed for the scan
+            const bool list = segs[s].list_mode != 0;
+            const uint32_t width = segs[s].width;
+            const int64_t seg0 = int64_t(w) * comp_N + ti.sp_off;
+            const float* e = spill_v + seg0 + d.x;
             for (int j0 = 0; j0 < d.y; j0 += 32 * kBatch) {
                 uint32_t key[kBatch];
 #pragma unroll
@@ -667,10 +685,35 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
                     const int j = j0 + q * 32 + lane;
                     key[q] = j < d.y ? abs_key(__ldcg(e + j)) : 0xFFFFFFFFu;
                 }
+                if (!list) {
+#pragma unroll
+                    for (int q = 0; q < kBatch; ++q) {
+                        gt += key[q] != 0xFFFFFFFFu && key[q] > T;
+                        eq += key[q] == T;
+                    }
+                    continue;
+                }
+                bool any_in = false;
 #pragma unroll
                 for (int q = 0; q < kBatch; ++q) {
-                    gt += key[q] != 0xFFFFFFFFu && key[q] > T;
-                    eq += key[q] == T;
+                    const bool valid = key[q] != 0xFFFFFFFFu;
+                    gt += valid && key[q] - T >= width && key[q] > T;
+                    any_in |= valid && key[q] - T < width;
+                }
+                if (!__any_sync(kFull, any_in)) continue;  // the usual batch
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    const bool in = key[q] != 0xFFFFFFFFu && key[q] - T < width;
+                    const unsigned m = __ballot_sync(kFull, in);
+                    if (m == 0u) continue;
+                    int pos = 0;
+                    if (lane == 0) pos = atomicAdd(&segs[s].list_n, __popc(m));
+                    pos = __shfl_sync(kFull, pos, 0) + __popc(m & lt_mask);
+                    if (in) {
+                        const int64_t o = seg0 + segs[s].count + pos;
+                        reinterpret_cast<uint32_t*>(spill_v)[o] = key[q];
+                        spill_i[o] = int32_t(t);
+                    }
                 }
             }
             gt = warp_sum(gt);
@@ -683,19 +726,86 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
 __global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restrict__ layers,
                                                        const int32_t* __restrict__ comp,
                                                        int32_t ncomp, int64_t S, int32_t tiles_pw,
-                                                       const TkSeg* __restrict__ segs,
-                                                       int2* __restrict__ tile_cnt) {
+                                                       int64_t comp_N, TkSeg* __restrict__ segs,
+                                                       int2* __restrict__ tile_cnt,
+                                                       const float* __restrict__ spill_v,
+                                                       const int32_t* __restrict__ spill_i) {
     grid_dependency_sync();
     __shared__ int s_warp[33];
+    __shared__ int32_t h[kTkBins];
+    __shared__ uint32_t s_key[1024];
+    __shared__ uint32_t s_T;
+    __shared__ int32_t s_need;
     for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
         if (segs[s].k == 0) continue;
         const int w = int(s / ncomp);
         const DevLayer L = layers[comp[s % ncomp]];
         int2* tc = tile_cnt + int64_t(w) * tiles_pw + L.tile0;
+        if (segs[s].list_mode) {
+            // fix T from the listed keys of level 1's bin [base, base + width),
+            // then add each listed key to its tile's counts
+            const uint32_t base = segs[s].prefix;
+            const int32_t need = segs[s].need, c = segs[s].list_n;
+            const int64_t o = int64_t(w) * comp_N + L.sp_off + segs[s].count;
+            const uint32_t* lk = reinterpret_cast<const uint32_t*>(spill_v) + o;
+            const int32_t* lt = spill_i + o;
+            if (c <= int(blockDim.x)) {
+                // a short list: each key counts the keys above and equal to
+                // it; T is the key whose count from the top reaches need (the
+                // first thread holding it writes)
+                if (threadIdx.x == 0) {
+                    s_T = base;
+                    s_need = need;
+                }
+                if (int(threadIdx.x) < c) s_key[threadIdx.x] = lk[threadIdx.x];
+                __syncthreads();
+                if (int(threadIdx.x) < c) {
+                    const uint32_t me = s_key[threadIdx.x];
+                    int gt = 0, eq = 0, eq_before = 0;
+                    for (int j = 0; j < c; ++j) {
+                        const uint32_t x = s_key[j];
+                        gt += x > me;
+                        eq += x == me;
+                        eq_before += x == me && j < int(threadIdx.x);
+                    }
+                    if (gt < need && need <= gt + eq && eq_before == 0) {
+                        s_T = me;
+                        s_need = need - gt;
+                    }
+                }
+            } else {
+                for (int b = threadIdx.x; b < kTkBins; b += blockDim.x) h[b] = 0;
+                __syncthreads();
+                for (int i = threadIdx.x; i < c; i += blockDim.x) atomicAdd(&h[lk[i] - base], 1);
+                __syncthreads();
+                if (threadIdx.x < 32) {
+                    int64_t above = 0;
+                    const int b = warp_find_from_top(h, kTkBins, need, &above);
+                    if (threadIdx.x == 0) {
+                        s_T = b >= 0 ? base + uint32_t(b) : base;
+                        s_need = b >= 0 ? need - int32_t(above) : need;
+                    }
+                }
+            }
+            __syncthreads();
+            const uint32_t T = s_T;
+            if (threadIdx.x == 0) {
+                segs[s].prefix = T;
+                segs[s].width = 1u;
+                segs[s].need = s_need;
+            }
+            for (int i = threadIdx.x; i < c; i += blockDim.x) {
+                const uint32_t key = lk[i];
+                if (key > T) atomicAdd(&tile_cnt[lt[i]].x, 1);
+                else if (key == T) atomicAdd(&tile_cnt[lt[i]].y, 1);
+            }
+            __syncthreads();
+        }
         int carry_gt = 0, carry_eq = 0;
         for (int b0 = 0; b0 < L.ntiles; b0 += blockDim.x) {
             const int i = b0 + threadIdx.x;
-            const int2 x = i < L.ntiles ? tc[i] : make_int2(0, 0);
+            // from L2, where the atomic additions above were made
+            const int2 x = i < L.ntiles ? __ldcg(tc + i) : make_int2(0, 0);
             int tg = 0, te = 0;
             const int eg = block_exclusive_scan(x.x, s_warp, &tg);
             const int ee = block_exclusive_scan(x.y, s_warp, &te);
@@ -705,6 +815,7 @@ __global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restric
         }
     }
 }
+
 
 __global__ void __launch_bounds__(256) tk_emit_kernel(
     const TileInfo* __restrict__ tile_info, int32_t tiles_pw,
@@ -849,9 +960,9 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
                    t->comp_N, segs, unit_start, unit_seg, hists, spill_v);
         const int64_t wwork = (lay.TT + 7) / 8;  // a warp per tile
         GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_tile_info,
-                   t->tiles_pw, W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v);
+                   t->tiles_pw, W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v, spill_i);
         GCE_LAUNCH(tk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
-                   lay.S, t->tiles_pw, segs, tile_cnt);
+                   lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, spill_v, spill_i);
         GCE_LAUNCH(tk_emit_kernel, wave_grid(wwork, 8, r_emit), 256, 0, st, t->d_tile_info,
                    t->tiles_pw, W, ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt,
                    spill_v, spill_i, mem, vals, idx);

@@ -16,6 +16,7 @@ constexpr int kTkSampleStride = 4096;              // one run per 4096 elements
 constexpr int64_t kTkSamplePart = int64_t(1) << 20; // elements covered by one sample unit
 constexpr int64_t kTkSampleMinN = 65536;           // smaller layers: exact histogram of all
 constexpr int kTkHUnit = 16384;                    // candidates per histogram unit
+constexpr int kTkListMax = 65536;                  // longest list of keys in T's level-1 bin
 
 // Per (worker, layer) state of one top-k step.
 struct TkSeg {
@@ -33,8 +34,10 @@ struct TkSeg {
     uint32_t top;        // T <= top almost surely (sample bound); level 1's fine bins
                          // span [lo, top]
     uint32_t width;      // keys in the range [prefix, prefix + width) that holds T
-    int32_t pad;
+    int32_t list_mode;   // 1: T is found from a list of the keys in level 1's bin
+    int32_t list_n;      // keys appended to that list by the count pass
+    int32_t pad[3];
 };
-static_assert(sizeof(TkSeg) == 64, "TkSeg is one 64-byte record");
+static_assert(sizeof(TkSeg) == 80, "TkSeg is one 80-byte record");
 
 }  // namespace gce

@@ -121,6 +121,22 @@ def test_ties_integer_gradients():
     run_and_compare(layers, W, 3, mk, eta=1.0)
 
 
+def test_short_list_with_ties_at_T():
+    """Gradients on a 1/64 grid: the value at the k-th place recurs a few hundred
+    times, so the short list of keys in T's level-1 bin, from which the scan
+    fixes T, holds ties at T that split across tiles.  Bit-exact, three steps."""
+    need_gpu()
+    layers = [dict(rows=300000, cols=1, kind="topk", cap=3000, sigma=1.0),
+              dict(rows=700, cols=900, kind="topk", cap=6300, sigma=1.0),
+              dict(rows=65536, cols=1, kind="topk", cap=655, sigma=1.0)]
+    W = 2
+
+    def mk(t):
+        return torch.round(workloads.gradients(layers, W, 109, t) * 64.0) / 64.0
+
+    run_and_compare(layers, W, 3, mk, eta=1.0)
+
+
 def test_all_equal_magnitudes_and_zeros():
     need_gpu()
     layers = [dict(rows=100000, cols=1, kind="topk", cap=777, sigma=1.0),
