@@ -189,6 +189,84 @@ def test_sweep_2p25_randk_oracle_whole_layer():
         del grad
 
 
+def _lsr(z, s):
+    """Logical right shift of int64 tensors (torch's >> is arithmetic)."""
+    return (z >> s) & ((1 << (64 - s)) - 1)
+
+
+def _as_i64(u):
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+def _randk_keys(base, i0, i1):
+    """rand-k keys of coordinates i0 .. i1-1 on the device: the high 32 bits of
+    SplitMix64 output i+1 from the unit's base state (modular int64 arithmetic,
+    logical shifts).  The test checks them against the oracle's key function."""
+    i = torch.arange(i0, i1, device="cuda", dtype=torch.int64)
+    z = _as_i64(base) + (i + 1) * _as_i64(0x9E3779B97F4A7C15)
+    z = z ^ _lsr(z, 30)
+    z = z * _as_i64(0xBF58476D1CE4E5B9)
+    z = z ^ _lsr(z, 27)
+    z = z * _as_i64(0x94D049BB133111EB)
+    z = z ^ _lsr(z, 31)
+    return _lsr(z, 32)
+
+
+def test_sweep_top_2p30_randk_properties():
+    """rand-k 1 % on a single 2^30-element layer (the bench's largest sweep
+    point), two steps (the second on the key pass the first ran ahead), every
+    element checked on the device: exactly k ascending indices; they are the k
+    smallest (key, index) pairs, the keys recomputed from the oracle's base
+    state; sent values are v's bits; memory is +0 on the sent set and v
+    elsewhere.  v = fl(m + fl(eta * g)) by two torch kernels (no contraction)."""
+    need_gpu()
+    g = gce()
+    layers = workloads.sweep(30, "randk", 10000)
+    t = g.Table(workloads.table_layers(layers))
+    n, k = t.N, layers[0]["cap"]
+    mem = torch.zeros((1, n), device="cuda")
+    vals = torch.zeros((1, t.vals_per_worker), device="cuda")
+    idx = torch.zeros((1, t.vals_per_worker), dtype=torch.int32, device="cuda")
+    ws = t.workspace(1, "randk")
+    seed = 9
+    for s in range(2):
+        base = oracle.randk_base(seed, 0, 0, 0, s)
+        probe = [0, 1, 12345, n // 2 + 7, n - 1]
+        got = _randk_keys(base, 0, 2).tolist() + [int(_randk_keys(base, i, i + 1)) for i in probe[2:]]
+        assert got == [oracle.randk_key(base, i) for i in probe], s
+        grad = workloads.gradients(layers, 1, 5, 400 + s)
+        mem_old = mem.clone()
+        g.ef_randk_step(t, 1, grad, mem, workloads.ETA, None, seed, s, vals, idx, ws)
+        torch.cuda.synchronize()
+        ix = idx[0, :k].long()
+        assert bool((ix[1:] > ix[:-1]).all()) and int(ix[0]) >= 0 and int(ix[-1]) < n
+        prod = grad[0] * torch.tensor(workloads.ETA, dtype=torch.float32, device="cuda")
+        v = mem_old[0] + prod
+        del prod, grad, mem_old
+        assert torch.equal(v[ix].view(torch.int32), vals[0, :k].view(torch.int32)), s
+        sel = torch.zeros(n, dtype=torch.bool, device="cuda")
+        sel[ix] = True
+        expect_mem = torch.where(sel, torch.zeros_like(v), v)
+        assert torch.equal(mem[0].view(torch.int32), expect_mem.view(torch.int32)), s
+        del expect_mem, v
+        # the chosen set is the k smallest (key, index): every chosen pair is
+        # below every other one (key * 2^31 + index orders the pairs)
+        top_chosen, low_other = -1, 1 << 64
+        step = 1 << 26
+        for i0 in range(0, n, step):
+            comb = _randk_keys(base, i0, i0 + step) * (1 << 31) + torch.arange(
+                i0, i0 + step, device="cuda", dtype=torch.int64)
+            c = sel[i0:i0 + step]
+            if bool(c.any()):
+                top_chosen = max(top_chosen, int(comb[c].max()))
+            if bool((~c).any()):
+                low_other = min(low_other, int(comb[~c].min()))
+            del comb
+        assert top_chosen < low_other, s
+        del sel
+        torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("rank", [1, 2, 4])
 def test_tall_2p26_powersgd_oracle_whole_matrix(rank):
     """PowerSGD rank 1 / 2 / 4 on a 32768 x 2048 matrix (2^26 elements; P is
