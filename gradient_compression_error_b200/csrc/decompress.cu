@@ -7,11 +7,15 @@
 // parallel replicas live in one GPU's HBM and the combination is a sum in
 // worker order from +0.0 with fp32 round-to-nearest adds, times `scale`.
 //
-// Design: each CTA owns one 4096-element tile of the output and accumulates
-// every worker's contribution to it in shared memory, in worker order, then
-// writes the tile once.  Sparse payloads are sorted by index, so a first
-// pass (bounds) turns each (worker, layer) list into per-tile entry ranges
-// by comparing neighbouring indices -- no searching.  DRAM traffic: the
+// Design: every output element is written once, after all workers'
+// contributions to it are summed on chip in worker order.  Sparse payloads
+// are sorted by index, so a first pass (bounds) turns each (worker, layer)
+// list into per-span entry ranges (1024 outputs a span) by comparing
+// neighbouring indices -- no searching; then a warp per span gathers its
+// entries and adds them into its own shared accumulator (dc_sparse_kernel).
+// Sign payloads of up to 8 workers are decoded by table lookup
+// (dc_sign8_kernel); other layers and more workers take a block per
+// 4096-output tile (dc_accum_kernel, dc_sign_kernel).  DRAM traffic: the
 // payload read once plus one 4-byte write per output element.
 #include <mutex>
 
