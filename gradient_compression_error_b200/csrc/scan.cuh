@@ -65,16 +65,27 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int* s_warp, int* tot
     return res;
 }
 
-// Run by one full warp.  h: nb >= 32 bins in shared memory, nb % 32 == 0.
+// Sum of lane l's run of `per` bins h[l*per .. l*per + per), a power of two.
+// Lane l starts its run at a different bin than its neighbours, so the 32
+// reads of each step fall in 32 banks when per is a multiple of 32.
+__device__ __forceinline__ int64_t warp_run_sum(const int32_t* h, int per) {
+    const int lane = threadIdx.x & 31;
+    int64_t mine = 0;
+    for (int i = 0; i < per; ++i) mine += h[lane * per + ((i + lane) & (per - 1))];
+    return mine;
+}
+
+// Run by one full warp.  h: nb bins in shared memory, nb a power of two >= 32.
 // Finds the bin b with above(b) < target <= above(b) + h[b], where above(b)
 // is the sum of all bins above b (the crossing of the count taken from the
 // top).  Returns -1 when the total is below target.  *above_out = above(b).
+// The run of the lane holding the crossing is then split over the warp, q
+// bins a lane, and only the q bins of the lane holding it are scanned in turn.
 __device__ __forceinline__ int warp_find_from_top(const int32_t* h, int nb, int64_t target,
                                                   int64_t* above_out) {
     const int lane = threadIdx.x & 31;
     const int per = nb >> 5;
-    int64_t mine = 0;
-    for (int i = 0; i < per; ++i) mine += h[lane * per + i];
+    const int64_t mine = warp_run_sum(h, per);
     // inclusive suffix sum over lanes (this lane and every higher one)
     int64_t incl = mine;
 #pragma unroll
@@ -89,11 +100,22 @@ __device__ __forceinline__ int warp_find_from_top(const int32_t* h, int nb, int6
         return -1;
     }
     const int src = __ffs(ball) - 1;
+    const int64_t above_src = __shfl_sync(kFull, excl, src);
+    // lane j takes the j-th group of q bins from the top of src's run
+    const int q = per >= 32 ? per >> 5 : 1;
+    const int top = src * per + per - lane * q;  // one past this lane's group
+    int64_t sub = 0;
+    if (lane * q < per)
+        for (int i = 1; i <= q; ++i) sub += h[top - i];
+    const int64_t pin = warp_inclusive_scan(sub);  // groups at or above this lane's
+    const int64_t t2 = target - above_src;
+    const unsigned b2 = __ballot_sync(kFull, pin - sub < t2 && t2 <= pin);
+    const int s2 = __ffs(b2) - 1;  // b2 is never empty: src's run holds the crossing
     int res = -1;
     int64_t above = 0;
-    if (lane == src) {
-        int64_t acc = excl;
-        for (int b = lane * per + per - 1; b >= lane * per; --b) {
+    if (lane == s2) {
+        int64_t acc = above_src + pin - sub;
+        for (int b = top - 1; b >= top - q; --b) {
             if (acc + h[b] >= target) {
                 res = b;
                 above = acc;
@@ -102,8 +124,8 @@ __device__ __forceinline__ int warp_find_from_top(const int32_t* h, int nb, int6
             acc += h[b];
         }
     }
-    res = __shfl_sync(kFull, res, src);
-    above = __shfl_sync(kFull, above, src);
+    res = __shfl_sync(kFull, res, s2);
+    above = __shfl_sync(kFull, above, s2);
     *above_out = above;
     return res;
 }
@@ -114,8 +136,7 @@ __device__ __forceinline__ int warp_find_from_bottom(const int32_t* h, int nb, i
                                                      int64_t* below_out) {
     const int lane = threadIdx.x & 31;
     const int per = nb >> 5;
-    int64_t mine = 0;
-    for (int i = 0; i < per; ++i) mine += h[lane * per + i];
+    const int64_t mine = warp_run_sum(h, per);
     const int64_t incl = warp_inclusive_scan(mine);
     const int64_t excl = incl - mine;
     const unsigned ball = __ballot_sync(kFull, excl < target && target <= incl);
@@ -124,11 +145,22 @@ __device__ __forceinline__ int warp_find_from_bottom(const int32_t* h, int nb, i
         return -1;
     }
     const int src = __ffs(ball) - 1;
+    const int64_t below_src = __shfl_sync(kFull, excl, src);
+    // lane j takes the j-th group of q bins from the bottom of src's run
+    const int q = per >= 32 ? per >> 5 : 1;
+    const int bot = src * per + lane * q;  // this lane's first bin
+    int64_t sub = 0;
+    if (lane * q < per)
+        for (int i = 0; i < q; ++i) sub += h[bot + i];
+    const int64_t pin = warp_inclusive_scan(sub);
+    const int64_t t2 = target - below_src;
+    const unsigned b2 = __ballot_sync(kFull, pin - sub < t2 && t2 <= pin);
+    const int s2 = __ffs(b2) - 1;  // never empty: src's run holds the crossing
     int res = -1;
     int64_t below = 0;
-    if (lane == src) {
-        int64_t acc = excl;
-        for (int b = lane * per; b < lane * per + per; ++b) {
+    if (lane == s2) {
+        int64_t acc = below_src + pin - sub;
+        for (int b = bot; b < bot + q; ++b) {
             if (acc + h[b] >= target) {
                 res = b;
                 below = acc;
@@ -137,8 +169,8 @@ __device__ __forceinline__ int warp_find_from_bottom(const int32_t* h, int nb, i
             acc += h[b];
         }
     }
-    res = __shfl_sync(kFull, res, src);
-    below = __shfl_sync(kFull, below, src);
+    res = __shfl_sync(kFull, res, s2);
+    below = __shfl_sync(kFull, below, s2);
     *below_out = below;
     return res;
 }
