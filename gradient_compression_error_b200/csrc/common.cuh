@@ -254,6 +254,30 @@ inline int wave_grid(int64_t work, int per_sm, int resident) {
     return int(work < 1 ? 1 : (work < cap ? work : cap));
 }
 
+// (worker, tile within the worker) along a grid-stride walk over W x tiles_pw
+// tiles: one division at the start, then each step adds the stride's whole
+// workers and remaining tiles, carrying one worker when the tile overflows.
+struct TileWalk {
+    int64_t t;
+    int32_t w, lt, dw, dlt, tiles_pw;
+    __device__ __forceinline__ TileWalk(int64_t t0, int64_t stride, int32_t tpw)
+        : t(t0), tiles_pw(tpw) {
+        w = int32_t(t0 / tpw);
+        lt = int32_t(t0 - int64_t(w) * tpw);
+        dw = int32_t(stride / tpw);
+        dlt = int32_t(stride - int64_t(dw) * tpw);
+    }
+    __device__ __forceinline__ void next(int64_t stride) {
+        t += stride;
+        w += dw;
+        lt += dlt;
+        if (lt >= tiles_pw) {
+            lt -= tiles_pw;
+            ++w;
+        }
+    }
+};
+
 // ---- workspace carving ------------------------------------------------------
 struct Carver {
     size_t off = GCE_WS_HEADER_BYTES;

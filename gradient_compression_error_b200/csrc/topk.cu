@@ -662,9 +662,10 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
     const unsigned lt_mask = (1u << lane) - 1u;
     const int64_t total = int64_t(tiles_pw) * W;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
-        const int w = int(t / tiles_pw);
-        const int lt = int(t % tiles_pw);
+    for (TileWalk tw(int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5), wstride, tiles_pw);
+         tw.t < total; tw.next(wstride)) {
+        const int64_t t = tw.t;
+        const int w = tw.w, lt = tw.lt;
         const TileInfo ti = tile_info[lt];
         const int2 d = tile_dir[t];
         const int64_t s = int64_t(w) * ncomp + ti.sidx;
@@ -817,7 +818,7 @@ __global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restric
 }
 
 
-__global__ void __launch_bounds__(256) tk_emit_kernel(
+__global__ void __launch_bounds__(256, 5) tk_emit_kernel(
     const TileInfo* __restrict__ tile_info, int32_t tiles_pw,
     int32_t W, int32_t ncomp, int64_t N, int64_t comp_N, int64_t vals_pw,
     const TkSeg* __restrict__ segs, const int2* __restrict__ tile_dir,
@@ -830,9 +831,10 @@ __global__ void __launch_bounds__(256) tk_emit_kernel(
     const unsigned lt_mask = (1u << lane) - 1u;
     const int64_t total = int64_t(tiles_pw) * W;
     const int64_t wstride = int64_t(gridDim.x) * (blockDim.x >> 5);
-    for (int64_t t = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < total; t += wstride) {
-        const int w = int(t / tiles_pw);
-        const int lt = int(t % tiles_pw);
+    for (TileWalk tw(int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5), wstride, tiles_pw);
+         tw.t < total; tw.next(wstride)) {
+        const int64_t t = tw.t;
+        const int w = tw.w, lt = tw.lt;
         const TileInfo ti = tile_info[lt];
         const int2 d = tile_dir[t];
         const int2 before = tile_cnt[t];    // (key > T, key == T) in earlier tiles
