@@ -136,7 +136,7 @@ __device__ __forceinline__ int64_t tk_sample_key(const int32_t* h, int64_t targe
     return key < bottom ? bottom : key;
 }
 
-__global__ void __launch_bounds__(256) tk_sample_kernel(
+__global__ void __launch_bounds__(256, 6) tk_sample_kernel(
     const DevLayer* __restrict__ layers, const int32_t* __restrict__ sunit_layer,
     const int32_t* __restrict__ sunit_part, int32_t sunits_pw, int32_t W, int32_t ncomp,
     int64_t S, int64_t N, const float* __restrict__ grad, const float* __restrict__ mem,
