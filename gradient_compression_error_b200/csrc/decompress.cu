@@ -45,7 +45,7 @@ __device__ __forceinline__ int32_t layer_k(const DevLayer& L, const int32_t* k_o
 // begin after an entry's predecessor and at or before the entry itself.
 constexpr int kDcBoundPer = 8;
 
-__global__ void __launch_bounds__(256) dc_bounds_kernel(const DevLayer* __restrict__ layers,
+__global__ void __launch_bounds__(256, 8) dc_bounds_kernel(const DevLayer* __restrict__ layers,
                                                         const int32_t* __restrict__ bunit_layer,
                                                         const int32_t* __restrict__ bunit_chunk,
                                                         int32_t bunits_pw, int32_t W,
