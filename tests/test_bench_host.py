@@ -86,3 +86,25 @@ def test_payload_bytes_per_worker():
     b = bench.payload_bytes_per_worker(bert, "topk")
     assert b == 8 * 1094775
     assert 49 < 4 * 109482240 / b < 51
+
+
+def test_workload_names():
+    """The bench's workload names: the BERT-base sets, and the sweep points with
+    an optional _w<W> worker count (the small W = 8 cases of the decoders)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    d = bench.workload_spec("bert_base_topk1pct_w8")
+    assert (d["W"], d["method"], len(d["layers"])) == (8, "topk", 90)
+    d = bench.workload_spec("sweep_topk_e24_ppm10000_w8")
+    assert (d["W"], d["method"], d["layers"][0]["rows"], d["layers"][0]["cap"]) == \
+        (8, "topk", 1 << 24, 167772)
+    d = bench.workload_spec("sweep_randk_e30_ppm10000")
+    assert (d["W"], d["method"], d["layers"][0]["rows"]) == (1, "randk", 1 << 30)
+    d = bench.workload_spec("sweep_sign_e25_w8")
+    assert (d["W"], d["method"], d["layers"][0]["kind"], d["layers"][0]["cap"]) == \
+        (8, "sign", "sign", 0)
+    d = bench.workload_spec("sweep_powersgd_e30_r2_lazy")
+    assert (d["W"], d["method"], d["layers"][0]["rows"], d["layers"][0]["cols"]) == \
+        (1, "powersgd_lazy", 1 << 15, 1 << 15)
+    with pytest.raises(SystemExit):
+        bench.workload_spec("no_such_workload")
