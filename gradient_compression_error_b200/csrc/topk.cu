@@ -245,6 +245,8 @@ __global__ void __launch_bounds__(256, 6) tk_sample_kernel(
                     segs[seg].top = top;
                 }
             }
+            int32_t* h1 = tk_hist(hists, S, 1, seg);  // level 1 starts at zero
+            for (int b = tid; b < kTkBins; b += blockDim.x) h1[b] = 0;
         }
         __syncthreads();
     }
@@ -724,7 +726,7 @@ __global__ void __launch_bounds__(256) tk_count_kernel(const TileInfo* __restric
     }
 }
 
-__global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restrict__ layers,
+__global__ void __launch_bounds__(512) tk_scan_kernel(const DevLayer* __restrict__ layers,
                                                        const int32_t* __restrict__ comp,
                                                        int32_t ncomp, int64_t S, int32_t tiles_pw,
                                                        int64_t comp_N, TkSeg* __restrict__ segs,
@@ -734,7 +736,7 @@ __global__ void __launch_bounds__(1024) tk_scan_kernel(const DevLayer* __restric
     grid_dependency_sync();
     __shared__ int s_warp[33];
     __shared__ int32_t h[kTkBins];
-    __shared__ uint32_t s_key[1024];
+    __shared__ uint32_t s_key[512];
     __shared__ uint32_t s_T;
     __shared__ int32_t s_need;
     for (int64_t s = blockIdx.x; s < S; s += gridDim.x) {
@@ -919,9 +921,10 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         int2* tile_cnt = at<int2>(ws, lay.tile_cnt);
         float* spill_v = at<float>(ws, lay.spill_v);
         int32_t* spill_i = at<int32_t>(ws, lay.spill_i);
-        // the sample and level-1 histograms; a level's last block clears the
-        // next level's histogram of its segment when that level has work
-        const int64_t n4 = lay.S * (kTkSBins + kTkBins) / 4;
+        // the sample histograms; the sample's last block of a segment clears
+        // its level-1 histogram, and a level's last block the next level's
+        // when that level has work
+        const int64_t n4 = lay.S * kTkSBins / 4;
 
         static const int r_setup = resident_blocks(tk_setup_kernel, 256);
         static const int r_sample = resident_blocks(tk_sample_kernel, 256);
@@ -932,7 +935,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         static const int r_h2 = resident_blocks(tk_hist_kernel<2>, 256);
         static const int r_h3 = resident_blocks(tk_hist_kernel<3>, 256);
         static const int r_count = resident_blocks(tk_count_kernel, 256);
-        static const int r_scan = resident_blocks(tk_scan_kernel, 1024);
+        static const int r_scan = resident_blocks(tk_scan_kernel, 512);
         static const int r_emit = resident_blocks(tk_emit_kernel, 256);
         GCE_LAUNCH(tk_setup_kernel, wave_grid((n4 + lay.S + 255) / 256, 8, r_setup), 256, 0, st, t->d_layers,
                    t->d_comp, ncomp, lay.S, k_or_rank, segs, reinterpret_cast<int4*>(hists), n4,
@@ -963,7 +966,7 @@ extern "C" int ef_topk_step(const gce_table* t, int32_t W, const float* grad, fl
         const int64_t wwork = (lay.TT + 7) / 8;  // a warp per tile
         GCE_LAUNCH(tk_count_kernel, wave_grid(wwork, 8, r_count), 256, 0, st, t->d_tile_info,
                    t->tiles_pw, W, ncomp, t->comp_N, segs, tile_dir, tile_cnt, spill_v, spill_i);
-        GCE_LAUNCH(tk_scan_kernel, wave_grid(lay.S, 2, r_scan), 1024, 0, st, t->d_layers, t->d_comp, ncomp,
+        GCE_LAUNCH(tk_scan_kernel, wave_grid(lay.S, 4, r_scan), 512, 0, st, t->d_layers, t->d_comp, ncomp,
                    lay.S, t->tiles_pw, t->comp_N, segs, tile_cnt, spill_v, spill_i);
         GCE_LAUNCH(tk_emit_kernel, wave_grid(wwork, 8, r_emit), 256, 0, st, t->d_tile_info,
                    t->tiles_pw, W, ncomp, t->N, t->comp_N, t->vals_pw, segs, tile_dir, tile_cnt,
