@@ -93,3 +93,31 @@ def test_sign_step_updates_memory_per_worker():
         s2, w2, m2 = oracle.ef_sign_unit(grad[w, :120], np.zeros(120, np.float32), 0.1)
         assert sc == s2 and np.array_equal(words, w2) and np.array_equal(mem[w, :120], m2)
         assert not mem[w, 120:].any()
+
+
+def test_sum_and_vote_at_forty_workers_against_numpy():
+    """The oracle's aggregates over 40 workers (more than one 32-bit lane's
+    worth) against their definitions written with numpy: the sum adds
+    +-s_w worker by worker in fp32 from +0.0; the vote is the sign of
+    (#positive - #negative) times the scale, 0 on a tie."""
+    W, n = 40, 77
+    layers = [dict(rows=n, cols=1, kind="sign")]
+    rng = np.random.default_rng(12)
+    neg = rng.integers(0, 2, (W, n)).astype(bool)
+    scales = rng.uniform(0.01, 3.0, W).astype(np.float32)
+    pay = {}
+    for w in range(W):
+        words = np.zeros((n + 31) // 32, np.uint32)
+        for i in np.nonzero(neg[w])[0]:
+            words[i // 32] |= np.uint32(1) << np.uint32(i % 32)
+        pay[(w, 0)] = (scales[w], words)
+    expect = np.zeros(n, np.float32)
+    for w in range(W):
+        expect = (expect + np.where(neg[w], -scales[w], scales[w])).astype(np.float32)
+    expect = (expect * np.float32(0.5)).astype(np.float32)
+    assert np.array_equal(steps.decompress(layers, W, pay, 0.5).view(np.uint32),
+                          expect.view(np.uint32))
+    margin = (~neg).sum(axis=0) - neg.sum(axis=0)
+    vote = np.where(margin > 0, np.float32(0.25),
+                    np.where(margin < 0, np.float32(-0.25), np.float32(0.0)))
+    assert np.array_equal(steps.vote(layers, W, pay, 0.25), vote)
